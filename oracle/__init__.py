@@ -1,0 +1,175 @@
+"""CPU oracle for block-scaled FP4 quantization -- TEST INFRASTRUCTURE ONLY.
+
+Plain, slow, single-threaded C (``fp4q_oracle.c``) behind ctypes.  Only ``tests/``,
+``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may import this
+package; the library's product path never does.  It shares no code with the CUDA path.
+
+Each function follows the passage its C counterpart cites:
+  ScaleSweep (gist.science/ko/paper/2606.07618) "Methodology": global scale, base scale,
+      candidate windows [-3,+7] (MSE) / [-8,+7] (WMSE), MSE and WMSE objectives.
+  Adaptive Block-Scaled Data Types (gist.science/ko/paper/2603.28765) "Methodology":
+      IF4 selection, 7/6 and 6/7, indicator in the scale sign bit; "Problem": 4/6.
+  Bridging the Gap ... Microscaling FP4 (gist.science/ko/paper/2509.23202) "Methodology":
+      MXFP4 (32-element blocks, power-of-two scales), block-wise Hadamard.
+  TORQ (gist.science/ko/paper/2605.19561) "Method", S-step: block max onto the largest code.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import numpy as np
+
+from . import build as _build
+
+ST_OK, ST_NONFINITE, ST_RANGE = 0, 1, 2
+OBJ = {"absmax": 0, "four_over_six": 1, "sweep_mse": 2, "sweep_wmse": 3, "brute_mse": 4, "brute_wmse": 5}
+FMT = {"nvfp4": 0, "if4": 1, "mxfp4": 2}
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = C.CDLL(path)
+        P = C.c_void_p
+        i64 = C.c_int64
+        L.fp4q_o_e4m3_value.restype = C.c_double
+        L.fp4q_o_e4m3_value.argtypes = [C.c_int]
+        L.fp4q_o_e4m3_encode.restype = C.c_int
+        L.fp4q_o_e4m3_encode.argtypes = [C.c_float]
+        L.fp4q_o_e2m1_value.restype = C.c_float
+        L.fp4q_o_e2m1_value.argtypes = [C.c_int]
+        L.fp4q_o_e2m1_encode.restype = C.c_int
+        L.fp4q_o_e2m1_encode.argtypes = [C.c_float]
+        L.fp4q_o_global_scale.restype = C.c_float
+        L.fp4q_o_global_scale.argtypes = [C.c_float]
+        L.fp4q_o_mx_exponent.restype = C.c_int
+        L.fp4q_o_mx_exponent.argtypes = [C.c_float, C.c_int]
+        L.fp4q_o_hadamard32.restype = None
+        L.fp4q_o_hadamard32.argtypes = [P]
+        L.fp4q_o_nvfp4_quantize.restype = C.c_int
+        L.fp4q_o_nvfp4_quantize.argtypes = [P, i64, i64, i64, C.c_int, P, C.c_int, P, P, P, P, P, P, P]
+        L.fp4q_o_if4_quantize.restype = C.c_int
+        L.fp4q_o_if4_quantize.argtypes = [P, i64, i64, i64, C.c_int, P, P, P, P, P]
+        L.fp4q_o_mxfp4_quantize.restype = C.c_int
+        L.fp4q_o_mxfp4_quantize.argtypes = [P, i64, i64, i64, C.c_int, C.c_int, P, P]
+        L.fp4q_o_dequantize.restype = C.c_int
+        L.fp4q_o_dequantize.argtypes = [P, P, C.c_float, i64, i64, C.c_int, C.c_int, P, C.c_int]
+        _lib = L
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(C.c_void_p)
+
+
+def _f32(x):
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    if x.ndim == 1:
+        x = x.reshape(1, -1)
+    return x
+
+
+# --- codec -------------------------------------------------------------------------
+def e4m3_value(p: int) -> float:
+    return lib().fp4q_o_e4m3_value(int(p))
+
+
+def e4m3_encode(v: float) -> int:
+    return lib().fp4q_o_e4m3_encode(float(v))
+
+
+def e2m1_value(code: int) -> float:
+    return lib().fp4q_o_e2m1_value(int(code))
+
+
+def e2m1_encode(y: float) -> int:
+    return lib().fp4q_o_e2m1_encode(float(y))
+
+
+def global_scale(amax: float) -> float:
+    return lib().fp4q_o_global_scale(float(amax))
+
+
+def mx_exponent(a: float, ocp_floor: bool = False) -> int:
+    return lib().fp4q_o_mx_exponent(float(a), int(ocp_floor))
+
+
+def hadamard32(v) -> np.ndarray:
+    v = np.ascontiguousarray(v, dtype=np.float32).copy()
+    assert v.size == 32
+    lib().fp4q_o_hadamard32(_p(v))
+    return v
+
+
+# --- quantizers --------------------------------------------------------------------
+def nvfp4_quantize(x, objective="sweep_mse", importance=None, S=None):
+    """NVFP4 quantization of a float32 [rows, cols] array; returns a dict with packed codes
+    [rows, cols/2], scale bytes [rows, cols/16], S, status and per-block diagnostics."""
+    x = _f32(x)
+    rows, cols = x.shape
+    nb = cols // 16
+    codes = np.zeros((rows, cols // 2), np.uint8)
+    scales = np.zeros((rows, nb), np.uint8)
+    Sarr = np.array([0.0 if S is None else S], np.float32)
+    bp = np.zeros((rows, nb), np.int32)
+    be = np.zeros((rows, nb), np.float32)
+    be2 = np.zeros((rows, nb), np.float32)
+    bn = np.zeros((rows, nb), np.int32)
+    w = None if importance is None else np.ascontiguousarray(importance, np.float32)
+    st = lib().fp4q_o_nvfp4_quantize(_p(x), rows, cols, cols, OBJ[objective], _p(w), int(S is not None),
+                                     _p(Sarr), _p(codes), _p(scales), _p(bp), _p(be), _p(be2), _p(bn))
+    if st < 0:
+        raise ValueError("oracle: bad shape")
+    return {"codes": codes, "scales": scales, "S": float(Sarr[0]), "S_f32": Sarr, "status": st,
+            "p": bp, "err": be, "err2": be2, "nvalid": bn}
+
+
+def if4_quantize(x, S=None):
+    x = _f32(x)
+    rows, cols = x.shape
+    nb = cols // 16
+    codes = np.zeros((rows, cols // 2), np.uint8)
+    scales = np.zeros((rows, nb), np.uint8)
+    Sarr = np.array([0.0 if S is None else S], np.float32)
+    ef = np.zeros((rows, nb), np.float32)
+    ei = np.zeros((rows, nb), np.float32)
+    st = lib().fp4q_o_if4_quantize(_p(x), rows, cols, cols, int(S is not None), _p(Sarr), _p(codes),
+                                   _p(scales), _p(ef), _p(ei))
+    if st < 0:
+        raise ValueError("oracle: bad shape")
+    return {"codes": codes, "scales": scales, "S": float(Sarr[0]), "S_f32": Sarr, "status": st,
+            "err_fp": ef, "err_int": ei}
+
+
+def mxfp4_quantize(x, hadamard=False, ocp_floor=False):
+    x = _f32(x)
+    rows, cols = x.shape
+    codes = np.zeros((rows, cols // 2), np.uint8)
+    scales = np.zeros((rows, cols // 32), np.uint8)
+    st = lib().fp4q_o_mxfp4_quantize(_p(x), rows, cols, cols, int(hadamard), int(ocp_floor), _p(codes),
+                                     _p(scales))
+    if st < 0:
+        raise ValueError("oracle: bad shape")
+    return {"codes": codes, "scales": scales, "status": st}
+
+
+def dequantize(codes, scales, S, fmt, inverse_hadamard=False, out_bf16=False):
+    codes = np.ascontiguousarray(codes, np.uint8)
+    scales = np.ascontiguousarray(scales, np.uint8)
+    rows, cols = codes.shape[0], codes.shape[1] * 2
+    out = np.zeros((rows, cols), np.uint16 if out_bf16 else np.float32)
+    st = lib().fp4q_o_dequantize(_p(codes), _p(scales), float(S), rows, cols, FMT[fmt], int(inverse_hadamard),
+                                 _p(out), int(out_bf16))
+    if st < 0:
+        raise ValueError("oracle: bad shape")
+    return out
+
+
+def widen_bf16(bits) -> np.ndarray:
+    """bf16 bit patterns -> float32 (exact), the oracle's own input widening."""
+    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return b.view(np.float32)
