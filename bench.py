@@ -1,0 +1,398 @@
+#!/usr/bin/env python
+"""Throughput benchmark: NVFP4 ScaleSweep-MSE dynamic activation quantization of a bf16
+8192x4096 activation tensor (amax pass + sweep quantization), on B200.
+
+One step = the whole hot path over one tensor: tensor scale S = max|x|/1536 (amax kernel),
+then base scale, 11-candidate sweep, RTN, error, argmin, nibble pack and scale write (sweep
+kernel).  value = algorithmic bytes per step (2 B/element read + 0.5 B codes + 1/16 B scales
++ 4 B S) x steps / device time.  Inputs rotate over distinct buffer sets whose total exceeds
+the 126 MB L2, so every step reads its input from HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Multi-GPU (torchrun): every rank quantizes its own tensor (weak scaling, no collective on
+the data path); time = max over ranks of the device time.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOADS = {
+    # name: (synth config, fmt, objective, description)
+    "cfg3": ("cfg3", "nvfp4", "sweep_mse",
+             "NVFP4 ScaleSweep-MSE dynamic activation quantization, bf16 8192x4096 (tokens x hidden), "
+             "Laplace values, lognormal(0,1.5) channel std, 8 outlier channels x50, dynamic S"),
+    "cfg2": ("cfg2", "nvfp4", "sweep_wmse",
+             "NVFP4 ScaleSweep-WMSE, bf16 weight 14336x4096, 0.02*t5, per-input-column importance"),
+    "cfg4": ("cfg4", "if4", None, "IF4 per-block FP4/INT4 selection, bf16 weight 4096x14336, 0.02*t4"),
+    "cfg5": ("cfg5", "mxfp4", None, "MXFP4, bf16 activations 16384x8192"),
+    "cfg5h": ("cfg5", "mxfp4_had", None, "MXFP4 after 32x32 block Hadamard, bf16 activations 16384x8192"),
+}
+METRIC = "quantize GB/s (input bf16) and % of B200 HBM peak, 1 GPU, vs CPU oracle"
+L2_BYTES = 126 * 2 ** 20
+
+
+def algorithmic_bytes(rows, cols, fmt, in_bytes=2, wmse=False):
+    B = 32 if fmt.startswith("mxfp4") else 16
+    n = rows * cols
+    b = n * in_bytes + n // 2 + n // B
+    if not fmt.startswith("mxfp4"):
+        b += 4
+    if wmse:
+        b += 4 * cols
+    return b
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("fp4_block_scaled_nvfp4_b200/csrc/fp4q.cu", "fp4_block_scaled_nvfp4_b200/csrc/fp4q_device.cuh"):
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel_key):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the current
+    kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel_key)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Polls NVML for SM clock and throttle reasons while the timed region runs."""
+
+    def __init__(self, index):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            uuid = str(torch.cuda.get_device_properties(index).uuid)
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # no NVML: report no samples
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        names = {
+            getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8): "hw_slowdown",
+            getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40): "hw_thermal_slowdown",
+            getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20): "sw_thermal_slowdown",
+            getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4): "sw_power_cap",
+            getattr(nv, "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80): "hw_power_brake_slowdown",
+        }
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in names.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                break
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.nv:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        return {"sm_mhz": (statistics.median(self.samples) if self.samples else None), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml polled every ~2 ms"}
+
+
+def device_tensor_from_bits(bits, torch):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+
+
+def cpu_baseline(w, fmt, obj, budget_s=12.0):
+    """The oracle as it stands, single-threaded, on whole rows of the same tensor until about
+    budget_s of CPU time has been spent; returns its throughput in the same unit."""
+    import oracle as O
+    x = O.widen_bf16(w["x"]) if w["dtype"] == "bf16" else w["x"]
+    rows, cols = x.shape
+    chunk = max(1, min(rows, 256))
+    done, t0 = 0, time.perf_counter()
+    imp = w.get("importance")
+    while done < rows and time.perf_counter() - t0 < budget_s:
+        xs = x[done:done + chunk]
+        if fmt == "nvfp4":
+            O.nvfp4_quantize(xs, obj, importance=imp)
+        elif fmt == "if4":
+            O.if4_quantize(xs)
+        else:
+            O.mxfp4_quantize(xs, hadamard=fmt.endswith("had"))
+        done += xs.shape[0]
+    dt = time.perf_counter() - t0
+    nbytes = algorithmic_bytes(done, cols, fmt, wmse=(obj == "sweep_wmse"))
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{done} of {rows} rows of the {rows}x{cols} tensor ({done * cols} elements), "
+                      f"S over the sampled rows, {dt:.1f} s single-threaded"}
+
+
+def run_reference(args, rank, world):
+    """The oracle on the host cores as the reference arm: K steps, each a bounded row sample."""
+    cfg, fmt, obj, desc = WORKLOADS[args.workload]
+    from fp4_block_scaled_nvfp4_b200 import synth
+    import oracle as O
+    if rank != 0:
+        return
+    w = synth.make(cfg)
+    x = O.widen_bf16(w["x"]) if w["dtype"] == "bf16" else w["x"]
+    rows, cols = x.shape
+    sample_rows = 16
+    imp = w.get("importance")
+
+    def step(i):
+        r0 = (i * sample_rows) % rows
+        xs = x[r0:r0 + sample_rows]
+        if fmt == "nvfp4":
+            O.nvfp4_quantize(xs, obj, importance=imp)
+        elif fmt == "if4":
+            O.if4_quantize(xs)
+        else:
+            O.mxfp4_quantize(xs, hadamard=fmt.endswith("had"))
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    dt = time.perf_counter() - t0
+    nbytes = algorithmic_bytes(sample_rows, cols, fmt, wmse=(obj == "sweep_wmse")) * args.steps
+    val = nbytes / dt / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": desc, "rows": rows, "cols": cols, "input_dtype": w["dtype"],
+                       "step_sample_rows": sample_rows},
+            "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{sample_rows} rows per step of the {rows}x{cols} tensor"},
+            "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world):
+    import torch
+    import torch.distributed as dist
+
+    import fp4_block_scaled_nvfp4_b200 as fq
+    from fp4_block_scaled_nvfp4_b200 import synth
+
+    cfg, fmt, obj, desc = WORKLOADS[args.workload]
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    fq.lib()
+
+    w = synth.make(cfg)
+    rows, cols = w["rows"], w["cols"]
+    x_host = device_tensor_from_bits(w["x"], torch)
+    in_bytes = x_host.numel() * 2
+    alg = algorithmic_bytes(rows, cols, fmt, wmse=(obj == "sweep_wmse"))
+    out_bytes = rows * cols // 2 + rows * cols // (32 if fmt.startswith("mxfp4") else 16)
+    nsets = max(2, int(np.ceil(2.5 * L2_BYTES / (in_bytes + out_bytes))))
+    xs = [x_host.to(dev) for _ in range(nsets)]
+    outs = [fq.alloc_outputs(rows, cols, "mxfp4" if fmt.startswith("mxfp4") else fmt, dev) for _ in range(nsets)]
+    imp = torch.from_numpy(w["importance"]).to(dev) if obj == "sweep_wmse" else None
+    ws = fq.new_workspace(dev)
+    launches_per_step = 0
+
+    def step(s, ev=None):
+        c, sc, g = outs[s]
+        if ev is not None:
+            ev[0].record()
+        if fmt.startswith("mxfp4"):
+            if fmt.endswith("had"):
+                fq.hadamard_quantize(xs[s], out=(c, sc, None), workspace=ws)
+            else:
+                fq.quantize(xs[s], "mxfp4", out=(c, sc, None), workspace=ws)
+            if ev is not None:
+                ev[1].record()
+                ev[2].record()
+            return 1
+        fq.global_scale(xs[s], out=g, workspace=ws)
+        if ev is not None:
+            ev[1].record()
+        fq.quantize(xs[s], fmt, obj or "absmax", importance=imp, global_scale=g, out=(c, sc, g), workspace=ws)
+        if ev is not None:
+            ev[2].record()
+        return 2
+
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            launches_per_step = step(i % nsets)
+    torch.cuda.synchronize()
+
+    # one CUDA graph per buffer set; external timing events inside each graph bracket the
+    # amax and the quantize kernel of that step
+    graphs, evs = [], []
+    for s in range(nsets):
+        ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(s, ev)
+        graphs.append(g)
+        evs.append(ev)
+    with torch.cuda.stream(stream):
+        for s in range(nsets):
+            graphs[s].replay()
+    torch.cuda.synchronize()
+
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            start.record()
+            for i in range(args.steps):
+                graphs[i % nsets].replay()
+            end.record()
+        end.synchronize()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = start.elapsed_time(end)
+    t_amax = [evs[s][0].elapsed_time(evs[s][1]) for s in range(nsets)]
+    t_q = [evs[s][1].elapsed_time(evs[s][2]) for s in range(nsets)]
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # status of the last step must be clean
+    st = fq.read_device_status(ws)
+
+    # end to end through the public API with host buffers: H2D of the input, quantize, D2H
+    e2e_steps = max(1, min(args.steps, 20))
+    x_pin = x_host.pin_memory()
+    dev_bufs = {"x": xs[0], "out": outs[0]}
+    host_out = fq.alloc_host_outputs(rows, cols, "mxfp4" if fmt.startswith("mxfp4") else fmt)
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            fq.quantize_host(x_pin, fmt, obj or "absmax", importance=imp, workspace=ws, dev_bufs=dev_bufs,
+                             host_out=host_out)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(e2e_steps):
+            fq.quantize_host(x_pin, fmt, obj or "absmax", importance=imp, workspace=ws, dev_bufs=dev_bufs,
+                             host_out=host_out)
+        e1.record()
+    e1.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = in_bytes
+    d2h = out_bytes + (4 if not fmt.startswith("mxfp4") else 0)
+
+    if rank != 0:
+        return
+    peak, peak_src = load_peaks()
+    per_step_ms = ms / args.steps
+    value = alg * args.steps * world / (ms * 1e-3) / 1e9
+    tq = statistics.mean(t_q)
+    kernel_key = f"{args.workload}:quantize"
+    achieved = alg / (tq * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(per_step_ms, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": desc, "rows": rows, "cols": cols, "input_dtype": w["dtype"],
+                   "method": obj or fmt, "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": f"{nsets} rotating input/output buffer sets, {nsets * (in_bytes + out_bytes) / 2**20:.0f} MB "
+                         f"total (> 2x the 126 MB L2)",
+                   "timing": "CUDA graph per step replayed on one stream; CUDA events on that stream"},
+        "hbm_frac": round(value / world / peak, 4),
+        "input_gbps": round(in_bytes * args.steps * world / (ms * 1e-3) / 1e9, 2),
+        "elements_per_s": round(rows * cols * args.steps * world / (ms * 1e-3), 1),
+        "kernels_ms": {"amax": round(statistics.mean(t_amax), 5), "quantize": round(tq, 5)},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": profiled_traffic(kernel_key),
+                     "kernel": "quantize (" + (obj or fmt) + ")",
+                     "peak_source": f"{peak_src} hbm_gbs (copy, burst) from MEASURED_PEAKS.json"},
+        "device_status": st,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+        "e2e": {"value": round(alg / (e2e_ms * 1e-3) / 1e9 * world, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
+    }
+    if args.cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(w, fmt, obj, budget_s=args.cpu_seconds)
+    elif args.cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, fmt, obj, budget_s=args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="cfg3")
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world > 1 and args.impl == "ours":
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world)
+    finally:
+        if world > 1 and args.impl == "ours":
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

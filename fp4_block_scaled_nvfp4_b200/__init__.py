@@ -1,0 +1,229 @@
+"""Block-scaled FP4 quantization (NVFP4 / IF4 / MXFP4) for NVIDIA B200.
+
+Thin ctypes binding over ``libfp4q.so`` (the C ABI in ``include/fp4q.h``).  Every step of
+the quantization runs in the library's sm_100a kernels; this module only marshals torch
+tensors (device memory and the current CUDA stream) into the C calls.  There is no CPU
+fallback: if the library is missing the functions raise.
+
+    codes, scales, S = quantize(x, fmt="nvfp4", objective="sweep_mse")
+    xh = dequantize(codes, scales, S, fmt="nvfp4")
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfp4q.so")
+
+OK, ERR_INVALID_ARG, ERR_SHAPE, ERR_ALIGNMENT, ERR_UNSUPPORTED, ERR_CUDA = range(6)
+DEVSTAT_OK, DEVSTAT_NONFINITE, DEVSTAT_RANGE = 0, 1, 2
+IN_F32, IN_BF16 = 0, 1
+FORMATS = {"nvfp4": 0, "if4": 1, "mxfp4": 2}
+OBJECTIVES = {"absmax": 0, "four_over_six": 1, "sweep_mse": 2, "sweep_wmse": 3}
+F_GLOBAL_SCALE_GIVEN, F_MX_OCP_FLOOR, F_OUT_BF16 = 0x1, 0x2, 0x4
+BLOCK = {"nvfp4": 16, "if4": 16, "mxfp4": 32}
+
+# Names of every function include/fp4q.h declares (checked against the header by the tests).
+EXPORTS = ("fp4q_workspace_bytes", "fp4q_global_scale", "fp4q_quantize", "fp4q_hadamard_quantize", "fp4q_dequantize",
+           "fp4q_read_device_status", "fp4q_last_launch_count", "fp4q_status_string")
+
+_lib = None
+
+
+class Fp4qError(RuntimeError):
+    pass
+
+
+def lib():
+    """Load libfp4q.so (built in-tree by __graft_entry__.build()); raise if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise Fp4qError(f"{LIB_PATH} is not built; run `python -c 'import __graft_entry__ as g; g.build()'`")
+        L = C.CDLL(LIB_PATH)
+        P, i64, u32, i32 = C.c_void_p, C.c_int64, C.c_uint32, C.c_int
+        L.fp4q_workspace_bytes.restype = C.c_size_t
+        L.fp4q_workspace_bytes.argtypes = []
+        L.fp4q_quantize.restype = i32
+        L.fp4q_quantize.argtypes = [P, i32, i64, i64, i64, i32, i32, P, P, P, P, P, u32, P]
+        L.fp4q_global_scale.restype = i32
+        L.fp4q_global_scale.argtypes = [P, i32, i64, i64, i64, P, P, P]
+        L.fp4q_hadamard_quantize.restype = i32
+        L.fp4q_hadamard_quantize.argtypes = [P, i32, i64, i64, i64, i32, P, P, P, u32, P]
+        L.fp4q_dequantize.restype = i32
+        L.fp4q_dequantize.argtypes = [P, P, P, i64, i64, i32, i32, P, u32, P]
+        L.fp4q_read_device_status.restype = i32
+        L.fp4q_read_device_status.argtypes = [P, C.POINTER(C.c_uint32), P]
+        L.fp4q_last_launch_count.restype = i32
+        L.fp4q_last_launch_count.argtypes = []
+        L.fp4q_status_string.restype = C.c_char_p
+        L.fp4q_status_string.argtypes = [i32]
+        _lib = L
+    return _lib
+
+
+def status_string(rc: int) -> str:
+    return lib().fp4q_status_string(int(rc)).decode()
+
+
+def _check(rc: int, what: str):
+    if rc != OK:
+        raise Fp4qError(f"{what}: {status_string(rc)} ({rc})")
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream_ptr(stream=None):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return C.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def workspace_bytes() -> int:
+    return int(lib().fp4q_workspace_bytes())
+
+
+def new_workspace(device="cuda"):
+    """A zero-filled workspace (the library leaves it zeroed after each call, except the
+    device status word)."""
+    torch = _torch()
+    return torch.zeros(max(workspace_bytes(), 16), dtype=torch.uint8, device=device)
+
+
+def _dtype_code(x):
+    torch = _torch()
+    if x.dtype == torch.bfloat16:
+        return IN_BF16
+    if x.dtype == torch.float32:
+        return IN_F32
+    raise Fp4qError(f"unsupported input dtype {x.dtype} (bf16 or fp32)")
+
+
+def alloc_outputs(rows: int, cols: int, fmt: str, device="cuda"):
+    torch = _torch()
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=device)
+    scales = torch.empty((rows, cols // BLOCK[fmt]), dtype=torch.uint8, device=device)
+    gs = torch.empty((1,), dtype=torch.float32, device=device)
+    return codes, scales, gs
+
+
+def quantize(x, fmt: str = "nvfp4", objective: str = "sweep_mse", importance=None, global_scale=None,
+             mx_ocp_floor: bool = False, out=None, workspace=None, stream=None):
+    """Quantize a 2-D bf16/fp32 CUDA tensor (row stride may exceed the width).
+
+    Returns (codes [rows, cols/2] uint8, scales [rows, cols/B] uint8, S [1] float32 or None).
+    global_scale: a [1] float32 CUDA tensor to use as S (skips the amax pass).
+    out: optional preallocated (codes, scales, S) tuple.
+    """
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise Fp4qError("x must be 2-D with unit column stride")
+    rows, cols = x.shape
+    codes, scales, gs = out if out is not None else alloc_outputs(rows, cols, fmt, x.device)
+    flags = 0
+    if global_scale is not None:
+        flags |= F_GLOBAL_SCALE_GIVEN
+        gs = global_scale
+    if mx_ocp_floor:
+        flags |= F_MX_OCP_FLOOR
+    ws = workspace if workspace is not None else new_workspace(x.device)
+    rc = lib().fp4q_quantize(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), FORMATS[fmt],
+                             OBJECTIVES.get(objective, 0), _ptr(importance), _ptr(codes), _ptr(scales),
+                             _ptr(gs) if fmt != "mxfp4" else None, _ptr(ws), flags, _stream_ptr(stream))
+    _check(rc, "fp4q_quantize")
+    return codes, scales, (gs if fmt != "mxfp4" else None)
+
+
+def global_scale(x, out=None, workspace=None, stream=None):
+    """Tensor scale S = RN(max|x| / 1536) as a [1] float32 CUDA tensor (amax pass only)."""
+    torch = _torch()
+    rows, cols = x.shape
+    gs = out if out is not None else torch.empty((1,), dtype=torch.float32, device=x.device)
+    ws = workspace if workspace is not None else new_workspace(x.device)
+    rc = lib().fp4q_global_scale(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), _ptr(gs), _ptr(ws),
+                                 _stream_ptr(stream))
+    _check(rc, "fp4q_global_scale")
+    return gs
+
+
+def hadamard_quantize(x, mx_ocp_floor: bool = False, out=None, workspace=None, stream=None):
+    """MXFP4 quantization after a normalized 32-point block Hadamard rotation."""
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise Fp4qError("x must be 2-D with unit column stride")
+    rows, cols = x.shape
+    codes, scales, _ = out if out is not None else alloc_outputs(rows, cols, "mxfp4", x.device)
+    ws = workspace if workspace is not None else new_workspace(x.device)
+    rc = lib().fp4q_hadamard_quantize(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), 32, _ptr(codes),
+                                      _ptr(scales), _ptr(ws), F_MX_OCP_FLOOR if mx_ocp_floor else 0,
+                                      _stream_ptr(stream))
+    _check(rc, "fp4q_hadamard_quantize")
+    return codes, scales
+
+
+def dequantize(codes, scales, global_scale, fmt: str = "nvfp4", inverse_hadamard: bool = False,
+               out_dtype=None, out=None, stream=None):
+    torch = _torch()
+    out_dtype = out_dtype or torch.float32
+    rows, cols = codes.shape[0], codes.shape[1] * 2
+    if out is None:
+        out = torch.empty((rows, cols), dtype=out_dtype, device=codes.device)
+    flags = F_OUT_BF16 if out.dtype == torch.bfloat16 else 0
+    rc = lib().fp4q_dequantize(_ptr(codes), _ptr(scales), _ptr(global_scale), rows, cols, FORMATS[fmt],
+                               int(inverse_hadamard), _ptr(out), flags, _stream_ptr(stream))
+    _check(rc, "fp4q_dequantize")
+    return out
+
+
+def read_device_status(workspace, stream=None) -> int:
+    st = C.c_uint32(0)
+    _check(lib().fp4q_read_device_status(_ptr(workspace), C.byref(st), _stream_ptr(stream)), "read_device_status")
+    return int(st.value)
+
+
+def last_launch_count() -> int:
+    return int(lib().fp4q_last_launch_count())
+
+
+def alloc_host_outputs(rows: int, cols: int, fmt: str):
+    """Pinned host buffers for (codes, scales, S)."""
+    torch = _torch()
+    fmt = "mxfp4" if fmt.startswith("mxfp4") else fmt
+    return (torch.empty((rows, cols // 2), dtype=torch.uint8, pin_memory=True),
+            torch.empty((rows, cols // BLOCK[fmt]), dtype=torch.uint8, pin_memory=True),
+            torch.empty((1,), dtype=torch.float32, pin_memory=True))
+
+
+def quantize_host(x_host, fmt="nvfp4", objective="sweep_mse", importance=None, stream=None, workspace=None,
+                  dev_bufs=None, host_out=None):
+    """End-to-end call on host (pinned) memory: copy the input in, quantize on the device,
+    copy codes, scales and S back (asynchronously on the current stream).
+    fmt "mxfp4_had" selects the Hadamard-rotated MXFP4 path.  Returns host (codes, scales, S)."""
+    torch = _torch()
+    rows, cols = x_host.shape
+    base = "mxfp4" if fmt.startswith("mxfp4") else fmt
+    if dev_bufs is None:
+        dev_bufs = {"x": torch.empty(x_host.shape, dtype=x_host.dtype, device="cuda"),
+                    "out": alloc_outputs(rows, cols, base, "cuda")}
+    if host_out is None:
+        host_out = alloc_host_outputs(rows, cols, base)
+    xd = dev_bufs["x"]
+    xd.copy_(x_host, non_blocking=True)
+    if fmt == "mxfp4_had":
+        codes, scales = hadamard_quantize(xd, out=dev_bufs["out"], workspace=workspace, stream=stream)
+        gs = None
+    else:
+        codes, scales, gs = quantize(xd, base, objective, importance=importance, out=dev_bufs["out"],
+                                     workspace=workspace, stream=stream)
+    hc, hs, hg = host_out
+    hc.copy_(codes, non_blocking=True)
+    hs.copy_(scales, non_blocking=True)
+    if gs is not None:
+        hg.copy_(gs, non_blocking=True)
+    return hc, hs, (hg if gs is not None else None)

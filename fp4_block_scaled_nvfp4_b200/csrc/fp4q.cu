@@ -1,0 +1,734 @@
+// fp4q.cu -- sm_100a kernels and the C ABI of libfp4q (declared in include/fp4q.h).
+//
+// Kernels (one CUDA thread owns one quantization block, so the per-block search runs in
+// registers without any cross-thread reduction):
+//   amax_kernel          tensor max|x| as an integer max over magnitude bit patterns
+//                        (NaN/Inf sort above every finite value), one atomicMax per CTA;
+//                        the last CTA to arrive computes S = RN(amax/1536) and the data
+//                        flags.  ScaleSweep (gist.science/ko/paper/2606.07618),
+//                        "Methodology", global scale S = max|x|/(256*6).
+//   nvfp4_kernel<OBJ>    base scale, candidate sweep, RTN, block error, argmin, nibble
+//                        pack, scale write.  ScaleSweep "Methodology" (offsets [-3,+7] MSE,
+//                        [-8,+7] WMSE), 4/6 (Adaptive Block-Scaled Data Types,
+//                        gist.science/ko/paper/2603.28765, "Problem").
+//   if4_kernel           FP4 vs scaled-INT4 per block, indicator in the scale sign bit.
+//                        Adaptive Block-Scaled Data Types, "Methodology", IF4 structure.
+//   mxfp4_kernel<HAD>    E8M0 scale + RTN over 32-element blocks, optional in-register
+//                        32-point fast Walsh-Hadamard rotation.  Bridging the Gap ...
+//                        Microscaling FP4 (gist.science/ko/paper/2509.23202),
+//                        "Methodology"; TORQ (gist.science/ko/paper/2605.19561) S-step.
+//   dequant kernels      codes + scales (+S) -> fp32 / bf16.
+// Status protocol (workspace words): each quantize kernel ORs its data flags into
+// PENDING, counts its CTAs in an arrival counter, and the last CTA publishes
+// STATUS = PENDING and zeroes PENDING and the counter, so the workspace is clean again
+// after every call.
+#include <cmath>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "fp4q.h"
+#include "fp4q_device.cuh"
+
+namespace fp4q {
+
+enum : int { WS_STATUS = 0, WS_PENDING = 1, WS_AMAX = 2, WS_CNT_AMAX = 3, WS_CNT_Q = 4 };
+constexpr size_t kWorkspaceBytes = 64;
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ bool scale_range_ok(float S) {
+    if (S == 0.0f) return true;
+    return S >= 0x1p-117f && S <= __fdiv_rn(0x1p125f, 1536.0f);
+}
+
+// Data flags implied by the tensor scale: NaN/Inf S -> NONFINITE, S outside the supported
+// range -> RANGE (every candidate scale must stay normal and every reciprocal finite).
+__device__ __forceinline__ uint32_t scale_flags(float S) {
+    if (!isfinite(S)) return FP4Q_DEVSTAT_NONFINITE;
+    return scale_range_ok(S) ? 0u : (uint32_t)FP4Q_DEVSTAT_RANGE;
+}
+
+// Publish this CTA's data flags; the last CTA of the grid writes the call's status word.
+__device__ __forceinline__ void finish_status(uint32_t* ws, uint32_t flag, int cnt) {
+    __shared__ uint32_t s_flag;
+    if (threadIdx.x == 0) s_flag = 0u;
+    __syncthreads();
+    if (flag) atomicOr(&s_flag, flag);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        if (s_flag) atomicOr(&ws[WS_PENDING], s_flag);
+        __threadfence();
+        const unsigned prev = atomicAdd(&ws[cnt], 1u);
+        if (prev == gridDim.x - 1) {
+            __threadfence();
+            const uint32_t all = atomicExch(&ws[WS_PENDING], 0u);
+            atomicExch(&ws[WS_STATUS], all);
+            atomicExch(&ws[cnt], 0u);
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// amax
+// ------------------------------------------------------------------------------------------
+template <int IN>
+__global__ void __launch_bounds__(kThreads) amax_kernel(const void* __restrict__ xv, int64_t rows, int64_t cols,
+                                                        int64_t ld, uint32_t* __restrict__ ws,
+                                                        float* __restrict__ gscale, int publish) {
+    const int64_t vpr = cols * (IN == FP4Q_IN_BF16 ? 2 : 4) / 16;   // 16-byte vectors per row
+    const int64_t total = rows * vpr;
+    const int64_t step = (int64_t)gridDim.x * blockDim.x;
+    uint32_t m = 0;
+    const uint4* base = reinterpret_cast<const uint4*>(xv);
+    const int64_t ldv = ld * (IN == FP4Q_IN_BF16 ? 2 : 4) / 16;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += step) {
+        int64_t off = i;
+        if (ldv != vpr) {
+            const int64_t r = i / vpr;
+            off = r * ldv + (i - r * vpr);
+        }
+        const uint4 v = __ldg(base + off);
+        if (IN == FP4Q_IN_BF16) {
+            uint32_t t;
+            const uint32_t mk = 0x7FFF7FFFu;
+            asm("max.u16x2 %0, %1, %2;" : "=r"(t) : "r"(v.x & mk), "r"(v.y & mk));
+            asm("max.u16x2 %0, %0, %1;" : "+r"(t) : "r"(v.z & mk));
+            asm("max.u16x2 %0, %0, %1;" : "+r"(t) : "r"(v.w & mk));
+            asm("max.u16x2 %0, %0, %1;" : "+r"(m) : "r"(t));
+        } else {
+            const uint32_t mk = 0x7FFFFFFFu;
+            m = max(m, max(max(v.x & mk, v.y & mk), max(v.z & mk, v.w & mk)));
+        }
+    }
+    if (IN == FP4Q_IN_BF16) m = max(m & 0xFFFFu, m >> 16) << 16;   // bf16 bits -> f32 bits
+    m = __reduce_max_sync(0xFFFFFFFFu, m);
+    __shared__ uint32_t red[kThreads / 32];
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < kThreads / 32; ++w) m = max(m, red[w]);
+        atomicMax(&ws[WS_AMAX], m);
+        __threadfence();
+        const unsigned prev = atomicAdd(&ws[WS_CNT_AMAX], 1u);
+        if (prev == gridDim.x - 1) {
+            __threadfence();
+            const uint32_t bits = atomicExch(&ws[WS_AMAX], 0u);
+            atomicExch(&ws[WS_CNT_AMAX], 0u);
+            const float S = bits >= 0x7F800000u ? __uint_as_float(0x7FC00000u)
+                                                : __fdiv_rn(__uint_as_float(bits), 1536.0f);
+            *gscale = S;
+            if (publish) atomicExch(&ws[WS_STATUS], scale_flags(S));
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// Shared pieces of the NVFP4 / IF4 kernels
+// ------------------------------------------------------------------------------------------
+struct Setup {
+    float S;
+    uint32_t flags;
+};
+
+// Tensor scale (given by the caller or written by the amax pass just before) and the data
+// flags it implies; every CTA derives the same values.
+__device__ __forceinline__ Setup read_setup(const float* gscale) {
+    Setup s;
+    s.S = *gscale;
+    s.flags = scale_flags(s.S);
+    return s;
+}
+
+// sv(p) = RN(e(p) * S) and inv(p) = RN(1/sv(p)) for every pattern p (0 for p = 0 and 127).
+__device__ __forceinline__ void build_scale_table(float S, float* s_sv, float* s_inv) {
+    for (int p = threadIdx.x; p < 128; p += blockDim.x) {
+        const float sv = (p == 0 || p == 127) ? 0.0f : __fmul_rn(e4m3_value(p), S);
+        s_sv[p] = sv;
+        s_inv[p] = sv == 0.0f ? 0.0f : __frcp_rn(sv);
+    }
+    __syncthreads();
+}
+
+// Load the 16 elements of one NVFP4 block as 8 float pairs (element 2k, 2k+1).
+template <int IN>
+__device__ __forceinline__ void load_block16(const void* xv, int64_t off, u64 (&xp)[8]) {
+    if (IN == FP4Q_IN_BF16) {
+        const uint4* p = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(xv) + off);
+        const uint4 a = __ldg(p), b = __ldg(p + 1);
+        xp[0] = bf16x2_to_pair(a.x); xp[1] = bf16x2_to_pair(a.y);
+        xp[2] = bf16x2_to_pair(a.z); xp[3] = bf16x2_to_pair(a.w);
+        xp[4] = bf16x2_to_pair(b.x); xp[5] = bf16x2_to_pair(b.y);
+        xp[6] = bf16x2_to_pair(b.z); xp[7] = bf16x2_to_pair(b.w);
+    } else {
+        const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(xv) + off);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float4 v = __ldg(p + j);
+            xp[2 * j] = pk(v.x, v.y);
+            xp[2 * j + 1] = pk(v.z, v.w);
+        }
+    }
+}
+
+__device__ __forceinline__ float block_absmax(const u64 (&xp)[8]) {
+    float m = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        float a, b;
+        upk(xp[j], a, b);
+        m = fmaxf(m, fmaxf(fabsf(a), fabsf(b)));
+    }
+    return m;
+}
+
+// Error of one candidate (sv, inv): residual d = fma(-q, sv, x) per element; squares summed
+// by fma into an (even, odd) pair of accumulators; result RN(even + odd).
+template <bool WEIGHTED>
+__device__ __forceinline__ float candidate_error(const u64 (&xp)[8], const u64 (&wp)[8], float sv, float inv) {
+    const u64 inv2 = pk(inv, inv), nsv2 = pk(-sv, -sv);
+    u64 acc = pk(0.0f, 0.0f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const u64 y = mul2(xp[j], inv2);
+        const u64 g = e2m1x2_decode(e2m1x2(y));
+        const u64 d = fma2(g, nsv2, xp[j]);
+        if (WEIGHTED) acc = fma2(mul2(wp[j], d), d, acc);
+        else acc = fma2(d, d, acc);
+    }
+    float a, b;
+    upk(acc, a, b);
+    return __fadd_rn(a, b);
+}
+
+// Packed codes of a block for a given reciprocal scale (8 bytes: elements 0..15).
+__device__ __forceinline__ uint2 block_codes(const u64 (&xp)[8], float inv) {
+    const u64 inv2 = pk(inv, inv);
+    uint32_t c[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) c[j] = e2m1x2(mul2(xp[j], inv2));
+    return make_uint2(c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24),
+                      c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24));
+}
+
+// ------------------------------------------------------------------------------------------
+// NVFP4: AbsMax / 4-over-6 / ScaleSweep MSE / ScaleSweep WMSE
+// ------------------------------------------------------------------------------------------
+template <int IN, int OBJ>
+__global__ void __launch_bounds__(kThreads) nvfp4_kernel(const void* __restrict__ xv, int64_t rows, int64_t cols,
+                                                         int64_t ld, const float* __restrict__ imp,
+                                                         uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                                                         const float* __restrict__ gscale, uint32_t* __restrict__ ws,
+                                                         int s_given) {
+    __shared__ float s_sv[128], s_inv[128];
+    const Setup su = read_setup(gscale);
+    build_scale_table(su.S, s_sv, s_inv);
+    const float S = su.S;
+    const float d6 = __fmul_rn(6.0f, S), d4 = __fmul_rn(4.0f, S);
+    const int64_t nb = cols / 16;
+    const int64_t total = rows * nb;
+    const int64_t step = (int64_t)gridDim.x * blockDim.x;
+    constexpr int LO = OBJ == FP4Q_SWEEP_MSE ? -3 : (OBJ == FP4Q_SWEEP_WMSE ? -8 : 0);
+    constexpr int HI = (OBJ == FP4Q_SWEEP_MSE || OBJ == FP4Q_SWEEP_WMSE) ? 7 : 0;
+    constexpr bool WEIGHTED = OBJ == FP4Q_SWEEP_WMSE;
+
+    for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < total; blk += step) {
+        const int64_t r = blk / nb, b = blk - r * nb;
+        uint2* cdst = reinterpret_cast<uint2*>(codes + r * (cols / 2) + b * 8);
+        if (su.flags) {   // data out of contract: zero-filled outputs
+            *cdst = make_uint2(0u, 0u);
+            scales[blk] = 0;
+            continue;
+        }
+        u64 xp[8];
+        load_block16<IN>(xv, r * ld + b * 16, xp);
+        int bp = 0;
+        if (S > 0.0f) {
+            const float ab = block_absmax(xp);
+            const int p0 = e4m3_rne(__fdiv_rn(ab, d6));
+            bp = p0;
+            if (OBJ == FP4Q_FOUR_OVER_SIX) {
+                const int p4 = e4m3_rne(__fdiv_rn(ab, d4));
+                if (p4 != p0) {
+                    u64 wp[8];
+                    const float e0 = candidate_error<false>(xp, wp, s_sv[p0], s_inv[p0]);
+                    const float e4 = candidate_error<false>(xp, wp, s_sv[p4], s_inv[p4]);
+                    if (e4 < e0) bp = p4;
+                }
+            } else if (OBJ == FP4Q_SWEEP_MSE || OBJ == FP4Q_SWEEP_WMSE) {
+                u64 wp[8];
+                if (WEIGHTED) {
+                    const float4* w4 = reinterpret_cast<const float4*>(imp + b * 16);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float4 v = __ldg(w4 + j);
+                        wp[2 * j] = pk(v.x, v.y);
+                        wp[2 * j + 1] = pk(v.z, v.w);
+                    }
+                }
+                float best = INFINITY;
+                bp = max(p0 + LO, 0);
+#pragma unroll 1
+                for (int k = LO; k <= HI; ++k) {
+                    const int p = p0 + k;
+                    const bool valid = (unsigned)p <= 126u;
+                    const int pc = valid ? p : 0;
+                    const float e = candidate_error<WEIGHTED>(xp, wp, s_sv[pc], s_inv[pc]);
+                    if (valid && e < best) {
+                        best = e;
+                        bp = p;
+                    }
+                }
+            }
+        }
+        *cdst = block_codes(xp, s_inv[bp]);
+        scales[blk] = (uint8_t)bp;
+    }
+    finish_status(ws, su.flags, WS_CNT_Q);
+}
+
+// ------------------------------------------------------------------------------------------
+// IF4
+// ------------------------------------------------------------------------------------------
+template <int IN>
+__global__ void __launch_bounds__(kThreads) if4_kernel(const void* __restrict__ xv, int64_t rows, int64_t cols,
+                                                       int64_t ld, uint8_t* __restrict__ codes,
+                                                       uint8_t* __restrict__ scales, const float* __restrict__ gscale,
+                                                       uint32_t* __restrict__ ws, int s_given) {
+    __shared__ float s_sv[128], s_inv[128];
+    const Setup su = read_setup(gscale);
+    build_scale_table(su.S, s_sv, s_inv);
+    const float S = su.S;
+    const float d6 = __fmul_rn(6.0f, S);
+    const float K76 = __fdiv_rn(7.0f, 6.0f), K67 = __fdiv_rn(6.0f, 7.0f);
+    const u64 k76 = pk(K76, K76), k67 = pk(K67, K67);
+    const int64_t nb = cols / 16;
+    const int64_t total = rows * nb;
+    const int64_t step = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < total; blk += step) {
+        const int64_t r = blk / nb, b = blk - r * nb;
+        uint2* cdst = reinterpret_cast<uint2*>(codes + r * (cols / 2) + b * 8);
+        if (su.flags) {
+            *cdst = make_uint2(0u, 0u);
+            scales[blk] = 0;
+            continue;
+        }
+        u64 xp[8];
+        load_block16<IN>(xv, r * ld + b * 16, xp);
+        const int p0 = S > 0.0f ? e4m3_rne(__fdiv_rn(block_absmax(xp), d6)) : 0;
+        const float sv = s_sv[p0], inv = s_inv[p0];
+        const u64 inv2 = pk(inv, inv), nsv2 = pk(-sv, -sv);
+        u64 accf = pk(0.0f, 0.0f), acci = pk(0.0f, 0.0f);
+        uint32_t cf[8], ci[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const u64 y = mul2(xp[j], inv2);
+            cf[j] = e2m1x2(y);
+            const u64 df = fma2(e2m1x2_decode(cf[j]), nsv2, xp[j]);
+            accf = fma2(df, df, accf);
+            float z0, z1;
+            upk(mul2(y, k76), z0, z1);
+            float n0, n1;
+            asm("cvt.rni.f32.f32 %0, %1;" : "=f"(n0) : "f"(z0));
+            asm("cvt.rni.f32.f32 %0, %1;" : "=f"(n1) : "f"(z1));
+            n0 = fminf(fmaxf(n0, -7.0f), 7.0f);
+            n1 = fminf(fmaxf(n1, -7.0f), 7.0f);
+            const u64 di = fma2(mul2(pk(n0, n1), k67), nsv2, xp[j]);
+            acci = fma2(di, di, acci);
+            ci[j] = ((uint32_t)__float2int_rn(n0) & 0xFu) | (((uint32_t)__float2int_rn(n1) & 0xFu) << 4);
+        }
+        float a, c;
+        upk(accf, a, c);
+        const float ef = __fadd_rn(a, c);
+        upk(acci, a, c);
+        const float ei = __fadd_rn(a, c);
+        const bool use_int = ei < ef;
+        const uint32_t* cc = use_int ? ci : cf;
+        *cdst = make_uint2(cc[0] | (cc[1] << 8) | (cc[2] << 16) | (cc[3] << 24),
+                           cc[4] | (cc[5] << 8) | (cc[6] << 16) | (cc[7] << 24));
+        scales[blk] = (uint8_t)(p0 | (use_int ? 0x80 : 0));
+    }
+    finish_status(ws, su.flags, WS_CNT_Q);
+}
+
+// ------------------------------------------------------------------------------------------
+// MXFP4 (+ 32-point Hadamard)
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ void fwht32(float (&v)[32]) {
+#pragma unroll
+    for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            if ((j & h) == 0) {
+                const float a = v[j], b = v[j + h];
+                v[j] = __fadd_rn(a, b);
+                v[j + h] = __fsub_rn(a, b);
+            }
+        }
+    }
+    const float KH = (float)0.17677669529663688110021109052621;   // RN(1/sqrt(32))
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __fmul_rn(v[j], KH);
+}
+
+// Smallest e with a <= 6*2^e (ceil rule) or floor(log2 a) - 2 (OCP rule), clamped to [-127,127].
+__device__ __forceinline__ int mx_exponent(float a, bool ocp) {
+    if (a == 0.0f) return -127;
+    int sh = 0;
+    if (a < 0x1p-126f) { a = __fmul_rn(a, 0x1p24f); sh = 24; }   // exact rescale of subnormals
+    const uint32_t u = __float_as_uint(a);
+    const int k = (int)(u >> 23) - 127 - sh;                     // floor(log2 a)
+    int e = ocp ? k - 2 : (k - 2 + ((u & 0x7FFFFFu) > 0x400000u ? 1 : 0));
+    return min(max(e, -127), 127);
+}
+
+template <int IN, bool HAD>
+__global__ void __launch_bounds__(kThreads) mxfp4_kernel(const void* __restrict__ xv, int64_t rows, int64_t cols,
+                                                         int64_t ld, uint8_t* __restrict__ codes,
+                                                         uint8_t* __restrict__ scales, uint32_t* __restrict__ ws,
+                                                         int ocp) {
+    const int64_t nb = cols / 32;
+    const int64_t total = rows * nb;
+    const int64_t step = (int64_t)gridDim.x * blockDim.x;
+    uint32_t flag = 0;
+    for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < total; blk += step) {
+        const int64_t r = blk / nb, b = blk - r * nb;
+        float v[32];
+        if (IN == FP4Q_IN_BF16) {
+            const uint4* p = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(xv) + r * ld + b * 32);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint4 w = __ldg(p + q);
+                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    v[q * 8 + 2 * t] = __uint_as_float(ww[t] << 16);
+                    v[q * 8 + 2 * t + 1] = __uint_as_float(ww[t] & 0xFFFF0000u);
+                }
+            }
+        } else {
+            const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(xv) + r * ld + b * 32);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float4 w = __ldg(p + q);
+                v[4 * q] = w.x; v[4 * q + 1] = w.y; v[4 * q + 2] = w.z; v[4 * q + 3] = w.w;
+            }
+        }
+        bool bad = false;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) bad |= !isfinite(v[i]);
+        uint4* cdst = reinterpret_cast<uint4*>(codes + r * (cols / 2) + b * 16);
+        if (bad) {
+            flag = FP4Q_DEVSTAT_NONFINITE;
+            *cdst = make_uint4(0u, 0u, 0u, 0u);
+            scales[blk] = 0xFF;
+            continue;
+        }
+        if (HAD) fwht32(v);
+        float ab = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ab = fmaxf(ab, fabsf(v[i]));
+        const int e = mx_exponent(ab, ocp != 0);
+        const float m = pow2i(-e);
+        uint32_t c[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) c[j] = e2m1x2(__fmul_rn(v[2 * j], m), __fmul_rn(v[2 * j + 1], m));
+        *cdst = make_uint4(c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24),
+                           c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24),
+                           c[8] | (c[9] << 8) | (c[10] << 16) | (c[11] << 24),
+                           c[12] | (c[13] << 8) | (c[14] << 16) | (c[15] << 24));
+        scales[blk] = (uint8_t)(e + 127);
+    }
+    finish_status(ws, flag, WS_CNT_Q);
+}
+
+// ------------------------------------------------------------------------------------------
+// Dequantize
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t bf16_bits(float f) {
+    if (isnan(f)) return 0x7FC0u;
+    const uint32_t u = __float_as_uint(f);
+    return (u + 0x7FFFu + ((u >> 16) & 1u)) >> 16;
+}
+
+template <bool OUT_BF16, int N>
+__device__ __forceinline__ void store_values(void* out, int64_t off, const float (&v)[N]) {
+    if (OUT_BF16) {
+        uint4* p = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(out) + off);
+#pragma unroll
+        for (int q = 0; q < N / 8; ++q) {
+            uint32_t w[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) w[t] = bf16_bits(v[8 * q + 2 * t]) | (bf16_bits(v[8 * q + 2 * t + 1]) << 16);
+            p[q] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    } else {
+        float4* p = reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + off);
+#pragma unroll
+        for (int q = 0; q < N / 4; ++q) p[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    }
+}
+
+template <bool OUT_BF16, bool IF4>
+__global__ void __launch_bounds__(kThreads) dequant16_kernel(const uint8_t* __restrict__ codes,
+                                                             const uint8_t* __restrict__ scales,
+                                                             const float* __restrict__ gscale, int64_t rows,
+                                                             int64_t cols, void* __restrict__ out) {
+    const float S = *gscale;
+    const float K67 = __fdiv_rn(6.0f, 7.0f);
+    const int64_t nb = cols / 16;
+    const int64_t total = rows * nb;
+    const int64_t step = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < total; blk += step) {
+        const int64_t r = blk / nb, b = blk - r * nb;
+        const uint2 c = __ldg(reinterpret_cast<const uint2*>(codes + r * (cols / 2) + b * 8));
+        const uint32_t sb = __ldg(scales + blk);
+        const int p = sb & 0x7F;
+        const float sv = p == 0 ? 0.0f : (p == 127 ? __uint_as_float(0x7FC00000u) : __fmul_rn(e4m3_value(p), S));
+        float v[16];
+        const uint32_t cw[2] = {c.x, c.y};
+        if (IF4 && (sb & 0x80)) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int nib = (cw[i >> 3] >> ((i & 7) * 4)) & 0xF;
+                const int n = nib >= 8 ? nib - 16 : nib;
+                v[i] = __fmul_rn(__fmul_rn((float)n, K67), sv);
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                float g0, g1;
+                e2m1x2_decode((cw[j >> 2] >> ((j & 3) * 8)) & 0xFFu, g0, g1);
+                v[2 * j] = __fmul_rn(g0, sv);
+                v[2 * j + 1] = __fmul_rn(g1, sv);
+            }
+        }
+        store_values<OUT_BF16>(out, r * cols + b * 16, v);
+    }
+}
+
+template <bool OUT_BF16, bool HAD>
+__global__ void __launch_bounds__(kThreads) dequant_mx_kernel(const uint8_t* __restrict__ codes,
+                                                              const uint8_t* __restrict__ scales, int64_t rows,
+                                                              int64_t cols, void* __restrict__ out) {
+    const int64_t nb = cols / 32;
+    const int64_t total = rows * nb;
+    const int64_t step = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < total; blk += step) {
+        const int64_t r = blk / nb, b = blk - r * nb;
+        const uint4 c = __ldg(reinterpret_cast<const uint4*>(codes + r * (cols / 2) + b * 16));
+        const uint32_t sb = __ldg(scales + blk);
+        const float m = sb == 0xFFu ? __uint_as_float(0x7FC00000u) : pow2i((int)sb - 127);
+        const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            float g0, g1;
+            e2m1x2_decode((cw[j >> 2] >> ((j & 3) * 8)) & 0xFFu, g0, g1);
+            v[2 * j] = __fmul_rn(g0, m);
+            v[2 * j + 1] = __fmul_rn(g1, m);
+        }
+        if (HAD) fwht32(v);
+        store_values<OUT_BF16>(out, r * cols + b * 32, v);
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// Host side
+// ------------------------------------------------------------------------------------------
+thread_local int g_launches = 0;
+
+int grid_for(int64_t work_items, int ctas_per_sm) {
+    static int sms = 0;
+    if (sms == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) sms = 148;
+    }
+    const int64_t need = (work_items + kThreads - 1) / kThreads;
+    const int64_t cap = (int64_t)sms * ctas_per_sm;
+    return (int)(need < cap ? (need > 0 ? need : 1) : cap);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int launched(int n) {
+    g_launches = n;
+    return cudaGetLastError() == cudaSuccess ? FP4Q_OK : FP4Q_ERR_CUDA;
+}
+
+int check_common(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld, int B, const uint8_t* codes,
+                 const uint8_t* scales, const void* workspace) {
+    if (dtype != FP4Q_IN_F32 && dtype != FP4Q_IN_BF16) return FP4Q_ERR_INVALID_ARG;
+    if (rows < 0 || cols < 0 || ld < cols || cols % B) return FP4Q_ERR_SHAPE;
+    if (rows > 0 && cols > 0 && rows > ((int64_t)1 << 40) / cols) return FP4Q_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return FP4Q_OK;
+    if (!x || !codes || !scales || !workspace) return FP4Q_ERR_INVALID_ARG;
+    const int es = dtype == FP4Q_IN_BF16 ? 2 : 4;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(workspace) || (ld * es) % 16) return FP4Q_ERR_ALIGNMENT;
+    return FP4Q_OK;
+}
+
+template <int IN>
+int launch_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, int fmt, int obj, const float* imp,
+                    uint8_t* codes, uint8_t* scales, float* gs, uint32_t* ws, uint32_t flags, cudaStream_t st) {
+    int n = 0;
+    if (fmt == FP4Q_MXFP4) {
+        const int ocp = (flags & FP4Q_F_MX_OCP_FLOOR) ? 1 : 0;
+        mxfp4_kernel<IN, false><<<grid_for(rows * (cols / 32), 8), kThreads, 0, st>>>(x, rows, cols, ld, codes,
+                                                                                   scales, ws, ocp);
+        return launched(1);
+    }
+    const int given = (flags & FP4Q_F_GLOBAL_SCALE_GIVEN) ? 1 : 0;
+    if (!given) {
+        const int64_t vecs = rows * cols * (IN == FP4Q_IN_BF16 ? 2 : 4) / 16;
+        amax_kernel<IN><<<grid_for(vecs, 8), kThreads, 0, st>>>(x, rows, cols, ld, ws, gs, 0);
+        ++n;
+    }
+    const int g = grid_for(rows * (cols / 16), 8);
+    if (fmt == FP4Q_IF4) {
+        if4_kernel<IN><<<g, kThreads, 0, st>>>(x, rows, cols, ld, codes, scales, gs, ws, given);
+    } else {
+        switch (obj) {
+            case FP4Q_ABSMAX:
+                nvfp4_kernel<IN, FP4Q_ABSMAX><<<g, kThreads, 0, st>>>(x, rows, cols, ld, imp, codes, scales, gs, ws, given);
+                break;
+            case FP4Q_FOUR_OVER_SIX:
+                nvfp4_kernel<IN, FP4Q_FOUR_OVER_SIX><<<g, kThreads, 0, st>>>(x, rows, cols, ld, imp, codes, scales, gs, ws,
+                                                                          given);
+                break;
+            case FP4Q_SWEEP_MSE:
+                nvfp4_kernel<IN, FP4Q_SWEEP_MSE><<<g, kThreads, 0, st>>>(x, rows, cols, ld, imp, codes, scales, gs, ws,
+                                                                      given);
+                break;
+            default:
+                nvfp4_kernel<IN, FP4Q_SWEEP_WMSE><<<g, kThreads, 0, st>>>(x, rows, cols, ld, imp, codes, scales, gs, ws,
+                                                                       given);
+                break;
+        }
+    }
+    return launched(n + 1);
+}
+
+}  // namespace fp4q
+
+using namespace fp4q;
+
+extern "C" {
+
+size_t fp4q_workspace_bytes(void) { return kWorkspaceBytes; }
+
+int fp4q_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld, int fmt, int objective,
+                  const float* importance, uint8_t* codes, uint8_t* scales, float* global_scale, void* workspace,
+                  uint32_t flags, void* stream) {
+    g_launches = 0;
+    if (fmt != FP4Q_NVFP4 && fmt != FP4Q_IF4 && fmt != FP4Q_MXFP4) return FP4Q_ERR_INVALID_ARG;
+    if (flags & ~(FP4Q_F_GLOBAL_SCALE_GIVEN | FP4Q_F_MX_OCP_FLOOR)) return FP4Q_ERR_INVALID_ARG;
+    if (fmt == FP4Q_NVFP4 && (objective < FP4Q_ABSMAX || objective > FP4Q_SWEEP_WMSE)) return FP4Q_ERR_INVALID_ARG;
+    const int B = fmt == FP4Q_MXFP4 ? 32 : 16;
+    int rc = check_common(x, dtype, rows, cols, ld, B, codes, scales, workspace);
+    if (rc != FP4Q_OK || rows == 0 || cols == 0) return rc;
+    if (fmt != FP4Q_MXFP4 && !global_scale) return FP4Q_ERR_INVALID_ARG;
+    if (fmt == FP4Q_NVFP4 && objective == FP4Q_SWEEP_WMSE) {
+        if (!importance) return FP4Q_ERR_INVALID_ARG;
+        if (!aligned16(importance)) return FP4Q_ERR_ALIGNMENT;
+    }
+    if (fmt == FP4Q_MXFP4 && (flags & FP4Q_F_GLOBAL_SCALE_GIVEN)) return FP4Q_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t* ws = reinterpret_cast<uint32_t*>(workspace);
+    if (dtype == FP4Q_IN_BF16)
+        return launch_quantize<FP4Q_IN_BF16>(x, rows, cols, ld, fmt, objective, importance, codes, scales, global_scale,
+                                             ws, flags, st);
+    return launch_quantize<FP4Q_IN_F32>(x, rows, cols, ld, fmt, objective, importance, codes, scales, global_scale, ws,
+                                        flags, st);
+}
+
+int fp4q_global_scale(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld, float* global_scale,
+                      void* workspace, void* stream) {
+    g_launches = 0;
+    if (dtype != FP4Q_IN_F32 && dtype != FP4Q_IN_BF16) return FP4Q_ERR_INVALID_ARG;
+    const int es = dtype == FP4Q_IN_BF16 ? 2 : 4;
+    if (rows < 0 || cols < 0 || ld < cols || (cols * es) % 16) return FP4Q_ERR_SHAPE;
+    if (rows > 0 && cols > 0 && rows > ((int64_t)1 << 40) / cols) return FP4Q_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return FP4Q_OK;
+    if (!x || !global_scale || !workspace) return FP4Q_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(workspace) || (ld * es) % 16) return FP4Q_ERR_ALIGNMENT;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t* ws = reinterpret_cast<uint32_t*>(workspace);
+    const int64_t vecs = rows * cols * (dtype == FP4Q_IN_BF16 ? 2 : 4) / 16;
+    if (dtype == FP4Q_IN_BF16)
+        amax_kernel<FP4Q_IN_BF16><<<grid_for(vecs, 8), kThreads, 0, st>>>(x, rows, cols, ld, ws, global_scale, 1);
+    else
+        amax_kernel<FP4Q_IN_F32><<<grid_for(vecs, 8), kThreads, 0, st>>>(x, rows, cols, ld, ws, global_scale, 1);
+    return launched(1);
+}
+
+int fp4q_hadamard_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld, int had_size,
+                           uint8_t* codes, uint8_t* scales, void* workspace, uint32_t flags, void* stream) {
+    g_launches = 0;
+    if (had_size != 32) return FP4Q_ERR_UNSUPPORTED;
+    if (flags & ~FP4Q_F_MX_OCP_FLOOR) return FP4Q_ERR_INVALID_ARG;
+    int rc = check_common(x, dtype, rows, cols, ld, 32, codes, scales, workspace);
+    if (rc != FP4Q_OK || rows == 0 || cols == 0) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t* ws = reinterpret_cast<uint32_t*>(workspace);
+    const int ocp = (flags & FP4Q_F_MX_OCP_FLOOR) ? 1 : 0;
+    const int g = grid_for(rows * (cols / 32), 8);
+    if (dtype == FP4Q_IN_BF16)
+        mxfp4_kernel<FP4Q_IN_BF16, true><<<g, kThreads, 0, st>>>(x, rows, cols, ld, codes, scales, ws, ocp);
+    else
+        mxfp4_kernel<FP4Q_IN_F32, true><<<g, kThreads, 0, st>>>(x, rows, cols, ld, codes, scales, ws, ocp);
+    return launched(1);
+}
+
+int fp4q_dequantize(const uint8_t* codes, const uint8_t* scales, const float* global_scale, int64_t rows,
+                    int64_t cols, int fmt, int inverse_hadamard, void* out, uint32_t flags, void* stream) {
+    g_launches = 0;
+    if (fmt != FP4Q_NVFP4 && fmt != FP4Q_IF4 && fmt != FP4Q_MXFP4) return FP4Q_ERR_INVALID_ARG;
+    if (flags & ~FP4Q_F_OUT_BF16) return FP4Q_ERR_INVALID_ARG;
+    if (inverse_hadamard && fmt != FP4Q_MXFP4) return FP4Q_ERR_UNSUPPORTED;
+    const int B = fmt == FP4Q_MXFP4 ? 32 : 16;
+    if (rows < 0 || cols < 0 || cols % B) return FP4Q_ERR_SHAPE;
+    if (rows > 0 && cols > 0 && rows > ((int64_t)1 << 40) / cols) return FP4Q_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return FP4Q_OK;
+    if (!codes || !scales || !out || (fmt != FP4Q_MXFP4 && !global_scale)) return FP4Q_ERR_INVALID_ARG;
+    if (!aligned16(codes) || !aligned16(out)) return FP4Q_ERR_ALIGNMENT;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const bool bf = (flags & FP4Q_F_OUT_BF16) != 0;
+    const int g = grid_for(rows * (cols / B), 8);
+    if (fmt == FP4Q_MXFP4) {
+        if (bf && inverse_hadamard) dequant_mx_kernel<true, true><<<g, kThreads, 0, st>>>(codes, scales, rows, cols, out);
+        else if (bf) dequant_mx_kernel<true, false><<<g, kThreads, 0, st>>>(codes, scales, rows, cols, out);
+        else if (inverse_hadamard) dequant_mx_kernel<false, true><<<g, kThreads, 0, st>>>(codes, scales, rows, cols, out);
+        else dequant_mx_kernel<false, false><<<g, kThreads, 0, st>>>(codes, scales, rows, cols, out);
+    } else if (fmt == FP4Q_IF4) {
+        if (bf) dequant16_kernel<true, true><<<g, kThreads, 0, st>>>(codes, scales, global_scale, rows, cols, out);
+        else dequant16_kernel<false, true><<<g, kThreads, 0, st>>>(codes, scales, global_scale, rows, cols, out);
+    } else {
+        if (bf) dequant16_kernel<true, false><<<g, kThreads, 0, st>>>(codes, scales, global_scale, rows, cols, out);
+        else dequant16_kernel<false, false><<<g, kThreads, 0, st>>>(codes, scales, global_scale, rows, cols, out);
+    }
+    return launched(1);
+}
+
+int fp4q_read_device_status(const void* workspace, uint32_t* status, void* stream) {
+    if (!workspace || !status) return FP4Q_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(status, workspace, sizeof(uint32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return FP4Q_ERR_CUDA;
+    return cudaStreamSynchronize(st) == cudaSuccess ? FP4Q_OK : FP4Q_ERR_CUDA;
+}
+
+int fp4q_last_launch_count(void) { return g_launches; }
+
+const char* fp4q_status_string(int s) {
+    switch (s) {
+        case FP4Q_OK: return "ok";
+        case FP4Q_ERR_INVALID_ARG: return "invalid argument";
+        case FP4Q_ERR_SHAPE: return "invalid shape";
+        case FP4Q_ERR_ALIGNMENT: return "misaligned pointer or row pitch (16 bytes required)";
+        case FP4Q_ERR_UNSUPPORTED: return "unsupported combination";
+        case FP4Q_ERR_CUDA: return "CUDA launch or runtime error";
+        default: return "unknown status";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,150 @@
+/*
+ * fp4q.h -- C ABI of libfp4q: block-scaled FP4 quantization on NVIDIA B200 (sm_100a).
+ *
+ * Formats and methods (each entry point cites the passage that defines what it computes):
+ *   NVFP4  16-element blocks of E2M1 codes {0,.5,1,1.5,2,3,4,6} with one E4M3 scale per
+ *          block and one FP32 scale S per tensor.  S = max|x| / (256*6) and the ScaleSweep
+ *          search over E4M3 bit-pattern offsets [-3,+7] (MSE) or [-8,+7] (WMSE):
+ *          ScaleSweep (gist.science/ko/paper/2606.07618), "Methodology".  AbsMax is the
+ *          base scale itself; 4/6 (max->6 or max->4, lower MSE): Adaptive Block-Scaled Data
+ *          Types (gist.science/ko/paper/2603.28765), "Problem".
+ *   IF4    NVFP4 layout; per block the lower-MSE of FP4 and scaled INT4 (x 7/6 before
+ *          rounding, x 6/7 on dequantization), flagged in the scale byte's sign bit
+ *          (1 = INT4): Adaptive Block-Scaled Data Types, "Methodology", IF4 structure.
+ *   MXFP4  32-element blocks of E2M1 codes with an E8M0 (power-of-two) scale, optionally
+ *          after a normalized 32-point block Hadamard rotation: Bridging the Gap ...
+ *          Microscaling FP4 (gist.science/ko/paper/2509.23202), "Methodology"; scale rule
+ *          "block maximum onto the largest codeword": TORQ (gist.science/ko/paper/
+ *          2605.19561), "Method", S-step.
+ *
+ * Arithmetic (identical on every path; every step one binary32 operation rounded to
+ * nearest even, no contraction, no flush-to-zero):
+ *   S = RN(amax/1536); p0 = E4M3_RNE(RN(a_b / RN(6 S))); p4 = E4M3_RNE(RN(a_b / RN(4 S)));
+ *   candidate p: sv = RN(e(p) S), inv = RN(1/sv) (sv = inv = 0 for p = 0);
+ *   y = RN(x inv); q = E2M1_RNE_satfinite(y); d = fma(-q, sv, x);
+ *   error = RN(acc_even + acc_odd), acc_par = fma(d, d, acc_par) over the block's even /
+ *   odd positions in order (WMSE: fma(RN(w d), d, acc)); the lowest offset wins a tie.
+ *   IF4 INT4: z = RN(y RN(7/6)), n = clamp(rint(z), -7, 7), v = RN(n RN(6/7)),
+ *   d = fma(-v, sv, x); INT4 iff its error is strictly lower.
+ *   MXFP4: e = smallest integer with a_b <= 6 * 2^e (flag FP4Q_F_MX_OCP_FLOOR: floor(log2
+ *   a_b) - 2), clamped to [-127,127]; y = RN(x 2^-e).
+ *
+ * Memory layout (all device memory, row-major, owned and allocated by the caller):
+ *   x        [rows][ld] bf16 or fp32; ld >= cols elements; x and the row pitch (ld * element
+ *            size) 16-byte aligned.
+ *   codes    [rows][cols/2] bytes; element 2k in the low nibble of byte k, 2k+1 in the high
+ *            nibble; nibble = sign << 3 | E2M1 magnitude index (IF4 INT4 blocks: 4-bit two's
+ *            complement of n).  16-byte aligned; cols/2 bytes per row, no padding.
+ *   scales   [rows][cols/B] bytes, B = 16 (NVFP4/IF4: E4M3 pattern, IF4 indicator in bit 7)
+ *            or 32 (MXFP4: E8M0 byte e+127, 0xFF marks a block with a non-finite input).
+ *   global_scale  one float (NVFP4/IF4): written with S, or read when
+ *            FP4Q_F_GLOBAL_SCALE_GIVEN is set.
+ *   workspace fp4q_workspace_bytes() bytes, 16-byte aligned, ZERO-FILLED ONCE by the caller
+ *            before its first use; every call leaves it zeroed again except word 0.  Word 0
+ *            (uint32) receives the device status (FP4Q_DEVSTAT_*) of the most recent call that
+ *            used it.  One workspace must not be shared by calls that may run concurrently.
+ *
+ * Errors: argument, shape and alignment problems are detected on the host before anything
+ * is launched and returned as fp4q_status; a failed launch returns FP4Q_ERR_CUDA.  Data
+ * conditions (a non-finite input, or a tensor scale S outside [2^-117, 2^125/1536]) are found
+ * on the device: the outputs of that call are zero-filled and the device status word is
+ * set; no call synchronizes the host, and no kernel traps.  Calls are asynchronous on
+ * `stream` (a cudaStream_t; NULL = the legacy default stream).
+ */
+#ifndef FP4Q_H
+#define FP4Q_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FP4Q_OK = 0,
+    FP4Q_ERR_INVALID_ARG = 1,   /* null pointer, unknown enum value, bad flag combination */
+    FP4Q_ERR_SHAPE = 2,         /* rows/cols/ld out of range or cols not a multiple of B    */
+    FP4Q_ERR_ALIGNMENT = 3,     /* a pointer or the row pitch is not 16-byte aligned        */
+    FP4Q_ERR_UNSUPPORTED = 4,   /* combination the library does not implement                */
+    FP4Q_ERR_CUDA = 5           /* a CUDA launch or runtime call failed                      */
+} fp4q_status;
+
+enum { FP4Q_DEVSTAT_OK = 0, FP4Q_DEVSTAT_NONFINITE = 1, FP4Q_DEVSTAT_RANGE = 2 };
+enum { FP4Q_IN_F32 = 0, FP4Q_IN_BF16 = 1 };
+enum { FP4Q_NVFP4 = 0, FP4Q_IF4 = 1, FP4Q_MXFP4 = 2 };
+enum { FP4Q_ABSMAX = 0, FP4Q_FOUR_OVER_SIX = 1, FP4Q_SWEEP_MSE = 2, FP4Q_SWEEP_WMSE = 3 };
+
+#define FP4Q_F_GLOBAL_SCALE_GIVEN 0x1u  /* quantize: read S from *global_scale (no amax pass) */
+#define FP4Q_F_MX_OCP_FLOOR       0x2u  /* MXFP4: e = floor(log2 a_b) - 2 instead of the ceil rule */
+#define FP4Q_F_OUT_BF16           0x4u  /* dequantize: write bf16 (RNE of the fp32 value)     */
+
+/* Size in bytes of the workspace every quantize call needs (a small constant). */
+size_t fp4q_workspace_bytes(void);
+
+/*
+ * Quantize x into codes + scales (+ S).
+ *   fmt FP4Q_NVFP4 with objective FP4Q_ABSMAX / FP4Q_FOUR_OVER_SIX / FP4Q_SWEEP_MSE /
+ *   FP4Q_SWEEP_WMSE (importance: device float[cols], one non-negative finite weight per
+ *   column, required for WMSE and ignored otherwise); fmt FP4Q_IF4 (objective ignored);
+ *   fmt FP4Q_MXFP4 (objective, importance and global_scale ignored; see also
+ *   fp4q_hadamard_quantize).
+ *   rows >= 0, cols a multiple of 16 (32 for MXFP4), ld >= cols; rows*cols < 2^40.
+ *   flags: FP4Q_F_GLOBAL_SCALE_GIVEN (NVFP4/IF4), FP4Q_F_MX_OCP_FLOOR (MXFP4).
+ * Launches: NVFP4/IF4 without a given S: an amax kernel then the quantize kernel;
+ * otherwise one kernel.  Empty tensors launch nothing.
+ */
+int fp4q_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                  int fmt, int objective, const float* importance,
+                  uint8_t* codes, uint8_t* scales, float* global_scale,
+                  void* workspace, uint32_t flags, void* stream);
+
+/*
+ * Tensor scale only: S = RN(max|x| / 1536) written to *global_scale (device float), the
+ * ScaleSweep global scale S = max|x|/(256*6) (ScaleSweep, gist.science/ko/paper/2606.07618,
+ * "Methodology").  A non-finite element gives S = NaN.  The workspace status word receives
+ * FP4Q_DEVSTAT_NONFINITE (S = NaN) or FP4Q_DEVSTAT_RANGE (S outside [2^-117, 2^125/1536]).
+ * Passing the result to fp4q_quantize with FP4Q_F_GLOBAL_SCALE_GIVEN performs exactly the
+ * work of a call without the flag.  cols * element size must be a multiple of 16 bytes.
+ */
+int fp4q_global_scale(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                      float* global_scale, void* workspace, void* stream);
+
+/*
+ * MXFP4 quantization of H x: each 32-element block (along the contiguous dimension) is
+ * rotated by the normalized Sylvester Hadamard matrix H_32 / sqrt(32) before the E8M0 scale
+ * and the E2M1 codes are chosen (Bridging the Gap ... Microscaling FP4, "Methodology",
+ * block-wise Hadamard transforms).  had_size must be 32.  The transform is computed as the
+ * fast Walsh-Hadamard butterflies h = 1, 2, 4, 8, 16 followed by one multiplication by
+ * RN(1/sqrt(32)).  Same layout, alignment and error rules as fp4q_quantize with
+ * fmt = FP4Q_MXFP4.  Dequantized values are in the rotated domain.
+ */
+int fp4q_hadamard_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                           int had_size, uint8_t* codes, uint8_t* scales,
+                           void* workspace, uint32_t flags, void* stream);
+
+/*
+ * Dequantize codes + scales (+ S for NVFP4/IF4) into out [rows][cols], fp32 or (flag
+ * FP4Q_F_OUT_BF16) bf16.  NVFP4: RN(q * RN(e(p) S)); IF4 blocks with bit 7 set:
+ * RN(RN(n RN(6/7)) * RN(e(p) S)); MXFP4: RN(q * 2^(byte-127)) (byte 0xFF gives NaN).
+ * inverse_hadamard (MXFP4 only): apply the same normalized 32-point transform to each
+ * dequantized block (it is its own inverse up to rounding).  global_scale is a device
+ * pointer (ignored for MXFP4).  out must be 16-byte aligned.
+ */
+int fp4q_dequantize(const uint8_t* codes, const uint8_t* scales, const float* global_scale,
+                    int64_t rows, int64_t cols, int fmt, int inverse_hadamard,
+                    void* out, uint32_t flags, void* stream);
+
+/* Copy the device status word of `workspace` to *status (blocks until `stream` is done). */
+int fp4q_read_device_status(const void* workspace, uint32_t* status, void* stream);
+
+/* Number of kernel launches the most recent successful call on this thread issued. */
+int fp4q_last_launch_count(void);
+
+/* Static description of a status code. */
+const char* fp4q_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FP4Q_H */

@@ -46,6 +46,8 @@ def lib():
         L.fp4q_o_e2m1_encode.argtypes = [C.c_float]
         L.fp4q_o_global_scale.restype = C.c_float
         L.fp4q_o_global_scale.argtypes = [C.c_float]
+        L.fp4q_o_tensor_scale.restype = C.c_int
+        L.fp4q_o_tensor_scale.argtypes = [P, i64, i64, i64, P]
         L.fp4q_o_mx_exponent.restype = C.c_int
         L.fp4q_o_mx_exponent.argtypes = [C.c_float, C.c_int]
         L.fp4q_o_hadamard32.restype = None
@@ -92,6 +94,14 @@ def e2m1_encode(y: float) -> int:
 
 def global_scale(amax: float) -> float:
     return lib().fp4q_o_global_scale(float(amax))
+
+
+def tensor_scale(x):
+    """(S, status) of a whole float32 tensor: S = RN(max|x| / 1536)."""
+    x = _f32(x)
+    S = np.zeros(1, np.float32)
+    st = lib().fp4q_o_tensor_scale(_p(x), x.shape[0], x.shape[1], x.shape[1], _p(S))
+    return float(S[0]), st
 
 
 def mx_exponent(a: float, ocp_floor: bool = False) -> int:

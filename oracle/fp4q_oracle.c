@@ -141,6 +141,17 @@ static int scale_range_ok(float S)
     return S >= ldexpf(1.0f, -117) && S <= ldexpf(1.0f, 125) / 1536.0f;
 }
 
+/* S of a whole tensor (status ST_NONFINITE if any element is not finite). */
+int fp4q_o_tensor_scale(const float* x, int64_t rows, int64_t cols, int64_t ld, float* S)
+{
+    float amax;
+    int st = tensor_amax(x, rows, cols, ld, &amax);
+    *S = st == ST_OK ? fp4q_o_global_scale(amax) : NAN;
+    if (st == ST_OK && !scale_range_ok(*S)) st = ST_RANGE;
+    return st;
+}
+
+
 /* ------------------------------------------------------------------------------------
  * NVFP4 candidate evaluation
  * ---------------------------------------------------------------------------------- */
@@ -197,7 +208,6 @@ int fp4q_o_nvfp4_quantize(const float* x, int64_t rows, int64_t cols, int64_t ld
         float amax;
         status = tensor_amax(x, rows, cols, ld, &amax);
         S = status == ST_OK ? fp4q_o_global_scale(amax) : NAN;
-        if (status == ST_OK && !(amax <= ldexpf(1.0f, 125))) status = ST_RANGE;
         *S_io = S;
     }
     if (status == ST_OK && !scale_range_ok(S)) status = ST_RANGE;
@@ -275,7 +285,6 @@ int fp4q_o_if4_quantize(const float* x, int64_t rows, int64_t cols, int64_t ld,
         float amax;
         status = tensor_amax(x, rows, cols, ld, &amax);
         S = status == ST_OK ? fp4q_o_global_scale(amax) : NAN;
-        if (status == ST_OK && !(amax <= ldexpf(1.0f, 125))) status = ST_RANGE;
         *S_io = S;
     }
     if (status == ST_OK && !scale_range_ok(S)) status = ST_RANGE;

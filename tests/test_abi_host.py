@@ -1,0 +1,88 @@
+"""Host-side checks of the C-ABI library (no GPU needed): the library loads, exports every
+function include/fp4q.h declares, and rejects bad arguments before launching anything."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+import fp4_block_scaled_nvfp4_b200 as fq
+
+HDR = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "fp4q.h")
+
+
+def declared_functions():
+    src = open(HDR).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fp4q_\w+)\s*\(", src)))
+
+
+def test_header_declarations_match_binding():
+    assert declared_functions() == sorted(fq.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    L = fq.lib()
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings_and_workspace():
+    assert fq.status_string(0) == "ok"
+    for rc in range(1, 6):
+        assert fq.status_string(rc) and fq.status_string(rc) != "unknown status"
+    assert fq.status_string(99) == "unknown status"
+    assert fq.workspace_bytes() >= 16
+
+
+FAKE = 0x10000   # 16-byte aligned non-null stand-in; validation rejects before any use
+
+
+@pytest.mark.parametrize("args,rc", [
+    # x, dtype, rows, cols, ld, fmt, obj, imp, codes, scales, gs, ws, flags
+    ((FAKE, 1, 4, 24, 24, 0, 2, None, FAKE, FAKE, FAKE, FAKE, 0), fq.ERR_SHAPE),        # cols % 16
+    ((FAKE, 1, 4, 32, 16, 0, 2, None, FAKE, FAKE, FAKE, FAKE, 0), fq.ERR_SHAPE),        # ld < cols
+    ((FAKE, 1, -1, 32, 32, 0, 2, None, FAKE, FAKE, FAKE, FAKE, 0), fq.ERR_SHAPE),       # rows < 0
+    ((FAKE, 1, 4, 48, 48, 2, 0, None, FAKE, FAKE, None, FAKE, 0), fq.ERR_SHAPE),        # MX cols % 32
+    ((FAKE, 7, 4, 32, 32, 0, 2, None, FAKE, FAKE, FAKE, FAKE, 0), fq.ERR_INVALID_ARG),  # dtype
+    ((FAKE, 1, 4, 32, 32, 5, 2, None, FAKE, FAKE, FAKE, FAKE, 0), fq.ERR_INVALID_ARG),  # fmt
+    ((FAKE, 1, 4, 32, 32, 0, 9, None, FAKE, FAKE, FAKE, FAKE, 0), fq.ERR_INVALID_ARG),  # objective
+    ((FAKE, 1, 4, 32, 32, 0, 3, None, FAKE, FAKE, FAKE, FAKE, 0), fq.ERR_INVALID_ARG),  # WMSE w/o weights
+    ((None, 1, 4, 32, 32, 0, 2, None, FAKE, FAKE, FAKE, FAKE, 0), fq.ERR_INVALID_ARG),  # null x
+    ((FAKE, 1, 4, 32, 32, 0, 2, None, FAKE, FAKE, None, FAKE, 0), fq.ERR_INVALID_ARG),  # null S
+    ((FAKE, 1, 4, 32, 32, 0, 2, None, FAKE, FAKE, FAKE, None, 0), fq.ERR_INVALID_ARG),  # null workspace
+    ((FAKE + 8, 1, 4, 32, 32, 0, 2, None, FAKE, FAKE, FAKE, FAKE, 0), fq.ERR_ALIGNMENT),  # x misaligned
+    ((FAKE, 1, 4, 32, 36, 0, 2, None, FAKE, FAKE, FAKE, FAKE, 0), fq.ERR_ALIGNMENT),    # row pitch 72 B
+    ((FAKE, 1, 4, 32, 32, 0, 2, None, FAKE + 4, FAKE, FAKE, FAKE, 0), fq.ERR_ALIGNMENT),  # codes
+    ((FAKE, 1, 4, 32, 32, 0, 3, FAKE + 4, FAKE, FAKE, FAKE, FAKE, 0), fq.ERR_ALIGNMENT),  # weights
+    ((FAKE, 1, 4, 32, 32, 0, 2, None, FAKE, FAKE, FAKE, FAKE, 0x80), fq.ERR_INVALID_ARG),  # unknown flag
+    ((FAKE, 1, 4, 32, 32, 2, 0, None, FAKE, FAKE, None, FAKE, 1), fq.ERR_INVALID_ARG),  # MX with given S
+    ((None, 1, 0, 32, 32, 0, 2, None, None, None, None, None, 0), fq.OK),               # empty: no launch
+])
+def test_quantize_rejects_before_launch(args, rc):
+    L = fq.lib()
+    assert L.fp4q_quantize(*args, None) == rc
+    if rc == fq.OK:
+        assert L.fp4q_last_launch_count() == 0
+
+
+def test_hadamard_and_dequant_validation():
+    L = fq.lib()
+    assert L.fp4q_hadamard_quantize(FAKE, 1, 4, 64, 64, 16, FAKE, FAKE, FAKE, 0, None) == fq.ERR_UNSUPPORTED
+    assert L.fp4q_hadamard_quantize(FAKE, 1, 4, 48, 48, 32, FAKE, FAKE, FAKE, 0, None) == fq.ERR_SHAPE
+    assert L.fp4q_dequantize(FAKE, FAKE, FAKE, 4, 24, 0, 0, FAKE, 0, None) == fq.ERR_SHAPE
+    assert L.fp4q_dequantize(FAKE, FAKE, FAKE, 4, 32, 0, 1, FAKE, 0, None) == fq.ERR_UNSUPPORTED
+    assert L.fp4q_dequantize(FAKE, FAKE, None, 4, 32, 0, 0, FAKE, 0, None) == fq.ERR_INVALID_ARG
+    assert L.fp4q_dequantize(FAKE, FAKE, FAKE, 4, 32, 0, 0, FAKE + 4, 0, None) == fq.ERR_ALIGNMENT
+    assert L.fp4q_dequantize(FAKE, FAKE, FAKE, 4, 32, 0, 0, FAKE, 8, None) == fq.ERR_INVALID_ARG
+    assert L.fp4q_dequantize(None, None, None, 0, 32, 0, 0, None, 0, None) == fq.OK
+    assert L.fp4q_read_device_status(None, None, None) == fq.ERR_INVALID_ARG
+
+
+def test_global_scale_validation():
+    L = fq.lib()
+    assert L.fp4q_global_scale(FAKE, 1, 4, 12, 12, FAKE, FAKE, None) == fq.ERR_SHAPE      # 24-byte rows
+    assert L.fp4q_global_scale(FAKE, 1, 4, 16, 20, FAKE, FAKE, None) == fq.ERR_ALIGNMENT  # 40-byte pitch
+    assert L.fp4q_global_scale(FAKE, 1, 4, 16, 16, None, FAKE, None) == fq.ERR_INVALID_ARG
+    assert L.fp4q_global_scale(FAKE, 3, 4, 16, 16, FAKE, FAKE, None) == fq.ERR_INVALID_ARG
+    assert L.fp4q_global_scale(None, 1, 0, 16, 16, None, None, None) == fq.OK
