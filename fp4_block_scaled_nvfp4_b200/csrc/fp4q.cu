@@ -80,13 +80,7 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const void* __restrict__
     uint32_t m = 0;
     const uint4* base = reinterpret_cast<const uint4*>(xv);
     const int64_t ldv = ld * (IN == FP4Q_IN_BF16 ? 2 : 4) / 16;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += step) {
-        int64_t off = i;
-        if (ldv != vpr) {
-            const int64_t r = i / vpr;
-            off = r * ldv + (i - r * vpr);
-        }
-        const uint4 v = __ldg(base + off);
+    auto fold = [&](const uint4 v) {
         if (IN == FP4Q_IN_BF16) {
             uint32_t t;
             const uint32_t mk = 0x7FFF7FFFu;
@@ -98,7 +92,18 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const void* __restrict__
             const uint32_t mk = 0x7FFFFFFFu;
             m = max(m, max(max(v.x & mk, v.y & mk), max(v.z & mk, v.w & mk)));
         }
+    };
+    auto at = [&](int64_t i) -> const uint4* {
+        if (ldv == vpr) return base + i;
+        const int64_t r = i / vpr;
+        return base + r * ldv + (i - r * vpr);
+    };
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    for (; i + 3 * step < total; i += 4 * step) {   // four independent 16-byte loads in flight
+        const uint4 v0 = __ldg(at(i)), v1 = __ldg(at(i + step)), v2 = __ldg(at(i + 2 * step)), v3 = __ldg(at(i + 3 * step));
+        fold(v0); fold(v1); fold(v2); fold(v3);
     }
+    for (; i < total; i += step) fold(__ldg(at(i)));
     if (IN == FP4Q_IN_BF16) m = max(m & 0xFFFFu, m >> 16) << 16;   // bf16 bits -> f32 bits
     m = __reduce_max_sync(0xFFFFFFFFu, m);
     __shared__ uint32_t red[kThreads / 32];
@@ -138,12 +143,14 @@ __device__ __forceinline__ Setup read_setup(const float* gscale) {
     return s;
 }
 
-// sv(p) = RN(e(p) * S) and inv(p) = RN(1/sv(p)) for every pattern p (0 for p = 0 and 127).
-__device__ __forceinline__ void build_scale_table(float S, float* s_sv, float* s_inv) {
+// sv(p) = RN(e(p) * S), inv(p) = RN(1/sv(p)) and s2(p) = RN(sv(p)^2) for every pattern p
+// (all 0 for p = 0 and 127).
+__device__ __forceinline__ void build_scale_table(float S, float* s_sv, float* s_inv, float* s_s2) {
     for (int p = threadIdx.x; p < 128; p += blockDim.x) {
         const float sv = (p == 0 || p == 127) ? 0.0f : __fmul_rn(e4m3_value(p), S);
         s_sv[p] = sv;
         s_inv[p] = sv == 0.0f ? 0.0f : __frcp_rn(sv);
+        s_s2[p] = __fmul_rn(sv, sv);
     }
     __syncthreads();
 }
@@ -180,23 +187,46 @@ __device__ __forceinline__ float block_absmax(const u64 (&xp)[8]) {
     return m;
 }
 
-// Error of one candidate (sv, inv): residual d = fma(-q, sv, x) per element; squares summed
-// by fma into an (even, odd) pair of accumulators; result RN(even + odd).
+// Error of one candidate: with y = RN(x inv) and codes q = E2M1(y), the residuals
+// r = RN(q - y) (units of the scale) are squared and summed by fma into an (even, odd) pair
+// of accumulators, combined once, and scaled by s2 = RN(sv^2).  For the zero scale (sv = 0)
+// every code is 0 and the error is the same fma sum over x itself (no scaling).
 template <bool WEIGHTED>
-__device__ __forceinline__ float candidate_error(const u64 (&xp)[8], const u64 (&wp)[8], float sv, float inv) {
-    const u64 inv2 = pk(inv, inv), nsv2 = pk(-sv, -sv);
-    u64 acc = pk(0.0f, 0.0f);
+__device__ __forceinline__ float candidate_error(const u64 (&xp)[8], const u64 (&wp)[8], float sv, float inv, float s2) {
+    float ae = 0.0f, ao = 0.0f;
+    if (sv == 0.0f) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            float a, b;
+            upk(xp[j], a, b);
+            if (WEIGHTED) {
+                float w0, w1;
+                upk(wp[j], w0, w1);
+                ae = __fmaf_rn(__fmul_rn(w0, a), a, ae);
+                ao = __fmaf_rn(__fmul_rn(w1, b), b, ao);
+            } else {
+                ae = __fmaf_rn(a, a, ae);
+                ao = __fmaf_rn(b, b, ao);
+            }
+        }
+        return __fadd_rn(ae, ao);
+    }
+    const u64 inv2 = pk(inv, inv);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-        const u64 y = mul2(xp[j], inv2);
-        const u64 g = e2m1x2_decode(e2m1x2(y));
-        const u64 d = fma2(g, nsv2, xp[j]);
-        if (WEIGHTED) acc = fma2(mul2(wp[j], d), d, acc);
-        else acc = fma2(d, d, acc);
+        float r0, r1;
+        e2m1x2_residual(mul2(xp[j], inv2), r0, r1);
+        if (WEIGHTED) {
+            float w0, w1;
+            upk(wp[j], w0, w1);
+            ae = __fmaf_rn(__fmul_rn(w0, r0), r0, ae);
+            ao = __fmaf_rn(__fmul_rn(w1, r1), r1, ao);
+        } else {
+            ae = __fmaf_rn(r0, r0, ae);
+            ao = __fmaf_rn(r1, r1, ao);
+        }
     }
-    float a, b;
-    upk(acc, a, b);
-    return __fadd_rn(a, b);
+    return __fmul_rn(s2, __fadd_rn(ae, ao));
 }
 
 // Packed codes of a block for a given reciprocal scale (8 bytes: elements 0..15).
@@ -218,9 +248,9 @@ __global__ void __launch_bounds__(kThreads) nvfp4_kernel(const void* __restrict_
                                                          uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
                                                          const float* __restrict__ gscale, uint32_t* __restrict__ ws,
                                                          int s_given) {
-    __shared__ float s_sv[128], s_inv[128];
+    __shared__ float s_sv[128], s_inv[128], s_s2[128];
     const Setup su = read_setup(gscale);
-    build_scale_table(su.S, s_sv, s_inv);
+    build_scale_table(su.S, s_sv, s_inv, s_s2);
     const float S = su.S;
     const float d6 = __fmul_rn(6.0f, S), d4 = __fmul_rn(4.0f, S);
     const int64_t nb = cols / 16;
@@ -249,8 +279,8 @@ __global__ void __launch_bounds__(kThreads) nvfp4_kernel(const void* __restrict_
                 const int p4 = e4m3_rne(__fdiv_rn(ab, d4));
                 if (p4 != p0) {
                     u64 wp[8];
-                    const float e0 = candidate_error<false>(xp, wp, s_sv[p0], s_inv[p0]);
-                    const float e4 = candidate_error<false>(xp, wp, s_sv[p4], s_inv[p4]);
+                    const float e0 = candidate_error<false>(xp, wp, s_sv[p0], s_inv[p0], s_s2[p0]);
+                    const float e4 = candidate_error<false>(xp, wp, s_sv[p4], s_inv[p4], s_s2[p4]);
                     if (e4 < e0) bp = p4;
                 }
             } else if (OBJ == FP4Q_SWEEP_MSE || OBJ == FP4Q_SWEEP_WMSE) {
@@ -271,7 +301,7 @@ __global__ void __launch_bounds__(kThreads) nvfp4_kernel(const void* __restrict_
                     const int p = p0 + k;
                     const bool valid = (unsigned)p <= 126u;
                     const int pc = valid ? p : 0;
-                    const float e = candidate_error<WEIGHTED>(xp, wp, s_sv[pc], s_inv[pc]);
+                    const float e = candidate_error<WEIGHTED>(xp, wp, s_sv[pc], s_inv[pc], s_s2[pc]);
                     if (valid && e < best) {
                         best = e;
                         bp = p;
@@ -293,13 +323,13 @@ __global__ void __launch_bounds__(kThreads) if4_kernel(const void* __restrict__ 
                                                        int64_t ld, uint8_t* __restrict__ codes,
                                                        uint8_t* __restrict__ scales, const float* __restrict__ gscale,
                                                        uint32_t* __restrict__ ws, int s_given) {
-    __shared__ float s_sv[128], s_inv[128];
+    __shared__ float s_sv[128], s_inv[128], s_s2[128];
     const Setup su = read_setup(gscale);
-    build_scale_table(su.S, s_sv, s_inv);
+    build_scale_table(su.S, s_sv, s_inv, s_s2);
     const float S = su.S;
     const float d6 = __fmul_rn(6.0f, S);
     const float K76 = __fdiv_rn(7.0f, 6.0f), K67 = __fdiv_rn(6.0f, 7.0f);
-    const u64 k76 = pk(K76, K76), k67 = pk(K67, K67);
+    const u64 k76 = pk(K76, K76);
     const int64_t nb = cols / 16;
     const int64_t total = rows * nb;
     const int64_t step = (int64_t)gridDim.x * blockDim.x;
@@ -314,32 +344,34 @@ __global__ void __launch_bounds__(kThreads) if4_kernel(const void* __restrict__ 
         u64 xp[8];
         load_block16<IN>(xv, r * ld + b * 16, xp);
         const int p0 = S > 0.0f ? e4m3_rne(__fdiv_rn(block_absmax(xp), d6)) : 0;
-        const float sv = s_sv[p0], inv = s_inv[p0];
-        const u64 inv2 = pk(inv, inv), nsv2 = pk(-sv, -sv);
-        u64 accf = pk(0.0f, 0.0f), acci = pk(0.0f, 0.0f);
+        const float inv = s_inv[p0];
+        const u64 inv2 = pk(inv, inv);
+        float fe = 0.0f, fo = 0.0f, ie = 0.0f, io = 0.0f;
         uint32_t cf[8], ci[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const u64 y = mul2(xp[j], inv2);
             cf[j] = e2m1x2(y);
-            const u64 df = fma2(e2m1x2_decode(cf[j]), nsv2, xp[j]);
-            accf = fma2(df, df, accf);
-            float z0, z1;
+            float r0, r1;
+            e2m1x2_residual(y, r0, r1);
+            fe = __fmaf_rn(r0, r0, fe);
+            fo = __fmaf_rn(r1, r1, fo);
+            float y0, y1, z0, z1;
+            upk(y, y0, y1);
             upk(mul2(y, k76), z0, z1);
             float n0, n1;
             asm("cvt.rni.f32.f32 %0, %1;" : "=f"(n0) : "f"(z0));
             asm("cvt.rni.f32.f32 %0, %1;" : "=f"(n1) : "f"(z1));
             n0 = fminf(fmaxf(n0, -7.0f), 7.0f);
             n1 = fminf(fmaxf(n1, -7.0f), 7.0f);
-            const u64 di = fma2(mul2(pk(n0, n1), k67), nsv2, xp[j]);
-            acci = fma2(di, di, acci);
+            const float v0 = __fmul_rn(n0, K67), v1 = __fmul_rn(n1, K67);
+            const float s0 = __fsub_rn(v0, y0), s1 = __fsub_rn(v1, y1);
+            ie = __fmaf_rn(s0, s0, ie);
+            io = __fmaf_rn(s1, s1, io);
             ci[j] = ((uint32_t)__float2int_rn(n0) & 0xFu) | (((uint32_t)__float2int_rn(n1) & 0xFu) << 4);
         }
-        float a, c;
-        upk(accf, a, c);
-        const float ef = __fadd_rn(a, c);
-        upk(acci, a, c);
-        const float ei = __fadd_rn(a, c);
+        const float ef = __fadd_rn(fe, fo);
+        const float ei = __fadd_rn(ie, io);
         const bool use_int = ei < ef;
         const uint32_t* cc = use_int ? ci : cf;
         *cdst = make_uint2(cc[0] | (cc[1] << 8) | (cc[2] << 16) | (cc[3] << 24),
@@ -580,7 +612,7 @@ int launch_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, int f
     const int given = (flags & FP4Q_F_GLOBAL_SCALE_GIVEN) ? 1 : 0;
     if (!given) {
         const int64_t vecs = rows * cols * (IN == FP4Q_IN_BF16 ? 2 : 4) / 16;
-        amax_kernel<IN><<<grid_for(vecs, 8), kThreads, 0, st>>>(x, rows, cols, ld, ws, gs, 0);
+        amax_kernel<IN><<<grid_for(vecs, 4), kThreads, 0, st>>>(x, rows, cols, ld, ws, gs, 0);
         ++n;
     }
     const int g = grid_for(rows * (cols / 16), 8);
@@ -655,9 +687,9 @@ int fp4q_global_scale(const void* x, int dtype, int64_t rows, int64_t cols, int6
     uint32_t* ws = reinterpret_cast<uint32_t*>(workspace);
     const int64_t vecs = rows * cols * (dtype == FP4Q_IN_BF16 ? 2 : 4) / 16;
     if (dtype == FP4Q_IN_BF16)
-        amax_kernel<FP4Q_IN_BF16><<<grid_for(vecs, 8), kThreads, 0, st>>>(x, rows, cols, ld, ws, global_scale, 1);
+        amax_kernel<FP4Q_IN_BF16><<<grid_for(vecs, 4), kThreads, 0, st>>>(x, rows, cols, ld, ws, global_scale, 1);
     else
-        amax_kernel<FP4Q_IN_F32><<<grid_for(vecs, 8), kThreads, 0, st>>>(x, rows, cols, ld, ws, global_scale, 1);
+        amax_kernel<FP4Q_IN_F32><<<grid_for(vecs, 4), kThreads, 0, st>>>(x, rows, cols, ld, ws, global_scale, 1);
     return launched(1);
 }
 

@@ -68,6 +68,21 @@ __device__ __forceinline__ u64 e2m1x2_decode(uint32_t c) {
     return pk(a, b);
 }
 
+// Quantizer residuals of a pair in units of the scale: with y = (y0, y1), codes
+// q = E2M1(y) and r = RN(q - y) per lane (q is exact in f16, the subtraction is one binary32
+// rounding).  Encode, decode and subtract in one block so no value leaves its register.
+__device__ __forceinline__ void e2m1x2_residual(u64 y, float& r0, float& r1) {
+    float a, b;
+    upk(y, a, b);
+    asm("{ .reg .b8 t; .reg .b32 h; .reg .f16 p, q;\n"
+        "  cvt.rn.satfinite.e2m1x2.f32 t, %3, %2;\n"
+        "  cvt.rn.f16x2.e2m1x2 h, t;\n"
+        "  mov.b32 {p, q}, h;\n"
+        "  sub.rn.f32.f16 %0, p, %2;\n"
+        "  sub.rn.f32.f16 %1, q, %3; }"
+        : "=f"(r0), "=f"(r1) : "f"(a), "f"(b));
+}
+
 // ---- E4M3 (FN) ----------------------------------------------------------------------------
 // Bit pattern of the nearest E4M3 value (ties to even, saturating at 448) of a finite v >= 0.
 __device__ __forceinline__ int e4m3_rne(float v) {

@@ -21,11 +21,14 @@
  * nearest even, no contraction, no flush-to-zero):
  *   S = RN(amax/1536); p0 = E4M3_RNE(RN(a_b / RN(6 S))); p4 = E4M3_RNE(RN(a_b / RN(4 S)));
  *   candidate p: sv = RN(e(p) S), inv = RN(1/sv) (sv = inv = 0 for p = 0);
- *   y = RN(x inv); q = E2M1_RNE_satfinite(y); d = fma(-q, sv, x);
- *   error = RN(acc_even + acc_odd), acc_par = fma(d, d, acc_par) over the block's even /
- *   odd positions in order (WMSE: fma(RN(w d), d, acc)); the lowest offset wins a tie.
+ *   y = RN(x inv); q = E2M1_RNE_satfinite(y); r = RN(q - y) (the quantizer's rounding error
+ *   in units of the scale); E = RN(acc_even + acc_odd), acc_par = fma(r, r, acc_par) over the
+ *   block's even / odd positions in order (WMSE: fma(RN(w r), r, acc)); error = RN(RN(sv^2) E),
+ *   i.e. the block MSE sum (x - q s)^2 = s^2 sum (x/s - q)^2 evaluated on the binary32
+ *   quotient y; for p = 0 the error is the same fma sum over x itself.  The lowest offset
+ *   wins a tie of the computed errors.
  *   IF4 INT4: z = RN(y RN(7/6)), n = clamp(rint(z), -7, 7), v = RN(n RN(6/7)),
- *   d = fma(-v, sv, x); INT4 iff its error is strictly lower.
+ *   r = RN(v - y); both paths share s, so INT4 iff E_int < E_fp.
  *   MXFP4: e = smallest integer with a_b <= 6 * 2^e (flag FP4Q_F_MX_OCP_FLOOR: floor(log2
  *   a_b) - 2), clamped to [-127,127]; y = RN(x 2^-e).
  *

@@ -33,13 +33,18 @@
  *   p0     = E4M3(RN(a_b / RN(6*S)))               (a_b = max |x| over the block)
  *   p4     = E4M3(RN(a_b / RN(4*S)))               (4/6 only)
  *   sv(p)  = RN(e(p) * S), inv(p) = RN(1 / sv(p)); sv(0) = inv(0) = 0
- *   y      = RN(x * inv),  q = E2M1(y),  d = fma(-q, sv, x)
- *   error  = two fp32 accumulators, even and odd element positions, each
- *            acc = fma(d, d, acc) (WMSE: acc = fma(RN(w*d), d, acc)) in element order,
- *            then RN(acc_even + acc_odd)
+ *   y      = RN(x * inv),  q = E2M1(y),  r = RN(q - y)   (the quantizer's own rounding
+ *            error, in units of the scale)
+ *   error  = RN(RN(sv*sv) * E) with E = RN(acc_even + acc_odd); acc_even / acc_odd are fp32
+ *            accumulators over the even / odd element positions, each acc = fma(r, r, acc)
+ *            (WMSE: acc = fma(RN(w*r), r, acc)) in element order.  For the zero scale
+ *            (p = 0) every code is 0 and the error is the same fma sum over x itself.
+ *            This is the block MSE sum (x - q*s)^2 = s^2 sum (x/s - q)^2 evaluated on the
+ *            binary32 quotient y the quantizer rounds.
  *   argmin = lexicographic (error, offset): the lowest offset wins a tie.
  *   IF4    = AbsMax scale p0; INT4 path z = RN(y*RN(7/6)), n = clamp(rint(z), -7, 7),
- *            v = RN(n*RN(6/7)), d = fma(-v, sv, x); INT4 iff err_int < err_fp.
+ *            v = RN(n*RN(6/7)), r = RN(v - y); both paths share s, so INT4 iff
+ *            E_int < E_fp.
  *   MXFP4  = e = smallest integer with a_b <= 6*2^e (clamped to [-127,127]), byte e+127,
  *            y = RN(x * 2^-e), q = E2M1(y), dequant q*2^e.
  *   Hadamard(32) = Sylvester fast Walsh-Hadamard butterflies for h = 1,2,4,8,16
@@ -163,19 +168,29 @@ static void scale_pair(int p, float S, float* sv, float* inv)
     *inv = 1.0f / *sv;
 }
 
-/* Error of one candidate scale for a block of B values: x-domain residuals, two
- * accumulators by element parity, combined at the end. */
+/* Error of one candidate scale for a block of B values.  p = 0 (sv = 0): every code is
+ * zero and the error is the sum of x^2 (WMSE: w x^2).  Otherwise: residuals of the
+ * quantizer in units of the scale, r = RN(q - y), squares summed by fma into two
+ * accumulators by element parity, combined once, then scaled by RN(sv^2). */
 static float block_error(const float* x, const float* w, int B, float sv, float inv)
 {
     float acc[2] = {0.0f, 0.0f};
+    if (sv == 0.0f) {
+        for (int i = 0; i < B; ++i) {
+            if (w) acc[i & 1] = fmaf(w[i] * x[i], x[i], acc[i & 1]);
+            else acc[i & 1] = fmaf(x[i], x[i], acc[i & 1]);
+        }
+        return acc[0] + acc[1];
+    }
     for (int i = 0; i < B; ++i) {
         float y = x[i] * inv;
         float q = fp4q_o_e2m1_value(fp4q_o_e2m1_encode(y));
-        float d = fmaf(-q, sv, x[i]);
-        if (w) acc[i & 1] = fmaf(w[i] * d, d, acc[i & 1]);
-        else acc[i & 1] = fmaf(d, d, acc[i & 1]);
+        float r = q - y;
+        if (w) acc[i & 1] = fmaf(w[i] * r, r, acc[i & 1]);
+        else acc[i & 1] = fmaf(r, r, acc[i & 1]);
     }
-    return acc[0] + acc[1];
+    float E = acc[0] + acc[1];
+    return (sv * sv) * E;
 }
 
 static uint8_t pack_codes_for(const float* x, int B, float inv, uint8_t* codes_row, int64_t c0)
@@ -310,15 +325,15 @@ int fp4q_o_if4_quantize(const float* x, int64_t rows, int64_t cols, int64_t ld,
                 float y = xb[i] * inv;
                 cf[i] = fp4q_o_e2m1_encode(y);
                 float q = fp4q_o_e2m1_value(cf[i]);
-                float df = fmaf(-q, sv, xb[i]);
-                accf[i & 1] = fmaf(df, df, accf[i & 1]);
+                float rf = q - y;
+                accf[i & 1] = fmaf(rf, rf, accf[i & 1]);
                 float z = y * K76;
                 float n = rint_even(z);
                 if (n > 7.0f) n = 7.0f;
                 if (n < -7.0f) n = -7.0f;
                 float v = n * K67;
-                float di = fmaf(-v, sv, xb[i]);
-                acci[i & 1] = fmaf(di, di, acci[i & 1]);
+                float ri = v - y;
+                acci[i & 1] = fmaf(ri, ri, acci[i & 1]);
                 ci[i] = ((int)n) & 0xF;   /* two's complement nibble */
             }
             float ef = accf[0] + accf[1], ei = acci[0] + acci[1];

@@ -136,21 +136,37 @@ def test_window_bounds_in_bit_pattern_space():
 # ---------------------------------------------------------------------------------
 # exact error arithmetic (rational brute force) and the sweep's argmin
 # ---------------------------------------------------------------------------------
+DELTA = Fr(1, 2 ** 22)   # |y - x/s| <= 2^-22 |x/s|: two binary32 roundings (1/s, then x * 1/s)
+
+
 def exact_block_errors(xb, S, cands, w=None):
-    """Exact squared error sum_i w_i (x_i - q_i s)^2 for each candidate pattern, with codes
-    from the binary32 quantizer y = RN(x * RN(1/s)) and a brute-force E2M1 rounding."""
+    """Exact rational errors of each candidate pattern with the codes of the binary32
+    quantizer y = RN(x * RN(1/s)) (brute-force E2M1 rounding):
+      'x': the block MSE sum w (x - q s)^2 (the method's objective),
+      'y': the contract's quantity s^2 sum w (q - y)^2 on the binary32 quotients y,
+      'e': sum w x^2 (energy, for the bound between the two)."""
     out = {}
     for p in cands:
         s = f32(float(E4M3[p])) * f32(S)
         inv = f32(1.0) / s if p else f32(0.0)
-        err = Fr(0)
+        ex, ey, en = Fr(0), Fr(0), Fr(0)
         for i, xv in enumerate(xb):
+            wi = Fr(float(w[i])) if w is not None else 1
             y = f32(xv) * inv
             q = nearest_e2m1(Fr(float(y)))
             d = Fr(float(xv)) - q * Fr(float(s))
-            err += (Fr(float(w[i])) if w is not None else 1) * d * d
-        out[p] = err
+            ex += wi * d * d
+            en += wi * Fr(float(xv)) ** 2
+            ey += wi * (q - Fr(float(y))) ** 2
+        ey = ey * Fr(float(s)) ** 2 if p else en
+        out[p] = {"x": ex, "y": ey, "e": en}
     return out
+
+
+def xy_bound(e):
+    """|y-domain - x-domain| <= 2 D sqrt(Ex En) + D^2 En, D = DELTA (Cauchy-Schwarz)."""
+    ex, en = float(e["x"]), float(e["e"])
+    return 2.0 * float(DELTA) * (ex * en) ** 0.5 + float(DELTA) ** 2 * en
 
 
 def _tensor_with(xb, amax=1536.0):
@@ -175,14 +191,21 @@ def test_error_matches_exact_and_argmin(cfg):
         cands = [p for p in range(p0 - 3, p0 + 8) if 0 <= p <= 0x7E]
         ex = exact_block_errors(xb, S, cands)
         chosen = int(r["p"][row, b])
-        # the oracle's float error for the chosen candidate is the exact error to fp32 accuracy
-        assert abs(Fr(float(r["err"][row, b])) - ex[chosen]) <= ex[chosen] * Fr(1, 10 ** 5) + Fr(1, 10 ** 30)
-        best = min(ex.values())
-        # chosen = exact argmin unless the exact gap is below the fp32 resolution
-        if ex[chosen] != best:
-            assert (ex[chosen] - best) <= best * Fr(1, 10 ** 5)
+        e = ex[chosen]
+        # the oracle's binary32 error is the contract's quantity to fp32 accumulation accuracy
+        assert abs(Fr(float(r["err"][row, b])) - e["y"]) <= e["y"] * Fr(1, 10 ** 5) + Fr(1, 10 ** 30)
+        # and the contract's quantity is the block MSE up to the rounding of y
+        for p in cands:
+            assert abs(float(ex[p]["y"] - ex[p]["x"])) <= xy_bound(ex[p]) * 1.0001 + 1e-30
+        # chosen = exact argmin of the contract's quantity unless the gap is below fp32 resolution
+        besty = min(v["y"] for v in ex.values())
+        if e["y"] != besty:
+            assert (e["y"] - besty) <= besty * Fr(1, 10 ** 5)
         else:
-            assert chosen == min(p for p in cands if ex[p] == best)
+            assert chosen == min(p for p in cands if ex[p]["y"] == besty)
+        # and it is within the y-rounding bound of the true MSE optimum
+        bestx = min(v["x"] for v in ex.values())
+        assert float(e["x"] - bestx) <= 2 * max(xy_bound(v) for v in ex.values()) + float(bestx) * 1e-5
 
 
 def test_weighted_error_matches_exact():
@@ -196,7 +219,9 @@ def test_weighted_error_matches_exact():
         wb = imp[b * 16:(b + 1) * 16]
         chosen = int(r["p"][row, b])
         ex = exact_block_errors(xb, S, [chosen], w=wb)
-        assert abs(Fr(float(r["err"][row, b])) - ex[chosen]) <= ex[chosen] * Fr(1, 10 ** 5) + Fr(1, 10 ** 30)
+        e = ex[chosen]
+        assert abs(Fr(float(r["err"][row, b])) - e["y"]) <= e["y"] * Fr(1, 10 ** 5) + Fr(1, 10 ** 30)
+        assert abs(float(e["y"] - e["x"])) <= xy_bound(e) * 1.0001 + 1e-30
 
 
 def test_bruteforce_all_126_scales_on_tiny_blocks():
@@ -208,9 +233,11 @@ def test_bruteforce_all_126_scales_on_tiny_blocks():
         x = _tensor_with(xb, amax=float(np.abs(xb).max()) * 3.0)
         r = O.nvfp4_quantize(x, "sweep_mse")
         ex = exact_block_errors(xb, r["S"], range(0x7F))
-        best = min(ex.values())
         chosen = int(r["p"][0, 0])
-        assert ex[chosen] - best <= best * Fr(1, 10 ** 5)
+        besty = min(v["y"] for v in ex.values())
+        bestx = min(v["x"] for v in ex.values())
+        assert ex[chosen]["y"] - besty <= besty * Fr(1, 10 ** 5)
+        assert float(ex[chosen]["x"] - bestx) <= 2 * max(xy_bound(v) for v in ex.values()) + float(bestx) * 1e-5
 
 
 @pytest.mark.parametrize("cfg,obj", [("cfg1", "sweep_mse"), ("cfg3", "sweep_mse"), ("cfg2", "sweep_wmse")])
@@ -263,7 +290,11 @@ def test_if4_invariants():
     ind = (r["scales"] >> 7).astype(bool)
     assert np.array_equal(r["scales"] & 0x7F, a["scales"])          # shared AbsMax scale
     assert np.array_equal(ind, r["err_int"] < r["err_fp"])           # lower error wins, tie -> FP4
-    assert np.array_equal(r["err_fp"], a["err"])
+    # IF4 compares both paths in units of the shared scale; AbsMax reports s^2 * E
+    S = r["S"]
+    s2 = np.array([[f32(f32(O.e4m3_value(p)) * f32(S)) ** 2 if p else 0 for p in row] for row in a["scales"]], np.float32)
+    nz = a["scales"] > 0
+    assert np.array_equal((s2 * r["err_fp"])[nz], a["err"][nz])
     assert 0 < ind.mean() < 1
     # FP4 blocks carry exactly the AbsMax codes
     cf = r["codes"].reshape(8, -1, 8)[~ind]
@@ -317,9 +348,12 @@ def test_exact_roundtrip_every_e2m1_x_e4m3_value():
     assert list(r["scales"][0]) == list(range(1, 0x79))
     xh = O.dequantize(r["codes"], r["scales"], r["S"], "nvfp4")
     assert np.array_equal(xh.view(np.uint32), x.view(np.uint32))
-    assert np.all(r["err"] == 0)
+    # the error is evaluated on y = RN(x * RN(1/s)), which equals the code only up to two
+    # roundings: an exactly representable block scores at most (6 * 2^-22)^2 * 16 * s^2
+    energy = (x.astype(np.float64).reshape(-1, 16) ** 2).sum(axis=1)
+    assert np.all(r["err"] <= energy * 2.0 ** -38)
     rs = O.nvfp4_quantize(x, "sweep_mse")
-    assert np.all(rs["err"] == 0)
+    assert np.all(rs["err"] <= energy * 2.0 ** -38)
     assert np.array_equal(O.dequantize(rs["codes"], rs["scales"], rs["S"], "nvfp4"), x)
     for p in range(0x79, 0x7F):
         codes = np.array([[k | (k << 4) for k in range(8)] + [(k | 8) | ((k | 8) << 4) for k in range(8)]], np.uint8)
@@ -355,7 +389,7 @@ def test_hand_worked(row):
         assert r["S"] == float(S)
         assert r["scales"][0, 0] == scale
         err = r["err_int"][0, 0] if scale & 0x80 else r["err_fp"][0, 0]
-        assert err == expect[0]
+        assert err == expect[0]          # zero errors are zero in either unit
         xh = O.dequantize(r["codes"], r["scales"], r["S"], "if4")
         if expect[0] == 0:
             assert np.array_equal(xh[0, :16], xb)
@@ -363,7 +397,9 @@ def test_hand_worked(row):
     r = O.nvfp4_quantize(x, method)
     assert r["S"] == float(S)
     assert r["scales"][0, 0] == scale
-    assert r["err"][0, 0] == expect[0]
+    # the hand-worked value is the exact block MSE; the contract evaluates it in binary32 on
+    # y = RN(x * RN(1/s)), so a nonzero value agrees to rounding, a zero one exactly
+    assert abs(r["err"][0, 0] - expect[0]) <= 1e-5 * expect[0]
 
 
 def test_status_paths():
