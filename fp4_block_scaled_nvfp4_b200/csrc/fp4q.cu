@@ -71,7 +71,7 @@ __device__ __forceinline__ void finish_status(uint32_t* ws, uint32_t flag, int c
 // amax
 // ------------------------------------------------------------------------------------------
 template <int IN>
-__global__ void __launch_bounds__(kThreads) amax_kernel(const void* __restrict__ xv, int64_t rows, int64_t cols,
+__global__ void __launch_bounds__(kThreads, 4) amax_kernel(const void* __restrict__ xv, int64_t rows, int64_t cols,
                                                         int64_t ld, uint32_t* __restrict__ ws,
                                                         float* __restrict__ gscale, int publish) {
     const int64_t vpr = cols * (IN == FP4Q_IN_BF16 ? 2 : 4) / 16;   // 16-byte vectors per row
@@ -99,9 +99,21 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const void* __restrict__
         return base + r * ldv + (i - r * vpr);
     };
     int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    for (; i + 3 * step < total; i += 4 * step) {   // four independent 16-byte loads in flight
-        const uint4 v0 = __ldg(at(i)), v1 = __ldg(at(i + step)), v2 = __ldg(at(i + 2 * step)), v3 = __ldg(at(i + 3 * step));
-        fold(v0); fold(v1); fold(v2); fold(v3);
+    if (ldv == vpr) {   // contiguous tensor: eight independent 16-byte loads in flight per thread
+        constexpr int U = 8;
+        for (; i + (U - 1) * step < total; i += U * step) {
+            uint4 v[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) v[u] = __ldg(base + i + u * step);
+#pragma unroll
+            for (int u = 0; u < U; ++u) fold(v[u]);
+        }
+    } else {
+        for (; i + 3 * step < total; i += 4 * step) {
+            const uint4 v0 = __ldg(at(i)), v1 = __ldg(at(i + step)), v2 = __ldg(at(i + 2 * step)),
+                        v3 = __ldg(at(i + 3 * step));
+            fold(v0); fold(v1); fold(v2); fold(v3);
+        }
     }
     for (; i < total; i += step) fold(__ldg(at(i)));
     if (IN == FP4Q_IN_BF16) m = max(m & 0xFFFFu, m >> 16) << 16;   // bf16 bits -> f32 bits
@@ -311,6 +323,91 @@ __global__ void __launch_bounds__(kThreads) nvfp4_kernel(const void* __restrict_
         }
         *cdst = block_codes(xp, s_inv[bp]);
         scales[blk] = (uint8_t)bp;
+    }
+    finish_status(ws, su.flags, WS_CNT_Q);
+}
+
+// ------------------------------------------------------------------------------------------
+// NVFP4 ScaleSweep (MSE window [-3,+7], WMSE window [-8,+7]): one thread per block, every
+// candidate evaluated in registers; the zero scale (only in the window of tiny blocks) is
+// scored once before the loop so the loop itself is branch-free.
+// ------------------------------------------------------------------------------------------
+template <bool WEIGHTED>
+__device__ __forceinline__ float sweep_error(const u64 (&xp)[8], const u64 (&wp)[8], float inv, float s2) {
+    const u64 inv2 = pk(inv, inv);
+    u64 acc = pk(0.0f, 0.0f);   // (even, odd) accumulators
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const u64 r = e2m1x2_residual2(mul2(xp[j], inv2));
+        acc = WEIGHTED ? fma2(mul2(wp[j], r), r, acc) : fma2(r, r, acc);
+    }
+    float a, b;
+    upk(acc, a, b);
+    return __fmul_rn(s2, __fadd_rn(a, b));
+}
+
+template <bool WEIGHTED>
+__device__ __forceinline__ float zero_scale_error(const u64 (&xp)[8], const u64 (&wp)[8]) {
+    u64 acc = pk(0.0f, 0.0f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc = WEIGHTED ? fma2(mul2(wp[j], xp[j]), xp[j], acc) : fma2(xp[j], xp[j], acc);
+    float a, b;
+    upk(acc, a, b);
+    return __fadd_rn(a, b);
+}
+
+template <int IN, bool WEIGHTED, typename IDX>
+__global__ void __launch_bounds__(kThreads, WEIGHTED ? 4 : 6) sweep_kernel(const void* __restrict__ xv, IDX rows, IDX cols, IDX ld,
+                                                            const float* __restrict__ imp,
+                                                            uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                                                            const float* __restrict__ gscale, uint32_t* __restrict__ ws) {
+    __shared__ float s_sv[128], s_inv[128], s_s2[128];
+    const Setup su = read_setup(gscale);
+    build_scale_table(su.S, s_sv, s_inv, s_s2);
+    const float S = su.S;
+    const float d6 = __fmul_rn(6.0f, S);
+    constexpr int LO = WEIGHTED ? -8 : -3, HI = 7;
+    const IDX nb = cols / 16;
+    const IDX total = rows * nb;
+    const IDX blk = (IDX)blockIdx.x * blockDim.x + threadIdx.x;
+    if (blk < total) {
+        const IDX r = blk / nb, b = blk - r * nb;
+        uint2* cdst = reinterpret_cast<uint2*>(codes + r * (cols / 2) + b * 8);
+        if (su.flags) {   // data out of contract: zero-filled outputs
+            *cdst = make_uint2(0u, 0u);
+            scales[blk] = 0;
+        } else {
+            u64 xp[8], wp[8];
+            load_block16<IN>(xv, (int64_t)r * ld + b * 16, xp);
+            if (WEIGHTED) {
+                const float4* w4 = reinterpret_cast<const float4*>(imp + b * 16);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float4 v = __ldg(w4 + j);
+                    wp[2 * j] = pk(v.x, v.y);
+                    wp[2 * j + 1] = pk(v.z, v.w);
+                }
+            }
+            int bp = 0;
+            if (S > 0.0f) {
+                const int p0 = e4m3_rne(__fdiv_rn(block_absmax(xp), d6));
+                float best = INFINITY;
+                bp = max(p0 + LO, 0);                      // first candidate if every error overflows
+                if (p0 + LO <= 0) best = zero_scale_error<WEIGHTED>(xp, wp);   // pattern 0 is the lowest offset
+                const int k0 = max(LO, 1 - p0), k1 = min(HI, 126 - p0);
+#pragma unroll 1
+                for (int k = k0; k <= k1; ++k) {
+                    const int p = p0 + k;
+                    const float e = sweep_error<WEIGHTED>(xp, wp, s_inv[p], s_s2[p]);
+                    if (e < best) {
+                        best = e;
+                        bp = p;
+                    }
+                }
+            }
+            *cdst = block_codes(xp, s_inv[bp]);
+            scales[blk] = (uint8_t)bp;
+        }
     }
     finish_status(ws, su.flags, WS_CNT_Q);
 }
@@ -568,15 +665,35 @@ __global__ void __launch_bounds__(kThreads) dequant_mx_kernel(const uint8_t* __r
 // ------------------------------------------------------------------------------------------
 thread_local int g_launches = 0;
 
-int grid_for(int64_t work_items, int ctas_per_sm) {
+int sm_count() {
     static int sms = 0;
     if (sms == 0) {
         int dev = 0;
         cudaGetDevice(&dev);
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) sms = 148;
     }
+    return sms;
+}
+
+// Grid for a grid-stride kernel: enough CTAs for the work, at most one full wave (the CTAs
+// the kernel's register and shared-memory use let every SM hold, and no more than
+// ctas_per_sm per SM).
+template <typename K>
+int grid_for(K kernel, int64_t work_items, int ctas_per_sm) {
+    // per-thread cache of the occupancy query, keyed by kernel address
+    thread_local const void* keys[32] = {};
+    thread_local int fits[32] = {};
+    const void* key = reinterpret_cast<const void*>(kernel);
+    int fit = 0, slot = 0;
+    for (; slot < 32 && keys[slot]; ++slot)
+        if (keys[slot] == key) { fit = fits[slot]; break; }
+    if (fit == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, kernel, kThreads, 0) != cudaSuccess || fit <= 0) fit = 1;
+        if (slot < 32) { keys[slot] = key; fits[slot] = fit; }
+    }
+    const int per_sm = fit < ctas_per_sm ? fit : ctas_per_sm;
     const int64_t need = (work_items + kThreads - 1) / kThreads;
-    const int64_t cap = (int64_t)sms * ctas_per_sm;
+    const int64_t cap = (int64_t)sm_count() * per_sm;
     return (int)(need < cap ? (need > 0 ? need : 1) : cap);
 }
 
@@ -599,23 +716,36 @@ int check_common(const void* x, int dtype, int64_t rows, int64_t cols, int64_t l
     return FP4Q_OK;
 }
 
+template <int IN, bool WEIGHTED>
+void launch_sweep(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* imp, uint8_t* codes,
+                  uint8_t* scales, float* gs, uint32_t* ws, cudaStream_t st) {
+    const int64_t total = rows * (cols / 16);
+    const int64_t ctas = (total + kThreads - 1) / kThreads;   // one quantization block per thread
+    if (total < ((int64_t)1 << 31) && rows * ld < ((int64_t)1 << 31))
+        sweep_kernel<IN, WEIGHTED, uint32_t><<<(unsigned)ctas, kThreads, 0, st>>>(
+            x, (uint32_t)rows, (uint32_t)cols, (uint32_t)ld, imp, codes, scales, gs, ws);
+    else
+        sweep_kernel<IN, WEIGHTED, int64_t><<<(unsigned)ctas, kThreads, 0, st>>>(x, rows, cols, ld, imp, codes, scales,
+                                                                                  gs, ws);
+}
+
 template <int IN>
 int launch_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, int fmt, int obj, const float* imp,
                     uint8_t* codes, uint8_t* scales, float* gs, uint32_t* ws, uint32_t flags, cudaStream_t st) {
     int n = 0;
     if (fmt == FP4Q_MXFP4) {
         const int ocp = (flags & FP4Q_F_MX_OCP_FLOOR) ? 1 : 0;
-        mxfp4_kernel<IN, false><<<grid_for(rows * (cols / 32), 8), kThreads, 0, st>>>(x, rows, cols, ld, codes,
-                                                                                   scales, ws, ocp);
+        mxfp4_kernel<IN, false><<<grid_for(mxfp4_kernel<IN, false>, rows * (cols / 32), 8), kThreads, 0, st>>>(
+            x, rows, cols, ld, codes, scales, ws, ocp);
         return launched(1);
     }
     const int given = (flags & FP4Q_F_GLOBAL_SCALE_GIVEN) ? 1 : 0;
     if (!given) {
         const int64_t vecs = rows * cols * (IN == FP4Q_IN_BF16 ? 2 : 4) / 16;
-        amax_kernel<IN><<<grid_for(vecs, 4), kThreads, 0, st>>>(x, rows, cols, ld, ws, gs, 0);
+        amax_kernel<IN><<<grid_for(amax_kernel<IN>, vecs, 4), kThreads, 0, st>>>(x, rows, cols, ld, ws, gs, 0);
         ++n;
     }
-    const int g = grid_for(rows * (cols / 16), 8);
+    const int g = grid_for(nvfp4_kernel<IN, FP4Q_ABSMAX>, rows * (cols / 16), 8);
     if (fmt == FP4Q_IF4) {
         if4_kernel<IN><<<g, kThreads, 0, st>>>(x, rows, cols, ld, codes, scales, gs, ws, given);
     } else {
@@ -628,12 +758,10 @@ int launch_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, int f
                                                                           given);
                 break;
             case FP4Q_SWEEP_MSE:
-                nvfp4_kernel<IN, FP4Q_SWEEP_MSE><<<g, kThreads, 0, st>>>(x, rows, cols, ld, imp, codes, scales, gs, ws,
-                                                                      given);
+                launch_sweep<IN, false>(x, rows, cols, ld, imp, codes, scales, gs, ws, st);
                 break;
             default:
-                nvfp4_kernel<IN, FP4Q_SWEEP_WMSE><<<g, kThreads, 0, st>>>(x, rows, cols, ld, imp, codes, scales, gs, ws,
-                                                                       given);
+                launch_sweep<IN, true>(x, rows, cols, ld, imp, codes, scales, gs, ws, st);
                 break;
         }
     }
@@ -687,9 +815,11 @@ int fp4q_global_scale(const void* x, int dtype, int64_t rows, int64_t cols, int6
     uint32_t* ws = reinterpret_cast<uint32_t*>(workspace);
     const int64_t vecs = rows * cols * (dtype == FP4Q_IN_BF16 ? 2 : 4) / 16;
     if (dtype == FP4Q_IN_BF16)
-        amax_kernel<FP4Q_IN_BF16><<<grid_for(vecs, 4), kThreads, 0, st>>>(x, rows, cols, ld, ws, global_scale, 1);
+        amax_kernel<FP4Q_IN_BF16><<<grid_for(amax_kernel<FP4Q_IN_BF16>, vecs, 4), kThreads, 0, st>>>(
+            x, rows, cols, ld, ws, global_scale, 1);
     else
-        amax_kernel<FP4Q_IN_F32><<<grid_for(vecs, 4), kThreads, 0, st>>>(x, rows, cols, ld, ws, global_scale, 1);
+        amax_kernel<FP4Q_IN_F32><<<grid_for(amax_kernel<FP4Q_IN_F32>, vecs, 4), kThreads, 0, st>>>(
+            x, rows, cols, ld, ws, global_scale, 1);
     return launched(1);
 }
 
@@ -703,7 +833,7 @@ int fp4q_hadamard_quantize(const void* x, int dtype, int64_t rows, int64_t cols,
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     uint32_t* ws = reinterpret_cast<uint32_t*>(workspace);
     const int ocp = (flags & FP4Q_F_MX_OCP_FLOOR) ? 1 : 0;
-    const int g = grid_for(rows * (cols / 32), 8);
+    const int g = grid_for(mxfp4_kernel<FP4Q_IN_BF16, true>, rows * (cols / 32), 8);
     if (dtype == FP4Q_IN_BF16)
         mxfp4_kernel<FP4Q_IN_BF16, true><<<g, kThreads, 0, st>>>(x, rows, cols, ld, codes, scales, ws, ocp);
     else
@@ -725,7 +855,7 @@ int fp4q_dequantize(const uint8_t* codes, const uint8_t* scales, const float* gl
     if (!aligned16(codes) || !aligned16(out)) return FP4Q_ERR_ALIGNMENT;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const bool bf = (flags & FP4Q_F_OUT_BF16) != 0;
-    const int g = grid_for(rows * (cols / B), 8);
+    const int g = grid_for(dequant_mx_kernel<false, true>, rows * (cols / B), 8);
     if (fmt == FP4Q_MXFP4) {
         if (bf && inverse_hadamard) dequant_mx_kernel<true, true><<<g, kThreads, 0, st>>>(codes, scales, rows, cols, out);
         else if (bf) dequant_mx_kernel<true, false><<<g, kThreads, 0, st>>>(codes, scales, rows, cols, out);

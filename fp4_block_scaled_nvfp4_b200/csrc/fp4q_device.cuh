@@ -83,6 +83,21 @@ __device__ __forceinline__ void e2m1x2_residual(u64 y, float& r0, float& r1) {
         : "=f"(r0), "=f"(r1) : "f"(a), "f"(b));
 }
 
+// The same residual pair returned as one packed register pair (for f32x2 accumulation).
+__device__ __forceinline__ u64 e2m1x2_residual2(u64 y) {
+    u64 r;
+    asm("{ .reg .b8 t; .reg .b32 h; .reg .f16 p, q; .reg .f32 a, b, r0, r1;\n"
+        "  mov.b64 {a, b}, %1;\n"
+        "  cvt.rn.satfinite.e2m1x2.f32 t, b, a;\n"
+        "  cvt.rn.f16x2.e2m1x2 h, t;\n"
+        "  mov.b32 {p, q}, h;\n"
+        "  sub.rn.f32.f16 r0, p, a;\n"
+        "  sub.rn.f32.f16 r1, q, b;\n"
+        "  mov.b64 %0, {r0, r1}; }"
+        : "=l"(r) : "l"(y));
+    return r;
+}
+
 // ---- E4M3 (FN) ----------------------------------------------------------------------------
 // Bit pattern of the nearest E4M3 value (ties to even, saturating at 448) of a finite v >= 0.
 __device__ __forceinline__ int e4m3_rne(float v) {
