@@ -26,7 +26,7 @@ BLOCK = {"nvfp4": 16, "if4": 16, "mxfp4": 32}
 
 # Names of every function include/fp4q.h declares (checked against the header by the tests).
 EXPORTS = ("fp4q_workspace_bytes", "fp4q_global_scale", "fp4q_quantize", "fp4q_hadamard_quantize", "fp4q_dequantize",
-           "fp4q_read_device_status", "fp4q_last_launch_count", "fp4q_status_string")
+           "fp4q_quantize_noalloc", "fp4q_read_device_status", "fp4q_last_launch_count", "fp4q_status_string")
 
 _lib = None
 
@@ -53,6 +53,8 @@ def lib():
         L.fp4q_hadamard_quantize.argtypes = [P, i32, i64, i64, i64, i32, P, P, P, u32, P]
         L.fp4q_dequantize.restype = i32
         L.fp4q_dequantize.argtypes = [P, P, P, i64, i64, i32, i32, P, u32, P]
+        L.fp4q_quantize_noalloc.restype = i32
+        L.fp4q_quantize_noalloc.argtypes = [P, i32, i64, i64, i64, i32, i32, P, P, P, P, P, u32, P]
         L.fp4q_read_device_status.restype = i32
         L.fp4q_read_device_status.argtypes = [P, C.POINTER(C.c_uint32), P]
         L.fp4q_last_launch_count.restype = i32
@@ -179,6 +181,29 @@ def dequantize(codes, scales, global_scale, fmt: str = "nvfp4", inverse_hadamard
                                int(inverse_hadamard), _ptr(out), flags, _stream_ptr(stream))
     _check(rc, "fp4q_dequantize")
     return out
+
+
+def quantize_noalloc(x, fmt: str = "nvfp4", objective: str = "sweep_mse", importance=None, global_scale=None,
+                     mx_ocp_floor: bool = False, out=None, device_status=None, stream=None):
+    """quantize() for callers that cannot allocate device memory: the library's own
+    per-GPU scratch replaces the workspace (see fp4q_quantize_noalloc in include/fp4q.h).
+    Outputs must be passed in `out`; device_status is an optional [1] int32 CUDA tensor."""
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise Fp4qError("x must be 2-D with unit column stride")
+    rows, cols = x.shape
+    codes, scales, gs = out
+    flags = 0
+    if global_scale is not None:
+        flags |= F_GLOBAL_SCALE_GIVEN
+        gs = global_scale
+    if mx_ocp_floor:
+        flags |= F_MX_OCP_FLOOR
+    rc = lib().fp4q_quantize_noalloc(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), FORMATS[fmt],
+                                     OBJECTIVES.get(objective, 0), _ptr(importance), _ptr(codes), _ptr(scales),
+                                     _ptr(gs) if fmt != "mxfp4" else None, _ptr(device_status), flags,
+                                     _stream_ptr(stream))
+    _check(rc, "fp4q_quantize_noalloc")
+    return codes, scales, (gs if fmt != "mxfp4" else None)
 
 
 def read_device_status(workspace, stream=None) -> int:

@@ -24,6 +24,7 @@
 // after every call.
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 #include <cuda_runtime.h>
 
 #include "fp4q.h"
@@ -768,6 +769,33 @@ int launch_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, int f
     return launched(n + 1);
 }
 
+// Scratch for fp4q_quantize_noalloc: the 64 bytes a quantize call keeps on the device
+// (status word, amax word, arrival counters) live in this file-scope array instead of a
+// caller-allocated workspace.  Every GPU that loads the library holds these 256 bytes until
+// the process exits.  In host code the name is only a stand-in for the symbol; the device
+// address comes from cudaGetSymbolAddress, looked up once per device.
+static __device__ __align__(256) uint32_t g_noalloc_scratch[64];
+constexpr size_t kNoAllocScratchBytes = sizeof(g_noalloc_scratch);
+static_assert(kWorkspaceBytes <= kNoAllocScratchBytes, "no-alloc scratch smaller than a workspace");
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (set up on first use).
+int noalloc_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FP4Q_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return FP4Q_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return FP4Q_ERR_CUDA;
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return FP4Q_OK;
+}
+
 }  // namespace fp4q
 
 using namespace fp4q;
@@ -869,6 +897,39 @@ int fp4q_dequantize(const uint8_t* codes, const uint8_t* scales, const float* gl
         else dequant16_kernel<false, false><<<g, kThreads, 0, st>>>(codes, scales, global_scale, rows, cols, out);
     }
     return launched(1);
+}
+
+int fp4q_quantize_noalloc(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld, int fmt,
+                          int objective, const float* importance, uint8_t* codes, uint8_t* scales,
+                          float* global_scale, uint32_t* device_status, uint32_t flags, void* stream) {
+    g_launches = 0;
+    // the same argument checks as fp4q_quantize, made before the scratch is touched
+    if (fmt != FP4Q_NVFP4 && fmt != FP4Q_IF4 && fmt != FP4Q_MXFP4) return FP4Q_ERR_INVALID_ARG;
+    if (flags & ~(FP4Q_F_GLOBAL_SCALE_GIVEN | FP4Q_F_MX_OCP_FLOOR)) return FP4Q_ERR_INVALID_ARG;
+    if (fmt == FP4Q_NVFP4 && (objective < FP4Q_ABSMAX || objective > FP4Q_SWEEP_WMSE)) return FP4Q_ERR_INVALID_ARG;
+    const int B = fmt == FP4Q_MXFP4 ? 32 : 16;
+    const void* aligned_stand_in = reinterpret_cast<const void*>(static_cast<uintptr_t>(256));
+    int rc0 = check_common(x, dtype, rows, cols, ld, B, codes, scales, aligned_stand_in);
+    if (rc0 != FP4Q_OK || rows == 0 || cols == 0) return rc0;
+    if (fmt != FP4Q_MXFP4 && !global_scale) return FP4Q_ERR_INVALID_ARG;
+    if (fmt == FP4Q_NVFP4 && objective == FP4Q_SWEEP_WMSE) {
+        if (!importance) return FP4Q_ERR_INVALID_ARG;
+        if (!aligned16(importance)) return FP4Q_ERR_ALIGNMENT;
+    }
+    if (fmt == FP4Q_MXFP4 && (flags & FP4Q_F_GLOBAL_SCALE_GIVEN)) return FP4Q_ERR_INVALID_ARG;
+    if (device_status && (reinterpret_cast<uintptr_t>(device_status) & 3u)) return FP4Q_ERR_ALIGNMENT;
+    void* scratch = nullptr;
+    int rc = noalloc_scratch(&scratch);
+    if (rc != FP4Q_OK) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // the previous call's words (and anything an interrupted call left) start from zero
+    if (cudaMemsetAsync(scratch, 0, kWorkspaceBytes, st) != cudaSuccess) return FP4Q_ERR_CUDA;
+    rc = fp4q_quantize(x, dtype, rows, cols, ld, fmt, objective, importance, codes, scales, global_scale, scratch,
+                       flags, stream);
+    if (rc == FP4Q_OK && device_status &&
+        cudaMemcpyAsync(device_status, scratch, sizeof(uint32_t), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+        return FP4Q_ERR_CUDA;
+    return rc;
 }
 
 int fp4q_read_device_status(const void* workspace, uint32_t* status, void* stream) {

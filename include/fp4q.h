@@ -138,6 +138,31 @@ int fp4q_dequantize(const uint8_t* codes, const uint8_t* scales, const float* gl
                     int64_t rows, int64_t cols, int fmt, int inverse_hadamard,
                     void* out, uint32_t flags, void* stream);
 
+/*
+ * fp4q_quantize for callers that cannot allocate device memory.  The pages have no
+ * counterpart; this is a deployment convenience.  Some callers run where the allocator is
+ * off limits: code inside another framework's stream capture or memory pool, a plugin that
+ * gets only the tensors it works on, or an inference engine that plans every allocation
+ * ahead of time.  They cannot hand over the zeroed workspace fp4q_quantize wants.  This
+ * entry point keeps that scratch (64 bytes: status word, amax word, arrival counters) in a
+ * 256-byte array compiled into the library, one per GPU, held until the process exits.
+ * It calls no cudaMalloc, cudaFree or other allocating routine.
+ *   Arguments and results are those of fp4q_quantize, minus `workspace`.  device_status is
+ *   an optional device uint32 (4-byte aligned, may be NULL); it receives the call's
+ *   FP4Q_DEVSTAT_* word, copied asynchronously on `stream`.
+ *   The scratch need does not grow with the tensor, so every shape fp4q_quantize accepts
+ *   fits; larger tensors (2^40 elements and up) are rejected with FP4Q_ERR_SHAPE as there.
+ *   The first call on a device looks up the array's address (cudaGetSymbolAddress) with
+ *   that device current.  Make that first call before any stream capture.
+ *   Every call clears the scratch on `stream` before using it, and all calls on a device
+ *   share it: calls that may run at the same time on the GPU (different streams, different
+ *   host threads) race and must be serialized by the caller.
+ */
+int fp4q_quantize_noalloc(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                          int fmt, int objective, const float* importance,
+                          uint8_t* codes, uint8_t* scales, float* global_scale,
+                          uint32_t* device_status, uint32_t flags, void* stream);
+
 /* Copy the device status word of `workspace` to *status (blocks until `stream` is done). */
 int fp4q_read_device_status(const void* workspace, uint32_t* status, void* stream);
 
