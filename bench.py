@@ -38,6 +38,11 @@ WORKLOADS = {
     "cfg5h": ("cfg5", "mxfp4_had", None, "MXFP4 after 32x32 block Hadamard, bf16 activations 16384x8192"),
 }
 METRIC = "quantize GB/s (input bf16) and % of B200 HBM peak, 1 GPU, vs CPU oracle"
+# Arithmetic the method itself needs per element for the ALU-bound searches: per candidate
+# scale one multiply (x/s), one E2M1 rounding, one subtraction (residual) and one fused
+# multiply-add (square-accumulate) -- plus, for WMSE, the weight multiply -- over 11 (MSE) or
+# 16 (WMSE) candidates, plus the block maximum and the final multiply + rounding.
+ALU_OPS_PER_ELEMENT = {"sweep_mse": 11 * 4 + 3, "sweep_wmse": 16 * 5 + 3}
 L2_BYTES = 126 * 2 ** 20
 
 
@@ -238,13 +243,14 @@ def run_ours(args, rank, world):
         c, sc, g = outs[s]
         if ev is not None:
             ev[0].record()
-        if fmt.startswith("mxfp4"):
+        if fmt.startswith("mxfp4"):   # one kernel, no tensor scale: the amax slot stays empty
+            if ev is not None:
+                ev[1].record()
             if fmt.endswith("had"):
                 fq.hadamard_quantize(xs[s], out=(c, sc, None), workspace=ws)
             else:
                 fq.quantize(xs[s], "mxfp4", out=(c, sc, None), workspace=ws)
             if ev is not None:
-                ev[1].record()
                 ev[2].record()
             return 1
         fq.global_scale(xs[s], out=g, workspace=ws)
@@ -335,6 +341,26 @@ def run_ours(args, rank, world):
     tq = statistics.mean(t_q)
     kernel_key = f"{args.workload}:quantize"
     achieved = alg / (tq * 1e-3) / 1e9
+    clocks = clk.summary()
+    traffic = profiled_traffic(kernel_key)
+    hbm_roof = {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": "quantize (" + (obj or fmt) + ")",
+                "peak_source": f"{peak_src} hbm_gbs (copy, burst) from MEASURED_PEAKS.json"}
+    ops = ALU_OPS_PER_ELEMENT.get(obj or fmt)
+    if ops is not None:
+        # the candidate search is bound by plain FP32/convert arithmetic, not by HBM: the peak is
+        # 148 SMs x 128 FP32 lanes x the SM clock sampled during the timed region
+        mhz = clocks["sm_mhz"] or clocks["sm_max_mhz"] or 1965.0
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        alu_peak = sms * 128 * mhz * 1e6 / 1e9
+        alu_ach = ops * rows * cols / (tq * 1e-3) / 1e9
+        roofline = {"bound": "alu", "achieved": round(alu_ach, 1), "peak": round(alu_peak, 1), "unit": "Gop/s",
+                    "frac": round(alu_ach / alu_peak, 4), "traffic": traffic, "kernel": "quantize (" + obj + ")",
+                    "ops_per_element": ops,
+                    "peak_source": f"{sms} SMs x 128 FP32 lanes x {mhz:.0f} MHz (median SM clock in the timed region)",
+                    "hbm": {k: hbm_roof[k] for k in ("achieved", "peak", "unit", "frac")}}
+    else:
+        roofline = hbm_roof
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(per_step_ms, 5), "higher_is_better": True, "scaling": "weak",
@@ -347,14 +373,12 @@ def run_ours(args, rank, world):
         "hbm_frac": round(value / world / peak, 4),
         "input_gbps": round(in_bytes * args.steps * world / (ms * 1e-3) / 1e9, 2),
         "elements_per_s": round(rows * cols * args.steps * world / (ms * 1e-3), 1),
-        "kernels_ms": {"amax": round(statistics.mean(t_amax), 5), "quantize": round(tq, 5)},
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": profiled_traffic(kernel_key),
-                     "kernel": "quantize (" + (obj or fmt) + ")",
-                     "peak_source": f"{peak_src} hbm_gbs (copy, burst) from MEASURED_PEAKS.json"},
+        "kernels_ms": {"amax": (None if fmt.startswith("mxfp4") else round(statistics.mean(t_amax), 5)),
+                       "quantize": round(tq, 5)},
+        "roofline": roofline,
         "device_status": st,
         "gpu_launches": launches_per_step * args.steps,
-        "clocks": clk.summary(),
+        "clocks": clocks,
         "e2e": {"value": round(alg / (e2e_ms * 1e-3) / 1e9 * world, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
     }

@@ -7,7 +7,7 @@
 //                        the last CTA to arrive computes S = RN(amax/1536) and the data
 //                        flags.  ScaleSweep (gist.science/ko/paper/2606.07618),
 //                        "Methodology", global scale S = max|x|/(256*6).
-//   nvfp4_kernel<OBJ>    base scale, candidate sweep, RTN, block error, argmin, nibble
+//   quant16_kernel<OBJ>  base scale, candidate sweep, RTN, block error, argmin, nibble
 //                        pack, scale write.  ScaleSweep "Methodology" (offsets [-3,+7] MSE,
 //                        [-8,+7] WMSE), 4/6 (Adaptive Block-Scaled Data Types,
 //                        gist.science/ko/paper/2603.28765, "Problem").
@@ -200,48 +200,6 @@ __device__ __forceinline__ float block_absmax(const u64 (&xp)[8]) {
     return m;
 }
 
-// Error of one candidate: with y = RN(x inv) and codes q = E2M1(y), the residuals
-// r = RN(q - y) (units of the scale) are squared and summed by fma into an (even, odd) pair
-// of accumulators, combined once, and scaled by s2 = RN(sv^2).  For the zero scale (sv = 0)
-// every code is 0 and the error is the same fma sum over x itself (no scaling).
-template <bool WEIGHTED>
-__device__ __forceinline__ float candidate_error(const u64 (&xp)[8], const u64 (&wp)[8], float sv, float inv, float s2) {
-    float ae = 0.0f, ao = 0.0f;
-    if (sv == 0.0f) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            float a, b;
-            upk(xp[j], a, b);
-            if (WEIGHTED) {
-                float w0, w1;
-                upk(wp[j], w0, w1);
-                ae = __fmaf_rn(__fmul_rn(w0, a), a, ae);
-                ao = __fmaf_rn(__fmul_rn(w1, b), b, ao);
-            } else {
-                ae = __fmaf_rn(a, a, ae);
-                ao = __fmaf_rn(b, b, ao);
-            }
-        }
-        return __fadd_rn(ae, ao);
-    }
-    const u64 inv2 = pk(inv, inv);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        float r0, r1;
-        e2m1x2_residual(mul2(xp[j], inv2), r0, r1);
-        if (WEIGHTED) {
-            float w0, w1;
-            upk(wp[j], w0, w1);
-            ae = __fmaf_rn(__fmul_rn(w0, r0), r0, ae);
-            ao = __fmaf_rn(__fmul_rn(w1, r1), r1, ao);
-        } else {
-            ae = __fmaf_rn(r0, r0, ae);
-            ao = __fmaf_rn(r1, r1, ao);
-        }
-    }
-    return __fmul_rn(s2, __fadd_rn(ae, ao));
-}
-
 // Packed codes of a block for a given reciprocal scale (8 bytes: elements 0..15).
 __device__ __forceinline__ uint2 block_codes(const u64 (&xp)[8], float inv) {
     const u64 inv2 = pk(inv, inv);
@@ -252,87 +210,9 @@ __device__ __forceinline__ uint2 block_codes(const u64 (&xp)[8], float inv) {
                       c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24));
 }
 
-// ------------------------------------------------------------------------------------------
-// NVFP4: AbsMax / 4-over-6 / ScaleSweep MSE / ScaleSweep WMSE
-// ------------------------------------------------------------------------------------------
-template <int IN, int OBJ>
-__global__ void __launch_bounds__(kThreads) nvfp4_kernel(const void* __restrict__ xv, int64_t rows, int64_t cols,
-                                                         int64_t ld, const float* __restrict__ imp,
-                                                         uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
-                                                         const float* __restrict__ gscale, uint32_t* __restrict__ ws,
-                                                         int s_given) {
-    __shared__ float s_sv[128], s_inv[128], s_s2[128];
-    const Setup su = read_setup(gscale);
-    build_scale_table(su.S, s_sv, s_inv, s_s2);
-    const float S = su.S;
-    const float d6 = __fmul_rn(6.0f, S), d4 = __fmul_rn(4.0f, S);
-    const int64_t nb = cols / 16;
-    const int64_t total = rows * nb;
-    const int64_t step = (int64_t)gridDim.x * blockDim.x;
-    constexpr int LO = OBJ == FP4Q_SWEEP_MSE ? -3 : (OBJ == FP4Q_SWEEP_WMSE ? -8 : 0);
-    constexpr int HI = (OBJ == FP4Q_SWEEP_MSE || OBJ == FP4Q_SWEEP_WMSE) ? 7 : 0;
-    constexpr bool WEIGHTED = OBJ == FP4Q_SWEEP_WMSE;
-
-    for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < total; blk += step) {
-        const int64_t r = blk / nb, b = blk - r * nb;
-        uint2* cdst = reinterpret_cast<uint2*>(codes + r * (cols / 2) + b * 8);
-        if (su.flags) {   // data out of contract: zero-filled outputs
-            *cdst = make_uint2(0u, 0u);
-            scales[blk] = 0;
-            continue;
-        }
-        u64 xp[8];
-        load_block16<IN>(xv, r * ld + b * 16, xp);
-        int bp = 0;
-        if (S > 0.0f) {
-            const float ab = block_absmax(xp);
-            const int p0 = e4m3_rne(__fdiv_rn(ab, d6));
-            bp = p0;
-            if (OBJ == FP4Q_FOUR_OVER_SIX) {
-                const int p4 = e4m3_rne(__fdiv_rn(ab, d4));
-                if (p4 != p0) {
-                    u64 wp[8];
-                    const float e0 = candidate_error<false>(xp, wp, s_sv[p0], s_inv[p0], s_s2[p0]);
-                    const float e4 = candidate_error<false>(xp, wp, s_sv[p4], s_inv[p4], s_s2[p4]);
-                    if (e4 < e0) bp = p4;
-                }
-            } else if (OBJ == FP4Q_SWEEP_MSE || OBJ == FP4Q_SWEEP_WMSE) {
-                u64 wp[8];
-                if (WEIGHTED) {
-                    const float4* w4 = reinterpret_cast<const float4*>(imp + b * 16);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const float4 v = __ldg(w4 + j);
-                        wp[2 * j] = pk(v.x, v.y);
-                        wp[2 * j + 1] = pk(v.z, v.w);
-                    }
-                }
-                float best = INFINITY;
-                bp = max(p0 + LO, 0);
-#pragma unroll 1
-                for (int k = LO; k <= HI; ++k) {
-                    const int p = p0 + k;
-                    const bool valid = (unsigned)p <= 126u;
-                    const int pc = valid ? p : 0;
-                    const float e = candidate_error<WEIGHTED>(xp, wp, s_sv[pc], s_inv[pc], s_s2[pc]);
-                    if (valid && e < best) {
-                        best = e;
-                        bp = p;
-                    }
-                }
-            }
-        }
-        *cdst = block_codes(xp, s_inv[bp]);
-        scales[blk] = (uint8_t)bp;
-    }
-    finish_status(ws, su.flags, WS_CNT_Q);
-}
-
-// ------------------------------------------------------------------------------------------
-// NVFP4 ScaleSweep (MSE window [-3,+7], WMSE window [-8,+7]): one thread per block, every
-// candidate evaluated in registers; the zero scale (only in the window of tiny blocks) is
-// scored once before the loop so the loop itself is branch-free.
-// ------------------------------------------------------------------------------------------
+// Error of one candidate with a nonzero scale: y = RN(x inv), residuals r = RN(q - y) in units
+// of the scale, squares summed by packed fma into (even, odd) accumulators, combined once and
+// scaled by s2 = RN(sv^2).  WMSE: acc = fma(RN(w r), r, acc).
 template <bool WEIGHTED>
 __device__ __forceinline__ float sweep_error(const u64 (&xp)[8], const u64 (&wp)[8], float inv, float s2) {
     const u64 inv2 = pk(inv, inv);
@@ -347,6 +227,8 @@ __device__ __forceinline__ float sweep_error(const u64 (&xp)[8], const u64 (&wp)
     return __fmul_rn(s2, __fadd_rn(a, b));
 }
 
+// Error of the zero scale (pattern 0): every code is 0, so the error is the fma sum of x^2
+// (WMSE: RN(w x) x) in the same (even, odd) order, unscaled.
 template <bool WEIGHTED>
 __device__ __forceinline__ float zero_scale_error(const u64 (&xp)[8], const u64 (&wp)[8]) {
     u64 acc = pk(0.0f, 0.0f);
@@ -357,126 +239,149 @@ __device__ __forceinline__ float zero_scale_error(const u64 (&xp)[8], const u64 
     return __fadd_rn(a, b);
 }
 
-template <int IN, bool WEIGHTED, typename IDX>
-__global__ void __launch_bounds__(kThreads, WEIGHTED ? 4 : 6) sweep_kernel(const void* __restrict__ xv, IDX rows, IDX cols, IDX ld,
-                                                            const float* __restrict__ imp,
-                                                            uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
-                                                            const float* __restrict__ gscale, uint32_t* __restrict__ ws) {
+// ------------------------------------------------------------------------------------------
+// NVFP4: AbsMax / 4-over-6 / ScaleSweep MSE [-3,+7] / ScaleSweep WMSE [-8,+7].
+// One thread owns one 16-element block and keeps it in registers for the whole candidate
+// search; one block per thread (no grid-stride tail).  The zero scale, which only enters
+// the window of tiny blocks, is scored once before the candidate loop so the loop is
+// branch-free.  The status word depends only on S, so CTA 0 writes it.
+// ScaleSweep (gist.science/ko/paper/2606.07618), Methodology; 4/6: Adaptive Block-Scaled
+// Data Types (gist.science/ko/paper/2603.28765), Problem.
+// ------------------------------------------------------------------------------------------
+template <int IN, int OBJ, typename IDX>
+__global__ void __launch_bounds__(kThreads, OBJ == FP4Q_SWEEP_WMSE ? 4 : 6)
+    quant16_kernel(const void* __restrict__ xv, IDX rows, IDX cols, IDX ld, const float* __restrict__ imp,
+                   uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, const float* __restrict__ gscale,
+                   uint32_t* __restrict__ ws) {
+    constexpr bool SWEEP = OBJ == FP4Q_SWEEP_MSE || OBJ == FP4Q_SWEEP_WMSE;
+    constexpr bool WEIGHTED = OBJ == FP4Q_SWEEP_WMSE;
+    constexpr int LO = WEIGHTED ? -8 : -3, HI = 7;
     __shared__ float s_sv[128], s_inv[128], s_s2[128];
     const Setup su = read_setup(gscale);
+    if (blockIdx.x == 0 && threadIdx.x == 0) ws[WS_STATUS] = su.flags;
     build_scale_table(su.S, s_sv, s_inv, s_s2);
     const float S = su.S;
-    const float d6 = __fmul_rn(6.0f, S);
-    constexpr int LO = WEIGHTED ? -8 : -3, HI = 7;
+    const float d6 = __fmul_rn(6.0f, S), d4 = __fmul_rn(4.0f, S);
     const IDX nb = cols / 16;
     const IDX total = rows * nb;
     const IDX blk = (IDX)blockIdx.x * blockDim.x + threadIdx.x;
-    if (blk < total) {
-        const IDX r = blk / nb, b = blk - r * nb;
-        uint2* cdst = reinterpret_cast<uint2*>(codes + r * (cols / 2) + b * 8);
-        if (su.flags) {   // data out of contract: zero-filled outputs
-            *cdst = make_uint2(0u, 0u);
-            scales[blk] = 0;
-        } else {
-            u64 xp[8], wp[8];
-            load_block16<IN>(xv, (int64_t)r * ld + b * 16, xp);
-            if (WEIGHTED) {
-                const float4* w4 = reinterpret_cast<const float4*>(imp + b * 16);
+    if (blk >= total) return;
+    const IDX r = blk / nb, b = blk - r * nb;
+    uint2* cdst = reinterpret_cast<uint2*>(codes + r * (cols / 2) + b * 8);
+    if (su.flags) {   // data out of contract: zero-filled outputs
+        *cdst = make_uint2(0u, 0u);
+        scales[blk] = 0;
+        return;
+    }
+    u64 xp[8], wp[8];
+    load_block16<IN>(xv, (int64_t)r * ld + b * 16, xp);
+    if (WEIGHTED) {
+        const float4* w4 = reinterpret_cast<const float4*>(imp + b * 16);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float4 v = __ldg(w4 + j);
-                    wp[2 * j] = pk(v.x, v.y);
-                    wp[2 * j + 1] = pk(v.z, v.w);
-                }
-            }
-            int bp = 0;
-            if (S > 0.0f) {
-                const int p0 = e4m3_rne(__fdiv_rn(block_absmax(xp), d6));
-                float best = INFINITY;
-                bp = max(p0 + LO, 0);                      // first candidate if every error overflows
-                if (p0 + LO <= 0) best = zero_scale_error<WEIGHTED>(xp, wp);   // pattern 0 is the lowest offset
-                const int k0 = max(LO, 1 - p0), k1 = min(HI, 126 - p0);
-#pragma unroll 1
-                for (int k = k0; k <= k1; ++k) {
-                    const int p = p0 + k;
-                    const float e = sweep_error<WEIGHTED>(xp, wp, s_inv[p], s_s2[p]);
-                    if (e < best) {
-                        best = e;
-                        bp = p;
-                    }
-                }
-            }
-            *cdst = block_codes(xp, s_inv[bp]);
-            scales[blk] = (uint8_t)bp;
+        for (int j = 0; j < 4; ++j) {
+            const float4 v = __ldg(w4 + j);
+            wp[2 * j] = pk(v.x, v.y);
+            wp[2 * j + 1] = pk(v.z, v.w);
         }
     }
-    finish_status(ws, su.flags, WS_CNT_Q);
+    int bp = 0;
+    if (S > 0.0f) {
+        const float ab = block_absmax(xp);
+        const int p0 = e4m3_rne(__fdiv_rn(ab, d6));
+        bp = p0;
+        if (OBJ == FP4Q_FOUR_OVER_SIX) {
+            const int p4 = e4m3_rne(__fdiv_rn(ab, d4));   // p4 >= p0
+            if (p4 != p0) {
+                const float e0 = p0 == 0 ? zero_scale_error<false>(xp, wp) : sweep_error<false>(xp, wp, s_inv[p0], s_s2[p0]);
+                const float e4 = sweep_error<false>(xp, wp, s_inv[p4], s_s2[p4]);
+                if (e4 < e0) bp = p4;
+            }
+        } else if (SWEEP) {
+            float best = INFINITY;
+            bp = max(p0 + LO, 0);                                   // first candidate if every error overflows
+            if (p0 + LO <= 0) best = zero_scale_error<WEIGHTED>(xp, wp);   // pattern 0 is the lowest offset
+            const int k0 = max(LO, 1 - p0), k1 = min(HI, 126 - p0);
+#pragma unroll 1
+            for (int k = k0; k <= k1; ++k) {
+                const int p = p0 + k;
+                const float e = sweep_error<WEIGHTED>(xp, wp, s_inv[p], s_s2[p]);
+                if (e < best) {
+                    best = e;
+                    bp = p;
+                }
+            }
+        }
+    }
+    *cdst = block_codes(xp, s_inv[bp]);
+    scales[blk] = (uint8_t)bp;
 }
 
 // ------------------------------------------------------------------------------------------
-// IF4
+// IF4: per block, FP4 (E2M1) vs scaled INT4 at the shared AbsMax scale, lower error kept,
+// indicator in bit 7 of the scale byte.  Adaptive Block-Scaled Data Types
+// (gist.science/ko/paper/2603.28765), Methodology, IF4 structure and the 6/7 method.
+// Both errors are in units of the shared scale: FP4 r = RN(q - y); INT4 z = RN(y RN(7/6)),
+// n = clamp(rint(z), -7, 7), r = RN(RN(n RN(6/7)) - y).
 // ------------------------------------------------------------------------------------------
-template <int IN>
-__global__ void __launch_bounds__(kThreads) if4_kernel(const void* __restrict__ xv, int64_t rows, int64_t cols,
-                                                       int64_t ld, uint8_t* __restrict__ codes,
-                                                       uint8_t* __restrict__ scales, const float* __restrict__ gscale,
-                                                       uint32_t* __restrict__ ws, int s_given) {
+template <int IN, typename IDX>
+__global__ void __launch_bounds__(kThreads, 4)
+    if4_kernel(const void* __restrict__ xv, IDX rows, IDX cols, IDX ld, uint8_t* __restrict__ codes,
+               uint8_t* __restrict__ scales, const float* __restrict__ gscale, uint32_t* __restrict__ ws) {
     __shared__ float s_sv[128], s_inv[128], s_s2[128];
     const Setup su = read_setup(gscale);
+    if (blockIdx.x == 0 && threadIdx.x == 0) ws[WS_STATUS] = su.flags;
     build_scale_table(su.S, s_sv, s_inv, s_s2);
     const float S = su.S;
     const float d6 = __fmul_rn(6.0f, S);
     const float K76 = __fdiv_rn(7.0f, 6.0f), K67 = __fdiv_rn(6.0f, 7.0f);
     const u64 k76 = pk(K76, K76);
-    const int64_t nb = cols / 16;
-    const int64_t total = rows * nb;
-    const int64_t step = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < total; blk += step) {
-        const int64_t r = blk / nb, b = blk - r * nb;
-        uint2* cdst = reinterpret_cast<uint2*>(codes + r * (cols / 2) + b * 8);
-        if (su.flags) {
-            *cdst = make_uint2(0u, 0u);
-            scales[blk] = 0;
-            continue;
-        }
-        u64 xp[8];
-        load_block16<IN>(xv, r * ld + b * 16, xp);
-        const int p0 = S > 0.0f ? e4m3_rne(__fdiv_rn(block_absmax(xp), d6)) : 0;
-        const float inv = s_inv[p0];
-        const u64 inv2 = pk(inv, inv);
-        float fe = 0.0f, fo = 0.0f, ie = 0.0f, io = 0.0f;
-        uint32_t cf[8], ci[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const u64 y = mul2(xp[j], inv2);
-            cf[j] = e2m1x2(y);
-            float r0, r1;
-            e2m1x2_residual(y, r0, r1);
-            fe = __fmaf_rn(r0, r0, fe);
-            fo = __fmaf_rn(r1, r1, fo);
-            float y0, y1, z0, z1;
-            upk(y, y0, y1);
-            upk(mul2(y, k76), z0, z1);
-            float n0, n1;
-            asm("cvt.rni.f32.f32 %0, %1;" : "=f"(n0) : "f"(z0));
-            asm("cvt.rni.f32.f32 %0, %1;" : "=f"(n1) : "f"(z1));
-            n0 = fminf(fmaxf(n0, -7.0f), 7.0f);
-            n1 = fminf(fmaxf(n1, -7.0f), 7.0f);
-            const float v0 = __fmul_rn(n0, K67), v1 = __fmul_rn(n1, K67);
-            const float s0 = __fsub_rn(v0, y0), s1 = __fsub_rn(v1, y1);
-            ie = __fmaf_rn(s0, s0, ie);
-            io = __fmaf_rn(s1, s1, io);
-            ci[j] = ((uint32_t)__float2int_rn(n0) & 0xFu) | (((uint32_t)__float2int_rn(n1) & 0xFu) << 4);
-        }
-        const float ef = __fadd_rn(fe, fo);
-        const float ei = __fadd_rn(ie, io);
-        const bool use_int = ei < ef;
-        const uint32_t* cc = use_int ? ci : cf;
-        *cdst = make_uint2(cc[0] | (cc[1] << 8) | (cc[2] << 16) | (cc[3] << 24),
-                           cc[4] | (cc[5] << 8) | (cc[6] << 16) | (cc[7] << 24));
-        scales[blk] = (uint8_t)(p0 | (use_int ? 0x80 : 0));
+    const IDX nb = cols / 16;
+    const IDX total = rows * nb;
+    const IDX blk = (IDX)blockIdx.x * blockDim.x + threadIdx.x;
+    if (blk >= total) return;
+    const IDX r = blk / nb, b = blk - r * nb;
+    uint2* cdst = reinterpret_cast<uint2*>(codes + r * (cols / 2) + b * 8);
+    if (su.flags) {
+        *cdst = make_uint2(0u, 0u);
+        scales[blk] = 0;
+        return;
     }
-    finish_status(ws, su.flags, WS_CNT_Q);
+    u64 xp[8];
+    load_block16<IN>(xv, (int64_t)r * ld + b * 16, xp);
+    const int p0 = S > 0.0f ? e4m3_rne(__fdiv_rn(block_absmax(xp), d6)) : 0;
+    const float inv = s_inv[p0];
+    const u64 inv2 = pk(inv, inv);
+    u64 accf = pk(0.0f, 0.0f), acci = pk(0.0f, 0.0f);
+    uint32_t cf[8], ci[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const u64 y = mul2(xp[j], inv2);
+        const u64 rf = e2m1x2_code_residual2(y, cf[j]);
+        accf = fma2(rf, rf, accf);
+        float z0, z1, n0, n1;
+        upk(mul2(y, k76), z0, z1);
+        asm("cvt.rni.f32.f32 %0, %1;" : "=f"(n0) : "f"(z0));
+        asm("cvt.rni.f32.f32 %0, %1;" : "=f"(n1) : "f"(z1));
+        n0 = fminf(fmaxf(n0, -7.0f), 7.0f);
+        n1 = fminf(fmaxf(n1, -7.0f), 7.0f);
+        // scalar .rn intrinsics: a packed multiply feeding a packed subtract can be contracted
+        // into one fused operation by the assembler, which would skip the rounding of v
+        float y0, y1;
+        upk(y, y0, y1);
+        const u64 ri = pk(__fsub_rn(__fmul_rn(n0, K67), y0), __fsub_rn(__fmul_rn(n1, K67), y1));
+        acci = fma2(ri, ri, acci);
+        ci[j] = ((uint32_t)__float2int_rn(n0) & 0xFu) | (((uint32_t)__float2int_rn(n1) & 0xFu) << 4);
+    }
+    float a, c;
+    upk(accf, a, c);
+    const float ef = __fadd_rn(a, c);
+    upk(acci, a, c);
+    const float ei = __fadd_rn(a, c);
+    const bool use_int = ei < ef;
+    const uint32_t* cc = use_int ? ci : cf;
+    *cdst = make_uint2(cc[0] | (cc[1] << 8) | (cc[2] << 16) | (cc[3] << 24),
+                       cc[4] | (cc[5] << 8) | (cc[6] << 16) | (cc[7] << 24));
+    scales[blk] = (uint8_t)(p0 | (use_int ? 0x80 : 0));
 }
 
 // ------------------------------------------------------------------------------------------
@@ -717,17 +622,29 @@ int check_common(const void* x, int dtype, int64_t rows, int64_t cols, int64_t l
     return FP4Q_OK;
 }
 
-template <int IN, bool WEIGHTED>
-void launch_sweep(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* imp, uint8_t* codes,
-                  uint8_t* scales, float* gs, uint32_t* ws, cudaStream_t st) {
+// One quantization block per thread; 32-bit index arithmetic when the tensor allows it.
+template <int IN, int OBJ>
+void launch_q16(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* imp, uint8_t* codes,
+                uint8_t* scales, float* gs, uint32_t* ws, cudaStream_t st) {
     const int64_t total = rows * (cols / 16);
-    const int64_t ctas = (total + kThreads - 1) / kThreads;   // one quantization block per thread
+    const unsigned ctas = (unsigned)((total + kThreads - 1) / kThreads);
     if (total < ((int64_t)1 << 31) && rows * ld < ((int64_t)1 << 31))
-        sweep_kernel<IN, WEIGHTED, uint32_t><<<(unsigned)ctas, kThreads, 0, st>>>(
-            x, (uint32_t)rows, (uint32_t)cols, (uint32_t)ld, imp, codes, scales, gs, ws);
+        quant16_kernel<IN, OBJ, uint32_t><<<ctas, kThreads, 0, st>>>(x, (uint32_t)rows, (uint32_t)cols, (uint32_t)ld,
+                                                                      imp, codes, scales, gs, ws);
     else
-        sweep_kernel<IN, WEIGHTED, int64_t><<<(unsigned)ctas, kThreads, 0, st>>>(x, rows, cols, ld, imp, codes, scales,
-                                                                                  gs, ws);
+        quant16_kernel<IN, OBJ, int64_t><<<ctas, kThreads, 0, st>>>(x, rows, cols, ld, imp, codes, scales, gs, ws);
+}
+
+template <int IN>
+void launch_if4(const void* x, int64_t rows, int64_t cols, int64_t ld, uint8_t* codes, uint8_t* scales, float* gs,
+                uint32_t* ws, cudaStream_t st) {
+    const int64_t total = rows * (cols / 16);
+    const unsigned ctas = (unsigned)((total + kThreads - 1) / kThreads);
+    if (total < ((int64_t)1 << 31) && rows * ld < ((int64_t)1 << 31))
+        if4_kernel<IN, uint32_t><<<ctas, kThreads, 0, st>>>(x, (uint32_t)rows, (uint32_t)cols, (uint32_t)ld, codes,
+                                                             scales, gs, ws);
+    else
+        if4_kernel<IN, int64_t><<<ctas, kThreads, 0, st>>>(x, rows, cols, ld, codes, scales, gs, ws);
 }
 
 template <int IN>
@@ -746,24 +663,16 @@ int launch_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, int f
         amax_kernel<IN><<<grid_for(amax_kernel<IN>, vecs, 4), kThreads, 0, st>>>(x, rows, cols, ld, ws, gs, 0);
         ++n;
     }
-    const int g = grid_for(nvfp4_kernel<IN, FP4Q_ABSMAX>, rows * (cols / 16), 8);
     if (fmt == FP4Q_IF4) {
-        if4_kernel<IN><<<g, kThreads, 0, st>>>(x, rows, cols, ld, codes, scales, gs, ws, given);
+        launch_if4<IN>(x, rows, cols, ld, codes, scales, gs, ws, st);
     } else {
         switch (obj) {
-            case FP4Q_ABSMAX:
-                nvfp4_kernel<IN, FP4Q_ABSMAX><<<g, kThreads, 0, st>>>(x, rows, cols, ld, imp, codes, scales, gs, ws, given);
-                break;
+            case FP4Q_ABSMAX: launch_q16<IN, FP4Q_ABSMAX>(x, rows, cols, ld, imp, codes, scales, gs, ws, st); break;
             case FP4Q_FOUR_OVER_SIX:
-                nvfp4_kernel<IN, FP4Q_FOUR_OVER_SIX><<<g, kThreads, 0, st>>>(x, rows, cols, ld, imp, codes, scales, gs, ws,
-                                                                          given);
+                launch_q16<IN, FP4Q_FOUR_OVER_SIX>(x, rows, cols, ld, imp, codes, scales, gs, ws, st);
                 break;
-            case FP4Q_SWEEP_MSE:
-                launch_sweep<IN, false>(x, rows, cols, ld, imp, codes, scales, gs, ws, st);
-                break;
-            default:
-                launch_sweep<IN, true>(x, rows, cols, ld, imp, codes, scales, gs, ws, st);
-                break;
+            case FP4Q_SWEEP_MSE: launch_q16<IN, FP4Q_SWEEP_MSE>(x, rows, cols, ld, imp, codes, scales, gs, ws, st); break;
+            default: launch_q16<IN, FP4Q_SWEEP_WMSE>(x, rows, cols, ld, imp, codes, scales, gs, ws, st); break;
         }
     }
     return launched(n + 1);

@@ -11,6 +11,10 @@ namespace fp4q {
 typedef unsigned long long u64;
 
 // ---- packed pairs of floats (sm_100 f32x2 instructions) ---------------------------------
+// Caution (measured on B200 with CUDA 12.9): a mul.rn.f32x2 whose result feeds an
+// add/sub.rn.f32x2 can be contracted by the assembler into one fused multiply-add, dropping
+// the rounding of the product despite the .rn qualifiers.  Where the contract rounds a
+// product before adding it, use the scalar __fmul_rn/__fadd_rn/__fsub_rn intrinsics.
 __device__ __forceinline__ u64 pk(float a, float b) {
     u64 r;
     asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
@@ -95,6 +99,24 @@ __device__ __forceinline__ u64 e2m1x2_residual2(u64 y) {
         "  sub.rn.f32.f16 r1, q, b;\n"
         "  mov.b64 %0, {r0, r1}; }"
         : "=l"(r) : "l"(y));
+    return r;
+}
+
+// Codes and residuals of a pair from one conversion: `code` receives the packed E2M1 byte
+// (low nibble = y0), the return value the pair r = RN(q - y).
+__device__ __forceinline__ u64 e2m1x2_code_residual2(u64 y, uint32_t& code) {
+    u64 r;
+    asm("{ .reg .b8 t; .reg .b16 c16; .reg .b32 h; .reg .f16 p, q; .reg .f32 a, b, r0, r1;\n"
+        "  mov.b64 {a, b}, %2;\n"
+        "  cvt.rn.satfinite.e2m1x2.f32 t, b, a;\n"
+        "  mov.b16 c16, {t, 0};\n"
+        "  cvt.u32.u16 %1, c16;\n"
+        "  cvt.rn.f16x2.e2m1x2 h, t;\n"
+        "  mov.b32 {p, q}, h;\n"
+        "  sub.rn.f32.f16 r0, p, a;\n"
+        "  sub.rn.f32.f16 r1, q, b;\n"
+        "  mov.b64 %0, {r0, r1}; }"
+        : "=l"(r), "=r"(code) : "l"(y));
     return r;
 }
 

@@ -181,6 +181,16 @@ def _edge_tensors():
     u[1] = np.arange(32, dtype=np.float32) * 0.25 - 4   # exact E2M1 midpoints at S = 1 scale steps
     u[0, 0] = 1536.0
     out["ties"] = u
+    # exact FP4/INT4 ties: one saturating outlier per block, every other |y| <= 0.25
+    v = (rng.laplace(size=(8, 256)) * 0.02).astype(np.float32)
+    v[:, ::16] = np.float32(102.5) * np.sign(rng.normal(size=(8, 16))).astype(np.float32)
+    out["outlier_ties"] = v
+    # exact sweep ties: [6*e, 0 ...] is reproduced exactly by two candidate scales
+    t2 = np.zeros((4, 128), np.float32)
+    t2[0, 0] = 1536.0                                   # S = 1
+    for k, e in enumerate([1.0, 0.5, 2.0, 0.75, 1.25, 3.0, 0.375]):
+        t2[1 + k % 3, 16 * (k + 1)] = np.float32(6 * e)
+    out["sweep_ties"] = t2
     return out
 
 
