@@ -32,6 +32,22 @@
 
 namespace fp4q {
 
+// Build-time tuning of the 16-element kernels (defaults are the measured best).
+#ifndef FP4Q_SWEEP_SCALAR_ACC
+#define FP4Q_SWEEP_SCALAR_ACC 0   // 1: square-accumulate with scalar FMAs instead of packed pairs
+#endif
+#ifndef FP4Q_SWEEP_UNROLL
+#define FP4Q_SWEEP_UNROLL 11    // MSE candidate-loop unroll factor (11 = the whole window)
+#endif
+#ifndef FP4Q_WMSE_UNROLL
+#define FP4Q_WMSE_UNROLL 1      // WMSE candidate-loop unroll factor
+#endif
+constexpr int kMseUnroll = FP4Q_SWEEP_UNROLL, kWmseUnroll = FP4Q_WMSE_UNROLL;
+
+#ifndef FP4Q_SWEEP_MIN_CTAS
+#define FP4Q_SWEEP_MIN_CTAS 6   // CTAs per SM the MSE/AbsMax/4-6 kernels are compiled for (register cap)
+#endif
+
 enum : int { WS_STATUS = 0, WS_PENDING = 1, WS_AMAX = 2, WS_CNT_AMAX = 3, WS_CNT_Q = 4 };
 constexpr size_t kWorkspaceBytes = 64;
 constexpr int kThreads = 256;
@@ -105,7 +121,11 @@ __global__ void __launch_bounds__(kThreads, 4) amax_kernel(const void* __restric
         for (; i + (U - 1) * step < total; i += U * step) {
             uint4 v[U];
 #pragma unroll
-            for (int u = 0; u < U; ++u) v[u] = __ldg(base + i + u * step);
+            for (int u = 0; u < U; ++u) {   // read-only, no L1 allocation, 256-byte L2 fetches
+                const uint4* src = base + i + u * step;
+                asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(v[u].x), "=r"(v[u].y), "=r"(v[u].z), "=r"(v[u].w) : "l"(src));
+            }
 #pragma unroll
             for (int u = 0; u < U; ++u) fold(v[u]);
         }
@@ -217,6 +237,24 @@ template <bool WEIGHTED>
 __device__ __forceinline__ float sweep_error(const u64 (&xp)[8], const u64 (&wp)[8], float inv, float s2) {
     const u64 inv2 = pk(inv, inv);
     u64 acc = pk(0.0f, 0.0f);   // (even, odd) accumulators
+#if FP4Q_SWEEP_SCALAR_ACC
+    float ae = 0.0f, ao = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        float r0, r1;
+        e2m1x2_residual(mul2(xp[j], inv2), r0, r1);
+        if (WEIGHTED) {
+            float w0, w1;
+            upk(wp[j], w0, w1);
+            ae = __fmaf_rn(__fmul_rn(w0, r0), r0, ae);
+            ao = __fmaf_rn(__fmul_rn(w1, r1), r1, ao);
+        } else {
+            ae = __fmaf_rn(r0, r0, ae);
+            ao = __fmaf_rn(r1, r1, ao);
+        }
+    }
+    return __fmul_rn(s2, __fadd_rn(ae, ao));
+#else
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         const u64 r = e2m1x2_residual2(mul2(xp[j], inv2));
@@ -225,6 +263,7 @@ __device__ __forceinline__ float sweep_error(const u64 (&xp)[8], const u64 (&wp)
     float a, b;
     upk(acc, a, b);
     return __fmul_rn(s2, __fadd_rn(a, b));
+#endif
 }
 
 // Error of the zero scale (pattern 0): every code is 0, so the error is the fma sum of x^2
@@ -249,7 +288,7 @@ __device__ __forceinline__ float zero_scale_error(const u64 (&xp)[8], const u64 
 // Data Types (gist.science/ko/paper/2603.28765), Problem.
 // ------------------------------------------------------------------------------------------
 template <int IN, int OBJ, typename IDX>
-__global__ void __launch_bounds__(kThreads, OBJ == FP4Q_SWEEP_WMSE ? 4 : 6)
+__global__ void __launch_bounds__(kThreads, OBJ == FP4Q_SWEEP_WMSE ? 4 : FP4Q_SWEEP_MIN_CTAS)
     quant16_kernel(const void* __restrict__ xv, IDX rows, IDX cols, IDX ld, const float* __restrict__ imp,
                    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, const float* __restrict__ gscale,
                    uint32_t* __restrict__ ws) {
@@ -301,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, OBJ == FP4Q_SWEEP_WMSE ? 4 : 6)
             bp = max(p0 + LO, 0);                                   // first candidate if every error overflows
             if (p0 + LO <= 0) best = zero_scale_error<WEIGHTED>(xp, wp);   // pattern 0 is the lowest offset
             const int k0 = max(LO, 1 - p0), k1 = min(HI, 126 - p0);
-#pragma unroll 1
+#pragma unroll(WEIGHTED ? kWmseUnroll : kMseUnroll)
             for (int k = k0; k <= k1; ++k) {
                 const int p = p0 + k;
                 const float e = sweep_error<WEIGHTED>(xp, wp, s_inv[p], s_s2[p]);
