@@ -44,6 +44,9 @@ namespace fp4q {
 #endif
 constexpr int kMseUnroll = FP4Q_SWEEP_UNROLL, kWmseUnroll = FP4Q_WMSE_UNROLL;
 
+#ifndef FP4Q_IF4_MIN_CTAS
+#define FP4Q_IF4_MIN_CTAS 6     // CTAs per SM the IF4 kernel is compiled for (register cap)
+#endif
 #ifndef FP4Q_SWEEP_MIN_CTAS
 #define FP4Q_SWEEP_MIN_CTAS 6   // CTAs per SM the MSE/AbsMax/4-6 kernels are compiled for (register cap)
 #endif
@@ -51,6 +54,7 @@ constexpr int kMseUnroll = FP4Q_SWEEP_UNROLL, kWmseUnroll = FP4Q_WMSE_UNROLL;
 enum : int { WS_STATUS = 0, WS_PENDING = 1, WS_AMAX = 2, WS_CNT_AMAX = 3, WS_CNT_Q = 4 };
 constexpr size_t kWorkspaceBytes = 64;
 constexpr int kThreads = 256;
+constexpr float kRintMagic = 12582912.0f;   // 1.5 * 2^23
 
 __device__ __forceinline__ bool scale_range_ok(float S) {
     if (S == 0.0f) return true;
@@ -363,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, OBJ == FP4Q_SWEEP_WMSE ? 4 : FP4Q_SW
 // n = clamp(rint(z), -7, 7), r = RN(RN(n RN(6/7)) - y).
 // ------------------------------------------------------------------------------------------
 template <int IN, typename IDX>
-__global__ void __launch_bounds__(kThreads, 4)
+__global__ void __launch_bounds__(kThreads, FP4Q_IF4_MIN_CTAS)
     if4_kernel(const void* __restrict__ xv, IDX rows, IDX cols, IDX ld, uint8_t* __restrict__ codes,
                uint8_t* __restrict__ scales, const float* __restrict__ gscale, uint32_t* __restrict__ ws) {
     __shared__ float s_sv[128], s_inv[128], s_s2[128];
@@ -373,7 +377,6 @@ __global__ void __launch_bounds__(kThreads, 4)
     const float S = su.S;
     const float d6 = __fmul_rn(6.0f, S);
     const float K76 = __fdiv_rn(7.0f, 6.0f), K67 = __fdiv_rn(6.0f, 7.0f);
-    const u64 k76 = pk(K76, K76);
     const IDX nb = cols / 16;
     const IDX total = rows * nb;
     const IDX blk = (IDX)blockIdx.x * blockDim.x + threadIdx.x;
@@ -397,19 +400,18 @@ __global__ void __launch_bounds__(kThreads, 4)
         const u64 y = mul2(xp[j], inv2);
         const u64 rf = e2m1x2_code_residual2(y, cf[j]);
         accf = fma2(rf, rf, accf);
-        float z0, z1, n0, n1;
-        upk(mul2(y, k76), z0, z1);
-        asm("cvt.rni.f32.f32 %0, %1;" : "=f"(n0) : "f"(z0));
-        asm("cvt.rni.f32.f32 %0, %1;" : "=f"(n1) : "f"(z1));
-        n0 = fminf(fmaxf(n0, -7.0f), 7.0f);
-        n1 = fminf(fmaxf(n1, -7.0f), 7.0f);
-        // scalar .rn intrinsics: a packed multiply feeding a packed subtract can be contracted
-        // into one fused operation by the assembler, which would skip the rounding of v
+        // INT4 path on scalar .rn intrinsics (no contraction): z = RN(y RN(7/6)); adding
+        // M = 1.5 * 2^23 rounds z to the nearest integer, ties to even (the sum's ulp is 1), so
+        // t = M + rint(z) exactly; clamping t to [M-7, M+7] clamps n; n = t - M is exact and the
+        // low four bits of t's encoding are n's two's-complement nibble.
         float y0, y1;
         upk(y, y0, y1);
+        const float t0 = fminf(fmaxf(__fadd_rn(__fmul_rn(y0, K76), kRintMagic), kRintMagic - 7.0f), kRintMagic + 7.0f);
+        const float t1 = fminf(fmaxf(__fadd_rn(__fmul_rn(y1, K76), kRintMagic), kRintMagic - 7.0f), kRintMagic + 7.0f);
+        const float n0 = __fsub_rn(t0, kRintMagic), n1 = __fsub_rn(t1, kRintMagic);
         const u64 ri = pk(__fsub_rn(__fmul_rn(n0, K67), y0), __fsub_rn(__fmul_rn(n1, K67), y1));
         acci = fma2(ri, ri, acci);
-        ci[j] = ((uint32_t)__float2int_rn(n0) & 0xFu) | (((uint32_t)__float2int_rn(n1) & 0xFu) << 4);
+        ci[j] = (__float_as_uint(t0) & 0xFu) | ((__float_as_uint(t1) & 0xFu) << 4);
     }
     float a, c;
     upk(accf, a, c);
@@ -427,20 +429,35 @@ __global__ void __launch_bounds__(kThreads, 4)
 // MXFP4 (+ 32-point Hadamard)
 // ------------------------------------------------------------------------------------------
 __device__ __forceinline__ void fwht32(float (&v)[32]) {
+    // h = 1 pairs neighbours within a register pair: scalar adds
 #pragma unroll
-    for (int h = 1; h < 32; h <<= 1) {
+    for (int j = 0; j < 32; j += 2) {
+        const float a = v[j], b = v[j + 1];
+        v[j] = __fadd_rn(a, b);
+        v[j + 1] = __fsub_rn(a, b);
+    }
+    // h = 2, 4, 8, 16: (v_j, v_j+1) and (v_j+h, v_j+h+1) butterfly as packed pairs
+    u64 w[16];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
+    for (int j = 0; j < 16; ++j) w[j] = pk(v[2 * j], v[2 * j + 1]);
+#pragma unroll
+    for (int h = 1; h < 16; h <<= 1) {   // h counts pairs: element stride 2h
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
             if ((j & h) == 0) {
-                const float a = v[j], b = v[j + h];
-                v[j] = __fadd_rn(a, b);
-                v[j + h] = __fsub_rn(a, b);
+                const u64 a = w[j], b = w[j + h];
+                w[j] = add2(a, b);
+                w[j + h] = sub2(a, b);
             }
         }
     }
     const float KH = (float)0.17677669529663688110021109052621;   // RN(1/sqrt(32))
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = __fmul_rn(v[j], KH);
+    for (int j = 0; j < 16; ++j) {
+        upk(w[j], v[2 * j], v[2 * j + 1]);
+        v[2 * j] = __fmul_rn(v[2 * j], KH);
+        v[2 * j + 1] = __fmul_rn(v[2 * j + 1], KH);
+    }
 }
 
 // Smallest e with a <= 6*2^e (ceil rule) or floor(log2 a) - 2 (OCP rule), clamped to [-127,127].
