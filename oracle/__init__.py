@@ -50,6 +50,10 @@ def lib():
         L.fp4q_o_tensor_scale.argtypes = [P, i64, i64, i64, P]
         L.fp4q_o_mx_exponent.restype = C.c_int
         L.fp4q_o_mx_exponent.argtypes = [C.c_float, C.c_int]
+        L.fp4q_o_hadamard16.restype = None
+        L.fp4q_o_hadamard16.argtypes = [P]
+        L.fp4q_o_rotate16.restype = C.c_int
+        L.fp4q_o_rotate16.argtypes = [P, i64, i64, i64, P]
         L.fp4q_o_hadamard32.restype = None
         L.fp4q_o_hadamard32.argtypes = [P]
         L.fp4q_o_nvfp4_quantize.restype = C.c_int
@@ -115,11 +119,28 @@ def hadamard32(v) -> np.ndarray:
     return v
 
 
-# --- quantizers --------------------------------------------------------------------
-def nvfp4_quantize(x, objective="sweep_mse", importance=None, S=None):
-    """NVFP4 quantization of a float32 [rows, cols] array; returns a dict with packed codes
-    [rows, cols/2], scale bytes [rows, cols/16], S, status and per-block diagnostics."""
+def hadamard16(v) -> np.ndarray:
+    v = np.ascontiguousarray(v, dtype=np.float32).copy()
+    assert v.size == 16
+    lib().fp4q_o_hadamard16(_p(v))
+    return v
+
+
+def rotate16(x) -> np.ndarray:
+    """Every 16-element block of every row rotated by the normalized 16-point Hadamard."""
     x = _f32(x)
+    out = np.empty_like(x)
+    if lib().fp4q_o_rotate16(_p(x), x.shape[0], x.shape[1], x.shape[1], _p(out)) < 0:
+        raise ValueError("oracle: bad shape")
+    return out
+
+
+# --- quantizers --------------------------------------------------------------------
+def nvfp4_quantize(x, objective="sweep_mse", importance=None, S=None, hadamard16=False):
+    """NVFP4 quantization of a float32 [rows, cols] array; returns a dict with packed codes
+    [rows, cols/2], scale bytes [rows, cols/16], S, status and per-block diagnostics.
+    hadamard16: quantize the blockwise-rotated tensor (S taken over the rotated values)."""
+    x = rotate16(x) if hadamard16 else _f32(x)
     rows, cols = x.shape
     nb = cols // 16
     codes = np.zeros((rows, cols // 2), np.uint8)
@@ -138,8 +159,8 @@ def nvfp4_quantize(x, objective="sweep_mse", importance=None, S=None):
             "p": bp, "err": be, "err2": be2, "nvalid": bn}
 
 
-def if4_quantize(x, S=None):
-    x = _f32(x)
+def if4_quantize(x, S=None, hadamard16=False):
+    x = rotate16(x) if hadamard16 else _f32(x)
     rows, cols = x.shape
     nb = cols // 16
     codes = np.zeros((rows, cols // 2), np.uint8)

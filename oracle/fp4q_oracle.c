@@ -368,6 +368,35 @@ void fp4q_o_hadamard32(float* v)
     for (int j = 0; j < 32; ++j) v[j] = v[j] * KH;
 }
 
+/* Normalized 16-point block Hadamard for NVFP4/IF4 (the rotation the MR-GPTQ page applies to
+ * both formats, with the block size of NVFP4): butterflies h = 1, 2, 4, 8 in binary32, then a
+ * multiplication by 1/sqrt(16) = 1/4, an exact power of two. */
+void fp4q_o_hadamard16(float* v)
+{
+    for (int h = 1; h < 16; h <<= 1)
+        for (int j = 0; j < 16; ++j)
+            if ((j & h) == 0) {
+                float a = v[j], b = v[j + h];
+                v[j] = a + b;
+                v[j + h] = a - b;
+            }
+    for (int j = 0; j < 16; ++j) v[j] = v[j] * 0.25f;
+}
+
+/* out[r][c] = the 16-point rotation of each 16-element block of row r of x (row stride ld). */
+int fp4q_o_rotate16(const float* x, int64_t rows, int64_t cols, int64_t ld, float* out)
+{
+    if (cols % 16) return -1;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; c += 16) {
+            float v[16];
+            memcpy(v, x + r * ld + c, sizeof v);
+            fp4q_o_hadamard16(v);
+            memcpy(out + r * cols + c, v, sizeof v);
+        }
+    return 0;
+}
+
 /* Smallest e with a <= 6*2^e (ocp_floor = 0), or floor(log2 a) - 2 (ocp_floor = 1). */
 int fp4q_o_mx_exponent(float a, int ocp_floor)
 {
@@ -431,7 +460,8 @@ static uint16_t f32_to_bf16(float f)
 
 /* fmt: 0 NVFP4, 1 IF4, 2 MXFP4.  out is float32 [rows][cols] (out_bf16 = 0) or uint16
  * bf16 bit patterns (out_bf16 = 1).  inverse_hadamard applies the 32-point transform to
- * every dequantized MXFP4 block (the normalized transform is its own inverse). */
+ * every dequantized MXFP4 block, the 16-point one to NVFP4/IF4 blocks (each normalized
+ * transform is its own inverse). */
 int fp4q_o_dequantize(const uint8_t* codes, const uint8_t* scales, float S,
                       int64_t rows, int64_t cols, int fmt, int inverse_hadamard,
                       void* out, int out_bf16)
@@ -463,6 +493,7 @@ int fp4q_o_dequantize(const uint8_t* codes, const uint8_t* scales, float S,
                 }
             }
             if (fmt == 2 && inverse_hadamard) fp4q_o_hadamard32(v);
+            if (fmt != 2 && inverse_hadamard) fp4q_o_hadamard16(v);
             for (int i = 0; i < B; ++i) {
                 int64_t idx = r * cols + b * B + i;
                 if (out_bf16) ((uint16_t*)out)[idx] = f32_to_bf16(v[i]);

@@ -331,6 +331,69 @@ def test_hadamard_is_normalized_sylvester():
         assert np.allclose(O.hadamard32(v), ref, rtol=1e-5, atol=1e-6)
 
 
+H16 = np.array([[(-1.0) ** bin(i & j).count("1") for j in range(16)] for i in range(16)]) / 4   # closed form
+
+
+def test_hadamard16_is_normalized_sylvester():
+    """The 16-point rotation NVFP4/IF4 blocks take is H_16 / 4 with H_16[i][j] =
+    (-1)^popcount(i & j) (Sylvester order): checked column by column, then as a matrix
+    product on integer blocks (every partial sum exact), as an involution, block by block
+    along a row, and within the summation error bound on random values."""
+    M = np.stack([O.hadamard16(np.eye(16, dtype=np.float32)[k]) for k in range(16)], axis=1).astype(np.float64)
+    assert np.array_equal(M, H16)
+    rng = np.random.default_rng(3)
+    x = rng.integers(-1000, 1000, size=(5, 64)).astype(np.float32)
+    rx = O.rotate16(x)
+    assert np.array_equal(rx.astype(np.float64), (x.astype(np.float64).reshape(5, 4, 16) @ H16.T).reshape(5, 64))
+    assert np.array_equal(O.rotate16(rx), x)
+    v = rng.normal(size=(64, 16)).astype(np.float32) * np.exp(rng.uniform(-20, 20, size=(64, 1))).astype(np.float32)
+    got = O.rotate16(v).astype(np.float64)
+    exact = v.astype(np.float64) @ H16.T
+    # four levels of binary32 additions, then an exact 1/4: |error| <= 4 u sum|v| / 4 (u = 2^-24)
+    bound = 4 * 2.0 ** -24 * np.abs(v.astype(np.float64)).sum(axis=1, keepdims=True) / 4 * 1.0001
+    assert np.all(np.abs(got - exact) <= bound)
+
+
+def _rotated_grid_tensor(seed, rows=6, cols=128):
+    """x = H y blockwise (closed-form matrix, exact: multiples of 1/8 below 2^5) with y on the
+    E2M1 grid and every block's largest magnitude 6."""
+    rng = np.random.default_rng(seed)
+    y = rng.choice([0, .5, 1, 1.5, 2, 3, 4, 6], size=(rows, cols)) * rng.choice([-1.0, 1.0], size=(rows, cols))
+    y[:, rng.integers(0, 16)::16] = 6.0 * rng.choice([-1.0, 1.0], size=(rows, cols // 16))
+    x = (y.reshape(rows, -1, 16) @ H16.T).reshape(rows, cols)
+    return x.astype(np.float32), y.astype(np.float32)
+
+
+@pytest.mark.parametrize("method", ["absmax", "four_over_six", "sweep_mse", "if4"])
+def test_hadamard16_quantize_is_exact_on_rotated_grid_values(method):
+    """If H x lies on the FP4 grid at scale 1 with block maxima 6, the rotated method must
+    take S = 6/1536 = 2^-8 from max|H x| (max|x| is larger), pick pattern 0x78 (e = 256,
+    sv = 1) in every block with zero error, reproduce H x exactly without the inverse
+    rotation and x exactly with it."""
+    x, y = _rotated_grid_tensor(5)
+    assert np.abs(x).max() > 6.0
+    fmt = "if4" if method == "if4" else "nvfp4"
+    r = O.if4_quantize(x, hadamard16=True) if fmt == "if4" else O.nvfp4_quantize(x, method, hadamard16=True)
+    assert r["S"] == 2.0 ** -8
+    assert np.all(r["scales"] == 0x78)
+    assert np.array_equal(O.dequantize(r["codes"], r["scales"], r["S"], fmt), y)
+    assert np.array_equal(O.dequantize(r["codes"], r["scales"], r["S"], fmt, inverse_hadamard=True), x)
+    # and the plain path on the same tensor sees max|x|, not max|H x|
+    plain = O.if4_quantize(x) if fmt == "if4" else O.nvfp4_quantize(x, method)
+    assert plain["S"] == np.float32(np.float32(np.abs(x).max()) / np.float32(1536))
+
+
+def test_hadamard16_spreads_an_outlier():
+    """One outlier c in a block becomes c/4 at all 16 positions: S = RN(RN(c/4) / 1536)."""
+    x = np.zeros((2, 32), np.float32)
+    x[1, 21] = -3000.0
+    x[0, 2] = 7.0
+    r = O.nvfp4_quantize(x, "sweep_mse", hadamard16=True)
+    assert r["S"] == np.float32(np.float32(750.0) / np.float32(1536.0))
+    xr = O.rotate16(x)
+    assert np.all(np.abs(xr[1, 16:]) == 750.0) and np.all(xr[1, :16] == 0)
+
+
 def test_exact_roundtrip_every_e2m1_x_e4m3_value():
     """With S = 1, every value q*e(p) is reproduced bit-exactly.  AbsMax reaches patterns
     1..0x78 (a_b/(6S) <= 256 by construction): a block whose max is 6*e(p) selects p and
