@@ -36,6 +36,10 @@ WORKLOADS = {
     "cfg4": ("cfg4", "if4", None, "IF4 per-block FP4/INT4 selection, bf16 weight 4096x14336, 0.02*t4"),
     "cfg5": ("cfg5", "mxfp4", None, "MXFP4, bf16 activations 16384x8192"),
     "cfg5h": ("cfg5", "mxfp4_had", None, "MXFP4 after 32x32 block Hadamard, bf16 activations 16384x8192"),
+    "cfg3h": ("cfg3", "nvfp4_had", "sweep_mse",
+              "NVFP4 ScaleSweep-MSE on 16x16 block-Hadamard-rotated blocks, bf16 activations 8192x4096, "
+              "dynamic S of the rotated tensor"),
+    "cfg4h": ("cfg4", "if4_had", None, "IF4 on 16x16 block-Hadamard-rotated blocks, bf16 weight 4096x14336"),
 }
 METRIC = "quantize GB/s (input bf16) and % of B200 HBM peak, 1 GPU, vs CPU oracle"
 # Arithmetic the method itself needs per element for the ALU-bound searches: per candidate
@@ -43,6 +47,15 @@ METRIC = "quantize GB/s (input bf16) and % of B200 HBM peak, 1 GPU, vs CPU oracl
 # multiply-add (square-accumulate) -- plus, for WMSE, the weight multiply -- over 11 (MSE) or
 # 16 (WMSE) candidates, plus the block maximum and the final multiply + rounding.
 ALU_OPS_PER_ELEMENT = {"sweep_mse": 11 * 4 + 3, "sweep_wmse": 16 * 5 + 3}
+# the 16-point rotation adds four butterfly additions and one multiplication per element
+ROTATION_OPS_PER_ELEMENT = 4 + 1
+
+
+def split_fmt(fmt):
+    """'nvfp4_had' -> ('nvfp4', True); MXFP4's rotated form keeps its own name."""
+    if fmt.endswith("_had") and not fmt.startswith("mxfp4"):
+        return fmt[:-4], True
+    return fmt, False
 L2_BYTES = 126 * 2 ** 20
 
 
@@ -155,12 +168,13 @@ def cpu_baseline(w, fmt, obj, budget_s=12.0):
     chunk = max(1, min(rows, 256))
     done, t0 = 0, time.perf_counter()
     imp = w.get("importance")
+    base, had16 = split_fmt(fmt)
     while done < rows and time.perf_counter() - t0 < budget_s:
         xs = x[done:done + chunk]
-        if fmt == "nvfp4":
-            O.nvfp4_quantize(xs, obj, importance=imp)
-        elif fmt == "if4":
-            O.if4_quantize(xs)
+        if base == "nvfp4":
+            O.nvfp4_quantize(xs, obj, importance=imp, hadamard16=had16)
+        elif base == "if4":
+            O.if4_quantize(xs, hadamard16=had16)
         else:
             O.mxfp4_quantize(xs, hadamard=fmt.endswith("had"))
         done += xs.shape[0]
@@ -183,14 +197,15 @@ def run_reference(args, rank, world):
     rows, cols = x.shape
     sample_rows = 16
     imp = w.get("importance")
+    base, had16 = split_fmt(fmt)
 
     def step(i):
         r0 = (i * sample_rows) % rows
         xs = x[r0:r0 + sample_rows]
-        if fmt == "nvfp4":
-            O.nvfp4_quantize(xs, obj, importance=imp)
-        elif fmt == "if4":
-            O.if4_quantize(xs)
+        if base == "nvfp4":
+            O.nvfp4_quantize(xs, obj, importance=imp, hadamard16=had16)
+        elif base == "if4":
+            O.if4_quantize(xs, hadamard16=had16)
         else:
             O.mxfp4_quantize(xs, hadamard=fmt.endswith("had"))
 
@@ -234,7 +249,8 @@ def run_ours(args, rank, world):
     out_bytes = rows * cols // 2 + rows * cols // (32 if fmt.startswith("mxfp4") else 16)
     nsets = max(2, int(np.ceil(2.5 * L2_BYTES / (in_bytes + out_bytes))))
     xs = [x_host.to(dev) for _ in range(nsets)]
-    outs = [fq.alloc_outputs(rows, cols, "mxfp4" if fmt.startswith("mxfp4") else fmt, dev) for _ in range(nsets)]
+    base, had16 = split_fmt(fmt)
+    outs = [fq.alloc_outputs(rows, cols, "mxfp4" if fmt.startswith("mxfp4") else base, dev) for _ in range(nsets)]
     imp = torch.from_numpy(w["importance"]).to(dev) if obj == "sweep_wmse" else None
     ws = fq.new_workspace(dev)
     launches_per_step = 0
@@ -253,10 +269,11 @@ def run_ours(args, rank, world):
             if ev is not None:
                 ev[2].record()
             return 1
-        fq.global_scale(xs[s], out=g, workspace=ws)
+        fq.global_scale(xs[s], out=g, workspace=ws, hadamard16=had16)
         if ev is not None:
             ev[1].record()
-        fq.quantize(xs[s], fmt, obj or "absmax", importance=imp, global_scale=g, out=(c, sc, g), workspace=ws)
+        fq.quantize(xs[s], base, obj or "absmax", importance=imp, global_scale=g, out=(c, sc, g), workspace=ws,
+                    hadamard16=had16)
         if ev is not None:
             ev[2].record()
         return 2
@@ -321,7 +338,7 @@ def run_ours(args, rank, world):
     e2e_steps = max(1, min(args.steps, 20))
     x_pin = x_host.pin_memory()
     dev_bufs = {"x": xs[0], "out": outs[0]}
-    host_out = fq.alloc_host_outputs(rows, cols, "mxfp4" if fmt.startswith("mxfp4") else fmt)
+    host_out = fq.alloc_host_outputs(rows, cols, fmt)
     with torch.cuda.stream(stream):
         for _ in range(2):
             fq.quantize_host(x_pin, fmt, obj or "absmax", importance=imp, workspace=ws, dev_bufs=dev_bufs,
@@ -356,6 +373,8 @@ def run_ours(args, rank, world):
                 "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": "quantize (" + (obj or fmt) + ")",
                 "peak_source": f"{peak_src} hbm_gbs (copy, burst) from MEASURED_PEAKS.json"}
     ops = ALU_OPS_PER_ELEMENT.get(obj or fmt)
+    if ops is not None and had16:
+        ops += ROTATION_OPS_PER_ELEMENT
     if ops is not None:
         # the candidate search is bound by plain FP32/convert arithmetic, not by HBM: the peak is
         # 148 SMs x 128 FP32 lanes x the SM clock sampled during the timed region

@@ -21,12 +21,12 @@ DEVSTAT_OK, DEVSTAT_NONFINITE, DEVSTAT_RANGE = 0, 1, 2
 IN_F32, IN_BF16 = 0, 1
 FORMATS = {"nvfp4": 0, "if4": 1, "mxfp4": 2}
 OBJECTIVES = {"absmax": 0, "four_over_six": 1, "sweep_mse": 2, "sweep_wmse": 3}
-F_GLOBAL_SCALE_GIVEN, F_MX_OCP_FLOOR, F_OUT_BF16 = 0x1, 0x2, 0x4
+F_GLOBAL_SCALE_GIVEN, F_MX_OCP_FLOOR, F_OUT_BF16, F_HADAMARD16 = 0x1, 0x2, 0x4, 0x8
 BLOCK = {"nvfp4": 16, "if4": 16, "mxfp4": 32}
 
 # Names of every function include/fp4q.h declares (checked against the header by the tests).
-EXPORTS = ("fp4q_workspace_bytes", "fp4q_global_scale", "fp4q_quantize", "fp4q_hadamard_quantize", "fp4q_dequantize",
-           "fp4q_quantize_noalloc", "fp4q_read_device_status", "fp4q_last_launch_count", "fp4q_status_string")
+EXPORTS = ("fp4q_workspace_bytes", "fp4q_global_scale", "fp4q_hadamard_global_scale", "fp4q_quantize",
+           "fp4q_hadamard_quantize", "fp4q_dequantize", "fp4q_quantize_noalloc", "fp4q_read_device_status", "fp4q_last_launch_count", "fp4q_status_string")
 
 _lib = None
 
@@ -49,6 +49,8 @@ def lib():
         L.fp4q_quantize.argtypes = [P, i32, i64, i64, i64, i32, i32, P, P, P, P, P, u32, P]
         L.fp4q_global_scale.restype = i32
         L.fp4q_global_scale.argtypes = [P, i32, i64, i64, i64, P, P, P]
+        L.fp4q_hadamard_global_scale.restype = i32
+        L.fp4q_hadamard_global_scale.argtypes = [P, i32, i64, i64, i64, i32, P, P, P]
         L.fp4q_hadamard_quantize.restype = i32
         L.fp4q_hadamard_quantize.argtypes = [P, i32, i64, i64, i64, i32, P, P, P, u32, P]
         L.fp4q_dequantize.restype = i32
@@ -117,24 +119,27 @@ def alloc_outputs(rows: int, cols: int, fmt: str, device="cuda"):
     return codes, scales, gs
 
 
+def _flags(global_scale, mx_ocp_floor, hadamard16):
+    return ((F_GLOBAL_SCALE_GIVEN if global_scale is not None else 0) | (F_MX_OCP_FLOOR if mx_ocp_floor else 0)
+            | (F_HADAMARD16 if hadamard16 else 0))
+
+
 def quantize(x, fmt: str = "nvfp4", objective: str = "sweep_mse", importance=None, global_scale=None,
-             mx_ocp_floor: bool = False, out=None, workspace=None, stream=None):
+             mx_ocp_floor: bool = False, out=None, workspace=None, stream=None, hadamard16: bool = False):
     """Quantize a 2-D bf16/fp32 CUDA tensor (row stride may exceed the width).
 
     Returns (codes [rows, cols/2] uint8, scales [rows, cols/B] uint8, S [1] float32 or None).
     global_scale: a [1] float32 CUDA tensor to use as S (skips the amax pass).
     out: optional preallocated (codes, scales, S) tuple.
+    hadamard16: NVFP4/IF4 on blocks rotated by the normalized 16-point Hadamard.
     """
     if x.dim() != 2 or x.stride(1) != 1:
         raise Fp4qError("x must be 2-D with unit column stride")
     rows, cols = x.shape
     codes, scales, gs = out if out is not None else alloc_outputs(rows, cols, fmt, x.device)
-    flags = 0
+    flags = _flags(global_scale, mx_ocp_floor, hadamard16)
     if global_scale is not None:
-        flags |= F_GLOBAL_SCALE_GIVEN
         gs = global_scale
-    if mx_ocp_floor:
-        flags |= F_MX_OCP_FLOOR
     ws = workspace if workspace is not None else new_workspace(x.device)
     rc = lib().fp4q_quantize(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), FORMATS[fmt],
                              OBJECTIVES.get(objective, 0), _ptr(importance), _ptr(codes), _ptr(scales),
@@ -143,14 +148,19 @@ def quantize(x, fmt: str = "nvfp4", objective: str = "sweep_mse", importance=Non
     return codes, scales, (gs if fmt != "mxfp4" else None)
 
 
-def global_scale(x, out=None, workspace=None, stream=None):
-    """Tensor scale S = RN(max|x| / 1536) as a [1] float32 CUDA tensor (amax pass only)."""
+def global_scale(x, out=None, workspace=None, stream=None, hadamard16: bool = False):
+    """Tensor scale S = RN(max|x| / 1536) as a [1] float32 CUDA tensor (amax pass only);
+    hadamard16: of the 16-point block-rotated tensor."""
     torch = _torch()
     rows, cols = x.shape
     gs = out if out is not None else torch.empty((1,), dtype=torch.float32, device=x.device)
     ws = workspace if workspace is not None else new_workspace(x.device)
-    rc = lib().fp4q_global_scale(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), _ptr(gs), _ptr(ws),
-                                 _stream_ptr(stream))
+    if hadamard16:
+        rc = lib().fp4q_hadamard_global_scale(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), 16, _ptr(gs),
+                                              _ptr(ws), _stream_ptr(stream))
+    else:
+        rc = lib().fp4q_global_scale(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), _ptr(gs), _ptr(ws),
+                                     _stream_ptr(stream))
     _check(rc, "fp4q_global_scale")
     return gs
 
@@ -184,7 +194,8 @@ def dequantize(codes, scales, global_scale, fmt: str = "nvfp4", inverse_hadamard
 
 
 def quantize_noalloc(x, fmt: str = "nvfp4", objective: str = "sweep_mse", importance=None, global_scale=None,
-                     mx_ocp_floor: bool = False, out=None, device_status=None, stream=None):
+                     mx_ocp_floor: bool = False, out=None, device_status=None, stream=None,
+                     hadamard16: bool = False):
     """quantize() for callers that cannot allocate device memory: the library's own
     per-GPU scratch replaces the workspace (see fp4q_quantize_noalloc in include/fp4q.h).
     Outputs must be passed in `out`; device_status is an optional [1] int32 CUDA tensor."""
@@ -192,12 +203,9 @@ def quantize_noalloc(x, fmt: str = "nvfp4", objective: str = "sweep_mse", import
         raise Fp4qError("x must be 2-D with unit column stride")
     rows, cols = x.shape
     codes, scales, gs = out
-    flags = 0
+    flags = _flags(global_scale, mx_ocp_floor, hadamard16)
     if global_scale is not None:
-        flags |= F_GLOBAL_SCALE_GIVEN
         gs = global_scale
-    if mx_ocp_floor:
-        flags |= F_MX_OCP_FLOOR
     rc = lib().fp4q_quantize_noalloc(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), FORMATS[fmt],
                                      OBJECTIVES.get(objective, 0), _ptr(importance), _ptr(codes), _ptr(scales),
                                      _ptr(gs) if fmt != "mxfp4" else None, _ptr(device_status), flags,
@@ -219,7 +227,7 @@ def last_launch_count() -> int:
 def alloc_host_outputs(rows: int, cols: int, fmt: str):
     """Pinned host buffers for (codes, scales, S)."""
     torch = _torch()
-    fmt = "mxfp4" if fmt.startswith("mxfp4") else fmt
+    fmt = fmt[:-4] if fmt.endswith("_had") else fmt
     return (torch.empty((rows, cols // 2), dtype=torch.uint8, pin_memory=True),
             torch.empty((rows, cols // BLOCK[fmt]), dtype=torch.uint8, pin_memory=True),
             torch.empty((1,), dtype=torch.float32, pin_memory=True))
@@ -229,10 +237,11 @@ def quantize_host(x_host, fmt="nvfp4", objective="sweep_mse", importance=None, s
                   dev_bufs=None, host_out=None):
     """End-to-end call on host (pinned) memory: copy the input in, quantize on the device,
     copy codes, scales and S back (asynchronously on the current stream).
-    fmt "mxfp4_had" selects the Hadamard-rotated MXFP4 path.  Returns host (codes, scales, S)."""
+    fmt "mxfp4_had" selects the Hadamard-rotated MXFP4 path, "nvfp4_had" / "if4_had" the
+    16-point rotated NVFP4 / IF4 paths.  Returns host (codes, scales, S)."""
     torch = _torch()
     rows, cols = x_host.shape
-    base = "mxfp4" if fmt.startswith("mxfp4") else fmt
+    base = fmt[:-4] if fmt.endswith("_had") else fmt
     if dev_bufs is None:
         dev_bufs = {"x": torch.empty(x_host.shape, dtype=x_host.dtype, device="cuda"),
                     "out": alloc_outputs(rows, cols, base, "cuda")}
@@ -245,7 +254,7 @@ def quantize_host(x_host, fmt="nvfp4", objective="sweep_mse", importance=None, s
         gs = None
     else:
         codes, scales, gs = quantize(xd, base, objective, importance=importance, out=dev_bufs["out"],
-                                     workspace=workspace, stream=stream)
+                                     workspace=workspace, stream=stream, hadamard16=fmt.endswith("_had"))
     hc, hs, hg = host_out
     hc.copy_(codes, non_blocking=True)
     hs.copy_(scales, non_blocking=True)

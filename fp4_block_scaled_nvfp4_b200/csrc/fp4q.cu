@@ -17,7 +17,11 @@
 //                        32-point fast Walsh-Hadamard rotation.  Bridging the Gap ...
 //                        Microscaling FP4 (gist.science/ko/paper/2509.23202),
 //                        "Methodology"; TORQ (gist.science/ko/paper/2605.19561) S-step.
-//   dequant kernels      codes + scales (+S) -> fp32 / bf16.
+//   HAD16 variants       amax, NVFP4 and IF4 kernels on blocks rotated by the normalized
+//                        16-point Hadamard H_16/4 (in registers, before the scale is chosen);
+//                        Bridging the Gap ..., "Methodology", block-wise Hadamard transforms,
+//                        which rotates for both NVFP4 and MXFP4.
+//   dequant kernels      codes + scales (+S) -> fp32 / bf16 (+ the inverse rotation).
 // Status protocol (workspace words): each quantize kernel ORs its data flags into
 // PENDING, counts its CTAs in an arrival counter, and the last CTA publishes
 // STATUS = PENDING and zeroes PENDING and the counter, so the workspace is clean again
@@ -91,6 +95,31 @@ __device__ __forceinline__ void finish_status(uint32_t* ws, uint32_t flag, int c
 // ------------------------------------------------------------------------------------------
 // amax
 // ------------------------------------------------------------------------------------------
+// Combine the per-thread maxima m (magnitude bit patterns) of the CTA, fold them into the
+// workspace word, and let the last CTA write S = RN(RN(amax * post) / 1536) (NaN when any
+// element was NaN or infinite) and, when publish is set, the status word.
+__device__ __forceinline__ void amax_finish(uint32_t m, float post, uint32_t* ws, float* gscale, int publish) {
+    m = __reduce_max_sync(0xFFFFFFFFu, m);
+    __shared__ uint32_t red[kThreads / 32];
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < kThreads / 32; ++w) m = max(m, red[w]);
+        atomicMax(&ws[WS_AMAX], m);
+        __threadfence();
+        const unsigned prev = atomicAdd(&ws[WS_CNT_AMAX], 1u);
+        if (prev == gridDim.x - 1) {
+            __threadfence();
+            const uint32_t bits = atomicExch(&ws[WS_AMAX], 0u);
+            atomicExch(&ws[WS_CNT_AMAX], 0u);
+            const float S = bits >= 0x7F800000u ? __uint_as_float(0x7FC00000u)
+                                                : __fdiv_rn(__fmul_rn(__uint_as_float(bits), post), 1536.0f);
+            *gscale = S;
+            if (publish) atomicExch(&ws[WS_STATUS], scale_flags(S));
+        }
+    }
+}
+
 template <int IN>
 __global__ void __launch_bounds__(kThreads, 4) amax_kernel(const void* __restrict__ xv, int64_t rows, int64_t cols,
                                                         int64_t ld, uint32_t* __restrict__ ws,
@@ -142,25 +171,7 @@ __global__ void __launch_bounds__(kThreads, 4) amax_kernel(const void* __restric
     }
     for (; i < total; i += step) fold(__ldg(at(i)));
     if (IN == FP4Q_IN_BF16) m = max(m & 0xFFFFu, m >> 16) << 16;   // bf16 bits -> f32 bits
-    m = __reduce_max_sync(0xFFFFFFFFu, m);
-    __shared__ uint32_t red[kThreads / 32];
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        for (int w = 1; w < kThreads / 32; ++w) m = max(m, red[w]);
-        atomicMax(&ws[WS_AMAX], m);
-        __threadfence();
-        const unsigned prev = atomicAdd(&ws[WS_CNT_AMAX], 1u);
-        if (prev == gridDim.x - 1) {
-            __threadfence();
-            const uint32_t bits = atomicExch(&ws[WS_AMAX], 0u);
-            atomicExch(&ws[WS_CNT_AMAX], 0u);
-            const float S = bits >= 0x7F800000u ? __uint_as_float(0x7FC00000u)
-                                                : __fdiv_rn(__uint_as_float(bits), 1536.0f);
-            *gscale = S;
-            if (publish) atomicExch(&ws[WS_STATUS], scale_flags(S));
-        }
-    }
+    amax_finish(m, 1.0f, ws, gscale, publish);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -222,6 +233,105 @@ __device__ __forceinline__ float block_absmax(const u64 (&xp)[8]) {
         m = fmaxf(m, fmaxf(fabsf(a), fabsf(b)));
     }
     return m;
+}
+
+// Fast Walsh-Hadamard butterflies h = 1, 2, 4, 8 over one 16-element block held as 8
+// (even, odd) pairs, without the normalization: h = 1 combines the two halves of a pair
+// (scalar), h = 2, 4, 8 combine whole pairs k and k + h/2 (packed).
+__device__ __forceinline__ void fwht16_butterflies(u64 (&xp)[8]) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        float a, b;
+        upk(xp[j], a, b);
+        xp[j] = pk(__fadd_rn(a, b), __fsub_rn(a, b));
+    }
+#pragma unroll
+    for (int h = 1; h < 8; h <<= 1) {   // h counts pairs: element stride 2h
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            if ((j & h) == 0) {
+                const u64 a = xp[j], b = xp[j + h];
+                xp[j] = add2(a, b);
+                xp[j + h] = sub2(a, b);
+            }
+        }
+    }
+}
+
+// Normalized 16-point Hadamard H_16 / 4 of one block: the butterflies, then each value times
+// 1/sqrt(16) = 1/4 (a single rounding, exact unless the product is subnormal).
+__device__ __forceinline__ void fwht16(u64 (&xp)[8]) {
+    fwht16_butterflies(xp);
+    const u64 q = pk(0.25f, 0.25f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) xp[j] = mul2(xp[j], q);
+}
+
+// Tensor amax of the rotated blocks.  Every thread rotates whole 16-element blocks and keeps
+// the largest unnormalized magnitude; the factor 1/4 is applied once to the maximum, which
+// gives the maximum of the normalized values because RN(a/4) is non-decreasing in a and
+// |RN(v/4)| = RN(|v|/4).  The raw 16-byte vectors of U blocks (eight loads for bf16, the
+// same bytes for fp32) are issued before any of them is converted, so the registers hold
+// the loads in flight rather than unpacked pairs.
+template <int IN>
+__global__ void __launch_bounds__(kThreads, 4) amax_had16_kernel(const void* __restrict__ xv, int64_t rows,
+                                                              int64_t cols, int64_t ld, uint32_t* __restrict__ ws,
+                                                              float* __restrict__ gscale, int publish) {
+    constexpr int VPB = IN == FP4Q_IN_BF16 ? 2 : 4;   // 16-byte vectors per block
+    constexpr int U = 8 / VPB;                        // blocks in flight per thread
+    const int64_t nb = cols / 16;
+    const int64_t total = rows * nb;
+    const int64_t step = (int64_t)gridDim.x * blockDim.x;
+    uint32_t m = 0;
+    auto src = [&](int64_t blk) {
+        const int64_t r = blk / nb;
+        const int64_t off = r * ld + (blk - r * nb) * 16;   // elements
+        return reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(xv) + off * (IN == FP4Q_IN_BF16 ? 2 : 4));
+    };
+    auto fold = [&](const uint4 (&v)[VPB]) {
+        u64 xp[8];
+        if (IN == FP4Q_IN_BF16) {
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                xp[4 * q] = bf16x2_to_pair(v[q].x); xp[4 * q + 1] = bf16x2_to_pair(v[q].y);
+                xp[4 * q + 2] = bf16x2_to_pair(v[q].z); xp[4 * q + 3] = bf16x2_to_pair(v[q].w);
+            }
+        } else {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                xp[2 * q] = pk(__uint_as_float(v[q].x), __uint_as_float(v[q].y));
+                xp[2 * q + 1] = pk(__uint_as_float(v[q].z), __uint_as_float(v[q].w));
+            }
+        }
+        fwht16_butterflies(xp);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            float a, b;
+            upk(xp[j], a, b);
+            m = max(m, max(__float_as_uint(a) & 0x7FFFFFFFu, __float_as_uint(b) & 0x7FFFFFFFu));
+        }
+    };
+    auto load = [&](int64_t blk, uint4 (&v)[VPB]) {
+        const uint4* p = src(blk);
+#pragma unroll
+        for (int q = 0; q < VPB; ++q)   // read-only, no L1 allocation, 256-byte L2 fetches
+            asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v[q].x), "=r"(v[q].y), "=r"(v[q].z), "=r"(v[q].w) : "l"(p + q));
+    };
+    int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    for (; blk + (U - 1) * step < total; blk += U * step) {
+        uint4 v[U][VPB];
+#pragma unroll
+        for (int u = 0; u < U; ++u) load(blk + u * step, v[u]);
+#pragma unroll
+        for (int u = 0; u < U; ++u) fold(v[u]);
+    }
+    for (; blk < total; blk += step) {
+        uint4 v[VPB];
+        load(blk, v);
+        fold(v);
+    }
+    amax_finish(m, 0.25f, ws, gscale, publish);
 }
 
 // Packed codes of a block for a given reciprocal scale (8 bytes: elements 0..15).
@@ -291,7 +401,7 @@ __device__ __forceinline__ float zero_scale_error(const u64 (&xp)[8], const u64 
 // ScaleSweep (gist.science/ko/paper/2606.07618), Methodology; 4/6: Adaptive Block-Scaled
 // Data Types (gist.science/ko/paper/2603.28765), Problem.
 // ------------------------------------------------------------------------------------------
-template <int IN, int OBJ, typename IDX>
+template <int IN, int OBJ, bool HAD, typename IDX>
 __global__ void __launch_bounds__(kThreads, OBJ == FP4Q_SWEEP_WMSE ? 4 : FP4Q_SWEEP_MIN_CTAS)
     quant16_kernel(const void* __restrict__ xv, IDX rows, IDX cols, IDX ld, const float* __restrict__ imp,
                    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, const float* __restrict__ gscale,
@@ -318,6 +428,7 @@ __global__ void __launch_bounds__(kThreads, OBJ == FP4Q_SWEEP_WMSE ? 4 : FP4Q_SW
     }
     u64 xp[8], wp[8];
     load_block16<IN>(xv, (int64_t)r * ld + b * 16, xp);
+    if (HAD) fwht16(xp);
     if (WEIGHTED) {
         const float4* w4 = reinterpret_cast<const float4*>(imp + b * 16);
 #pragma unroll
@@ -366,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, OBJ == FP4Q_SWEEP_WMSE ? 4 : FP4Q_SW
 // Both errors are in units of the shared scale: FP4 r = RN(q - y); INT4 z = RN(y RN(7/6)),
 // n = clamp(rint(z), -7, 7), r = RN(RN(n RN(6/7)) - y).
 // ------------------------------------------------------------------------------------------
-template <int IN, typename IDX>
+template <int IN, bool HAD, typename IDX>
 __global__ void __launch_bounds__(kThreads, FP4Q_IF4_MIN_CTAS)
     if4_kernel(const void* __restrict__ xv, IDX rows, IDX cols, IDX ld, uint8_t* __restrict__ codes,
                uint8_t* __restrict__ scales, const float* __restrict__ gscale, uint32_t* __restrict__ ws) {
@@ -390,6 +501,7 @@ __global__ void __launch_bounds__(kThreads, FP4Q_IF4_MIN_CTAS)
     }
     u64 xp[8];
     load_block16<IN>(xv, (int64_t)r * ld + b * 16, xp);
+    if (HAD) fwht16(xp);
     const int p0 = S > 0.0f ? e4m3_rne(__fdiv_rn(block_absmax(xp), d6)) : 0;
     const float inv = s_inv[p0];
     const u64 inv2 = pk(inv, inv);
@@ -558,7 +670,7 @@ __device__ __forceinline__ void store_values(void* out, int64_t off, const float
     }
 }
 
-template <bool OUT_BF16, bool IF4>
+template <bool OUT_BF16, bool IF4, bool HAD>
 __global__ void __launch_bounds__(kThreads) dequant16_kernel(const uint8_t* __restrict__ codes,
                                                              const uint8_t* __restrict__ scales,
                                                              const float* __restrict__ gscale, int64_t rows,
@@ -591,6 +703,14 @@ __global__ void __launch_bounds__(kThreads) dequant16_kernel(const uint8_t* __re
                 v[2 * j] = __fmul_rn(g0, sv);
                 v[2 * j + 1] = __fmul_rn(g1, sv);
             }
+        }
+        if (HAD) {   // inverse rotation: H_16 / 4 is its own inverse
+            u64 vp[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) vp[j] = pk(v[2 * j], v[2 * j + 1]);
+            fwht16(vp);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) upk(vp[j], v[2 * j], v[2 * j + 1]);
         }
         store_values<OUT_BF16>(out, r * cols + b * 16, v);
     }
@@ -679,28 +799,63 @@ int check_common(const void* x, int dtype, int64_t rows, int64_t cols, int64_t l
 }
 
 // One quantization block per thread; 32-bit index arithmetic when the tensor allows it.
-template <int IN, int OBJ>
+template <int IN, int OBJ, bool HAD>
 void launch_q16(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* imp, uint8_t* codes,
                 uint8_t* scales, float* gs, uint32_t* ws, cudaStream_t st) {
     const int64_t total = rows * (cols / 16);
     const unsigned ctas = (unsigned)((total + kThreads - 1) / kThreads);
     if (total < ((int64_t)1 << 31) && rows * ld < ((int64_t)1 << 31))
-        quant16_kernel<IN, OBJ, uint32_t><<<ctas, kThreads, 0, st>>>(x, (uint32_t)rows, (uint32_t)cols, (uint32_t)ld,
-                                                                      imp, codes, scales, gs, ws);
+        quant16_kernel<IN, OBJ, HAD, uint32_t><<<ctas, kThreads, 0, st>>>(
+            x, (uint32_t)rows, (uint32_t)cols, (uint32_t)ld, imp, codes, scales, gs, ws);
     else
-        quant16_kernel<IN, OBJ, int64_t><<<ctas, kThreads, 0, st>>>(x, rows, cols, ld, imp, codes, scales, gs, ws);
+        quant16_kernel<IN, OBJ, HAD, int64_t><<<ctas, kThreads, 0, st>>>(x, rows, cols, ld, imp, codes, scales, gs,
+                                                                         ws);
 }
 
-template <int IN>
+template <int IN, bool HAD>
 void launch_if4(const void* x, int64_t rows, int64_t cols, int64_t ld, uint8_t* codes, uint8_t* scales, float* gs,
                 uint32_t* ws, cudaStream_t st) {
     const int64_t total = rows * (cols / 16);
     const unsigned ctas = (unsigned)((total + kThreads - 1) / kThreads);
     if (total < ((int64_t)1 << 31) && rows * ld < ((int64_t)1 << 31))
-        if4_kernel<IN, uint32_t><<<ctas, kThreads, 0, st>>>(x, (uint32_t)rows, (uint32_t)cols, (uint32_t)ld, codes,
-                                                             scales, gs, ws);
+        if4_kernel<IN, HAD, uint32_t><<<ctas, kThreads, 0, st>>>(x, (uint32_t)rows, (uint32_t)cols, (uint32_t)ld,
+                                                                  codes, scales, gs, ws);
     else
-        if4_kernel<IN, int64_t><<<ctas, kThreads, 0, st>>>(x, rows, cols, ld, codes, scales, gs, ws);
+        if4_kernel<IN, HAD, int64_t><<<ctas, kThreads, 0, st>>>(x, rows, cols, ld, codes, scales, gs, ws);
+}
+
+// Tensor scale pass: plain amax, or the amax of the 16-point rotated blocks.
+template <int IN>
+void launch_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, uint32_t* ws, float* gs, int publish,
+                 bool had16, cudaStream_t st) {
+    if (had16) {
+        amax_had16_kernel<IN><<<grid_for(amax_had16_kernel<IN>, rows * (cols / 16), 4), kThreads, 0, st>>>(
+            x, rows, cols, ld, ws, gs, publish);
+    } else {
+        const int64_t vecs = rows * cols * (IN == FP4Q_IN_BF16 ? 2 : 4) / 16;
+        amax_kernel<IN><<<grid_for(amax_kernel<IN>, vecs, 4), kThreads, 0, st>>>(x, rows, cols, ld, ws, gs, publish);
+    }
+}
+
+template <int IN, bool HAD>
+void launch_nvfp4_if4(const void* x, int64_t rows, int64_t cols, int64_t ld, int fmt, int obj, const float* imp,
+                      uint8_t* codes, uint8_t* scales, float* gs, uint32_t* ws, cudaStream_t st) {
+    if (fmt == FP4Q_IF4) {
+        launch_if4<IN, HAD>(x, rows, cols, ld, codes, scales, gs, ws, st);
+        return;
+    }
+    switch (obj) {
+        case FP4Q_ABSMAX: launch_q16<IN, FP4Q_ABSMAX, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, st); break;
+        case FP4Q_FOUR_OVER_SIX:
+            launch_q16<IN, FP4Q_FOUR_OVER_SIX, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, st);
+            break;
+        case FP4Q_SWEEP_MSE:
+            launch_q16<IN, FP4Q_SWEEP_MSE, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, st);
+            break;
+        default:   // WMSE is rejected with the rotation before any launch
+            if (!HAD) launch_q16<IN, FP4Q_SWEEP_WMSE, false>(x, rows, cols, ld, imp, codes, scales, gs, ws, st);
+            break;
+    }
 }
 
 template <int IN>
@@ -713,24 +868,13 @@ int launch_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, int f
             x, rows, cols, ld, codes, scales, ws, ocp);
         return launched(1);
     }
-    const int given = (flags & FP4Q_F_GLOBAL_SCALE_GIVEN) ? 1 : 0;
-    if (!given) {
-        const int64_t vecs = rows * cols * (IN == FP4Q_IN_BF16 ? 2 : 4) / 16;
-        amax_kernel<IN><<<grid_for(amax_kernel<IN>, vecs, 4), kThreads, 0, st>>>(x, rows, cols, ld, ws, gs, 0);
+    const bool had16 = (flags & FP4Q_F_HADAMARD16) != 0;
+    if (!(flags & FP4Q_F_GLOBAL_SCALE_GIVEN)) {
+        launch_amax<IN>(x, rows, cols, ld, ws, gs, 0, had16, st);
         ++n;
     }
-    if (fmt == FP4Q_IF4) {
-        launch_if4<IN>(x, rows, cols, ld, codes, scales, gs, ws, st);
-    } else {
-        switch (obj) {
-            case FP4Q_ABSMAX: launch_q16<IN, FP4Q_ABSMAX>(x, rows, cols, ld, imp, codes, scales, gs, ws, st); break;
-            case FP4Q_FOUR_OVER_SIX:
-                launch_q16<IN, FP4Q_FOUR_OVER_SIX>(x, rows, cols, ld, imp, codes, scales, gs, ws, st);
-                break;
-            case FP4Q_SWEEP_MSE: launch_q16<IN, FP4Q_SWEEP_MSE>(x, rows, cols, ld, imp, codes, scales, gs, ws, st); break;
-            default: launch_q16<IN, FP4Q_SWEEP_WMSE>(x, rows, cols, ld, imp, codes, scales, gs, ws, st); break;
-        }
-    }
+    if (had16) launch_nvfp4_if4<IN, true>(x, rows, cols, ld, fmt, obj, imp, codes, scales, gs, ws, st);
+    else launch_nvfp4_if4<IN, false>(x, rows, cols, ld, fmt, obj, imp, codes, scales, gs, ws, st);
     return launched(n + 1);
 }
 
@@ -761,6 +905,28 @@ int noalloc_scratch(void** out) {
     return FP4Q_OK;
 }
 
+template <bool HAD>
+void launch_dequant16(const uint8_t* codes, const uint8_t* scales, const float* gs, int64_t rows, int64_t cols,
+                      bool if4, bool bf, void* out, int g, cudaStream_t st) {
+    if (if4 && bf) dequant16_kernel<true, true, HAD><<<g, kThreads, 0, st>>>(codes, scales, gs, rows, cols, out);
+    else if (if4) dequant16_kernel<false, true, HAD><<<g, kThreads, 0, st>>>(codes, scales, gs, rows, cols, out);
+    else if (bf) dequant16_kernel<true, false, HAD><<<g, kThreads, 0, st>>>(codes, scales, gs, rows, cols, out);
+    else dequant16_kernel<false, false, HAD><<<g, kThreads, 0, st>>>(codes, scales, gs, rows, cols, out);
+}
+
+// Format, objective and flag checks shared by fp4q_quantize and fp4q_quantize_noalloc.
+int check_quantize_args(int fmt, int objective, uint32_t flags) {
+    if (fmt != FP4Q_NVFP4 && fmt != FP4Q_IF4 && fmt != FP4Q_MXFP4) return FP4Q_ERR_INVALID_ARG;
+    if (flags & ~(FP4Q_F_GLOBAL_SCALE_GIVEN | FP4Q_F_MX_OCP_FLOOR | FP4Q_F_HADAMARD16)) return FP4Q_ERR_INVALID_ARG;
+    if (fmt == FP4Q_NVFP4 && (objective < FP4Q_ABSMAX || objective > FP4Q_SWEEP_WMSE)) return FP4Q_ERR_INVALID_ARG;
+    if (fmt == FP4Q_MXFP4 && (flags & FP4Q_F_GLOBAL_SCALE_GIVEN)) return FP4Q_ERR_INVALID_ARG;
+    if (flags & FP4Q_F_HADAMARD16) {
+        if (fmt == FP4Q_MXFP4) return FP4Q_ERR_UNSUPPORTED;
+        if (fmt == FP4Q_NVFP4 && objective == FP4Q_SWEEP_WMSE) return FP4Q_ERR_UNSUPPORTED;
+    }
+    return FP4Q_OK;
+}
+
 }  // namespace fp4q
 
 using namespace fp4q;
@@ -773,18 +939,16 @@ int fp4q_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int64_t 
                   const float* importance, uint8_t* codes, uint8_t* scales, float* global_scale, void* workspace,
                   uint32_t flags, void* stream) {
     g_launches = 0;
-    if (fmt != FP4Q_NVFP4 && fmt != FP4Q_IF4 && fmt != FP4Q_MXFP4) return FP4Q_ERR_INVALID_ARG;
-    if (flags & ~(FP4Q_F_GLOBAL_SCALE_GIVEN | FP4Q_F_MX_OCP_FLOOR)) return FP4Q_ERR_INVALID_ARG;
-    if (fmt == FP4Q_NVFP4 && (objective < FP4Q_ABSMAX || objective > FP4Q_SWEEP_WMSE)) return FP4Q_ERR_INVALID_ARG;
+    int rc = check_quantize_args(fmt, objective, flags);
+    if (rc != FP4Q_OK) return rc;
     const int B = fmt == FP4Q_MXFP4 ? 32 : 16;
-    int rc = check_common(x, dtype, rows, cols, ld, B, codes, scales, workspace);
+    rc = check_common(x, dtype, rows, cols, ld, B, codes, scales, workspace);
     if (rc != FP4Q_OK || rows == 0 || cols == 0) return rc;
     if (fmt != FP4Q_MXFP4 && !global_scale) return FP4Q_ERR_INVALID_ARG;
     if (fmt == FP4Q_NVFP4 && objective == FP4Q_SWEEP_WMSE) {
         if (!importance) return FP4Q_ERR_INVALID_ARG;
         if (!aligned16(importance)) return FP4Q_ERR_ALIGNMENT;
     }
-    if (fmt == FP4Q_MXFP4 && (flags & FP4Q_F_GLOBAL_SCALE_GIVEN)) return FP4Q_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     uint32_t* ws = reinterpret_cast<uint32_t*>(workspace);
     if (dtype == FP4Q_IN_BF16)
@@ -794,26 +958,41 @@ int fp4q_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int64_t 
                                         flags, st);
 }
 
-int fp4q_global_scale(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld, float* global_scale,
-                      void* workspace, void* stream) {
+}  // extern "C"
+
+namespace fp4q {
+// fp4q_global_scale (plain, granule = 16 bytes of a row) and fp4q_hadamard_global_scale
+// (rotated blocks, granule = 16 elements).
+int global_scale_impl(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld, bool had16,
+                      float* global_scale, void* workspace, void* stream) {
     g_launches = 0;
     if (dtype != FP4Q_IN_F32 && dtype != FP4Q_IN_BF16) return FP4Q_ERR_INVALID_ARG;
     const int es = dtype == FP4Q_IN_BF16 ? 2 : 4;
-    if (rows < 0 || cols < 0 || ld < cols || (cols * es) % 16) return FP4Q_ERR_SHAPE;
+    if (rows < 0 || cols < 0 || ld < cols || (cols * es) % 16 || (had16 && cols % 16)) return FP4Q_ERR_SHAPE;
     if (rows > 0 && cols > 0 && rows > ((int64_t)1 << 40) / cols) return FP4Q_ERR_SHAPE;
     if (rows == 0 || cols == 0) return FP4Q_OK;
     if (!x || !global_scale || !workspace) return FP4Q_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(workspace) || (ld * es) % 16) return FP4Q_ERR_ALIGNMENT;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     uint32_t* ws = reinterpret_cast<uint32_t*>(workspace);
-    const int64_t vecs = rows * cols * (dtype == FP4Q_IN_BF16 ? 2 : 4) / 16;
-    if (dtype == FP4Q_IN_BF16)
-        amax_kernel<FP4Q_IN_BF16><<<grid_for(amax_kernel<FP4Q_IN_BF16>, vecs, 4), kThreads, 0, st>>>(
-            x, rows, cols, ld, ws, global_scale, 1);
-    else
-        amax_kernel<FP4Q_IN_F32><<<grid_for(amax_kernel<FP4Q_IN_F32>, vecs, 4), kThreads, 0, st>>>(
-            x, rows, cols, ld, ws, global_scale, 1);
+    if (dtype == FP4Q_IN_BF16) launch_amax<FP4Q_IN_BF16>(x, rows, cols, ld, ws, global_scale, 1, had16, st);
+    else launch_amax<FP4Q_IN_F32>(x, rows, cols, ld, ws, global_scale, 1, had16, st);
     return launched(1);
+}
+}  // namespace fp4q
+
+extern "C" {
+
+int fp4q_global_scale(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld, float* global_scale,
+                      void* workspace, void* stream) {
+    return global_scale_impl(x, dtype, rows, cols, ld, false, global_scale, workspace, stream);
+}
+
+int fp4q_hadamard_global_scale(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld, int had_size,
+                               float* global_scale, void* workspace, void* stream) {
+    g_launches = 0;
+    if (had_size != 16) return FP4Q_ERR_UNSUPPORTED;
+    return global_scale_impl(x, dtype, rows, cols, ld, true, global_scale, workspace, stream);
 }
 
 int fp4q_hadamard_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld, int had_size,
@@ -839,7 +1018,6 @@ int fp4q_dequantize(const uint8_t* codes, const uint8_t* scales, const float* gl
     g_launches = 0;
     if (fmt != FP4Q_NVFP4 && fmt != FP4Q_IF4 && fmt != FP4Q_MXFP4) return FP4Q_ERR_INVALID_ARG;
     if (flags & ~FP4Q_F_OUT_BF16) return FP4Q_ERR_INVALID_ARG;
-    if (inverse_hadamard && fmt != FP4Q_MXFP4) return FP4Q_ERR_UNSUPPORTED;
     const int B = fmt == FP4Q_MXFP4 ? 32 : 16;
     if (rows < 0 || cols < 0 || cols % B) return FP4Q_ERR_SHAPE;
     if (rows > 0 && cols > 0 && rows > ((int64_t)1 << 40) / cols) return FP4Q_ERR_SHAPE;
@@ -854,12 +1032,10 @@ int fp4q_dequantize(const uint8_t* codes, const uint8_t* scales, const float* gl
         else if (bf) dequant_mx_kernel<true, false><<<g, kThreads, 0, st>>>(codes, scales, rows, cols, out);
         else if (inverse_hadamard) dequant_mx_kernel<false, true><<<g, kThreads, 0, st>>>(codes, scales, rows, cols, out);
         else dequant_mx_kernel<false, false><<<g, kThreads, 0, st>>>(codes, scales, rows, cols, out);
-    } else if (fmt == FP4Q_IF4) {
-        if (bf) dequant16_kernel<true, true><<<g, kThreads, 0, st>>>(codes, scales, global_scale, rows, cols, out);
-        else dequant16_kernel<false, true><<<g, kThreads, 0, st>>>(codes, scales, global_scale, rows, cols, out);
+    } else if (inverse_hadamard) {
+        launch_dequant16<true>(codes, scales, global_scale, rows, cols, fmt == FP4Q_IF4, bf, out, g, st);
     } else {
-        if (bf) dequant16_kernel<true, false><<<g, kThreads, 0, st>>>(codes, scales, global_scale, rows, cols, out);
-        else dequant16_kernel<false, false><<<g, kThreads, 0, st>>>(codes, scales, global_scale, rows, cols, out);
+        launch_dequant16<false>(codes, scales, global_scale, rows, cols, fmt == FP4Q_IF4, bf, out, g, st);
     }
     return launched(1);
 }
@@ -869,9 +1045,8 @@ int fp4q_quantize_noalloc(const void* x, int dtype, int64_t rows, int64_t cols, 
                           float* global_scale, uint32_t* device_status, uint32_t flags, void* stream) {
     g_launches = 0;
     // the same argument checks as fp4q_quantize, made before the scratch is touched
-    if (fmt != FP4Q_NVFP4 && fmt != FP4Q_IF4 && fmt != FP4Q_MXFP4) return FP4Q_ERR_INVALID_ARG;
-    if (flags & ~(FP4Q_F_GLOBAL_SCALE_GIVEN | FP4Q_F_MX_OCP_FLOOR)) return FP4Q_ERR_INVALID_ARG;
-    if (fmt == FP4Q_NVFP4 && (objective < FP4Q_ABSMAX || objective > FP4Q_SWEEP_WMSE)) return FP4Q_ERR_INVALID_ARG;
+    const int rca = check_quantize_args(fmt, objective, flags);
+    if (rca != FP4Q_OK) return rca;
     const int B = fmt == FP4Q_MXFP4 ? 32 : 16;
     const void* aligned_stand_in = reinterpret_cast<const void*>(static_cast<uintptr_t>(256));
     int rc0 = check_common(x, dtype, rows, cols, ld, B, codes, scales, aligned_stand_in);
@@ -881,7 +1056,6 @@ int fp4q_quantize_noalloc(const void* x, int dtype, int64_t rows, int64_t cols, 
         if (!importance) return FP4Q_ERR_INVALID_ARG;
         if (!aligned16(importance)) return FP4Q_ERR_ALIGNMENT;
     }
-    if (fmt == FP4Q_MXFP4 && (flags & FP4Q_F_GLOBAL_SCALE_GIVEN)) return FP4Q_ERR_INVALID_ARG;
     if (device_status && (reinterpret_cast<uintptr_t>(device_status) & 3u)) return FP4Q_ERR_ALIGNMENT;
     void* scratch = nullptr;
     int rc = noalloc_scratch(&scratch);

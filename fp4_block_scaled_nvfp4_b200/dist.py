@@ -26,19 +26,21 @@ def reduce_global_scale(s_local, group=None):
 
 
 def sharded_quantize(x_local, fmt: str = "nvfp4", objective: str = "sweep_mse", importance=None, group=None,
-                     workspace=None, out=None):
+                     workspace=None, out=None, hadamard16: bool = False):
     """Quantize this rank's rows of a row-sharded tensor with the whole tensor's S.
 
-    Two kernels and one collective per call: the local amax pass (fp4q_global_scale), the
-    4-byte all-reduce-MAX, then fp4q_quantize with FP4Q_F_GLOBAL_SCALE_GIVEN.  MXFP4 has no
-    tensor scale and needs no collective.  Returns (codes, scales, S)."""
+    Two kernels and one collective per call: the local amax pass (fp4q_global_scale, or
+    fp4q_hadamard_global_scale for the 16-point rotated blocks), the 4-byte
+    all-reduce-MAX, then fp4q_quantize with FP4Q_F_GLOBAL_SCALE_GIVEN.  MXFP4 has no tensor
+    scale and needs no collective.  Returns (codes, scales, S)."""
     from . import global_scale, new_workspace, quantize
 
     ws = workspace if workspace is not None else new_workspace(x_local.device)
     if fmt == "mxfp4":
         return quantize(x_local, fmt, objective, out=out, workspace=ws)
-    s_all = reduce_global_scale(global_scale(x_local, workspace=ws), group)
-    return quantize(x_local, fmt, objective, importance=importance, global_scale=s_all, out=out, workspace=ws)
+    s_all = reduce_global_scale(global_scale(x_local, workspace=ws, hadamard16=hadamard16), group)
+    return quantize(x_local, fmt, objective, importance=importance, global_scale=s_all, out=out, workspace=ws,
+                    hadamard16=hadamard16)
 
 
 def max_over_ranks(value: float, device="cpu", group=None) -> float:

@@ -81,6 +81,8 @@ enum { FP4Q_ABSMAX = 0, FP4Q_FOUR_OVER_SIX = 1, FP4Q_SWEEP_MSE = 2, FP4Q_SWEEP_W
 #define FP4Q_F_GLOBAL_SCALE_GIVEN 0x1u  /* quantize: read S from *global_scale (no amax pass) */
 #define FP4Q_F_MX_OCP_FLOOR       0x2u  /* MXFP4: e = floor(log2 a_b) - 2 instead of the ceil rule */
 #define FP4Q_F_OUT_BF16           0x4u  /* dequantize: write bf16 (RNE of the fp32 value)     */
+#define FP4Q_F_HADAMARD16         0x8u  /* NVFP4/IF4 quantize: rotate every 16-element block by
+                                           H_16/4 first (see fp4q_hadamard_global_scale)      */
 
 /* Size in bytes of the workspace every quantize call needs (a small constant). */
 size_t fp4q_workspace_bytes(void);
@@ -93,7 +95,18 @@ size_t fp4q_workspace_bytes(void);
  *   fmt FP4Q_MXFP4 (objective, importance and global_scale ignored; see also
  *   fp4q_hadamard_quantize).
  *   rows >= 0, cols a multiple of 16 (32 for MXFP4), ld >= cols; rows*cols < 2^40.
- *   flags: FP4Q_F_GLOBAL_SCALE_GIVEN (NVFP4/IF4), FP4Q_F_MX_OCP_FLOOR (MXFP4).
+ *   flags: FP4Q_F_GLOBAL_SCALE_GIVEN (NVFP4/IF4), FP4Q_F_MX_OCP_FLOOR (MXFP4),
+ *   FP4Q_F_HADAMARD16 (NVFP4 with ABSMAX / FOUR_OVER_SIX / SWEEP_MSE, and IF4).
+ * FP4Q_F_HADAMARD16: every 16-element block is first rotated by the normalized Sylvester
+ *   Hadamard matrix H_16 / 4 (butterflies h = 1, 2, 4, 8 in binary32, then one exact
+ *   multiplication by 1/4 per value), and the whole method -- S, the block scales, the
+ *   scale search and the codes -- runs on the rotated values, so S = RN(max|H x| / 1536).
+ *   Bridging the Gap ... Microscaling FP4 (gist.science/ko/paper/2509.23202),
+ *   "Methodology", block-wise Hadamard transforms, which rotates NVFP4 as well as MXFP4.
+ *   A given S (FP4Q_F_GLOBAL_SCALE_GIVEN) must then be the rotated tensor's, e.g. from
+ *   fp4q_hadamard_global_scale.  SWEEP_WMSE with the flag returns FP4Q_ERR_UNSUPPORTED (a
+ *   per-column importance has no meaning once the columns of a block are mixed), and so
+ *   does MXFP4 (use fp4q_hadamard_quantize).  Dequantize with inverse_hadamard = 1.
  * Launches: NVFP4/IF4 without a given S: an amax kernel then the quantize kernel;
  * otherwise one kernel.  Empty tensors launch nothing.
  */
@@ -114,6 +127,18 @@ int fp4q_global_scale(const void* x, int dtype, int64_t rows, int64_t cols, int6
                       float* global_scale, void* workspace, void* stream);
 
 /*
+ * Tensor scale of the block-rotated tensor: S = RN(max|H x| / 1536), H x being every
+ * 16-element block of every row rotated by H_16 / 4 exactly as fp4q_quantize does under
+ * FP4Q_F_HADAMARD16 (so this S with FP4Q_F_GLOBAL_SCALE_GIVEN | FP4Q_F_HADAMARD16
+ * reproduces a call without the first flag).  had_size must be 16 (else
+ * FP4Q_ERR_UNSUPPORTED); cols a multiple of 16.  A non-finite element, or a rotation that
+ * overflows, gives S = NaN.  Status, workspace and errors as fp4q_global_scale.  Use: a
+ * row-sharded tensor reduces the per-shard S values by maximum.
+ */
+int fp4q_hadamard_global_scale(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                               int had_size, float* global_scale, void* workspace, void* stream);
+
+/*
  * MXFP4 quantization of H x: each 32-element block (along the contiguous dimension) is
  * rotated by the normalized Sylvester Hadamard matrix H_32 / sqrt(32) before the E8M0 scale
  * and the E2M1 codes are chosen (Bridging the Gap ... Microscaling FP4, "Methodology",
@@ -130,8 +155,9 @@ int fp4q_hadamard_quantize(const void* x, int dtype, int64_t rows, int64_t cols,
  * Dequantize codes + scales (+ S for NVFP4/IF4) into out [rows][cols], fp32 or (flag
  * FP4Q_F_OUT_BF16) bf16.  NVFP4: RN(q * RN(e(p) S)); IF4 blocks with bit 7 set:
  * RN(RN(n RN(6/7)) * RN(e(p) S)); MXFP4: RN(q * 2^(byte-127)) (byte 0xFF gives NaN).
- * inverse_hadamard (MXFP4 only): apply the same normalized 32-point transform to each
- * dequantized block (it is its own inverse up to rounding).  global_scale is a device
+ * inverse_hadamard: apply the normalized transform of the format's block size (32-point for
+ * MXFP4, 16-point H_16 / 4 for NVFP4/IF4) to each dequantized block, as butterflies then
+ * one multiplication per value (it is its own inverse up to rounding).  global_scale is a device
  * pointer (ignored for MXFP4).  out must be 16-byte aligned.
  */
 int fp4q_dequantize(const uint8_t* codes, const uint8_t* scales, const float* global_scale,

@@ -57,6 +57,11 @@ FAKE = 0x10000   # 16-byte aligned non-null stand-in; validation rejects before 
     ((FAKE, 1, 4, 32, 32, 0, 3, FAKE + 4, FAKE, FAKE, FAKE, FAKE, 0), fq.ERR_ALIGNMENT),  # weights
     ((FAKE, 1, 4, 32, 32, 0, 2, None, FAKE, FAKE, FAKE, FAKE, 0x80), fq.ERR_INVALID_ARG),  # unknown flag
     ((FAKE, 1, 4, 32, 32, 2, 0, None, FAKE, FAKE, None, FAKE, 1), fq.ERR_INVALID_ARG),  # MX with given S
+    ((FAKE, 1, 4, 32, 32, 0, 2, None, FAKE, FAKE, FAKE, FAKE, 0x10), fq.ERR_INVALID_ARG),  # unknown flag
+    ((FAKE, 1, 4, 64, 64, 2, 0, None, FAKE, FAKE, None, FAKE, 8), fq.ERR_UNSUPPORTED),  # MX + 16-point rotation
+    ((FAKE, 1, 4, 32, 32, 0, 3, FAKE, FAKE, FAKE, FAKE, FAKE, 8), fq.ERR_UNSUPPORTED),  # WMSE + rotation
+    ((FAKE, 1, 4, 24, 24, 1, 0, None, FAKE, FAKE, FAKE, FAKE, 8), fq.ERR_SHAPE),        # IF4 + rotation, cols % 16
+    ((None, 1, 0, 32, 32, 0, 2, None, None, None, None, None, 8), fq.OK),               # rotated, empty
     ((None, 1, 0, 32, 32, 0, 2, None, None, None, None, None, 0), fq.OK),               # empty: no launch
 ])
 def test_quantize_rejects_before_launch(args, rc):
@@ -71,7 +76,7 @@ def test_hadamard_and_dequant_validation():
     assert L.fp4q_hadamard_quantize(FAKE, 1, 4, 64, 64, 16, FAKE, FAKE, FAKE, 0, None) == fq.ERR_UNSUPPORTED
     assert L.fp4q_hadamard_quantize(FAKE, 1, 4, 48, 48, 32, FAKE, FAKE, FAKE, 0, None) == fq.ERR_SHAPE
     assert L.fp4q_dequantize(FAKE, FAKE, FAKE, 4, 24, 0, 0, FAKE, 0, None) == fq.ERR_SHAPE
-    assert L.fp4q_dequantize(FAKE, FAKE, FAKE, 4, 32, 0, 1, FAKE, 0, None) == fq.ERR_UNSUPPORTED
+    assert L.fp4q_dequantize(FAKE, FAKE, FAKE, 4, 24, 1, 1, FAKE, 0, None) == fq.ERR_SHAPE   # rotated IF4
     assert L.fp4q_dequantize(FAKE, FAKE, None, 4, 32, 0, 0, FAKE, 0, None) == fq.ERR_INVALID_ARG
     assert L.fp4q_dequantize(FAKE, FAKE, FAKE, 4, 32, 0, 0, FAKE + 4, 0, None) == fq.ERR_ALIGNMENT
     assert L.fp4q_dequantize(FAKE, FAKE, FAKE, 4, 32, 0, 0, FAKE, 8, None) == fq.ERR_INVALID_ARG
@@ -86,3 +91,9 @@ def test_global_scale_validation():
     assert L.fp4q_global_scale(FAKE, 1, 4, 16, 16, None, FAKE, None) == fq.ERR_INVALID_ARG
     assert L.fp4q_global_scale(FAKE, 3, 4, 16, 16, FAKE, FAKE, None) == fq.ERR_INVALID_ARG
     assert L.fp4q_global_scale(None, 1, 0, 16, 16, None, None, None) == fq.OK
+    # rotated tensor scale: 16-point only, whole blocks
+    assert L.fp4q_hadamard_global_scale(FAKE, 1, 4, 32, 32, 32, FAKE, FAKE, None) == fq.ERR_UNSUPPORTED
+    assert L.fp4q_hadamard_global_scale(FAKE, 1, 4, 8, 8, 16, FAKE, FAKE, None) == fq.ERR_SHAPE   # 16-byte rows
+    assert L.fp4q_hadamard_global_scale(FAKE, 1, 4, 32, 36, 16, FAKE, FAKE, None) == fq.ERR_ALIGNMENT  # 72-byte pitch
+    assert L.fp4q_hadamard_global_scale(FAKE, 1, 4, 32, 32, 16, None, FAKE, None) == fq.ERR_INVALID_ARG
+    assert L.fp4q_hadamard_global_scale(None, 1, 0, 16, 16, 16, None, None, None) == fq.OK

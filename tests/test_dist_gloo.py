@@ -46,8 +46,13 @@ def _worker(rank, world, port, results):
         s_bad_loc, _ = O.tensor_scale(bad)
         s_bad = reduce_global_scale(torch.tensor([s_bad_loc], dtype=torch.float32))
         slowest = max_over_ranks(1.5 + rank)
+        # the 16-point rotated path: S of the rotated shard, reduced the same way
+        s_rot_loc, _ = O.tensor_scale(O.rotate16(shard))
+        s_rot = reduce_global_scale(torch.tensor([s_rot_loc], dtype=torch.float32))
+        rot = O.nvfp4_quantize(shard, "sweep_mse", S=float(s_rot.item()), hadamard16=True)
         results[rank] = (float(s_all.item()), codes["codes"].tobytes(), codes["scales"].tobytes(),
-                         float(s_bad.item()), slowest)
+                         float(s_bad.item()), slowest, float(s_rot.item()), rot["codes"].tobytes(),
+                         rot["scales"].tobytes())
     finally:
         dist.destroy_process_group()
 
@@ -63,8 +68,13 @@ def test_sharded_scale_matches_whole_tensor():
     w = synth.make("cfg3", rows=32, cols=256)
     x = O.widen_bf16(w["x"])
     whole = O.nvfp4_quantize(x, "sweep_mse")
+    whole_rot = O.nvfp4_quantize(x, "sweep_mse", hadamard16=True)
+    assert whole_rot["S"] != whole["S"]
     for rank in range(world):
-        s_all, c, sc, s_bad, slowest = results[rank]
+        s_all, c, sc, s_bad, slowest, s_rot, c_rot, sc_rot = results[rank]
+        assert np.float32(s_rot).view(np.uint32) == np.float32(whole_rot["S"]).view(np.uint32)
+        assert c_rot == whole_rot["codes"][rank * 16:(rank + 1) * 16].tobytes()
+        assert sc_rot == whole_rot["scales"][rank * 16:(rank + 1) * 16].tobytes()
         assert np.float32(s_all).view(np.uint32) == np.float32(whole["S"]).view(np.uint32)
         assert c == whole["codes"][rank * 16:(rank + 1) * 16].tobytes()
         assert sc == whole["scales"][rank * 16:(rank + 1) * 16].tobytes()
