@@ -21,12 +21,12 @@ DEVSTAT_OK, DEVSTAT_NONFINITE, DEVSTAT_RANGE = 0, 1, 2
 IN_F32, IN_BF16 = 0, 1
 FORMATS = {"nvfp4": 0, "if4": 1, "mxfp4": 2}
 OBJECTIVES = {"absmax": 0, "four_over_six": 1, "sweep_mse": 2, "sweep_wmse": 3}
-F_GLOBAL_SCALE_GIVEN, F_MX_OCP_FLOOR, F_OUT_BF16, F_HADAMARD16 = 0x1, 0x2, 0x4, 0x8
+F_GLOBAL_SCALE_GIVEN, F_MX_OCP_FLOOR, F_OUT_BF16, F_HADAMARD16, F_HADAMARD32 = 0x1, 0x2, 0x4, 0x8, 0x10
 BLOCK = {"nvfp4": 16, "if4": 16, "mxfp4": 32}
 
 # Names of every function include/fp4q.h declares (checked against the header by the tests).
 EXPORTS = ("fp4q_workspace_bytes", "fp4q_global_scale", "fp4q_hadamard_global_scale", "fp4q_quantize",
-           "fp4q_hadamard_quantize", "fp4q_dequantize", "fp4q_quantize_noalloc", "fp4q_read_device_status", "fp4q_last_launch_count", "fp4q_status_string")
+           "fp4q_hadamard_quantize", "fp4q_dequantize", "fp4q_quantize_noalloc", "fp4q_quantize_host_async", "fp4q_read_device_status", "fp4q_last_launch_count", "fp4q_status_string")
 
 _lib = None
 
@@ -57,6 +57,8 @@ def lib():
         L.fp4q_dequantize.argtypes = [P, P, P, i64, i64, i32, i32, P, u32, P]
         L.fp4q_quantize_noalloc.restype = i32
         L.fp4q_quantize_noalloc.argtypes = [P, i32, i64, i64, i64, i32, i32, P, P, P, P, P, u32, P]
+        L.fp4q_quantize_host_async.restype = i32
+        L.fp4q_quantize_host_async.argtypes = [P, i32, i64, i64, i32, i32, P, P, P, P, P, P, P, P, P, u32, P, P, P, P]
         L.fp4q_read_device_status.restype = i32
         L.fp4q_read_device_status.argtypes = [P, C.POINTER(C.c_uint32), P]
         L.fp4q_last_launch_count.restype = i32
@@ -224,40 +226,78 @@ def last_launch_count() -> int:
     return int(lib().fp4q_last_launch_count())
 
 
+def split_fmt(fmt: str):
+    """'nvfp4_had' / 'if4_had' -> 16-point rotated NVFP4 / IF4, 'mxfp4_had' -> rotated MXFP4;
+    returns (base format, flags)."""
+    if not fmt.endswith("_had"):
+        return fmt, 0
+    base = fmt[:-4]
+    return base, (F_HADAMARD32 if base == "mxfp4" else F_HADAMARD16)
+
+
 def alloc_host_outputs(rows: int, cols: int, fmt: str):
     """Pinned host buffers for (codes, scales, S)."""
     torch = _torch()
-    fmt = fmt[:-4] if fmt.endswith("_had") else fmt
+    base, _ = split_fmt(fmt)
     return (torch.empty((rows, cols // 2), dtype=torch.uint8, pin_memory=True),
-            torch.empty((rows, cols // BLOCK[fmt]), dtype=torch.uint8, pin_memory=True),
+            torch.empty((rows, cols // BLOCK[base]), dtype=torch.uint8, pin_memory=True),
             torch.empty((1,), dtype=torch.float32, pin_memory=True))
 
 
-def quantize_host(x_host, fmt="nvfp4", objective="sweep_mse", importance=None, stream=None, workspace=None,
-                  dev_bufs=None, host_out=None):
-    """End-to-end call on host (pinned) memory: copy the input in, quantize on the device,
-    copy codes, scales and S back (asynchronously on the current stream).
-    fmt "mxfp4_had" selects the Hadamard-rotated MXFP4 path, "nvfp4_had" / "if4_had" the
-    16-point rotated NVFP4 / IF4 paths.  Returns host (codes, scales, S)."""
-    torch = _torch()
-    rows, cols = x_host.shape
-    base = fmt[:-4] if fmt.endswith("_had") else fmt
-    if dev_bufs is None:
-        dev_bufs = {"x": torch.empty(x_host.shape, dtype=x_host.dtype, device="cuda"),
-                    "out": alloc_outputs(rows, cols, base, "cuda")}
-    if host_out is None:
-        host_out = alloc_host_outputs(rows, cols, base)
-    xd = dev_bufs["x"]
-    xd.copy_(x_host, non_blocking=True)
-    if fmt == "mxfp4_had":
-        codes, scales = hadamard_quantize(xd, out=dev_bufs["out"], workspace=workspace, stream=stream)
-        gs = None
-    else:
-        codes, scales, gs = quantize(xd, base, objective, importance=importance, out=dev_bufs["out"],
-                                     workspace=workspace, stream=stream, hadamard16=fmt.endswith("_had"))
-    hc, hs, hg = host_out
-    hc.copy_(codes, non_blocking=True)
-    hs.copy_(scales, non_blocking=True)
-    if gs is not None:
-        hg.copy_(gs, non_blocking=True)
-    return hc, hs, (hg if gs is not None else None)
+class HostQuantizer:
+    """Quantize tensors that live in pinned host memory (fp4q_quantize_host_async).
+
+    Holds `depth` device staging sets (input, codes, scales, S, workspace and two events)
+    used in turn, a copy stream for the input copies and a compute stream for the kernels
+    and the output copies, so the input copy of one call overlaps the previous call's
+    kernels and output copies.  Each call returns the host (codes, scales, S) it will fill;
+    they are valid once `synchronize()` (or the compute stream) has passed the call.
+    fmt: "nvfp4", "if4", "mxfp4", or the rotated "nvfp4_had", "if4_had", "mxfp4_had"."""
+
+    def __init__(self, rows, cols, fmt="nvfp4", objective="sweep_mse", importance=None, dtype=None, depth=2,
+                 device="cuda", copy_stream=None, compute_stream=None):
+        torch = _torch()
+        self.rows, self.cols, self.fmt, self.objective = rows, cols, fmt, objective
+        self.base, self.flags = split_fmt(fmt)
+        self.dtype = dtype or torch.bfloat16
+        self.importance = importance
+        self.copy_stream = copy_stream or torch.cuda.Stream(device=device)
+        self.compute_stream = compute_stream or torch.cuda.Stream(device=device)
+        self.sets = []
+        for _ in range(max(1, depth)):
+            codes, scales, gs = alloc_outputs(rows, cols, self.base, device)
+            st = {"x": torch.empty((rows, cols), dtype=self.dtype, device=device), "codes": codes, "scales": scales,
+                  "S": gs, "ws": new_workspace(device), "staged": torch.cuda.Event(), "free": torch.cuda.Event()}
+            st["free"].record(self.compute_stream)   # the first use of the set waits on nothing
+            st["staged"].record(self.copy_stream)
+            self.sets.append(st)
+        self.turn = 0
+
+    def __call__(self, x_host, host_out=None):
+        if tuple(x_host.shape) != (self.rows, self.cols) or x_host.dtype != self.dtype or not x_host.is_contiguous():
+            raise Fp4qError("x_host must be a contiguous [rows, cols] tensor of the quantizer's dtype")
+        st = self.sets[self.turn]
+        self.turn = (self.turn + 1) % len(self.sets)
+        hc, hs, hg = host_out if host_out is not None else alloc_host_outputs(self.rows, self.cols, self.fmt)
+        rc = lib().fp4q_quantize_host_async(
+            _ptr(x_host), _dtype_code(x_host), self.rows, self.cols, FORMATS[self.base],
+            OBJECTIVES.get(self.objective or "absmax", 0), _ptr(self.importance), _ptr(hc), _ptr(hs),
+            _ptr(hg) if self.base != "mxfp4" else None, _ptr(st["x"]), _ptr(st["codes"]), _ptr(st["scales"]),
+            _ptr(st["S"]) if self.base != "mxfp4" else None, _ptr(st["ws"]), self.flags,
+            C.c_void_p(self.copy_stream.cuda_stream), C.c_void_p(self.compute_stream.cuda_stream),
+            C.c_void_p(st["staged"].cuda_event), C.c_void_p(st["free"].cuda_event))
+        _check(rc, "fp4q_quantize_host_async")
+        return hc, hs, (hg if self.base != "mxfp4" else None)
+
+    def synchronize(self):
+        self.compute_stream.synchronize()
+
+
+def quantize_host(x_host, fmt="nvfp4", objective="sweep_mse", importance=None, host_out=None):
+    """One end-to-end call on host (pinned) memory: copy in, quantize, copy codes, scales and
+    S back; returns the host (codes, scales, S) after the copies have completed."""
+    q = HostQuantizer(x_host.shape[0], x_host.shape[1], fmt, objective, importance=importance, dtype=x_host.dtype,
+                      depth=1)
+    out = q(x_host, host_out)
+    q.synchronize()
+    return out

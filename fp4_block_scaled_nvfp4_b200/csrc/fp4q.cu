@@ -864,8 +864,12 @@ int launch_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, int f
     int n = 0;
     if (fmt == FP4Q_MXFP4) {
         const int ocp = (flags & FP4Q_F_MX_OCP_FLOOR) ? 1 : 0;
-        mxfp4_kernel<IN, false><<<grid_for(mxfp4_kernel<IN, false>, rows * (cols / 32), 8), kThreads, 0, st>>>(
-            x, rows, cols, ld, codes, scales, ws, ocp);
+        if (flags & FP4Q_F_HADAMARD32)
+            mxfp4_kernel<IN, true><<<grid_for(mxfp4_kernel<IN, true>, rows * (cols / 32), 8), kThreads, 0, st>>>(
+                x, rows, cols, ld, codes, scales, ws, ocp);
+        else
+            mxfp4_kernel<IN, false><<<grid_for(mxfp4_kernel<IN, false>, rows * (cols / 32), 8), kThreads, 0, st>>>(
+                x, rows, cols, ld, codes, scales, ws, ocp);
         return launched(1);
     }
     const bool had16 = (flags & FP4Q_F_HADAMARD16) != 0;
@@ -917,13 +921,15 @@ void launch_dequant16(const uint8_t* codes, const uint8_t* scales, const float* 
 // Format, objective and flag checks shared by fp4q_quantize and fp4q_quantize_noalloc.
 int check_quantize_args(int fmt, int objective, uint32_t flags) {
     if (fmt != FP4Q_NVFP4 && fmt != FP4Q_IF4 && fmt != FP4Q_MXFP4) return FP4Q_ERR_INVALID_ARG;
-    if (flags & ~(FP4Q_F_GLOBAL_SCALE_GIVEN | FP4Q_F_MX_OCP_FLOOR | FP4Q_F_HADAMARD16)) return FP4Q_ERR_INVALID_ARG;
+    if (flags & ~(FP4Q_F_GLOBAL_SCALE_GIVEN | FP4Q_F_MX_OCP_FLOOR | FP4Q_F_HADAMARD16 | FP4Q_F_HADAMARD32))
+        return FP4Q_ERR_INVALID_ARG;
     if (fmt == FP4Q_NVFP4 && (objective < FP4Q_ABSMAX || objective > FP4Q_SWEEP_WMSE)) return FP4Q_ERR_INVALID_ARG;
     if (fmt == FP4Q_MXFP4 && (flags & FP4Q_F_GLOBAL_SCALE_GIVEN)) return FP4Q_ERR_INVALID_ARG;
     if (flags & FP4Q_F_HADAMARD16) {
         if (fmt == FP4Q_MXFP4) return FP4Q_ERR_UNSUPPORTED;
         if (fmt == FP4Q_NVFP4 && objective == FP4Q_SWEEP_WMSE) return FP4Q_ERR_UNSUPPORTED;
     }
+    if ((flags & FP4Q_F_HADAMARD32) && fmt != FP4Q_MXFP4) return FP4Q_ERR_UNSUPPORTED;
     return FP4Q_OK;
 }
 
@@ -1000,17 +1006,8 @@ int fp4q_hadamard_quantize(const void* x, int dtype, int64_t rows, int64_t cols,
     g_launches = 0;
     if (had_size != 32) return FP4Q_ERR_UNSUPPORTED;
     if (flags & ~FP4Q_F_MX_OCP_FLOOR) return FP4Q_ERR_INVALID_ARG;
-    int rc = check_common(x, dtype, rows, cols, ld, 32, codes, scales, workspace);
-    if (rc != FP4Q_OK || rows == 0 || cols == 0) return rc;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    uint32_t* ws = reinterpret_cast<uint32_t*>(workspace);
-    const int ocp = (flags & FP4Q_F_MX_OCP_FLOOR) ? 1 : 0;
-    const int g = grid_for(mxfp4_kernel<FP4Q_IN_BF16, true>, rows * (cols / 32), 8);
-    if (dtype == FP4Q_IN_BF16)
-        mxfp4_kernel<FP4Q_IN_BF16, true><<<g, kThreads, 0, st>>>(x, rows, cols, ld, codes, scales, ws, ocp);
-    else
-        mxfp4_kernel<FP4Q_IN_F32, true><<<g, kThreads, 0, st>>>(x, rows, cols, ld, codes, scales, ws, ocp);
-    return launched(1);
+    return fp4q_quantize(x, dtype, rows, cols, ld, FP4Q_MXFP4, 0, nullptr, codes, scales, nullptr, workspace,
+                         flags | FP4Q_F_HADAMARD32, stream);
 }
 
 int fp4q_dequantize(const uint8_t* codes, const uint8_t* scales, const float* global_scale, int64_t rows,
@@ -1069,6 +1066,50 @@ int fp4q_quantize_noalloc(const void* x, int dtype, int64_t rows, int64_t cols, 
         cudaMemcpyAsync(device_status, scratch, sizeof(uint32_t), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
         return FP4Q_ERR_CUDA;
     return rc;
+}
+
+int fp4q_quantize_host_async(const void* x_host, int dtype, int64_t rows, int64_t cols, int fmt, int objective,
+                             const float* importance, uint8_t* codes_host, uint8_t* scales_host, float* S_host,
+                             void* x_dev, uint8_t* codes_dev, uint8_t* scales_dev, float* S_dev, void* workspace,
+                             uint32_t flags, void* copy_stream, void* compute_stream, void* staged_event,
+                             void* free_event) {
+    g_launches = 0;
+    int rc = check_quantize_args(fmt, objective, flags);
+    if (rc != FP4Q_OK) return rc;
+    const int B = fmt == FP4Q_MXFP4 ? 32 : 16;
+    rc = check_common(x_dev, dtype, rows, cols, cols, B, codes_dev, scales_dev, workspace);
+    if (rc != FP4Q_OK || rows == 0 || cols == 0) return rc;
+    if (!x_host || !codes_host || !scales_host || !staged_event || !free_event) return FP4Q_ERR_INVALID_ARG;
+    if (fmt != FP4Q_MXFP4 && (!S_dev || !S_host)) return FP4Q_ERR_INVALID_ARG;
+    if (fmt == FP4Q_NVFP4 && objective == FP4Q_SWEEP_WMSE) {
+        if (!importance) return FP4Q_ERR_INVALID_ARG;
+        if (!aligned16(importance)) return FP4Q_ERR_ALIGNMENT;
+    }
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(copy_stream);
+    cudaStream_t ks = reinterpret_cast<cudaStream_t>(compute_stream);
+    cudaEvent_t staged = reinterpret_cast<cudaEvent_t>(staged_event);
+    cudaEvent_t freed = reinterpret_cast<cudaEvent_t>(free_event);
+    const size_t in_bytes = (size_t)rows * (size_t)cols * (dtype == FP4Q_IN_BF16 ? 2 : 4);
+    // the staging input is overwritten only once the kernels of its previous use have read it
+    if (cudaStreamWaitEvent(cs, freed, 0) != cudaSuccess) return FP4Q_ERR_CUDA;
+    if (cudaMemcpyAsync(x_dev, x_host, in_bytes, cudaMemcpyHostToDevice, cs) != cudaSuccess) return FP4Q_ERR_CUDA;
+    if (cudaEventRecord(staged, cs) != cudaSuccess || cudaStreamWaitEvent(ks, staged, 0) != cudaSuccess)
+        return FP4Q_ERR_CUDA;
+    rc = fp4q_quantize(x_dev, dtype, rows, cols, cols, fmt, objective, importance, codes_dev, scales_dev,
+                       fmt == FP4Q_MXFP4 ? nullptr : S_dev, workspace, flags, compute_stream);
+    if (rc != FP4Q_OK) return rc;
+    const int n = g_launches;
+    if (cudaEventRecord(freed, ks) != cudaSuccess) return FP4Q_ERR_CUDA;
+    if (cudaMemcpyAsync(codes_host, codes_dev, (size_t)rows * (size_t)(cols / 2), cudaMemcpyDeviceToHost, ks) !=
+            cudaSuccess ||
+        cudaMemcpyAsync(scales_host, scales_dev, (size_t)rows * (size_t)(cols / B), cudaMemcpyDeviceToHost, ks) !=
+            cudaSuccess)
+        return FP4Q_ERR_CUDA;
+    if (fmt != FP4Q_MXFP4 &&
+        cudaMemcpyAsync(S_host, S_dev, sizeof(float), cudaMemcpyDeviceToHost, ks) != cudaSuccess)
+        return FP4Q_ERR_CUDA;
+    g_launches = n;
+    return FP4Q_OK;
 }
 
 int fp4q_read_device_status(const void* workspace, uint32_t* status, void* stream) {

@@ -166,10 +166,11 @@ def cfg5(rows=16384, cols=8192, seed=4):
 CONFIGS = {"cfg1": cfg1, "cfg2": cfg2, "cfg3": cfg3, "cfg4": cfg4, "cfg5": cfg5}
 
 
-def make(name: str, rows: int | None = None, cols: int | None = None):
-    """Build a workload; rows/cols override the full size (same distribution, smaller tensor)."""
+def make(name: str, rows: int | None = None, cols: int | None = None, seed: int | None = None):
+    """Build a workload; rows/cols override the full size (same distribution, smaller tensor),
+    seed another draw of the same distribution."""
     fn = CONFIGS[name]
-    kw = {}
+    kw = {} if seed is None else {"seed": seed}
     if rows is not None:
         kw["rows"] = rows
     if cols is not None:

@@ -83,6 +83,8 @@ enum { FP4Q_ABSMAX = 0, FP4Q_FOUR_OVER_SIX = 1, FP4Q_SWEEP_MSE = 2, FP4Q_SWEEP_W
 #define FP4Q_F_OUT_BF16           0x4u  /* dequantize: write bf16 (RNE of the fp32 value)     */
 #define FP4Q_F_HADAMARD16         0x8u  /* NVFP4/IF4 quantize: rotate every 16-element block by
                                            H_16/4 first (see fp4q_hadamard_global_scale)      */
+#define FP4Q_F_HADAMARD32         0x10u /* MXFP4 quantize: rotate every 32-element block first,
+                                           as fp4q_hadamard_quantize does                     */
 
 /* Size in bytes of the workspace every quantize call needs (a small constant). */
 size_t fp4q_workspace_bytes(void);
@@ -96,7 +98,9 @@ size_t fp4q_workspace_bytes(void);
  *   fp4q_hadamard_quantize).
  *   rows >= 0, cols a multiple of 16 (32 for MXFP4), ld >= cols; rows*cols < 2^40.
  *   flags: FP4Q_F_GLOBAL_SCALE_GIVEN (NVFP4/IF4), FP4Q_F_MX_OCP_FLOOR (MXFP4),
- *   FP4Q_F_HADAMARD16 (NVFP4 with ABSMAX / FOUR_OVER_SIX / SWEEP_MSE, and IF4).
+ *   FP4Q_F_HADAMARD16 (NVFP4 with ABSMAX / FOUR_OVER_SIX / SWEEP_MSE, and IF4),
+ *   FP4Q_F_HADAMARD32 (MXFP4 only, else FP4Q_ERR_UNSUPPORTED; identical to
+ *   fp4q_hadamard_quantize).
  * FP4Q_F_HADAMARD16: every 16-element block is first rotated by the normalized Sylvester
  *   Hadamard matrix H_16 / 4 (butterflies h = 1, 2, 4, 8 in binary32, then one exact
  *   multiplication by 1/4 per value), and the whole method -- S, the block scales, the
@@ -150,6 +154,40 @@ int fp4q_hadamard_global_scale(const void* x, int dtype, int64_t rows, int64_t c
 int fp4q_hadamard_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld,
                            int had_size, uint8_t* codes, uint8_t* scales,
                            void* workspace, uint32_t flags, void* stream);
+
+/*
+ * Quantize a tensor that lives in host memory: copy it in, quantize, copy codes, scales
+ * (and S) out, all enqueued asynchronously; the call returns before any of it completes.
+ * The pages have no counterpart; this is the end-to-end form of fp4q_quantize for callers
+ * whose tensors arrive in host memory, built so that consecutive calls overlap.
+ *   x_host [rows][cols] (contiguous, bf16 or fp32), codes_host [rows][cols/2],
+ *   scales_host [rows][cols/B], S_host [1] (NVFP4/IF4; may be NULL for MXFP4): host
+ *   memory, page-locked (cudaHostAlloc / pinned) for the copies to be asynchronous.
+ *   x_dev, codes_dev, scales_dev, S_dev, workspace: one caller-owned device staging set
+ *   (same sizes, contiguous; alignment and zeroed workspace as fp4q_quantize).
+ *   fmt, objective, importance (device), flags: as fp4q_quantize (S_dev is read, not
+ *   written, under FP4Q_F_GLOBAL_SCALE_GIVEN).
+ *   copy_stream: carries the host-to-device copy; compute_stream: the kernels and the
+ *   device-to-host copies (cudaStream_t; they may be equal, which serialises them).
+ *   staged_event, free_event: two cudaEvent_t owned by the staging set (created by the
+ *   caller, timing disabled is fine).  The call records staged_event on copy_stream after
+ *   the input copy and makes compute_stream wait for it; it records free_event on
+ *   compute_stream after the kernels and, on its next use with the same set, makes
+ *   copy_stream wait for it before overwriting x_dev.  free_event must have been recorded
+ *   once (e.g. on compute_stream) before the set's first use.
+ * With two staging sets used alternately, the input copy of one call runs while the
+ * previous call's kernels and output copies run, so a stream of calls is bound by the
+ * host-to-device bandwidth instead of the sum of both copies.  The host output buffers of
+ * a call may be read once compute_stream has passed the call (synchronize or record an
+ * event after it).  Errors as fp4q_quantize; the device status lands in the set's
+ * workspace.  Launch count as fp4q_quantize (copies are not counted).
+ */
+int fp4q_quantize_host_async(const void* x_host, int dtype, int64_t rows, int64_t cols,
+                             int fmt, int objective, const float* importance,
+                             uint8_t* codes_host, uint8_t* scales_host, float* S_host,
+                             void* x_dev, uint8_t* codes_dev, uint8_t* scales_dev, float* S_dev,
+                             void* workspace, uint32_t flags, void* copy_stream,
+                             void* compute_stream, void* staged_event, void* free_event);
 
 /*
  * Dequantize codes + scales (+ S for NVFP4/IF4) into out [rows][cols], fp32 or (flag

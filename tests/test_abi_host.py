@@ -57,7 +57,8 @@ FAKE = 0x10000   # 16-byte aligned non-null stand-in; validation rejects before 
     ((FAKE, 1, 4, 32, 32, 0, 3, FAKE + 4, FAKE, FAKE, FAKE, FAKE, 0), fq.ERR_ALIGNMENT),  # weights
     ((FAKE, 1, 4, 32, 32, 0, 2, None, FAKE, FAKE, FAKE, FAKE, 0x80), fq.ERR_INVALID_ARG),  # unknown flag
     ((FAKE, 1, 4, 32, 32, 2, 0, None, FAKE, FAKE, None, FAKE, 1), fq.ERR_INVALID_ARG),  # MX with given S
-    ((FAKE, 1, 4, 32, 32, 0, 2, None, FAKE, FAKE, FAKE, FAKE, 0x10), fq.ERR_INVALID_ARG),  # unknown flag
+    ((FAKE, 1, 4, 32, 32, 0, 2, None, FAKE, FAKE, FAKE, FAKE, 0x20), fq.ERR_INVALID_ARG),  # unknown flag
+    ((FAKE, 1, 4, 32, 32, 0, 2, None, FAKE, FAKE, FAKE, FAKE, 0x10), fq.ERR_UNSUPPORTED),  # 32-point rotation, NVFP4
     ((FAKE, 1, 4, 64, 64, 2, 0, None, FAKE, FAKE, None, FAKE, 8), fq.ERR_UNSUPPORTED),  # MX + 16-point rotation
     ((FAKE, 1, 4, 32, 32, 0, 3, FAKE, FAKE, FAKE, FAKE, FAKE, 8), fq.ERR_UNSUPPORTED),  # WMSE + rotation
     ((FAKE, 1, 4, 24, 24, 1, 0, None, FAKE, FAKE, FAKE, FAKE, 8), fq.ERR_SHAPE),        # IF4 + rotation, cols % 16
@@ -97,3 +98,32 @@ def test_global_scale_validation():
     assert L.fp4q_hadamard_global_scale(FAKE, 1, 4, 32, 36, 16, FAKE, FAKE, None) == fq.ERR_ALIGNMENT  # 72-byte pitch
     assert L.fp4q_hadamard_global_scale(FAKE, 1, 4, 32, 32, 16, None, FAKE, None) == fq.ERR_INVALID_ARG
     assert L.fp4q_hadamard_global_scale(None, 1, 0, 16, 16, 16, None, None, None) == fq.OK
+
+
+def test_host_async_validation():
+    """fp4q_quantize_host_async rejects bad arguments before any copy or launch."""
+    L = fq.lib()
+    # x_host, dtype, rows, cols, fmt, obj, imp, codes_h, scales_h, S_h, x_dev, codes_dev, scales_dev, S_dev,
+    # ws, flags, copy_stream, compute_stream, staged_event, free_event
+    ok = [FAKE, 1, 4, 32, 0, 2, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, None, None, FAKE, FAKE]
+
+    def call(**kw):
+        a = list(ok)
+        names = ["x_host", "dtype", "rows", "cols", "fmt", "obj", "imp", "codes_h", "scales_h", "S_h", "x_dev",
+                 "codes_dev", "scales_dev", "S_dev", "ws", "flags", "cs", "ks", "staged", "free"]
+        for k, v in kw.items():
+            a[names.index(k)] = v
+        return L.fp4q_quantize_host_async(*a)
+
+    assert call(cols=24) == fq.ERR_SHAPE
+    assert call(fmt=2, cols=48, S_h=None, S_dev=None) == fq.ERR_SHAPE
+    assert call(x_host=None) == fq.ERR_INVALID_ARG
+    assert call(codes_h=None) == fq.ERR_INVALID_ARG
+    assert call(S_h=None) == fq.ERR_INVALID_ARG
+    assert call(staged=None) == fq.ERR_INVALID_ARG
+    assert call(free=None) == fq.ERR_INVALID_ARG
+    assert call(obj=3) == fq.ERR_INVALID_ARG                     # WMSE without weights
+    assert call(x_dev=FAKE + 8) == fq.ERR_ALIGNMENT
+    assert call(flags=0x8, fmt=2, cols=64) == fq.ERR_UNSUPPORTED  # 16-point rotation on MXFP4
+    assert call(flags=0x20) == fq.ERR_INVALID_ARG
+    assert call(rows=0, x_host=None, x_dev=None) == fq.OK and L.fp4q_last_launch_count() == 0
