@@ -255,28 +255,24 @@ def run_ours(args, rank, world):
     ws = fq.new_workspace(dev)
     launches_per_step = 0
 
-    def step(s, ev=None):
+    def amax(s):
+        fq.global_scale(xs[s], out=outs[s][2], workspace=ws, hadamard16=had16)
+        return 1
+
+    def quant(s):
         c, sc, g = outs[s]
-        if ev is not None:
-            ev[0].record()
-        if fmt.startswith("mxfp4"):   # one kernel, no tensor scale: the amax slot stays empty
-            if ev is not None:
-                ev[1].record()
+        if fmt.startswith("mxfp4"):   # one kernel, no tensor scale
             if fmt.endswith("had"):
                 fq.hadamard_quantize(xs[s], out=(c, sc, None), workspace=ws)
             else:
                 fq.quantize(xs[s], "mxfp4", out=(c, sc, None), workspace=ws)
-            if ev is not None:
-                ev[2].record()
-            return 1
-        fq.global_scale(xs[s], out=g, workspace=ws, hadamard16=had16)
-        if ev is not None:
-            ev[1].record()
-        fq.quantize(xs[s], base, obj or "absmax", importance=imp, global_scale=g, out=(c, sc, g), workspace=ws,
-                    hadamard16=had16)
-        if ev is not None:
-            ev[2].record()
-        return 2
+        else:
+            fq.quantize(xs[s], base, obj or "absmax", importance=imp, global_scale=g, out=(c, sc, g), workspace=ws,
+                        hadamard16=had16)
+        return 1
+
+    def step(s):
+        return (0 if fmt.startswith("mxfp4") else amax(s)) + quant(s)
 
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
@@ -285,21 +281,17 @@ def run_ours(args, rank, world):
             launches_per_step = step(i % nsets)
     torch.cuda.synchronize()
 
-    # CUDA graphs: one per buffer set (for a remainder of steps) and one that runs every set
-    # once in turn; external timing events inside the graphs bracket the amax and the quantize
-    # kernel of each step
-    graphs, evs = [], []
-    for s in range(nsets):
-        ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
+    def capture(body):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            step(s, ev)
-        graphs.append(g)
-        evs.append(ev)
-    cycle = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(cycle, stream=stream):
-        for s in range(nsets):
-            step(s, evs[s])
+            body()
+        return g
+
+    # CUDA graphs without timing nodes inside (an event recorded between two kernels of a graph
+    # costs several microseconds): one per buffer set, for a remainder of steps, and one that
+    # runs every set once in turn
+    graphs = [capture(lambda s=s: step(s)) for s in range(nsets)]
+    cycle = capture(lambda: [step(s) for s in range(nsets)])
     with torch.cuda.stream(stream):
         for s in range(nsets):
             graphs[s].replay()
@@ -324,12 +316,32 @@ def run_ours(args, rank, world):
     if world > 1:
         dist.barrier()
     ms = start.elapsed_time(end)
-    t_amax = [evs[s][0].elapsed_time(evs[s][1]) for s in range(nsets)]
-    t_q = [evs[s][1].elapsed_time(evs[s][2]) for s in range(nsets)]
     if world > 1:
         t = torch.tensor([ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
+
+    # per-kernel launch durations for the roofline: the same launches, one kernel kind at a
+    # time (every buffer set in turn, so reads still come from HBM), timed with CUDA events on
+    # the launching stream over kernel_reps launches
+    kernel_reps = max(nsets, (min(args.steps, 400) // nsets) * nsets)
+
+    def time_kernel(fn):
+        g = capture(lambda: [fn(s) for s in range(nsets)])
+        with torch.cuda.stream(stream):
+            g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            a.record()
+            for _ in range(kernel_reps // nsets):
+                g.replay()
+            b.record()
+        b.synchronize()
+        return a.elapsed_time(b) / kernel_reps
+
+    t_q = time_kernel(quant)
+    t_amax = None if fmt.startswith("mxfp4") else time_kernel(amax)
 
     # status of the last step must be clean
     st = fq.read_device_status(ws)
@@ -366,7 +378,7 @@ def run_ours(args, rank, world):
     peak, peak_src = load_peaks()
     per_step_ms = ms / args.steps
     value = alg * args.steps * world / (ms * 1e-3) / 1e9
-    tq = statistics.mean(t_q)
+    tq = t_q
     kernel_key = f"{args.workload}:quantize"
     achieved = alg / (tq * 1e-3) / 1e9
     clocks = clk.summary()
@@ -399,12 +411,13 @@ def run_ours(args, rank, world):
                    "method": obj or fmt, "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": f"{nsets} rotating input/output buffer sets, {nsets * (in_bytes + out_bytes) / 2**20:.0f} MB "
                          f"total (> 2x the 126 MB L2)",
-                   "timing": "CUDA graph of one step per buffer set, replayed in turn on one stream; CUDA events on that stream"},
+                   "timing": "CUDA graph of one step per buffer set (no timing nodes inside), replayed in turn on one "
+                             "stream; CUDA events on that stream"},
         "hbm_frac": round(value / world / peak, 4),
         "input_gbps": round(in_bytes * args.steps * world / (ms * 1e-3) / 1e9, 2),
         "elements_per_s": round(rows * cols * args.steps * world / (ms * 1e-3), 1),
-        "kernels_ms": {"amax": (None if fmt.startswith("mxfp4") else round(statistics.mean(t_amax), 5)),
-                       "quantize": round(tq, 5)},
+        "kernels_ms": {"amax": (None if t_amax is None else round(t_amax, 5)), "quantize": round(tq, 5),
+                       "how": f"each kernel alone, {kernel_reps} launches over the rotating buffer sets, CUDA events"},
         "roofline": roofline,
         "device_status": st,
         "gpu_launches": launches_per_step * args.steps,

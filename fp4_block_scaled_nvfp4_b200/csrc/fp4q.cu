@@ -191,16 +191,78 @@ __device__ __forceinline__ Setup read_setup(const float* gscale) {
     return s;
 }
 
-// sv(p) = RN(e(p) * S), inv(p) = RN(1/sv(p)) and s2(p) = RN(sv(p)^2) for every pattern p
-// (all 0 for p = 0 and 127).
-__device__ __forceinline__ void build_scale_table(float S, float* s_sv, float* s_inv, float* s_s2) {
-    for (int p = threadIdx.x; p < 128; p += blockDim.x) {
-        const float sv = (p == 0 || p == 127) ? 0.0f : __fmul_rn(e4m3_value(p), S);
-        s_sv[p] = sv;
-        s_inv[p] = sv == 0.0f ? 0.0f : __frcp_rn(sv);
-        s_s2[p] = __fmul_rn(sv, sv);
+// Per-pattern scale table {inv, s2} with inv = RN(1/sv), s2 = RN(sv^2), sv = RN(e(p) * S),
+// indexed by p + kTabPad for p = -kTabPad .. 126 + kTabPad, so that a candidate window
+// [p0 - 8, p0 + 7] never leaves it.  Entries for patterns that are not candidates (p <= 0 or
+// p >= 127) hold inv = 0 and s2 = NaN: their error is NaN, which never compares below the
+// best, so the candidate loop needs no bounds.  inv = 0 is also the zero scale's reciprocal,
+// which makes the codes of pattern 0 the signs of the elements.
+constexpr int kTabPad = 8;
+constexpr int kTabLen = 127 + 2 * kTabPad;
+__device__ __forceinline__ void build_scale_table(float S, float2* tab) {
+    for (int i = threadIdx.x; i < kTabLen; i += blockDim.x) {
+        const int p = i - kTabPad;
+        float2 t = make_float2(0.0f, __uint_as_float(0x7FC00000u));
+        if (p >= 1 && p <= 126) {
+            const float sv = __fmul_rn(e4m3_value(p), S);
+            t = make_float2(__frcp_rn(sv), __fmul_rn(sv, sv));
+        }
+        tab[i] = t;
     }
     __syncthreads();
+}
+
+// Raw 16-byte vectors of one 16-element block (2 for bf16, 4 for fp32), loaded ahead of the
+// scale table so that their latency overlaps it, and their conversion to 8 float pairs.
+template <int IN>
+struct RawBlock16 {
+    uint4 v[IN == FP4Q_IN_BF16 ? 2 : 4];
+};
+template <int IN>
+__device__ __forceinline__ void load_raw16(const void* xv, int64_t off, RawBlock16<IN>& rb) {
+    const uint4* p = reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(xv) + off * (IN == FP4Q_IN_BF16 ? 2 : 4));
+#pragma unroll
+    for (int q = 0; q < (IN == FP4Q_IN_BF16 ? 2 : 4); ++q) rb.v[q] = __ldg(p + q);
+}
+template <int IN>
+__device__ __forceinline__ void unpack16(const RawBlock16<IN>& rb, u64 (&xp)[8]) {
+    if (IN == FP4Q_IN_BF16) {
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            xp[4 * q] = bf16x2_to_pair(rb.v[q].x); xp[4 * q + 1] = bf16x2_to_pair(rb.v[q].y);
+            xp[4 * q + 2] = bf16x2_to_pair(rb.v[q].z); xp[4 * q + 3] = bf16x2_to_pair(rb.v[q].w);
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            xp[2 * q] = pk(__uint_as_float(rb.v[q].x), __uint_as_float(rb.v[q].y));
+            xp[2 * q + 1] = pk(__uint_as_float(rb.v[q].z), __uint_as_float(rb.v[q].w));
+        }
+    }
+}
+
+// Where block blk of a rows x cols tensor with row pitch ld lives: element offset of its
+// first value, its column block b, and its byte offset in the codes.  Contiguous rows
+// (ld == cols) need no division.
+template <typename IDX>
+struct BlockAt {
+    int64_t xoff, coff;
+    IDX b;
+};
+template <typename IDX, bool NEED_COL>
+__device__ __forceinline__ BlockAt<IDX> block_at(IDX blk, IDX cols, IDX ld, IDX nb) {
+    BlockAt<IDX> a;
+    if (ld == cols) {
+        a.xoff = (int64_t)blk * 16;
+        a.coff = (int64_t)blk * 8;
+        a.b = NEED_COL ? blk % nb : 0;
+    } else {
+        const IDX r = blk / nb, b = blk - r * nb;
+        a.xoff = (int64_t)r * ld + (int64_t)b * 16;
+        a.coff = (int64_t)blk * 8;
+        a.b = b;
+    }
+    return a;
 }
 
 // Load the 16 elements of one NVFP4 block as 8 float pairs (element 2k, 2k+1).
@@ -409,28 +471,35 @@ __global__ void __launch_bounds__(kThreads, OBJ == FP4Q_SWEEP_WMSE ? 4 : FP4Q_SW
     constexpr bool SWEEP = OBJ == FP4Q_SWEEP_MSE || OBJ == FP4Q_SWEEP_WMSE;
     constexpr bool WEIGHTED = OBJ == FP4Q_SWEEP_WMSE;
     constexpr int LO = WEIGHTED ? -8 : -3, HI = 7;
-    __shared__ float s_sv[128], s_inv[128], s_s2[128];
-    const Setup su = read_setup(gscale);
-    if (blockIdx.x == 0 && threadIdx.x == 0) ws[WS_STATUS] = su.flags;
-    build_scale_table(su.S, s_sv, s_inv, s_s2);
-    const float S = su.S;
-    const float d6 = __fmul_rn(6.0f, S), d4 = __fmul_rn(4.0f, S);
+    __shared__ float2 s_tab[kTabLen];
     const IDX nb = cols / 16;
     const IDX total = rows * nb;
     const IDX blk = (IDX)blockIdx.x * blockDim.x + threadIdx.x;
-    if (blk >= total) return;
-    const IDX r = blk / nb, b = blk - r * nb;
-    uint2* cdst = reinterpret_cast<uint2*>(codes + r * (cols / 2) + b * 8);
+    const bool live = blk < total;
+    const BlockAt<IDX> at = block_at<IDX, WEIGHTED>(live ? blk : 0, cols, ld, nb);
+    // bf16 blocks (8 registers) are loaded before S and the table so the load latency overlaps
+    // them; fp32 blocks (16 registers) would not fit the register cap across the table build
+    RawBlock16<IN> rb;
+    if (IN == FP4Q_IN_BF16 && live) load_raw16<IN>(xv, at.xoff, rb);
+    const Setup su = read_setup(gscale);
+    if (blockIdx.x == 0 && threadIdx.x == 0) ws[WS_STATUS] = su.flags;
+    build_scale_table(su.S, s_tab);
+    const float2* tab = s_tab + kTabPad;
+    const float S = su.S;
+    const float d6 = __fmul_rn(6.0f, S), d4 = __fmul_rn(4.0f, S);
+    if (!live) return;
+    uint2* cdst = reinterpret_cast<uint2*>(codes + at.coff);
     if (su.flags) {   // data out of contract: zero-filled outputs
         *cdst = make_uint2(0u, 0u);
         scales[blk] = 0;
         return;
     }
     u64 xp[8], wp[8];
-    load_block16<IN>(xv, (int64_t)r * ld + b * 16, xp);
+    if (IN != FP4Q_IN_BF16) load_raw16<IN>(xv, at.xoff, rb);
+    unpack16<IN>(rb, xp);
     if (HAD) fwht16(xp);
     if (WEIGHTED) {
-        const float4* w4 = reinterpret_cast<const float4*>(imp + b * 16);
+        const float4* w4 = reinterpret_cast<const float4*>(imp + (int64_t)at.b * 16);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const float4 v = __ldg(w4 + j);
@@ -446,27 +515,32 @@ __global__ void __launch_bounds__(kThreads, OBJ == FP4Q_SWEEP_WMSE ? 4 : FP4Q_SW
         if (OBJ == FP4Q_FOUR_OVER_SIX) {
             const int p4 = e4m3_rne(__fdiv_rn(ab, d4));   // p4 >= p0
             if (p4 != p0) {
-                const float e0 = p0 == 0 ? zero_scale_error<false>(xp, wp) : sweep_error<false>(xp, wp, s_inv[p0], s_s2[p0]);
-                const float e4 = sweep_error<false>(xp, wp, s_inv[p4], s_s2[p4]);
+                const float e0 = p0 == 0 ? zero_scale_error<false>(xp, wp) : sweep_error<false>(xp, wp, tab[p0].x, tab[p0].y);
+                const float e4 = sweep_error<false>(xp, wp, tab[p4].x, tab[p4].y);
                 if (e4 < e0) bp = p4;
             }
         } else if (SWEEP) {
+            // Candidates p0 + k, k = LO .. HI, in increasing offset with strict improvement
+            // (ties keep the lowest offset).  Patterns outside 1 .. 126 score NaN and are never
+            // taken; the zero scale (pattern 0), when it is in the window, is scored first as
+            // the lowest offset.  If every error is +inf the first candidate is kept.
             float best = INFINITY;
-            bp = max(p0 + LO, 0);                                   // first candidate if every error overflows
-            if (p0 + LO <= 0) best = zero_scale_error<WEIGHTED>(xp, wp);   // pattern 0 is the lowest offset
-            const int k0 = max(LO, 1 - p0), k1 = min(HI, 126 - p0);
+            int kb = max(LO, -p0);
+            if (p0 + LO <= 0) best = zero_scale_error<WEIGHTED>(xp, wp);
+            const float2* t = tab + p0;
 #pragma unroll(WEIGHTED ? kWmseUnroll : kMseUnroll)
-            for (int k = k0; k <= k1; ++k) {
-                const int p = p0 + k;
-                const float e = sweep_error<WEIGHTED>(xp, wp, s_inv[p], s_s2[p]);
+            for (int k = LO; k <= HI; ++k) {
+                const float2 c = t[k];
+                const float e = sweep_error<WEIGHTED>(xp, wp, c.x, c.y);
                 if (e < best) {
                     best = e;
-                    bp = p;
+                    kb = k;
                 }
             }
+            bp = p0 + kb;
         }
     }
-    *cdst = block_codes(xp, s_inv[bp]);
+    *cdst = block_codes(xp, tab[bp].x);
     scales[blk] = (uint8_t)bp;
 }
 
@@ -481,29 +555,36 @@ template <int IN, bool HAD, typename IDX>
 __global__ void __launch_bounds__(kThreads, FP4Q_IF4_MIN_CTAS)
     if4_kernel(const void* __restrict__ xv, IDX rows, IDX cols, IDX ld, uint8_t* __restrict__ codes,
                uint8_t* __restrict__ scales, const float* __restrict__ gscale, uint32_t* __restrict__ ws) {
-    __shared__ float s_sv[128], s_inv[128], s_s2[128];
-    const Setup su = read_setup(gscale);
-    if (blockIdx.x == 0 && threadIdx.x == 0) ws[WS_STATUS] = su.flags;
-    build_scale_table(su.S, s_sv, s_inv, s_s2);
-    const float S = su.S;
-    const float d6 = __fmul_rn(6.0f, S);
-    const float K76 = __fdiv_rn(7.0f, 6.0f), K67 = __fdiv_rn(6.0f, 7.0f);
+    __shared__ float2 s_tab[kTabLen];
     const IDX nb = cols / 16;
     const IDX total = rows * nb;
     const IDX blk = (IDX)blockIdx.x * blockDim.x + threadIdx.x;
-    if (blk >= total) return;
-    const IDX r = blk / nb, b = blk - r * nb;
-    uint2* cdst = reinterpret_cast<uint2*>(codes + r * (cols / 2) + b * 8);
+    const bool live = blk < total;
+    const BlockAt<IDX> at = block_at<IDX, false>(live ? blk : 0, cols, ld, nb);
+    // bf16 blocks (8 registers) are loaded before S and the table so the load latency overlaps
+    // them; fp32 blocks (16 registers) would not fit the register cap across the table build
+    RawBlock16<IN> rb;
+    if (IN == FP4Q_IN_BF16 && live) load_raw16<IN>(xv, at.xoff, rb);
+    const Setup su = read_setup(gscale);
+    if (blockIdx.x == 0 && threadIdx.x == 0) ws[WS_STATUS] = su.flags;
+    build_scale_table(su.S, s_tab);
+    const float2* tab = s_tab + kTabPad;
+    const float S = su.S;
+    const float d6 = __fmul_rn(6.0f, S);
+    const float K76 = __fdiv_rn(7.0f, 6.0f), K67 = __fdiv_rn(6.0f, 7.0f);
+    if (!live) return;
+    uint2* cdst = reinterpret_cast<uint2*>(codes + at.coff);
     if (su.flags) {
         *cdst = make_uint2(0u, 0u);
         scales[blk] = 0;
         return;
     }
     u64 xp[8];
-    load_block16<IN>(xv, (int64_t)r * ld + b * 16, xp);
+    if (IN != FP4Q_IN_BF16) load_raw16<IN>(xv, at.xoff, rb);
+    unpack16<IN>(rb, xp);
     if (HAD) fwht16(xp);
     const int p0 = S > 0.0f ? e4m3_rne(__fdiv_rn(block_absmax(xp), d6)) : 0;
-    const float inv = s_inv[p0];
+    const float inv = tab[p0].x;
     const u64 inv2 = pk(inv, inv);
     u64 accf = pk(0.0f, 0.0f), acci = pk(0.0f, 0.0f);
     uint32_t cf[8], ci[8];
