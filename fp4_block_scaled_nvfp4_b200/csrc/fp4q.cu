@@ -48,11 +48,14 @@ namespace fp4q {
 #endif
 constexpr int kMseUnroll = FP4Q_SWEEP_UNROLL, kWmseUnroll = FP4Q_WMSE_UNROLL;
 
-#ifndef FP4Q_IF4_MIN_CTAS
-#define FP4Q_IF4_MIN_CTAS 6     // CTAs per SM the IF4 kernel is compiled for (register cap)
+#ifndef FP4Q_PERSIST_MIN_CTAS
+#define FP4Q_PERSIST_MIN_CTAS 5 // CTAs per SM of the persistent IF4 / AbsMax / 4-6 kernels (register cap)
+#endif
+#ifndef FP4Q_SWEEP_PERSISTENT
+#define FP4Q_SWEEP_PERSISTENT 1 // 0: the MSE sweep runs one block per thread instead of as one persistent wave
 #endif
 #ifndef FP4Q_SWEEP_MIN_CTAS
-#define FP4Q_SWEEP_MIN_CTAS 6   // CTAs per SM the MSE/AbsMax/4-6 kernels are compiled for (register cap)
+#define FP4Q_SWEEP_MIN_CTAS 6   // CTAs per SM of a one-block-per-thread MSE sweep (register cap)
 #endif
 
 enum : int { WS_STATUS = 0, WS_PENDING = 1, WS_AMAX = 2, WS_CNT_AMAX = 3, WS_CNT_Q = 4 };
@@ -120,13 +123,14 @@ __device__ __forceinline__ void amax_finish(uint32_t m, float post, uint32_t* ws
     }
 }
 
-template <int IN>
-__global__ void __launch_bounds__(kThreads, 4) amax_kernel(const void* __restrict__ xv, int64_t rows, int64_t cols,
-                                                        int64_t ld, uint32_t* __restrict__ ws,
-                                                        float* __restrict__ gscale, int publish) {
+// Largest magnitude of the elements in the 16-byte vectors first, first + step, ... of a
+// rows x cols tensor with row pitch ld, as float bits (NaN and Inf order above every finite
+// value as integers).  U loads are kept in flight per thread on contiguous tensors.
+template <int IN, int U>
+__device__ __forceinline__ uint32_t amax_partial(const void* __restrict__ xv, int64_t rows, int64_t cols, int64_t ld,
+                                                 int64_t first, int64_t step) {
     const int64_t vpr = cols * (IN == FP4Q_IN_BF16 ? 2 : 4) / 16;   // 16-byte vectors per row
     const int64_t total = rows * vpr;
-    const int64_t step = (int64_t)gridDim.x * blockDim.x;
     uint32_t m = 0;
     const uint4* base = reinterpret_cast<const uint4*>(xv);
     const int64_t ldv = ld * (IN == FP4Q_IN_BF16 ? 2 : 4) / 16;
@@ -148,9 +152,8 @@ __global__ void __launch_bounds__(kThreads, 4) amax_kernel(const void* __restric
         const int64_t r = i / vpr;
         return base + r * ldv + (i - r * vpr);
     };
-    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (ldv == vpr) {   // contiguous tensor: eight independent 16-byte loads in flight per thread
-        constexpr int U = 8;
+    int64_t i = first;
+    if (ldv == vpr) {   // contiguous tensor: U independent 16-byte loads in flight per thread
         for (; i + (U - 1) * step < total; i += U * step) {
             uint4 v[U];
 #pragma unroll
@@ -171,26 +174,21 @@ __global__ void __launch_bounds__(kThreads, 4) amax_kernel(const void* __restric
     }
     for (; i < total; i += step) fold(__ldg(at(i)));
     if (IN == FP4Q_IN_BF16) m = max(m & 0xFFFFu, m >> 16) << 16;   // bf16 bits -> f32 bits
+    return m;
+}
+
+template <int IN>
+__global__ void __launch_bounds__(kThreads, 4) amax_kernel(const void* __restrict__ xv, int64_t rows, int64_t cols,
+                                                        int64_t ld, uint32_t* __restrict__ ws,
+                                                        float* __restrict__ gscale, int publish) {
+    const uint32_t m = amax_partial<IN, 8>(xv, rows, cols, ld, (int64_t)blockIdx.x * blockDim.x + threadIdx.x,
+                                           (int64_t)gridDim.x * blockDim.x);
     amax_finish(m, 1.0f, ws, gscale, publish);
 }
 
 // ------------------------------------------------------------------------------------------
 // Shared pieces of the NVFP4 / IF4 kernels
 // ------------------------------------------------------------------------------------------
-struct Setup {
-    float S;
-    uint32_t flags;
-};
-
-// Tensor scale (given by the caller or written by the amax pass just before) and the data
-// flags it implies; every CTA derives the same values.
-__device__ __forceinline__ Setup read_setup(const float* gscale) {
-    Setup s;
-    s.S = *gscale;
-    s.flags = scale_flags(s.S);
-    return s;
-}
-
 // Per-pattern scale table {inv, s2} with inv = RN(1/sv), s2 = RN(sv^2), sv = RN(e(p) * S),
 // indexed by p + kTabPad for p = -kTabPad .. 126 + kTabPad, so that a candidate window
 // [p0 - 8, p0 + 7] never leaves it.  Entries for patterns that are not candidates (p <= 0 or
@@ -265,27 +263,6 @@ __device__ __forceinline__ BlockAt<IDX> block_at(IDX blk, IDX cols, IDX ld, IDX 
     return a;
 }
 
-// Load the 16 elements of one NVFP4 block as 8 float pairs (element 2k, 2k+1).
-template <int IN>
-__device__ __forceinline__ void load_block16(const void* xv, int64_t off, u64 (&xp)[8]) {
-    if (IN == FP4Q_IN_BF16) {
-        const uint4* p = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(xv) + off);
-        const uint4 a = __ldg(p), b = __ldg(p + 1);
-        xp[0] = bf16x2_to_pair(a.x); xp[1] = bf16x2_to_pair(a.y);
-        xp[2] = bf16x2_to_pair(a.z); xp[3] = bf16x2_to_pair(a.w);
-        xp[4] = bf16x2_to_pair(b.x); xp[5] = bf16x2_to_pair(b.y);
-        xp[6] = bf16x2_to_pair(b.z); xp[7] = bf16x2_to_pair(b.w);
-    } else {
-        const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(xv) + off);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float4 v = __ldg(p + j);
-            xp[2 * j] = pk(v.x, v.y);
-            xp[2 * j + 1] = pk(v.z, v.w);
-        }
-    }
-}
-
 __device__ __forceinline__ float block_absmax(const u64 (&xp)[8]) {
     float m = 0.0f;
 #pragma unroll
@@ -329,21 +306,13 @@ __device__ __forceinline__ void fwht16(u64 (&xp)[8]) {
     for (int j = 0; j < 8; ++j) xp[j] = mul2(xp[j], q);
 }
 
-// Tensor amax of the rotated blocks.  Every thread rotates whole 16-element blocks and keeps
-// the largest unnormalized magnitude; the factor 1/4 is applied once to the maximum, which
-// gives the maximum of the normalized values because RN(a/4) is non-decreasing in a and
-// |RN(v/4)| = RN(|v|/4).  The raw 16-byte vectors of U blocks (eight loads for bf16, the
-// same bytes for fp32) are issued before any of them is converted, so the registers hold
-// the loads in flight rather than unpacked pairs.
 template <int IN>
-__global__ void __launch_bounds__(kThreads, 4) amax_had16_kernel(const void* __restrict__ xv, int64_t rows,
-                                                              int64_t cols, int64_t ld, uint32_t* __restrict__ ws,
-                                                              float* __restrict__ gscale, int publish) {
+__device__ __forceinline__ uint32_t amax_had16_partial(const void* __restrict__ xv, int64_t rows, int64_t cols,
+                                                       int64_t ld, int64_t first, int64_t step) {
     constexpr int VPB = IN == FP4Q_IN_BF16 ? 2 : 4;   // 16-byte vectors per block
     constexpr int U = 8 / VPB;                        // blocks in flight per thread
     const int64_t nb = cols / 16;
     const int64_t total = rows * nb;
-    const int64_t step = (int64_t)gridDim.x * blockDim.x;
     uint32_t m = 0;
     auto src = [&](int64_t blk) {
         const int64_t r = blk / nb;
@@ -380,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, 4) amax_had16_kernel(const void* __r
             asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
                          : "=r"(v[q].x), "=r"(v[q].y), "=r"(v[q].z), "=r"(v[q].w) : "l"(p + q));
     };
-    int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    int64_t blk = first;
     for (; blk + (U - 1) * step < total; blk += U * step) {
         uint4 v[U][VPB];
 #pragma unroll
@@ -393,6 +362,21 @@ __global__ void __launch_bounds__(kThreads, 4) amax_had16_kernel(const void* __r
         load(blk, v);
         fold(v);
     }
+    return m;
+}
+
+// Tensor amax of the rotated blocks.  Every thread rotates whole 16-element blocks and keeps
+// the largest unnormalized magnitude; the factor 1/4 is applied once to the maximum, which
+// gives the maximum of the normalized values because RN(a/4) is non-decreasing in a and
+// |RN(v/4)| = RN(|v|/4).  The raw 16-byte vectors of several blocks (eight loads for bf16,
+// the same bytes for fp32) are issued before any of them is converted, so the registers hold
+// the loads in flight rather than unpacked pairs.
+template <int IN>
+__global__ void __launch_bounds__(kThreads, 4) amax_had16_kernel(const void* __restrict__ xv, int64_t rows,
+                                                              int64_t cols, int64_t ld, uint32_t* __restrict__ ws,
+                                                              float* __restrict__ gscale, int publish) {
+    const uint32_t m = amax_had16_partial<IN>(xv, rows, cols, ld, (int64_t)blockIdx.x * blockDim.x + threadIdx.x,
+                                              (int64_t)gridDim.x * blockDim.x);
     amax_finish(m, 0.25f, ws, gscale, publish);
 }
 
@@ -455,51 +439,22 @@ __device__ __forceinline__ float zero_scale_error(const u64 (&xp)[8], const u64 
 }
 
 // ------------------------------------------------------------------------------------------
-// NVFP4: AbsMax / 4-over-6 / ScaleSweep MSE [-3,+7] / ScaleSweep WMSE [-8,+7].
-// One thread owns one 16-element block and keeps it in registers for the whole candidate
-// search; one block per thread (no grid-stride tail).  The zero scale, which only enters
-// the window of tiny blocks, is scored once before the candidate loop so the loop is
-// branch-free.  The status word depends only on S, so CTA 0 writes it.
-// ScaleSweep (gist.science/ko/paper/2606.07618), Methodology; 4/6: Adaptive Block-Scaled
-// Data Types (gist.science/ko/paper/2603.28765), Problem.
+// NVFP4: AbsMax / 4-over-6 / ScaleSweep MSE [-3,+7] / ScaleSweep WMSE [-8,+7] of one block.
+// The block stays in registers for the whole candidate search.  The zero scale, which only
+// enters the window of tiny blocks, is scored before the candidate loop so the loop is
+// branch-free.  ScaleSweep (gist.science/ko/paper/2606.07618), Methodology; 4/6: Adaptive
+// Block-Scaled Data Types (gist.science/ko/paper/2603.28765), Problem.
 // ------------------------------------------------------------------------------------------
-template <int IN, int OBJ, bool HAD, typename IDX>
-__global__ void __launch_bounds__(kThreads, OBJ == FP4Q_SWEEP_WMSE ? 4 : FP4Q_SWEEP_MIN_CTAS)
-    quant16_kernel(const void* __restrict__ xv, IDX rows, IDX cols, IDX ld, const float* __restrict__ imp,
-                   uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, const float* __restrict__ gscale,
-                   uint32_t* __restrict__ ws) {
+template <int OBJ, bool HAD>
+__device__ __forceinline__ void nvfp4_block(u64 (&xp)[8], const float* __restrict__ imp, int64_t colblk, float S,
+                                            float d6, float d4, const float2* tab, uint2* cdst, uint8_t* sdst) {
     constexpr bool SWEEP = OBJ == FP4Q_SWEEP_MSE || OBJ == FP4Q_SWEEP_WMSE;
     constexpr bool WEIGHTED = OBJ == FP4Q_SWEEP_WMSE;
     constexpr int LO = WEIGHTED ? -8 : -3, HI = 7;
-    __shared__ float2 s_tab[kTabLen];
-    const IDX nb = cols / 16;
-    const IDX total = rows * nb;
-    const IDX blk = (IDX)blockIdx.x * blockDim.x + threadIdx.x;
-    const bool live = blk < total;
-    const BlockAt<IDX> at = block_at<IDX, WEIGHTED>(live ? blk : 0, cols, ld, nb);
-    // bf16 blocks (8 registers) are loaded before S and the table so the load latency overlaps
-    // them; fp32 blocks (16 registers) would not fit the register cap across the table build
-    RawBlock16<IN> rb;
-    if (IN == FP4Q_IN_BF16 && live) load_raw16<IN>(xv, at.xoff, rb);
-    const Setup su = read_setup(gscale);
-    if (blockIdx.x == 0 && threadIdx.x == 0) ws[WS_STATUS] = su.flags;
-    build_scale_table(su.S, s_tab);
-    const float2* tab = s_tab + kTabPad;
-    const float S = su.S;
-    const float d6 = __fmul_rn(6.0f, S), d4 = __fmul_rn(4.0f, S);
-    if (!live) return;
-    uint2* cdst = reinterpret_cast<uint2*>(codes + at.coff);
-    if (su.flags) {   // data out of contract: zero-filled outputs
-        *cdst = make_uint2(0u, 0u);
-        scales[blk] = 0;
-        return;
-    }
-    u64 xp[8], wp[8];
-    if (IN != FP4Q_IN_BF16) load_raw16<IN>(xv, at.xoff, rb);
-    unpack16<IN>(rb, xp);
+    u64 wp[8];
     if (HAD) fwht16(xp);
     if (WEIGHTED) {
-        const float4* w4 = reinterpret_cast<const float4*>(imp + (int64_t)at.b * 16);
+        const float4* w4 = reinterpret_cast<const float4*>(imp + colblk * 16);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const float4 v = __ldg(w4 + j);
@@ -541,47 +496,19 @@ __global__ void __launch_bounds__(kThreads, OBJ == FP4Q_SWEEP_WMSE ? 4 : FP4Q_SW
         }
     }
     *cdst = block_codes(xp, tab[bp].x);
-    scales[blk] = (uint8_t)bp;
+    *sdst = (uint8_t)bp;
 }
 
 // ------------------------------------------------------------------------------------------
-// IF4: per block, FP4 (E2M1) vs scaled INT4 at the shared AbsMax scale, lower error kept,
+// IF4 of one block: FP4 (E2M1) vs scaled INT4 at the shared AbsMax scale, lower error kept,
 // indicator in bit 7 of the scale byte.  Adaptive Block-Scaled Data Types
 // (gist.science/ko/paper/2603.28765), Methodology, IF4 structure and the 6/7 method.
 // Both errors are in units of the shared scale: FP4 r = RN(q - y); INT4 z = RN(y RN(7/6)),
 // n = clamp(rint(z), -7, 7), r = RN(RN(n RN(6/7)) - y).
 // ------------------------------------------------------------------------------------------
-template <int IN, bool HAD, typename IDX>
-__global__ void __launch_bounds__(kThreads, FP4Q_IF4_MIN_CTAS)
-    if4_kernel(const void* __restrict__ xv, IDX rows, IDX cols, IDX ld, uint8_t* __restrict__ codes,
-               uint8_t* __restrict__ scales, const float* __restrict__ gscale, uint32_t* __restrict__ ws) {
-    __shared__ float2 s_tab[kTabLen];
-    const IDX nb = cols / 16;
-    const IDX total = rows * nb;
-    const IDX blk = (IDX)blockIdx.x * blockDim.x + threadIdx.x;
-    const bool live = blk < total;
-    const BlockAt<IDX> at = block_at<IDX, false>(live ? blk : 0, cols, ld, nb);
-    // bf16 blocks (8 registers) are loaded before S and the table so the load latency overlaps
-    // them; fp32 blocks (16 registers) would not fit the register cap across the table build
-    RawBlock16<IN> rb;
-    if (IN == FP4Q_IN_BF16 && live) load_raw16<IN>(xv, at.xoff, rb);
-    const Setup su = read_setup(gscale);
-    if (blockIdx.x == 0 && threadIdx.x == 0) ws[WS_STATUS] = su.flags;
-    build_scale_table(su.S, s_tab);
-    const float2* tab = s_tab + kTabPad;
-    const float S = su.S;
-    const float d6 = __fmul_rn(6.0f, S);
-    const float K76 = __fdiv_rn(7.0f, 6.0f), K67 = __fdiv_rn(6.0f, 7.0f);
-    if (!live) return;
-    uint2* cdst = reinterpret_cast<uint2*>(codes + at.coff);
-    if (su.flags) {
-        *cdst = make_uint2(0u, 0u);
-        scales[blk] = 0;
-        return;
-    }
-    u64 xp[8];
-    if (IN != FP4Q_IN_BF16) load_raw16<IN>(xv, at.xoff, rb);
-    unpack16<IN>(rb, xp);
+template <bool HAD>
+__device__ __forceinline__ void if4_block(u64 (&xp)[8], float S, float d6, float K76, float K67, const float2* tab,
+                                          uint2* cdst, uint8_t* sdst) {
     if (HAD) fwht16(xp);
     const int p0 = S > 0.0f ? e4m3_rne(__fdiv_rn(block_absmax(xp), d6)) : 0;
     const float inv = tab[p0].x;
@@ -615,7 +542,72 @@ __global__ void __launch_bounds__(kThreads, FP4Q_IF4_MIN_CTAS)
     const uint32_t* cc = use_int ? ci : cf;
     *cdst = make_uint2(cc[0] | (cc[1] << 8) | (cc[2] << 16) | (cc[3] << 24),
                        cc[4] | (cc[5] << 8) | (cc[6] << 16) | (cc[7] << 24));
-    scales[blk] = (uint8_t)(p0 | (use_int ? 0x80 : 0));
+    *sdst = (uint8_t)(p0 | (use_int ? 0x80 : 0));
+}
+
+// ------------------------------------------------------------------------------------------
+// The NVFP4 / IF4 quantize kernel (KIND = the NVFP4 objective, or KIND_IF4).  Each thread
+// walks the blocks tid, tid + G, ... (G threads in the grid) with the next block's loads in
+// flight while the current one is searched; the CTA builds its scale table once.  The host
+// picks the grid per kind: one block per thread (G >= blocks: the loop runs once) for the
+// ScaleSweep searches, one persistent wave for the light IF4 / AbsMax / 4-6 kinds, whose
+// per-CTA start-up (S, table, first loads) would otherwise not be amortized.  The status
+// word depends only on S, so CTA 0 writes it.
+// ------------------------------------------------------------------------------------------
+enum : int { KIND_IF4 = 4 };   // kinds 0..3 are the NVFP4 objectives
+
+template <int KIND>
+__host__ __device__ constexpr bool q16_persistent() {
+    return KIND == KIND_IF4 || KIND == FP4Q_ABSMAX || KIND == FP4Q_FOUR_OVER_SIX ||
+           (KIND == FP4Q_SWEEP_MSE && FP4Q_SWEEP_PERSISTENT);
+}
+template <int KIND>
+__host__ __device__ constexpr int q16_min_ctas() {   // register cap: CTAs per SM the kernel is compiled for
+    return KIND == FP4Q_SWEEP_WMSE ? 4 : (q16_persistent<KIND>() ? FP4Q_PERSIST_MIN_CTAS : FP4Q_SWEEP_MIN_CTAS);
+}
+
+template <int IN, int KIND, bool HAD, typename IDX>
+__global__ void __launch_bounds__(kThreads, q16_min_ctas<KIND>())
+    q16_kernel(const void* __restrict__ xv, IDX rows, IDX cols, IDX ld, const float* __restrict__ imp,
+               uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, const float* __restrict__ gscale,
+               uint32_t* __restrict__ ws) {
+    __shared__ float2 s_tab[kTabLen];
+    const IDX nb = cols / 16;
+    const IDX total = rows * nb;
+    const IDX G = (IDX)gridDim.x * blockDim.x;
+    IDX blk = (IDX)blockIdx.x * blockDim.x + threadIdx.x;
+    // bf16 blocks (8 registers) are loaded before S and the table so the load latency overlaps
+    // them; fp32 blocks (16 registers) would not fit the register cap across the table build
+    RawBlock16<IN> rb;
+    if (IN == FP4Q_IN_BF16 && blk < total) load_raw16<IN>(xv, block_at<IDX, false>(blk, cols, ld, nb).xoff, rb);
+    const float S = *gscale;
+    const uint32_t flags = scale_flags(S);
+    if (blockIdx.x == 0 && threadIdx.x == 0) ws[WS_STATUS] = flags;
+    build_scale_table(S, s_tab);
+    const float2* tab = s_tab + kTabPad;
+    const float d6 = __fmul_rn(6.0f, S), d4 = __fmul_rn(4.0f, S);
+    const float K76 = __fdiv_rn(7.0f, 6.0f), K67 = __fdiv_rn(6.0f, 7.0f);
+    auto one_block = [&](IDX b) {
+        const BlockAt<IDX> at = block_at<IDX, KIND == FP4Q_SWEEP_WMSE>(b, cols, ld, nb);
+        uint2* cdst = reinterpret_cast<uint2*>(codes + at.coff);
+        if (flags) {   // data out of contract: zero-filled outputs
+            *cdst = make_uint2(0u, 0u);
+            scales[b] = 0;
+            return;
+        }
+        if (IN != FP4Q_IN_BF16) load_raw16<IN>(xv, at.xoff, rb);
+        u64 xp[8];
+        unpack16<IN>(rb, xp);
+        if (q16_persistent<KIND>() && IN == FP4Q_IN_BF16 && b + G < total)   // next block's loads in flight
+            load_raw16<IN>(xv, block_at<IDX, false>(b + G, cols, ld, nb).xoff, rb);
+        if (KIND == KIND_IF4) if4_block<HAD>(xp, S, d6, K76, K67, tab, cdst, scales + b);
+        else nvfp4_block<KIND, HAD>(xp, imp, at.b, S, d6, d4, tab, cdst, scales + b);
+    };
+    if (q16_persistent<KIND>()) {
+        for (; blk < total; blk += G) one_block(blk);
+    } else if (blk < total) {
+        one_block(blk);
+    }
 }
 
 // ------------------------------------------------------------------------------------------
@@ -879,30 +871,25 @@ int check_common(const void* x, int dtype, int64_t rows, int64_t cols, int64_t l
     return FP4Q_OK;
 }
 
-// One quantization block per thread; 32-bit index arithmetic when the tensor allows it.
-template <int IN, int OBJ, bool HAD>
+// The NVFP4 / IF4 kernel; 32-bit index arithmetic when the tensor allows it.
+template <int IN, int KIND, bool HAD, typename IDX>
+void launch_q16_as(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* imp, uint8_t* codes,
+                   uint8_t* scales, float* gs, uint32_t* ws, cudaStream_t st) {
+    auto kernel = q16_kernel<IN, KIND, HAD, IDX>;
+    const int64_t total = rows * (cols / 16);
+    const int grid = q16_persistent<KIND>() ? grid_for(kernel, total, q16_min_ctas<KIND>())
+                                            : (int)((total + kThreads - 1) / kThreads);
+    kernel<<<grid, kThreads, 0, st>>>(x, (IDX)rows, (IDX)cols, (IDX)ld, imp, codes, scales, gs, ws);
+}
+
+template <int IN, int KIND, bool HAD>
 void launch_q16(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* imp, uint8_t* codes,
                 uint8_t* scales, float* gs, uint32_t* ws, cudaStream_t st) {
     const int64_t total = rows * (cols / 16);
-    const unsigned ctas = (unsigned)((total + kThreads - 1) / kThreads);
     if (total < ((int64_t)1 << 31) && rows * ld < ((int64_t)1 << 31))
-        quant16_kernel<IN, OBJ, HAD, uint32_t><<<ctas, kThreads, 0, st>>>(
-            x, (uint32_t)rows, (uint32_t)cols, (uint32_t)ld, imp, codes, scales, gs, ws);
+        launch_q16_as<IN, KIND, HAD, uint32_t>(x, rows, cols, ld, imp, codes, scales, gs, ws, st);
     else
-        quant16_kernel<IN, OBJ, HAD, int64_t><<<ctas, kThreads, 0, st>>>(x, rows, cols, ld, imp, codes, scales, gs,
-                                                                         ws);
-}
-
-template <int IN, bool HAD>
-void launch_if4(const void* x, int64_t rows, int64_t cols, int64_t ld, uint8_t* codes, uint8_t* scales, float* gs,
-                uint32_t* ws, cudaStream_t st) {
-    const int64_t total = rows * (cols / 16);
-    const unsigned ctas = (unsigned)((total + kThreads - 1) / kThreads);
-    if (total < ((int64_t)1 << 31) && rows * ld < ((int64_t)1 << 31))
-        if4_kernel<IN, HAD, uint32_t><<<ctas, kThreads, 0, st>>>(x, (uint32_t)rows, (uint32_t)cols, (uint32_t)ld,
-                                                                  codes, scales, gs, ws);
-    else
-        if4_kernel<IN, HAD, int64_t><<<ctas, kThreads, 0, st>>>(x, rows, cols, ld, codes, scales, gs, ws);
+        launch_q16_as<IN, KIND, HAD, int64_t>(x, rows, cols, ld, imp, codes, scales, gs, ws, st);
 }
 
 // Tensor scale pass: plain amax, or the amax of the 16-point rotated blocks.
@@ -922,7 +909,7 @@ template <int IN, bool HAD>
 void launch_nvfp4_if4(const void* x, int64_t rows, int64_t cols, int64_t ld, int fmt, int obj, const float* imp,
                       uint8_t* codes, uint8_t* scales, float* gs, uint32_t* ws, cudaStream_t st) {
     if (fmt == FP4Q_IF4) {
-        launch_if4<IN, HAD>(x, rows, cols, ld, codes, scales, gs, ws, st);
+        launch_q16<IN, KIND_IF4, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, st);
         return;
     }
     switch (obj) {
@@ -930,9 +917,7 @@ void launch_nvfp4_if4(const void* x, int64_t rows, int64_t cols, int64_t ld, int
         case FP4Q_FOUR_OVER_SIX:
             launch_q16<IN, FP4Q_FOUR_OVER_SIX, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, st);
             break;
-        case FP4Q_SWEEP_MSE:
-            launch_q16<IN, FP4Q_SWEEP_MSE, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, st);
-            break;
+        case FP4Q_SWEEP_MSE: launch_q16<IN, FP4Q_SWEEP_MSE, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, st); break;
         default:   // WMSE is rejected with the rotation before any launch
             if (!HAD) launch_q16<IN, FP4Q_SWEEP_WMSE, false>(x, rows, cols, ld, imp, codes, scales, gs, ws, st);
             break;
@@ -942,7 +927,6 @@ void launch_nvfp4_if4(const void* x, int64_t rows, int64_t cols, int64_t ld, int
 template <int IN>
 int launch_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, int fmt, int obj, const float* imp,
                     uint8_t* codes, uint8_t* scales, float* gs, uint32_t* ws, uint32_t flags, cudaStream_t st) {
-    int n = 0;
     if (fmt == FP4Q_MXFP4) {
         const int ocp = (flags & FP4Q_F_MX_OCP_FLOOR) ? 1 : 0;
         if (flags & FP4Q_F_HADAMARD32)
@@ -954,6 +938,7 @@ int launch_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, int f
         return launched(1);
     }
     const bool had16 = (flags & FP4Q_F_HADAMARD16) != 0;
+    int n = 0;
     if (!(flags & FP4Q_F_GLOBAL_SCALE_GIVEN)) {
         launch_amax<IN>(x, rows, cols, ld, ws, gs, 0, had16, st);
         ++n;
