@@ -44,7 +44,7 @@ namespace fp4q {
 #define FP4Q_SWEEP_UNROLL 11    // MSE candidate-loop unroll factor (11 = the whole window)
 #endif
 #ifndef FP4Q_WMSE_UNROLL
-#define FP4Q_WMSE_UNROLL 1      // WMSE candidate-loop unroll factor
+#define FP4Q_WMSE_UNROLL 16     // WMSE candidate-loop unroll factor (16 = the whole window)
 #endif
 constexpr int kMseUnroll = FP4Q_SWEEP_UNROLL, kWmseUnroll = FP4Q_WMSE_UNROLL;
 
