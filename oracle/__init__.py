@@ -61,7 +61,9 @@ def lib():
         L.fp4q_o_if4_quantize.restype = C.c_int
         L.fp4q_o_if4_quantize.argtypes = [P, i64, i64, i64, C.c_int, P, P, P, P, P]
         L.fp4q_o_mxfp4_quantize.restype = C.c_int
-        L.fp4q_o_mxfp4_quantize.argtypes = [P, i64, i64, i64, C.c_int, C.c_int, P, P]
+        L.fp4q_o_mxfp4_quantize.argtypes = [P, i64, i64, i64, C.c_int, C.c_int, C.c_int, P, P]
+        L.fp4q_o_mx_block_errors.restype = C.c_int
+        L.fp4q_o_mx_block_errors.argtypes = [P, i64, i64, i64, C.c_int, P, P]
         L.fp4q_o_dequantize.restype = C.c_int
         L.fp4q_o_dequantize.argtypes = [P, P, C.c_float, i64, i64, C.c_int, C.c_int, P, C.c_int]
         _lib = L
@@ -176,16 +178,32 @@ def if4_quantize(x, S=None, hadamard16=False):
             "err_fp": ef, "err_int": ei}
 
 
-def mxfp4_quantize(x, hadamard=False, ocp_floor=False):
+MX_SWEEP = {"rule": 0, "sweep": 1, "brute": 2}
+
+
+def mxfp4_quantize(x, hadamard=False, ocp_floor=False, sweep="rule"):
+    """MXFP4 codes and E8M0 scale bytes.  sweep: "rule" (the max rule, ceil or OCP floor),
+    "sweep" (the MX scale sweep over e_c - 2 .. e_c), "brute" (every exponent)."""
     x = _f32(x)
     rows, cols = x.shape
     codes = np.zeros((rows, cols // 2), np.uint8)
     scales = np.zeros((rows, cols // 32), np.uint8)
-    st = lib().fp4q_o_mxfp4_quantize(_p(x), rows, cols, cols, int(hadamard), int(ocp_floor), _p(codes),
-                                     _p(scales))
+    st = lib().fp4q_o_mxfp4_quantize(_p(x), rows, cols, cols, int(hadamard), int(ocp_floor), MX_SWEEP[sweep],
+                                     _p(codes), _p(scales))
     if st < 0:
         raise ValueError("oracle: bad shape")
     return {"codes": codes, "scales": scales, "status": st}
+
+
+def mx_block_errors(x, scales, hadamard=False):
+    """Per-block error E (units of 4^e) of MXFP4 blocks at the exponents of `scales`."""
+    x = _f32(x)
+    rows, cols = x.shape
+    scales = np.ascontiguousarray(scales, np.uint8)
+    err = np.zeros((rows, cols // 32), np.float32)
+    if lib().fp4q_o_mx_block_errors(_p(x), rows, cols, cols, int(hadamard), _p(scales), _p(err)) < 0:
+        raise ValueError("oracle: bad shape")
+    return err
 
 
 def dequantize(codes, scales, S, fmt, inverse_hadamard=False, out_bf16=False):

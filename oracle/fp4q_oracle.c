@@ -47,6 +47,9 @@
  *            E_int < E_fp.
  *   MXFP4  = e = smallest integer with a_b <= 6*2^e (clamped to [-127,127]), byte e+127,
  *            y = RN(x * 2^-e), q = E2M1(y), dequant q*2^e.
+ *   MX sweep = e among e_c - 2 .. e_c (e_c the rule above) minimizing RN(E * 4^(e - e_c)),
+ *            E = RN(acc_even + acc_odd) of fma(r, r, acc), r = RN(q - y) at that e; lowest e
+ *            wins a tie.
  *   Hadamard(32) = Sylvester fast Walsh-Hadamard butterflies for h = 1,2,4,8,16
  *            (v_j, v_j+h) <- (RN(v_j + v_j+h), RN(v_j - v_j+h)), then RN(v * RN(1/sqrt(32))).
  *   dequant NVFP4 x^ = RN(q * sv); IF4-INT4 x^ = RN(RN(n*RN(6/7)) * sv); MXFP4 x^ = RN(q*2^e).
@@ -409,8 +412,72 @@ int fp4q_o_mx_exponent(float a, int ocp_floor)
     return e;
 }
 
+/* MX scale sweep [MR] ("Scale Fitting" for MXFP4: the page fits the power-of-two scale grid
+ * to the data to cut the error that E8M0's coarse, over-wide grid causes, without giving the
+ * rule; the plainest reading is ScaleSweep's search carried over to E8M0).  Error of one
+ * 32-element block at scale 2^e, in units of 4^e: y = RN(x*2^-e), q = E2M1(y), r = RN(q - y),
+ * E = RN(acc_even + acc_odd) with acc = fma(r, r, acc) over the even / odd positions in order,
+ * as for NVFP4.  Multiplying by 2^-e is exact for normal results, so r is the rounding error
+ * of the block in units of the scale. */
+static float mx_block_error(const float* v, int e)
+{
+    const float m = ldexpf(1.0f, -e);
+    float acc[2] = {0.0f, 0.0f};
+    for (int i = 0; i < 32; ++i) {
+        float y = v[i] * m;
+        float q = fp4q_o_e2m1_value(fp4q_o_e2m1_encode(y));
+        float r = q - y;
+        acc[i & 1] = fmaf(r, r, acc[i & 1]);
+    }
+    return acc[0] + acc[1];
+}
+
+/* Exponent of one block under mode: 0 the max rule (ceil, or OCP floor with ocp_floor);
+ * 1 the sweep over e_c + k, k = -2..0, e_c = the ceil rule, patterns below -127 skipped,
+ * comparing RN(E_k * 4^k) (the block error in units of 4^e_c; the power-of-two factor is
+ * exact) lexicographically with the lowest k winning a tie;
+ * 2 brute force over every e in [-127, 127] on the reconstruction error itself,
+ * sum (x - q * 2^e)^2 accumulated in double (each term exact), lowest e winning a tie (checks
+ * that the window of mode 1 holds the optimum; away from the window the scaled error of
+ * mode 1 would underflow, the absolute one does not). */
+static double mx_block_abs_error(const float* v, int e)
+{
+    const float m = ldexpf(1.0f, -e);
+    double err = 0.0;
+    for (int i = 0; i < 32; ++i) {
+        double d = (double)v[i] - ldexp((double)fp4q_o_e2m1_value(fp4q_o_e2m1_encode(v[i] * m)), e);
+        err += d * d;
+    }
+    return err;
+}
+
+static int mx_block_exponent(const float* v, float ab, int ocp_floor, int mode)
+{
+    const int ec = fp4q_o_mx_exponent(ab, 0);
+    if (mode == 0) return ocp_floor ? fp4q_o_mx_exponent(ab, 1) : ec;
+    if (mode == 1) {
+        int be = ec + (ec - 2 < -127 ? -127 - ec : -2);   /* the first candidate */
+        float best = INFINITY;
+        for (int k = -2; k <= 0; ++k) {
+            if (ec + k < -127) continue;
+            float err = mx_block_error(v, ec + k) * ldexpf(1.0f, 2 * k);
+            if (err < best) { best = err; be = ec + k; }
+        }
+        return be;
+    }
+    int be = -127;
+    double best = INFINITY;
+    for (int e = -127; e <= 127; ++e) {
+        double err = mx_block_abs_error(v, e);
+        if (err < best) { best = err; be = e; }
+    }
+    return be;
+}
+
+/* sweep: 0 the max rule, 1 the MX scale sweep (window [-2, 0]), 2 brute force over all
+ * exponents; ocp_floor applies to sweep = 0 only. */
 int fp4q_o_mxfp4_quantize(const float* x, int64_t rows, int64_t cols, int64_t ld,
-                          int hadamard, int ocp_floor, uint8_t* codes, uint8_t* scales)
+                          int hadamard, int ocp_floor, int sweep, uint8_t* codes, uint8_t* scales)
 {
     const int B = 32;
     if (cols % B) return -1;
@@ -432,7 +499,7 @@ int fp4q_o_mxfp4_quantize(const float* x, int64_t rows, int64_t cols, int64_t ld
             if (hadamard) fp4q_o_hadamard32(v);
             float ab = 0.0f;
             for (int i = 0; i < B; ++i) ab = fmaxf(ab, fabsf(v[i]));
-            int e = fp4q_o_mx_exponent(ab, ocp_floor);
+            int e = mx_block_exponent(v, ab, ocp_floor, sweep);
             float m = ldexpf(1.0f, -e);   /* exact power of two (subnormal for e = 127) */
             for (int i = 0; i < B; i += 2) {
                 int lo = fp4q_o_e2m1_encode(v[i] * m), hi = fp4q_o_e2m1_encode(v[i + 1] * m);
@@ -442,6 +509,23 @@ int fp4q_o_mxfp4_quantize(const float* x, int64_t rows, int64_t cols, int64_t ld
         }
     }
     return status;
+}
+
+/* Block errors of MXFP4 blocks (after the optional rotation) at the exponents given by the
+ * scale bytes, in units of 4^e: the E of mx_block_error.  Returns -1 on a bad shape. */
+int fp4q_o_mx_block_errors(const float* x, int64_t rows, int64_t cols, int64_t ld, int hadamard,
+                           const uint8_t* scales, float* err)
+{
+    if (cols % 32) return -1;
+    const int64_t nb = cols / 32;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t b = 0; b < nb; ++b) {
+            float v[32];
+            memcpy(v, x + r * ld + b * 32, sizeof v);
+            if (hadamard) fp4q_o_hadamard32(v);
+            err[r * nb + b] = mx_block_error(v, (int)scales[r * nb + b] - 127);
+        }
+    return 0;
 }
 
 /* ------------------------------------------------------------------------------------

@@ -316,6 +316,66 @@ def test_mx_exponent_closed_form():
     assert O.mx_exponent(0.0) == -127
 
 
+def _mx_blocks(seed, n):
+    """Blocks of 32 from several distributions: Laplace with per-channel scales (the activation
+    workload's shape), Gaussian, exact E2M1 grid values times a power of two, and blocks with one
+    large outlier."""
+    rng = np.random.default_rng(seed)
+    lap = rng.laplace(size=(n, 32)) * np.exp(rng.normal(0, 1.5, size=(1, 32)))
+    gau = rng.normal(size=(n, 32))
+    grid = rng.choice(GRID, size=(n, 32)) * rng.choice([-1.0, 1.0], size=(n, 32)) * 2.0 ** rng.integers(-4, 5, (n, 1))
+    out = rng.normal(size=(n, 32)) * 0.1
+    out[:, 0] = rng.uniform(3, 40, n)
+    return np.concatenate([lap, gau, grid, out]).astype(np.float32)
+
+
+def test_mx_sweep_never_prefers_a_larger_exponent():
+    # Above the max rule e_c every |x| <= 6*2^e_c, and the grid at 2^(e_c+1) restricted to
+    # [0, 6*2^e_c] is {0,1,2,3,4,6}*2^e_c, a subset of the grid at 2^e_c: a larger scale can only
+    # tie.  The brute-force optimum over all 255 exponents therefore never exceeds e_c.
+    x = _mx_blocks(11, 500)
+    rule = O.mxfp4_quantize(x, sweep="rule")["scales"].astype(int)
+    brute = O.mxfp4_quantize(x, sweep="brute")["scales"].astype(int)
+    assert (brute <= rule).all()
+
+
+@pytest.mark.parametrize("had", [False, True])
+def test_mx_sweep_window_holds_the_optimum(had):
+    # The window [e_c - 2, e_c] against the brute force over every exponent (exact float64 errors),
+    # on config-shaped activations (Laplace, lognormal(0,1.5) channel std, outlier channels x100)
+    # and on the synthetic mixtures: the optimum is always inside, and the sweep picks it except
+    # where the two best candidates are within binary32 rounding of each other.
+    w = synth.make("cfg5", rows=64, cols=8192)
+    x = np.concatenate([O.widen_bf16(w["x"]).reshape(-1, 32), _mx_blocks(12, 300)])
+    rule = O.mxfp4_quantize(x, hadamard=had, sweep="rule")["scales"].astype(int)
+    sw = O.mxfp4_quantize(x, hadamard=had, sweep="sweep")["scales"].astype(int)
+    brute = O.mxfp4_quantize(x, hadamard=had, sweep="brute")["scales"].astype(int)
+    assert ((brute >= rule - 2) & (brute <= rule)).all()
+    assert ((sw >= rule - 2) & (sw <= rule)).all()
+    diff = np.nonzero((sw != brute).ravel())[0]
+    assert len(diff) <= 1e-3 * sw.size
+    if len(diff):
+        e_sw = O.mx_block_errors(x, (sw.reshape(-1, 1) + 127).astype(np.uint8), had).ravel().astype(np.float64)
+        e_bf = O.mx_block_errors(x, (brute.reshape(-1, 1) + 127).astype(np.uint8), had).ravel().astype(np.float64)
+        a = e_sw[diff] * 4.0 ** (sw.ravel()[diff] - rule.ravel()[diff])
+        b = e_bf[diff] * 4.0 ** (brute.ravel()[diff] - rule.ravel()[diff])
+        assert (np.abs(a - b) <= 1e-5 * np.maximum(a, b)).all()
+
+
+def test_mx_sweep_error_never_above_either_rule():
+    x = _mx_blocks(13, 500)
+    sw = O.mxfp4_quantize(x, sweep="sweep")["scales"]
+    for ocp in (False, True):
+        ru = O.mxfp4_quantize(x, sweep="rule", ocp_floor=ocp)["scales"]
+        # compare the exact reconstruction errors of the two choices, from the dequantized values
+        xs = O.dequantize(O.mxfp4_quantize(x, sweep="sweep")["codes"], sw, 0.0, "mxfp4").astype(np.float64)
+        xr = O.dequantize(O.mxfp4_quantize(x, sweep="rule", ocp_floor=ocp)["codes"], ru, 0.0, "mxfp4").astype(np.float64)
+        es = ((x.astype(np.float64) - xs) ** 2).sum(1)
+        er = ((x.astype(np.float64) - xr) ** 2).sum(1)
+        assert (es <= er * (1 + 1e-6) + 1e-30).all()
+        assert (es < er).any()
+
+
 def test_hadamard_is_normalized_sylvester():
     H = np.array([[1.0]])
     while H.shape[0] < 32:
@@ -441,7 +501,8 @@ def _parse_golden():
 def test_hand_worked(row):
     _, method, S, xb, scale, expect = row
     if method.startswith("mxfp4"):
-        r = O.mxfp4_quantize(xb.reshape(1, -1), ocp_floor=method.endswith("ocp"))
+        r = O.mxfp4_quantize(xb.reshape(1, -1), ocp_floor=method.endswith("ocp"),
+                             sweep="sweep" if method.endswith("sweep") else "rule")
         assert r["scales"][0, 0] == scale
         xh = O.dequantize(r["codes"], r["scales"], 0.0, "mxfp4")
         assert np.array_equal(xh[0], expect)
