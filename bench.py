@@ -36,6 +36,10 @@ WORKLOADS = {
     "cfg4": ("cfg4", "if4", None, "IF4 per-block FP4/INT4 selection, bf16 weight 4096x14336, 0.02*t4"),
     "cfg5": ("cfg5", "mxfp4", None, "MXFP4, bf16 activations 16384x8192"),
     "cfg5h": ("cfg5", "mxfp4_had", None, "MXFP4 after 32x32 block Hadamard, bf16 activations 16384x8192"),
+    "cfg5s": ("cfg5", "mxfp4", "mx_sweep",
+              "MXFP4 with the MX scale sweep (E8M0 exponents e_c-2..e_c by block MSE), bf16 activations 16384x8192"),
+    "cfg5hs": ("cfg5", "mxfp4_had", "mx_sweep",
+               "MXFP4 with the MX scale sweep after 32x32 block Hadamard, bf16 activations 16384x8192"),
     "cfg3h": ("cfg3", "nvfp4_had", "sweep_mse",
               "NVFP4 ScaleSweep-MSE on 16x16 block-Hadamard-rotated blocks, bf16 activations 8192x4096, "
               "dynamic S of the rotated tensor"),
@@ -176,7 +180,7 @@ def cpu_baseline(w, fmt, obj, budget_s=12.0):
         elif base == "if4":
             O.if4_quantize(xs, hadamard16=had16)
         else:
-            O.mxfp4_quantize(xs, hadamard=fmt.endswith("had"))
+            O.mxfp4_quantize(xs, hadamard=fmt.endswith("had"), sweep="sweep" if obj == "mx_sweep" else "rule")
         done += xs.shape[0]
     dt = time.perf_counter() - t0
     nbytes = algorithmic_bytes(done, cols, fmt, wmse=(obj == "sweep_wmse"))
@@ -207,7 +211,7 @@ def run_reference(args, rank, world):
         elif base == "if4":
             O.if4_quantize(xs, hadamard16=had16)
         else:
-            O.mxfp4_quantize(xs, hadamard=fmt.endswith("had"))
+            O.mxfp4_quantize(xs, hadamard=fmt.endswith("had"), sweep="sweep" if obj == "mx_sweep" else "rule")
 
     for i in range(args.warmup):
         step(i)
@@ -263,9 +267,9 @@ def run_ours(args, rank, world):
         c, sc, g = outs[s]
         if fmt.startswith("mxfp4"):   # one kernel, no tensor scale
             if fmt.endswith("had"):
-                fq.hadamard_quantize(xs[s], out=(c, sc, None), workspace=ws)
+                fq.hadamard_quantize(xs[s], out=(c, sc, None), workspace=ws, mx_sweep=(obj == "mx_sweep"))
             else:
-                fq.quantize(xs[s], "mxfp4", out=(c, sc, None), workspace=ws)
+                fq.quantize(xs[s], "mxfp4", out=(c, sc, None), workspace=ws, mx_sweep=(obj == "mx_sweep"))
         else:
             fq.quantize(xs[s], base, obj or "absmax", importance=imp, global_scale=g, out=(c, sc, g), workspace=ws,
                         hadamard16=had16)
@@ -352,7 +356,7 @@ def run_ours(args, rank, world):
     e2e_steps = max(1, min(args.steps, 50))
     x_pin = x_host.pin_memory()
     hq = fq.HostQuantizer(rows, cols, fmt, obj or "absmax", importance=imp, dtype=x_host.dtype, depth=2,
-                          device=dev)
+                          device=dev, mx_sweep=(obj == "mx_sweep"))
     host_outs = [fq.alloc_host_outputs(rows, cols, fmt) for _ in range(2)]
     for i in range(3):
         hq(x_pin, host_outs[i % 2])

@@ -656,7 +656,40 @@ __device__ __forceinline__ int mx_exponent(float a, bool ocp) {
     return min(max(e, -127), 127);
 }
 
-template <int IN, bool HAD>
+// MX scale sweep of one 32-element block (pairs vp): the exponent among e_c - 2 .. e_c with
+// the lowest block error, e_c the ceil rule.  Error at e in units of 4^e: r = RN(q - y) with
+// y = RN(x 2^-e), q = E2M1(y), E = RN(acc_even + acc_odd) of fma(r, r, acc); candidates are
+// compared on RN(E 4^(e - e_c)) (an exact power-of-two factor) in increasing e, strict
+// improvement, so the lowest exponent wins a tie.  Exponents below -127 are not candidates.
+// Bridging the Gap ... Microscaling FP4 (gist.science/ko/paper/2509.23202), Methodology:
+// MXFP4 "Scale Fitting" of the power-of-two scale grid to the data.
+__device__ __forceinline__ int mx_sweep_exponent(const u64 (&vp)[16], int ec) {
+    int be = max(ec - 2, -127);
+    float best = INFINITY;
+#pragma unroll
+    for (int k = -2; k <= 0; ++k) {
+        const int e = ec + k;
+        if (e < -127) continue;
+        const float m = pow2i(-e);
+        const u64 m2 = pk(m, m);
+        u64 acc = pk(0.0f, 0.0f);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const u64 r = e2m1x2_residual2(mul2(vp[j], m2));
+            acc = fma2(r, r, acc);
+        }
+        float a, b;
+        upk(acc, a, b);
+        const float err = __fmul_rn(__fadd_rn(a, b), k == -2 ? 0.0625f : (k == -1 ? 0.25f : 1.0f));
+        if (err < best) {
+            best = err;
+            be = e;
+        }
+    }
+    return be;
+}
+
+template <int IN, bool HAD, bool SWEEP>
 __global__ void __launch_bounds__(kThreads) mxfp4_kernel(const void* __restrict__ xv, int64_t rows, int64_t cols,
                                                          int64_t ld, uint8_t* __restrict__ codes,
                                                          uint8_t* __restrict__ scales, uint32_t* __restrict__ ws,
@@ -702,7 +735,15 @@ __global__ void __launch_bounds__(kThreads) mxfp4_kernel(const void* __restrict_
         float ab = 0.0f;
 #pragma unroll
         for (int i = 0; i < 32; ++i) ab = fmaxf(ab, fabsf(v[i]));
-        const int e = mx_exponent(ab, ocp != 0);
+        int e;
+        if (SWEEP) {
+            u64 vp[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) vp[j] = pk(v[2 * j], v[2 * j + 1]);
+            e = mx_sweep_exponent(vp, mx_exponent(ab, false));
+        } else {
+            e = mx_exponent(ab, ocp != 0);
+        }
         const float m = pow2i(-e);
         uint32_t c[16];
 #pragma unroll
@@ -929,11 +970,19 @@ int launch_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, int f
                     uint8_t* codes, uint8_t* scales, float* gs, uint32_t* ws, uint32_t flags, cudaStream_t st) {
     if (fmt == FP4Q_MXFP4) {
         const int ocp = (flags & FP4Q_F_MX_OCP_FLOOR) ? 1 : 0;
-        if (flags & FP4Q_F_HADAMARD32)
-            mxfp4_kernel<IN, true><<<grid_for(mxfp4_kernel<IN, true>, rows * (cols / 32), 8), kThreads, 0, st>>>(
+        const bool had = (flags & FP4Q_F_HADAMARD32) != 0, sweep = (flags & FP4Q_F_MX_SWEEP) != 0;
+        const int64_t nblk = rows * (cols / 32);
+        if (had && sweep)
+            mxfp4_kernel<IN, true, true><<<grid_for(mxfp4_kernel<IN, true, true>, nblk, 8), kThreads, 0, st>>>(
+                x, rows, cols, ld, codes, scales, ws, ocp);
+        else if (had)
+            mxfp4_kernel<IN, true, false><<<grid_for(mxfp4_kernel<IN, true, false>, nblk, 8), kThreads, 0, st>>>(
+                x, rows, cols, ld, codes, scales, ws, ocp);
+        else if (sweep)
+            mxfp4_kernel<IN, false, true><<<grid_for(mxfp4_kernel<IN, false, true>, nblk, 8), kThreads, 0, st>>>(
                 x, rows, cols, ld, codes, scales, ws, ocp);
         else
-            mxfp4_kernel<IN, false><<<grid_for(mxfp4_kernel<IN, false>, rows * (cols / 32), 8), kThreads, 0, st>>>(
+            mxfp4_kernel<IN, false, false><<<grid_for(mxfp4_kernel<IN, false, false>, nblk, 8), kThreads, 0, st>>>(
                 x, rows, cols, ld, codes, scales, ws, ocp);
         return launched(1);
     }
@@ -987,8 +1036,11 @@ void launch_dequant16(const uint8_t* codes, const uint8_t* scales, const float* 
 // Format, objective and flag checks shared by fp4q_quantize and fp4q_quantize_noalloc.
 int check_quantize_args(int fmt, int objective, uint32_t flags) {
     if (fmt != FP4Q_NVFP4 && fmt != FP4Q_IF4 && fmt != FP4Q_MXFP4) return FP4Q_ERR_INVALID_ARG;
-    if (flags & ~(FP4Q_F_GLOBAL_SCALE_GIVEN | FP4Q_F_MX_OCP_FLOOR | FP4Q_F_HADAMARD16 | FP4Q_F_HADAMARD32))
+    if (flags & ~(FP4Q_F_GLOBAL_SCALE_GIVEN | FP4Q_F_MX_OCP_FLOOR | FP4Q_F_HADAMARD16 | FP4Q_F_HADAMARD32 |
+                  FP4Q_F_MX_SWEEP))
         return FP4Q_ERR_INVALID_ARG;
+    if ((flags & FP4Q_F_MX_SWEEP) && (flags & FP4Q_F_MX_OCP_FLOOR)) return FP4Q_ERR_INVALID_ARG;
+    if ((flags & FP4Q_F_MX_SWEEP) && fmt != FP4Q_MXFP4) return FP4Q_ERR_UNSUPPORTED;
     if (fmt == FP4Q_NVFP4 && (objective < FP4Q_ABSMAX || objective > FP4Q_SWEEP_WMSE)) return FP4Q_ERR_INVALID_ARG;
     if (fmt == FP4Q_MXFP4 && (flags & FP4Q_F_GLOBAL_SCALE_GIVEN)) return FP4Q_ERR_INVALID_ARG;
     if (flags & FP4Q_F_HADAMARD16) {
@@ -1071,7 +1123,7 @@ int fp4q_hadamard_quantize(const void* x, int dtype, int64_t rows, int64_t cols,
                            uint8_t* codes, uint8_t* scales, void* workspace, uint32_t flags, void* stream) {
     g_launches = 0;
     if (had_size != 32) return FP4Q_ERR_UNSUPPORTED;
-    if (flags & ~FP4Q_F_MX_OCP_FLOOR) return FP4Q_ERR_INVALID_ARG;
+    if (flags & ~(FP4Q_F_MX_OCP_FLOOR | FP4Q_F_MX_SWEEP)) return FP4Q_ERR_INVALID_ARG;
     return fp4q_quantize(x, dtype, rows, cols, ld, FP4Q_MXFP4, 0, nullptr, codes, scales, nullptr, workspace,
                          flags | FP4Q_F_HADAMARD32, stream);
 }

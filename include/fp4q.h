@@ -31,6 +31,12 @@
  *   r = RN(v - y); both paths share s, so INT4 iff E_int < E_fp.
  *   MXFP4: e = smallest integer with a_b <= 6 * 2^e (flag FP4Q_F_MX_OCP_FLOOR: floor(log2
  *   a_b) - 2), clamped to [-127,127]; y = RN(x 2^-e).
+ *   MX scale sweep (flag FP4Q_F_MX_SWEEP): e among e_c - 2 .. e_c (e_c the ceil rule, none
+ *   below -127) minimizing RN(E 4^(e - e_c)), E = RN(acc_even + acc_odd) of fma(r, r, acc),
+ *   r = RN(q - y) at that e; the lowest e wins a tie.  Bridging the Gap ... Microscaling FP4,
+ *   "Methodology": MXFP4 "Scale Fitting" of the power-of-two grid to the data, read as
+ *   ScaleSweep's block-MSE search over E8M0 neighbours; exponents above e_c can only tie (the
+ *   grid at 2^(e_c+1) below 6*2^e_c is a subset of the grid at 2^e_c).
  *
  * Memory layout (all device memory, row-major, owned and allocated by the caller):
  *   x        [rows][ld] bf16 or fp32; ld >= cols elements; x and the row pitch (ld * element
@@ -85,6 +91,10 @@ enum { FP4Q_ABSMAX = 0, FP4Q_FOUR_OVER_SIX = 1, FP4Q_SWEEP_MSE = 2, FP4Q_SWEEP_W
                                            H_16/4 first (see fp4q_hadamard_global_scale)      */
 #define FP4Q_F_HADAMARD32         0x10u /* MXFP4 quantize: rotate every 32-element block first,
                                            as fp4q_hadamard_quantize does                     */
+#define FP4Q_F_MX_SWEEP           0x20u /* MXFP4 quantize (fp4q_quantize, fp4q_hadamard_quantize):
+                                           MX scale sweep -- each block's exponent is the one
+                                           among e_c-2 .. e_c (e_c = the ceil rule) with the
+                                           lowest block error; not with FP4Q_F_MX_OCP_FLOOR    */
 
 /* Size in bytes of the workspace every quantize call needs (a small constant). */
 size_t fp4q_workspace_bytes(void);
@@ -100,7 +110,8 @@ size_t fp4q_workspace_bytes(void);
  *   flags: FP4Q_F_GLOBAL_SCALE_GIVEN (NVFP4/IF4), FP4Q_F_MX_OCP_FLOOR (MXFP4),
  *   FP4Q_F_HADAMARD16 (NVFP4 with ABSMAX / FOUR_OVER_SIX / SWEEP_MSE, and IF4),
  *   FP4Q_F_HADAMARD32 (MXFP4 only, else FP4Q_ERR_UNSUPPORTED; identical to
- *   fp4q_hadamard_quantize).
+ *   fp4q_hadamard_quantize), FP4Q_F_MX_SWEEP (MXFP4 only, else FP4Q_ERR_UNSUPPORTED;
+ *   with FP4Q_F_MX_OCP_FLOOR: FP4Q_ERR_INVALID_ARG).
  * FP4Q_F_HADAMARD16: every 16-element block is first rotated by the normalized Sylvester
  *   Hadamard matrix H_16 / 4 (butterflies h = 1, 2, 4, 8 in binary32, then one exact
  *   multiplication by 1/4 per value), and the whole method -- S, the block scales, the
@@ -149,7 +160,8 @@ int fp4q_hadamard_global_scale(const void* x, int dtype, int64_t rows, int64_t c
  * block-wise Hadamard transforms).  had_size must be 32.  The transform is computed as the
  * fast Walsh-Hadamard butterflies h = 1, 2, 4, 8, 16 followed by one multiplication by
  * RN(1/sqrt(32)).  Same layout, alignment and error rules as fp4q_quantize with
- * fmt = FP4Q_MXFP4.  Dequantized values are in the rotated domain.
+ * fmt = FP4Q_MXFP4.  Dequantized values are in the rotated domain.  flags: 0,
+ * FP4Q_F_MX_OCP_FLOOR or FP4Q_F_MX_SWEEP (the MX scale sweep on the rotated blocks).
  */
 int fp4q_hadamard_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld,
                            int had_size, uint8_t* codes, uint8_t* scales,

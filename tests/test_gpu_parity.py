@@ -36,15 +36,16 @@ def oracle_x(w, rows=None):
     return x if rows is None else x[rows]
 
 
-def run_gpu(xd, fmt, obj="sweep_mse", imp=None, S=None, ocp=False, had=False):
+def run_gpu(xd, fmt, obj="sweep_mse", imp=None, S=None, ocp=False, had=False, mx_sweep=False):
     ws = fq.new_workspace()
     impd = None if imp is None else torch.from_numpy(np.ascontiguousarray(imp)).cuda()
     gs = None if S is None else torch.tensor([S], dtype=torch.float32, device="cuda")
     if had:
-        codes, scales = fq.hadamard_quantize(xd, mx_ocp_floor=ocp, workspace=ws)
+        codes, scales = fq.hadamard_quantize(xd, mx_ocp_floor=ocp, workspace=ws, mx_sweep=mx_sweep)
         out = (codes, scales, None)
     else:
-        out = fq.quantize(xd, fmt, obj, importance=impd, global_scale=gs, mx_ocp_floor=ocp, workspace=ws)
+        out = fq.quantize(xd, fmt, obj, importance=impd, global_scale=gs, mx_ocp_floor=ocp, workspace=ws,
+                          mx_sweep=mx_sweep)
     torch.cuda.synchronize()
     st = fq.read_device_status(ws)
     c, s, g = out
@@ -140,6 +141,22 @@ def test_mxfp4_parity(cfg, rows, cols, had, ocp):
         check_dequant(out, None, "mxfp4", r["codes"], r["scales"], had=True)
 
 
+@pytest.mark.parametrize("had", [False, True])
+@pytest.mark.parametrize("cfg,rows,cols", [("cfg5", 24, 8192), ("cfg5", 5, 96), ("cfg1", None, None)])
+def test_mx_sweep_parity(cfg, rows, cols, had):
+    # MX scale sweep (exponents e_c-2 .. e_c by block error) against the oracle, bit for bit
+    w = synth.make(cfg, rows=rows, cols=cols)
+    gc, gsc, _, st, out = run_gpu(to_dev(w), "mxfp4", had=had, mx_sweep=True)
+    x = oracle_x(w)
+    r = O.mxfp4_quantize(x, hadamard=had, sweep="sweep")
+    assert st == 0 and r["status"] == 0
+    assert_same_codes(gc, gsc, r["codes"], r["scales"])
+    check_dequant(out, None, "mxfp4", r["codes"], r["scales"], had=had)
+    rule = O.mxfp4_quantize(x, hadamard=had)["scales"].astype(int)
+    moved = gsc.astype(int) - rule
+    assert ((moved >= -2) & (moved <= 0)).all() and (moved != 0).any()
+
+
 def test_padded_rows_and_given_scale():
     w = synth.make("cfg3", rows=16, cols=1024)
     full = torch.from_numpy(w["x"].view(np.int16)).view(torch.bfloat16).cuda()
@@ -195,14 +212,15 @@ def _edge_tensors():
 
 
 @pytest.mark.parametrize("name", list(_edge_tensors()))
-@pytest.mark.parametrize("method", ["absmax", "four_over_six", "sweep_mse", "sweep_wmse", "if4", "mxfp4", "mxfp4_had"])
+@pytest.mark.parametrize("method", ["absmax", "four_over_six", "sweep_mse", "sweep_wmse", "if4", "mxfp4", "mxfp4_had",
+                                    "mxfp4_sweep", "mxfp4_had_sweep"])
 def test_edge_tensors(name, method):
     x = _edge_tensors()[name]
     xd = torch.from_numpy(x).cuda()
     if method.startswith("mxfp4"):
-        had = method.endswith("had")
-        gc, gsc, _, st, _ = run_gpu(xd, "mxfp4", had=had)
-        r = O.mxfp4_quantize(x, hadamard=had)
+        had, sw = "had" in method, method.endswith("sweep")
+        gc, gsc, _, st, _ = run_gpu(xd, "mxfp4", had=had, mx_sweep=sw)
+        r = O.mxfp4_quantize(x, hadamard=had, sweep="sweep" if sw else "rule")
     elif method == "if4":
         gc, gsc, gS, st, _ = run_gpu(xd, "if4")
         r = O.if4_quantize(x)
@@ -253,7 +271,8 @@ def test_launch_counts():
 # full workload sizes, sampled rows
 # ------------------------------------------------------------------------------------------
 FULL = [("cfg2", "nvfp4", "sweep_wmse"), ("cfg3", "nvfp4", "sweep_mse"), ("cfg4", "if4", None),
-        ("cfg5", "mxfp4", None), ("cfg5", "mxfp4_had", None)]
+        ("cfg5", "mxfp4", None), ("cfg5", "mxfp4_had", None), ("cfg5", "mxfp4", "mx_sweep"),
+        ("cfg5", "mxfp4_had", "mx_sweep")]
 
 
 @pytest.mark.parametrize("cfg,fmt,obj", FULL)
@@ -263,9 +282,9 @@ def test_full_size_sampled(cfg, fmt, obj):
     rng = np.random.default_rng(99)
     rows = np.sort(rng.choice(w["rows"], size=48, replace=False))
     if fmt.startswith("mxfp4"):
-        had = fmt.endswith("had")
-        gc, gsc, _, st, _ = run_gpu(xd, "mxfp4", had=had)
-        r = O.mxfp4_quantize(oracle_x(w, rows), hadamard=had)
+        had, sw = fmt.endswith("had"), obj == "mx_sweep"
+        gc, gsc, _, st, _ = run_gpu(xd, "mxfp4", had=had, mx_sweep=sw)
+        r = O.mxfp4_quantize(oracle_x(w, rows), hadamard=had, sweep="sweep" if sw else "rule")
     else:
         imp = w.get("importance")
         gc, gsc, gS, st, _ = run_gpu(xd, fmt, obj or "absmax", imp=imp)
