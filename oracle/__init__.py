@@ -59,7 +59,7 @@ def lib():
         L.fp4q_o_nvfp4_quantize.restype = C.c_int
         L.fp4q_o_nvfp4_quantize.argtypes = [P, i64, i64, i64, C.c_int, P, C.c_int, P, P, P, P, P, P, P]
         L.fp4q_o_if4_quantize.restype = C.c_int
-        L.fp4q_o_if4_quantize.argtypes = [P, i64, i64, i64, C.c_int, P, P, P, P, P]
+        L.fp4q_o_if4_quantize.argtypes = [P, i64, i64, i64, C.c_int, C.c_int, P, P, P, P, P]
         L.fp4q_o_mxfp4_quantize.restype = C.c_int
         L.fp4q_o_mxfp4_quantize.argtypes = [P, i64, i64, i64, C.c_int, C.c_int, C.c_int, P, P]
         L.fp4q_o_mx_block_errors.restype = C.c_int
@@ -161,7 +161,12 @@ def nvfp4_quantize(x, objective="sweep_mse", importance=None, S=None, hadamard16
             "p": bp, "err": be, "err2": be2, "nvalid": bn}
 
 
-def if4_quantize(x, S=None, hadamard16=False):
+IF4_SWEEP = {"absmax": 0, "sweep": 1, "brute": 2}
+
+
+def if4_quantize(x, S=None, hadamard16=False, sweep="absmax"):
+    """IF4 codes, scale bytes (indicator in bit 7) and S.  sweep: "absmax" (the AbsMax scale),
+    "sweep" (IF4 x ScaleSweep over the MSE window), "brute" (every E4M3 pattern)."""
     x = rotate16(x) if hadamard16 else _f32(x)
     rows, cols = x.shape
     nb = cols // 16
@@ -170,8 +175,8 @@ def if4_quantize(x, S=None, hadamard16=False):
     Sarr = np.array([0.0 if S is None else S], np.float32)
     ef = np.zeros((rows, nb), np.float32)
     ei = np.zeros((rows, nb), np.float32)
-    st = lib().fp4q_o_if4_quantize(_p(x), rows, cols, cols, int(S is not None), _p(Sarr), _p(codes),
-                                   _p(scales), _p(ef), _p(ei))
+    st = lib().fp4q_o_if4_quantize(_p(x), rows, cols, cols, IF4_SWEEP[sweep], int(S is not None), _p(Sarr),
+                                   _p(codes), _p(scales), _p(ef), _p(ei))
     if st < 0:
         raise ValueError("oracle: bad shape")
     return {"codes": codes, "scales": scales, "S": float(Sarr[0]), "S_f32": Sarr, "status": st,

@@ -45,6 +45,9 @@
  *   IF4    = AbsMax scale p0; INT4 path z = RN(y*RN(7/6)), n = clamp(rint(z), -7, 7),
  *            v = RN(n*RN(6/7)), r = RN(v - y); both paths share s, so INT4 iff
  *            E_int < E_fp.
+ *   IF4 sweep = every MSE-window candidate p0-3 .. p0+7 under both types, error
+ *            RN(RN(sv*sv) * E) as for the NVFP4 sweep; (error, offset, FP4-before-INT4)
+ *            lexicographic.
  *   MXFP4  = e = smallest integer with a_b <= 6*2^e (clamped to [-127,127]), byte e+127,
  *            y = RN(x * 2^-e), q = E2M1(y), dequant q*2^e.
  *   MX sweep = e among e_c - 2 .. e_c (e_c the rule above) minimizing RN(E * 4^(e - e_c)),
@@ -288,7 +291,41 @@ int fp4q_o_nvfp4_quantize(const float* x, int64_t rows, int64_t cols, int64_t ld
 
 static float rint_even(float z) { return nearbyintf(z); } /* default rounding mode: to nearest even */
 
-int fp4q_o_if4_quantize(const float* x, int64_t rows, int64_t cols, int64_t ld,
+/* FP4 and scaled-INT4 residual sums of one block at reciprocal scale inv, in units of the
+ * scale (E = RN(acc_even + acc_odd), fma accumulation in element order), and the codes of both
+ * paths.  [IF4]: INT4 z = RN(y*RN(7/6)), n = clamp(rint(z), -7, 7), v = RN(n*RN(6/7)). */
+static void if4_block_sums(const float* xb, float inv, float* ef, float* ei, int* cf, int* ci)
+{
+    const float K76 = 7.0f / 6.0f, K67 = 6.0f / 7.0f;   /* RN of each ratio */
+    float accf[2] = {0, 0}, acci[2] = {0, 0};
+    for (int i = 0; i < 16; ++i) {
+        float y = xb[i] * inv;
+        cf[i] = fp4q_o_e2m1_encode(y);
+        float q = fp4q_o_e2m1_value(cf[i]);
+        float rf = q - y;
+        accf[i & 1] = fmaf(rf, rf, accf[i & 1]);
+        float z = y * K76;
+        float n = rint_even(z);
+        if (n > 7.0f) n = 7.0f;
+        if (n < -7.0f) n = -7.0f;
+        float v = n * K67;
+        float ri = v - y;
+        acci[i & 1] = fmaf(ri, ri, acci[i & 1]);
+        ci[i] = ((int)n) & 0xF;   /* two's complement nibble */
+    }
+    *ef = accf[0] + accf[1];
+    *ei = acci[0] + acci[1];
+}
+
+/* sweep: 0 = IF4 at the AbsMax scale p0 (INT4 iff E_int < E_fp);
+ *        1 = IF4 x ScaleSweep: every candidate p0 + k, k = -3..+7 (patterns 0..126), under
+ *            both element types; error = RN(RN(sv^2) * E) (the zero scale: the fma sum of x^2,
+ *            both types alike); lexicographic (error, offset, type) with FP4 before INT4, so
+ *            the lowest offset and then FP4 win ties;
+ *        2 = the same over all patterns 0..126 (window check).
+ * blk_err_fp / blk_err_int receive both types' errors at the chosen pattern (mode 0: the
+ * unscaled E; modes 1-2: the scaled errors). */
+int fp4q_o_if4_quantize(const float* x, int64_t rows, int64_t cols, int64_t ld, int sweep,
                         int scale_given, float* S_io, uint8_t* codes, uint8_t* scales,
                         float* blk_err_fp, float* blk_err_int)
 {
@@ -312,7 +349,6 @@ int fp4q_o_if4_quantize(const float* x, int64_t rows, int64_t cols, int64_t ld,
         memset(scales, 0, (size_t)(rows * nb));
         return status;
     }
-    const float K76 = 7.0f / 6.0f, K67 = 6.0f / 7.0f;   /* RN of each ratio */
     const float d6 = 6.0f * S;
     for (int64_t r = 0; r < rows; ++r) {
         for (int64_t b = 0; b < nb; ++b) {
@@ -320,33 +356,50 @@ int fp4q_o_if4_quantize(const float* x, int64_t rows, int64_t cols, int64_t ld,
             float ab = 0.0f;
             for (int i = 0; i < B; ++i) ab = fmaxf(ab, fabsf(xb[i]));
             int p0 = S > 0.0f ? fp4q_o_e4m3_encode(ab / d6) : 0;
-            float sv, inv;
-            scale_pair(p0, S, &sv, &inv);
-            float accf[2] = {0, 0}, acci[2] = {0, 0};
+            int bp = p0, use_int = 0;
+            float ef, ei;
             int cf[16], ci[16];
-            for (int i = 0; i < B; ++i) {
-                float y = xb[i] * inv;
-                cf[i] = fp4q_o_e2m1_encode(y);
-                float q = fp4q_o_e2m1_value(cf[i]);
-                float rf = q - y;
-                accf[i & 1] = fmaf(rf, rf, accf[i & 1]);
-                float z = y * K76;
-                float n = rint_even(z);
-                if (n > 7.0f) n = 7.0f;
-                if (n < -7.0f) n = -7.0f;
-                float v = n * K67;
-                float ri = v - y;
-                acci[i & 1] = fmaf(ri, ri, acci[i & 1]);
-                ci[i] = ((int)n) & 0xF;   /* two's complement nibble */
+            if (sweep == 0) {
+                float sv, inv;
+                scale_pair(p0, S, &sv, &inv);
+                if4_block_sums(xb, inv, &ef, &ei, cf, ci);
+                use_int = ei < ef;
+            } else {
+                int lo = sweep == 1 ? p0 - 3 : 0, hi = sweep == 1 ? p0 + 7 : 0x7E;
+                if (lo < 0) lo = 0;
+                if (hi > 0x7E) hi = 0x7E;
+                if (S == 0.0f) lo = hi = 0;
+                float best = INFINITY, bf = 0.0f, bi = 0.0f;
+                bp = lo;
+                for (int p = lo; p <= hi; ++p) {
+                    float e_fp, e_int;
+                    if (p == 0) {
+                        float acc[2] = {0, 0};
+                        for (int i = 0; i < B; ++i) acc[i & 1] = fmaf(xb[i], xb[i], acc[i & 1]);
+                        e_fp = e_int = acc[0] + acc[1];
+                    } else {
+                        float sv, inv, E_f, E_i;
+                        scale_pair(p, S, &sv, &inv);
+                        if4_block_sums(xb, inv, &E_f, &E_i, cf, ci);
+                        const float s2 = sv * sv;
+                        e_fp = s2 * E_f;
+                        e_int = s2 * E_i;
+                    }
+                    if (e_fp < best) { best = e_fp; bp = p; use_int = 0; bf = e_fp; bi = e_int; }
+                    if (e_int < best) { best = e_int; bp = p; use_int = 1; bf = e_fp; bi = e_int; }
+                }
+                float sv, inv;
+                scale_pair(bp, S, &sv, &inv);
+                if4_block_sums(xb, inv, &ef, &ei, cf, ci);   /* codes of the chosen scale */
+                ef = bf;
+                ei = bi;
             }
-            float ef = accf[0] + accf[1], ei = acci[0] + acci[1];
-            int use_int = ei < ef;
             uint8_t* crow = codes + r * (cols / 2) + b * B / 2;
             for (int i = 0; i < B; i += 2) {
                 int lo = use_int ? ci[i] : cf[i], hi = use_int ? ci[i + 1] : cf[i + 1];
                 crow[i / 2] = (uint8_t)(lo | (hi << 4));
             }
-            scales[r * nb + b] = (uint8_t)(p0 | (use_int ? 0x80 : 0));
+            scales[r * nb + b] = (uint8_t)(bp | (use_int ? 0x80 : 0));
             if (blk_err_fp) blk_err_fp[r * nb + b] = ef;
             if (blk_err_int) blk_err_int[r * nb + b] = ei;
         }

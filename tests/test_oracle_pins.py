@@ -376,6 +376,54 @@ def test_mx_sweep_error_never_above_either_rule():
         assert (es < er).any()
 
 
+def _if4_blocks(seed, n):
+    """Tensors of 16-element blocks for the IF4 sweep: Student-t weights (the IF4 workload's
+    shape), Laplace activations with per-channel scales, and INT4 / E2M1 grid points at random
+    E4M3 scales, each tensor carrying its own S."""
+    rng = np.random.default_rng(seed)
+    t = (rng.standard_t(4, size=(n, 64)) * 0.02).astype(np.float32)
+    lap = (rng.laplace(size=(n, 64)) * np.exp(rng.normal(0, 1.5, size=(1, 64)))).astype(np.float32)
+    k67 = np.float32(6.0) / np.float32(7.0)
+    ints = (rng.integers(-7, 8, size=(n, 64)).astype(np.float32) * k67).astype(np.float32)
+    ints *= np.float32(2.0) ** rng.integers(-3, 3, size=(n, 4)).repeat(16, axis=1).astype(np.float32)
+    return [t, lap, ints]
+
+
+def test_if4_sweep_window_holds_the_optimum():
+    # IF4 x ScaleSweep over the MSE window against the brute force over all 127 patterns under
+    # both types, on config-shaped weights and activations and on exact INT4 grids
+    w4 = synth.make("cfg4", rows=8, cols=14336)
+    w3 = synth.make("cfg3", rows=8, cols=4096)
+    for x in [synth.as_f32(w4), synth.as_f32(w3)] + _if4_blocks(21, 64):
+        sw = O.if4_quantize(x, sweep="sweep")
+        bf = O.if4_quantize(x, sweep="brute")
+        a = O.if4_quantize(x)
+        off = (sw["scales"] & 0x7F).astype(int) - (a["scales"] & 0x7F).astype(int)
+        assert ((off >= -3) & (off <= 7)).all()
+        assert np.array_equal(sw["scales"], bf["scales"])
+        assert np.array_equal(sw["codes"], bf["codes"])
+
+
+def test_if4_sweep_dominates_if4_and_the_nvfp4_sweep():
+    # Under the contract the IF4 sweep's candidate set contains the NVFP4 sweep's (same FP4
+    # errors) and IF4's own (both types at p0), so its chosen error is never larger -- exactly.
+    w4 = synth.make("cfg4", rows=8, cols=14336)
+    for x in [synth.as_f32(w4)] + _if4_blocks(22, 32):
+        sw = O.if4_quantize(x, sweep="sweep")
+        chosen = np.where(sw["scales"] >> 7, sw["err_int"], sw["err_fp"])
+        nv = O.nvfp4_quantize(x, "sweep_mse", S=sw["S"])
+        assert (chosen <= nv["err"]).all()
+        a = O.if4_quantize(x, S=sw["S"])
+        p0 = (a["scales"] & 0x7F).astype(int)
+        sv = (np.array([O.lib().fp4q_o_e4m3_value(int(p)) for p in range(128)], np.float32)[p0]
+              * np.float32(sw["S"])).astype(np.float32)
+        s2 = (sv * sv).astype(np.float32)
+        at_p0 = np.where(p0 == 0, np.minimum(a["err_fp"], a["err_int"]),
+                         (s2 * np.minimum(a["err_fp"], a["err_int"])).astype(np.float32))
+        assert (chosen[p0 > 0] <= at_p0[p0 > 0]).all()
+        assert (chosen < nv["err"]).any() and (chosen < at_p0).any()
+
+
 def test_hadamard_is_normalized_sylvester():
     H = np.array([[1.0]])
     while H.shape[0] < 32:
@@ -508,8 +556,8 @@ def test_hand_worked(row):
         assert np.array_equal(xh[0], expect)
         return
     x = _tensor_with(xb)
-    if method == "if4":
-        r = O.if4_quantize(x)
+    if method.startswith("if4"):
+        r = O.if4_quantize(x, sweep="sweep" if method.endswith("sweep") else "absmax")
         assert r["S"] == float(S)
         assert r["scales"][0, 0] == scale
         err = r["err_int"][0, 0] if scale & 0x80 else r["err_fp"][0, 0]
