@@ -34,6 +34,9 @@ WORKLOADS = {
     "cfg2": ("cfg2", "nvfp4", "sweep_wmse",
              "NVFP4 ScaleSweep-WMSE, bf16 weight 14336x4096, 0.02*t5, per-input-column importance"),
     "cfg4": ("cfg4", "if4", None, "IF4 per-block FP4/INT4 selection, bf16 weight 4096x14336, 0.02*t4"),
+    "cfg4s": ("cfg4", "if4", "if4_sweep",
+              "IF4 x ScaleSweep (scale and FP4/INT4 type chosen together over offsets [-3,+7]), bf16 weight "
+              "4096x14336, 0.02*t4"),
     "cfg5": ("cfg5", "mxfp4", None, "MXFP4, bf16 activations 16384x8192"),
     "cfg5h": ("cfg5", "mxfp4_had", None, "MXFP4 after 32x32 block Hadamard, bf16 activations 16384x8192"),
     "cfg5s": ("cfg5", "mxfp4", "mx_sweep",
@@ -50,7 +53,10 @@ METRIC = "quantize GB/s (input bf16) and % of B200 HBM peak, 1 GPU, vs CPU oracl
 # scale one multiply (x/s), one E2M1 rounding, one subtraction (residual) and one fused
 # multiply-add (square-accumulate) -- plus, for WMSE, the weight multiply -- over 11 (MSE) or
 # 16 (WMSE) candidates, plus the block maximum and the final multiply + rounding.
-ALU_OPS_PER_ELEMENT = {"sweep_mse": 11 * 4 + 3, "sweep_wmse": 16 * 5 + 3}
+ALU_OPS_PER_ELEMENT = {"sweep_mse": 11 * 4 + 3, "sweep_wmse": 16 * 5 + 3,
+                       # IF4 x ScaleSweep: per candidate the FP4 four plus the INT4 pre-scale,
+                       # rounding, clamp, de-scale, residual and square-accumulate
+                       "if4_sweep": 11 * (4 + 6) + 3}
 # the 16-point rotation adds four butterfly additions and one multiplication per element
 ROTATION_OPS_PER_ELEMENT = 4 + 1
 
@@ -178,7 +184,7 @@ def cpu_baseline(w, fmt, obj, budget_s=12.0):
         if base == "nvfp4":
             O.nvfp4_quantize(xs, obj, importance=imp, hadamard16=had16)
         elif base == "if4":
-            O.if4_quantize(xs, hadamard16=had16)
+            O.if4_quantize(xs, hadamard16=had16, sweep="sweep" if obj == "if4_sweep" else "absmax")
         else:
             O.mxfp4_quantize(xs, hadamard=fmt.endswith("had"), sweep="sweep" if obj == "mx_sweep" else "rule")
         done += xs.shape[0]
@@ -209,7 +215,7 @@ def run_reference(args, rank, world):
         if base == "nvfp4":
             O.nvfp4_quantize(xs, obj, importance=imp, hadamard16=had16)
         elif base == "if4":
-            O.if4_quantize(xs, hadamard16=had16)
+            O.if4_quantize(xs, hadamard16=had16, sweep="sweep" if obj == "if4_sweep" else "absmax")
         else:
             O.mxfp4_quantize(xs, hadamard=fmt.endswith("had"), sweep="sweep" if obj == "mx_sweep" else "rule")
 
@@ -272,7 +278,7 @@ def run_ours(args, rank, world):
                 fq.quantize(xs[s], "mxfp4", out=(c, sc, None), workspace=ws, mx_sweep=(obj == "mx_sweep"))
         else:
             fq.quantize(xs[s], base, obj or "absmax", importance=imp, global_scale=g, out=(c, sc, g), workspace=ws,
-                        hadamard16=had16)
+                        hadamard16=had16, if4_sweep=(obj == "if4_sweep"))
         return 1
 
     def step(s):
@@ -356,7 +362,7 @@ def run_ours(args, rank, world):
     e2e_steps = max(1, min(args.steps, 50))
     x_pin = x_host.pin_memory()
     hq = fq.HostQuantizer(rows, cols, fmt, obj or "absmax", importance=imp, dtype=x_host.dtype, depth=2,
-                          device=dev, mx_sweep=(obj == "mx_sweep"))
+                          device=dev, mx_sweep=(obj == "mx_sweep"), if4_sweep=(obj == "if4_sweep"))
     host_outs = [fq.alloc_host_outputs(rows, cols, fmt) for _ in range(2)]
     for i in range(3):
         hq(x_pin, host_outs[i % 2])

@@ -21,7 +21,8 @@ DEVSTAT_OK, DEVSTAT_NONFINITE, DEVSTAT_RANGE = 0, 1, 2
 IN_F32, IN_BF16 = 0, 1
 FORMATS = {"nvfp4": 0, "if4": 1, "mxfp4": 2}
 OBJECTIVES = {"absmax": 0, "four_over_six": 1, "sweep_mse": 2, "sweep_wmse": 3}
-F_GLOBAL_SCALE_GIVEN, F_MX_OCP_FLOOR, F_OUT_BF16, F_HADAMARD16, F_HADAMARD32, F_MX_SWEEP = 0x1, 0x2, 0x4, 0x8, 0x10, 0x20
+F_GLOBAL_SCALE_GIVEN, F_MX_OCP_FLOOR, F_OUT_BF16, F_HADAMARD16, F_HADAMARD32, F_MX_SWEEP, F_IF4_SWEEP = (
+    0x1, 0x2, 0x4, 0x8, 0x10, 0x20, 0x40)
 BLOCK = {"nvfp4": 16, "if4": 16, "mxfp4": 32}
 
 # Names of every function include/fp4q.h declares (checked against the header by the tests).
@@ -121,14 +122,15 @@ def alloc_outputs(rows: int, cols: int, fmt: str, device="cuda"):
     return codes, scales, gs
 
 
-def _flags(global_scale, mx_ocp_floor, hadamard16, mx_sweep=False):
+def _flags(global_scale, mx_ocp_floor, hadamard16, mx_sweep=False, if4_sweep=False):
     return ((F_GLOBAL_SCALE_GIVEN if global_scale is not None else 0) | (F_MX_OCP_FLOOR if mx_ocp_floor else 0)
-            | (F_HADAMARD16 if hadamard16 else 0) | (F_MX_SWEEP if mx_sweep else 0))
+            | (F_HADAMARD16 if hadamard16 else 0) | (F_MX_SWEEP if mx_sweep else 0)
+            | (F_IF4_SWEEP if if4_sweep else 0))
 
 
 def quantize(x, fmt: str = "nvfp4", objective: str = "sweep_mse", importance=None, global_scale=None,
              mx_ocp_floor: bool = False, out=None, workspace=None, stream=None, hadamard16: bool = False,
-             mx_sweep: bool = False):
+             mx_sweep: bool = False, if4_sweep: bool = False):
     """Quantize a 2-D bf16/fp32 CUDA tensor (row stride may exceed the width).
 
     Returns (codes [rows, cols/2] uint8, scales [rows, cols/B] uint8, S [1] float32 or None).
@@ -136,12 +138,13 @@ def quantize(x, fmt: str = "nvfp4", objective: str = "sweep_mse", importance=Non
     out: optional preallocated (codes, scales, S) tuple.
     hadamard16: NVFP4/IF4 on blocks rotated by the normalized 16-point Hadamard.
     mx_sweep: MXFP4 with the MX scale sweep (exponents e_c-2 .. e_c by block error).
+    if4_sweep: IF4 x ScaleSweep (scale and element type chosen together over the MSE window).
     """
     if x.dim() != 2 or x.stride(1) != 1:
         raise Fp4qError("x must be 2-D with unit column stride")
     rows, cols = x.shape
     codes, scales, gs = out if out is not None else alloc_outputs(rows, cols, fmt, x.device)
-    flags = _flags(global_scale, mx_ocp_floor, hadamard16, mx_sweep)
+    flags = _flags(global_scale, mx_ocp_floor, hadamard16, mx_sweep, if4_sweep)
     if global_scale is not None:
         gs = global_scale
     ws = workspace if workspace is not None else new_workspace(x.device)
@@ -200,7 +203,7 @@ def dequantize(codes, scales, global_scale, fmt: str = "nvfp4", inverse_hadamard
 
 def quantize_noalloc(x, fmt: str = "nvfp4", objective: str = "sweep_mse", importance=None, global_scale=None,
                      mx_ocp_floor: bool = False, out=None, device_status=None, stream=None,
-                     hadamard16: bool = False, mx_sweep: bool = False):
+                     hadamard16: bool = False, mx_sweep: bool = False, if4_sweep: bool = False):
     """quantize() for callers that cannot allocate device memory: the library's own
     per-GPU scratch replaces the workspace (see fp4q_quantize_noalloc in include/fp4q.h).
     Outputs must be passed in `out`; device_status is an optional [1] int32 CUDA tensor."""
@@ -208,7 +211,7 @@ def quantize_noalloc(x, fmt: str = "nvfp4", objective: str = "sweep_mse", import
         raise Fp4qError("x must be 2-D with unit column stride")
     rows, cols = x.shape
     codes, scales, gs = out
-    flags = _flags(global_scale, mx_ocp_floor, hadamard16, mx_sweep)
+    flags = _flags(global_scale, mx_ocp_floor, hadamard16, mx_sweep, if4_sweep)
     if global_scale is not None:
         gs = global_scale
     rc = lib().fp4q_quantize_noalloc(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), FORMATS[fmt],
@@ -256,15 +259,18 @@ class HostQuantizer:
     kernels and output copies.  Each call returns the host (codes, scales, S) it will fill;
     they are valid once `synchronize()` (or the compute stream) has passed the call.
     fmt: "nvfp4", "if4", "mxfp4", or the rotated "nvfp4_had", "if4_had", "mxfp4_had";
-    mx_sweep: MXFP4 with the MX scale sweep."""
+    mx_sweep: MXFP4 with the MX scale sweep; if4_sweep: IF4 x ScaleSweep."""
 
     def __init__(self, rows, cols, fmt="nvfp4", objective="sweep_mse", importance=None, dtype=None, depth=2,
-                 device="cuda", copy_stream=None, compute_stream=None, mx_sweep: bool = False):
+                 device="cuda", copy_stream=None, compute_stream=None, mx_sweep: bool = False,
+                 if4_sweep: bool = False):
         torch = _torch()
         self.rows, self.cols, self.fmt, self.objective = rows, cols, fmt, objective
         self.base, self.flags = split_fmt(fmt)
         if mx_sweep:
             self.flags |= F_MX_SWEEP
+        if if4_sweep:
+            self.flags |= F_IF4_SWEEP
         self.dtype = dtype or torch.bfloat16
         self.importance = importance
         self.copy_stream = copy_stream or torch.cuda.Stream(device=device)

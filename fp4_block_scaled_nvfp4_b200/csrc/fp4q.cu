@@ -546,6 +546,85 @@ __device__ __forceinline__ void if4_block(u64 (&xp)[8], float S, float d6, float
 }
 
 // ------------------------------------------------------------------------------------------
+// IF4 x ScaleSweep of one block: every candidate scale of the MSE window p0 - 3 .. p0 + 7 is
+// scored under both element types, error = RN(RN(sv^2) E) (E the residual sum of that type in
+// units of the scale, as above); the zero scale (when in the window) scores the fma sum of x^2
+// for both types.  Candidates in increasing offset, FP4 before INT4, strict improvement: the
+// lowest offset and then FP4 win ties.  Adaptive Block-Scaled Data Types
+// (gist.science/ko/paper/2603.28765), Methodology (IF4 per-block type choice) searched jointly
+// with ScaleSweep (gist.science/ko/paper/2606.07618), Methodology (MSE window).
+// ------------------------------------------------------------------------------------------
+// Residual sums of one block at reciprocal scale inv: FP4 into accf, scaled INT4 into acci
+// (z = RN(y RN(7/6)), n = clamp(rint(z), -7, 7), r = RN(RN(n RN(6/7)) - y)); the INT4 products
+// feeding a subtraction use the scalar .rn intrinsics, which are never contracted.
+__device__ __forceinline__ void if4_sums(const u64 (&xp)[8], float inv, float K76, float K67, float& ef, float& ei) {
+    const u64 inv2 = pk(inv, inv), k76 = pk(K76, K76);
+    u64 accf = pk(0.0f, 0.0f), acci = pk(0.0f, 0.0f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const u64 y = mul2(xp[j], inv2);
+        const u64 rf = e2m1x2_residual2(y);
+        accf = fma2(rf, rf, accf);
+        float y0, y1, z0, z1;
+        upk(y, y0, y1);
+        upk(mul2(y, k76), z0, z1);   // feeds only the rounding, never an addition
+        const float n0 = fminf(fmaxf(rintf(z0), -7.0f), 7.0f), n1 = fminf(fmaxf(rintf(z1), -7.0f), 7.0f);
+        const u64 ri = pk(__fsub_rn(__fmul_rn(n0, K67), y0), __fsub_rn(__fmul_rn(n1, K67), y1));
+        acci = fma2(ri, ri, acci);
+    }
+    float a, b;
+    upk(accf, a, b);
+    ef = __fadd_rn(a, b);
+    upk(acci, a, b);
+    ei = __fadd_rn(a, b);
+}
+
+template <bool HAD>
+__device__ __forceinline__ void if4_sweep_block(u64 (&xp)[8], float S, float d6, float K76, float K67,
+                                                const float2* tab, uint2* cdst, uint8_t* sdst) {
+    if (HAD) fwht16(xp);
+    int bp = 0;
+    bool use_int = false;
+    if (S > 0.0f) {
+        const int p0 = e4m3_rne(__fdiv_rn(block_absmax(xp), d6));
+        float best = INFINITY;
+        int kb = max(-3, -p0);   // the first candidate (FP4) if every error is +inf
+        bool ib = false;
+        if (p0 - 3 <= 0) best = zero_scale_error<false>(xp, xp);   // pattern 0: both types alike, FP4 first
+        const float2* t = tab + p0;
+#pragma unroll
+        for (int k = -3; k <= 7; ++k) {
+            const float2 c = t[k];
+            float ef, ei;
+            if4_sums(xp, c.x, K76, K67, ef, ei);
+            ef = __fmul_rn(c.y, ef);   // RN(sv^2) E; NaN for the non-candidate patterns
+            ei = __fmul_rn(c.y, ei);
+            if (ef < best) { best = ef; kb = k; ib = false; }
+            if (ei < best) { best = ei; kb = k; ib = true; }
+        }
+        bp = p0 + kb;
+        use_int = ib;
+    }
+    const float inv = tab[bp].x;
+    if (!use_int) {
+        *cdst = block_codes(xp, inv);
+    } else {
+        uint32_t ci[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            float y0, y1;
+            upk(mul2(xp[j], pk(inv, inv)), y0, y1);
+            const int n0 = (int)fminf(fmaxf(rintf(__fmul_rn(y0, K76)), -7.0f), 7.0f);
+            const int n1 = (int)fminf(fmaxf(rintf(__fmul_rn(y1, K76)), -7.0f), 7.0f);
+            ci[j] = ((uint32_t)n0 & 0xFu) | (((uint32_t)n1 & 0xFu) << 4);
+        }
+        *cdst = make_uint2(ci[0] | (ci[1] << 8) | (ci[2] << 16) | (ci[3] << 24),
+                           ci[4] | (ci[5] << 8) | (ci[6] << 16) | (ci[7] << 24));
+    }
+    *sdst = (uint8_t)(bp | (use_int ? 0x80 : 0));
+}
+
+// ------------------------------------------------------------------------------------------
 // The NVFP4 / IF4 quantize kernel (KIND = the NVFP4 objective, or KIND_IF4).  Each thread
 // walks the blocks tid, tid + G, ... (G threads in the grid) with the next block's loads in
 // flight while the current one is searched; the CTA builds its scale table once.  The host
@@ -554,12 +633,12 @@ __device__ __forceinline__ void if4_block(u64 (&xp)[8], float S, float d6, float
 // per-CTA start-up (S, table, first loads) would otherwise not be amortized.  The status
 // word depends only on S, so CTA 0 writes it.
 // ------------------------------------------------------------------------------------------
-enum : int { KIND_IF4 = 4 };   // kinds 0..3 are the NVFP4 objectives
+enum : int { KIND_IF4 = 4, KIND_IF4_SWEEP = 5 };   // kinds 0..3 are the NVFP4 objectives
 
 template <int KIND>
 __host__ __device__ constexpr bool q16_persistent() {
     return KIND == KIND_IF4 || KIND == FP4Q_ABSMAX || KIND == FP4Q_FOUR_OVER_SIX ||
-           (KIND == FP4Q_SWEEP_MSE && FP4Q_SWEEP_PERSISTENT);
+           ((KIND == FP4Q_SWEEP_MSE || KIND == KIND_IF4_SWEEP) && FP4Q_SWEEP_PERSISTENT);
 }
 template <int KIND>
 __host__ __device__ constexpr int q16_min_ctas() {   // register cap: CTAs per SM the kernel is compiled for
@@ -601,6 +680,7 @@ __global__ void __launch_bounds__(kThreads, q16_min_ctas<KIND>())
         if (q16_persistent<KIND>() && IN == FP4Q_IN_BF16 && b + G < total)   // next block's loads in flight
             load_raw16<IN>(xv, block_at<IDX, false>(b + G, cols, ld, nb).xoff, rb);
         if (KIND == KIND_IF4) if4_block<HAD>(xp, S, d6, K76, K67, tab, cdst, scales + b);
+        else if (KIND == KIND_IF4_SWEEP) if4_sweep_block<HAD>(xp, S, d6, K76, K67, tab, cdst, scales + b);
         else nvfp4_block<KIND, HAD>(xp, imp, at.b, S, d6, d4, tab, cdst, scales + b);
     };
     if (q16_persistent<KIND>()) {
@@ -948,9 +1028,10 @@ void launch_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, uint32_t
 
 template <int IN, bool HAD>
 void launch_nvfp4_if4(const void* x, int64_t rows, int64_t cols, int64_t ld, int fmt, int obj, const float* imp,
-                      uint8_t* codes, uint8_t* scales, float* gs, uint32_t* ws, cudaStream_t st) {
+                      uint8_t* codes, uint8_t* scales, float* gs, uint32_t* ws, uint32_t flags, cudaStream_t st) {
     if (fmt == FP4Q_IF4) {
-        launch_q16<IN, KIND_IF4, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, st);
+        if (flags & FP4Q_F_IF4_SWEEP) launch_q16<IN, KIND_IF4_SWEEP, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, st);
+        else launch_q16<IN, KIND_IF4, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, st);
         return;
     }
     switch (obj) {
@@ -992,8 +1073,8 @@ int launch_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, int f
         launch_amax<IN>(x, rows, cols, ld, ws, gs, 0, had16, st);
         ++n;
     }
-    if (had16) launch_nvfp4_if4<IN, true>(x, rows, cols, ld, fmt, obj, imp, codes, scales, gs, ws, st);
-    else launch_nvfp4_if4<IN, false>(x, rows, cols, ld, fmt, obj, imp, codes, scales, gs, ws, st);
+    if (had16) launch_nvfp4_if4<IN, true>(x, rows, cols, ld, fmt, obj, imp, codes, scales, gs, ws, flags, st);
+    else launch_nvfp4_if4<IN, false>(x, rows, cols, ld, fmt, obj, imp, codes, scales, gs, ws, flags, st);
     return launched(n + 1);
 }
 
@@ -1037,8 +1118,9 @@ void launch_dequant16(const uint8_t* codes, const uint8_t* scales, const float* 
 int check_quantize_args(int fmt, int objective, uint32_t flags) {
     if (fmt != FP4Q_NVFP4 && fmt != FP4Q_IF4 && fmt != FP4Q_MXFP4) return FP4Q_ERR_INVALID_ARG;
     if (flags & ~(FP4Q_F_GLOBAL_SCALE_GIVEN | FP4Q_F_MX_OCP_FLOOR | FP4Q_F_HADAMARD16 | FP4Q_F_HADAMARD32 |
-                  FP4Q_F_MX_SWEEP))
+                  FP4Q_F_MX_SWEEP | FP4Q_F_IF4_SWEEP))
         return FP4Q_ERR_INVALID_ARG;
+    if ((flags & FP4Q_F_IF4_SWEEP) && fmt != FP4Q_IF4) return FP4Q_ERR_UNSUPPORTED;
     if ((flags & FP4Q_F_MX_SWEEP) && (flags & FP4Q_F_MX_OCP_FLOOR)) return FP4Q_ERR_INVALID_ARG;
     if ((flags & FP4Q_F_MX_SWEEP) && fmt != FP4Q_MXFP4) return FP4Q_ERR_UNSUPPORTED;
     if (fmt == FP4Q_NVFP4 && (objective < FP4Q_ABSMAX || objective > FP4Q_SWEEP_WMSE)) return FP4Q_ERR_INVALID_ARG;

@@ -29,6 +29,10 @@
  *   wins a tie of the computed errors.
  *   IF4 INT4: z = RN(y RN(7/6)), n = clamp(rint(z), -7, 7), v = RN(n RN(6/7)),
  *   r = RN(v - y); both paths share s, so INT4 iff E_int < E_fp.
+ *   IF4 x ScaleSweep (flag FP4Q_F_IF4_SWEEP): every MSE-window candidate p0-3 .. p0+7 under both
+ *   types, error RN(RN(sv^2) E_type) (the zero scale: the fma sum of x^2 for both); the
+ *   lowest (error, offset, type) wins with FP4 before INT4.  Adaptive Block-Scaled Data Types,
+ *   "Methodology" (IF4 type choice) searched jointly with ScaleSweep, "Methodology".
  *   MXFP4: e = smallest integer with a_b <= 6 * 2^e (flag FP4Q_F_MX_OCP_FLOOR: floor(log2
  *   a_b) - 2), clamped to [-127,127]; y = RN(x 2^-e).
  *   MX scale sweep (flag FP4Q_F_MX_SWEEP): e among e_c - 2 .. e_c (e_c the ceil rule, none
@@ -95,6 +99,9 @@ enum { FP4Q_ABSMAX = 0, FP4Q_FOUR_OVER_SIX = 1, FP4Q_SWEEP_MSE = 2, FP4Q_SWEEP_W
                                            MX scale sweep -- each block's exponent is the one
                                            among e_c-2 .. e_c (e_c = the ceil rule) with the
                                            lowest block error; not with FP4Q_F_MX_OCP_FLOOR    */
+#define FP4Q_F_IF4_SWEEP          0x40u /* IF4 quantize: IF4 x ScaleSweep -- the block scale and
+                                           the element type are chosen together over the MSE
+                                           window p0-3 .. p0+7 (see the arithmetic above)      */
 
 /* Size in bytes of the workspace every quantize call needs (a small constant). */
 size_t fp4q_workspace_bytes(void);
@@ -111,7 +118,8 @@ size_t fp4q_workspace_bytes(void);
  *   FP4Q_F_HADAMARD16 (NVFP4 with ABSMAX / FOUR_OVER_SIX / SWEEP_MSE, and IF4),
  *   FP4Q_F_HADAMARD32 (MXFP4 only, else FP4Q_ERR_UNSUPPORTED; identical to
  *   fp4q_hadamard_quantize), FP4Q_F_MX_SWEEP (MXFP4 only, else FP4Q_ERR_UNSUPPORTED;
- *   with FP4Q_F_MX_OCP_FLOOR: FP4Q_ERR_INVALID_ARG).
+ *   with FP4Q_F_MX_OCP_FLOOR: FP4Q_ERR_INVALID_ARG), FP4Q_F_IF4_SWEEP (IF4 only, else
+ *   FP4Q_ERR_UNSUPPORTED; combines with FP4Q_F_HADAMARD16 and FP4Q_F_GLOBAL_SCALE_GIVEN).
  * FP4Q_F_HADAMARD16: every 16-element block is first rotated by the normalized Sylvester
  *   Hadamard matrix H_16 / 4 (butterflies h = 1, 2, 4, 8 in binary32, then one exact
  *   multiplication by 1/4 per value), and the whole method -- S, the block scales, the

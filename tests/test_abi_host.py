@@ -57,7 +57,8 @@ FAKE = 0x10000   # 16-byte aligned non-null stand-in; validation rejects before 
     ((FAKE, 1, 4, 32, 32, 0, 3, FAKE + 4, FAKE, FAKE, FAKE, FAKE, 0), fq.ERR_ALIGNMENT),  # weights
     ((FAKE, 1, 4, 32, 32, 0, 2, None, FAKE, FAKE, FAKE, FAKE, 0x80), fq.ERR_INVALID_ARG),  # unknown flag
     ((FAKE, 1, 4, 32, 32, 2, 0, None, FAKE, FAKE, None, FAKE, 1), fq.ERR_INVALID_ARG),  # MX with given S
-    ((FAKE, 1, 4, 32, 32, 0, 2, None, FAKE, FAKE, FAKE, FAKE, 0x40), fq.ERR_INVALID_ARG),  # unknown flag
+    ((FAKE, 1, 4, 32, 32, 0, 2, None, FAKE, FAKE, FAKE, FAKE, 0x40), fq.ERR_UNSUPPORTED),  # IF4 sweep, NVFP4
+    ((FAKE, 1, 4, 64, 64, 2, 0, None, FAKE, FAKE, None, FAKE, 0x40), fq.ERR_UNSUPPORTED),  # IF4 sweep, MXFP4
     ((FAKE, 1, 4, 32, 32, 0, 2, None, FAKE, FAKE, FAKE, FAKE, 0x20), fq.ERR_UNSUPPORTED),  # MX sweep, NVFP4
     ((FAKE, 1, 4, 32, 32, 2, 0, None, FAKE, FAKE, None, FAKE, 0x22), fq.ERR_INVALID_ARG),  # MX sweep + OCP floor
     ((None, 1, 0, 32, 32, 2, 0, None, None, None, None, None, 0x20), fq.OK),             # MX sweep, empty
@@ -128,6 +129,7 @@ def test_host_async_validation():
     assert call(obj=3) == fq.ERR_INVALID_ARG                     # WMSE without weights
     assert call(x_dev=FAKE + 8) == fq.ERR_ALIGNMENT
     assert call(flags=0x8, fmt=2, cols=64) == fq.ERR_UNSUPPORTED  # 16-point rotation on MXFP4
-    assert call(flags=0x40) == fq.ERR_INVALID_ARG
+    assert call(flags=0x80) == fq.ERR_INVALID_ARG
+    assert call(flags=0x40) == fq.ERR_UNSUPPORTED                 # IF4 sweep on NVFP4
     assert call(flags=0x20) == fq.ERR_UNSUPPORTED                 # MX sweep on NVFP4
     assert call(rows=0, x_host=None, x_dev=None) == fq.OK and L.fp4q_last_launch_count() == 0

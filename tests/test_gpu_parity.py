@@ -36,7 +36,8 @@ def oracle_x(w, rows=None):
     return x if rows is None else x[rows]
 
 
-def run_gpu(xd, fmt, obj="sweep_mse", imp=None, S=None, ocp=False, had=False, mx_sweep=False):
+def run_gpu(xd, fmt, obj="sweep_mse", imp=None, S=None, ocp=False, had=False, mx_sweep=False, if4_sweep=False,
+            had16=False):
     ws = fq.new_workspace()
     impd = None if imp is None else torch.from_numpy(np.ascontiguousarray(imp)).cuda()
     gs = None if S is None else torch.tensor([S], dtype=torch.float32, device="cuda")
@@ -45,7 +46,7 @@ def run_gpu(xd, fmt, obj="sweep_mse", imp=None, S=None, ocp=False, had=False, mx
         out = (codes, scales, None)
     else:
         out = fq.quantize(xd, fmt, obj, importance=impd, global_scale=gs, mx_ocp_floor=ocp, workspace=ws,
-                          mx_sweep=mx_sweep)
+                          mx_sweep=mx_sweep, if4_sweep=if4_sweep, hadamard16=had16)
     torch.cuda.synchronize()
     st = fq.read_device_status(ws)
     c, s, g = out
@@ -141,6 +142,21 @@ def test_mxfp4_parity(cfg, rows, cols, had, ocp):
         check_dequant(out, None, "mxfp4", r["codes"], r["scales"], had=True)
 
 
+@pytest.mark.parametrize("had16", [False, True])
+@pytest.mark.parametrize("cfg,rows,cols", [("cfg4", 24, 14336), ("cfg4", 3, 48), ("cfg3", 17, 2048), ("cfg1", None, None)])
+def test_if4_sweep_parity(cfg, rows, cols, had16):
+    # IF4 x ScaleSweep (scale and type chosen together over the MSE window) against the oracle
+    w = synth.make(cfg, rows=rows, cols=cols)
+    gc, gsc, gS, st, out = run_gpu(to_dev(w), "if4", if4_sweep=True, had16=had16)
+    x = oracle_x(w)
+    r = O.if4_quantize(x, sweep="sweep", hadamard16=had16)
+    a = O.if4_quantize(x, hadamard16=had16)
+    assert st == 0 and f32_bits(gS) == f32_bits(r["S"])
+    assert_same_codes(gc, gsc, r["codes"], r["scales"])
+    check_dequant(out, r["S"], "if4", r["codes"], r["scales"], had=had16)
+    assert (gsc != a["scales"]).any()
+
+
 @pytest.mark.parametrize("had", [False, True])
 @pytest.mark.parametrize("cfg,rows,cols", [("cfg5", 24, 8192), ("cfg5", 5, 96), ("cfg1", None, None)])
 def test_mx_sweep_parity(cfg, rows, cols, had):
@@ -212,8 +228,8 @@ def _edge_tensors():
 
 
 @pytest.mark.parametrize("name", list(_edge_tensors()))
-@pytest.mark.parametrize("method", ["absmax", "four_over_six", "sweep_mse", "sweep_wmse", "if4", "mxfp4", "mxfp4_had",
-                                    "mxfp4_sweep", "mxfp4_had_sweep"])
+@pytest.mark.parametrize("method", ["absmax", "four_over_six", "sweep_mse", "sweep_wmse", "if4", "if4_sweep", "mxfp4",
+                                    "mxfp4_had", "mxfp4_sweep", "mxfp4_had_sweep"])
 def test_edge_tensors(name, method):
     x = _edge_tensors()[name]
     xd = torch.from_numpy(x).cuda()
@@ -221,9 +237,10 @@ def test_edge_tensors(name, method):
         had, sw = "had" in method, method.endswith("sweep")
         gc, gsc, _, st, _ = run_gpu(xd, "mxfp4", had=had, mx_sweep=sw)
         r = O.mxfp4_quantize(x, hadamard=had, sweep="sweep" if sw else "rule")
-    elif method == "if4":
-        gc, gsc, gS, st, _ = run_gpu(xd, "if4")
-        r = O.if4_quantize(x)
+    elif method.startswith("if4"):
+        sw = method.endswith("sweep")
+        gc, gsc, gS, st, _ = run_gpu(xd, "if4", if4_sweep=sw)
+        r = O.if4_quantize(x, sweep="sweep" if sw else "absmax")
         assert f32_bits(gS) == f32_bits(r["S"])
     else:
         imp = np.linspace(0.01, 5, x.shape[1]).astype(np.float32) if method == "sweep_wmse" else None
@@ -270,7 +287,7 @@ def test_launch_counts():
 # ------------------------------------------------------------------------------------------
 # full workload sizes, sampled rows
 # ------------------------------------------------------------------------------------------
-FULL = [("cfg2", "nvfp4", "sweep_wmse"), ("cfg3", "nvfp4", "sweep_mse"), ("cfg4", "if4", None),
+FULL = [("cfg2", "nvfp4", "sweep_wmse"), ("cfg3", "nvfp4", "sweep_mse"), ("cfg4", "if4", None), ("cfg4", "if4", "if4_sweep"),
         ("cfg5", "mxfp4", None), ("cfg5", "mxfp4_had", None), ("cfg5", "mxfp4", "mx_sweep"),
         ("cfg5", "mxfp4_had", "mx_sweep")]
 
@@ -287,11 +304,11 @@ def test_full_size_sampled(cfg, fmt, obj):
         r = O.mxfp4_quantize(oracle_x(w, rows), hadamard=had, sweep="sweep" if sw else "rule")
     else:
         imp = w.get("importance")
-        gc, gsc, gS, st, _ = run_gpu(xd, fmt, obj or "absmax", imp=imp)
+        gc, gsc, gS, st, _ = run_gpu(xd, fmt, obj or "absmax", imp=imp, if4_sweep=(obj == "if4_sweep"))
         S, ost = O.tensor_scale(oracle_x(w))
         assert ost == 0 and f32_bits(gS) == f32_bits(S)
         if fmt == "if4":
-            r = O.if4_quantize(oracle_x(w, rows), S=S)
+            r = O.if4_quantize(oracle_x(w, rows), S=S, sweep="sweep" if obj == "if4_sweep" else "absmax")
         else:
             r = O.nvfp4_quantize(oracle_x(w, rows), obj, importance=imp, S=S)
             nt = (r["err2"] - r["err"]) / np.maximum(r["err"], np.finfo(np.float32).tiny)
