@@ -23,10 +23,11 @@ FORMATS = {"nvfp4": 0, "if4": 1, "mxfp4": 2}
 OBJECTIVES = {"absmax": 0, "four_over_six": 1, "sweep_mse": 2, "sweep_wmse": 3}
 F_GLOBAL_SCALE_GIVEN, F_MX_OCP_FLOOR, F_OUT_BF16, F_HADAMARD16, F_HADAMARD32, F_MX_SWEEP, F_IF4_SWEEP = (
     0x1, 0x2, 0x4, 0x8, 0x10, 0x20, 0x40)
+F_SCALE_TILED = 0x80
 BLOCK = {"nvfp4": 16, "if4": 16, "mxfp4": 32}
 
 # Names of every function include/fp4q.h declares (checked against the header by the tests).
-EXPORTS = ("fp4q_workspace_bytes", "fp4q_global_scale", "fp4q_hadamard_global_scale", "fp4q_quantize",
+EXPORTS = ("fp4q_workspace_bytes", "fp4q_scale_bytes", "fp4q_global_scale", "fp4q_hadamard_global_scale", "fp4q_quantize",
            "fp4q_hadamard_quantize", "fp4q_dequantize", "fp4q_quantize_noalloc", "fp4q_quantize_host_async", "fp4q_read_device_status", "fp4q_last_launch_count", "fp4q_status_string")
 
 _lib = None
@@ -46,6 +47,8 @@ def lib():
         P, i64, u32, i32 = C.c_void_p, C.c_int64, C.c_uint32, C.c_int
         L.fp4q_workspace_bytes.restype = C.c_size_t
         L.fp4q_workspace_bytes.argtypes = []
+        L.fp4q_scale_bytes.restype = i64
+        L.fp4q_scale_bytes.argtypes = [i64, i64, i32, u32]
         L.fp4q_quantize.restype = i32
         L.fp4q_quantize.argtypes = [P, i32, i64, i64, i64, i32, i32, P, P, P, P, P, u32, P]
         L.fp4q_global_scale.restype = i32
@@ -114,23 +117,36 @@ def _dtype_code(x):
     raise Fp4qError(f"unsupported input dtype {x.dtype} (bf16 or fp32)")
 
 
-def alloc_outputs(rows: int, cols: int, fmt: str, device="cuda"):
+def alloc_outputs(rows: int, cols: int, fmt: str, device="cuda", tiled: bool = False):
+    """(codes, scales, S) device buffers; tiled: a zero-filled 1-D scales buffer in the tiled
+    layout of block-scaled GEMMs (scale_bytes(..., tiled=True) bytes)."""
     torch = _torch()
     codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=device)
-    scales = torch.empty((rows, cols // BLOCK[fmt]), dtype=torch.uint8, device=device)
+    if tiled:
+        scales = torch.zeros((scale_bytes(rows, cols, fmt, True),), dtype=torch.uint8, device=device)
+    else:
+        scales = torch.empty((rows, cols // BLOCK[fmt]), dtype=torch.uint8, device=device)
     gs = torch.empty((1,), dtype=torch.float32, device=device)
     return codes, scales, gs
 
 
-def _flags(global_scale, mx_ocp_floor, hadamard16, mx_sweep=False, if4_sweep=False):
+def _flags(global_scale, mx_ocp_floor, hadamard16, mx_sweep=False, if4_sweep=False, tiled=False):
     return ((F_GLOBAL_SCALE_GIVEN if global_scale is not None else 0) | (F_MX_OCP_FLOOR if mx_ocp_floor else 0)
             | (F_HADAMARD16 if hadamard16 else 0) | (F_MX_SWEEP if mx_sweep else 0)
-            | (F_IF4_SWEEP if if4_sweep else 0))
+            | (F_IF4_SWEEP if if4_sweep else 0) | (F_SCALE_TILED if tiled else 0))
+
+
+def scale_bytes(rows: int, cols: int, fmt: str, tiled: bool = False) -> int:
+    """Bytes of the scales buffer: rows * cols/B, or the padded tiled layout (tiled=True)."""
+    n = int(lib().fp4q_scale_bytes(rows, cols, FORMATS[fmt], F_SCALE_TILED if tiled else 0))
+    if n < 0:
+        raise Fp4qError("fp4q_scale_bytes: bad format or shape")
+    return n
 
 
 def quantize(x, fmt: str = "nvfp4", objective: str = "sweep_mse", importance=None, global_scale=None,
              mx_ocp_floor: bool = False, out=None, workspace=None, stream=None, hadamard16: bool = False,
-             mx_sweep: bool = False, if4_sweep: bool = False):
+             mx_sweep: bool = False, if4_sweep: bool = False, tiled_scales: bool = False):
     """Quantize a 2-D bf16/fp32 CUDA tensor (row stride may exceed the width).
 
     Returns (codes [rows, cols/2] uint8, scales [rows, cols/B] uint8, S [1] float32 or None).
@@ -139,12 +155,13 @@ def quantize(x, fmt: str = "nvfp4", objective: str = "sweep_mse", importance=Non
     hadamard16: NVFP4/IF4 on blocks rotated by the normalized 16-point Hadamard.
     mx_sweep: MXFP4 with the MX scale sweep (exponents e_c-2 .. e_c by block error).
     if4_sweep: IF4 x ScaleSweep (scale and element type chosen together over the MSE window).
+    tiled_scales: NVFP4/MXFP4 scales in the 128x4-tiled layout of block-scaled GEMMs (1-D buffer).
     """
     if x.dim() != 2 or x.stride(1) != 1:
         raise Fp4qError("x must be 2-D with unit column stride")
     rows, cols = x.shape
-    codes, scales, gs = out if out is not None else alloc_outputs(rows, cols, fmt, x.device)
-    flags = _flags(global_scale, mx_ocp_floor, hadamard16, mx_sweep, if4_sweep)
+    codes, scales, gs = out if out is not None else alloc_outputs(rows, cols, fmt, x.device, tiled=tiled_scales)
+    flags = _flags(global_scale, mx_ocp_floor, hadamard16, mx_sweep, if4_sweep, tiled_scales)
     if global_scale is not None:
         gs = global_scale
     ws = workspace if workspace is not None else new_workspace(x.device)
@@ -172,29 +189,31 @@ def global_scale(x, out=None, workspace=None, stream=None, hadamard16: bool = Fa
     return gs
 
 
-def hadamard_quantize(x, mx_ocp_floor: bool = False, out=None, workspace=None, stream=None, mx_sweep: bool = False):
+def hadamard_quantize(x, mx_ocp_floor: bool = False, out=None, workspace=None, stream=None, mx_sweep: bool = False,
+                      tiled_scales: bool = False):
     """MXFP4 quantization after a normalized 32-point block Hadamard rotation (mx_sweep: with
     the MX scale sweep)."""
     if x.dim() != 2 or x.stride(1) != 1:
         raise Fp4qError("x must be 2-D with unit column stride")
     rows, cols = x.shape
-    codes, scales, _ = out if out is not None else alloc_outputs(rows, cols, "mxfp4", x.device)
+    codes, scales, _ = out if out is not None else alloc_outputs(rows, cols, "mxfp4", x.device, tiled=tiled_scales)
     ws = workspace if workspace is not None else new_workspace(x.device)
     rc = lib().fp4q_hadamard_quantize(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), 32, _ptr(codes),
-                                      _ptr(scales), _ptr(ws), _flags(None, mx_ocp_floor, False, mx_sweep),
+                                      _ptr(scales), _ptr(ws), _flags(None, mx_ocp_floor, False, mx_sweep,
+                                                                     tiled=tiled_scales),
                                       _stream_ptr(stream))
     _check(rc, "fp4q_hadamard_quantize")
     return codes, scales
 
 
 def dequantize(codes, scales, global_scale, fmt: str = "nvfp4", inverse_hadamard: bool = False,
-               out_dtype=None, out=None, stream=None):
+               out_dtype=None, out=None, stream=None, tiled_scales: bool = False):
     torch = _torch()
     out_dtype = out_dtype or torch.float32
     rows, cols = codes.shape[0], codes.shape[1] * 2
     if out is None:
         out = torch.empty((rows, cols), dtype=out_dtype, device=codes.device)
-    flags = F_OUT_BF16 if out.dtype == torch.bfloat16 else 0
+    flags = (F_OUT_BF16 if out.dtype == torch.bfloat16 else 0) | (F_SCALE_TILED if tiled_scales else 0)
     rc = lib().fp4q_dequantize(_ptr(codes), _ptr(scales), _ptr(global_scale), rows, cols, FORMATS[fmt],
                                int(inverse_hadamard), _ptr(out), flags, _stream_ptr(stream))
     _check(rc, "fp4q_dequantize")

@@ -95,6 +95,24 @@ __device__ __forceinline__ void finish_status(uint32_t* ws, uint32_t flag, int c
     }
 }
 
+// Byte offset of the scale of block (r, j) -- row r, column block j of jblocks -- in the tiled
+// layout that block-scaled tensor-core GEMMs read their scale factors in: 128-row x 4-column
+// tiles of 512 bytes, tiles row-major over (r / 128, j / 4), and inside a tile row r%32 at
+// 16 (r%32) + 4 ((r/32)%4) + j%4.  The scale tensor is padded to whole tiles.
+template <typename IDX>
+__device__ __forceinline__ int64_t tiled_scale_offset(IDX r, IDX j, IDX jblocks) {
+    const int64_t jt = ((int64_t)jblocks + 3) >> 2;
+    return ((int64_t)r >> 7) * (jt * 512) + ((int64_t)j >> 2) * 512 + ((int64_t)r & 31) * 16 +
+           (((int64_t)r >> 5) & 3) * 4 + ((int64_t)j & 3);
+}
+// Scale offset of linear block index blk of a tensor with jblocks blocks per row.
+template <typename IDX>
+__device__ __forceinline__ int64_t scale_offset(IDX blk, IDX jblocks, bool tiled) {
+    if (!tiled) return (int64_t)blk;
+    const IDX r = blk / jblocks;
+    return tiled_scale_offset<IDX>(r, blk - r * jblocks, jblocks);
+}
+
 // ------------------------------------------------------------------------------------------
 // amax
 // ------------------------------------------------------------------------------------------
@@ -649,7 +667,7 @@ template <int IN, int KIND, bool HAD, typename IDX>
 __global__ void __launch_bounds__(kThreads, q16_min_ctas<KIND>())
     q16_kernel(const void* __restrict__ xv, IDX rows, IDX cols, IDX ld, const float* __restrict__ imp,
                uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, const float* __restrict__ gscale,
-               uint32_t* __restrict__ ws) {
+               uint32_t* __restrict__ ws, int tiled) {
     __shared__ float2 s_tab[kTabLen];
     const IDX nb = cols / 16;
     const IDX total = rows * nb;
@@ -669,9 +687,10 @@ __global__ void __launch_bounds__(kThreads, q16_min_ctas<KIND>())
     auto one_block = [&](IDX b) {
         const BlockAt<IDX> at = block_at<IDX, KIND == FP4Q_SWEEP_WMSE>(b, cols, ld, nb);
         uint2* cdst = reinterpret_cast<uint2*>(codes + at.coff);
+        uint8_t* sdst = scales + scale_offset<IDX>(b, nb, tiled != 0);
         if (flags) {   // data out of contract: zero-filled outputs
             *cdst = make_uint2(0u, 0u);
-            scales[b] = 0;
+            *sdst = 0;
             return;
         }
         if (IN != FP4Q_IN_BF16) load_raw16<IN>(xv, at.xoff, rb);
@@ -679,9 +698,9 @@ __global__ void __launch_bounds__(kThreads, q16_min_ctas<KIND>())
         unpack16<IN>(rb, xp);
         if (q16_persistent<KIND>() && IN == FP4Q_IN_BF16 && b + G < total)   // next block's loads in flight
             load_raw16<IN>(xv, block_at<IDX, false>(b + G, cols, ld, nb).xoff, rb);
-        if (KIND == KIND_IF4) if4_block<HAD>(xp, S, d6, K76, K67, tab, cdst, scales + b);
-        else if (KIND == KIND_IF4_SWEEP) if4_sweep_block<HAD>(xp, S, d6, K76, K67, tab, cdst, scales + b);
-        else nvfp4_block<KIND, HAD>(xp, imp, at.b, S, d6, d4, tab, cdst, scales + b);
+        if (KIND == KIND_IF4) if4_block<HAD>(xp, S, d6, K76, K67, tab, cdst, sdst);
+        else if (KIND == KIND_IF4_SWEEP) if4_sweep_block<HAD>(xp, S, d6, K76, K67, tab, cdst, sdst);
+        else nvfp4_block<KIND, HAD>(xp, imp, at.b, S, d6, d4, tab, cdst, sdst);
     };
     if (q16_persistent<KIND>()) {
         for (; blk < total; blk += G) one_block(blk);
@@ -773,7 +792,7 @@ template <int IN, bool HAD, bool SWEEP>
 __global__ void __launch_bounds__(kThreads) mxfp4_kernel(const void* __restrict__ xv, int64_t rows, int64_t cols,
                                                          int64_t ld, uint8_t* __restrict__ codes,
                                                          uint8_t* __restrict__ scales, uint32_t* __restrict__ ws,
-                                                         int ocp) {
+                                                         int ocp, int tiled) {
     const int64_t nb = cols / 32;
     const int64_t total = rows * nb;
     const int64_t step = (int64_t)gridDim.x * blockDim.x;
@@ -805,10 +824,11 @@ __global__ void __launch_bounds__(kThreads) mxfp4_kernel(const void* __restrict_
 #pragma unroll
         for (int i = 0; i < 32; ++i) bad |= !isfinite(v[i]);
         uint4* cdst = reinterpret_cast<uint4*>(codes + r * (cols / 2) + b * 16);
+        uint8_t* sdst = scales + (tiled ? tiled_scale_offset<int64_t>(r, b, nb) : blk);
         if (bad) {
             flag = FP4Q_DEVSTAT_NONFINITE;
             *cdst = make_uint4(0u, 0u, 0u, 0u);
-            scales[blk] = 0xFF;
+            *sdst = 0xFF;
             continue;
         }
         if (HAD) fwht32(v);
@@ -832,7 +852,7 @@ __global__ void __launch_bounds__(kThreads) mxfp4_kernel(const void* __restrict_
                            c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24),
                            c[8] | (c[9] << 8) | (c[10] << 16) | (c[11] << 24),
                            c[12] | (c[13] << 8) | (c[14] << 16) | (c[15] << 24));
-        scales[blk] = (uint8_t)(e + 127);
+        *sdst = (uint8_t)(e + 127);
     }
     finish_status(ws, flag, WS_CNT_Q);
 }
@@ -868,7 +888,7 @@ template <bool OUT_BF16, bool IF4, bool HAD>
 __global__ void __launch_bounds__(kThreads) dequant16_kernel(const uint8_t* __restrict__ codes,
                                                              const uint8_t* __restrict__ scales,
                                                              const float* __restrict__ gscale, int64_t rows,
-                                                             int64_t cols, void* __restrict__ out) {
+                                                             int64_t cols, void* __restrict__ out, int tiled) {
     const float S = *gscale;
     const float K67 = __fdiv_rn(6.0f, 7.0f);
     const int64_t nb = cols / 16;
@@ -877,7 +897,7 @@ __global__ void __launch_bounds__(kThreads) dequant16_kernel(const uint8_t* __re
     for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < total; blk += step) {
         const int64_t r = blk / nb, b = blk - r * nb;
         const uint2 c = __ldg(reinterpret_cast<const uint2*>(codes + r * (cols / 2) + b * 8));
-        const uint32_t sb = __ldg(scales + blk);
+        const uint32_t sb = __ldg(scales + (tiled ? tiled_scale_offset<int64_t>(r, b, nb) : blk));
         const int p = sb & 0x7F;
         const float sv = p == 0 ? 0.0f : (p == 127 ? __uint_as_float(0x7FC00000u) : __fmul_rn(e4m3_value(p), S));
         float v[16];
@@ -913,14 +933,14 @@ __global__ void __launch_bounds__(kThreads) dequant16_kernel(const uint8_t* __re
 template <bool OUT_BF16, bool HAD>
 __global__ void __launch_bounds__(kThreads) dequant_mx_kernel(const uint8_t* __restrict__ codes,
                                                               const uint8_t* __restrict__ scales, int64_t rows,
-                                                              int64_t cols, void* __restrict__ out) {
+                                                              int64_t cols, void* __restrict__ out, int tiled) {
     const int64_t nb = cols / 32;
     const int64_t total = rows * nb;
     const int64_t step = (int64_t)gridDim.x * blockDim.x;
     for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < total; blk += step) {
         const int64_t r = blk / nb, b = blk - r * nb;
         const uint4 c = __ldg(reinterpret_cast<const uint4*>(codes + r * (cols / 2) + b * 16));
-        const uint32_t sb = __ldg(scales + blk);
+        const uint32_t sb = __ldg(scales + (tiled ? tiled_scale_offset<int64_t>(r, b, nb) : blk));
         const float m = sb == 0xFFu ? __uint_as_float(0x7FC00000u) : pow2i((int)sb - 127);
         const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
         float v[32];
@@ -995,22 +1015,22 @@ int check_common(const void* x, int dtype, int64_t rows, int64_t cols, int64_t l
 // The NVFP4 / IF4 kernel; 32-bit index arithmetic when the tensor allows it.
 template <int IN, int KIND, bool HAD, typename IDX>
 void launch_q16_as(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* imp, uint8_t* codes,
-                   uint8_t* scales, float* gs, uint32_t* ws, cudaStream_t st) {
+                   uint8_t* scales, float* gs, uint32_t* ws, int tiled, cudaStream_t st) {
     auto kernel = q16_kernel<IN, KIND, HAD, IDX>;
     const int64_t total = rows * (cols / 16);
     const int grid = q16_persistent<KIND>() ? grid_for(kernel, total, q16_min_ctas<KIND>())
                                             : (int)((total + kThreads - 1) / kThreads);
-    kernel<<<grid, kThreads, 0, st>>>(x, (IDX)rows, (IDX)cols, (IDX)ld, imp, codes, scales, gs, ws);
+    kernel<<<grid, kThreads, 0, st>>>(x, (IDX)rows, (IDX)cols, (IDX)ld, imp, codes, scales, gs, ws, tiled);
 }
 
 template <int IN, int KIND, bool HAD>
 void launch_q16(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* imp, uint8_t* codes,
-                uint8_t* scales, float* gs, uint32_t* ws, cudaStream_t st) {
+                uint8_t* scales, float* gs, uint32_t* ws, int tiled, cudaStream_t st) {
     const int64_t total = rows * (cols / 16);
     if (total < ((int64_t)1 << 31) && rows * ld < ((int64_t)1 << 31))
-        launch_q16_as<IN, KIND, HAD, uint32_t>(x, rows, cols, ld, imp, codes, scales, gs, ws, st);
+        launch_q16_as<IN, KIND, HAD, uint32_t>(x, rows, cols, ld, imp, codes, scales, gs, ws, tiled, st);
     else
-        launch_q16_as<IN, KIND, HAD, int64_t>(x, rows, cols, ld, imp, codes, scales, gs, ws, st);
+        launch_q16_as<IN, KIND, HAD, int64_t>(x, rows, cols, ld, imp, codes, scales, gs, ws, tiled, st);
 }
 
 // Tensor scale pass: plain amax, or the amax of the 16-point rotated blocks.
@@ -1029,19 +1049,20 @@ void launch_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, uint32_t
 template <int IN, bool HAD>
 void launch_nvfp4_if4(const void* x, int64_t rows, int64_t cols, int64_t ld, int fmt, int obj, const float* imp,
                       uint8_t* codes, uint8_t* scales, float* gs, uint32_t* ws, uint32_t flags, cudaStream_t st) {
+    const int tiled = (flags & FP4Q_F_SCALE_TILED) ? 1 : 0;
     if (fmt == FP4Q_IF4) {
-        if (flags & FP4Q_F_IF4_SWEEP) launch_q16<IN, KIND_IF4_SWEEP, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, st);
-        else launch_q16<IN, KIND_IF4, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, st);
+        if (flags & FP4Q_F_IF4_SWEEP) launch_q16<IN, KIND_IF4_SWEEP, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, tiled, st);
+        else launch_q16<IN, KIND_IF4, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, tiled, st);
         return;
     }
     switch (obj) {
-        case FP4Q_ABSMAX: launch_q16<IN, FP4Q_ABSMAX, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, st); break;
+        case FP4Q_ABSMAX: launch_q16<IN, FP4Q_ABSMAX, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, tiled, st); break;
         case FP4Q_FOUR_OVER_SIX:
-            launch_q16<IN, FP4Q_FOUR_OVER_SIX, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, st);
+            launch_q16<IN, FP4Q_FOUR_OVER_SIX, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, tiled, st);
             break;
-        case FP4Q_SWEEP_MSE: launch_q16<IN, FP4Q_SWEEP_MSE, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, st); break;
+        case FP4Q_SWEEP_MSE: launch_q16<IN, FP4Q_SWEEP_MSE, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, tiled, st); break;
         default:   // WMSE is rejected with the rotation before any launch
-            if (!HAD) launch_q16<IN, FP4Q_SWEEP_WMSE, false>(x, rows, cols, ld, imp, codes, scales, gs, ws, st);
+            if (!HAD) launch_q16<IN, FP4Q_SWEEP_WMSE, false>(x, rows, cols, ld, imp, codes, scales, gs, ws, tiled, st);
             break;
     }
 }
@@ -1052,19 +1073,20 @@ int launch_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, int f
     if (fmt == FP4Q_MXFP4) {
         const int ocp = (flags & FP4Q_F_MX_OCP_FLOOR) ? 1 : 0;
         const bool had = (flags & FP4Q_F_HADAMARD32) != 0, sweep = (flags & FP4Q_F_MX_SWEEP) != 0;
+        const int tiled = (flags & FP4Q_F_SCALE_TILED) ? 1 : 0;
         const int64_t nblk = rows * (cols / 32);
         if (had && sweep)
             mxfp4_kernel<IN, true, true><<<grid_for(mxfp4_kernel<IN, true, true>, nblk, 8), kThreads, 0, st>>>(
-                x, rows, cols, ld, codes, scales, ws, ocp);
+                x, rows, cols, ld, codes, scales, ws, ocp, tiled);
         else if (had)
             mxfp4_kernel<IN, true, false><<<grid_for(mxfp4_kernel<IN, true, false>, nblk, 8), kThreads, 0, st>>>(
-                x, rows, cols, ld, codes, scales, ws, ocp);
+                x, rows, cols, ld, codes, scales, ws, ocp, tiled);
         else if (sweep)
             mxfp4_kernel<IN, false, true><<<grid_for(mxfp4_kernel<IN, false, true>, nblk, 8), kThreads, 0, st>>>(
-                x, rows, cols, ld, codes, scales, ws, ocp);
+                x, rows, cols, ld, codes, scales, ws, ocp, tiled);
         else
             mxfp4_kernel<IN, false, false><<<grid_for(mxfp4_kernel<IN, false, false>, nblk, 8), kThreads, 0, st>>>(
-                x, rows, cols, ld, codes, scales, ws, ocp);
+                x, rows, cols, ld, codes, scales, ws, ocp, tiled);
         return launched(1);
     }
     const bool had16 = (flags & FP4Q_F_HADAMARD16) != 0;
@@ -1107,19 +1129,20 @@ int noalloc_scratch(void** out) {
 
 template <bool HAD>
 void launch_dequant16(const uint8_t* codes, const uint8_t* scales, const float* gs, int64_t rows, int64_t cols,
-                      bool if4, bool bf, void* out, int g, cudaStream_t st) {
-    if (if4 && bf) dequant16_kernel<true, true, HAD><<<g, kThreads, 0, st>>>(codes, scales, gs, rows, cols, out);
-    else if (if4) dequant16_kernel<false, true, HAD><<<g, kThreads, 0, st>>>(codes, scales, gs, rows, cols, out);
-    else if (bf) dequant16_kernel<true, false, HAD><<<g, kThreads, 0, st>>>(codes, scales, gs, rows, cols, out);
-    else dequant16_kernel<false, false, HAD><<<g, kThreads, 0, st>>>(codes, scales, gs, rows, cols, out);
+                      bool if4, bool bf, void* out, int g, int tiled, cudaStream_t st) {
+    if (if4 && bf) dequant16_kernel<true, true, HAD><<<g, kThreads, 0, st>>>(codes, scales, gs, rows, cols, out, tiled);
+    else if (if4) dequant16_kernel<false, true, HAD><<<g, kThreads, 0, st>>>(codes, scales, gs, rows, cols, out, tiled);
+    else if (bf) dequant16_kernel<true, false, HAD><<<g, kThreads, 0, st>>>(codes, scales, gs, rows, cols, out, tiled);
+    else dequant16_kernel<false, false, HAD><<<g, kThreads, 0, st>>>(codes, scales, gs, rows, cols, out, tiled);
 }
 
 // Format, objective and flag checks shared by fp4q_quantize and fp4q_quantize_noalloc.
 int check_quantize_args(int fmt, int objective, uint32_t flags) {
     if (fmt != FP4Q_NVFP4 && fmt != FP4Q_IF4 && fmt != FP4Q_MXFP4) return FP4Q_ERR_INVALID_ARG;
     if (flags & ~(FP4Q_F_GLOBAL_SCALE_GIVEN | FP4Q_F_MX_OCP_FLOOR | FP4Q_F_HADAMARD16 | FP4Q_F_HADAMARD32 |
-                  FP4Q_F_MX_SWEEP | FP4Q_F_IF4_SWEEP))
+                  FP4Q_F_MX_SWEEP | FP4Q_F_IF4_SWEEP | FP4Q_F_SCALE_TILED))
         return FP4Q_ERR_INVALID_ARG;
+    if ((flags & FP4Q_F_SCALE_TILED) && fmt == FP4Q_IF4) return FP4Q_ERR_UNSUPPORTED;
     if ((flags & FP4Q_F_IF4_SWEEP) && fmt != FP4Q_IF4) return FP4Q_ERR_UNSUPPORTED;
     if ((flags & FP4Q_F_MX_SWEEP) && (flags & FP4Q_F_MX_OCP_FLOOR)) return FP4Q_ERR_INVALID_ARG;
     if ((flags & FP4Q_F_MX_SWEEP) && fmt != FP4Q_MXFP4) return FP4Q_ERR_UNSUPPORTED;
@@ -1140,6 +1163,16 @@ using namespace fp4q;
 extern "C" {
 
 size_t fp4q_workspace_bytes(void) { return kWorkspaceBytes; }
+
+int64_t fp4q_scale_bytes(int64_t rows, int64_t cols, int fmt, uint32_t flags) {
+    if (fmt != FP4Q_NVFP4 && fmt != FP4Q_IF4 && fmt != FP4Q_MXFP4) return -1;
+    const int64_t B = fmt == FP4Q_MXFP4 ? 32 : 16;
+    if (rows < 0 || cols < 0 || cols % B) return -1;
+    if (rows > 0 && cols > 0 && rows > ((int64_t)1 << 40) / cols) return -1;
+    const int64_t J = cols / B;
+    if (!(flags & FP4Q_F_SCALE_TILED)) return rows * J;
+    return ((rows + 127) / 128) * 128 * ((J + 3) / 4) * 4;
+}
 
 int fp4q_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld, int fmt, int objective,
                   const float* importance, uint8_t* codes, uint8_t* scales, float* global_scale, void* workspace,
@@ -1205,7 +1238,7 @@ int fp4q_hadamard_quantize(const void* x, int dtype, int64_t rows, int64_t cols,
                            uint8_t* codes, uint8_t* scales, void* workspace, uint32_t flags, void* stream) {
     g_launches = 0;
     if (had_size != 32) return FP4Q_ERR_UNSUPPORTED;
-    if (flags & ~(FP4Q_F_MX_OCP_FLOOR | FP4Q_F_MX_SWEEP)) return FP4Q_ERR_INVALID_ARG;
+    if (flags & ~(FP4Q_F_MX_OCP_FLOOR | FP4Q_F_MX_SWEEP | FP4Q_F_SCALE_TILED)) return FP4Q_ERR_INVALID_ARG;
     return fp4q_quantize(x, dtype, rows, cols, ld, FP4Q_MXFP4, 0, nullptr, codes, scales, nullptr, workspace,
                          flags | FP4Q_F_HADAMARD32, stream);
 }
@@ -1214,7 +1247,9 @@ int fp4q_dequantize(const uint8_t* codes, const uint8_t* scales, const float* gl
                     int64_t cols, int fmt, int inverse_hadamard, void* out, uint32_t flags, void* stream) {
     g_launches = 0;
     if (fmt != FP4Q_NVFP4 && fmt != FP4Q_IF4 && fmt != FP4Q_MXFP4) return FP4Q_ERR_INVALID_ARG;
-    if (flags & ~FP4Q_F_OUT_BF16) return FP4Q_ERR_INVALID_ARG;
+    if (flags & ~(FP4Q_F_OUT_BF16 | FP4Q_F_SCALE_TILED)) return FP4Q_ERR_INVALID_ARG;
+    if ((flags & FP4Q_F_SCALE_TILED) && fmt == FP4Q_IF4) return FP4Q_ERR_UNSUPPORTED;
+    const int tiled = (flags & FP4Q_F_SCALE_TILED) ? 1 : 0;
     const int B = fmt == FP4Q_MXFP4 ? 32 : 16;
     if (rows < 0 || cols < 0 || cols % B) return FP4Q_ERR_SHAPE;
     if (rows > 0 && cols > 0 && rows > ((int64_t)1 << 40) / cols) return FP4Q_ERR_SHAPE;
@@ -1225,14 +1260,14 @@ int fp4q_dequantize(const uint8_t* codes, const uint8_t* scales, const float* gl
     const bool bf = (flags & FP4Q_F_OUT_BF16) != 0;
     const int g = grid_for(dequant_mx_kernel<false, true>, rows * (cols / B), 8);
     if (fmt == FP4Q_MXFP4) {
-        if (bf && inverse_hadamard) dequant_mx_kernel<true, true><<<g, kThreads, 0, st>>>(codes, scales, rows, cols, out);
-        else if (bf) dequant_mx_kernel<true, false><<<g, kThreads, 0, st>>>(codes, scales, rows, cols, out);
-        else if (inverse_hadamard) dequant_mx_kernel<false, true><<<g, kThreads, 0, st>>>(codes, scales, rows, cols, out);
-        else dequant_mx_kernel<false, false><<<g, kThreads, 0, st>>>(codes, scales, rows, cols, out);
+        if (bf && inverse_hadamard) dequant_mx_kernel<true, true><<<g, kThreads, 0, st>>>(codes, scales, rows, cols, out, tiled);
+        else if (bf) dequant_mx_kernel<true, false><<<g, kThreads, 0, st>>>(codes, scales, rows, cols, out, tiled);
+        else if (inverse_hadamard) dequant_mx_kernel<false, true><<<g, kThreads, 0, st>>>(codes, scales, rows, cols, out, tiled);
+        else dequant_mx_kernel<false, false><<<g, kThreads, 0, st>>>(codes, scales, rows, cols, out, tiled);
     } else if (inverse_hadamard) {
-        launch_dequant16<true>(codes, scales, global_scale, rows, cols, fmt == FP4Q_IF4, bf, out, g, st);
+        launch_dequant16<true>(codes, scales, global_scale, rows, cols, fmt == FP4Q_IF4, bf, out, g, tiled, st);
     } else {
-        launch_dequant16<false>(codes, scales, global_scale, rows, cols, fmt == FP4Q_IF4, bf, out, g, st);
+        launch_dequant16<false>(codes, scales, global_scale, rows, cols, fmt == FP4Q_IF4, bf, out, g, tiled, st);
     }
     return launched(1);
 }

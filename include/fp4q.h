@@ -99,12 +99,30 @@ enum { FP4Q_ABSMAX = 0, FP4Q_FOUR_OVER_SIX = 1, FP4Q_SWEEP_MSE = 2, FP4Q_SWEEP_W
                                            MX scale sweep -- each block's exponent is the one
                                            among e_c-2 .. e_c (e_c = the ceil rule) with the
                                            lowest block error; not with FP4Q_F_MX_OCP_FLOOR    */
+#define FP4Q_F_SCALE_TILED        0x80u /* NVFP4/MXFP4 quantize and dequantize: scale bytes in the
+                                           128x4-tiled layout of block-scaled tensor-core GEMMs
+                                           (see fp4q_scale_bytes) instead of row-major         */
 #define FP4Q_F_IF4_SWEEP          0x40u /* IF4 quantize: IF4 x ScaleSweep -- the block scale and
                                            the element type are chosen together over the MSE
                                            window p0-3 .. p0+7 (see the arithmetic above)      */
 
 /* Size in bytes of the workspace every quantize call needs (a small constant). */
 size_t fp4q_workspace_bytes(void);
+
+/*
+ * Size in bytes of the scales buffer of a rows x cols tensor in format fmt: rows * cols/B
+ * row-major, or with FP4Q_F_SCALE_TILED in flags the tiled layout that block-scaled tensor-core
+ * GEMMs (the consumer of these codes and scales on B200) read: the [rows][cols/B] scale matrix
+ * padded to whole tiles of 128 rows x 4 scale columns (512 bytes each), tiles row-major over
+ * (row/128, col/4), and inside a tile the scale of row r, column c at byte
+ * 16*(r%32) + 4*((r/32)%4) + c%4.  A quantize call writes only the entries of real blocks; the
+ * padding keeps whatever the caller put there (zero it if the consumer reads it).  The pages
+ * give no scale layout; this one is the public layout of NVIDIA's block-scaled GEMMs
+ * (cuBLASLt's "32x4x4" scale-factor tiles), kept byte for byte so that a GEMM can read the
+ * scales as written.  IF4 has no tiled form (its indicator bit is not a consumer format).
+ * Returns -1 for an unknown format or a bad shape.
+ */
+int64_t fp4q_scale_bytes(int64_t rows, int64_t cols, int fmt, uint32_t flags);
 
 /*
  * Quantize x into codes + scales (+ S).
@@ -119,7 +137,9 @@ size_t fp4q_workspace_bytes(void);
  *   FP4Q_F_HADAMARD32 (MXFP4 only, else FP4Q_ERR_UNSUPPORTED; identical to
  *   fp4q_hadamard_quantize), FP4Q_F_MX_SWEEP (MXFP4 only, else FP4Q_ERR_UNSUPPORTED;
  *   with FP4Q_F_MX_OCP_FLOOR: FP4Q_ERR_INVALID_ARG), FP4Q_F_IF4_SWEEP (IF4 only, else
- *   FP4Q_ERR_UNSUPPORTED; combines with FP4Q_F_HADAMARD16 and FP4Q_F_GLOBAL_SCALE_GIVEN).
+ *   FP4Q_ERR_UNSUPPORTED; combines with FP4Q_F_HADAMARD16 and FP4Q_F_GLOBAL_SCALE_GIVEN),
+ *   FP4Q_F_SCALE_TILED (NVFP4 and MXFP4: scales in the tiled layout of fp4q_scale_bytes; IF4:
+ *   FP4Q_ERR_UNSUPPORTED).
  * FP4Q_F_HADAMARD16: every 16-element block is first rotated by the normalized Sylvester
  *   Hadamard matrix H_16 / 4 (butterflies h = 1, 2, 4, 8 in binary32, then one exact
  *   multiplication by 1/4 per value), and the whole method -- S, the block scales, the
@@ -216,7 +236,8 @@ int fp4q_quantize_host_async(const void* x_host, int dtype, int64_t rows, int64_
  * inverse_hadamard: apply the normalized transform of the format's block size (32-point for
  * MXFP4, 16-point H_16 / 4 for NVFP4/IF4) to each dequantized block, as butterflies then
  * one multiplication per value (it is its own inverse up to rounding).  global_scale is a device
- * pointer (ignored for MXFP4).  out must be 16-byte aligned.
+ * pointer (ignored for MXFP4).  out must be 16-byte aligned.  flags: FP4Q_F_OUT_BF16 and
+ * FP4Q_F_SCALE_TILED (scales in the tiled layout of fp4q_scale_bytes; NVFP4 and MXFP4).
  */
 int fp4q_dequantize(const uint8_t* codes, const uint8_t* scales, const float* global_scale,
                     int64_t rows, int64_t cols, int fmt, int inverse_hadamard,

@@ -223,6 +223,23 @@ def dequantize(codes, scales, S, fmt, inverse_hadamard=False, out_bf16=False):
     return out
 
 
+def tile_scales(scales) -> np.ndarray:
+    """Row-major [rows][J] scale bytes -> the 1-D tiled layout block-scaled tensor-core GEMMs read
+    (the library's FP4Q_F_SCALE_TILED): the matrix padded with zeros to whole 128-row x 4-column
+    tiles of 512 bytes, tiles in row-major order over (row / 128, column / 4), and inside a tile
+    the byte of row r, column c at 16 * (r % 32) + 4 * ((r // 32) % 4) + c % 4.  Written as the
+    plain element-by-element placement."""
+    scales = np.asarray(scales, np.uint8)
+    rows, J = scales.shape
+    rt, jt = (rows + 127) // 128, (J + 3) // 4
+    out = np.zeros(rt * 128 * jt * 4, np.uint8)
+    for r in range(rows):
+        for c in range(J):
+            off = (r // 128) * (jt * 512) + (c // 4) * 512 + (r % 32) * 16 + ((r // 32) % 4) * 4 + c % 4
+            out[off] = scales[r, c]
+    return out
+
+
 def widen_bf16(bits) -> np.ndarray:
     """bf16 bit patterns -> float32 (exact), the oracle's own input widening."""
     b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)

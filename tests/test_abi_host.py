@@ -27,6 +27,18 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(L, name), name
 
 
+def test_scale_bytes():
+    # row-major: rows * cols/B; tiled: padded to 128-row x 4-column tiles of 512 bytes
+    assert fq.scale_bytes(256, 1024, "nvfp4") == 256 * 64
+    assert fq.scale_bytes(256, 1024, "nvfp4", tiled=True) == 256 * 64
+    assert fq.scale_bytes(100, 48, "nvfp4", tiled=True) == 128 * 4          # 3 scale columns -> 4
+    assert fq.scale_bytes(129, 80, "nvfp4", tiled=True) == 256 * 8          # 5 scale columns -> 8
+    assert fq.scale_bytes(300, 8192, "mxfp4", tiled=True) == 384 * 256
+    assert fq.scale_bytes(0, 64, "mxfp4", tiled=True) == 0
+    L = fq.lib()
+    assert L.fp4q_scale_bytes(4, 24, 0, 0) == -1 and L.fp4q_scale_bytes(4, 32, 7, 0) == -1
+
+
 def test_status_strings_and_workspace():
     assert fq.status_string(0) == "ok"
     for rc in range(1, 6):
@@ -55,7 +67,8 @@ FAKE = 0x10000   # 16-byte aligned non-null stand-in; validation rejects before 
     ((FAKE, 1, 4, 32, 36, 0, 2, None, FAKE, FAKE, FAKE, FAKE, 0), fq.ERR_ALIGNMENT),    # row pitch 72 B
     ((FAKE, 1, 4, 32, 32, 0, 2, None, FAKE + 4, FAKE, FAKE, FAKE, 0), fq.ERR_ALIGNMENT),  # codes
     ((FAKE, 1, 4, 32, 32, 0, 3, FAKE + 4, FAKE, FAKE, FAKE, FAKE, 0), fq.ERR_ALIGNMENT),  # weights
-    ((FAKE, 1, 4, 32, 32, 0, 2, None, FAKE, FAKE, FAKE, FAKE, 0x80), fq.ERR_INVALID_ARG),  # unknown flag
+    ((FAKE, 1, 4, 32, 32, 0, 2, None, FAKE, FAKE, FAKE, FAKE, 0x100), fq.ERR_INVALID_ARG),  # unknown flag
+    ((FAKE, 1, 4, 32, 32, 1, 0, None, FAKE, FAKE, FAKE, FAKE, 0x80), fq.ERR_UNSUPPORTED),  # tiled scales, IF4
     ((FAKE, 1, 4, 32, 32, 2, 0, None, FAKE, FAKE, None, FAKE, 1), fq.ERR_INVALID_ARG),  # MX with given S
     ((FAKE, 1, 4, 32, 32, 0, 2, None, FAKE, FAKE, FAKE, FAKE, 0x40), fq.ERR_UNSUPPORTED),  # IF4 sweep, NVFP4
     ((FAKE, 1, 4, 64, 64, 2, 0, None, FAKE, FAKE, None, FAKE, 0x40), fq.ERR_UNSUPPORTED),  # IF4 sweep, MXFP4
@@ -129,7 +142,7 @@ def test_host_async_validation():
     assert call(obj=3) == fq.ERR_INVALID_ARG                     # WMSE without weights
     assert call(x_dev=FAKE + 8) == fq.ERR_ALIGNMENT
     assert call(flags=0x8, fmt=2, cols=64) == fq.ERR_UNSUPPORTED  # 16-point rotation on MXFP4
-    assert call(flags=0x80) == fq.ERR_INVALID_ARG
+    assert call(flags=0x100) == fq.ERR_INVALID_ARG
     assert call(flags=0x40) == fq.ERR_UNSUPPORTED                 # IF4 sweep on NVFP4
     assert call(flags=0x20) == fq.ERR_UNSUPPORTED                 # MX sweep on NVFP4
     assert call(rows=0, x_host=None, x_dev=None) == fq.OK and L.fp4q_last_launch_count() == 0

@@ -424,6 +424,25 @@ def test_if4_sweep_dominates_if4_and_the_nvfp4_sweep():
         assert (chosen < nv["err"]).any() and (chosen < at_p0).any()
 
 
+@pytest.mark.parametrize("rows,J", [(128, 4), (256, 64), (200, 6), (1, 1), (130, 257)])
+def test_tiled_scale_layout(rows, J):
+    # The consumer layout restated as NVIDIA's block-scaled GEMMs describe it: pad to 128 x 4 tiles,
+    # view each tile's 128 rows as 4 groups of 32, and store (tile row, tile column, row-in-group,
+    # group, column) -- a reshape and an axis permutation, independent of the oracle's loop.
+    rng = np.random.default_rng(rows * 1000 + J)
+    sc = rng.integers(1, 255, size=(rows, J), dtype=np.uint8)
+    got = O.tile_scales(sc)
+    rt, jt = (rows + 127) // 128, (J + 3) // 4
+    pad = np.zeros((rt * 128, jt * 4), np.uint8)
+    pad[:rows, :J] = sc
+    want = pad.reshape(rt, 4, 32, jt, 4).transpose(0, 3, 2, 1, 4).ravel()
+    assert np.array_equal(got, want)
+    # a bijection of the padded matrix onto the buffer: every byte placed once
+    ids = np.arange(rt * 128 * jt * 4).reshape(rt * 128, jt * 4)
+    placed = ids.reshape(rt, 4, 32, jt, 4).transpose(0, 3, 2, 1, 4).ravel()
+    assert np.array_equal(np.sort(placed), np.arange(placed.size))
+
+
 def test_hadamard_is_normalized_sylvester():
     H = np.array([[1.0]])
     while H.shape[0] < 32:
