@@ -240,6 +240,24 @@ def tile_scales(scales) -> np.ndarray:
     return out
 
 
+def nvfp4_gemm(a_codes, a_scales, Sa, b_codes, b_scales, Sb):
+    """D[m][n] = Sa * Sb * sum_k qa[m][k] e(pa[m][k/16]) qb[n][k] e(pb[n][k/16]) in float64: the
+    product of two NVFP4 operands stored with K contiguous (codes [rows][K/2], row-major scale
+    bytes [rows][K/16]), every element value q * e(p) formed from the oracle's own code tables.
+    Each term is exact in float64 and the sums are a float64 matmul."""
+    def values(codes, scales):
+        codes = np.asarray(codes, np.uint8)
+        rows, half = codes.shape
+        q = np.empty((rows, 2 * half), np.float64)
+        tab = np.array([lib().fp4q_o_e2m1_value(c) for c in range(16)], np.float64)
+        q[:, 0::2] = tab[codes & 0xF]
+        q[:, 1::2] = tab[codes >> 4]
+        e = np.array([lib().fp4q_o_e4m3_value(p) for p in range(128)], np.float64)
+        sc = e[np.asarray(scales, np.uint8) & 0x7F]
+        return q * np.repeat(sc, 16, axis=1)
+    return float(Sa) * float(Sb) * (values(a_codes, a_scales) @ values(b_codes, b_scales).T)
+
+
 def widen_bf16(bits) -> np.ndarray:
     """bf16 bit patterns -> float32 (exact), the oracle's own input widening."""
     b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)

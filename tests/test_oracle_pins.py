@@ -443,6 +443,29 @@ def test_tiled_scale_layout(rows, J):
     assert np.array_equal(np.sort(placed), np.arange(placed.size))
 
 
+def test_nvfp4_gemm_oracle():
+    # against a triple loop over exact rationals on a tiny problem, and against the float64
+    # product of the dequantized operands (each dequantized value is one rounding of the exact one)
+    rng = np.random.default_rng(5)
+    a = rng.normal(size=(3, 32)).astype(np.float32)
+    b = rng.normal(size=(2, 32)).astype(np.float32)
+    ra, rb = O.nvfp4_quantize(a, "sweep_mse"), O.nvfp4_quantize(b, "sweep_mse")
+    d = O.nvfp4_gemm(ra["codes"], ra["scales"], ra["S"], rb["codes"], rb["scales"], rb["S"])
+    def val(codes, scales, S, r, k):
+        c = (int(codes[r, k // 2]) >> (4 * (k % 2))) & 0xF
+        g = GRID[c & 7] * (-1 if c & 8 else 1)
+        return g * E4M3[int(scales[r, k // 16])] * Fr(S)
+    for m in range(3):
+        for n in range(2):
+            exact = sum(val(ra["codes"], ra["scales"], ra["S"], m, k) * val(rb["codes"], rb["scales"], rb["S"], n, k)
+                        for k in range(32))
+            assert abs(d[m, n] - float(exact)) <= 1e-12 * max(1.0, abs(float(exact)))
+    da = O.dequantize(ra["codes"], ra["scales"], ra["S"], "nvfp4").astype(np.float64)
+    db = O.dequantize(rb["codes"], rb["scales"], rb["S"], "nvfp4").astype(np.float64)
+    mag = np.abs(da) @ np.abs(db).T
+    assert np.all(np.abs(d - da @ db.T) <= 2 ** -22 * mag)
+
+
 def test_hadamard_is_normalized_sylvester():
     H = np.array([[1.0]])
     while H.shape[0] < 32:
