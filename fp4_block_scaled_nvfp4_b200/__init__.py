@@ -17,7 +17,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfp4q.so")
 
 OK, ERR_INVALID_ARG, ERR_SHAPE, ERR_ALIGNMENT, ERR_UNSUPPORTED, ERR_CUDA = range(6)
-DEVSTAT_OK, DEVSTAT_NONFINITE, DEVSTAT_RANGE = 0, 1, 2
+DEVSTAT_OK, DEVSTAT_NONFINITE, DEVSTAT_RANGE, DEVSTAT_TIMEOUT = 0, 1, 2, 4
 IN_F32, IN_BF16 = 0, 1
 FORMATS = {"nvfp4": 0, "if4": 1, "mxfp4": 2}
 OBJECTIVES = {"absmax": 0, "four_over_six": 1, "sweep_mse": 2, "sweep_wmse": 3}
@@ -27,7 +27,7 @@ F_SCALE_TILED = 0x80
 BLOCK = {"nvfp4": 16, "if4": 16, "mxfp4": 32}
 
 # Names of every function include/fp4q.h declares (checked against the header by the tests).
-EXPORTS = ("fp4q_workspace_bytes", "fp4q_scale_bytes", "fp4q_global_scale", "fp4q_hadamard_global_scale", "fp4q_quantize",
+EXPORTS = ("fp4q_workspace_bytes", "fp4q_scale_bytes", "fp4q_nvfp4_gemm", "fp4q_global_scale", "fp4q_hadamard_global_scale", "fp4q_quantize",
            "fp4q_hadamard_quantize", "fp4q_dequantize", "fp4q_quantize_noalloc", "fp4q_quantize_host_async", "fp4q_read_device_status", "fp4q_last_launch_count", "fp4q_status_string")
 
 _lib = None
@@ -49,6 +49,8 @@ def lib():
         L.fp4q_workspace_bytes.argtypes = []
         L.fp4q_scale_bytes.restype = i64
         L.fp4q_scale_bytes.argtypes = [i64, i64, i32, u32]
+        L.fp4q_nvfp4_gemm.restype = i32
+        L.fp4q_nvfp4_gemm.argtypes = [P, P, P, P, P, P, i64, i64, i64, P, i64, P, P]
         L.fp4q_quantize.restype = i32
         L.fp4q_quantize.argtypes = [P, i32, i64, i64, i64, i32, i32, P, P, P, P, P, u32, P]
         L.fp4q_global_scale.restype = i32
@@ -239,6 +241,25 @@ def quantize_noalloc(x, fmt: str = "nvfp4", objective: str = "sweep_mse", import
                                      _stream_ptr(stream))
     _check(rc, "fp4q_quantize_noalloc")
     return codes, scales, (gs if fmt != "mxfp4" else None)
+
+
+def nvfp4_gemm(a, b, out=None, workspace=None, stream=None):
+    """Block-scaled NVFP4 GEMM on the tensor cores: a = (codes [M, K/2], tiled scales, S) and
+    b = (codes [N, K/2], tiled scales, S) as returned by quantize(..., tiled_scales=True);
+    returns fp32 [M, N] = S_a S_b A B^T.  M, N multiples of 128, K a multiple of 256."""
+    torch = _torch()
+    ac, asc, ag = a
+    bc, bsc, bg = b
+    M, K = ac.shape[0], ac.shape[1] * 2
+    N = bc.shape[0]
+    if bc.shape[1] * 2 != K:
+        raise Fp4qError("a and b must have the same K")
+    d = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=ac.device)
+    ws = workspace if workspace is not None else new_workspace(ac.device)
+    rc = lib().fp4q_nvfp4_gemm(_ptr(ac), _ptr(asc), _ptr(ag), _ptr(bc), _ptr(bsc), _ptr(bg), M, N, K, _ptr(d),
+                               d.stride(0), _ptr(ws), _stream_ptr(stream))
+    _check(rc, "fp4q_nvfp4_gemm")
+    return d
 
 
 def read_device_status(workspace, stream=None) -> int:

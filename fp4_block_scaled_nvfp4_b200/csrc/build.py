@@ -6,7 +6,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 PKG = os.path.dirname(HERE)
 ROOT = os.path.dirname(PKG)
-SRCS = [os.path.join(HERE, "fp4q.cu")]
+SRCS = [os.path.join(HERE, "fp4q.cu"), os.path.join(HERE, "fp4q_gemm.cu")]
 DEPS = SRCS + [os.path.join(HERE, "fp4q_device.cuh"), os.path.join(ROOT, "include", "fp4q.h")]
 LIB = os.path.join(PKG, "libfp4q.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -1,0 +1,232 @@
+// fp4q_gemm.cu -- block-scaled NVFP4 GEMM on the sm_100a tensor cores (tcgen05), the consumer
+// of the quantizer's outputs: D[m][n] = S_a S_b sum_k A[m][k] B[n][k], with A and B NVFP4
+// tensors stored exactly as fp4q_quantize writes them (codes [rows][K/2], element 2j in the
+// low nibble; E4M3 scales in the 128x4-tiled layout of FP4Q_F_SCALE_TILED; one fp32 tensor
+// scale each).  Both operands have K contiguous.
+//
+// One CTA of 128 threads computes a 128 x 128 tile of D:
+//   * per K stage of 256 elements, all threads copy the A and B tiles (128 rows x 128 bytes
+//     each) into shared memory in the 128-byte-swizzled K-major layout the MMA descriptor
+//     describes, and the four 512-byte scale-factor atoms of each operand as they are;
+//   * one thread moves the scale atoms into tensor memory (tcgen05.cp 32x128b, broadcast to
+//     the four lane quarters) and issues four block-scaled MMAs of K = 64
+//     (tcgen05.mma kind::mxf4nvf4, 16-element scale blocks) accumulating in tensor memory,
+//     then commits them to an mbarrier that every thread waits on (bounded) before the shared
+//     buffers are refilled;
+//   * the epilogue reads the fp32 accumulator back with tcgen05.ld (each warp its 32 lanes),
+//     multiplies by S_a S_b and stores D.
+// A wait that runs out sets FP4Q_DEVSTAT_TIMEOUT in the status word, skips the rest of the
+// work, and still frees the CTA's tensor memory.
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "fp4q.h"
+
+namespace fp4q {
+
+extern thread_local int g_launches;
+
+namespace gemm {
+
+constexpr int kTM = 128, kTN = 128, kTK = 256;     // CTA tile and K per stage
+constexpr int kThreads = 128;
+constexpr uint32_t kTmemCols = 256;                // accumulator 128 + scale factors 16 + 16
+constexpr uint32_t kColSFA = 128, kColSFB = 144;
+constexpr int kTileBytes = kTM * kTK / 2;          // 16 KB of codes per operand and stage
+constexpr int kSfBytes = 4 * 512;                  // four 128x4 scale atoms per operand and stage
+constexpr int kSmemBytes = 2 * kTileBytes + 2 * kSfBytes + 64;
+// The request is padded so that at most two CTAs share an SM: two allocations of 256 tensor
+// memory columns fill the 512 an SM has, so no allocation ever waits for another CTA.
+constexpr int kSmemAlloc = (kSmemBytes + 1024) > 100 * 1024 ? (kSmemBytes + 1024) : 100 * 1024;
+constexpr uint32_t kWaitPolls = 1u << 22;          // bounded mbarrier wait
+
+// Shared-memory matrix descriptor (sm_100 tensor-core operand): start address, leading and
+// stride byte offsets in 16-byte units, descriptor version 1, and the layout type in bits
+// 61..63 (0 = no swizzle, 2 = 128-byte swizzle).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
+    return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | ((uint64_t)1 << 46) | ((uint64_t)layout << 61);
+}
+
+// Instruction descriptor of the block-scaled FP4 MMA: E2M1 A and B (format 1), K-major
+// operands, N / 8 in bits 17..22, UE4M3 scale factors (bit 23 = 0), M / 16 in bits 24..28,
+// dense K = 64.
+constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(kTN >> 3) << 17) | ((uint32_t)(kTM >> 4) << 24);
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+    for (uint32_t i = 0; i < kWaitPolls; ++i) {
+        uint32_t done;
+        asm volatile(
+            "{ .reg .pred p;\n"
+            "  mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+            "  selp.u32 %0, 1, 0, p; }"
+            : "=r"(done) : "r"(bar), "r"(parity) : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    nvfp4_gemm_kernel(const uint8_t* __restrict__ a, const uint8_t* __restrict__ sfa, const float* __restrict__ sa,
+                      const uint8_t* __restrict__ b, const uint8_t* __restrict__ sfb, const float* __restrict__ sb,
+                      int K, float* __restrict__ d, int64_t ldd, uint32_t* __restrict__ status) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + kTileBytes;
+    uint8_t* sSFA = smem + 2 * kTileBytes;
+    uint8_t* sSFB = sSFA + kSfBytes;
+    uint64_t* mbar = reinterpret_cast<uint64_t*>(sSFB + kSfBytes);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mbar + 1);
+    __shared__ int s_fail;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t m0 = (int64_t)blockIdx.y * kTM, n0 = (int64_t)blockIdx.x * kTN;
+    const int64_t rowbytes = K / 2;
+    const int64_t jt = K / 64;                        // scale atoms per 128-row tile along K
+
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     :: "r"(smem_u32(tmem_slot)), "r"(kTmemCols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (tid == 0) {
+        s_fail = 0;
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" :: "r"(smem_u32(mbar)) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = *tmem_slot;
+
+    const int KT = K / kTK;
+    uint32_t parity = 0;
+    for (int kt = 0; kt < KT; ++kt) {
+        // operand tiles: 16-byte chunk c of row r goes to chunk c ^ (r % 8) of that row
+        const uint8_t* ga = a + m0 * rowbytes + (int64_t)kt * (kTK / 2);
+        const uint8_t* gb = b + n0 * rowbytes + (int64_t)kt * (kTK / 2);
+        for (int i = tid; i < kTM * 8; i += kThreads) {
+            const int r = i >> 3, c = i & 7;
+            const uint4 va = __ldg(reinterpret_cast<const uint4*>(ga + r * rowbytes + c * 16));
+            const uint4 vb = __ldg(reinterpret_cast<const uint4*>(gb + r * rowbytes + c * 16));
+            *reinterpret_cast<uint4*>(sA + r * 128 + ((c ^ (r & 7)) << 4)) = va;
+            *reinterpret_cast<uint4*>(sB + r * 128 + ((c ^ (r & 7)) << 4)) = vb;
+        }
+        // scale atoms of this stage: atoms 4 kt .. 4 kt + 3 of the row tile, contiguous
+        {
+            const uint4* gsa = reinterpret_cast<const uint4*>(sfa + ((int64_t)blockIdx.y * jt + 4 * kt) * 512);
+            const uint4* gsb = reinterpret_cast<const uint4*>(sfb + ((int64_t)blockIdx.x * jt + 4 * kt) * 512);
+            reinterpret_cast<uint4*>(sSFA)[tid] = __ldg(gsa + tid);
+            reinterpret_cast<uint4*>(sSFB)[tid] = __ldg(gsb + tid);
+        }
+        // the tensor core reads shared memory through the async proxy
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncthreads();
+        if (tid == 0) {
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t da = smem_desc(smem_u32(sSFA + kk * 512), 16, 128, 0);
+                const uint64_t db = smem_desc(smem_u32(sSFB + kk * 512), 16, 128, 0);
+                asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" :: "r"(tmem + kColSFA + 4 * kk), "l"(da)
+                             : "memory");
+                asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" :: "r"(tmem + kColSFB + 4 * kk), "l"(db)
+                             : "memory");
+            }
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t adesc = smem_desc(smem_u32(sA + kk * 32), 16, 1024, 2);
+                const uint64_t bdesc = smem_desc(smem_u32(sB + kk * 32), 16, 1024, 2);
+                const uint32_t accumulate = (kt > 0 || kk > 0) ? 1u : 0u;
+                asm volatile(
+                    "{ .reg .pred p;\n"
+                    "  setp.ne.b32 p, %4, 0;\n"
+                    "  tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p; }"
+                    :: "r"(tmem), "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate),
+                       "r"(tmem + kColSFA + 4 * kk), "r"(tmem + kColSFB + 4 * kk)
+                    : "memory");
+            }
+            asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                         :: "r"(smem_u32(mbar)) : "memory");
+        }
+        // the MMAs have read the shared tiles before anyone refills them
+        if (!mbar_wait(smem_u32(mbar), parity)) s_fail = 1;
+        parity ^= 1u;
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        __syncthreads();
+        if (s_fail) break;
+    }
+
+    if (!s_fail) {
+        const float scale = __fmul_rn(*sa, *sb);
+        float* drow = d + (m0 + warp * 32 + lane) * ldd + n0;
+#pragma unroll 1
+        for (int c0 = 0; c0 < kTN; c0 += 32) {
+            uint32_t v[32];
+            asm volatile(
+                "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+                "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+                "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+                : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+                  "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
+                  "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
+                  "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
+                  "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+                : "r"(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0)
+                : "memory");
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+                *reinterpret_cast<float4*>(drow + c0 + j) =
+                    make_float4(__fmul_rn(__uint_as_float(v[j]), scale), __fmul_rn(__uint_as_float(v[j + 1]), scale),
+                                __fmul_rn(__uint_as_float(v[j + 2]), scale), __fmul_rn(__uint_as_float(v[j + 3]), scale));
+        }
+    } else if (tid == 0) {
+        atomicOr(status, (uint32_t)FP4Q_DEVSTAT_TIMEOUT);
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(kTmemCols) : "memory");
+}
+
+}  // namespace gemm
+}  // namespace fp4q
+
+extern "C" int fp4q_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global_scale,
+                               const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global_scale,
+                               int64_t M, int64_t N, int64_t K, float* d, int64_t ldd, void* workspace,
+                               void* stream) {
+    using namespace fp4q;
+    g_launches = 0;
+    if (M < 0 || N < 0 || K < 0 || M % gemm::kTM || N % gemm::kTN || K % gemm::kTK || ldd < N) return FP4Q_ERR_SHAPE;
+    if (M / gemm::kTM > 65535 || K > (1 << 30)) return FP4Q_ERR_SHAPE;
+    if (M == 0 || N == 0 || K == 0) return FP4Q_OK;
+    if (!a_codes || !a_scales || !a_global_scale || !b_codes || !b_scales || !b_global_scale || !d || !workspace)
+        return FP4Q_ERR_INVALID_ARG;
+    auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+    if (!al16(a_codes) || !al16(a_scales) || !al16(b_codes) || !al16(b_scales) || !al16(d) || !al16(workspace) ||
+        ldd % 4)
+        return FP4Q_ERR_ALIGNMENT;
+    static bool attr_set = false;
+    if (!attr_set) {
+        if (cudaFuncSetAttribute(gemm::nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 gemm::kSmemAlloc) != cudaSuccess)
+            return FP4Q_ERR_CUDA;
+        attr_set = true;
+    }
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t* status = reinterpret_cast<uint32_t*>(workspace);
+    if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return FP4Q_ERR_CUDA;
+    const dim3 grid((unsigned)(N / gemm::kTN), (unsigned)(M / gemm::kTM));
+    gemm::nvfp4_gemm_kernel<<<grid, gemm::kThreads, gemm::kSmemAlloc, st>>>(
+        a_codes, a_scales, a_global_scale, b_codes, b_scales, b_global_scale, (int)K, d, ldd, status);
+    if (cudaGetLastError() != cudaSuccess) return FP4Q_ERR_CUDA;
+    g_launches = 1;
+    return FP4Q_OK;
+}

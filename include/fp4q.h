@@ -83,7 +83,9 @@ typedef enum {
     FP4Q_ERR_CUDA = 5           /* a CUDA launch or runtime call failed                      */
 } fp4q_status;
 
-enum { FP4Q_DEVSTAT_OK = 0, FP4Q_DEVSTAT_NONFINITE = 1, FP4Q_DEVSTAT_RANGE = 2 };
+/* Device status bits.  TIMEOUT: fp4q_nvfp4_gemm gave up a bounded wait for its tensor-core
+ * work (its output is then incomplete). */
+enum { FP4Q_DEVSTAT_OK = 0, FP4Q_DEVSTAT_NONFINITE = 1, FP4Q_DEVSTAT_RANGE = 2, FP4Q_DEVSTAT_TIMEOUT = 4 };
 enum { FP4Q_IN_F32 = 0, FP4Q_IN_BF16 = 1 };
 enum { FP4Q_NVFP4 = 0, FP4Q_IF4 = 1, FP4Q_MXFP4 = 2 };
 enum { FP4Q_ABSMAX = 0, FP4Q_FOUR_OVER_SIX = 1, FP4Q_SWEEP_MSE = 2, FP4Q_SWEEP_WMSE = 3 };
@@ -276,6 +278,27 @@ int fp4q_last_launch_count(void);
 
 /* Static description of a status code. */
 const char* fp4q_status_string(int status);
+
+/*
+ * Block-scaled NVFP4 GEMM on the B200 tensor cores (tcgen05), the consumer of two quantized
+ * operands: d[m][n] = S_a * S_b * sum_k A[m][k] * B[n][k] in fp32, where A (M x K) and B (N x K)
+ * are NVFP4 tensors exactly as fp4q_quantize writes them with FP4Q_F_SCALE_TILED:
+ *   a_codes [M][K/2], b_codes [N][K/2] (K contiguous, element 2j in the low nibble),
+ *   a_scales, b_scales: E4M3 scale bytes in the tiled layout of fp4q_scale_bytes,
+ *   a_global_scale, b_global_scale: device pointers to the two tensor scales S.
+ * Every product of two element values q_a e_a * q_b e_b is formed exactly by the tensor core
+ * and accumulated in fp32; the result is multiplied by RN(S_a S_b) once.  The pages give no
+ * GEMM: this is the step after the quantizer (Bridging the Gap ... Microscaling FP4,
+ * "Methodology", the FP4 GEMM kernels whose operands the quantizer produces).
+ * d: fp32 [M][ldd], ldd >= N, ldd a multiple of 4; all pointers device memory, 16-byte
+ * aligned.  M and N multiples of 128, K a multiple of 256 (FP4Q_ERR_SHAPE otherwise).
+ * workspace: fp4q_workspace_bytes() bytes; its word 0 receives the device status
+ * (FP4Q_DEVSTAT_TIMEOUT if a bounded wait for the tensor cores ran out).  One launch.
+ */
+int fp4q_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global_scale,
+                    const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global_scale,
+                    int64_t M, int64_t N, int64_t K, float* d, int64_t ldd, void* workspace,
+                    void* stream);
 
 #ifdef __cplusplus
 }

@@ -39,6 +39,23 @@ def test_scale_bytes():
     assert L.fp4q_scale_bytes(4, 24, 0, 0) == -1 and L.fp4q_scale_bytes(4, 32, 7, 0) == -1
 
 
+def test_gemm_rejects_before_launch():
+    L = fq.lib()
+    F = FAKE
+    call = lambda M, N, K, ldd=None, **kw: L.fp4q_nvfp4_gemm(kw.get("a", F), F, F, F, F, F, M, N, K,
+                                                             kw.get("d", F), N if ldd is None else ldd,
+                                                             kw.get("ws", F), None)
+    assert call(100, 128, 256) == fq.ERR_SHAPE          # M % 128
+    assert call(128, 64, 256) == fq.ERR_SHAPE           # N % 128
+    assert call(128, 128, 128) == fq.ERR_SHAPE          # K % 256
+    assert call(128, 128, 256, ldd=64) == fq.ERR_SHAPE  # ldd < N
+    assert call(128, 128, 256, a=None) == fq.ERR_INVALID_ARG
+    assert call(128, 128, 256, ws=None) == fq.ERR_INVALID_ARG
+    assert call(128, 128, 256, d=F + 4) == fq.ERR_ALIGNMENT
+    assert call(128, 128, 256, ldd=130) == fq.ERR_ALIGNMENT
+    assert call(0, 128, 256, a=None, d=None, ws=None) == fq.OK and L.fp4q_last_launch_count() == 0
+
+
 def test_status_strings_and_workspace():
     assert fq.status_string(0) == "ok"
     for rc in range(1, 6):

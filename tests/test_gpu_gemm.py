@@ -1,0 +1,61 @@
+"""The block-scaled NVFP4 GEMM (fp4q_nvfp4_gemm, tcgen05 tensor cores) consuming the quantizer's
+codes and tiled scales, against the oracle's float64 product of the same operands: every product
+of two element values is exact, so the difference is the fp32 accumulation alone, bounded here by
+2e-5 of sum |a||b| per output."""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+import oracle as O
+import fp4_block_scaled_nvfp4_b200 as fq
+from fp4_block_scaled_nvfp4_b200 import synth
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    fq.lib()
+
+
+def _operand(cfg, rows, cols, obj):
+    w = synth.make(cfg, rows=rows, cols=cols)
+    xd = torch.from_numpy(w["x"].view(np.int16)).view(torch.bfloat16).cuda()
+    q = fq.quantize(xd, "nvfp4", obj, tiled_scales=True)
+    r = O.nvfp4_quantize(O.widen_bf16(w["x"]), obj)
+    return q, r
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 128, 256), (256, 384, 1024), (128, 256, 4096)])
+def test_nvfp4_gemm_matches_the_oracle_product(M, N, K):
+    (qa, ra), (qb, rb) = _operand("cfg3", M, K, "sweep_mse"), _operand("cfg2", N, K, "sweep_mse")
+    ws = fq.new_workspace()
+    d = fq.nvfp4_gemm(qa, qb, workspace=ws)
+    torch.cuda.synchronize()
+    assert fq.read_device_status(ws) == fq.DEVSTAT_OK
+    assert fq.last_launch_count() == 1
+    # the operands are the oracle's bit for bit (checked elsewhere); the product from its tables
+    assert np.array_equal(qa[0].cpu().numpy(), ra["codes"]) and np.array_equal(qb[0].cpu().numpy(), rb["codes"])
+    ref = O.nvfp4_gemm(ra["codes"], ra["scales"], ra["S"], rb["codes"], rb["scales"], rb["S"])
+    da = O.dequantize(ra["codes"], ra["scales"], ra["S"], "nvfp4").astype(np.float64)
+    db = O.dequantize(rb["codes"], rb["scales"], rb["S"], "nvfp4").astype(np.float64)
+    mag = np.abs(da) @ np.abs(db).T
+    got = d.cpu().numpy().astype(np.float64)
+    err = np.abs(got - ref)
+    assert np.all(err <= 2e-5 * mag + 1e-30), float(np.max(err / (mag + 1e-30)))
+
+
+def test_nvfp4_gemm_other_objectives_and_padding_rows():
+    # AbsMax and 4/6 operands, and an output with a row pitch wider than N
+    (qa, ra), (qb, rb) = _operand("cfg3", 128, 512, "absmax"), _operand("cfg4", 128, 512, "four_over_six")
+    d = torch.full((128, 160), 7.0, device="cuda")
+    fq.nvfp4_gemm(qa, qb, out=d[:, :128])
+    torch.cuda.synchronize()
+    ref = O.nvfp4_gemm(ra["codes"], ra["scales"], ra["S"], rb["codes"], rb["scales"], rb["S"])
+    da = O.dequantize(ra["codes"], ra["scales"], ra["S"], "nvfp4").astype(np.float64)
+    db = O.dequantize(rb["codes"], rb["scales"], rb["S"], "nvfp4").astype(np.float64)
+    got = d.cpu().numpy()
+    assert np.all(np.abs(got[:, :128] - ref) <= 2e-5 * (np.abs(da) @ np.abs(db).T) + 1e-30)
+    assert np.all(got[:, 128:] == 7.0)
