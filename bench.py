@@ -49,6 +49,11 @@ WORKLOADS = {
     "cfg4h": ("cfg4", "if4_had", None, "IF4 on 16x16 block-Hadamard-rotated blocks, bf16 weight 4096x14336"),
 }
 METRIC = "quantize GB/s (input bf16) and % of B200 HBM peak, 1 GPU, vs CPU oracle"
+# The consumer of the quantized operands (--workload gemm): the block-scaled NVFP4 GEMM on the
+# tcgen05 tensor cores, activations [M][K] (the 8192x4096 activation workload) times a weight
+# [N][K] (Llama-3-8B-shaped MLP up-projection, 14336x4096, Student-t weights), K contiguous.
+GEMM_METRIC = "NVFP4 block-scaled GEMM TFLOP/s (tcgen05), 1 GPU"
+GEMM_SHAPE = (8192, 14336, 4096)
 # Arithmetic the method itself needs per element for the ALU-bound searches: per candidate
 # scale one multiply (x/s), one E2M1 rounding, one subtraction (residual) and one fused
 # multiply-add (square-accumulate) -- plus, for WMSE, the weight multiply -- over 11 (MSE) or
@@ -197,6 +202,8 @@ def cpu_baseline(w, fmt, obj, budget_s=12.0):
 
 def run_reference(args, rank, world):
     """The oracle on the host cores as the reference arm: K steps, each a bounded row sample."""
+    if args.workload == "gemm":
+        return run_reference_gemm(args, rank, world)
     cfg, fmt, obj, desc = WORKLOADS[args.workload]
     from fp4_block_scaled_nvfp4_b200 import synth
     import oracle as O
@@ -445,13 +452,148 @@ def run_ours(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def fp4_peak_tflops():
+    """Dense FP4 tensor peak: the measured bf16 GEMM peak times the nominal FP4 / bf16 ratio (4)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return 4.0 * float(json.load(f)["bf16_tflops"]), "measured bf16_tflops (burst) x 4, the nominal FP4/bf16 ratio"
+    return 4.0 * 1590.0, "fallback bf16 1.59 PFLOP/s x 4"
+
+
+def gemm_operands(torch, fq, synth, dev):
+    M, N, K = GEMM_SHAPE
+    wa = synth.make("cfg3", rows=M, cols=K)
+    wb = synth.make("cfg2", rows=N, cols=K)
+    xa = device_tensor_from_bits(wa["x"], torch).to(dev)
+    xb = device_tensor_from_bits(wb["x"], torch).to(dev)
+    qa = fq.quantize(xa, "nvfp4", "sweep_mse", tiled_scales=True)
+    qb = fq.quantize(xb, "nvfp4", "sweep_mse", tiled_scales=True)
+    return (M, N, K), qa, qb, wa, wb
+
+
+def run_reference_gemm(args, rank, world):
+    """The oracle's float64 NVFP4 product on the host: each step 16 activation rows times a
+    1024-row slice of the weight."""
+    from fp4_block_scaled_nvfp4_b200 import synth
+    import oracle as O
+    if rank != 0:
+        return
+    M, N, K = GEMM_SHAPE
+    wa = synth.make("cfg3", rows=16 * max(1, args.steps + args.warmup), cols=K)
+    wb = synth.make("cfg2", rows=1024, cols=K)
+    ra = O.nvfp4_quantize(O.widen_bf16(wa["x"]), "sweep_mse")
+    rb = O.nvfp4_quantize(O.widen_bf16(wb["x"]), "sweep_mse")
+    def step(i):
+        sl = slice(16 * i, 16 * i + 16)
+        O.nvfp4_gemm(ra["codes"][sl], ra["scales"][sl], ra["S"], rb["codes"], rb["scales"], rb["S"])
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    dt = time.perf_counter() - t0
+    val = 2.0 * 16 * 1024 * K * args.steps / dt / 1e12
+    line = {"impl": "reference", "metric": GEMM_METRIC, "value": round(val, 6), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "NVFP4 GEMM on the oracle", "M": M, "N": N, "K": K, "step_sample": "16 x 1024 x K"},
+            "cpu_baseline": {"value": round(val, 6), "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                             "sample": "16 activation rows times 1024 weight rows per step"},
+            "e2e": {"value": round(val, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_gemm(args, rank, world):
+    import torch
+    import fp4_block_scaled_nvfp4_b200 as fq
+    from fp4_block_scaled_nvfp4_b200 import synth
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    fq.lib()
+    (M, N, K), qa, qb, wa, wb = gemm_operands(torch, fq, synth, dev)
+    d = torch.empty((M, N), dtype=torch.float32, device=dev)
+    ws = fq.new_workspace(dev)
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            fq.nvfp4_gemm(qa, qb, out=d, workspace=ws)
+    torch.cuda.synchronize()
+    flops = 2.0 * M * N * K
+    steps = args.steps
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            start.record()
+            for _ in range(steps):
+                fq.nvfp4_gemm(qa, qb, out=d, workspace=ws)
+            end.record()
+        end.synchronize()
+    ms = start.elapsed_time(end) / steps
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    st = fq.read_device_status(ws)
+    # end to end through the public API: operands (codes, tiled scales, S) copied in from pinned
+    # host memory, the GEMM, and the fp32 product copied back, every step
+    hosts = [t.cpu().pin_memory() for t in (*qa, *qb)]
+    d_host = torch.empty((M, N), dtype=torch.float32, pin_memory=True)
+    devs = [torch.empty_like(t, device=dev) for t in hosts]
+    e_steps = max(1, min(steps, 5))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record()
+        for _ in range(e_steps):
+            for h, g in zip(hosts, devs):
+                g.copy_(h, non_blocking=True)
+            fq.nvfp4_gemm(tuple(devs[:3]), tuple(devs[3:]), out=d, workspace=ws)
+            d_host.copy_(d, non_blocking=True)
+        e1.record()
+    e1.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e_steps
+    if rank != 0:
+        return
+    peak, peak_src = fp4_peak_tflops()
+    tf = flops / (ms * 1e-3) / 1e12
+    line = {"metric": GEMM_METRIC, "value": round(tf * world, 1), "unit": "TFLOP/s", "n_gpus": world, "steps": steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "e2m1xe2m1->f32", "data": "synthetic",
+            "config": {"workload": "NVFP4 GEMM, activations 8192x4096 (activation workload, sweep-MSE) times weight "
+                                   "14336x4096 (Student-t, sweep-MSE), K contiguous, tiled scales, fp32 out",
+                       "M": M, "N": N, "K": K, "parallelism": f"replicas{world}" if world > 1 else "single",
+                       "l2": "operands 46 MB stay L2-resident across steps (a GEMM reuses them by design)",
+                       "timing": "CUDA events around back-to-back launches on one stream"},
+            "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
+                         "frac": round(tf / peak, 4), "traffic": None, "kernel": "nvfp4_gemm_kernel",
+                         "peak_source": peak_src},
+            "device_status": st, "gpu_launches": steps, "clocks": clk.summary(),
+            "e2e": {"value": round(flops / (e2e_ms * 1e-3) / 1e12 * world, 3), "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": int(sum(h.numel() * h.element_size() for h in hosts)),
+                    "d2h_bytes_per_step": M * N * 4, "ms_per_step": round(e2e_ms, 3), "steps": e_steps,
+                    "api": "operands from pinned host memory, fp4q_nvfp4_gemm, product back to pinned host memory"}}
+    if args.cpu_baseline:
+        import oracle as O
+        ra = O.nvfp4_quantize(O.widen_bf16(wa["x"][:64]), "sweep_mse", S=float(qa[2].cpu()[0]))
+        rb = O.nvfp4_quantize(O.widen_bf16(wb["x"]), "sweep_mse")
+        t0 = time.perf_counter()
+        O.nvfp4_gemm(ra["codes"], ra["scales"], ra["S"], rb["codes"], rb["scales"], rb["S"])
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": round(2.0 * 64 * N * K / dt / 1e12, 6), "unit": "TFLOP/s", "cores": 1,
+                                "kind": "oracle", "sample": f"64 of {M} activation rows times the whole weight, "
+                                                            f"float64 matmul of the decoded operands, {dt:.1f} s"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="cfg3")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["gemm"], default="cfg3")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()
@@ -466,6 +608,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, rank, world)
+        elif args.workload == "gemm":
+            run_gemm(args, rank, world)
         else:
             run_ours(args, rank, world)
     finally:

@@ -18,9 +18,15 @@
 // A wait that runs out sets FP4Q_DEVSTAT_TIMEOUT in the status word, skips the rest of the
 // work, and still frees the CTA's tensor memory.
 #include <cstdint>
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include "fp4q.h"
+
+#ifndef FP4Q_GEMM_SIMPLE
+#define FP4Q_GEMM_SIMPLE 0   // 1: the single-stage kernel with plain loads instead of the pipelined one
+#endif
 
 namespace fp4q {
 
@@ -37,7 +43,7 @@ constexpr int kSfBytes = 4 * 512;                  // four 128x4 scale atoms per
 constexpr int kSmemBytes = 2 * kTileBytes + 2 * kSfBytes + 64;
 // The request is padded so that at most two CTAs share an SM: two allocations of 256 tensor
 // memory columns fill the 512 an SM has, so no allocation ever waits for another CTA.
-constexpr int kSmemAlloc = (kSmemBytes + 1024) > 100 * 1024 ? (kSmemBytes + 1024) : 100 * 1024;
+[[maybe_unused]] constexpr int kSmemAlloc = (kSmemBytes + 1024) > 100 * 1024 ? (kSmemBytes + 1024) : 100 * 1024;
 constexpr uint32_t kWaitPolls = 1u << 22;          // bounded mbarrier wait
 
 // Shared-memory matrix descriptor (sm_100 tensor-core operand): start address, leading and
@@ -195,6 +201,178 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(kTmemCols) : "memory");
 }
 
+// ------------------------------------------------------------------------------------------
+// Pipelined form: the same tile and MMA sequence with the shared-memory operands in a ring of
+// kStages stages, filled by the tensor-memory-access engine and consumed by the tensor cores
+// while the next stages load.  Roles inside the CTA of 128 threads:
+//   thread 0 (producer): per K stage waits until the ring slot is free (its "empty" mbarrier),
+//     posts the slot's byte count on its "full" mbarrier, and issues two 2-D tensor copies
+//     (A and B tiles, 128 rows x 128 bytes, written 128-byte-swizzled by the copy engine) and
+//     two 2048-byte bulk copies (the scale atoms), all completing on "full";
+//   thread 32 (MMA issuer): waits on "full", copies the scale atoms into tensor memory, issues
+//     the four block-scaled MMAs, and commits them to the slot's "empty" mbarrier, which
+//     releases the slot once the tensor cores are done reading it; after the last stage it
+//     commits to the "done" mbarrier;
+//   all four warps: wait on "done" and run the epilogue.
+// Every wait is bounded; a wait that runs out marks the CTA failed, which stops its loops,
+// skips the epilogue and reports FP4Q_DEVSTAT_TIMEOUT.
+// ------------------------------------------------------------------------------------------
+constexpr int kStages = 4;
+constexpr int kStageBytes = 2 * kTileBytes + 2 * kSfBytes;                      // 36 KB
+constexpr int kPipeSmem = kStages * kStageBytes + 1024 /* align */ + 256 /* barriers */;
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count) : "memory");
+}
+
+template <bool UNUSED = true>
+__global__ void __launch_bounds__(kThreads, 1)
+    nvfp4_gemm_tma_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
+                          const uint8_t* __restrict__ sfa, const float* __restrict__ sa,
+                          const uint8_t* __restrict__ sfb, const float* __restrict__ sb, int K,
+                          float* __restrict__ d, int64_t ldd, uint32_t* __restrict__ status) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+    uint64_t* empty = full + kStages;
+    uint64_t* done = empty + kStages;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    __shared__ int s_fail;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t m0 = (int64_t)blockIdx.y * kTM, n0 = (int64_t)blockIdx.x * kTN;
+    const int64_t jt = K / 64;
+    const int KT = K / kTK;
+
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     :: "r"(smem_u32(tmem_slot)), "r"(kTmemCols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (tid == 0) {
+        s_fail = 0;
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(smem_u32(full + i), 1);
+            mbar_init(smem_u32(empty + i), 1);
+        }
+        mbar_init(smem_u32(done), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(&tma_a)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(&tma_b)) : "memory");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = *tmem_slot;
+
+    if (tid == 0) {
+        // producer
+        for (int kt = 0; kt < KT; ++kt) {
+            const int s = kt % kStages;
+            const uint32_t round = (uint32_t)(kt / kStages);
+            if (!mbar_wait(smem_u32(empty + s), (round & 1u) ^ 1u)) { s_fail = 1; break; }
+            uint8_t* st = smem + s * kStageBytes;
+            const uint32_t fb = smem_u32(full + s);
+            asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(fb), "r"((uint32_t)kStageBytes)
+                         : "memory");
+            const int x = kt * (kTK / 2);   // byte column of the stage, a multiple of 16
+            asm volatile(
+                "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+                :: "r"(smem_u32(st)), "l"(reinterpret_cast<uint64_t>(&tma_a)), "r"(x), "r"((int)m0), "r"(fb)
+                : "memory");
+            asm volatile(
+                "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+                :: "r"(smem_u32(st + kTileBytes)), "l"(reinterpret_cast<uint64_t>(&tma_b)), "r"(x), "r"((int)n0), "r"(fb)
+                : "memory");
+            const uint8_t* gsa = sfa + ((int64_t)blockIdx.y * jt + 4 * kt) * 512;
+            const uint8_t* gsb = sfb + ((int64_t)blockIdx.x * jt + 4 * kt) * 512;
+            asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                         :: "r"(smem_u32(st + 2 * kTileBytes)), "l"(gsa), "r"((uint32_t)kSfBytes), "r"(fb) : "memory");
+            asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                         :: "r"(smem_u32(st + 2 * kTileBytes + kSfBytes)), "l"(gsb), "r"((uint32_t)kSfBytes), "r"(fb)
+                         : "memory");
+        }
+    } else if (tid == 32) {
+        // MMA issuer
+        bool ok = true;
+        for (int kt = 0; kt < KT && ok; ++kt) {
+            const int s = kt % kStages;
+            const uint32_t round = (uint32_t)(kt / kStages);
+            if (!mbar_wait(smem_u32(full + s), round & 1u)) { s_fail = 1; ok = false; break; }
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            uint8_t* st = smem + s * kStageBytes;
+            uint8_t* sA = st;
+            uint8_t* sB = st + kTileBytes;
+            uint8_t* sSFA = st + 2 * kTileBytes;
+            uint8_t* sSFB = sSFA + kSfBytes;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t da = smem_desc(smem_u32(sSFA + kk * 512), 16, 128, 0);
+                const uint64_t db = smem_desc(smem_u32(sSFB + kk * 512), 16, 128, 0);
+                asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" :: "r"(tmem + kColSFA + 4 * kk), "l"(da)
+                             : "memory");
+                asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" :: "r"(tmem + kColSFB + 4 * kk), "l"(db)
+                             : "memory");
+            }
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t adesc = smem_desc(smem_u32(sA + kk * 32), 16, 1024, 2);
+                const uint64_t bdesc = smem_desc(smem_u32(sB + kk * 32), 16, 1024, 2);
+                const uint32_t accumulate = (kt > 0 || kk > 0) ? 1u : 0u;
+                asm volatile(
+                    "{ .reg .pred p;\n"
+                    "  setp.ne.b32 p, %4, 0;\n"
+                    "  tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p; }"
+                    :: "r"(tmem), "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate),
+                       "r"(tmem + kColSFA + 4 * kk), "r"(tmem + kColSFB + 4 * kk)
+                    : "memory");
+            }
+            asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                         :: "r"(smem_u32(empty + s)) : "memory");
+        }
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                     :: "r"(smem_u32(done)) : "memory");
+    }
+    __syncwarp();
+    // everyone waits for the accumulator (the MMA issuer commits "done" even after a failure,
+    // so this wait ends unless the tensor cores themselves stall)
+    if (!mbar_wait(smem_u32(done), 0)) s_fail = 1;
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    __syncthreads();
+
+    if (!s_fail) {
+        const float scale = __fmul_rn(*sa, *sb);
+        float* drow = d + (m0 + warp * 32 + lane) * ldd + n0;
+#pragma unroll 1
+        for (int c0 = 0; c0 < kTN; c0 += 32) {
+            uint32_t v[32];
+            asm volatile(
+                "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+                "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+                "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+                : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+                  "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
+                  "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
+                  "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
+                  "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+                : "r"(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0)
+                : "memory");
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+                *reinterpret_cast<float4*>(drow + c0 + j) =
+                    make_float4(__fmul_rn(__uint_as_float(v[j]), scale), __fmul_rn(__uint_as_float(v[j + 1]), scale),
+                                __fmul_rn(__uint_as_float(v[j + 2]), scale), __fmul_rn(__uint_as_float(v[j + 3]), scale));
+        }
+    } else if (tid == 0) {
+        atomicOr(status, (uint32_t)FP4Q_DEVSTAT_TIMEOUT);
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(kTmemCols) : "memory");
+}
+
 }  // namespace gemm
 }  // namespace fp4q
 
@@ -213,6 +391,11 @@ extern "C" int fp4q_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, 
     if (!al16(a_codes) || !al16(a_scales) || !al16(b_codes) || !al16(b_scales) || !al16(d) || !al16(workspace) ||
         ldd % 4)
         return FP4Q_ERR_ALIGNMENT;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t* status = reinterpret_cast<uint32_t*>(workspace);
+    if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return FP4Q_ERR_CUDA;
+    const dim3 grid((unsigned)(N / gemm::kTN), (unsigned)(M / gemm::kTM));
+#if FP4Q_GEMM_SIMPLE
     static bool attr_set = false;
     if (!attr_set) {
         if (cudaFuncSetAttribute(gemm::nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -220,12 +403,40 @@ extern "C" int fp4q_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, 
             return FP4Q_ERR_CUDA;
         attr_set = true;
     }
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    uint32_t* status = reinterpret_cast<uint32_t*>(workspace);
-    if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return FP4Q_ERR_CUDA;
-    const dim3 grid((unsigned)(N / gemm::kTN), (unsigned)(M / gemm::kTM));
     gemm::nvfp4_gemm_kernel<<<grid, gemm::kThreads, gemm::kSmemAlloc, st>>>(
         a_codes, a_scales, a_global_scale, b_codes, b_scales, b_global_scale, (int)K, d, ldd, status);
+#else
+    // the tensor-copy descriptors of A and B: [rows][K/2] bytes, 128 x 128-byte boxes, 128-byte swizzle
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    static bool attr_set = false;
+    if (!encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn)
+            return FP4Q_ERR_CUDA;
+        encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    if (!attr_set) {
+        if (cudaFuncSetAttribute(gemm::nvfp4_gemm_tma_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 gemm::kPipeSmem) != cudaSuccess)
+            return FP4Q_ERR_CUDA;
+        attr_set = true;
+    }
+    CUtensorMap ta, tb;
+    auto make = [&](CUtensorMap* m, const uint8_t* base, int64_t rows) {
+        const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
+        const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+        const cuuint32_t box[2] = {(cuuint32_t)(gemm::kTK / 2), (cuuint32_t)gemm::kTM};
+        const cuuint32_t estr[2] = {1, 1};
+        return encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    };
+    if (!make(&ta, a_codes, M) || !make(&tb, b_codes, N)) return FP4Q_ERR_CUDA;
+    gemm::nvfp4_gemm_tma_kernel<true><<<grid, gemm::kThreads, gemm::kPipeSmem, st>>>(
+        ta, tb, a_scales, a_global_scale, b_scales, b_global_scale, (int)K, d, ldd, status);
+#endif
     if (cudaGetLastError() != cudaSuccess) return FP4Q_ERR_CUDA;
     g_launches = 1;
     return FP4Q_OK;
