@@ -4,19 +4,21 @@
 // low nibble; E4M3 scales in the 128x4-tiled layout of FP4Q_F_SCALE_TILED; one fp32 tensor
 // scale each).  Both operands have K contiguous.
 //
-// One CTA of 128 threads computes a 128 x 128 tile of D:
-//   * per K stage of 256 elements, all threads copy the A and B tiles (128 rows x 128 bytes
-//     each) into shared memory in the 128-byte-swizzled K-major layout the MMA descriptor
-//     describes, and the four 512-byte scale-factor atoms of each operand as they are;
-//   * one thread moves the scale atoms into tensor memory (tcgen05.cp 32x128b, broadcast to
-//     the four lane quarters) and issues four block-scaled MMAs of K = 64
-//     (tcgen05.mma kind::mxf4nvf4, 16-element scale blocks) accumulating in tensor memory,
-//     then commits them to an mbarrier that every thread waits on (bounded) before the shared
-//     buffers are refilled;
-//   * the epilogue reads the fp32 accumulator back with tcgen05.ld (each warp its 32 lanes),
-//     multiplies by S_a S_b and stores D.
-// A wait that runs out sets FP4Q_DEVSTAT_TIMEOUT in the status word, skips the rest of the
-// work, and still frees the CTA's tensor memory.
+// Each output tile of 128 x 128 is built from K stages of 256 elements: per stage the A and B
+// tiles (128 rows x 128 bytes each) sit in shared memory in the 128-byte-swizzled K-major
+// layout the MMA descriptor describes, and the four 512-byte scale-factor atoms of each operand
+// as they are; one thread moves the atoms into tensor memory (tcgen05.cp 32x128b, broadcast to
+// the four lane quarters) and issues four block-scaled MMAs of K = 64 (tcgen05.mma
+// kind::mxf4nvf4, 16-element scale blocks) accumulating fp32 in tensor memory; the epilogue
+// reads the accumulator back with tcgen05.ld (each warp its lane quarter), multiplies by
+// RN(S_a S_b) and stores D.
+//   nvfp4_gemm_persistent_kernel (the one launched): one CTA per SM over all tiles, a
+//     five-stage ring filled by tensor copies, producer / MMA / epilogue warps, two
+//     accumulators so the epilogue of a tile overlaps the next tile's MMAs.
+//   nvfp4_gemm_kernel (build flag FP4Q_GEMM_SIMPLE): the same arithmetic in one stage with
+//     plain loads, kept as the reference form of the sequence.
+// Every wait is bounded; one that runs out sets FP4Q_DEVSTAT_TIMEOUT in the status word, stops
+// the CTA's loops, and the CTA still frees its tensor memory.
 #include <cstdint>
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -201,61 +203,67 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(kTmemCols) : "memory");
 }
 
-// ------------------------------------------------------------------------------------------
-// Pipelined form: the same tile and MMA sequence with the shared-memory operands in a ring of
-// kStages stages, filled by the tensor-memory-access engine and consumed by the tensor cores
-// while the next stages load.  Roles inside the CTA of 128 threads:
-//   thread 0 (producer): per K stage waits until the ring slot is free (its "empty" mbarrier),
-//     posts the slot's byte count on its "full" mbarrier, and issues two 2-D tensor copies
-//     (A and B tiles, 128 rows x 128 bytes, written 128-byte-swizzled by the copy engine) and
-//     two 2048-byte bulk copies (the scale atoms), all completing on "full";
-//   thread 32 (MMA issuer): waits on "full", copies the scale atoms into tensor memory, issues
-//     the four block-scaled MMAs, and commits them to the slot's "empty" mbarrier, which
-//     releases the slot once the tensor cores are done reading it; after the last stage it
-//     commits to the "done" mbarrier;
-//   all four warps: wait on "done" and run the epilogue.
-// Every wait is bounded; a wait that runs out marks the CTA failed, which stops its loops,
-// skips the epilogue and reports FP4Q_DEVSTAT_TIMEOUT.
-// ------------------------------------------------------------------------------------------
-constexpr int kStages = 4;
-constexpr int kStageBytes = 2 * kTileBytes + 2 * kSfBytes;                      // 36 KB
-constexpr int kPipeSmem = kStages * kStageBytes + 1024 /* align */ + 256 /* barriers */;
+constexpr int kStageBytes = 2 * kTileBytes + 2 * kSfBytes;                      // 36 KB per ring stage
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count) : "memory");
 }
 
-template <bool UNUSED = true>
-__global__ void __launch_bounds__(kThreads, 1)
-    nvfp4_gemm_tma_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
-                          const uint8_t* __restrict__ sfa, const float* __restrict__ sa,
-                          const uint8_t* __restrict__ sfb, const float* __restrict__ sb, int K,
-                          float* __restrict__ d, int64_t ldd, uint32_t* __restrict__ status) {
+// ------------------------------------------------------------------------------------------
+// Pipelined, persistent form (the one fp4q_nvfp4_gemm launches): the same 128 x 128 tile and
+// MMA sequence, with the shared-memory operands in a ring of kPStages stages filled by the
+// tensor-memory-access engine (A and B tiles as 2-D tensor copies written 128-byte-swizzled by
+// the copy engine, the scale atoms as 2048-byte bulk copies, all completing on the stage's
+// "full" mbarrier) and released by the MMAs' commit to the stage's "empty" mbarrier.  One CTA
+// per SM walks the output tiles t = blockIdx.x, + gridDim.x, ...
+// (row-major over (m tile, n tile)), with two fp32 accumulators in tensor memory so that the
+// epilogue of one tile overlaps the MMAs of the next.  192 threads, six warps:
+//   warp 0 lane 0 -- producer over the (tile, K stage) sequence, filling the kPStages ring;
+//   warp 1 lane 0 -- MMA issuer: per tile waits for a free accumulator ("acc_empty"), runs the
+//     K loop into it, and commits "acc_full";
+//   warps 2..5 -- epilogue: per tile wait "acc_full", read the accumulator (each warp the lane
+//     quarter warp % 4, as tensor memory requires), scale by S_a S_b, store, arrive "acc_empty".
+// ------------------------------------------------------------------------------------------
+constexpr int kPStages = 5;
+constexpr int kPThreads = 192;
+constexpr uint32_t kPTmemCols = 512;                  // two accumulators of 128 + scale factors
+constexpr uint32_t kPColSFA = 256, kPColSFB = 272;
+constexpr int kPersistSmem = kPStages * kStageBytes + 1024 + 256;
+
+__global__ void __launch_bounds__(kPThreads, 1)
+    nvfp4_gemm_persistent_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
+                                 const uint8_t* __restrict__ sfa, const float* __restrict__ sa,
+                                 const uint8_t* __restrict__ sfb, const float* __restrict__ sb, int K, int m_tiles,
+                                 int n_tiles, float* __restrict__ d, int64_t ldd, uint32_t* __restrict__ status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
-    uint64_t* empty = full + kStages;
-    uint64_t* done = empty + kStages;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
-    __shared__ int s_fail;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kPStages * kStageBytes);
+    uint64_t* empty = full + kPStages;
+    uint64_t* acc_full = empty + kPStages;     // [2]
+    uint64_t* acc_empty = acc_full + 2;        // [2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+    __shared__ volatile int s_fail;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t m0 = (int64_t)blockIdx.y * kTM, n0 = (int64_t)blockIdx.x * kTN;
     const int64_t jt = K / 64;
     const int KT = K / kTK;
+    const int tiles = m_tiles * n_tiles;
 
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                     :: "r"(smem_u32(tmem_slot)), "r"(kTmemCols) : "memory");
+                     :: "r"(smem_u32(tmem_slot)), "r"(kPTmemCols) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (tid == 0) {
         s_fail = 0;
-        for (int i = 0; i < kStages; ++i) {
+        for (int i = 0; i < kPStages; ++i) {
             mbar_init(smem_u32(full + i), 1);
             mbar_init(smem_u32(empty + i), 1);
         }
-        mbar_init(smem_u32(done), 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_u32(acc_full + i), 1);
+            mbar_init(smem_u32(acc_empty + i), 4);   // one arrival per epilogue warp
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(&tma_a)) : "memory");
         asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(&tma_b)) : "memory");
@@ -267,110 +275,130 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (tid == 0) {
         // producer
-        for (int kt = 0; kt < KT; ++kt) {
-            const int s = kt % kStages;
-            const uint32_t round = (uint32_t)(kt / kStages);
-            if (!mbar_wait(smem_u32(empty + s), (round & 1u) ^ 1u)) { s_fail = 1; break; }
-            uint8_t* st = smem + s * kStageBytes;
-            const uint32_t fb = smem_u32(full + s);
-            asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(fb), "r"((uint32_t)kStageBytes)
-                         : "memory");
-            const int x = kt * (kTK / 2);   // byte column of the stage, a multiple of 16
-            asm volatile(
-                "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-                :: "r"(smem_u32(st)), "l"(reinterpret_cast<uint64_t>(&tma_a)), "r"(x), "r"((int)m0), "r"(fb)
-                : "memory");
-            asm volatile(
-                "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-                :: "r"(smem_u32(st + kTileBytes)), "l"(reinterpret_cast<uint64_t>(&tma_b)), "r"(x), "r"((int)n0), "r"(fb)
-                : "memory");
-            const uint8_t* gsa = sfa + ((int64_t)blockIdx.y * jt + 4 * kt) * 512;
-            const uint8_t* gsb = sfb + ((int64_t)blockIdx.x * jt + 4 * kt) * 512;
-            asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                         :: "r"(smem_u32(st + 2 * kTileBytes)), "l"(gsa), "r"((uint32_t)kSfBytes), "r"(fb) : "memory");
-            asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                         :: "r"(smem_u32(st + 2 * kTileBytes + kSfBytes)), "l"(gsb), "r"((uint32_t)kSfBytes), "r"(fb)
-                         : "memory");
+        uint32_t g = 0;
+        for (int t = blockIdx.x; t < tiles && !s_fail; t += gridDim.x) {
+            const int mt = t / n_tiles, nt = t - mt * n_tiles;
+            for (int kt = 0; kt < KT; ++kt, ++g) {
+                const uint32_t s = g % kPStages, round = g / kPStages;
+                if (!mbar_wait(smem_u32(empty + s), (round & 1u) ^ 1u)) { s_fail = 1; break; }
+                uint8_t* st = smem + s * kStageBytes;
+                const uint32_t fb = smem_u32(full + s);
+                asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+                             :: "r"(fb), "r"((uint32_t)kStageBytes) : "memory");
+                const int x = kt * (kTK / 2);
+                asm volatile(
+                    "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+                    :: "r"(smem_u32(st)), "l"(reinterpret_cast<uint64_t>(&tma_a)), "r"(x), "r"(mt * kTM), "r"(fb)
+                    : "memory");
+                asm volatile(
+                    "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+                    :: "r"(smem_u32(st + kTileBytes)), "l"(reinterpret_cast<uint64_t>(&tma_b)), "r"(x), "r"(nt * kTN), "r"(fb)
+                    : "memory");
+                const uint8_t* gsa = sfa + ((int64_t)mt * jt + 4 * kt) * 512;
+                const uint8_t* gsb = sfb + ((int64_t)nt * jt + 4 * kt) * 512;
+                asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                             :: "r"(smem_u32(st + 2 * kTileBytes)), "l"(gsa), "r"((uint32_t)kSfBytes), "r"(fb) : "memory");
+                asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                             :: "r"(smem_u32(st + 2 * kTileBytes + kSfBytes)), "l"(gsb), "r"((uint32_t)kSfBytes), "r"(fb)
+                             : "memory");
+            }
         }
     } else if (tid == 32) {
         // MMA issuer
-        bool ok = true;
-        for (int kt = 0; kt < KT && ok; ++kt) {
-            const int s = kt % kStages;
-            const uint32_t round = (uint32_t)(kt / kStages);
-            if (!mbar_wait(smem_u32(full + s), round & 1u)) { s_fail = 1; ok = false; break; }
+        uint32_t g = 0;
+        int j = 0;
+        for (int t = blockIdx.x; t < tiles && !s_fail; t += gridDim.x, ++j) {
+            const uint32_t acc = (uint32_t)(j & 1), around = (uint32_t)(j >> 1);
+            if (!mbar_wait(smem_u32(acc_empty + acc), (around & 1u) ^ 1u)) { s_fail = 1; break; }
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            uint8_t* st = smem + s * kStageBytes;
-            uint8_t* sA = st;
-            uint8_t* sB = st + kTileBytes;
-            uint8_t* sSFA = st + 2 * kTileBytes;
-            uint8_t* sSFB = sSFA + kSfBytes;
+            const uint32_t tacc = tmem + acc * kTN;
+            for (int kt = 0; kt < KT; ++kt, ++g) {
+                const uint32_t s = g % kPStages, round = g / kPStages;
+                if (!mbar_wait(smem_u32(full + s), round & 1u)) { s_fail = 1; break; }
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                uint8_t* st = smem + s * kStageBytes;
+                uint8_t* sSFA = st + 2 * kTileBytes;
+                uint8_t* sSFB = sSFA + kSfBytes;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t da = smem_desc(smem_u32(sSFA + kk * 512), 16, 128, 0);
-                const uint64_t db = smem_desc(smem_u32(sSFB + kk * 512), 16, 128, 0);
-                asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" :: "r"(tmem + kColSFA + 4 * kk), "l"(da)
-                             : "memory");
-                asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" :: "r"(tmem + kColSFB + 4 * kk), "l"(db)
-                             : "memory");
-            }
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t da = smem_desc(smem_u32(sSFA + kk * 512), 16, 128, 0);
+                    const uint64_t db = smem_desc(smem_u32(sSFB + kk * 512), 16, 128, 0);
+                    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;"
+                                 :: "r"(tmem + kPColSFA + 4 * kk), "l"(da) : "memory");
+                    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;"
+                                 :: "r"(tmem + kPColSFB + 4 * kk), "l"(db) : "memory");
+                }
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t adesc = smem_desc(smem_u32(sA + kk * 32), 16, 1024, 2);
-                const uint64_t bdesc = smem_desc(smem_u32(sB + kk * 32), 16, 1024, 2);
-                const uint32_t accumulate = (kt > 0 || kk > 0) ? 1u : 0u;
-                asm volatile(
-                    "{ .reg .pred p;\n"
-                    "  setp.ne.b32 p, %4, 0;\n"
-                    "  tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p; }"
-                    :: "r"(tmem), "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate),
-                       "r"(tmem + kColSFA + 4 * kk), "r"(tmem + kColSFB + 4 * kk)
-                    : "memory");
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t adesc = smem_desc(smem_u32(st + kk * 32), 16, 1024, 2);
+                    const uint64_t bdesc = smem_desc(smem_u32(st + kTileBytes + kk * 32), 16, 1024, 2);
+                    const uint32_t accumulate = (kt > 0 || kk > 0) ? 1u : 0u;
+                    asm volatile(
+                        "{ .reg .pred p;\n"
+                        "  setp.ne.b32 p, %4, 0;\n"
+                        "  tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p; }"
+                        :: "r"(tacc), "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate),
+                           "r"(tmem + kPColSFA + 4 * kk), "r"(tmem + kPColSFB + 4 * kk)
+                        : "memory");
+                }
+                asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                             :: "r"(smem_u32(empty + s)) : "memory");
             }
+            // the accumulator is complete once every MMA above has finished (also after a failure,
+            // so that the epilogue's wait ends)
             asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-                         :: "r"(smem_u32(empty + s)) : "memory");
+                         :: "r"(smem_u32(acc_full + acc)) : "memory");
         }
-        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-                     :: "r"(smem_u32(done)) : "memory");
+    } else if (warp >= 2) {
+        // epilogue: this warp owns tensor-memory lanes 32 (warp % 4) .. + 31
+        const int q = warp & 3;
+        const float scale = __fmul_rn(*sa, *sb);
+        int j = 0;
+        for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++j) {
+            const uint32_t acc = (uint32_t)(j & 1), around = (uint32_t)(j >> 1);
+            // warp-uniform decisions: the tensor-memory loads below are warp-collective
+            const int ok = __all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(acc_full + acc), around & 1u) ? 1 : 0);
+            const int failed = __shfl_sync(0xFFFFFFFFu, s_fail, 0);
+            if (!ok || failed) {
+                s_fail = 1;
+                break;
+            }
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            const int mt = t / n_tiles, nt = t - mt * n_tiles;
+            float* drow = d + ((int64_t)mt * kTM + q * 32 + lane) * ldd + (int64_t)nt * kTN;
+#pragma unroll 1
+            for (int c0 = 0; c0 < kTN; c0 += 32) {
+                uint32_t v[32];
+                asm volatile(
+                    "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+                    "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+                    "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+                    : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+                      "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
+                      "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
+                      "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
+                      "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+                    : "r"(tmem + ((uint32_t)(q * 32) << 16) + acc * kTN + (uint32_t)c0)
+                    : "memory");
+                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+                for (int c = 0; c < 32; c += 4)
+                    *reinterpret_cast<float4*>(drow + c0 + c) = make_float4(
+                        __fmul_rn(__uint_as_float(v[c]), scale), __fmul_rn(__uint_as_float(v[c + 1]), scale),
+                        __fmul_rn(__uint_as_float(v[c + 2]), scale), __fmul_rn(__uint_as_float(v[c + 3]), scale));
+            }
+            // the accumulator may be overwritten once this warp's reads are done
+            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_u32(acc_empty + acc)) : "memory");
+        }
     }
     __syncwarp();
-    // everyone waits for the accumulator (the MMA issuer commits "done" even after a failure,
-    // so this wait ends unless the tensor cores themselves stall)
-    if (!mbar_wait(smem_u32(done), 0)) s_fail = 1;
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    __syncthreads();
-
-    if (!s_fail) {
-        const float scale = __fmul_rn(*sa, *sb);
-        float* drow = d + (m0 + warp * 32 + lane) * ldd + n0;
-#pragma unroll 1
-        for (int c0 = 0; c0 < kTN; c0 += 32) {
-            uint32_t v[32];
-            asm volatile(
-                "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-                "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-                "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-                : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-                  "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
-                  "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
-                  "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
-                  "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-                : "r"(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0)
-                : "memory");
-            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-            for (int j = 0; j < 32; j += 4)
-                *reinterpret_cast<float4*>(drow + c0 + j) =
-                    make_float4(__fmul_rn(__uint_as_float(v[j]), scale), __fmul_rn(__uint_as_float(v[j + 1]), scale),
-                                __fmul_rn(__uint_as_float(v[j + 2]), scale), __fmul_rn(__uint_as_float(v[j + 3]), scale));
-        }
-    } else if (tid == 0) {
-        atomicOr(status, (uint32_t)FP4Q_DEVSTAT_TIMEOUT);
-    }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
+    if (s_fail && tid == 0) atomicOr(status, (uint32_t)FP4Q_DEVSTAT_TIMEOUT);
     if (warp == 0)
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(kTmemCols) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(kPTmemCols) : "memory");
 }
 
 }  // namespace gemm
@@ -418,8 +446,8 @@ extern "C" int fp4q_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, 
         encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
     if (!attr_set) {
-        if (cudaFuncSetAttribute(gemm::nvfp4_gemm_tma_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 gemm::kPipeSmem) != cudaSuccess)
+        if (cudaFuncSetAttribute(gemm::nvfp4_gemm_persistent_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 gemm::kPersistSmem) != cudaSuccess)
             return FP4Q_ERR_CUDA;
         attr_set = true;
     }
@@ -434,8 +462,17 @@ extern "C" int fp4q_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, 
                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
     };
     if (!make(&ta, a_codes, M) || !make(&tb, b_codes, N)) return FP4Q_ERR_CUDA;
-    gemm::nvfp4_gemm_tma_kernel<true><<<grid, gemm::kThreads, gemm::kPipeSmem, st>>>(
-        ta, tb, a_scales, a_global_scale, b_scales, b_global_scale, (int)K, d, ldd, status);
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+            return FP4Q_ERR_CUDA;
+    }
+    const int m_tiles = (int)(M / gemm::kTM), n_tiles = (int)(N / gemm::kTN);
+    const int tiles = m_tiles * n_tiles;
+    gemm::nvfp4_gemm_persistent_kernel<<<tiles < sms ? tiles : sms, gemm::kPThreads, gemm::kPersistSmem, st>>>(
+        ta, tb, a_scales, a_global_scale, b_scales, b_global_scale, (int)K, m_tiles, n_tiles, d, ldd, status);
 #endif
     if (cudaGetLastError() != cudaSuccess) return FP4Q_ERR_CUDA;
     g_launches = 1;
