@@ -203,51 +203,79 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(kTmemCols) : "memory");
 }
 
-constexpr int kStageBytes = 2 * kTileBytes + 2 * kSfBytes;                      // 36 KB per ring stage
-
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count) : "memory");
 }
 
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
 // ------------------------------------------------------------------------------------------
-// Pipelined, persistent form (the one fp4q_nvfp4_gemm launches): the same 128 x 128 tile and
-// MMA sequence, with the shared-memory operands in a ring of kPStages stages filled by the
-// tensor-memory-access engine (A and B tiles as 2-D tensor copies written 128-byte-swizzled by
-// the copy engine, the scale atoms as 2048-byte bulk copies, all completing on the stage's
-// "full" mbarrier) and released by the MMAs' commit to the stage's "empty" mbarrier.  One CTA
-// per SM walks the output tiles t = blockIdx.x, + gridDim.x, ...
-// (row-major over (m tile, n tile)), with two fp32 accumulators in tensor memory so that the
-// epilogue of one tile overlaps the MMAs of the next.  192 threads, six warps:
-//   warp 0 lane 0 -- producer over the (tile, K stage) sequence, filling the kPStages ring;
-//   warp 1 lane 0 -- MMA issuer: per tile waits for a free accumulator ("acc_empty"), runs the
-//     K loop into it, and commits "acc_full";
+// Pipelined, persistent form (the one fp4q_nvfp4_gemm launches).  Output tiles are 128 x 256
+// (the last tile of a row of tiles is 128 x 128 when N is an odd multiple of 128): per K stage
+// of 256 elements one MMA of N = 256 (or 128) per K = 64 reads the A tile (128 rows) and the
+// B tile (256 rows), so every byte brought into shared memory feeds twice the products of a
+// 128 x 128 tile.  The operands sit in a ring of kPStages stages filled by the tensor-memory-
+// access engine (A and B tiles as 2-D tensor copies written 128-byte-swizzled by the copy
+// engine, B rows past N read as zeros; scale atoms as 2048-byte bulk copies), completing on the
+// stage's "full" mbarrier, and released by the MMAs' commit to the stage's "empty" mbarrier.
+// One CTA per SM walks the tiles t = blockIdx.x, + gridDim.x, ... (row-major over (m tile,
+// n tile)).  192 threads, six warps:
+//   warp 0 lane 0 -- producer over the (tile, K stage) sequence;
+//   warp 1 lane 0 -- MMA issuer: copies each stage's scale atoms into tensor memory and issues
+//     the four MMAs, then commits "acc_full" per tile;
 //   warps 2..5 -- epilogue: per tile wait "acc_full", read the accumulator (each warp the lane
-//     quarter warp % 4, as tensor memory requires), scale by S_a S_b, store, arrive "acc_empty".
+//     quarter warp % 4, as tensor memory requires), scale by S_a S_b and store.
+// Tensor memory (512 columns): two accumulators of 256 columns cannot both fit beside the
+// scale factors, so they overlap: tile j accumulates at column 0 (j even) or 192 (j odd), and
+// the 64 columns [192, 256) are shared.  The epilogue of each tile reads its shared 64 columns
+// first and then arrives on "acc_free"; the MMAs of the next tile start on that arrival and
+// overlap the rest of the epilogue.  Scale factors: A at column 448 (4 per K = 64), B at 464
+// (8 per K = 64: B rows 32 c .. 32 c + 31 in column c).
 // ------------------------------------------------------------------------------------------
-constexpr int kPStages = 5;
+constexpr int kBN = 256;                                   // tile N
+constexpr int kPStages = 4;
+constexpr int kBTileBytes = kBN * kTK / 2;                 // 32 KB of B codes per stage
+constexpr int kPStageBytes = kTileBytes + kBTileBytes + 3 * kSfBytes;   // 54 KB per ring stage
 constexpr int kPThreads = 192;
-constexpr uint32_t kPTmemCols = 512;                  // two accumulators of 128 + scale factors
-constexpr uint32_t kPColSFA = 256, kPColSFB = 272;
-constexpr int kPersistSmem = kPStages * kStageBytes + 1024 + 256;
+constexpr uint32_t kPTmemCols = 512;
+constexpr uint32_t kAcc1 = 192;                            // first column of the odd tiles' accumulator
+constexpr uint32_t kPColSFA = 448, kPColSFB = 464;
+constexpr int kPersistSmem = kPStages * kPStageBytes + 1024 + 256;
+constexpr uint32_t kIdescN256 = (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(kTM >> 4) << 24);
 
 __global__ void __launch_bounds__(kPThreads, 1)
     nvfp4_gemm_persistent_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                                  const uint8_t* __restrict__ sfa, const float* __restrict__ sa,
                                  const uint8_t* __restrict__ sfb, const float* __restrict__ sb, int K, int m_tiles,
-                                 int n_tiles, float* __restrict__ d, int64_t ldd, uint32_t* __restrict__ status) {
+                                 int n_tiles, int n_last_wide, float* __restrict__ d, int64_t ldd,
+                                 uint32_t* __restrict__ status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kPStages * kStageBytes);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kPStages * kPStageBytes);
     uint64_t* empty = full + kPStages;
-    uint64_t* acc_full = empty + kPStages;     // [2]
-    uint64_t* acc_empty = acc_full + 2;        // [2]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+    uint64_t* acc_full = empty + kPStages;
+    uint64_t* acc_free = acc_full + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_free + 1);
     __shared__ volatile int s_fail;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t jt = K / 64;
     const int KT = K / kTK;
     const int tiles = m_tiles * n_tiles;
+    // the last tile of each row of tiles is 128 wide unless N is a multiple of 256
+    auto wide_tile = [&](int nt) { return nt + 1 < n_tiles || n_last_wide; };
 
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -260,10 +288,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
             mbar_init(smem_u32(full + i), 1);
             mbar_init(smem_u32(empty + i), 1);
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(smem_u32(acc_full + i), 1);
-            mbar_init(smem_u32(acc_empty + i), 4);   // one arrival per epilogue warp
-        }
+        mbar_init(smem_u32(acc_full), 1);
+        mbar_init(smem_u32(acc_free), 4);   // one arrival per epilogue warp
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(&tma_a)) : "memory");
         asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(&tma_b)) : "memory");
@@ -278,13 +304,15 @@ __global__ void __launch_bounds__(kPThreads, 1)
         uint32_t g = 0;
         for (int t = blockIdx.x; t < tiles && !s_fail; t += gridDim.x) {
             const int mt = t / n_tiles, nt = t - mt * n_tiles;
+            const bool wide = wide_tile(nt);
+            // a tensor copy's transaction count is its whole box, rows past N included
+            const uint32_t bytes = (uint32_t)(kTileBytes + kBTileBytes + (wide ? 3 : 2) * kSfBytes);
             for (int kt = 0; kt < KT; ++kt, ++g) {
                 const uint32_t s = g % kPStages, round = g / kPStages;
                 if (!mbar_wait(smem_u32(empty + s), (round & 1u) ^ 1u)) { s_fail = 1; break; }
-                uint8_t* st = smem + s * kStageBytes;
+                uint8_t* st = smem + s * kPStageBytes;
                 const uint32_t fb = smem_u32(full + s);
-                asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
-                             :: "r"(fb), "r"((uint32_t)kStageBytes) : "memory");
+                asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(fb), "r"(bytes) : "memory");
                 const int x = kt * (kTK / 2);
                 asm volatile(
                     "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
@@ -292,15 +320,20 @@ __global__ void __launch_bounds__(kPThreads, 1)
                     : "memory");
                 asm volatile(
                     "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-                    :: "r"(smem_u32(st + kTileBytes)), "l"(reinterpret_cast<uint64_t>(&tma_b)), "r"(x), "r"(nt * kTN), "r"(fb)
+                    :: "r"(smem_u32(st + kTileBytes)), "l"(reinterpret_cast<uint64_t>(&tma_b)), "r"(x), "r"(nt * kBN),
+                       "r"(fb)
                     : "memory");
+                uint8_t* ssf = st + kTileBytes + kBTileBytes;
                 const uint8_t* gsa = sfa + ((int64_t)mt * jt + 4 * kt) * 512;
-                const uint8_t* gsb = sfb + ((int64_t)nt * jt + 4 * kt) * 512;
+                const uint8_t* gsb = sfb + ((int64_t)(2 * nt) * jt + 4 * kt) * 512;
                 asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                             :: "r"(smem_u32(st + 2 * kTileBytes)), "l"(gsa), "r"((uint32_t)kSfBytes), "r"(fb) : "memory");
+                             :: "r"(smem_u32(ssf)), "l"(gsa), "r"((uint32_t)kSfBytes), "r"(fb) : "memory");
                 asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                             :: "r"(smem_u32(st + 2 * kTileBytes + kSfBytes)), "l"(gsb), "r"((uint32_t)kSfBytes), "r"(fb)
-                             : "memory");
+                             :: "r"(smem_u32(ssf + kSfBytes)), "l"(gsb), "r"((uint32_t)kSfBytes), "r"(fb) : "memory");
+                if (wide)
+                    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                                 :: "r"(smem_u32(ssf + 2 * kSfBytes)), "l"(gsb + jt * 512), "r"((uint32_t)kSfBytes), "r"(fb)
+                                 : "memory");
             }
         }
     } else if (tid == 32) {
@@ -308,25 +341,32 @@ __global__ void __launch_bounds__(kPThreads, 1)
         uint32_t g = 0;
         int j = 0;
         for (int t = blockIdx.x; t < tiles && !s_fail; t += gridDim.x, ++j) {
-            const uint32_t acc = (uint32_t)(j & 1), around = (uint32_t)(j >> 1);
-            if (!mbar_wait(smem_u32(acc_empty + acc), (around & 1u) ^ 1u)) { s_fail = 1; break; }
+            const int nt = t % n_tiles;
+            const bool wide = wide_tile(nt);
+            const uint32_t idesc = wide ? kIdescN256 : kIdesc;
+            // the previous tile's epilogue has read the columns this accumulator shares with it
+            if (j > 0 && !mbar_wait(smem_u32(acc_free), (uint32_t)((j - 1) & 1))) { s_fail = 1; break; }
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            const uint32_t tacc = tmem + acc * kTN;
+            const uint32_t tacc = tmem + ((j & 1) ? kAcc1 : 0u);
             for (int kt = 0; kt < KT; ++kt, ++g) {
                 const uint32_t s = g % kPStages, round = g / kPStages;
                 if (!mbar_wait(smem_u32(full + s), round & 1u)) { s_fail = 1; break; }
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-                uint8_t* st = smem + s * kStageBytes;
-                uint8_t* sSFA = st + 2 * kTileBytes;
-                uint8_t* sSFB = sSFA + kSfBytes;
+                uint8_t* st = smem + s * kPStageBytes;
+                uint8_t* ssf = st + kTileBytes + kBTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t da = smem_desc(smem_u32(sSFA + kk * 512), 16, 128, 0);
-                    const uint64_t db = smem_desc(smem_u32(sSFB + kk * 512), 16, 128, 0);
+                    const uint64_t da = smem_desc(smem_u32(ssf + kk * 512), 16, 128, 0);
+                    const uint64_t db0 = smem_desc(smem_u32(ssf + kSfBytes + kk * 512), 16, 128, 0);
                     asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;"
                                  :: "r"(tmem + kPColSFA + 4 * kk), "l"(da) : "memory");
                     asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;"
-                                 :: "r"(tmem + kPColSFB + 4 * kk), "l"(db) : "memory");
+                                 :: "r"(tmem + kPColSFB + 8 * kk), "l"(db0) : "memory");
+                    if (wide) {
+                        const uint64_t db1 = smem_desc(smem_u32(ssf + 2 * kSfBytes + kk * 512), 16, 128, 0);
+                        asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;"
+                                     :: "r"(tmem + kPColSFB + 8 * kk + 4), "l"(db1) : "memory");
+                    }
                 }
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
@@ -337,8 +377,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
                         "{ .reg .pred p;\n"
                         "  setp.ne.b32 p, %4, 0;\n"
                         "  tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p; }"
-                        :: "r"(tacc), "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate),
-                           "r"(tmem + kPColSFA + 4 * kk), "r"(tmem + kPColSFB + 4 * kk)
+                        :: "r"(tacc), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate),
+                           "r"(tmem + kPColSFA + 4 * kk), "r"(tmem + kPColSFB + 8 * kk)
                         : "memory");
                 }
                 asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
@@ -347,7 +387,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
             // the accumulator is complete once every MMA above has finished (also after a failure,
             // so that the epilogue's wait ends)
             asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-                         :: "r"(smem_u32(acc_full + acc)) : "memory");
+                         :: "r"(smem_u32(acc_full)) : "memory");
         }
     } else if (warp >= 2) {
         // epilogue: this warp owns tensor-memory lanes 32 (warp % 4) .. + 31
@@ -355,9 +395,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
         const float scale = __fmul_rn(*sa, *sb);
         int j = 0;
         for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++j) {
-            const uint32_t acc = (uint32_t)(j & 1), around = (uint32_t)(j >> 1);
             // warp-uniform decisions: the tensor-memory loads below are warp-collective
-            const int ok = __all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(acc_full + acc), around & 1u) ? 1 : 0);
+            const int ok = __all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(acc_full), (uint32_t)(j & 1)) ? 1 : 0);
             const int failed = __shfl_sync(0xFFFFFFFFu, s_fail, 0);
             if (!ok || failed) {
                 s_fail = 1;
@@ -365,32 +404,30 @@ __global__ void __launch_bounds__(kPThreads, 1)
             }
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
             const int mt = t / n_tiles, nt = t - mt * n_tiles;
-            float* drow = d + ((int64_t)mt * kTM + q * 32 + lane) * ldd + (int64_t)nt * kTN;
-#pragma unroll 1
-            for (int c0 = 0; c0 < kTN; c0 += 32) {
+            const bool odd = (j & 1) != 0;
+            const int nchunks = wide_tile(nt) ? kBN / 32 : kTN / 32;
+            // chunks (of 32 columns) shared with the other accumulator are read first: the last
+            // two of an even tile's 256 columns, the first two of an odd tile's
+            const int first = (!odd && nchunks == 8) ? 6 : 0;
+            const int shared_chunks = odd ? 2 : (nchunks == 8 ? 2 : 0);
+            const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (odd ? kAcc1 : 0u);
+            float* drow = d + ((int64_t)mt * kTM + q * 32 + lane) * ldd + (int64_t)nt * kBN;
+            for (int i = 0; i <= nchunks; ++i) {
+                if (i == shared_chunks) {
+                    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_u32(acc_free)) : "memory");
+                }
+                if (i == nchunks) break;
+                const int c = (first + i) % nchunks;
                 uint32_t v[32];
-                asm volatile(
-                    "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-                    "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-                    "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-                    : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-                      "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
-                      "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
-                      "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
-                      "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-                    : "r"(tmem + ((uint32_t)(q * 32) << 16) + acc * kTN + (uint32_t)c0)
-                    : "memory");
-                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                tmem_ld32(tbase + (uint32_t)(c * 32), v);
 #pragma unroll
-                for (int c = 0; c < 32; c += 4)
-                    *reinterpret_cast<float4*>(drow + c0 + c) = make_float4(
-                        __fmul_rn(__uint_as_float(v[c]), scale), __fmul_rn(__uint_as_float(v[c + 1]), scale),
-                        __fmul_rn(__uint_as_float(v[c + 2]), scale), __fmul_rn(__uint_as_float(v[c + 3]), scale));
+                for (int e = 0; e < 32; e += 4)
+                    *reinterpret_cast<float4*>(drow + c * 32 + e) = make_float4(
+                        __fmul_rn(__uint_as_float(v[e]), scale), __fmul_rn(__uint_as_float(v[e + 1]), scale),
+                        __fmul_rn(__uint_as_float(v[e + 2]), scale), __fmul_rn(__uint_as_float(v[e + 3]), scale));
             }
-            // the accumulator may be overwritten once this warp's reads are done
-            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-            __syncwarp();
-            if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_u32(acc_empty + acc)) : "memory");
         }
     }
     __syncwarp();
@@ -452,16 +489,16 @@ extern "C" int fp4q_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, 
         attr_set = true;
     }
     CUtensorMap ta, tb;
-    auto make = [&](CUtensorMap* m, const uint8_t* base, int64_t rows) {
+    auto make = [&](CUtensorMap* m, const uint8_t* base, int64_t rows, int box_rows) {
         const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
         const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
-        const cuuint32_t box[2] = {(cuuint32_t)(gemm::kTK / 2), (cuuint32_t)gemm::kTM};
+        const cuuint32_t box[2] = {(cuuint32_t)(gemm::kTK / 2), (cuuint32_t)box_rows};
         const cuuint32_t estr[2] = {1, 1};
         return encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
     };
-    if (!make(&ta, a_codes, M) || !make(&tb, b_codes, N)) return FP4Q_ERR_CUDA;
+    if (!make(&ta, a_codes, M, gemm::kTM) || !make(&tb, b_codes, N, gemm::kBN)) return FP4Q_ERR_CUDA;
     static int sms = 0;
     if (!sms) {
         int dev = 0;
@@ -469,10 +506,11 @@ extern "C" int fp4q_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, 
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
             return FP4Q_ERR_CUDA;
     }
-    const int m_tiles = (int)(M / gemm::kTM), n_tiles = (int)(N / gemm::kTN);
+    const int m_tiles = (int)(M / gemm::kTM), n_tiles = (int)((N + gemm::kBN - 1) / gemm::kBN);
     const int tiles = m_tiles * n_tiles;
     gemm::nvfp4_gemm_persistent_kernel<<<tiles < sms ? tiles : sms, gemm::kPThreads, gemm::kPersistSmem, st>>>(
-        ta, tb, a_scales, a_global_scale, b_scales, b_global_scale, (int)K, m_tiles, n_tiles, d, ldd, status);
+        ta, tb, a_scales, a_global_scale, b_scales, b_global_scale, (int)K, m_tiles, n_tiles,
+        (int)(N % gemm::kBN == 0), d, ldd, status);
 #endif
     if (cudaGetLastError() != cudaSuccess) return FP4Q_ERR_CUDA;
     g_launches = 1;

@@ -47,6 +47,24 @@ def test_nvfp4_gemm_matches_the_oracle_product(M, N, K):
     assert np.all(err <= 2e-5 * mag + 1e-30), float(np.max(err / (mag + 1e-30)))
 
 
+@pytest.mark.parametrize("M,N,K", [(4096, 2432, 512), (2048, 4096, 768)])
+def test_nvfp4_gemm_several_tiles_per_cta(M, N, K):
+    # more tiles than two per SM: the two overlapping accumulators alternate, 128-wide last tiles
+    # (N = 2432) mix with 256-wide ones, and the operand ring wraps across tiles (K = 768 is three
+    # stages per tile)
+    (qa, ra), (qb, rb) = _operand("cfg3", M, K, "sweep_mse"), _operand("cfg4", N, K, "absmax")
+    ws = fq.new_workspace()
+    d = fq.nvfp4_gemm(qa, qb, workspace=ws)
+    torch.cuda.synchronize()
+    assert fq.read_device_status(ws) == fq.DEVSTAT_OK
+    ref = O.nvfp4_gemm(ra["codes"], ra["scales"], ra["S"], rb["codes"], rb["scales"], rb["S"])
+    da = O.dequantize(ra["codes"], ra["scales"], ra["S"], "nvfp4").astype(np.float64)
+    db = O.dequantize(rb["codes"], rb["scales"], rb["S"], "nvfp4").astype(np.float64)
+    mag = np.abs(da) @ np.abs(db).T
+    err = np.abs(d.cpu().numpy().astype(np.float64) - ref)
+    assert np.all(err <= 2e-5 * mag + 1e-30), float(np.max(err / (mag + 1e-30)))
+
+
 def test_nvfp4_gemm_other_objectives_and_padding_rows():
     # AbsMax and 4/6 operands, and an output with a row pitch wider than N
     (qa, ra), (qb, rb) = _operand("cfg3", 128, 512, "absmax"), _operand("cfg4", 128, 512, "four_over_six")
