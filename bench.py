@@ -94,15 +94,19 @@ def load_peaks():
     return 6650.0, "fallback"
 
 
-def kernel_source_hash():
+QUANT_SOURCES = ("fp4_block_scaled_nvfp4_b200/csrc/fp4q.cu", "fp4_block_scaled_nvfp4_b200/csrc/fp4q_device.cuh")
+GEMM_SOURCES = ("fp4_block_scaled_nvfp4_b200/csrc/fp4q_gemm.cu",)
+
+
+def kernel_source_hash(files=QUANT_SOURCES):
     h = hashlib.sha256()
-    for f in ("fp4_block_scaled_nvfp4_b200/csrc/fp4q.cu", "fp4_block_scaled_nvfp4_b200/csrc/fp4q_device.cuh"):
+    for f in files:
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel_key):
+def profiled_traffic(kernel_key, files=QUANT_SOURCES):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on the current
     kernel source (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
@@ -111,7 +115,7 @@ def profiled_traffic(kernel_key):
     with open(p) as f:
         d = json.load(f)
     e = d.get(kernel_key)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(files):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -567,7 +571,8 @@ def run_gemm(args, rank, world):
                        "l2": "operands 46 MB stay L2-resident across steps (a GEMM reuses them by design)",
                        "timing": "CUDA events around back-to-back launches on one stream"},
             "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
-                         "frac": round(tf / peak, 4), "traffic": None, "kernel": "nvfp4_gemm_kernel",
+                         "frac": round(tf / peak, 4), "traffic": profiled_traffic("gemm:gemm", GEMM_SOURCES),
+                         "kernel": "nvfp4_gemm_persistent_kernel",
                          "peak_source": peak_src},
             "device_status": st, "gpu_launches": steps, "clocks": clk.summary(),
             "e2e": {"value": round(flops / (e2e_ms * 1e-3) / 1e12 * world, 3), "unit": "TFLOP/s",

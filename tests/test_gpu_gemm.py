@@ -47,11 +47,11 @@ def test_nvfp4_gemm_matches_the_oracle_product(M, N, K):
     assert np.all(err <= 2e-5 * mag + 1e-30), float(np.max(err / (mag + 1e-30)))
 
 
-@pytest.mark.parametrize("M,N,K", [(4096, 2432, 512), (2048, 4096, 768)])
+@pytest.mark.parametrize("M,N,K", [(256, 256, 512), (4096, 2432, 512), (2048, 4096, 768), (4096, 4096, 512)])
 def test_nvfp4_gemm_several_tiles_per_cta(M, N, K):
-    # more tiles than two per SM: the two overlapping accumulators alternate, 128-wide last tiles
-    # (N = 2432) mix with 256-wide ones, and the operand ring wraps across tiles (K = 768 is three
-    # stages per tile)
+    # one tile, and more tiles than two per SM: the two overlapping accumulators alternate,
+    # 128-wide last tiles (N = 2432) mix with 256-wide ones, and the operand ring wraps across
+    # tiles (K = 768 is three stages per tile)
     (qa, ra), (qb, rb) = _operand("cfg3", M, K, "sweep_mse"), _operand("cfg4", N, K, "absmax")
     ws = fq.new_workspace()
     d = fq.nvfp4_gemm(qa, qb, workspace=ws)
