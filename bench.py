@@ -53,6 +53,8 @@ METRIC = "quantize GB/s (input bf16) and % of B200 HBM peak, 1 GPU, vs CPU oracl
 # tcgen05 tensor cores, activations [M][K] (the 8192x4096 activation workload) times a weight
 # [N][K] (Llama-3-8B-shaped MLP up-projection, 14336x4096, Student-t weights), K contiguous.
 GEMM_METRIC = "NVFP4 block-scaled GEMM TFLOP/s (tcgen05), 1 GPU"
+GEMM_MX_METRIC = "MXFP4 block-scaled GEMM TFLOP/s (tcgen05), 1 GPU"
+GEMM_WORKLOADS = ("gemm", "gemm_mx")
 GEMM_SHAPE = (8192, 14336, 4096)
 # Arithmetic the method itself needs per element for the ALU-bound searches: per candidate
 # scale one multiply (x/s), one E2M1 rounding, one subtraction (residual) and one fused
@@ -206,7 +208,7 @@ def cpu_baseline(w, fmt, obj, budget_s=12.0):
 
 def run_reference(args, rank, world):
     """The oracle on the host cores as the reference arm: K steps, each a bounded row sample."""
-    if args.workload == "gemm":
+    if args.workload in GEMM_WORKLOADS:
         return run_reference_gemm(args, rank, world)
     cfg, fmt, obj, desc = WORKLOADS[args.workload]
     from fp4_block_scaled_nvfp4_b200 import synth
@@ -465,14 +467,19 @@ def fp4_peak_tflops():
     return 4.0 * 1590.0, "fallback bf16 1.59 PFLOP/s x 4"
 
 
-def gemm_operands(torch, fq, synth, dev):
+def gemm_operands(torch, fq, synth, dev, mx=False):
     M, N, K = GEMM_SHAPE
     wa = synth.make("cfg3", rows=M, cols=K)
     wb = synth.make("cfg2", rows=N, cols=K)
     xa = device_tensor_from_bits(wa["x"], torch).to(dev)
     xb = device_tensor_from_bits(wb["x"], torch).to(dev)
-    qa = fq.quantize(xa, "nvfp4", "sweep_mse", tiled_scales=True)
-    qb = fq.quantize(xb, "nvfp4", "sweep_mse", tiled_scales=True)
+    if mx:
+        # MXFP4 with the 32-point rotation on both operands (it cancels in the product)
+        qa = fq.hadamard_quantize(xa, tiled_scales=True)[:2]
+        qb = fq.hadamard_quantize(xb, tiled_scales=True)[:2]
+    else:
+        qa = fq.quantize(xa, "nvfp4", "sweep_mse", tiled_scales=True)
+        qb = fq.quantize(xb, "nvfp4", "sweep_mse", tiled_scales=True)
     return (M, N, K), qa, qb, wa, wb
 
 
@@ -484,13 +491,21 @@ def run_reference_gemm(args, rank, world):
     if rank != 0:
         return
     M, N, K = GEMM_SHAPE
+    mx = args.workload == "gemm_mx"
     wa = synth.make("cfg3", rows=16 * max(1, args.steps + args.warmup), cols=K)
     wb = synth.make("cfg2", rows=1024, cols=K)
-    ra = O.nvfp4_quantize(O.widen_bf16(wa["x"]), "sweep_mse")
-    rb = O.nvfp4_quantize(O.widen_bf16(wb["x"]), "sweep_mse")
+    if mx:
+        ra = O.mxfp4_quantize(O.widen_bf16(wa["x"]), hadamard=True)
+        rb = O.mxfp4_quantize(O.widen_bf16(wb["x"]), hadamard=True)
+    else:
+        ra = O.nvfp4_quantize(O.widen_bf16(wa["x"]), "sweep_mse")
+        rb = O.nvfp4_quantize(O.widen_bf16(wb["x"]), "sweep_mse")
     def step(i):
         sl = slice(16 * i, 16 * i + 16)
-        O.nvfp4_gemm(ra["codes"][sl], ra["scales"][sl], ra["S"], rb["codes"], rb["scales"], rb["S"])
+        if mx:
+            O.mxfp4_gemm(ra["codes"][sl], ra["scales"][sl], rb["codes"], rb["scales"])
+        else:
+            O.nvfp4_gemm(ra["codes"][sl], ra["scales"][sl], ra["S"], rb["codes"], rb["scales"], rb["S"])
     for i in range(args.warmup):
         step(i)
     t0 = time.perf_counter()
@@ -498,10 +513,12 @@ def run_reference_gemm(args, rank, world):
         step(args.warmup + i)
     dt = time.perf_counter() - t0
     val = 2.0 * 16 * 1024 * K * args.steps / dt / 1e12
-    line = {"impl": "reference", "metric": GEMM_METRIC, "value": round(val, 6), "unit": "TFLOP/s", "n_gpus": world,
+    line = {"impl": "reference", "metric": GEMM_MX_METRIC if mx else GEMM_METRIC, "value": round(val, 6),
+            "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "NVFP4 GEMM on the oracle", "M": M, "N": N, "K": K, "step_sample": "16 x 1024 x K"},
+            "config": {"workload": ("MXFP4 (rotated)" if mx else "NVFP4") + " GEMM on the oracle", "M": M, "N": N,
+                       "K": K, "step_sample": "16 x 1024 x K"},
             "cpu_baseline": {"value": round(val, 6), "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
                              "sample": "16 activation rows times 1024 weight rows per step"},
             "e2e": {"value": round(val, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -516,13 +533,15 @@ def run_gemm(args, rank, world):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     fq.lib()
-    (M, N, K), qa, qb, wa, wb = gemm_operands(torch, fq, synth, dev)
+    mx = args.workload == "gemm_mx"
+    gemm = fq.mxfp4_gemm if mx else fq.nvfp4_gemm
+    (M, N, K), qa, qb, wa, wb = gemm_operands(torch, fq, synth, dev, mx=mx)
     d = torch.empty((M, N), dtype=torch.float32, device=dev)
     ws = fq.new_workspace(dev)
     stream = torch.cuda.Stream(device=dev)
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
-            fq.nvfp4_gemm(qa, qb, out=d, workspace=ws)
+            gemm(qa, qb, out=d, workspace=ws)
     torch.cuda.synchronize()
     flops = 2.0 * M * N * K
     steps = args.steps
@@ -531,7 +550,7 @@ def run_gemm(args, rank, world):
         with torch.cuda.stream(stream):
             start.record()
             for _ in range(steps):
-                fq.nvfp4_gemm(qa, qb, out=d, workspace=ws)
+                gemm(qa, qb, out=d, workspace=ws)
             end.record()
         end.synchronize()
     ms = start.elapsed_time(end) / steps
@@ -553,7 +572,8 @@ def run_gemm(args, rank, world):
         for _ in range(e_steps):
             for h, g in zip(hosts, devs):
                 g.copy_(h, non_blocking=True)
-            fq.nvfp4_gemm(tuple(devs[:3]), tuple(devs[3:]), out=d, workspace=ws)
+            na = len(qa)
+            gemm(tuple(devs[:na]), tuple(devs[na:]), out=d, workspace=ws)
             d_host.copy_(d, non_blocking=True)
         e1.record()
     e1.synchronize()
@@ -562,29 +582,40 @@ def run_gemm(args, rank, world):
         return
     peak, peak_src = fp4_peak_tflops()
     tf = flops / (ms * 1e-3) / 1e12
-    line = {"metric": GEMM_METRIC, "value": round(tf * world, 1), "unit": "TFLOP/s", "n_gpus": world, "steps": steps,
+    line = {"metric": GEMM_MX_METRIC if mx else GEMM_METRIC, "value": round(tf * world, 1), "unit": "TFLOP/s",
+            "n_gpus": world, "steps": steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "e2m1xe2m1->f32", "data": "synthetic",
-            "config": {"workload": "NVFP4 GEMM, activations 8192x4096 (activation workload, sweep-MSE) times weight "
-                                   "14336x4096 (Student-t, sweep-MSE), K contiguous, tiled scales, fp32 out",
+            "config": {"workload": ("MXFP4 GEMM, activations 8192x4096 (activation workload) times weight 14336x4096 "
+                                    "(Student-t), both rotated by the 32-point block Hadamard, K contiguous, tiled "
+                                    "E8M0 scales, fp32 out") if mx else
+                                   ("NVFP4 GEMM, activations 8192x4096 (activation workload, sweep-MSE) times weight "
+                                    "14336x4096 (Student-t, sweep-MSE), K contiguous, tiled scales, fp32 out"),
                        "M": M, "N": N, "K": K, "parallelism": f"replicas{world}" if world > 1 else "single",
                        "l2": "operands 46 MB stay L2-resident across steps (a GEMM reuses them by design)",
                        "timing": "CUDA events around back-to-back launches on one stream"},
             "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
-                         "frac": round(tf / peak, 4), "traffic": profiled_traffic("gemm:gemm", GEMM_SOURCES),
-                         "kernel": "nvfp4_gemm_persistent_kernel",
+                         "frac": round(tf / peak, 4), "traffic": profiled_traffic(f"{args.workload}:gemm", GEMM_SOURCES),
+                         "kernel": f"fp4_gemm_kernel<{'true' if mx else 'false'}>",
                          "peak_source": peak_src},
             "device_status": st, "gpu_launches": steps, "clocks": clk.summary(),
             "e2e": {"value": round(flops / (e2e_ms * 1e-3) / 1e12 * world, 3), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": int(sum(h.numel() * h.element_size() for h in hosts)),
                     "d2h_bytes_per_step": M * N * 4, "ms_per_step": round(e2e_ms, 3), "steps": e_steps,
-                    "api": "operands from pinned host memory, fp4q_nvfp4_gemm, product back to pinned host memory"}}
+                    "api": f"operands from pinned host memory, fp4q_{'mx' if mx else 'nv'}fp4_gemm, product back to "
+                           "pinned host memory"}}
     if args.cpu_baseline:
         import oracle as O
-        ra = O.nvfp4_quantize(O.widen_bf16(wa["x"][:64]), "sweep_mse", S=float(qa[2].cpu()[0]))
-        rb = O.nvfp4_quantize(O.widen_bf16(wb["x"]), "sweep_mse")
-        t0 = time.perf_counter()
-        O.nvfp4_gemm(ra["codes"], ra["scales"], ra["S"], rb["codes"], rb["scales"], rb["S"])
+        if mx:
+            ra = O.mxfp4_quantize(O.widen_bf16(wa["x"][:64]), hadamard=True)
+            rb = O.mxfp4_quantize(O.widen_bf16(wb["x"]), hadamard=True)
+            t0 = time.perf_counter()
+            O.mxfp4_gemm(ra["codes"], ra["scales"], rb["codes"], rb["scales"])
+        else:
+            ra = O.nvfp4_quantize(O.widen_bf16(wa["x"][:64]), "sweep_mse", S=float(qa[2].cpu()[0]))
+            rb = O.nvfp4_quantize(O.widen_bf16(wb["x"]), "sweep_mse")
+            t0 = time.perf_counter()
+            O.nvfp4_gemm(ra["codes"], ra["scales"], ra["S"], rb["codes"], rb["scales"], rb["S"])
         dt = time.perf_counter() - t0
         line["cpu_baseline"] = {"value": round(2.0 * 64 * N * K / dt / 1e12, 6), "unit": "TFLOP/s", "cores": 1,
                                 "kind": "oracle", "sample": f"64 of {M} activation rows times the whole weight, "
@@ -598,7 +629,7 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["gemm"], default="cfg3")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + list(GEMM_WORKLOADS), default="cfg3")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()
@@ -613,7 +644,7 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, rank, world)
-        elif args.workload == "gemm":
+        elif args.workload in GEMM_WORKLOADS:
             run_gemm(args, rank, world)
         else:
             run_ours(args, rank, world)

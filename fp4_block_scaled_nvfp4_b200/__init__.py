@@ -27,7 +27,7 @@ F_SCALE_TILED = 0x80
 BLOCK = {"nvfp4": 16, "if4": 16, "mxfp4": 32}
 
 # Names of every function include/fp4q.h declares (checked against the header by the tests).
-EXPORTS = ("fp4q_workspace_bytes", "fp4q_scale_bytes", "fp4q_nvfp4_gemm", "fp4q_global_scale", "fp4q_hadamard_global_scale", "fp4q_quantize",
+EXPORTS = ("fp4q_workspace_bytes", "fp4q_scale_bytes", "fp4q_nvfp4_gemm", "fp4q_mxfp4_gemm", "fp4q_global_scale", "fp4q_hadamard_global_scale", "fp4q_quantize",
            "fp4q_hadamard_quantize", "fp4q_dequantize", "fp4q_quantize_noalloc", "fp4q_quantize_host_async", "fp4q_read_device_status", "fp4q_last_launch_count", "fp4q_status_string")
 
 _lib = None
@@ -51,6 +51,8 @@ def lib():
         L.fp4q_scale_bytes.argtypes = [i64, i64, i32, u32]
         L.fp4q_nvfp4_gemm.restype = i32
         L.fp4q_nvfp4_gemm.argtypes = [P, P, P, P, P, P, i64, i64, i64, P, i64, P, P]
+        L.fp4q_mxfp4_gemm.restype = i32
+        L.fp4q_mxfp4_gemm.argtypes = [P, P, P, P, i64, i64, i64, P, i64, P, P]
         L.fp4q_quantize.restype = i32
         L.fp4q_quantize.argtypes = [P, i32, i64, i64, i64, i32, i32, P, P, P, P, P, u32, P]
         L.fp4q_global_scale.restype = i32
@@ -259,6 +261,26 @@ def nvfp4_gemm(a, b, out=None, workspace=None, stream=None):
     rc = lib().fp4q_nvfp4_gemm(_ptr(ac), _ptr(asc), _ptr(ag), _ptr(bc), _ptr(bsc), _ptr(bg), M, N, K, _ptr(d),
                                d.stride(0), _ptr(ws), _stream_ptr(stream))
     _check(rc, "fp4q_nvfp4_gemm")
+    return d
+
+
+def mxfp4_gemm(a, b, out=None, workspace=None, stream=None):
+    """Block-scaled MXFP4 GEMM on the tensor cores: a = (codes [M, K/2], tiled E8M0 scales) and
+    b = (codes [N, K/2], tiled E8M0 scales) as returned by quantize / hadamard_quantize(...,
+    "mxfp4", tiled_scales=True) (a third element, the absent tensor scale, is ignored);
+    returns fp32 [M, N] = A B^T.  M, N multiples of 128, K a multiple of 256."""
+    torch = _torch()
+    ac, asc = a[0], a[1]
+    bc, bsc = b[0], b[1]
+    M, K = ac.shape[0], ac.shape[1] * 2
+    N = bc.shape[0]
+    if bc.shape[1] * 2 != K:
+        raise Fp4qError("a and b must have the same K")
+    d = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=ac.device)
+    ws = workspace if workspace is not None else new_workspace(ac.device)
+    rc = lib().fp4q_mxfp4_gemm(_ptr(ac), _ptr(asc), _ptr(bc), _ptr(bsc), M, N, K, _ptr(d), d.stride(0), _ptr(ws),
+                               _stream_ptr(stream))
+    _check(rc, "fp4q_mxfp4_gemm")
     return d
 
 

@@ -12,7 +12,7 @@
 // kind::mxf4nvf4, 16-element scale blocks) accumulating fp32 in tensor memory; the epilogue
 // reads the accumulator back with tcgen05.ld (each warp its lane quarter), multiplies by
 // RN(S_a S_b) and stores D.
-//   nvfp4_gemm_persistent_kernel (the one launched): one CTA per SM over all tiles, a
+//   fp4_gemm_kernel<MX> (the one launched; MX selects MXFP4 operands): one CTA per SM over all tiles, a
 //     five-stage ring filled by tensor copies, producer / MMA / epilogue warps, two
 //     accumulators so the epilogue of a tile overlaps the next tile's MMAs.
 //   nvfp4_gemm_kernel (build flag FP4Q_GEMM_SIMPLE): the same arithmetic in one stage with
@@ -255,8 +255,15 @@ constexpr uint32_t kPColSFA = 448, kPColSFB = 464;
 constexpr int kPersistSmem = kPStages * kPStageBytes + 1024 + 256;
 constexpr uint32_t kIdescN256 = (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(kTM >> 4) << 24);
 
+// MX = false: NVFP4 operands (E4M3 factor per 16 elements, tensor scales S_a, S_b); MX = true:
+// MXFP4 operands (E8M0 factor per 32 elements, no tensor scale).  An MXFP4 scale atom covers
+// K = 128 (four 32-element blocks per row), so a stage holds two atoms per 128 rows instead of
+// four, and each K = 64 MMA reads two of a 32-bit column's four factor bytes: the byte offset
+// (0 or 2) goes into the tensor-memory address's top bits and the instruction descriptor's
+// factor-id fields.
+template <bool MX>
 __global__ void __launch_bounds__(kPThreads, 1)
-    nvfp4_gemm_persistent_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
+    fp4_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                                  const uint8_t* __restrict__ sfa, const float* __restrict__ sa,
                                  const uint8_t* __restrict__ sfb, const float* __restrict__ sb, int K, int m_tiles,
                                  int n_tiles, int n_last_wide, float* __restrict__ d, int64_t ldd,
@@ -271,7 +278,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
     __shared__ volatile int s_fail;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t jt = K / 64;
+    constexpr int kAtoms = MX ? 2 : 4;                     // scale atoms per 128 rows and stage
+    constexpr uint32_t kSfCopy = kAtoms * 512;
+    const int64_t jt = K / (MX ? 128 : 64);                // scale atoms per 128 rows
     const int KT = K / kTK;
     const int tiles = m_tiles * n_tiles;
     // the last tile of each row of tiles is 128 wide unless N is a multiple of 256
@@ -306,7 +315,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
             const int mt = t / n_tiles, nt = t - mt * n_tiles;
             const bool wide = wide_tile(nt);
             // a tensor copy's transaction count is its whole box, rows past N included
-            const uint32_t bytes = (uint32_t)(kTileBytes + kBTileBytes + (wide ? 3 : 2) * kSfBytes);
+            const uint32_t bytes = (uint32_t)(kTileBytes + kBTileBytes) + (wide ? 3u : 2u) * kSfCopy;
             for (int kt = 0; kt < KT; ++kt, ++g) {
                 const uint32_t s = g % kPStages, round = g / kPStages;
                 if (!mbar_wait(smem_u32(empty + s), (round & 1u) ^ 1u)) { s_fail = 1; break; }
@@ -324,15 +333,15 @@ __global__ void __launch_bounds__(kPThreads, 1)
                        "r"(fb)
                     : "memory");
                 uint8_t* ssf = st + kTileBytes + kBTileBytes;
-                const uint8_t* gsa = sfa + ((int64_t)mt * jt + 4 * kt) * 512;
-                const uint8_t* gsb = sfb + ((int64_t)(2 * nt) * jt + 4 * kt) * 512;
+                const uint8_t* gsa = sfa + ((int64_t)mt * jt + kAtoms * kt) * 512;
+                const uint8_t* gsb = sfb + ((int64_t)(2 * nt) * jt + kAtoms * kt) * 512;
                 asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                             :: "r"(smem_u32(ssf)), "l"(gsa), "r"((uint32_t)kSfBytes), "r"(fb) : "memory");
+                             :: "r"(smem_u32(ssf)), "l"(gsa), "r"(kSfCopy), "r"(fb) : "memory");
                 asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                             :: "r"(smem_u32(ssf + kSfBytes)), "l"(gsb), "r"((uint32_t)kSfBytes), "r"(fb) : "memory");
+                             :: "r"(smem_u32(ssf + kSfBytes)), "l"(gsb), "r"(kSfCopy), "r"(fb) : "memory");
                 if (wide)
                     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                                 :: "r"(smem_u32(ssf + 2 * kSfBytes)), "l"(gsb + jt * 512), "r"((uint32_t)kSfBytes), "r"(fb)
+                                 :: "r"(smem_u32(ssf + 2 * kSfBytes)), "l"(gsb + jt * 512), "r"(kSfCopy), "r"(fb)
                                  : "memory");
             }
         }
@@ -343,7 +352,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
         for (int t = blockIdx.x; t < tiles && !s_fail; t += gridDim.x, ++j) {
             const int nt = t % n_tiles;
             const bool wide = wide_tile(nt);
-            const uint32_t idesc = wide ? kIdescN256 : kIdesc;
+            const uint32_t idesc = (wide ? kIdescN256 : kIdesc) | (MX ? (1u << 23) : 0u);   // E8M0 factors
             // the previous tile's epilogue has read the columns this accumulator shares with it
             if (j > 0 && !mbar_wait(smem_u32(acc_free), (uint32_t)((j - 1) & 1))) { s_fail = 1; break; }
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
@@ -355,7 +364,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 uint8_t* st = smem + s * kPStageBytes;
                 uint8_t* ssf = st + kTileBytes + kBTileBytes;
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
+                for (int kk = 0; kk < kAtoms; ++kk) {
                     const uint64_t da = smem_desc(smem_u32(ssf + kk * 512), 16, 128, 0);
                     const uint64_t db0 = smem_desc(smem_u32(ssf + kSfBytes + kk * 512), 16, 128, 0);
                     asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;"
@@ -373,13 +382,26 @@ __global__ void __launch_bounds__(kPThreads, 1)
                     const uint64_t adesc = smem_desc(smem_u32(st + kk * 32), 16, 1024, 2);
                     const uint64_t bdesc = smem_desc(smem_u32(st + kTileBytes + kk * 32), 16, 1024, 2);
                     const uint32_t accumulate = (kt > 0 || kk > 0) ? 1u : 0u;
-                    asm volatile(
-                        "{ .reg .pred p;\n"
-                        "  setp.ne.b32 p, %4, 0;\n"
-                        "  tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p; }"
-                        :: "r"(tacc), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate),
-                           "r"(tmem + kPColSFA + 4 * kk), "r"(tmem + kPColSFB + 8 * kk)
-                        : "memory");
+                    if constexpr (MX) {
+                        const uint32_t id = (uint32_t)(kk & 1) * 2u;   // factor bytes 2 kk % 4 .. + 1
+                        const uint32_t sfa_t = (tmem + kPColSFA + 4 * (kk >> 1)) | (id << 30);
+                        const uint32_t sfb_t = (tmem + kPColSFB + 8 * (kk >> 1)) | (id << 30);
+                        asm volatile(
+                            "{ .reg .pred p;\n"
+                            "  setp.ne.b32 p, %4, 0;\n"
+                            "  tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p; }"
+                            :: "r"(tacc), "l"(adesc), "l"(bdesc), "r"(idesc | (id << 29) | (id << 4)), "r"(accumulate),
+                               "r"(sfa_t), "r"(sfb_t)
+                            : "memory");
+                    } else {
+                        asm volatile(
+                            "{ .reg .pred p;\n"
+                            "  setp.ne.b32 p, %4, 0;\n"
+                            "  tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p; }"
+                            :: "r"(tacc), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate),
+                               "r"(tmem + kPColSFA + 4 * kk), "r"(tmem + kPColSFB + 8 * kk)
+                            : "memory");
+                    }
                 }
                 asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                              :: "r"(smem_u32(empty + s)) : "memory");
@@ -392,7 +414,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     } else if (warp >= 2) {
         // epilogue: this warp owns tensor-memory lanes 32 (warp % 4) .. + 31
         const int q = warp & 3;
-        const float scale = __fmul_rn(*sa, *sb);
+        const float scale = MX ? 1.0f : __fmul_rn(*sa, *sb);
         int j = 0;
         for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++j) {
             // warp-uniform decisions: the tensor-memory loads below are warp-collective
@@ -441,17 +463,20 @@ __global__ void __launch_bounds__(kPThreads, 1)
 }  // namespace gemm
 }  // namespace fp4q
 
-extern "C" int fp4q_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global_scale,
-                               const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global_scale,
-                               int64_t M, int64_t N, int64_t K, float* d, int64_t ldd, void* workspace,
-                               void* stream) {
-    using namespace fp4q;
+namespace fp4q {
+namespace gemm {
+
+// Shared host path of the two entry points: argument checks, tensor maps, launch.
+template <bool MX>
+int launch(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global_scale, const uint8_t* b_codes,
+           const uint8_t* b_scales, const float* b_global_scale, int64_t M, int64_t N, int64_t K, float* d, int64_t ldd,
+           void* workspace, void* stream) {
     g_launches = 0;
-    if (M < 0 || N < 0 || K < 0 || M % gemm::kTM || N % gemm::kTN || K % gemm::kTK || ldd < N) return FP4Q_ERR_SHAPE;
-    if (M / gemm::kTM > 65535 || K > (1 << 30)) return FP4Q_ERR_SHAPE;
+    if (M < 0 || N < 0 || K < 0 || M % kTM || N % kTN || K % kTK || ldd < N) return FP4Q_ERR_SHAPE;
+    if (M / kTM > 65535 || K > (1 << 30)) return FP4Q_ERR_SHAPE;
     if (M == 0 || N == 0 || K == 0) return FP4Q_OK;
-    if (!a_codes || !a_scales || !a_global_scale || !b_codes || !b_scales || !b_global_scale || !d || !workspace)
-        return FP4Q_ERR_INVALID_ARG;
+    if (!a_codes || !a_scales || !b_codes || !b_scales || !d || !workspace) return FP4Q_ERR_INVALID_ARG;
+    if (!MX && (!a_global_scale || !b_global_scale)) return FP4Q_ERR_INVALID_ARG;
     auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
     if (!al16(a_codes) || !al16(a_scales) || !al16(b_codes) || !al16(b_scales) || !al16(d) || !al16(workspace) ||
         ldd % 4)
@@ -459,21 +484,22 @@ extern "C" int fp4q_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     uint32_t* status = reinterpret_cast<uint32_t*>(workspace);
     if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return FP4Q_ERR_CUDA;
-    const dim3 grid((unsigned)(N / gemm::kTN), (unsigned)(M / gemm::kTM));
 #if FP4Q_GEMM_SIMPLE
+    if (MX) return FP4Q_ERR_UNSUPPORTED;
     static bool attr_set = false;
     if (!attr_set) {
-        if (cudaFuncSetAttribute(gemm::nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 gemm::kSmemAlloc) != cudaSuccess)
+        if (cudaFuncSetAttribute(nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc) !=
+            cudaSuccess)
             return FP4Q_ERR_CUDA;
         attr_set = true;
     }
-    gemm::nvfp4_gemm_kernel<<<grid, gemm::kThreads, gemm::kSmemAlloc, st>>>(
-        a_codes, a_scales, a_global_scale, b_codes, b_scales, b_global_scale, (int)K, d, ldd, status);
+    const dim3 grid((unsigned)(N / kTN), (unsigned)(M / kTM));
+    nvfp4_gemm_kernel<<<grid, kThreads, kSmemAlloc, st>>>(a_codes, a_scales, a_global_scale, b_codes, b_scales,
+                                                          b_global_scale, (int)K, d, ldd, status);
 #else
-    // the tensor-copy descriptors of A and B: [rows][K/2] bytes, 128 x 128-byte boxes, 128-byte swizzle
+    // the tensor-copy descriptors of A and B: [rows][K/2] bytes, 128-byte-wide boxes of 128 (A) or
+    // 256 (B) rows, 128-byte swizzle
     static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
-    static bool attr_set = false;
     if (!encode) {
         void* fn = nullptr;
         cudaDriverEntryPointQueryResult q;
@@ -482,9 +508,10 @@ extern "C" int fp4q_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, 
             return FP4Q_ERR_CUDA;
         encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
+    static bool attr_set = false;
     if (!attr_set) {
-        if (cudaFuncSetAttribute(gemm::nvfp4_gemm_persistent_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 gemm::kPersistSmem) != cudaSuccess)
+        if (cudaFuncSetAttribute(fp4_gemm_kernel<MX>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPersistSmem) !=
+            cudaSuccess)
             return FP4Q_ERR_CUDA;
         attr_set = true;
     }
@@ -492,13 +519,13 @@ extern "C" int fp4q_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, 
     auto make = [&](CUtensorMap* m, const uint8_t* base, int64_t rows, int box_rows) {
         const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
         const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
-        const cuuint32_t box[2] = {(cuuint32_t)(gemm::kTK / 2), (cuuint32_t)box_rows};
+        const cuuint32_t box[2] = {(cuuint32_t)(kTK / 2), (cuuint32_t)box_rows};
         const cuuint32_t estr[2] = {1, 1};
         return encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
     };
-    if (!make(&ta, a_codes, M, gemm::kTM) || !make(&tb, b_codes, N, gemm::kBN)) return FP4Q_ERR_CUDA;
+    if (!make(&ta, a_codes, M, kTM) || !make(&tb, b_codes, N, kBN)) return FP4Q_ERR_CUDA;
     static int sms = 0;
     if (!sms) {
         int dev = 0;
@@ -506,13 +533,31 @@ extern "C" int fp4q_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, 
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
             return FP4Q_ERR_CUDA;
     }
-    const int m_tiles = (int)(M / gemm::kTM), n_tiles = (int)((N + gemm::kBN - 1) / gemm::kBN);
+    const int m_tiles = (int)(M / kTM), n_tiles = (int)((N + kBN - 1) / kBN);
     const int tiles = m_tiles * n_tiles;
-    gemm::nvfp4_gemm_persistent_kernel<<<tiles < sms ? tiles : sms, gemm::kPThreads, gemm::kPersistSmem, st>>>(
-        ta, tb, a_scales, a_global_scale, b_scales, b_global_scale, (int)K, m_tiles, n_tiles,
-        (int)(N % gemm::kBN == 0), d, ldd, status);
+    fp4_gemm_kernel<MX><<<tiles < sms ? tiles : sms, kPThreads, kPersistSmem, st>>>(
+        ta, tb, a_scales, a_global_scale, b_scales, b_global_scale, (int)K, m_tiles, n_tiles, (int)(N % kBN == 0), d,
+        ldd, status);
 #endif
     if (cudaGetLastError() != cudaSuccess) return FP4Q_ERR_CUDA;
     g_launches = 1;
     return FP4Q_OK;
+}
+
+}  // namespace gemm
+}  // namespace fp4q
+
+extern "C" int fp4q_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global_scale,
+                               const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global_scale,
+                               int64_t M, int64_t N, int64_t K, float* d, int64_t ldd, void* workspace,
+                               void* stream) {
+    return fp4q::gemm::launch<false>(a_codes, a_scales, a_global_scale, b_codes, b_scales, b_global_scale, M, N, K, d,
+                                     ldd, workspace, stream);
+}
+
+extern "C" int fp4q_mxfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* b_codes,
+                               const uint8_t* b_scales, int64_t M, int64_t N, int64_t K, float* d, int64_t ldd,
+                               void* workspace, void* stream) {
+    return fp4q::gemm::launch<true>(a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, M, N, K, d, ldd, workspace,
+                                    stream);
 }

@@ -300,6 +300,20 @@ int fp4q_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float
                     int64_t M, int64_t N, int64_t K, float* d, int64_t ldd, void* workspace,
                     void* stream);
 
+/*
+ * The same GEMM for two MXFP4 operands: d[m][n] = sum_k A[m][k] * B[n][k] in fp32, where
+ * A and B are MXFP4 tensors as fp4q_quantize or fp4q_hadamard_quantize writes them with
+ * FP4Q_F_SCALE_TILED (E8M0 scale bytes, one per 32 elements, in the tiled layout of
+ * fp4q_scale_bytes); MXFP4 has no tensor scale.  When both operands were rotated with the
+ * same 32-point block Hadamard along K, the rotations cancel in the product (the normalized
+ * transform is orthogonal), so d approximates the product of the unrotated tensors (Bridging
+ * the Gap ... Microscaling FP4, "Methodology": rotations folded into the adjacent weights).
+ * Shapes, alignment, layout of d, workspace and errors as for fp4q_nvfp4_gemm.
+ */
+int fp4q_mxfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* b_codes,
+                    const uint8_t* b_scales, int64_t M, int64_t N, int64_t K, float* d, int64_t ldd,
+                    void* workspace, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -258,6 +258,25 @@ def nvfp4_gemm(a_codes, a_scales, Sa, b_codes, b_scales, Sb):
     return float(Sa) * float(Sb) * (values(a_codes, a_scales) @ values(b_codes, b_scales).T)
 
 
+def mxfp4_gemm(a_codes, a_scales, b_codes, b_scales):
+    """D[m][n] = sum_k qa[m][k] 2^(sa[m][k/32]-127) qb[n][k] 2^(sb[n][k/32]-127) in float64: the
+    product of two MXFP4 operands stored with K contiguous (codes [rows][K/2], row-major E8M0
+    scale bytes [rows][K/32]); MXFP4 has no tensor scale.  Element values from the oracle's own
+    E2M1 table times the E8M0 power of two (byte 0xFF, E8M0's NaN, gives NaN).  Each term is
+    exact in float64 (the products span far fewer than 2^10 binades here) and the sums are a
+    float64 matmul."""
+    def values(codes, scales):
+        codes = np.asarray(codes, np.uint8)
+        rows, half = codes.shape
+        q = np.empty((rows, 2 * half), np.float64)
+        tab = np.array([lib().fp4q_o_e2m1_value(c) for c in range(16)], np.float64)
+        q[:, 0::2] = tab[codes & 0xF]
+        q[:, 1::2] = tab[codes >> 4]
+        e = np.array([np.ldexp(1.0, b - 127) if b != 0xFF else np.nan for b in range(256)], np.float64)
+        return q * np.repeat(e[np.asarray(scales, np.uint8)], 32, axis=1)
+    return values(a_codes, a_scales) @ values(b_codes, b_scales).T
+
+
 def widen_bf16(bits) -> np.ndarray:
     """bf16 bit patterns -> float32 (exact), the oracle's own input widening."""
     b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)

@@ -54,6 +54,16 @@ def test_gemm_rejects_before_launch():
     assert call(128, 128, 256, d=F + 4) == fq.ERR_ALIGNMENT
     assert call(128, 128, 256, ldd=130) == fq.ERR_ALIGNMENT
     assert call(0, 128, 256, a=None, d=None, ws=None) == fq.OK and L.fp4q_last_launch_count() == 0
+    # the MXFP4 form: the same checks, no tensor scales
+    mx = lambda M, N, K, ldd=None, **kw: L.fp4q_mxfp4_gemm(kw.get("a", F), F, F, kw.get("bs", F), M, N, K,
+                                                           kw.get("d", F), N if ldd is None else ldd,
+                                                           kw.get("ws", F), None)
+    assert mx(100, 128, 256) == fq.ERR_SHAPE
+    assert mx(128, 128, 384) == fq.ERR_SHAPE
+    assert mx(128, 128, 256, a=None) == fq.ERR_INVALID_ARG
+    assert mx(128, 128, 256, bs=None) == fq.ERR_INVALID_ARG
+    assert mx(128, 128, 256, d=F + 8) == fq.ERR_ALIGNMENT
+    assert mx(0, 128, 256, a=None, d=None, ws=None) == fq.OK and L.fp4q_last_launch_count() == 0
 
 
 def test_status_strings_and_workspace():

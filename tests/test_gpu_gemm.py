@@ -77,3 +77,36 @@ def test_nvfp4_gemm_other_objectives_and_padding_rows():
     got = d.cpu().numpy()
     assert np.all(np.abs(got[:, :128] - ref) <= 2e-5 * (np.abs(da) @ np.abs(db).T) + 1e-30)
     assert np.all(got[:, 128:] == 7.0)
+
+
+def _mx_operand(cfg, rows, cols, had, sweep=False):
+    w = synth.make(cfg, rows=rows, cols=cols)
+    xd = torch.from_numpy(w["x"].view(np.int16)).view(torch.bfloat16).cuda()
+    if had:
+        q = fq.hadamard_quantize(xd, mx_sweep=sweep, tiled_scales=True)
+    else:
+        q = fq.quantize(xd, "mxfp4", mx_sweep=sweep, tiled_scales=True)
+    x = O.widen_bf16(w["x"])
+    r = O.mxfp4_quantize(x, hadamard=had, sweep="sweep" if sweep else "rule")
+    return q, r, x
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 128, 256), (256, 384, 1024), (4096, 2432, 512)])
+@pytest.mark.parametrize("had", [False, True])
+def test_mxfp4_gemm_matches_the_oracle_product(M, N, K, had):
+    (qa, ra, xa), (qb, rb, xb) = _mx_operand("cfg5", M, K, had), _mx_operand("cfg4", N, K, had, sweep=True)
+    assert np.array_equal(qa[0].cpu().numpy(), ra["codes"]) and np.array_equal(qb[0].cpu().numpy(), rb["codes"])
+    ws = fq.new_workspace()
+    d = fq.mxfp4_gemm(qa, qb, workspace=ws)
+    torch.cuda.synchronize()
+    assert fq.read_device_status(ws) == fq.DEVSTAT_OK
+    assert fq.last_launch_count() == 1
+    ref = O.mxfp4_gemm(ra["codes"], ra["scales"], rb["codes"], rb["scales"])
+    da = O.dequantize(ra["codes"], ra["scales"], 0.0, "mxfp4").astype(np.float64)
+    db = O.dequantize(rb["codes"], rb["scales"], 0.0, "mxfp4").astype(np.float64)
+    mag = np.abs(da) @ np.abs(db).T
+    got = d.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(got - ref) <= 2e-5 * mag + 1e-30), float(np.max(np.abs(got - ref) / (mag + 1e-30)))
+    # the rotations cancel in the product: either way it approximates the unrotated product
+    exact = xa.astype(np.float64) @ xb.astype(np.float64).T
+    assert np.linalg.norm(got - exact) <= 0.25 * np.linalg.norm(exact)

@@ -466,6 +466,28 @@ def test_nvfp4_gemm_oracle():
     assert np.all(np.abs(d - da @ db.T) <= 2 ** -22 * mag)
 
 
+def test_mxfp4_gemm_oracle():
+    # against a triple loop over exact rationals (E8M0 byte b is the power of two 2^(b - 127)),
+    # and against the float64 product of the dequantized operands, plain and rotated
+    rng = np.random.default_rng(6)
+    a = (rng.normal(size=(3, 64)) * 3).astype(np.float32)
+    b = (rng.normal(size=(2, 64)) * 0.01).astype(np.float32)
+    for had in (False, True):
+        ra, rb = O.mxfp4_quantize(a, hadamard=had), O.mxfp4_quantize(b, hadamard=had)
+        d = O.mxfp4_gemm(ra["codes"], ra["scales"], rb["codes"], rb["scales"])
+        def val(codes, scales, r, k):
+            c = (int(codes[r, k // 2]) >> (4 * (k % 2))) & 0xF
+            g = GRID[c & 7] * (-1 if c & 8 else 1)
+            return g * Fr(2) ** (int(scales[r, k // 32]) - 127)
+        for m in range(3):
+            for n in range(2):
+                exact = sum(val(ra["codes"], ra["scales"], m, k) * val(rb["codes"], rb["scales"], n, k) for k in range(64))
+                assert abs(d[m, n] - float(exact)) <= 1e-12 * max(1.0, abs(float(exact)))
+        da = O.dequantize(ra["codes"], ra["scales"], 0.0, "mxfp4").astype(np.float64)
+        db = O.dequantize(rb["codes"], rb["scales"], 0.0, "mxfp4").astype(np.float64)
+        assert np.array_equal(d, da @ db.T)   # the dequantized values are exact here
+
+
 def test_hadamard_is_normalized_sylvester():
     H = np.array([[1.0]])
     while H.shape[0] < 32:
