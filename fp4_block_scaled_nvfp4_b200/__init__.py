@@ -27,7 +27,7 @@ F_SCALE_TILED = 0x80
 BLOCK = {"nvfp4": 16, "if4": 16, "mxfp4": 32}
 
 # Names of every function include/fp4q.h declares (checked against the header by the tests).
-EXPORTS = ("fp4q_workspace_bytes", "fp4q_scale_bytes", "fp4q_nvfp4_gemm", "fp4q_mxfp4_gemm", "fp4q_global_scale", "fp4q_hadamard_global_scale", "fp4q_quantize",
+EXPORTS = ("fp4q_workspace_bytes", "fp4q_scale_bytes", "fp4q_nvfp4_gemm", "fp4q_mxfp4_gemm", "fp4q_encode", "fp4q_global_scale", "fp4q_hadamard_global_scale", "fp4q_quantize",
            "fp4q_hadamard_quantize", "fp4q_dequantize", "fp4q_quantize_noalloc", "fp4q_quantize_host_async", "fp4q_read_device_status", "fp4q_last_launch_count", "fp4q_status_string")
 
 _lib = None
@@ -52,6 +52,8 @@ def lib():
         L.fp4q_nvfp4_gemm.restype = i32
         L.fp4q_nvfp4_gemm.argtypes = [P, P, P, P, P, P, i64, i64, i64, P, i64, P, P]
         L.fp4q_mxfp4_gemm.restype = i32
+        L.fp4q_encode.restype = i32
+        L.fp4q_encode.argtypes = [P, i64, i32, P, P]
         L.fp4q_mxfp4_gemm.argtypes = [P, P, P, P, i64, i64, i64, P, i64, P, P]
         L.fp4q_quantize.restype = i32
         L.fp4q_quantize.argtypes = [P, i32, i64, i64, i64, i32, i32, P, P, P, P, P, u32, P]
@@ -282,6 +284,17 @@ def mxfp4_gemm(a, b, out=None, workspace=None, stream=None):
                                _stream_ptr(stream))
     _check(rc, "fp4q_mxfp4_gemm")
     return d
+
+
+def encode(x, kind: str, out=None, stream=None):
+    """The hardware element codec on a CUDA fp32 tensor: kind "e2m1" -> 4-bit E2M1 codes (sign
+    in bit 3), "e4m3" -> E4M3FN bytes; both round to nearest even and saturate."""
+    torch = _torch()
+    x = x.contiguous().view(-1)
+    out = out if out is not None else torch.empty(x.numel(), dtype=torch.uint8, device=x.device)
+    rc = lib().fp4q_encode(_ptr(x), x.numel(), {"e2m1": 0, "e4m3": 1}[kind], _ptr(out), _stream_ptr(stream))
+    _check(rc, "fp4q_encode")
+    return out
 
 
 def read_device_status(workspace, stream=None) -> int:

@@ -957,6 +957,39 @@ __global__ void __launch_bounds__(kThreads) dequant_mx_kernel(const uint8_t* __r
 }
 
 // ------------------------------------------------------------------------------------------
+// Element codec: the hardware conversions every quantize path uses, applied element by element
+// (KIND 0: E2M1 round to nearest even, saturating, the 4-bit code with the sign in bit 3;
+// KIND 1: E4M3FN round to nearest even, saturating, the whole byte).  Four elements per thread
+// and step, one 4-byte store.
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t e4m3_byte(float v) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(v));
+    return r & 0xFFu;
+}
+
+template <int KIND>
+__global__ void __launch_bounds__(kThreads) encode_kernel(const float* __restrict__ x, int64_t n,
+                                                          uint8_t* __restrict__ out) {
+    const int64_t step = (int64_t)gridDim.x * blockDim.x;
+    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t n4 = n / 4;
+    for (int64_t i = tid; i < n4; i += step) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(x) + i);
+        uint32_t w;
+        if (KIND == 0) {
+            const uint32_t c01 = e2m1x2(v.x, v.y), c23 = e2m1x2(v.z, v.w);   // low nibble = first element
+            w = (c01 & 0xFu) | ((c01 >> 4) << 8) | ((c23 & 0xFu) << 16) | ((c23 >> 4) << 24);
+        } else {
+            w = e4m3_byte(v.x) | (e4m3_byte(v.y) << 8) | (e4m3_byte(v.z) << 16) | (e4m3_byte(v.w) << 24);
+        }
+        reinterpret_cast<uint32_t*>(out)[i] = w;
+    }
+    for (int64_t i = 4 * n4 + tid; i < n; i += step)
+        out[i] = (uint8_t)(KIND == 0 ? (e2m1x2(x[i], 0.0f) & 0xFu) : e4m3_byte(x[i]));
+}
+
+// ------------------------------------------------------------------------------------------
 // Host side
 // ------------------------------------------------------------------------------------------
 thread_local int g_launches = 0;
@@ -1345,6 +1378,22 @@ int fp4q_quantize_host_async(const void* x_host, int dtype, int64_t rows, int64_
         return FP4Q_ERR_CUDA;
     g_launches = n;
     return FP4Q_OK;
+}
+
+int fp4q_encode(const float* x, int64_t n, int kind, uint8_t* out, void* stream) {
+    g_launches = 0;
+    if (kind != FP4Q_CODEC_E2M1 && kind != FP4Q_CODEC_E4M3) return FP4Q_ERR_INVALID_ARG;
+    if (n < 0 || n > ((int64_t)1 << 40)) return FP4Q_ERR_SHAPE;
+    if (n == 0) return FP4Q_OK;
+    if (!x || !out) return FP4Q_ERR_INVALID_ARG;
+    if (!aligned16(x) || (reinterpret_cast<uintptr_t>(out) & 3u)) return FP4Q_ERR_ALIGNMENT;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t items = n / 4 > 0 ? n / 4 : 1;
+    if (kind == FP4Q_CODEC_E2M1)
+        encode_kernel<0><<<grid_for(encode_kernel<0>, items, 8), kThreads, 0, st>>>(x, n, out);
+    else
+        encode_kernel<1><<<grid_for(encode_kernel<1>, items, 8), kThreads, 0, st>>>(x, n, out);
+    return launched(1);
 }
 
 int fp4q_read_device_status(const void* workspace, uint32_t* status, void* stream) {

@@ -270,6 +270,21 @@ int fp4q_quantize_noalloc(const void* x, int dtype, int64_t rows, int64_t cols, 
                           uint8_t* codes, uint8_t* scales, float* global_scale,
                           uint32_t* device_status, uint32_t flags, void* stream);
 
+/*
+ * Element codec: the hardware conversions every quantize path uses, applied to n fp32 values.
+ *   kind FP4Q_CODEC_E2M1: out[i] = E2M1 code of x[i], round to nearest with ties to the even
+ *     code, saturating at +-6, sign kept (-0 -> 0x8): the low nibble holds sign << 3 | index of
+ *     the magnitude in {0, .5, 1, 1.5, 2, 3, 4, 6} (ScaleSweep, gist.science/ko/paper/2606.07618,
+ *     Contributions: round-to-nearest FP4 codes).
+ *   kind FP4Q_CODEC_E4M3: out[i] = E4M3FN byte of x[i], round to nearest even, saturating at
+ *     +-448 (the 126 positive finite values the ScaleSweep page counts, Methodology).
+ * x: device fp32 [n], 16-byte aligned; out: device uint8 [n], 4-byte aligned.  One launch.
+ * Errors: FP4Q_ERR_INVALID_ARG (unknown kind, NULL), FP4Q_ERR_SHAPE (n < 0 or n > 2^40),
+ * FP4Q_ERR_ALIGNMENT.  NaN inputs give whatever the hardware conversion gives.
+ */
+enum { FP4Q_CODEC_E2M1 = 0, FP4Q_CODEC_E4M3 = 1 };
+int fp4q_encode(const float* x, int64_t n, int kind, uint8_t* out, void* stream);
+
 /* Copy the device status word of `workspace` to *status (blocks until `stream` is done). */
 int fp4q_read_device_status(const void* workspace, uint32_t* status, void* stream);
 

@@ -44,6 +44,8 @@ def lib():
         L.fp4q_o_e2m1_value.argtypes = [C.c_int]
         L.fp4q_o_e2m1_encode.restype = C.c_int
         L.fp4q_o_e2m1_encode.argtypes = [C.c_float]
+        L.fp4q_o_encode.restype = C.c_int
+        L.fp4q_o_encode.argtypes = [P, i64, C.c_int, P]
         L.fp4q_o_global_scale.restype = C.c_float
         L.fp4q_o_global_scale.argtypes = [C.c_float]
         L.fp4q_o_tensor_scale.restype = C.c_int
@@ -256,6 +258,18 @@ def nvfp4_gemm(a_codes, a_scales, Sa, b_codes, b_scales, Sb):
         sc = e[np.asarray(scales, np.uint8) & 0x7F]
         return q * np.repeat(sc, 16, axis=1)
     return float(Sa) * float(Sb) * (values(a_codes, a_scales) @ values(b_codes, b_scales).T)
+
+
+def encode(x, kind: str) -> np.ndarray:
+    """Element codec over an fp32 array: kind "e2m1" gives the 4-bit E2M1 code of each value
+    (sign << 3 | magnitude index), "e4m3" the E4M3FN byte (sign in bit 7); both round to
+    nearest with ties to even and saturate."""
+    x = np.ascontiguousarray(x, np.float32).ravel()
+    out = np.empty(x.size, np.uint8)
+    st = lib().fp4q_o_encode(_p(x), x.size, {"e2m1": 0, "e4m3": 1}[kind], _p(out))
+    if st != 0:
+        raise ValueError(kind)
+    return out
 
 
 def mxfp4_gemm(a_codes, a_scales, b_codes, b_scales):

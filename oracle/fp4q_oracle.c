@@ -124,6 +124,40 @@ int fp4q_o_e2m1_encode(float y)
     return s | k;
 }
 
+/* Batch codec over n values (the reference the hardware conversions are checked against).
+ * kind 0: fp4q_o_e2m1_encode of each value.  kind 1: E4M3FN byte, sign in bit 7, magnitude
+ * rounded to the nearest of the 127 values 0 .. 448 with ties to the even pattern and
+ * saturation at 448 (infinities included); NaN gives 0x7F.  The magnitude's pattern is found by
+ * bisection over the increasing value table (the values of fp4q_o_e4m3_value), then the nearer
+ * of the two bracketing patterns is taken; this equals fp4q_o_e4m3_encode, which scans all
+ * patterns (a pin checks the two against each other). */
+int fp4q_o_encode(const float* x, int64_t n, int kind, uint8_t* out)
+{
+    if (kind == 0) {
+        for (int64_t i = 0; i < n; ++i) out[i] = (uint8_t)fp4q_o_e2m1_encode(x[i]);
+        return ST_OK;
+    }
+    if (kind != 1) return -1;
+    double tab[127];
+    for (int p = 0; p <= 0x7E; ++p) tab[p] = fp4q_o_e4m3_value(p);
+    for (int64_t i = 0; i < n; ++i) {
+        const float v = x[i];
+        const int s = signbit(v) ? 0x80 : 0;
+        if (isnan(v)) { out[i] = (uint8_t)(s | 0x7F); continue; }
+        const double a = fabs((double)v);
+        if (a >= 448.0) { out[i] = (uint8_t)(s | 0x7E); continue; }
+        int lo = 0, hi = 0x7E;          /* tab[lo] <= a < tab[hi] */
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) / 2;
+            if (tab[mid] <= a) lo = mid; else hi = mid;
+        }
+        const double dl = a - tab[lo], dh = tab[hi] - a;
+        const int p = dl < dh ? lo : (dh < dl ? hi : ((lo & 1) == 0 ? lo : hi));
+        out[i] = (uint8_t)(s | p);
+    }
+    return ST_OK;
+}
+
 /* ------------------------------------------------------------------------------------
  * Global scale  [SS] S = max|x|/(256*6)
  * ---------------------------------------------------------------------------------- */

@@ -466,6 +466,24 @@ def test_nvfp4_gemm_oracle():
     assert np.all(np.abs(d - da @ db.T) <= 2 ** -22 * mag)
 
 
+def test_batch_codec_matches_the_scalar_encoders():
+    # the batch codec (E4M3 by bisection) against the scalar encoders (E4M3 by a scan over all
+    # patterns): every E4M3 value and midpoint and their fp32 neighbours, both signs, and random
+    # values over the whole range, subnormals, saturation and infinities included
+    vals = np.array([O.lib().fp4q_o_e4m3_value(p) for p in range(127)])
+    pts = np.concatenate([vals, (vals[:-1] + vals[1:]) / 2, [448.0, 464.0, 480.0, 1e30, np.inf]]).astype(np.float32)
+    near = np.concatenate([np.nextafter(pts, np.float32(np.inf)), np.nextafter(pts, np.float32(0)), pts])
+    rng = np.random.default_rng(9)
+    rnd = (rng.random(200000) * 2.0 ** rng.integers(-20, 12, 200000)).astype(np.float32)
+    x = np.concatenate([near, rnd]).astype(np.float32)
+    x = np.concatenate([x, -x])
+    got = O.encode(x, "e4m3")
+    ref = np.array([(0x80 if np.signbit(v) else 0) | O.lib().fp4q_o_e4m3_encode(abs(float(v))) for v in x], np.uint8)
+    assert np.array_equal(got, ref)
+    got = O.encode(x, "e2m1")
+    assert np.array_equal(got, np.array([O.lib().fp4q_o_e2m1_encode(float(v)) for v in x], np.uint8))
+
+
 def test_mxfp4_gemm_oracle():
     # against a triple loop over exact rationals (E8M0 byte b is the power of two 2^(b - 127)),
     # and against the float64 product of the dequantized operands, plain and rotated
