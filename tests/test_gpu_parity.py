@@ -251,6 +251,26 @@ def test_edge_tensors(name, method):
     assert_same_codes(gc, gsc, r["codes"], r["scales"])
 
 
+def test_exact_roundtrip_every_representable_value():
+    # with S = 1, a block whose maximum is 6 e(p) and whose other elements are the signed grid
+    # values times e(p) selects pattern p under AbsMax and the sweep, and dequantizes bit-exactly:
+    # every E2M1 x E4M3 value for the patterns AbsMax reaches (1 .. 0x78)
+    grid = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0]
+    blocks = []
+    for p in range(1, 0x79):
+        e = O.lib().fp4q_o_e4m3_value(p)
+        vals = [6 * e] + [s * g * e for g in grid for s in (1, -1)] + [0.0]
+        blocks.append(np.array(vals[:16], np.float32))
+    x = np.concatenate(blocks).reshape(1, -1)
+    for obj in ("absmax", "sweep_mse"):
+        gc, gsc, gS, st, out = run_gpu(torch.from_numpy(x).cuda(), "nvfp4", obj)
+        assert st == 0 and gS == 1.0
+        if obj == "absmax":
+            assert list(gsc[0]) == list(range(1, 0x79))
+        xg = fq.dequantize(out[0], out[1], out[2], "nvfp4").cpu().numpy()
+        assert np.array_equal(xg.view(np.uint32), x.view(np.uint32))
+
+
 def test_bad_data_sets_status_and_zero_fills():
     x = np.random.default_rng(1).normal(size=(4, 64)).astype(np.float32)
     x[2, 7] = np.nan
