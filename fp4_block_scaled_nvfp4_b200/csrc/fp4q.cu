@@ -800,8 +800,12 @@ __global__ void __launch_bounds__(kThreads) mxfp4_kernel(const void* __restrict_
     for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < total; blk += step) {
         const int64_t r = blk / nb, b = blk - r * nb;
         float v[32];
+        // magnitude bits compared as unsigned integers (NaN > Inf > every finite value): one
+        // maximum gives both the finiteness check and, unrotated, the block maximum
+        uint32_t mb;
         if (IN == FP4Q_IN_BF16) {
             const uint4* p = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(xv) + r * ld + b * 32);
+            uint32_t m2 = 0;   // two 16-bit maxima
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const uint4 w = __ldg(p + q);
@@ -810,44 +814,46 @@ __global__ void __launch_bounds__(kThreads) mxfp4_kernel(const void* __restrict_
                 for (int t = 0; t < 4; ++t) {
                     v[q * 8 + 2 * t] = __uint_as_float(ww[t] << 16);
                     v[q * 8 + 2 * t + 1] = __uint_as_float(ww[t] & 0xFFFF0000u);
+                    m2 = __vmaxu2(m2, ww[t] & 0x7FFF7FFFu);
                 }
             }
+            mb = max(m2 & 0xFFFFu, m2 >> 16) << 16;
         } else {
             const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(xv) + r * ld + b * 32);
+            mb = 0;
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 const float4 w = __ldg(p + q);
                 v[4 * q] = w.x; v[4 * q + 1] = w.y; v[4 * q + 2] = w.z; v[4 * q + 3] = w.w;
             }
-        }
-        bool bad = false;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) bad |= !isfinite(v[i]);
+            for (int i = 0; i < 32; ++i) mb = max(mb, __float_as_uint(v[i]) & 0x7FFFFFFFu);
+        }
         uint4* cdst = reinterpret_cast<uint4*>(codes + r * (cols / 2) + b * 16);
         uint8_t* sdst = scales + (tiled ? tiled_scale_offset<int64_t>(r, b, nb) : blk);
-        if (bad) {
+        if (mb >= 0x7F800000u) {   // a NaN or an infinity in the block
             flag = FP4Q_DEVSTAT_NONFINITE;
             *cdst = make_uint4(0u, 0u, 0u, 0u);
             *sdst = 0xFF;
             continue;
         }
-        if (HAD) fwht32(v);
-        float ab = 0.0f;
+        float ab = __uint_as_float(mb);
+        if (HAD) {
+            // the rotated maximum ignores a NaN that an overflowing butterfly can produce
+            fwht32(v);
+            ab = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) ab = fmaxf(ab, fabsf(v[i]));
-        int e;
-        if (SWEEP) {
-            u64 vp[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) vp[j] = pk(v[2 * j], v[2 * j + 1]);
-            e = mx_sweep_exponent(vp, mx_exponent(ab, false));
-        } else {
-            e = mx_exponent(ab, ocp != 0);
+            for (int i = 0; i < 32; ++i) ab = fmaxf(ab, fabsf(v[i]));
         }
+        u64 vp[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) vp[j] = pk(v[2 * j], v[2 * j + 1]);
+        const int e = SWEEP ? mx_sweep_exponent(vp, mx_exponent(ab, false)) : mx_exponent(ab, ocp != 0);
         const float m = pow2i(-e);
+        const u64 m2 = pk(m, m);
         uint32_t c[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) c[j] = e2m1x2(__fmul_rn(v[2 * j], m), __fmul_rn(v[2 * j + 1], m));
+        for (int j = 0; j < 16; ++j) c[j] = e2m1x2(mul2(vp[j], m2));   // x 2^-e is exact
         *cdst = make_uint4(c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24),
                            c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24),
                            c[8] | (c[9] << 8) | (c[10] << 16) | (c[11] << 24),
