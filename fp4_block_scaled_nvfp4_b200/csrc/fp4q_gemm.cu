@@ -1,22 +1,23 @@
-// fp4q_gemm.cu -- block-scaled NVFP4 GEMM on the sm_100a tensor cores (tcgen05), the consumer
-// of the quantizer's outputs: D[m][n] = S_a S_b sum_k A[m][k] B[n][k], with A and B NVFP4
-// tensors stored exactly as fp4q_quantize writes them (codes [rows][K/2], element 2j in the
-// low nibble; E4M3 scales in the 128x4-tiled layout of FP4Q_F_SCALE_TILED; one fp32 tensor
-// scale each).  Both operands have K contiguous.
+// fp4q_gemm.cu -- block-scaled FP4 GEMMs on the sm_100a tensor cores (tcgen05), the consumer
+// of the quantizer's outputs: D[m][n] = S_a S_b sum_k A[m][k] B[n][k] for NVFP4 operands, and
+// D[m][n] = sum_k A[m][k] B[n][k] for MXFP4 operands, with A and B stored exactly as
+// fp4q_quantize writes them (codes [rows][K/2], element 2j in the low nibble; scales in the
+// 128x4-tiled layout of FP4Q_F_SCALE_TILED; NVFP4: one fp32 tensor scale each).  Both operands
+// have K contiguous.
 //
-// Each output tile of 128 x 128 is built from K stages of 256 elements: per stage the A and B
-// tiles (128 rows x 128 bytes each) sit in shared memory in the 128-byte-swizzled K-major
-// layout the MMA descriptor describes, and the four 512-byte scale-factor atoms of each operand
-// as they are; one thread moves the atoms into tensor memory (tcgen05.cp 32x128b, broadcast to
-// the four lane quarters) and issues four block-scaled MMAs of K = 64 (tcgen05.mma
-// kind::mxf4nvf4, 16-element scale blocks) accumulating fp32 in tensor memory; the epilogue
-// reads the accumulator back with tcgen05.ld (each warp its lane quarter), multiplies by
-// RN(S_a S_b) and stores D.
-//   fp4_gemm_kernel<MX> (the one launched; MX selects MXFP4 operands): one CTA per SM over all tiles, a
-//     five-stage ring filled by tensor copies, producer / MMA / epilogue warps, two
-//     accumulators so the epilogue of a tile overlaps the next tile's MMAs.
-//   nvfp4_gemm_kernel (build flag FP4Q_GEMM_SIMPLE): the same arithmetic in one stage with
-//     plain loads, kept as the reference form of the sequence.
+// Per K stage of 256 elements the A and B tiles (128-byte rows) sit in shared memory in the
+// 128-byte-swizzled K-major layout the MMA descriptors describe, and the operands' 512-byte
+// scale-factor atoms as they are; one thread moves the atoms into tensor memory (tcgen05.cp
+// 32x128b, broadcast to the four lane quarters) and issues four block-scaled MMAs of K = 64
+// (tcgen05.mma kind::mxf4nvf4, 16-element E4M3 or 32-element E8M0 scale blocks) accumulating
+// fp32 in tensor memory; the epilogue reads the accumulator back with tcgen05.ld (each warp
+// its lane quarter), multiplies by RN(S_a S_b) (NVFP4) and stores D.
+//   fp4_gemm_kernel<MX> (the one launched; MX selects MXFP4 operands): one CTA per SM over
+//     128 x 256 output tiles, a four-stage ring filled by tensor copies, producer / MMA /
+//     epilogue warps, two overlapping accumulators so the epilogue of a tile overlaps the next
+//     tile's MMAs.
+//   nvfp4_gemm_kernel (build flag FP4Q_GEMM_SIMPLE): 128 x 128 tiles, the same arithmetic in
+//     one stage with plain loads, kept as the reference form of the sequence.
 // Every wait is bounded; one that runs out sets FP4Q_DEVSTAT_TIMEOUT in the status word, stops
 // the CTA's loops, and the CTA still frees its tensor memory.
 #include <cstdint>
