@@ -546,6 +546,10 @@ def run_gemm(args, rank, world):
     flops = 2.0 * M * N * K
     steps = args.steps
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         with torch.cuda.stream(stream):
             start.record()
@@ -553,9 +557,11 @@ def run_gemm(args, rank, world):
                 gemm(qa, qb, out=d, workspace=ws)
             end.record()
         end.synchronize()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
     ms = start.elapsed_time(end) / steps
     if world > 1:
-        import torch.distributed as dist
         t = torch.tensor([ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
@@ -578,6 +584,10 @@ def run_gemm(args, rank, world):
         e1.record()
     e1.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
     if rank != 0:
         return
     peak, peak_src = fp4_peak_tflops()
