@@ -20,6 +20,7 @@
 //     one stage with plain loads, kept as the reference form of the sequence.
 // Every wait is bounded; one that runs out sets FP4Q_DEVSTAT_TIMEOUT in the status word, stops
 // the CTA's loops, and the CTA still frees its tensor memory.
+#include <atomic>
 #include <cstdint>
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -467,6 +468,20 @@ __global__ void __launch_bounds__(kPThreads, 1)
 namespace fp4q {
 namespace gemm {
 
+// The kernel's dynamic shared-memory limit, raised once per kernel and device (the attribute
+// belongs to the current device's context); one bit per device ordinal below 64.
+template <auto kernel>
+bool smem_attribute_set(int bytes) {
+    static std::atomic<uint64_t> done{0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return false;
+    const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
+    if (bit && (done.load(std::memory_order_relaxed) & bit)) return true;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+    done.fetch_or(bit, std::memory_order_relaxed);
+    return true;
+}
+
 // Shared host path of the two entry points: argument checks, tensor maps, launch.
 template <bool MX>
 int launch(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global_scale, const uint8_t* b_codes,
@@ -487,13 +502,7 @@ int launch(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_globa
     if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return FP4Q_ERR_CUDA;
 #if FP4Q_GEMM_SIMPLE
     if (MX) return FP4Q_ERR_UNSUPPORTED;
-    static bool attr_set = false;
-    if (!attr_set) {
-        if (cudaFuncSetAttribute(nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc) !=
-            cudaSuccess)
-            return FP4Q_ERR_CUDA;
-        attr_set = true;
-    }
+    if (!smem_attribute_set<nvfp4_gemm_kernel>(kSmemAlloc)) return FP4Q_ERR_CUDA;
     const dim3 grid((unsigned)(N / kTN), (unsigned)(M / kTM));
     nvfp4_gemm_kernel<<<grid, kThreads, kSmemAlloc, st>>>(a_codes, a_scales, a_global_scale, b_codes, b_scales,
                                                           b_global_scale, (int)K, d, ldd, status);
@@ -509,13 +518,7 @@ int launch(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_globa
             return FP4Q_ERR_CUDA;
         encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
-    static bool attr_set = false;
-    if (!attr_set) {
-        if (cudaFuncSetAttribute(fp4_gemm_kernel<MX>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPersistSmem) !=
-            cudaSuccess)
-            return FP4Q_ERR_CUDA;
-        attr_set = true;
-    }
+    if (!smem_attribute_set<fp4_gemm_kernel<MX>>(kPersistSmem)) return FP4Q_ERR_CUDA;
     CUtensorMap ta, tb;
     auto make = [&](CUtensorMap* m, const uint8_t* base, int64_t rows, int box_rows) {
         const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
