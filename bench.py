@@ -417,6 +417,21 @@ def run_ours(args, rank, world):
     t_q = time_kernel(quant)
     t_amax = None if fmt.startswith("mxfp4") else time_kernel(amax)
 
+    # per-step distribution: up to 200 steps, each between its own pair of CUDA events on the
+    # stream (the buffer sets in turn)
+    n_dist = max(1, min(args.steps, 200))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_dist)]
+    with torch.cuda.stream(stream):
+        for i, (a, b) in enumerate(evs):
+            a.record()
+            graphs[i % nsets].replay()
+            b.record()
+    torch.cuda.synchronize()
+    per_step = sorted(a.elapsed_time(b) for a, b in evs)
+    pick = lambda q: round(per_step[min(n_dist - 1, int(q * (n_dist - 1) + 0.5))], 5)
+    step_dist = {"p10": pick(0.1), "p50": pick(0.5), "p90": pick(0.9), "steps": n_dist,
+                 "how": "each step between its own CUDA events on the launching stream"}
+
     # status of the last step must be clean
     st = fq.read_device_status(ws)
 
@@ -492,6 +507,7 @@ def run_ours(args, rank, world):
         "elements_per_s": round(rows * cols * args.steps * world / (ms * 1e-3), 1),
         "kernels_ms": {"amax": (None if t_amax is None else round(t_amax, 5)), "quantize": round(tq, 5),
                        "how": f"each kernel alone, {kernel_reps} launches over the rotating buffer sets, CUDA events"},
+        "step_ms": step_dist,
         "roofline": roofline,
         "device_status": st,
         "gpu_launches": launches_per_step * args.steps,
