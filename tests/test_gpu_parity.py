@@ -331,8 +331,5 @@ def test_full_size_sampled(cfg, fmt, obj):
             r = O.if4_quantize(oracle_x(w, rows), S=S, sweep="sweep" if obj == "if4_sweep" else "absmax")
         else:
             r = O.nvfp4_quantize(oracle_x(w, rows), obj, importance=imp, S=S)
-            nt = (r["err2"] - r["err"]) / np.maximum(r["err"], np.finfo(np.float32).tiny)
-            near = int(np.sum((r["nvalid"] >= 2) & (nt < 1e-6)))
-            assert near <= max(1, int(1e-5 * r["err"].size)) or True   # reported by the bench
     assert st == 0
     assert_same_codes(gc[rows], gsc[rows], r["codes"], r["scales"])
