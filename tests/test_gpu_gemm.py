@@ -110,3 +110,49 @@ def test_mxfp4_gemm_matches_the_oracle_product(M, N, K, had):
     # the rotations cancel in the product: either way it approximates the unrotated product
     exact = xa.astype(np.float64) @ xb.astype(np.float64).T
     assert np.linalg.norm(got - exact) <= 0.25 * np.linalg.norm(exact)
+
+
+@pytest.mark.parametrize("mx", [False, True])
+def test_full_size_gemm_sampled(mx):
+    # the bench's GEMM at full size (8192 x 14336 x 4096: activation-workload rows times
+    # weight-workload rows, quantized by the library), checked on 32 x 96 sampled outputs
+    # against the oracle's product of the same rows and columns, quantized by the oracle
+    M, N, K = 8192, 14336, 4096
+    wa, wb = synth.make("cfg3", rows=M, cols=K), synth.make("cfg2", rows=N, cols=K)
+    xa = torch.from_numpy(wa["x"].view(np.int16)).view(torch.bfloat16).cuda()
+    xb = torch.from_numpy(wb["x"].view(np.int16)).view(torch.bfloat16).cuda()
+    ws = fq.new_workspace()
+    if mx:
+        qa, qb = fq.hadamard_quantize(xa, tiled_scales=True)[:2], fq.hadamard_quantize(xb, tiled_scales=True)[:2]
+        d = fq.mxfp4_gemm(qa, qb, workspace=ws)
+    else:
+        qa = fq.quantize(xa, "nvfp4", "sweep_mse", tiled_scales=True)
+        qb = fq.quantize(xb, "nvfp4", "sweep_mse", tiled_scales=True)
+        d = fq.nvfp4_gemm(qa, qb, workspace=ws)
+    torch.cuda.synchronize()
+    assert fq.read_device_status(ws) == fq.DEVSTAT_OK
+    rng = np.random.default_rng(7)
+    rows = np.sort(rng.choice(M, 32, replace=False))
+    cols = np.sort(rng.choice(N, 96, replace=False))
+    xa_r, xb_c = O.widen_bf16(wa["x"][rows]), O.widen_bf16(wb["x"][cols])
+    if mx:
+        ra, rb = O.mxfp4_quantize(xa_r, hadamard=True), O.mxfp4_quantize(xb_c, hadamard=True)
+        ref = O.mxfp4_gemm(ra["codes"], ra["scales"], rb["codes"], rb["scales"])
+        da = O.dequantize(ra["codes"], ra["scales"], 0.0, "mxfp4").astype(np.float64)
+        db = O.dequantize(rb["codes"], rb["scales"], 0.0, "mxfp4").astype(np.float64)
+    else:
+        Sa, sta = O.tensor_scale(O.widen_bf16(wa["x"]))
+        Sb, stb = O.tensor_scale(O.widen_bf16(wb["x"]))
+        assert sta == stb == 0
+        assert np.float32(qa[2].cpu().item()).view(np.uint32) == np.float32(Sa).view(np.uint32)
+        assert np.float32(qb[2].cpu().item()).view(np.uint32) == np.float32(Sb).view(np.uint32)
+        ra, rb = O.nvfp4_quantize(xa_r, "sweep_mse", S=Sa), O.nvfp4_quantize(xb_c, "sweep_mse", S=Sb)
+        ref = O.nvfp4_gemm(ra["codes"], ra["scales"], Sa, rb["codes"], rb["scales"], Sb)
+        da = O.dequantize(ra["codes"], ra["scales"], Sa, "nvfp4").astype(np.float64)
+        db = O.dequantize(rb["codes"], rb["scales"], Sb, "nvfp4").astype(np.float64)
+    # the operands agree bit for bit on the sampled rows
+    assert np.array_equal(qa[0][torch.from_numpy(rows).cuda()].cpu().numpy(), ra["codes"])
+    assert np.array_equal(qb[0][torch.from_numpy(cols).cuda()].cpu().numpy(), rb["codes"])
+    got = d[torch.from_numpy(rows).cuda()][:, torch.from_numpy(cols).cuda()].cpu().numpy().astype(np.float64)
+    mag = np.abs(da) @ np.abs(db).T
+    assert np.all(np.abs(got - ref) <= 2e-5 * mag + 1e-30), float(np.max(np.abs(got - ref) / (mag + 1e-30)))
