@@ -1,5 +1,6 @@
 /*
- * fp4q.h -- C ABI of libfp4q: block-scaled FP4 quantization on NVIDIA B200 (sm_100a).
+ * fp4q.h -- C ABI of libfp4q: block-scaled FP4 quantization on NVIDIA B200 (sm_100a), and the
+ * block-scaled NVFP4 / MXFP4 GEMMs (tcgen05 tensor cores) that consume the quantized operands.
  *
  * Formats and methods (each entry point cites the passage that defines what it computes):
  *   NVFP4  16-element blocks of E2M1 codes {0,.5,1,1.5,2,3,4,6} with one E4M3 scale per
@@ -83,8 +84,8 @@ typedef enum {
     FP4Q_ERR_CUDA = 5           /* a CUDA launch or runtime call failed                      */
 } fp4q_status;
 
-/* Device status bits.  TIMEOUT: fp4q_nvfp4_gemm gave up a bounded wait for its tensor-core
- * work (its output is then incomplete). */
+/* Device status bits.  TIMEOUT: fp4q_nvfp4_gemm / fp4q_mxfp4_gemm gave up a bounded wait for
+ * its tensor-core work (its output is then incomplete). */
 enum { FP4Q_DEVSTAT_OK = 0, FP4Q_DEVSTAT_NONFINITE = 1, FP4Q_DEVSTAT_RANGE = 2, FP4Q_DEVSTAT_TIMEOUT = 4 };
 enum { FP4Q_IN_F32 = 0, FP4Q_IN_BF16 = 1 };
 enum { FP4Q_NVFP4 = 0, FP4Q_IF4 = 1, FP4Q_MXFP4 = 2 };
@@ -121,7 +122,7 @@ size_t fp4q_workspace_bytes(void);
  * padding keeps whatever the caller put there (zero it if the consumer reads it).  The pages
  * give no scale layout; this one is the public layout of NVIDIA's block-scaled GEMMs
  * (cuBLASLt's "32x4x4" scale-factor tiles), kept byte for byte so that a GEMM can read the
- * scales as written.  IF4 has no tiled form (its indicator bit is not a consumer format).
+ * scales as written (fp4q_nvfp4_gemm and fp4q_mxfp4_gemm do).  IF4 has no tiled form (its indicator bit is not a consumer format).
  * Returns -1 for an unknown format or a bad shape.
  */
 int64_t fp4q_scale_bytes(int64_t rows, int64_t cols, int fmt, uint32_t flags);
