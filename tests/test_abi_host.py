@@ -66,6 +66,19 @@ def test_gemm_rejects_before_launch():
     assert mx(0, 128, 256, a=None, d=None, ws=None) == fq.OK and L.fp4q_last_launch_count() == 0
 
 
+def test_encode_rejects_before_launch():
+    L = fq.lib()
+    F = FAKE
+    assert L.fp4q_encode(F, 8, 2, F, None) == fq.ERR_INVALID_ARG      # unknown kind
+    assert L.fp4q_encode(F, -1, 0, F, None) == fq.ERR_SHAPE
+    assert L.fp4q_encode(F, 1 << 41, 1, F, None) == fq.ERR_SHAPE
+    assert L.fp4q_encode(None, 8, 0, F, None) == fq.ERR_INVALID_ARG
+    assert L.fp4q_encode(F, 8, 0, None, None) == fq.ERR_INVALID_ARG
+    assert L.fp4q_encode(F + 4, 8, 0, F, None) == fq.ERR_ALIGNMENT    # x must be 16-byte aligned
+    assert L.fp4q_encode(F, 8, 1, F + 2, None) == fq.ERR_ALIGNMENT    # out must be 4-byte aligned
+    assert L.fp4q_encode(None, 0, 0, None, None) == fq.OK and L.fp4q_last_launch_count() == 0
+
+
 def test_status_strings_and_workspace():
     assert fq.status_string(0) == "ok"
     for rc in range(1, 6):
