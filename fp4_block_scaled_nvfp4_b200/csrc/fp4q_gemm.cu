@@ -309,10 +309,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const uint32_t tmem = *tmem_slot;
+    uint32_t issued = 0;   // stages the producer has armed (thread 0)
 
     if (tid == 0) {
         // producer
-        uint32_t g = 0;
+        uint32_t& g = issued;
         for (int t = blockIdx.x; t < tiles && !s_fail; t += gridDim.x) {
             const int mt = t / n_tiles, nt = t - mt * n_tiles;
             const bool wide = wide_tile(nt);
@@ -457,7 +458,16 @@ __global__ void __launch_bounds__(kPThreads, 1)
     __syncwarp();
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
-    if (s_fail && tid == 0) atomicOr(status, (uint32_t)FP4Q_DEVSTAT_TIMEOUT);
+    if (s_fail && tid == 0) {
+        atomicOr(status, (uint32_t)FP4Q_DEVSTAT_TIMEOUT);
+        // a wait gave up: before the CTA leaves, let the copies it armed land in its shared
+        // memory (the last stage armed in each ring slot; each wait is again bounded)
+        for (uint32_t i = 0; i < (uint32_t)kPStages && i < issued; ++i) {
+            const uint32_t gi = issued - 1 - i;
+            mbar_wait(smem_u32(full + gi % kPStages), (gi / kPStages) & 1u);
+        }
+    }
+    __syncwarp();
     if (warp == 0)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(kPTmemCols) : "memory");
 }
