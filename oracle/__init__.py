@@ -12,6 +12,13 @@ Each function follows the passage its C counterpart cites:
   Bridging the Gap ... Microscaling FP4 (gist.science/ko/paper/2509.23202) "Methodology":
       MXFP4 (32-element blocks, power-of-two scales), block-wise Hadamard.
   TORQ (gist.science/ko/paper/2605.19561) "Method", S-step: block max onto the largest code.
+The GEMM products (``nvfp4_gemm``, ``mxfp4_gemm``) are the plain definition of the product of
+two quantized operands, in float64 from the oracle's own code tables; ``encode`` is the
+oracle's element codec over arrays.
+
+Pins (tests/test_oracle_pins.py): exact rationals, brute-force argmins, closed forms and
+hand-worked blocks.  Parity unpinned against the pages for end-to-end reconstruction MSE
+values per configuration: the pages print no worked numbers.
 """
 from __future__ import annotations
 

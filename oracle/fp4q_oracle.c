@@ -1,7 +1,9 @@
 /*
  * fp4q_oracle.c -- plain, slow, single-threaded CPU oracle for block-scaled FP4
  * quantization (NVFP4 AbsMax / 4-over-6 / ScaleSweep MSE and WMSE, IF4, MXFP4 with an
- * optional block Hadamard, and dequantization).
+ * optional block Hadamard, and dequantization), and its element codec.  Parity unpinned
+ * against the pages for end-to-end MSE values (they print no worked numbers); every function
+ * is pinned by the tests to exact rationals, brute force, closed forms or hand-worked blocks.
  *
  * TEST INFRASTRUCTURE ONLY.  Only the test-suite, the smoke check and the benchmark's
  * CPU-baseline leg may load this library.  It shares no code with the CUDA path: it has
