@@ -316,6 +316,23 @@ def test_mx_exponent_closed_form():
     assert O.mx_exponent(0.0) == -127
 
 
+def test_e8m0_roundtrip_every_exponent():
+    # a block whose maximum is 6 * 2^e and whose other elements are signed E2M1 grid values
+    # times 2^e selects E8M0 byte e + 127 and dequantizes exactly, for every exponent whose
+    # block fits in binary32 (-127 .. 125; 2^-128 and below are exact fp32 subnormals)
+    blocks = []
+    exps = list(range(-127, 126))
+    for e in exps:
+        p = 2.0 ** e
+        vals = [6 * p] + [sg * float(g) * p for g in GRID for sg in (1, -1)] + [0.0] * 15
+        blocks.append(np.array(vals[:32], np.float32))
+    x = np.concatenate(blocks).reshape(1, -1)
+    r = O.mxfp4_quantize(x)
+    assert list(r["scales"][0]) == [e + 127 for e in exps]
+    xh = O.dequantize(r["codes"], r["scales"], 0.0, "mxfp4")
+    assert np.array_equal(xh.view(np.uint32), x.view(np.uint32))
+
+
 def _mx_blocks(seed, n):
     """Blocks of 32 from several distributions: Laplace with per-channel scales (the activation
     workload's shape), Gaussian, exact E2M1 grid values times a power of two, and blocks with one
