@@ -204,10 +204,12 @@ def _oracle_rows(args):
     return xs.shape[0]
 
 
-def cpu_baseline_all_cores(w, fmt, obj, budget_s=6.0):
+def cpu_baseline_all_cores(w, fmt, obj, budget_s=6.0, cpu_budget_s=30.0):
     """The same oracle on row shards over the host cores this process may run on (at most 128):
     one process per core (started with spawn), each quantizing a contiguous shard of rows (rows
-    are independent); whole passes over the tensor until about budget_s of wall time."""
+    are independent); whole passes over the tensor until about min(budget_s, cpu_budget_s /
+    cores) of wall time (at least one pass), so that the sample stays near cpu_budget_s of CPU
+    work."""
     import multiprocessing as mp
     from concurrent.futures import ProcessPoolExecutor
     import oracle as O
@@ -215,6 +217,7 @@ def cpu_baseline_all_cores(w, fmt, obj, budget_s=6.0):
     x = O.widen_bf16(w["x"]) if w["dtype"] == "bf16" else w["x"]
     rows, cols = x.shape
     n = max(1, min(128, len(os.sched_getaffinity(0))))
+    budget_s = min(budget_s, cpu_budget_s / n)
     step = -(-rows // n)
     shards = [(np.ascontiguousarray(x[a:a + step]), fmt, obj, w.get("importance")) for a in range(0, rows, step)]
     # a worker that dies raises BrokenProcessPool here instead of leaving the map waiting
