@@ -66,11 +66,17 @@ def lib():
         L.fp4q_o_hadamard32.restype = None
         L.fp4q_o_hadamard32.argtypes = [P]
         L.fp4q_o_nvfp4_quantize.restype = C.c_int
-        L.fp4q_o_nvfp4_quantize.argtypes = [P, i64, i64, i64, C.c_int, P, C.c_int, P, P, P, P, P, P, P]
+        L.fp4q_o_nvfp4_quantize.argtypes = [P, i64, i64, i64, C.c_int, P, C.c_int, P, P, P, P, P, P, P, P, P]
         L.fp4q_o_if4_quantize.restype = C.c_int
-        L.fp4q_o_if4_quantize.argtypes = [P, i64, i64, i64, C.c_int, C.c_int, P, P, P, P, P]
+        L.fp4q_o_if4_quantize.argtypes = [P, i64, i64, i64, C.c_int, C.c_int, P, P, P, P, P, P, P]
         L.fp4q_o_mxfp4_quantize.restype = C.c_int
-        L.fp4q_o_mxfp4_quantize.argtypes = [P, i64, i64, i64, C.c_int, C.c_int, C.c_int, P, P]
+        L.fp4q_o_mxfp4_quantize.argtypes = [P, i64, i64, i64, C.c_int, C.c_int, C.c_int, P, P, P, P]
+        L.fp4q_o_f32_to_bf16.restype = None
+        L.fp4q_o_f32_to_bf16.argtypes = [P, i64, P]
+        L.fp4q_o_undecided.restype = C.c_long
+        L.fp4q_o_undecided.argtypes = []
+        L.fp4q_o_inexact.restype = C.c_long
+        L.fp4q_o_inexact.argtypes = []
         L.fp4q_o_mx_block_errors.restype = C.c_int
         L.fp4q_o_mx_block_errors.argtypes = [P, i64, i64, i64, C.c_int, P, P]
         L.fp4q_o_dequantize.restype = C.c_int
@@ -147,9 +153,28 @@ def rotate16(x) -> np.ndarray:
 
 
 # --- quantizers --------------------------------------------------------------------
+class OracleUndecided(RuntimeError):
+    """Two candidates came within the rounding of an inexact (brute-force-only) evaluation."""
+
+
+def _decided():
+    n = lib().fp4q_o_undecided()
+    if n:
+        raise OracleUndecided(f"oracle: {n} comparisons too close to decide without exact sums")
+
+
+def inexact_count() -> int:
+    """Exact-error evaluations since the last call whose sums did not stay exact (the windows
+    never produce one; only the brute-force window checks may)."""
+    return int(lib().fp4q_o_inexact())
+
+
 def nvfp4_quantize(x, objective="sweep_mse", importance=None, S=None, hadamard16=False):
     """NVFP4 quantization of a float32 [rows, cols] array; returns a dict with packed codes
-    [rows, cols/2], scale bytes [rows, cols/16], S, status and per-block diagnostics.
+    [rows, cols/2], scale bytes [rows, cols/16], S, status and per-block diagnostics:
+    p (chosen pattern), err (the exact block error E as float64; WMSE: the binary32 weighted
+    accumulator), gap (runner-up's (E2 - E1) / max(E1, FLT_MIN), +inf with one candidate),
+    tie (runner-up exactly equal), p2 (runner-up's pattern), nvalid (candidates).
     hadamard16: quantize the blockwise-rotated tensor (S taken over the rotated values)."""
     x = rotate16(x) if hadamard16 else _f32(x)
     rows, cols = x.shape
@@ -158,16 +183,19 @@ def nvfp4_quantize(x, objective="sweep_mse", importance=None, S=None, hadamard16
     scales = np.zeros((rows, nb), np.uint8)
     Sarr = np.array([0.0 if S is None else S], np.float32)
     bp = np.zeros((rows, nb), np.int32)
-    be = np.zeros((rows, nb), np.float32)
-    be2 = np.zeros((rows, nb), np.float32)
+    be = np.zeros((rows, nb), np.float64)
+    bg = np.zeros((rows, nb), np.float64)
+    bt = np.zeros((rows, nb), np.int32)
+    b2 = np.zeros((rows, nb), np.int32)
     bn = np.zeros((rows, nb), np.int32)
     w = None if importance is None else np.ascontiguousarray(importance, np.float32)
     st = lib().fp4q_o_nvfp4_quantize(_p(x), rows, cols, cols, OBJ[objective], _p(w), int(S is not None),
-                                     _p(Sarr), _p(codes), _p(scales), _p(bp), _p(be), _p(be2), _p(bn))
+                                     _p(Sarr), _p(codes), _p(scales), _p(bp), _p(be), _p(bg), _p(bt), _p(b2), _p(bn))
     if st < 0:
         raise ValueError("oracle: bad shape")
+    _decided()
     return {"codes": codes, "scales": scales, "S": float(Sarr[0]), "S_f32": Sarr, "status": st,
-            "p": bp, "err": be, "err2": be2, "nvalid": bn}
+            "p": bp, "err": be, "gap": bg, "tie": bt.astype(bool), "p2": b2, "nvalid": bn}
 
 
 IF4_SWEEP = {"absmax": 0, "sweep": 1, "brute": 2}
@@ -175,21 +203,26 @@ IF4_SWEEP = {"absmax": 0, "sweep": 1, "brute": 2}
 
 def if4_quantize(x, S=None, hadamard16=False, sweep="absmax"):
     """IF4 codes, scale bytes (indicator in bit 7) and S.  sweep: "absmax" (the AbsMax scale),
-    "sweep" (IF4 x ScaleSweep over the MSE window), "brute" (every E4M3 pattern)."""
+    "sweep" (IF4 x ScaleSweep over the MSE window), "brute" (every E4M3 pattern).  Diagnostics:
+    err_fp / err_int (both types' exact block errors at the chosen pattern), gap / tie (the
+    runner-up over every (pattern, type) candidate)."""
     x = rotate16(x) if hadamard16 else _f32(x)
     rows, cols = x.shape
     nb = cols // 16
     codes = np.zeros((rows, cols // 2), np.uint8)
     scales = np.zeros((rows, nb), np.uint8)
     Sarr = np.array([0.0 if S is None else S], np.float32)
-    ef = np.zeros((rows, nb), np.float32)
-    ei = np.zeros((rows, nb), np.float32)
+    ef = np.zeros((rows, nb), np.float64)
+    ei = np.zeros((rows, nb), np.float64)
+    bg = np.zeros((rows, nb), np.float64)
+    bt = np.zeros((rows, nb), np.int32)
     st = lib().fp4q_o_if4_quantize(_p(x), rows, cols, cols, IF4_SWEEP[sweep], int(S is not None), _p(Sarr),
-                                   _p(codes), _p(scales), _p(ef), _p(ei))
+                                   _p(codes), _p(scales), _p(ef), _p(ei), _p(bg), _p(bt))
     if st < 0:
         raise ValueError("oracle: bad shape")
+    _decided()
     return {"codes": codes, "scales": scales, "S": float(Sarr[0]), "S_f32": Sarr, "status": st,
-            "err_fp": ef, "err_int": ei}
+            "err_fp": ef, "err_int": ei, "gap": bg, "tie": bt.astype(bool)}
 
 
 MX_SWEEP = {"rule": 0, "sweep": 1, "brute": 2}
@@ -197,27 +230,48 @@ MX_SWEEP = {"rule": 0, "sweep": 1, "brute": 2}
 
 def mxfp4_quantize(x, hadamard=False, ocp_floor=False, sweep="rule"):
     """MXFP4 codes and E8M0 scale bytes.  sweep: "rule" (the max rule, ceil or OCP floor),
-    "sweep" (the MX scale sweep over e_c - 2 .. e_c), "brute" (every exponent)."""
+    "sweep" (the MX scale sweep over e_c - 2 .. e_c), "brute" (every exponent); gap / tie: the
+    near-tie statistic of the sweep modes."""
     x = _f32(x)
     rows, cols = x.shape
     codes = np.zeros((rows, cols // 2), np.uint8)
     scales = np.zeros((rows, cols // 32), np.uint8)
+    bg = np.zeros((rows, cols // 32), np.float64)
+    bt = np.zeros((rows, cols // 32), np.int32)
     st = lib().fp4q_o_mxfp4_quantize(_p(x), rows, cols, cols, int(hadamard), int(ocp_floor), MX_SWEEP[sweep],
-                                     _p(codes), _p(scales))
+                                     _p(codes), _p(scales), _p(bg), _p(bt))
     if st < 0:
         raise ValueError("oracle: bad shape")
-    return {"codes": codes, "scales": scales, "status": st}
+    _decided()
+    return {"codes": codes, "scales": scales, "status": st, "gap": bg, "tie": bt.astype(bool)}
 
 
 def mx_block_errors(x, scales, hadamard=False):
-    """Per-block error E (units of 4^e) of MXFP4 blocks at the exponents of `scales`."""
+    """Exact block errors sum (v - q 2^e)^2 (float64) of MXFP4 blocks at the exponents of `scales`."""
     x = _f32(x)
     rows, cols = x.shape
     scales = np.ascontiguousarray(scales, np.uint8)
-    err = np.zeros((rows, cols // 32), np.float32)
+    err = np.zeros((rows, cols // 32), np.float64)
     if lib().fp4q_o_mx_block_errors(_p(x), rows, cols, cols, int(hadamard), _p(scales), _p(err)) < 0:
         raise ValueError("oracle: bad shape")
     return err
+
+
+def near_ties(r, threshold=1e-6):
+    """The near-tie statistic of a quantizer result: among blocks with a runner-up, those whose
+    runner-up is within `threshold` relative of the best ((E2 - E1) / max(E1, FLT_MIN) <
+    threshold), and, separately, exact ties."""
+    gap = np.asarray(r["gap"]).ravel()
+    has = np.isfinite(gap) | np.asarray(r["tie"]).ravel()
+    near = (gap < threshold) & has
+    out = {"blocks": int(gap.size), "with_runner_up": int(has.sum()), "near": int(near.sum()),
+           "exact": int(np.asarray(r["tie"]).ravel().sum())}
+    out["near_frac"] = out["near"] / max(out["blocks"], 1)
+    if "p2" in r:
+        p, p2 = np.asarray(r["p"]).ravel(), np.asarray(r["p2"]).ravel()
+        t = np.asarray(r["tie"]).ravel()
+        out["exact_octave_pairs"] = int(np.sum(t & (np.abs(p2 - p) == 8)))
+    return out
 
 
 def dequantize(codes, scales, S, fmt, inverse_hadamard=False, out_bf16=False):
@@ -296,6 +350,15 @@ def mxfp4_gemm(a_codes, a_scales, b_codes, b_scales):
         e = np.array([np.ldexp(1.0, b - 127) if b != 0xFF else np.nan for b in range(256)], np.float64)
         return q * np.repeat(e[np.asarray(scales, np.uint8)], 32, axis=1)
     return values(a_codes, a_scales) @ values(b_codes, b_scales).T
+
+
+def f32_to_bf16(x) -> np.ndarray:
+    """The oracle's own float32 -> bf16 rounding (nearest, ties to even; NaN stays NaN), as bit
+    patterns: the reference for the bf16 dequantize output."""
+    x = np.ascontiguousarray(x, np.float32).ravel()
+    out = np.empty(x.size, np.uint16)
+    lib().fp4q_o_f32_to_bf16(_p(x), x.size, _p(out))
+    return out
 
 
 def widen_bf16(bits) -> np.ndarray:

@@ -28,41 +28,39 @@
  * "lowest offset wins a tie" rule are fixed by the workload specification that
  * accompanies the pages.
  *
- * Arithmetic contract (the readings where the pages are silent; every floating point
- * step is one IEEE-754 binary32 operation rounded to nearest even, written RN below;
- * no contraction, no flush-to-zero):
+ * Arithmetic (the readings where the pages are silent).  RN is one IEEE-754 binary32
+ * operation rounded to nearest even; no contraction, no flush-to-zero.
  *   S      = RN(amax / 1536)                      (amax = max |x| over the tensor)
  *   p0     = E4M3(RN(a_b / RN(6*S)))               (a_b = max |x| over the block)
  *   p4     = E4M3(RN(a_b / RN(4*S)))               (4/6 only)
- *   sv(p)  = RN(e(p) * S), inv(p) = RN(1 / sv(p)); sv(0) = inv(0) = 0
- *   y      = RN(x * inv),  q = E2M1(y),  r = RN(q - y)   (the quantizer's own rounding
- *            error, in units of the scale)
- *   error  = RN(RN(sv*sv) * E) with E = RN(acc_even + acc_odd); acc_even / acc_odd are fp32
- *            accumulators over the even / odd element positions, each acc = fma(r, r, acc)
- *            (WMSE: acc = fma(RN(w*r), r, acc)) in element order.  For the zero scale
- *            (p = 0) every code is 0 and the error is the same fma sum over x itself.
- *            This is the block MSE sum (x - q*s)^2 = s^2 sum (x/s - q)^2 evaluated on the
- *            binary32 quotient y the quantizer rounds.
- *   argmin = lexicographic (error, offset): the lowest offset wins a tie.
- *   IF4    = AbsMax scale p0; INT4 path z = RN(y*RN(7/6)), n = clamp(rint(z), -7, 7),
- *            v = RN(n*RN(6/7)), r = RN(v - y); both paths share s, so INT4 iff
- *            E_int < E_fp.
- *   IF4 sweep = every MSE-window candidate p0-3 .. p0+7 under both types, error
- *            RN(RN(sv*sv) * E) as for the NVFP4 sweep; (error, offset, FP4-before-INT4)
- *            lexicographic.
- *   MXFP4  = e = smallest integer with a_b <= 6*2^e (clamped to [-127,127]), byte e+127,
- *            y = RN(x * 2^-e), q = E2M1(y), dequant q*2^e.
- *   MX sweep = e among e_c - 2 .. e_c (e_c the rule above) minimizing RN(E * 4^(e - e_c)),
- *            E = RN(acc_even + acc_odd) of fma(r, r, acc), r = RN(q - y) at that e; lowest e
- *            wins a tie.
+ *   sv(p)  = RN(e(p) * S), inv(p) = RN(1 / sv(p)); sv(0) = inv(0) = 0   (the block scale the
+ *            quantizer holds in binary32, and its reciprocal)
+ *   codes  : FP4  q = E2M1(RN(x * inv));  INT4 n = clamp(rint(RN(RN(x * inv) * RN(7/6))), -7, 7);
+ *            MXFP4 q = E2M1(RN(x * 2^-e))
+ *   reconstruction (exact real products): FP4 xhat = q * sv; INT4 xhat = n * RN(6/7) * sv;
+ *            MXFP4 xhat = q * 2^e
+ *   MSE objective (AbsMax has none; 4/6, the MSE sweep, IF4, the IF4 sweep, the MX sweep):
+ *            the block's squared reconstruction error E = sum_i (x_i - xhat_i)^2, compared
+ *            EXACTLY (no rounding anywhere in the comparison; see exact_F below).  Ties go to
+ *            the lowest offset (4/6: the max->6 scale; IF4: FP4; the IF4 sweep: lowest offset,
+ *            then FP4; the MX sweep: the lowest exponent).
+ *   WMSE objective (importance-weighted; exact sums are out of reach with arbitrary weights, so
+ *            binary32 with one accumulator per candidate, in element order):
+ *            xhat = RN(q * sv), d = RN(x - xhat), acc = fma(RN(w * d), d, acc) for i = 0..15;
+ *            argmin (acc, offset) lexicographic; NaN never wins; if every acc is +inf the first
+ *            candidate is kept.
+ *   MXFP4  = e = smallest integer with a_b <= 6*2^e (clamped to [-127,127]), byte e+127.
+ *   MX sweep = e among e_c - 2 .. e_c (e_c the rule above, none below -127), exact MSE.
  *   Hadamard(32) = Sylvester fast Walsh-Hadamard butterflies for h = 1,2,4,8,16
  *            (v_j, v_j+h) <- (RN(v_j + v_j+h), RN(v_j - v_j+h)), then RN(v * RN(1/sqrt(32))).
- *   dequant NVFP4 x^ = RN(q * sv); IF4-INT4 x^ = RN(RN(n*RN(6/7)) * sv); MXFP4 x^ = RN(q*2^e).
+ *   dequant NVFP4 x^ = RN(q * sv); IF4-INT4 x^ = RN(RN(n*RN(6/7)) * sv); MXFP4 x^ = RN(q*2^e)
+ *            (the binary32 output rounds the exact reconstruction of the objective).
  */
 #include <math.h>
 #include <stdint.h>
 #include <string.h>
 #include <float.h>
+#include <stdlib.h>
 
 #define ST_OK 0
 #define ST_NONFINITE 1
@@ -200,7 +198,103 @@ int fp4q_o_tensor_scale(const float* x, int64_t rows, int64_t cols, int64_t ld, 
 
 
 /* ------------------------------------------------------------------------------------
- * NVFP4 candidate evaluation
+ * Exact block errors
+ * ---------------------------------------------------------------------------------- */
+
+/* long double carries at least 64 significand bits on the hosts this runs on (x86-64 extended
+ * precision, or binary128); every exactness bound below relies on it. */
+_Static_assert(LDBL_MANT_DIG >= 64, "the exact block errors need a 64-bit long double significand");
+
+/* The block error of one candidate relative to the block energy, held exactly:
+ *   E = sum_i (|x_i| - m_i g)^2 = sum_i x_i^2 + F,   F = g (g Q - 2 X),
+ * with m_i >= 0 the magnitude of element i's code (FP4: E2M1 value; INT4: |n|; MX: E2M1 value),
+ * g the grid step (FP4: sv; INT4: RN(6/7) * sv; MX: 2^e), Q = sum m_i^2, X = sum |x_i| m_i.
+ * sum x_i^2 is the same for every candidate of a block, so candidates are ordered by F.
+ * Why no step rounds (x_i binary32, so |x_i| = M 2^E with M < 2^24):
+ *  - an element with m_i > 0 has |x_i| >= g/4 (its quotient reached the first rounding
+ *    threshold: 0.25 for E2M1, 0.5 for INT4 before the 7/6 pre-scale), so every term |x_i| m_i
+ *    (exact: 24 + 3 bits) is a multiple of 2^(floor(log2 g) - 27); within the windows the block
+ *    maximum is at most 27 g (the worst case is p0 = 4 with offset -3 to pattern 1), so X < 2^13 g
+ *    and spans at most 41 bit positions: an exact long double sum (the brute-force modes reach
+ *    max|x| <= 2^20 g, still under 64 positions for FP4); Q is a multiple of 1/4 below 2^10;
+ *  - g Q is exact (g has at most 48 significand bits, Q at most 12), and u = g Q - 2 X spans
+ *    at most 62 bit positions in the windows (48-bit INT4 steps included), so it is exact too;
+ *  - F = g u is kept as hi + lo with hi = RN(g u) and lo = fma(g, u, -hi), the exact remainder.
+ * Comparing (hi, lo) lexicographically therefore compares the exact block errors. */
+typedef struct { long double hi, lo; int exact; } exact_F;
+
+/* Candidates compared with an inexact F (possible only in the brute-force window checks, for
+ * scales far below the block's, where X outgrows the span bound) are decided on hi alone; if
+ * two such values come within 2^-56 of each other the oracle cannot decide and counts it here
+ * (the bindings raise).  Every window mode is exact by the bounds above, which this also checks. */
+static long g_undecided = 0, g_inexact = 0;
+long fp4q_o_undecided(void) { long n = g_undecided; g_undecided = 0; return n; }
+long fp4q_o_inexact(void) { long n = g_inexact; g_inexact = 0; return n; }
+
+/* s = RN(a + b) is exactly a + b (Knuth's TwoSum remainder is zero). */
+static int sum_is_exact(long double a, long double b, long double s)
+{
+    const long double bb = s - a;
+    return ((a - (s - bb)) + (b - bb)) == 0.0L;
+}
+
+static exact_F block_F(const float* x, int B, const float* m, long double g)
+{
+    long double Q = 0.0L, X = 0.0L;
+    int exact = 1;
+    for (int i = 0; i < B; ++i) {
+        if (m[i] == 0.0f) continue;
+        Q += (long double)m[i] * (long double)m[i];
+        const long double t = fabsl((long double)x[i]) * (long double)m[i], s = X + t;
+        exact &= sum_is_exact(X, t, s);
+        X = s;
+    }
+    const long double p = g * Q;
+    exact &= fmal(g, Q, -p) == 0.0L;
+    const long double u = p - 2.0L * X;
+    exact &= sum_is_exact(p, -2.0L * X, u);
+    exact_F f;
+    f.hi = g * u;
+    f.lo = fmal(g, u, -f.hi);
+    f.exact = exact;
+    if (!exact) ++g_inexact;
+    return f;
+}
+
+static int F_less(exact_F a, exact_F b)
+{
+    if (a.exact && b.exact) return a.hi < b.hi || (a.hi == b.hi && a.lo < b.lo);
+    const long double m = fmaxl(fabsl(a.hi), fabsl(b.hi));
+    if (fabsl(a.hi - b.hi) <= ldexpl(m, -56)) ++g_undecided;
+    return a.hi < b.hi;
+}
+static int F_equal(exact_F a, exact_F b) { return a.exact && b.exact && a.hi == b.hi && a.lo == b.lo; }
+/* (b - a) as a long double (accurate to the last bits; used only for reporting). */
+static long double F_diff(exact_F a, exact_F b) { return (b.hi - a.hi) + (b.lo - a.lo); }
+
+/* The block error E itself, for reporting: the sum of the squared differences, each difference
+ * exact in long double (it spans fewer than 64 bit positions), the squares rounded to 64 bits.
+ * E is exactly 0 for a block the candidate reproduces. */
+static double block_E(const float* x, int B, const float* m, long double g)
+{
+    long double e = 0.0L;
+    for (int i = 0; i < B; ++i) {
+        const long double d = fabsl((long double)x[i]) - (long double)m[i] * g;
+        e += d * d;
+    }
+    return (double)e;
+}
+
+/* Relative gap of the runner-up to the best, (E2 - E1) / max(E1, FLT_MIN), the near-tie
+ * statistic; +inf when there is no runner-up. */
+static double rel_gap(double E1, long double diff)
+{
+    const double den = E1 > FLT_MIN ? E1 : FLT_MIN;
+    return (double)(diff / den);
+}
+
+/* ------------------------------------------------------------------------------------
+ * NVFP4
  * ---------------------------------------------------------------------------------- */
 
 static void scale_pair(int p, float S, float* sv, float* inv)
@@ -210,49 +304,47 @@ static void scale_pair(int p, float S, float* sv, float* inv)
     *inv = 1.0f / *sv;
 }
 
-/* Error of one candidate scale for a block of B values.  p = 0 (sv = 0): every code is
- * zero and the error is the sum of x^2 (WMSE: w x^2).  Otherwise: residuals of the
- * quantizer in units of the scale, r = RN(q - y), squares summed by fma into two
- * accumulators by element parity, combined once, then scaled by RN(sv^2). */
-static float block_error(const float* x, const float* w, int B, float sv, float inv)
+/* E2M1 magnitudes of a block's codes at reciprocal scale inv (the quantizer: RN(x * inv), then
+ * round to nearest even on the E2M1 grid). */
+static void fp4_mags(const float* x, int B, float inv, float* m)
 {
-    float acc[2] = {0.0f, 0.0f};
-    if (sv == 0.0f) {
-        for (int i = 0; i < B; ++i) {
-            if (w) acc[i & 1] = fmaf(w[i] * x[i], x[i], acc[i & 1]);
-            else acc[i & 1] = fmaf(x[i], x[i], acc[i & 1]);
-        }
-        return acc[0] + acc[1];
-    }
-    for (int i = 0; i < B; ++i) {
-        float y = x[i] * inv;
-        float q = fp4q_o_e2m1_value(fp4q_o_e2m1_encode(y));
-        float r = q - y;
-        if (w) acc[i & 1] = fmaf(w[i] * r, r, acc[i & 1]);
-        else acc[i & 1] = fmaf(r, r, acc[i & 1]);
-    }
-    float E = acc[0] + acc[1];
-    return (sv * sv) * E;
+    for (int i = 0; i < B; ++i) m[i] = E2M1_MAG[fp4q_o_e2m1_encode(x[i] * inv) & 7];
 }
 
-static uint8_t pack_codes_for(const float* x, int B, float inv, uint8_t* codes_row, int64_t c0)
+/* WMSE error of one candidate: binary32, one accumulator, element order.  The zero scale
+ * (sv = inv = 0) needs no special case: every code is +-0, xhat = 0, d = x. */
+static float wmse_error(const float* x, const float* w, int B, float sv, float inv)
+{
+    float acc = 0.0f;
+    for (int i = 0; i < B; ++i) {
+        const float q = fp4q_o_e2m1_value(fp4q_o_e2m1_encode(x[i] * inv));
+        const float xh = q * sv;
+        const float d = x[i] - xh;
+        acc = fmaf(w[i] * d, d, acc);
+    }
+    return acc;
+}
+
+static void pack_codes_for(const float* x, int B, float inv, uint8_t* codes_row, int64_t c0)
 {
     for (int i = 0; i < B; i += 2) {
         int lo = fp4q_o_e2m1_encode(x[i] * inv);
         int hi = fp4q_o_e2m1_encode(x[i + 1] * inv);
         codes_row[(c0 + i) / 2] = (uint8_t)(lo | (hi << 4));
     }
-    return 0;
 }
 
 /* objective: 0 AbsMax, 1 4/6, 2 sweep MSE [-3,7], 3 sweep WMSE [-8,7],
  *            4 brute-force MSE over all patterns 0..126, 5 brute-force WMSE.
- * Per block outputs (optional, may be NULL): chosen pattern, its error, runner-up error
- * (+inf when only one candidate), number of valid candidates. */
+ * Per block outputs (optional, may be NULL): chosen pattern; its error (MSE kinds: the exact
+ * block error E rounded to double; WMSE: the binary32 accumulator); the relative gap of the
+ * runner-up, (E2 - E1) / max(E1, FLT_MIN) (+inf with one candidate); whether the runner-up
+ * ties the best exactly; the runner-up's pattern (-1 with one candidate); the number of valid
+ * candidates. */
 int fp4q_o_nvfp4_quantize(const float* x, int64_t rows, int64_t cols, int64_t ld,
                           int objective, const float* importance, int scale_given,
                           float* S_io, uint8_t* codes, uint8_t* scales,
-                          int* blk_p, float* blk_err, float* blk_err2, int* blk_nvalid)
+                          int* blk_p, double* blk_err, double* blk_gap, int* blk_tie, int* blk_p2, int* blk_nvalid)
 {
     const int B = 16;
     if (cols % B) return -1;
@@ -299,22 +391,45 @@ int fp4q_o_nvfp4_quantize(const float* x, int64_t rows, int64_t cols, int64_t ld
             else { for (int k = lo; k <= hi; ++k) { int p = p0 + k; if (p >= 0 && p <= 0x7E) cand[nc++] = p; } }
             if (S == 0.0f) { nc = 1; cand[0] = 0; }
 
-            int bestp = cand[0];
-            float best = INFINITY, second = INFINITY;
-            for (int c = 0; c < nc; ++c) {
+            int bestp = cand[0], secp = -1, tie = 0;
+            double err = 0.0, gap = INFINITY;
+            if (weighted) {
+                float best = INFINITY, second = INFINITY;
+                for (int c = 0; c < nc; ++c) {
+                    float sv, inv;
+                    scale_pair(cand[c], S, &sv, &inv);
+                    const float e = wmse_error(xb, wb, B, sv, inv);
+                    if (c == 0 || e < best) { if (c) { second = best; secp = bestp; } best = e; bestp = cand[c]; }
+                    else if (c == 1 || e < second) { second = e; secp = cand[c]; }
+                }
+                err = best;
+                if (nc > 1) { gap = rel_gap(best, (long double)second - (long double)best); tie = second == best; }
+            } else {
+                exact_F best = {0.0L, 0.0L, 1}, second = {INFINITY, 0.0L, 1};
+                float m[16];
+                for (int c = 0; c < nc; ++c) {
+                    float sv, inv;
+                    scale_pair(cand[c], S, &sv, &inv);
+                    fp4_mags(xb, B, inv, m);
+                    const exact_F f = block_F(xb, B, m, (long double)sv);
+                    if (c == 0 || F_less(f, best)) { if (c) { second = best; secp = bestp; } best = f; bestp = cand[c]; }
+                    else if (c == 1 || F_less(f, second)) { second = f; secp = cand[c]; }
+                }
                 float sv, inv;
-                scale_pair(cand[c], S, &sv, &inv);
-                float e = block_error(xb, wb, B, sv, inv);
-                if (e < best) { second = best; best = e; bestp = cand[c]; }
-                else if (e < second) second = e;
+                scale_pair(bestp, S, &sv, &inv);
+                fp4_mags(xb, B, inv, m);
+                err = block_E(xb, B, m, (long double)sv);
+                if (nc > 1) { gap = rel_gap(err, F_diff(best, second)); tie = F_equal(best, second); }
             }
             float sv, inv;
             scale_pair(bestp, S, &sv, &inv);
             pack_codes_for(xb, B, inv, codes + r * (cols / 2), b * B);
             scales[r * nb + b] = (uint8_t)bestp;
             if (blk_p) blk_p[r * nb + b] = bestp;
-            if (blk_err) blk_err[r * nb + b] = best;
-            if (blk_err2) blk_err2[r * nb + b] = second;
+            if (blk_err) blk_err[r * nb + b] = err;
+            if (blk_gap) blk_gap[r * nb + b] = gap;
+            if (blk_tie) blk_tie[r * nb + b] = tie;
+            if (blk_p2) blk_p2[r * nb + b] = secp;
             if (blk_nvalid) blk_nvalid[r * nb + b] = nc;
         }
     }
@@ -327,43 +442,43 @@ int fp4q_o_nvfp4_quantize(const float* x, int64_t rows, int64_t cols, int64_t ld
 
 static float rint_even(float z) { return nearbyintf(z); } /* default rounding mode: to nearest even */
 
-/* FP4 and scaled-INT4 residual sums of one block at reciprocal scale inv, in units of the
- * scale (E = RN(acc_even + acc_odd), fma accumulation in element order), and the codes of both
- * paths.  [IF4]: INT4 z = RN(y*RN(7/6)), n = clamp(rint(z), -7, 7), v = RN(n*RN(6/7)). */
-static void if4_block_sums(const float* xb, float inv, float* ef, float* ei, int* cf, int* ci)
+/* The scaled-INT4 code of x at reciprocal scale inv: n = clamp(rint(RN(RN(x*inv) * RN(7/6))), -7, 7). */
+static int int4_code(float x, float inv)
 {
-    const float K76 = 7.0f / 6.0f, K67 = 6.0f / 7.0f;   /* RN of each ratio */
-    float accf[2] = {0, 0}, acci[2] = {0, 0};
-    for (int i = 0; i < 16; ++i) {
-        float y = xb[i] * inv;
-        cf[i] = fp4q_o_e2m1_encode(y);
-        float q = fp4q_o_e2m1_value(cf[i]);
-        float rf = q - y;
-        accf[i & 1] = fmaf(rf, rf, accf[i & 1]);
-        float z = y * K76;
-        float n = rint_even(z);
-        if (n > 7.0f) n = 7.0f;
-        if (n < -7.0f) n = -7.0f;
-        float v = n * K67;
-        float ri = v - y;
-        acci[i & 1] = fmaf(ri, ri, acci[i & 1]);
-        ci[i] = ((int)n) & 0xF;   /* two's complement nibble */
-    }
-    *ef = accf[0] + accf[1];
-    *ei = acci[0] + acci[1];
+    const float K76 = 7.0f / 6.0f;   /* RN(7/6) */
+    const float y = x * inv;
+    float n = rint_even(y * K76);
+    if (n > 7.0f) n = 7.0f;
+    if (n < -7.0f) n = -7.0f;
+    return (int)n;
 }
 
-/* sweep: 0 = IF4 at the AbsMax scale p0 (INT4 iff E_int < E_fp);
+/* Both types of one candidate pattern: their exact F values and their magnitudes. */
+static void if4_candidate(const float* xb, float S, int p, exact_F* ffp, exact_F* fint, float* mfp, float* mint,
+                          long double* gfp, long double* gint)
+{
+    float sv, inv;
+    scale_pair(p, S, &sv, &inv);
+    const float K67 = 6.0f / 7.0f;   /* RN(6/7) */
+    fp4_mags(xb, 16, inv, mfp);
+    for (int i = 0; i < 16; ++i) mint[i] = (float)abs(int4_code(xb[i], inv));
+    *gfp = (long double)sv;
+    *gint = (long double)K67 * (long double)sv;   /* exact: 24 x 24 bits */
+    *ffp = block_F(xb, 16, mfp, *gfp);
+    *fint = block_F(xb, 16, mint, *gint);
+}
+
+/* sweep: 0 = IF4 at the AbsMax scale p0 (INT4 iff E_int < E_fp, exactly);
  *        1 = IF4 x ScaleSweep: every candidate p0 + k, k = -3..+7 (patterns 0..126), under
- *            both element types; error = RN(RN(sv^2) * E) (the zero scale: the fma sum of x^2,
- *            both types alike); lexicographic (error, offset, type) with FP4 before INT4, so
- *            the lowest offset and then FP4 win ties;
+ *            both element types, exact errors, lexicographic (error, offset, type) with FP4 before
+ *            INT4, so the lowest offset and then FP4 win ties;
  *        2 = the same over all patterns 0..126 (window check).
- * blk_err_fp / blk_err_int receive both types' errors at the chosen pattern (mode 0: the
- * unscaled E; modes 1-2: the scaled errors). */
+ * blk_err_fp / blk_err_int receive both types' exact errors E at the chosen pattern (rounded to
+ * double); blk_gap / blk_tie the runner-up's relative gap and exact-tie flag over all (pattern,
+ * type) candidates. */
 int fp4q_o_if4_quantize(const float* x, int64_t rows, int64_t cols, int64_t ld, int sweep,
                         int scale_given, float* S_io, uint8_t* codes, uint8_t* scales,
-                        float* blk_err_fp, float* blk_err_int)
+                        double* blk_err_fp, double* blk_err_int, double* blk_gap, int* blk_tie)
 {
     const int B = 16;
     if (cols % B) return -1;
@@ -391,53 +506,47 @@ int fp4q_o_if4_quantize(const float* x, int64_t rows, int64_t cols, int64_t ld, 
             const float* xb = x + r * ld + b * B;
             float ab = 0.0f;
             for (int i = 0; i < B; ++i) ab = fmaxf(ab, fabsf(xb[i]));
-            int p0 = S > 0.0f ? fp4q_o_e4m3_encode(ab / d6) : 0;
-            int bp = p0, use_int = 0;
-            float ef, ei;
-            int cf[16], ci[16];
-            if (sweep == 0) {
-                float sv, inv;
-                scale_pair(p0, S, &sv, &inv);
-                if4_block_sums(xb, inv, &ef, &ei, cf, ci);
-                use_int = ei < ef;
-            } else {
-                int lo = sweep == 1 ? p0 - 3 : 0, hi = sweep == 1 ? p0 + 7 : 0x7E;
-                if (lo < 0) lo = 0;
-                if (hi > 0x7E) hi = 0x7E;
-                if (S == 0.0f) lo = hi = 0;
-                float best = INFINITY, bf = 0.0f, bi = 0.0f;
-                bp = lo;
-                for (int p = lo; p <= hi; ++p) {
-                    float e_fp, e_int;
-                    if (p == 0) {
-                        float acc[2] = {0, 0};
-                        for (int i = 0; i < B; ++i) acc[i & 1] = fmaf(xb[i], xb[i], acc[i & 1]);
-                        e_fp = e_int = acc[0] + acc[1];
-                    } else {
-                        float sv, inv, E_f, E_i;
-                        scale_pair(p, S, &sv, &inv);
-                        if4_block_sums(xb, inv, &E_f, &E_i, cf, ci);
-                        const float s2 = sv * sv;
-                        e_fp = s2 * E_f;
-                        e_int = s2 * E_i;
+            const int p0 = S > 0.0f ? fp4q_o_e4m3_encode(ab / d6) : 0;
+            int plo = p0, phi = p0;
+            if (sweep == 1) { plo = p0 - 3; phi = p0 + 7; }
+            if (sweep == 2) { plo = 0; phi = 0x7E; }
+            if (plo < 0) plo = 0;
+            if (phi > 0x7E) phi = 0x7E;
+            int bp = plo, use_int = 0, first = 1, tie = 0;
+            exact_F best = {0.0L, 0.0L, 1}, second = {INFINITY, 0.0L, 1};
+            for (int p = plo; p <= phi; ++p) {
+                exact_F f[2];
+                float mf[16], mi[16];
+                long double gf, gi;
+                if4_candidate(xb, S, p, &f[0], &f[1], mf, mi, &gf, &gi);
+                for (int t = 0; t < 2; ++t) {
+                    if (first || F_less(f[t], best)) {
+                        if (!first) second = best;
+                        best = f[t]; bp = p; use_int = t; first = 0;
+                    } else if (F_less(f[t], second)) {
+                        second = f[t];
                     }
-                    if (e_fp < best) { best = e_fp; bp = p; use_int = 0; bf = e_fp; bi = e_int; }
-                    if (e_int < best) { best = e_int; bp = p; use_int = 1; bf = e_fp; bi = e_int; }
                 }
-                float sv, inv;
-                scale_pair(bp, S, &sv, &inv);
-                if4_block_sums(xb, inv, &ef, &ei, cf, ci);   /* codes of the chosen scale */
-                ef = bf;
-                ei = bi;
             }
+            exact_F ff, fi;
+            float mf[16], mi[16];
+            long double gf, gi;
+            if4_candidate(xb, S, bp, &ff, &fi, mf, mi, &gf, &gi);
+            const double ef = block_E(xb, B, mf, gf), ei = block_E(xb, B, mi, gi);
+            float sv, inv;
+            scale_pair(bp, S, &sv, &inv);
             uint8_t* crow = codes + r * (cols / 2) + b * B / 2;
             for (int i = 0; i < B; i += 2) {
-                int lo = use_int ? ci[i] : cf[i], hi = use_int ? ci[i + 1] : cf[i + 1];
+                int lo = use_int ? (int4_code(xb[i], inv) & 0xF) : fp4q_o_e2m1_encode(xb[i] * inv);
+                int hi = use_int ? (int4_code(xb[i + 1], inv) & 0xF) : fp4q_o_e2m1_encode(xb[i + 1] * inv);
                 crow[i / 2] = (uint8_t)(lo | (hi << 4));
             }
+            tie = F_equal(best, second);
             scales[r * nb + b] = (uint8_t)(bp | (use_int ? 0x80 : 0));
             if (blk_err_fp) blk_err_fp[r * nb + b] = ef;
             if (blk_err_int) blk_err_int[r * nb + b] = ei;
+            if (blk_gap) blk_gap[r * nb + b] = rel_gap(use_int ? ei : ef, F_diff(best, second));
+            if (blk_tie) blk_tie[r * nb + b] = tie;
         }
     }
     return ST_OK;
@@ -501,72 +610,53 @@ int fp4q_o_mx_exponent(float a, int ocp_floor)
     return e;
 }
 
+/* E2M1 magnitudes of a 32-element block at scale 2^e: y = RN(v * 2^-e), exact for normal
+ * results. */
+static void mx_mags(const float* v, int e, float* m)
+{
+    const float s = ldexpf(1.0f, -e);
+    for (int i = 0; i < 32; ++i) m[i] = E2M1_MAG[fp4q_o_e2m1_encode(v[i] * s) & 7];
+}
+
 /* MX scale sweep [MR] ("Scale Fitting" for MXFP4: the page fits the power-of-two scale grid
  * to the data to cut the error that E8M0's coarse, over-wide grid causes, without giving the
- * rule; the plainest reading is ScaleSweep's search carried over to E8M0).  Error of one
- * 32-element block at scale 2^e, in units of 4^e: y = RN(x*2^-e), q = E2M1(y), r = RN(q - y),
- * E = RN(acc_even + acc_odd) with acc = fma(r, r, acc) over the even / odd positions in order,
- * as for NVFP4.  Multiplying by 2^-e is exact for normal results, so r is the rounding error
- * of the block in units of the scale. */
-static float mx_block_error(const float* v, int e)
-{
-    const float m = ldexpf(1.0f, -e);
-    float acc[2] = {0.0f, 0.0f};
-    for (int i = 0; i < 32; ++i) {
-        float y = v[i] * m;
-        float q = fp4q_o_e2m1_value(fp4q_o_e2m1_encode(y));
-        float r = q - y;
-        acc[i & 1] = fmaf(r, r, acc[i & 1]);
-    }
-    return acc[0] + acc[1];
-}
-
-/* Exponent of one block under mode: 0 the max rule (ceil, or OCP floor with ocp_floor);
- * 1 the sweep over e_c + k, k = -2..0, e_c = the ceil rule, patterns below -127 skipped,
- * comparing RN(E_k * 4^k) (the block error in units of 4^e_c; the power-of-two factor is
- * exact) lexicographically with the lowest k winning a tie;
- * 2 brute force over every e in [-127, 127] on the reconstruction error itself,
- * sum (x - q * 2^e)^2 accumulated in double (each term exact), lowest e winning a tie (checks
- * that the window of mode 1 holds the optimum; away from the window the scaled error of
- * mode 1 would underflow, the absolute one does not). */
-static double mx_block_abs_error(const float* v, int e)
-{
-    const float m = ldexpf(1.0f, -e);
-    double err = 0.0;
-    for (int i = 0; i < 32; ++i) {
-        double d = (double)v[i] - ldexp((double)fp4q_o_e2m1_value(fp4q_o_e2m1_encode(v[i] * m)), e);
-        err += d * d;
-    }
-    return err;
-}
-
-static int mx_block_exponent(const float* v, float ab, int ocp_floor, int mode)
+ * rule; the plainest reading is ScaleSweep's search carried over to E8M0).  Exponent of one
+ * block under mode: 0 the max rule (ceil, or OCP floor with ocp_floor); 1 the sweep over
+ * e_c + k, k = -2..0, e_c = the ceil rule, exponents below -127 skipped, the exact block error
+ * sum (v - q 2^e)^2 compared exactly, the lowest exponent winning a tie; 2 the same over every
+ * e in [-127, 127] (checks that the window of mode 1 holds the optimum).  gap / tie: the
+ * runner-up's relative gap and exact-tie flag (modes 1 and 2). */
+static int mx_block_exponent(const float* v, float ab, int ocp_floor, int mode, double* gap, int* tie)
 {
     const int ec = fp4q_o_mx_exponent(ab, 0);
+    *gap = INFINITY;
+    *tie = 0;
     if (mode == 0) return ocp_floor ? fp4q_o_mx_exponent(ab, 1) : ec;
-    if (mode == 1) {
-        int be = ec + (ec - 2 < -127 ? -127 - ec : -2);   /* the first candidate */
-        float best = INFINITY;
-        for (int k = -2; k <= 0; ++k) {
-            if (ec + k < -127) continue;
-            float err = mx_block_error(v, ec + k) * ldexpf(1.0f, 2 * k);
-            if (err < best) { best = err; be = ec + k; }
-        }
-        return be;
+    const int lo = mode == 1 ? (ec - 2 < -127 ? -127 : ec - 2) : -127, hi = mode == 1 ? ec : 127;
+    int be = lo, n = 0;
+    exact_F best = {0.0L, 0.0L, 1}, second = {INFINITY, 0.0L, 1};
+    float m[32];
+    for (int e = lo; e <= hi; ++e) {
+        mx_mags(v, e, m);
+        const exact_F f = block_F(v, 32, m, ldexpl(1.0L, e));
+        if (n == 0 || F_less(f, best)) { if (n) second = best; best = f; be = e; }
+        else if (F_less(f, second)) second = f;
+        ++n;
     }
-    int be = -127;
-    double best = INFINITY;
-    for (int e = -127; e <= 127; ++e) {
-        double err = mx_block_abs_error(v, e);
-        if (err < best) { best = err; be = e; }
+    if (n > 1) {
+        mx_mags(v, be, m);
+        *gap = rel_gap(block_E(v, 32, m, ldexpl(1.0L, be)), F_diff(best, second));
+        *tie = F_equal(best, second);
     }
     return be;
 }
 
 /* sweep: 0 the max rule, 1 the MX scale sweep (window [-2, 0]), 2 brute force over all
- * exponents; ocp_floor applies to sweep = 0 only. */
+ * exponents; ocp_floor applies to sweep = 0 only.  blk_gap / blk_tie (optional): the near-tie
+ * statistic of the sweep modes. */
 int fp4q_o_mxfp4_quantize(const float* x, int64_t rows, int64_t cols, int64_t ld,
-                          int hadamard, int ocp_floor, int sweep, uint8_t* codes, uint8_t* scales)
+                          int hadamard, int ocp_floor, int sweep, uint8_t* codes, uint8_t* scales,
+                          double* blk_gap, int* blk_tie)
 {
     const int B = 32;
     if (cols % B) return -1;
@@ -579,40 +669,46 @@ int fp4q_o_mxfp4_quantize(const float* x, int64_t rows, int64_t cols, int64_t ld
             int bad = 0;
             for (int i = 0; i < B; ++i) if (!isfinite(v[i])) bad = 1;
             uint8_t* crow = codes + r * (cols / 2) + b * B / 2;
+            double gap = INFINITY;
+            int tie = 0;
             if (bad) {
                 status |= ST_NONFINITE;
                 memset(crow, 0, B / 2);
                 scales[r * nb + b] = 0xFF;   /* E8M0 NaN */
-                continue;
+            } else {
+                if (hadamard) fp4q_o_hadamard32(v);
+                float ab = 0.0f;
+                for (int i = 0; i < B; ++i) ab = fmaxf(ab, fabsf(v[i]));
+                int e = mx_block_exponent(v, ab, ocp_floor, sweep, &gap, &tie);
+                float m = ldexpf(1.0f, -e);   /* exact power of two (subnormal for e = 127) */
+                for (int i = 0; i < B; i += 2) {
+                    int lo = fp4q_o_e2m1_encode(v[i] * m), hi = fp4q_o_e2m1_encode(v[i + 1] * m);
+                    crow[i / 2] = (uint8_t)(lo | (hi << 4));
+                }
+                scales[r * nb + b] = (uint8_t)(e + 127);
             }
-            if (hadamard) fp4q_o_hadamard32(v);
-            float ab = 0.0f;
-            for (int i = 0; i < B; ++i) ab = fmaxf(ab, fabsf(v[i]));
-            int e = mx_block_exponent(v, ab, ocp_floor, sweep);
-            float m = ldexpf(1.0f, -e);   /* exact power of two (subnormal for e = 127) */
-            for (int i = 0; i < B; i += 2) {
-                int lo = fp4q_o_e2m1_encode(v[i] * m), hi = fp4q_o_e2m1_encode(v[i + 1] * m);
-                crow[i / 2] = (uint8_t)(lo | (hi << 4));
-            }
-            scales[r * nb + b] = (uint8_t)(e + 127);
+            if (blk_gap) blk_gap[r * nb + b] = gap;
+            if (blk_tie) blk_tie[r * nb + b] = tie;
         }
     }
     return status;
 }
 
-/* Block errors of MXFP4 blocks (after the optional rotation) at the exponents given by the
- * scale bytes, in units of 4^e: the E of mx_block_error.  Returns -1 on a bad shape. */
+/* Exact block errors sum (v - q 2^e)^2 (rounded to double) of MXFP4 blocks (after the optional
+ * rotation) at the exponents given by the scale bytes.  Returns -1 on a bad shape. */
 int fp4q_o_mx_block_errors(const float* x, int64_t rows, int64_t cols, int64_t ld, int hadamard,
-                           const uint8_t* scales, float* err)
+                           const uint8_t* scales, double* err)
 {
     if (cols % 32) return -1;
     const int64_t nb = cols / 32;
     for (int64_t r = 0; r < rows; ++r)
         for (int64_t b = 0; b < nb; ++b) {
-            float v[32];
+            float v[32], m[32];
             memcpy(v, x + r * ld + b * 32, sizeof v);
             if (hadamard) fp4q_o_hadamard32(v);
-            err[r * nb + b] = mx_block_error(v, (int)scales[r * nb + b] - 127);
+            const int e = (int)scales[r * nb + b] - 127;
+            mx_mags(v, e, m);
+            err[r * nb + b] = block_E(v, 32, m, ldexpl(1.0L, e));
         }
     return 0;
 }
@@ -629,6 +725,12 @@ static uint16_t f32_to_bf16(float f)
     if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x7FFFFFu)) return (uint16_t)((u >> 16) | 0x40);
     u += 0x7FFFu + ((u >> 16) & 1u);
     return (uint16_t)(u >> 16);
+}
+
+/* Batch form of the bf16 rounding (for its pin). */
+void fp4q_o_f32_to_bf16(const float* x, int64_t n, uint16_t* out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = f32_to_bf16(x[i]);
 }
 
 /* fmt: 0 NVFP4, 1 IF4, 2 MXFP4.  out is float32 [rows][cols] (out_bf16 = 0) or uint16
