@@ -37,8 +37,9 @@
  *            quantizer holds in binary32, and its reciprocal)
  *   codes  : FP4  q = E2M1(RN(x * inv));  INT4 n = clamp(rint(RN(RN(x * inv) * RN(7/6))), -7, 7);
  *            MXFP4 q = E2M1(RN(x * 2^-e))
- *   reconstruction (exact real products): FP4 xhat = q * sv; INT4 xhat = n * RN(6/7) * sv;
- *            MXFP4 xhat = q * 2^e
+ *   reconstruction (exact real products): FP4 xhat = q * sv; INT4 xhat = n * g with
+ *            g = RN(RN(6/7) * sv), the INT4 block's scale (the 6/7 dequantization folded into the
+ *            block scale, held in binary32 like every scale); MXFP4 xhat = q * 2^e
  *   MSE objective (AbsMax has none; 4/6, the MSE sweep, IF4, the IF4 sweep, the MX sweep):
  *            the block's squared reconstruction error E = sum_i (x_i - xhat_i)^2, compared
  *            EXACTLY (no rounding anywhere in the comparison; see exact_F below).  Ties go to
@@ -53,8 +54,8 @@
  *   MX sweep = e among e_c - 2 .. e_c (e_c the rule above, none below -127), exact MSE.
  *   Hadamard(32) = Sylvester fast Walsh-Hadamard butterflies for h = 1,2,4,8,16
  *            (v_j, v_j+h) <- (RN(v_j + v_j+h), RN(v_j - v_j+h)), then RN(v * RN(1/sqrt(32))).
- *   dequant NVFP4 x^ = RN(q * sv); IF4-INT4 x^ = RN(RN(n*RN(6/7)) * sv); MXFP4 x^ = RN(q*2^e)
- *            (the binary32 output rounds the exact reconstruction of the objective).
+ *   dequant NVFP4 x^ = RN(q * sv); IF4-INT4 x^ = RN(n * RN(RN(6/7) * sv)); MXFP4 x^ = RN(q*2^e)
+ *            (the binary32 output is the rounding of the objective's exact reconstruction).
  */
 #include <math.h>
 #include <stdint.h>
@@ -208,7 +209,7 @@ _Static_assert(LDBL_MANT_DIG >= 64, "the exact block errors need a 64-bit long d
 /* The block error of one candidate relative to the block energy, held exactly:
  *   E = sum_i (|x_i| - m_i g)^2 = sum_i x_i^2 + F,   F = g (g Q - 2 X),
  * with m_i >= 0 the magnitude of element i's code (FP4: E2M1 value; INT4: |n|; MX: E2M1 value),
- * g the grid step (FP4: sv; INT4: RN(6/7) * sv; MX: 2^e), Q = sum m_i^2, X = sum |x_i| m_i.
+ * g the grid step (FP4: sv; INT4: RN(RN(6/7) * sv); MX: 2^e), Q = sum m_i^2, X = sum |x_i| m_i.
  * sum x_i^2 is the same for every candidate of a block, so candidates are ordered by F.
  * Why no step rounds (x_i binary32, so |x_i| = M 2^E with M < 2^24):
  *  - an element with m_i > 0 has |x_i| >= g/4 (its quotient reached the first rounding
@@ -217,8 +218,8 @@ _Static_assert(LDBL_MANT_DIG >= 64, "the exact block errors need a 64-bit long d
  *    maximum is at most 27 g (the worst case is p0 = 4 with offset -3 to pattern 1), so X < 2^13 g
  *    and spans at most 41 bit positions: an exact long double sum (the brute-force modes reach
  *    max|x| <= 2^20 g, still under 64 positions for FP4); Q is a multiple of 1/4 below 2^10;
- *  - g Q is exact (g has at most 48 significand bits, Q at most 12), and u = g Q - 2 X spans
- *    at most 62 bit positions in the windows (48-bit INT4 steps included), so it is exact too;
+ *  - g Q is exact (g is a binary32 value, Q has at most 12 bits), and u = g Q - 2 X spans at
+ *    most 44 bit positions in the windows (58 in the FP4 brute force), so it is exact too;
  *  - F = g u is kept as hi + lo with hi = RN(g u) and lo = fma(g, u, -hi), the exact remainder.
  * Comparing (hi, lo) lexicographically therefore compares the exact block errors. */
 typedef struct { long double hi, lo; int exact; } exact_F;
@@ -463,7 +464,7 @@ static void if4_candidate(const float* xb, float S, int p, exact_F* ffp, exact_F
     fp4_mags(xb, 16, inv, mfp);
     for (int i = 0; i < 16; ++i) mint[i] = (float)abs(int4_code(xb[i], inv));
     *gfp = (long double)sv;
-    *gint = (long double)K67 * (long double)sv;   /* exact: 24 x 24 bits */
+    *gint = (long double)(K67 * sv);   /* the INT4 block scale RN(RN(6/7) * sv) */
     *ffp = block_F(xb, 16, mfp, *gfp);
     *fint = block_F(xb, 16, mint, *gint);
 }
@@ -761,7 +762,7 @@ int fp4q_o_dequantize(const uint8_t* codes, const uint8_t* scales, float S,
                     scale_pair(sb & 0x7F, S, &sv, &inv);
                     if (fmt == 1 && (sb & 0x80)) {
                         int n = code >= 8 ? code - 16 : code;
-                        v[i] = ((float)n * K67) * sv;
+                        v[i] = (float)n * (K67 * sv);
                     } else {
                         v[i] = fp4q_o_e2m1_value(code) * sv;
                     }

@@ -176,7 +176,8 @@ def exact_int4_error(xb, p, S):
     s = sv_of(p, S)
     if not p:
         return exact_error(xb, [0] * len(xb))
-    return exact_error(xb, [n * Fr(float(K67)) * Fr(s) for n in int4_codes_exact(xb, s)])
+    g = Fr(float(f32(K67 * f32(s))))       # the INT4 block scale RN(RN(6/7) * sv)
+    return exact_error(xb, [n * g for n in int4_codes_exact(xb, s)])
 
 
 def _tensor_with(xb, amax=1536.0):
@@ -362,7 +363,8 @@ def test_wmse_with_unit_weights_tracks_mse():
 
 def test_if4_errors_are_exact():
     """IF4 at the AbsMax scale: both types' reported errors are the exact rational block MSE
-    (INT4 reconstruction n * RN(6/7) * sv, the integer times the 6/7 constant times the scale),
+    (INT4 reconstruction n * RN(RN(6/7) * sv): the integer times the block scale with the 6/7
+    dequantization folded in, in binary32 like every scale),
     and INT4 is chosen exactly when its exact error is lower (a tie keeps FP4)."""
     wl = synth.make("cfg4", rows=2, cols=1024)
     x = synth.as_f32(wl)
