@@ -136,6 +136,63 @@ def alloc_outputs(rows: int, cols: int, fmt: str, device="cuda", tiled: bool = F
     return codes, scales, gs
 
 
+def _objective(name) -> int:
+    if name is None:
+        return 0
+    if name not in OBJECTIVES:
+        raise Fp4qError(f"unknown objective {name!r} (one of {sorted(OBJECTIVES)})")
+    return OBJECTIVES[name]
+
+
+def _format(name) -> int:
+    if name not in FORMATS:
+        raise Fp4qError(f"unknown format {name!r} (one of {sorted(FORMATS)})")
+    return FORMATS[name]
+
+
+def _need(t, what, device, dtypes, numel=None, min_numel=None, contiguous=True):
+    """Raise Fp4qError unless t is a CUDA tensor on `device` of one of `dtypes` with the given
+    element count (exact, or at least min_numel), contiguous unless told otherwise.  Every
+    wrapper checks its tensors this way before calling into the library, so no pointer the
+    kernels would read or write out of bounds ever reaches them."""
+    if t is None:
+        raise Fp4qError(f"{what} is required")
+    if not t.is_cuda or t.device != device:
+        raise Fp4qError(f"{what} must be a CUDA tensor on {device} (got {t.device})")
+    if t.dtype not in dtypes:
+        raise Fp4qError(f"{what} must have dtype {' or '.join(str(d) for d in dtypes)} (got {t.dtype})")
+    if contiguous and not t.is_contiguous():
+        raise Fp4qError(f"{what} must be contiguous")
+    if numel is not None and t.numel() != numel:
+        raise Fp4qError(f"{what} must hold {numel} elements (got {t.numel()})")
+    if min_numel is not None and t.numel() < min_numel:
+        raise Fp4qError(f"{what} must hold at least {min_numel} elements (got {t.numel()})")
+
+
+def _check_quantize(x, fmt, objective, importance, codes, scales, gs, tiled, workspace=None, device_status=None):
+    torch = _torch()
+    if x is None or not x.is_cuda:
+        raise Fp4qError("x must be a CUDA tensor")
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise Fp4qError("x must be 2-D with unit column stride")
+    _dtype_code(x)
+    rows, cols = x.shape
+    dev = x.device
+    _need(codes, "codes", dev, (torch.uint8,), numel=rows * (cols // 2))
+    _need(scales, "scales", dev, (torch.uint8,), numel=scale_bytes(rows, cols, fmt, tiled))
+    if fmt != "mxfp4":
+        _need(gs, "global scale", dev, (torch.float32,), min_numel=1)
+    if fmt == "nvfp4" and objective == "sweep_wmse":
+        _need(importance, "importance", dev, (torch.float32,), min_numel=cols)
+    if workspace is not None:
+        _need(workspace, "workspace", dev, (torch.uint8, torch.int32, torch.int64, torch.float32),
+              contiguous=True)
+        if workspace.numel() * workspace.element_size() < workspace_bytes():
+            raise Fp4qError(f"workspace must hold at least {workspace_bytes()} bytes")
+    if device_status is not None:
+        _need(device_status, "device_status", dev, (torch.int32, torch.uint32), min_numel=1)
+
+
 def _flags(global_scale, mx_ocp_floor, hadamard16, mx_sweep=False, if4_sweep=False, tiled=False):
     return ((F_GLOBAL_SCALE_GIVEN if global_scale is not None else 0) | (F_MX_OCP_FLOOR if mx_ocp_floor else 0)
             | (F_HADAMARD16 if hadamard16 else 0) | (F_MX_SWEEP if mx_sweep else 0)
@@ -163,16 +220,20 @@ def quantize(x, fmt: str = "nvfp4", objective: str = "sweep_mse", importance=Non
     if4_sweep: IF4 x ScaleSweep (scale and element type chosen together over the MSE window).
     tiled_scales: NVFP4/MXFP4 scales in the 128x4-tiled layout of block-scaled GEMMs (1-D buffer).
     """
-    if x.dim() != 2 or x.stride(1) != 1:
-        raise Fp4qError("x must be 2-D with unit column stride")
+    fcode, ocode = _format(fmt), _objective(objective)
+    if x is None or not x.is_cuda or x.dim() != 2 or x.stride(1) != 1:
+        raise Fp4qError("x must be a 2-D CUDA tensor with unit column stride")
     rows, cols = x.shape
+    if cols % BLOCK[fmt]:
+        raise Fp4qError(f"cols must be a multiple of {BLOCK[fmt]}")
     codes, scales, gs = out if out is not None else alloc_outputs(rows, cols, fmt, x.device, tiled=tiled_scales)
     flags = _flags(global_scale, mx_ocp_floor, hadamard16, mx_sweep, if4_sweep, tiled_scales)
     if global_scale is not None:
         gs = global_scale
     ws = workspace if workspace is not None else new_workspace(x.device)
-    rc = lib().fp4q_quantize(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), FORMATS[fmt],
-                             OBJECTIVES.get(objective, 0), _ptr(importance), _ptr(codes), _ptr(scales),
+    _check_quantize(x, fmt, objective, importance, codes, scales, gs, tiled_scales, workspace=ws)
+    rc = lib().fp4q_quantize(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), fcode,
+                             ocode, _ptr(importance), _ptr(codes), _ptr(scales),
                              _ptr(gs) if fmt != "mxfp4" else None, _ptr(ws), flags, _stream_ptr(stream))
     _check(rc, "fp4q_quantize")
     return codes, scales, (gs if fmt != "mxfp4" else None)
@@ -182,9 +243,14 @@ def global_scale(x, out=None, workspace=None, stream=None, hadamard16: bool = Fa
     """Tensor scale S = RN(max|x| / 1536) as a [1] float32 CUDA tensor (amax pass only);
     hadamard16: of the 16-point block-rotated tensor."""
     torch = _torch()
+    if x is None or not x.is_cuda or x.dim() != 2 or x.stride(1) != 1:
+        raise Fp4qError("x must be a 2-D CUDA tensor with unit column stride")
+    _dtype_code(x)
     rows, cols = x.shape
     gs = out if out is not None else torch.empty((1,), dtype=torch.float32, device=x.device)
     ws = workspace if workspace is not None else new_workspace(x.device)
+    _need(gs, "out", x.device, (torch.float32,), min_numel=1)
+    _need(ws, "workspace", x.device, (torch.uint8,), min_numel=workspace_bytes())
     if hadamard16:
         rc = lib().fp4q_hadamard_global_scale(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), 16, _ptr(gs),
                                               _ptr(ws), _stream_ptr(stream))
@@ -199,11 +265,14 @@ def hadamard_quantize(x, mx_ocp_floor: bool = False, out=None, workspace=None, s
                       tiled_scales: bool = False):
     """MXFP4 quantization after a normalized 32-point block Hadamard rotation (mx_sweep: with
     the MX scale sweep)."""
-    if x.dim() != 2 or x.stride(1) != 1:
-        raise Fp4qError("x must be 2-D with unit column stride")
+    if x is None or not x.is_cuda or x.dim() != 2 or x.stride(1) != 1:
+        raise Fp4qError("x must be a 2-D CUDA tensor with unit column stride")
     rows, cols = x.shape
+    if cols % 32:
+        raise Fp4qError("cols must be a multiple of 32")
     codes, scales, _ = out if out is not None else alloc_outputs(rows, cols, "mxfp4", x.device, tiled=tiled_scales)
     ws = workspace if workspace is not None else new_workspace(x.device)
+    _check_quantize(x, "mxfp4", None, None, codes, scales, None, tiled_scales, workspace=ws)
     rc = lib().fp4q_hadamard_quantize(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), 32, _ptr(codes),
                                       _ptr(scales), _ptr(ws), _flags(None, mx_ocp_floor, False, mx_sweep,
                                                                      tiled=tiled_scales),
@@ -215,12 +284,24 @@ def hadamard_quantize(x, mx_ocp_floor: bool = False, out=None, workspace=None, s
 def dequantize(codes, scales, global_scale, fmt: str = "nvfp4", inverse_hadamard: bool = False,
                out_dtype=None, out=None, stream=None, tiled_scales: bool = False):
     torch = _torch()
+    fcode = _format(fmt)
     out_dtype = out_dtype or torch.float32
+    if codes is None or not codes.is_cuda or codes.dim() != 2:
+        raise Fp4qError("codes must be a 2-D CUDA tensor [rows, cols/2]")
     rows, cols = codes.shape[0], codes.shape[1] * 2
+    dev = codes.device
+    if cols % BLOCK[fmt]:
+        raise Fp4qError(f"cols must be a multiple of {BLOCK[fmt]}")
+    _need(codes, "codes", dev, (torch.uint8,), numel=rows * (cols // 2))
+    _need(scales, "scales", dev, (torch.uint8,), numel=scale_bytes(rows, cols, fmt, tiled_scales))
+    if fmt != "mxfp4":
+        _need(global_scale, "global_scale", dev, (torch.float32,), min_numel=1)
     if out is None:
-        out = torch.empty((rows, cols), dtype=out_dtype, device=codes.device)
+        out = torch.empty((rows, cols), dtype=out_dtype, device=dev)
+    _need(out, "out", dev, (torch.float32, torch.bfloat16), numel=rows * cols)
     flags = (F_OUT_BF16 if out.dtype == torch.bfloat16 else 0) | (F_SCALE_TILED if tiled_scales else 0)
-    rc = lib().fp4q_dequantize(_ptr(codes), _ptr(scales), _ptr(global_scale), rows, cols, FORMATS[fmt],
+    rc = lib().fp4q_dequantize(_ptr(codes), _ptr(scales), _ptr(global_scale) if fmt != "mxfp4" else None,
+                               rows, cols, fcode,
                                int(inverse_hadamard), _ptr(out), flags, _stream_ptr(stream))
     _check(rc, "fp4q_dequantize")
     return out
@@ -228,23 +309,54 @@ def dequantize(codes, scales, global_scale, fmt: str = "nvfp4", inverse_hadamard
 
 def quantize_noalloc(x, fmt: str = "nvfp4", objective: str = "sweep_mse", importance=None, global_scale=None,
                      mx_ocp_floor: bool = False, out=None, device_status=None, stream=None,
-                     hadamard16: bool = False, mx_sweep: bool = False, if4_sweep: bool = False):
+                     hadamard16: bool = False, mx_sweep: bool = False, if4_sweep: bool = False,
+                     tiled_scales: bool = False):
     """quantize() for callers that cannot allocate device memory: the library's own
     per-GPU scratch replaces the workspace (see fp4q_quantize_noalloc in include/fp4q.h).
     Outputs must be passed in `out`; device_status is an optional [1] int32 CUDA tensor."""
-    if x.dim() != 2 or x.stride(1) != 1:
-        raise Fp4qError("x must be 2-D with unit column stride")
+    fcode, ocode = _format(fmt), _objective(objective)
+    if x is None or not x.is_cuda or x.dim() != 2 or x.stride(1) != 1:
+        raise Fp4qError("x must be a 2-D CUDA tensor with unit column stride")
+    if out is None:
+        raise Fp4qError("quantize_noalloc needs preallocated outputs (codes, scales, S)")
     rows, cols = x.shape
+    if cols % BLOCK[fmt]:
+        raise Fp4qError(f"cols must be a multiple of {BLOCK[fmt]}")
     codes, scales, gs = out
-    flags = _flags(global_scale, mx_ocp_floor, hadamard16, mx_sweep, if4_sweep)
+    flags = _flags(global_scale, mx_ocp_floor, hadamard16, mx_sweep, if4_sweep, tiled_scales)
     if global_scale is not None:
         gs = global_scale
-    rc = lib().fp4q_quantize_noalloc(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), FORMATS[fmt],
-                                     OBJECTIVES.get(objective, 0), _ptr(importance), _ptr(codes), _ptr(scales),
+    _check_quantize(x, fmt, objective, importance, codes, scales, gs, tiled_scales, device_status=device_status)
+    rc = lib().fp4q_quantize_noalloc(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), fcode,
+                                     ocode, _ptr(importance), _ptr(codes), _ptr(scales),
                                      _ptr(gs) if fmt != "mxfp4" else None, _ptr(device_status), flags,
                                      _stream_ptr(stream))
     _check(rc, "fp4q_quantize_noalloc")
     return codes, scales, (gs if fmt != "mxfp4" else None)
+
+
+def _check_gemm_operands(ac, asc, bc, bsc, fmt):
+    torch = _torch()
+    if ac is None or not ac.is_cuda or ac.dim() != 2 or bc is None or bc.dim() != 2:
+        raise Fp4qError("operand codes must be 2-D CUDA tensors [rows, K/2]")
+    M, K, N = ac.shape[0], ac.shape[1] * 2, bc.shape[0]
+    if bc.shape[1] * 2 != K:
+        raise Fp4qError("a and b must have the same K")
+    dev = ac.device
+    _need(ac, "a codes", dev, (torch.uint8,))
+    _need(bc, "b codes", dev, (torch.uint8,))
+    _need(asc, "a scales", dev, (torch.uint8,), numel=scale_bytes(M, K, fmt, True))
+    _need(bsc, "b scales", dev, (torch.uint8,), numel=scale_bytes(N, K, fmt, True))
+    return M, K, N
+
+
+def _check_gemm_out(d, M, N, ws):
+    torch = _torch()
+    if not d.is_cuda or d.dim() != 2 or d.shape[0] != M or d.shape[1] != N or d.stride(1) != 1:
+        raise Fp4qError(f"out must be a CUDA [{M}, {N}] tensor with unit column stride")
+    if d.dtype != torch.float32:
+        raise Fp4qError("out must be float32")
+    _need(ws, "workspace", d.device, (torch.uint8,), min_numel=workspace_bytes())
 
 
 def nvfp4_gemm(a, b, out=None, workspace=None, stream=None):
@@ -254,12 +366,12 @@ def nvfp4_gemm(a, b, out=None, workspace=None, stream=None):
     torch = _torch()
     ac, asc, ag = a
     bc, bsc, bg = b
-    M, K = ac.shape[0], ac.shape[1] * 2
-    N = bc.shape[0]
-    if bc.shape[1] * 2 != K:
-        raise Fp4qError("a and b must have the same K")
+    M, K, N = _check_gemm_operands(ac, asc, bc, bsc, "nvfp4")
     d = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=ac.device)
     ws = workspace if workspace is not None else new_workspace(ac.device)
+    _need(ag, "a's S", ac.device, (torch.float32,), min_numel=1)
+    _need(bg, "b's S", ac.device, (torch.float32,), min_numel=1)
+    _check_gemm_out(d, M, N, ws)
     rc = lib().fp4q_nvfp4_gemm(_ptr(ac), _ptr(asc), _ptr(ag), _ptr(bc), _ptr(bsc), _ptr(bg), M, N, K, _ptr(d),
                                d.stride(0), _ptr(ws), _stream_ptr(stream))
     _check(rc, "fp4q_nvfp4_gemm")
@@ -274,12 +386,10 @@ def mxfp4_gemm(a, b, out=None, workspace=None, stream=None):
     torch = _torch()
     ac, asc = a[0], a[1]
     bc, bsc = b[0], b[1]
-    M, K = ac.shape[0], ac.shape[1] * 2
-    N = bc.shape[0]
-    if bc.shape[1] * 2 != K:
-        raise Fp4qError("a and b must have the same K")
+    M, K, N = _check_gemm_operands(ac, asc, bc, bsc, "mxfp4")
     d = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=ac.device)
     ws = workspace if workspace is not None else new_workspace(ac.device)
+    _check_gemm_out(d, M, N, ws)
     rc = lib().fp4q_mxfp4_gemm(_ptr(ac), _ptr(asc), _ptr(bc), _ptr(bsc), M, N, K, _ptr(d), d.stride(0), _ptr(ws),
                                _stream_ptr(stream))
     _check(rc, "fp4q_mxfp4_gemm")
@@ -290,8 +400,11 @@ def encode(x, kind: str, out=None, stream=None):
     """The hardware element codec on a CUDA fp32 tensor: kind "e2m1" -> 4-bit E2M1 codes (sign
     in bit 3), "e4m3" -> E4M3FN bytes; both round to nearest even and saturate."""
     torch = _torch()
+    if x is None or not x.is_cuda or x.dtype != torch.float32:
+        raise Fp4qError("x must be a float32 CUDA tensor")
     x = x.contiguous().view(-1)
     out = out if out is not None else torch.empty(x.numel(), dtype=torch.uint8, device=x.device)
+    _need(out, "out", x.device, (torch.uint8,), numel=x.numel())
     rc = lib().fp4q_encode(_ptr(x), x.numel(), {"e2m1": 0, "e4m3": 1}[kind], _ptr(out), _stream_ptr(stream))
     _check(rc, "fp4q_encode")
     return out
@@ -368,7 +481,7 @@ class HostQuantizer:
         hc, hs, hg = host_out if host_out is not None else alloc_host_outputs(self.rows, self.cols, self.fmt)
         rc = lib().fp4q_quantize_host_async(
             _ptr(x_host), _dtype_code(x_host), self.rows, self.cols, FORMATS[self.base],
-            OBJECTIVES.get(self.objective or "absmax", 0), _ptr(self.importance), _ptr(hc), _ptr(hs),
+            _objective(self.objective), _ptr(self.importance), _ptr(hc), _ptr(hs),
             _ptr(hg) if self.base != "mxfp4" else None, _ptr(st["x"]), _ptr(st["codes"]), _ptr(st["scales"]),
             _ptr(st["S"]) if self.base != "mxfp4" else None, _ptr(st["ws"]), self.flags,
             C.c_void_p(self.copy_stream.cuda_stream), C.c_void_p(self.compute_stream.cuda_stream),

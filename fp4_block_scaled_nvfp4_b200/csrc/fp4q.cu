@@ -36,28 +36,6 @@
 
 namespace fp4q {
 
-// Build-time tuning of the 16-element kernels (defaults are the measured best).
-#ifndef FP4Q_SWEEP_SCALAR_ACC
-#define FP4Q_SWEEP_SCALAR_ACC 0   // 1: square-accumulate with scalar FMAs instead of packed pairs
-#endif
-#ifndef FP4Q_SWEEP_UNROLL
-#define FP4Q_SWEEP_UNROLL 11    // MSE candidate-loop unroll factor (11 = the whole window)
-#endif
-#ifndef FP4Q_WMSE_UNROLL
-#define FP4Q_WMSE_UNROLL 16     // WMSE candidate-loop unroll factor (16 = the whole window)
-#endif
-constexpr int kMseUnroll = FP4Q_SWEEP_UNROLL, kWmseUnroll = FP4Q_WMSE_UNROLL;
-
-#ifndef FP4Q_PERSIST_MIN_CTAS
-#define FP4Q_PERSIST_MIN_CTAS 5 // CTAs per SM of the persistent IF4 / AbsMax / 4-6 kernels (register cap)
-#endif
-#ifndef FP4Q_SWEEP_PERSISTENT
-#define FP4Q_SWEEP_PERSISTENT 1 // 0: the MSE sweep runs one block per thread instead of as one persistent wave
-#endif
-#ifndef FP4Q_SWEEP_MIN_CTAS
-#define FP4Q_SWEEP_MIN_CTAS 6   // CTAs per SM of a one-block-per-thread MSE sweep (register cap)
-#endif
-
 enum : int { WS_STATUS = 0, WS_PENDING = 1, WS_AMAX = 2, WS_CNT_AMAX = 3, WS_CNT_Q = 4 };
 constexpr size_t kWorkspaceBytes = 64;
 constexpr int kThreads = 256;
@@ -207,21 +185,22 @@ __global__ void __launch_bounds__(kThreads, 4) amax_kernel(const void* __restric
 // ------------------------------------------------------------------------------------------
 // Shared pieces of the NVFP4 / IF4 kernels
 // ------------------------------------------------------------------------------------------
-// Per-pattern scale table {inv, s2} with inv = RN(1/sv), s2 = RN(sv^2), sv = RN(e(p) * S),
-// indexed by p + kTabPad for p = -kTabPad .. 126 + kTabPad, so that a candidate window
-// [p0 - 8, p0 + 7] never leaves it.  Entries for patterns that are not candidates (p <= 0 or
-// p >= 127) hold inv = 0 and s2 = NaN: their error is NaN, which never compares below the
-// best, so the candidate loop needs no bounds.  inv = 0 is also the zero scale's reciprocal,
-// which makes the codes of pattern 0 the signs of the elements.
+// Per-pattern scale table {inv, e} with e = the E4M3 value of pattern p and inv = RN(1/sv),
+// sv = RN(e S), indexed by p + kTabPad for p = -kTabPad .. 126 + kTabPad, so that a candidate
+// window [p0 - 8, p0 + 7] never leaves it.  Entries for patterns that are not candidates (p < 0 or
+// p >= 127) hold inv = 0 and e = NaN: every score built from e is NaN and never wins, so the
+// candidate loops need no bounds.  Pattern 0, the zero scale, holds inv = 0 and e = 0: its codes
+// are the signs of the elements and its reconstruction is 0.
 constexpr int kTabPad = 8;
 constexpr int kTabLen = 127 + 2 * kTabPad;
 __device__ __forceinline__ void build_scale_table(float S, float2* tab) {
     for (int i = threadIdx.x; i < kTabLen; i += blockDim.x) {
         const int p = i - kTabPad;
         float2 t = make_float2(0.0f, __uint_as_float(0x7FC00000u));
+        if (p == 0) t.y = 0.0f;
         if (p >= 1 && p <= 126) {
-            const float sv = __fmul_rn(e4m3_value(p), S);
-            t = make_float2(__frcp_rn(sv), __fmul_rn(sv, sv));
+            const float e = e4m3_value(p);
+            t = make_float2(__frcp_rn(__fmul_rn(e, S)), e);
         }
         tab[i] = t;
     }
@@ -398,7 +377,280 @@ __global__ void __launch_bounds__(kThreads, 4) amax_had16_kernel(const void* __r
     amax_finish(m, 0.25f, ws, gscale, publish);
 }
 
-// Packed codes of a block for a given reciprocal scale (8 bytes: elements 0..15).
+// ------------------------------------------------------------------------------------------
+// Exact block errors
+// ------------------------------------------------------------------------------------------
+// A candidate with grid step g (FP4: sv; INT4: RN(RN(6/7) sv); MXFP4: 2^e) gives element i the
+// code magnitude m_i, and the block error is
+//   E = sum (|x_i| - m_i g)^2 = sum x_i^2 + g (g Q - 2 X),   Q = sum m_i^2,  X = sum |x_i| m_i.
+// The kernels evaluate it in fixed point.  Per block a shift k puts the magnitudes on integers
+// A_i = |x_i| 2^k (exact for every element that any candidate of the window can give a nonzero
+// code: those lie within a factor 2^7 of the block maximum, and bf16 values carry 8 significant
+// bits, so 15-bit integers hold them; binary32 values need 31 bits), and M_i = 2 m_i is a byte
+// (E2M1: 0,1,2,3,4,6,8,12; INT4: 0,2,...,14).  Q4 = sum M_i^2 and Xi = sum A_i M_i are exact
+// integer dot products (dp4a / dp2a), and with sigma4 = g 2^(k-2),
+//   G = sigma4 (sigma4 Q4 - Xi) = (E - sum x^2) 2^(2k) / 4,
+// the same positive multiple of E - sum x^2 for every candidate of the block, so candidates are
+// ranked by G.  In binary32, t = fma(sigma4, Q4, -Xi) and G~ = sigma4 t are each one rounding of
+// an exact value, so |G~ - G| <= 2^-22.9 |G|: a candidate whose G~ exceeds min G~ + 2^-20 |min G~|
+// is certainly worse.  When two or more candidates lie inside that margin (exact ties among
+// them), the block is decided on the exact G = hi + lo held in binary64: u = sigma4 Q4 - Xi is
+// exact there (fewer than 45 significant bits), hi = RN(sigma4 u), lo = fma(sigma4, u, -hi).
+// ScaleSweep (gist.science/ko/paper/2606.07618), Methodology: the objective is the block's
+// reconstruction error.
+
+constexpr uint32_t kLutE2M1Lo = 0x03020100u, kLutE2M1Hi = 0x0C080604u;   // 2 m for E2M1 codes 0..7
+constexpr uint32_t kMagicInt = 0x4B000000u;                              // bits of 2^23: ints < 2^23 ride in the mantissa
+constexpr float kTwo23 = 8388608.0f;
+
+// floor(log2 a) of a finite a > 0 (subnormals included).
+__device__ __forceinline__ int ilog2f(float a) {
+    const uint32_t u = __float_as_uint(a);
+    return u >= 0x00800000u ? (int)(u >> 23) - 127 : -118 - __clz(u);
+}
+// 2^k as two factors that are normal floats for k in [-250, 250].
+__device__ __forceinline__ void pow2_split(int k, float& fa, float& fb) {
+    const int ka = k >> 1;
+    fa = pow2i(ka);
+    fb = pow2i(k - ka);
+}
+
+// Fixed-point magnitudes of one block of 2 NP elements.  B16 (bf16 values): w[j] = A_{2j} | A_{2j+1} << 16
+// (15-bit integers).  Otherwise (binary32 values, 31-bit integers): w[4g + b] = byte b of A_{4g},
+// A_{4g+1}, A_{4g+2}, A_{4g+3} (byte planes, so that each plane is one dp4a operand).
+template <bool B16, int NP = 8>
+struct Fixed16 {
+    uint32_t w[B16 ? NP : 2 * NP];
+};
+
+// ap: the block's magnitudes (pairs), k: the shift, from a block maximum a with a 2^k in
+// [2^14, 2^15) (B16) or [2^30, 2^31).
+template <bool B16, int NP = 8>
+__device__ __forceinline__ void fixed_point(const u64 (&ap)[NP], int k, Fixed16<B16, NP>& A) {
+    float fa, fb;
+    pow2_split(k, fa, fb);
+    const u64 fa2 = pk(fa, fa);
+    if (B16) {
+        const u64 fb2 = pk(fb, fb), mg = pk(kTwo23, kTwo23);
+#pragma unroll
+        for (int j = 0; j < NP; ++j) {   // RN(|x| 2^k + 2^23): the integer sits in the low mantissa bits
+            float v0, v1;
+            upk(fma2(mul2(ap[j], fa2), fb2, mg), v0, v1);
+            A.w[j] = __byte_perm(__float_as_uint(v0), __float_as_uint(v1), 0x5410);
+        }
+    } else {
+#pragma unroll
+        for (int g = 0; g < NP / 2; ++g) {
+            uint32_t a[4];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float v0, v1;
+                upk(mul2(ap[2 * g + h], fa2), v0, v1);
+                a[2 * h] = __float2uint_rz(__fmul_rn(v0, fb));       // exact integers below 2^31
+                a[2 * h + 1] = __float2uint_rz(__fmul_rn(v1, fb));
+            }
+            const uint32_t t01 = __byte_perm(a[0], a[1], 0x5140), t23 = __byte_perm(a[2], a[3], 0x5140);
+            const uint32_t u01 = __byte_perm(a[0], a[1], 0x7362), u23 = __byte_perm(a[2], a[3], 0x7362);
+            A.w[4 * g + 0] = __byte_perm(t01, t23, 0x5410);
+            A.w[4 * g + 1] = __byte_perm(t01, t23, 0x7632);
+            A.w[4 * g + 2] = __byte_perm(u01, u23, 0x5410);
+            A.w[4 * g + 3] = __byte_perm(u01, u23, 0x7632);
+        }
+    }
+}
+
+// 2m of the E2M1 codes of four quotients (bytes in element order): two conversions to E2M1 (round
+// to nearest even, saturating; the quotients are >= 0) and one byte-permute lookup.
+__device__ __forceinline__ uint32_t mags4_fp4(u64 y01, u64 y23) {
+    float y0, y1, y2, y3;
+    upk(y01, y0, y1);
+    upk(y23, y2, y3);
+    uint32_t m;
+    asm("{ .reg .b8 c0, c1; .reg .b16 h; .reg .b32 s;\n"
+        "  cvt.rn.satfinite.e2m1x2.f32 c0, %2, %1;\n"
+        "  cvt.rn.satfinite.e2m1x2.f32 c1, %4, %3;\n"
+        "  mov.b16 h, {c0, c1};\n"
+        "  cvt.u32.u16 s, h;\n"
+        "  prmt.b32 %0, %5, %6, s; }"
+        : "=r"(m) : "f"(y0), "f"(y1), "f"(y2), "f"(y3), "r"(kLutE2M1Lo), "r"(kLutE2M1Hi));
+    return m;
+}
+
+// 2|n| of the INT4 codes of four quotients y >= 0: n = min(rint(RN(y RN(7/6))), 7), each step a
+// separate binary32 rounding (scalar intrinsics are never contracted); adding 1.5 2^23 rounds to
+// an integer (ties to even) that sits in the low mantissa bits.
+__device__ __forceinline__ uint32_t mags4_int4(u64 y01, u64 y23, float K76) {
+    float y[4];
+    upk(y01, y[0], y[1]);
+    upk(y23, y[2], y[3]);
+    uint32_t t[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        t[i] = __float_as_uint(fminf(__fadd_rn(__fmul_rn(y[i], K76), kRintMagic), kRintMagic + 7.0f));
+    const uint32_t n = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
+    return (n & 0x07070707u) << 1;
+}
+
+// Exact integer sums of one candidate: Q4 = sum M^2 and the X partials (B16: one sum; binary32
+// values: one per byte plane).  q and x start at the caller's value (kMagicInt for B16).
+template <bool B16, bool INT4, int NP = 8>
+__device__ __forceinline__ void cand_sums(const u64 (&ap)[NP], const Fixed16<B16, NP>& A, float inv, float K76, uint32_t& q,
+                                          uint32_t (&x)[B16 ? 1 : 4]) {
+    const u64 inv2 = pk(inv, inv);
+#pragma unroll
+    for (int g = 0; g < NP / 2; ++g) {
+        const u64 y01 = mul2(ap[2 * g], inv2), y23 = mul2(ap[2 * g + 1], inv2);
+        const uint32_t m4 = INT4 ? mags4_int4(y01, y23, K76) : mags4_fp4(y01, y23);
+        q = __dp4a(m4, m4, q);
+        if (B16) {
+            x[0] = __dp2a_lo(A.w[2 * g], m4, x[0]);
+            x[0] = __dp2a_hi(A.w[2 * g + 1], m4, x[0]);
+        } else {
+#pragma unroll
+            for (int b = 0; b < 4; ++b) x[b] = __dp4a(A.w[4 * g + b], m4, x[b]);
+        }
+    }
+}
+
+// The fast score G~ of a candidate from its sums, and its exact value in binary64.
+template <bool B16>
+__device__ __forceinline__ float fast_G(float s4, uint32_t q, const uint32_t (&x)[B16 ? 1 : 4]) {
+    if (B16) {
+        const float q4 = __fsub_rn(__uint_as_float(q), kTwo23), xi = __fsub_rn(__uint_as_float(x[0]), kTwo23);
+        return __fmul_rn(s4, __fmaf_rn(s4, q4, -xi));
+    }
+    // X = xh + xl exactly (each below 2^24 times a power of two); t = RN(RN(s4 Q4 - xh) - xl) is
+    // within 2^-23.9 (1 + 2^-12) |t| of the exact value, since xl < 2^-12 |t| wherever it matters
+    const float xh = __fmul_rn((float)(x[3] * 256u + x[2]), 65536.0f), xl = (float)(x[1] * 256u + x[0]);
+    return __fmul_rn(s4, __fsub_rn(__fmaf_rn(s4, (float)q, -xh), xl));
+}
+struct ExactG {
+    double hi, lo;
+};
+template <bool B16>
+__device__ __forceinline__ ExactG exact_G(float s4, uint32_t q, const uint32_t (&x)[B16 ? 1 : 4]) {
+    double xi;
+    double q4;
+    if (B16) {
+        xi = (double)(x[0] - kMagicInt);
+        q4 = (double)(q - kMagicInt);
+    } else {
+        xi = (double)x[3] * 16777216.0 + (double)x[2] * 65536.0 + (double)x[1] * 256.0 + (double)x[0];
+        q4 = (double)q;
+    }
+    const double s = (double)s4;
+    const double u = __fma_rn(s, q4, -xi);   // exact: fewer than 45 significant bits
+    ExactG g;
+    g.hi = __dmul_rn(s, u);
+    g.lo = __fma_rn(s, u, -g.hi);
+    return g;
+}
+__device__ __forceinline__ bool exact_less(const ExactG& a, const ExactG& b) {
+    return a.hi < b.hi || (a.hi == b.hi && a.lo < b.lo);
+}
+
+// Candidates within 2^-20 of the smallest fast score (NaN scores, which mark patterns outside
+// 0..126, are never inside): bit c of the result.
+template <int N>
+__device__ __forceinline__ uint32_t near_min_mask(const float (&g)[N]) {
+    float m = g[0];
+#pragma unroll
+    for (int c = 1; c < N; ++c) m = fminf(m, g[c]);
+    const float thr = __fmaf_rn(fabsf(m), 0x1p-20f, m);
+    uint32_t mask = 0;
+#pragma unroll
+    for (int c = 0; c < N; ++c) mask |= (g[c] <= thr ? 1u : 0u) << c;
+    return mask;
+}
+
+// Per-block context of the searches: magnitudes, fixed point, the per-tensor table base.
+// Table entry of pattern p: {inv = RN(1/sv), e = the E4M3 value}, sv = RN(e S); patterns outside
+// 1..126 hold inv = 0 and e = NaN (pattern 0, the zero scale, holds e = 0).
+template <bool B16>
+struct BlockCtx {
+    u64 ap[8];          // |x| pairs
+    Fixed16<B16> A;
+    float T;            // S 2^(k-2): sigma4 of pattern p is RN(e(p) T) = sv(p) 2^(k-2)
+};
+
+template <bool B16>
+__device__ __forceinline__ void block_ctx(const u64 (&xp)[8], float ab, float S, BlockCtx<B16>& c) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        float a, b;
+        upk(xp[j], a, b);
+        c.ap[j] = pk(fabsf(a), fabsf(b));
+    }
+    // an element reaches a nonzero code only from |x| >= sv/4 >= 2^-11 S, so a maximum below that
+    // is raised to it (all codes are zero then, and the integers need not be exact)
+    const float aeff = fmaxf(ab, __fmul_rn(S, 0x1p-11f));
+    const int k = (B16 ? 14 : 30) - ilog2f(aeff);
+    fixed_point<B16>(c.ap, k, c.A);
+    float fa, fb;
+    pow2_split(k - 2, fa, fb);
+    c.T = __fmul_rn(__fmul_rn(S, fa), fb);
+}
+
+// Exact comparison of the candidates in `mask` (bit c = window offset c, INT4 at odd bits when
+// TWO_TYPES); the lowest index wins a tie.
+template <bool B16, bool TWO_TYPES>
+__device__ __noinline__ int exact_pick(const BlockCtx<B16>& c, const float2* t, uint32_t mask, float K76, float K67) {
+    int best = -1;
+    ExactG bg = {0.0, 0.0};
+    for (; mask; mask &= mask - 1) {
+        const int i = __ffs(mask) - 1;
+        const int off = TWO_TYPES ? i >> 1 : i;
+        const bool int4 = TWO_TYPES && (i & 1);
+        const float2 e = t[off];
+        uint32_t q = B16 ? kMagicInt : 0u, x[B16 ? 1 : 4];
+#pragma unroll
+        for (int b = 0; b < (B16 ? 1 : 4); ++b) x[b] = B16 ? kMagicInt : 0u;
+        float s4 = __fmul_rn(e.y, c.T);
+        if (int4) {
+            cand_sums<B16, true>(c.ap, c.A, e.x, K76, q, x);
+            s4 = __fmul_rn(K67, s4);
+        } else {
+            cand_sums<B16, false>(c.ap, c.A, e.x, K76, q, x);
+        }
+        const ExactG g = exact_G<B16>(s4, q, x);
+        if (best < 0 || exact_less(g, bg)) {
+            bg = g;
+            best = i;
+        }
+    }
+    return best;
+}
+
+// The window search of the NVFP4 MSE sweep (offsets LO..HI around p0, table t = base + p0) or of
+// the IF4 sweep (TWO_TYPES: FP4 and INT4 at each offset, FP4 first); returns the winning index.
+template <bool B16, bool TWO_TYPES, int NOFF>
+__device__ __forceinline__ int window_search(const BlockCtx<B16>& c, const float2* t, float K76, float K67) {
+    constexpr int N = TWO_TYPES ? 2 * NOFF : NOFF;
+    float g[N];
+#pragma unroll
+    for (int o = 0; o < NOFF; ++o) {
+        const float2 e = t[o];
+        const float s4 = __fmul_rn(e.y, c.T);
+        uint32_t q = B16 ? kMagicInt : 0u, x[B16 ? 1 : 4];
+#pragma unroll
+        for (int b = 0; b < (B16 ? 1 : 4); ++b) x[b] = B16 ? kMagicInt : 0u;
+        cand_sums<B16, false>(c.ap, c.A, e.x, K76, q, x);
+        g[TWO_TYPES ? 2 * o : o] = fast_G<B16>(s4, q, x);
+        if (TWO_TYPES) {
+            const float s4i = __fmul_rn(K67, s4);
+            q = B16 ? kMagicInt : 0u;
+#pragma unroll
+            for (int b = 0; b < (B16 ? 1 : 4); ++b) x[b] = B16 ? kMagicInt : 0u;
+            cand_sums<B16, true>(c.ap, c.A, e.x, K76, q, x);
+            g[2 * o + 1] = fast_G<B16>(s4i, q, x);
+        }
+    }
+    const uint32_t mask = near_min_mask<N>(g);
+    if ((mask & (mask - 1)) == 0) return __ffs(mask) - 1;
+    return exact_pick<B16, TWO_TYPES>(c, t, mask, K76, K67);
+}
+
+// Packed codes of a block (signed values xp) at reciprocal scale inv: 8 bytes, elements 0..15.
 __device__ __forceinline__ uint2 block_codes(const u64 (&xp)[8], float inv) {
     const u64 inv2 = pk(inv, inv);
     uint32_t c[8];
@@ -407,79 +659,53 @@ __device__ __forceinline__ uint2 block_codes(const u64 (&xp)[8], float inv) {
     return make_uint2(c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24),
                       c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24));
 }
-
-// Error of one candidate with a nonzero scale: y = RN(x inv), residuals r = RN(q - y) in units
-// of the scale, squares summed by packed fma into (even, odd) accumulators, combined once and
-// scaled by s2 = RN(sv^2).  WMSE: acc = fma(RN(w r), r, acc).
-template <bool WEIGHTED>
-__device__ __forceinline__ float sweep_error(const u64 (&xp)[8], const u64 (&wp)[8], float inv, float s2) {
+// INT4 codes of a block at reciprocal scale inv: n = clamp(rint(RN(RN(x inv) RN(7/6))), -7, 7) as
+// 4-bit two's complement nibbles (the low bits of 1.5 2^23 + n).
+__device__ __forceinline__ uint2 block_codes_int4(const u64 (&xp)[8], float inv, float K76) {
     const u64 inv2 = pk(inv, inv);
-    u64 acc = pk(0.0f, 0.0f);   // (even, odd) accumulators
-#if FP4Q_SWEEP_SCALAR_ACC
-    float ae = 0.0f, ao = 0.0f;
+    uint32_t ci[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-        float r0, r1;
-        e2m1x2_residual(mul2(xp[j], inv2), r0, r1);
-        if (WEIGHTED) {
-            float w0, w1;
-            upk(wp[j], w0, w1);
-            ae = __fmaf_rn(__fmul_rn(w0, r0), r0, ae);
-            ao = __fmaf_rn(__fmul_rn(w1, r1), r1, ao);
-        } else {
-            ae = __fmaf_rn(r0, r0, ae);
-            ao = __fmaf_rn(r1, r1, ao);
-        }
+        float y0, y1;
+        upk(mul2(xp[j], inv2), y0, y1);
+        const float t0 = fminf(fmaxf(__fadd_rn(__fmul_rn(y0, K76), kRintMagic), kRintMagic - 7.0f), kRintMagic + 7.0f);
+        const float t1 = fminf(fmaxf(__fadd_rn(__fmul_rn(y1, K76), kRintMagic), kRintMagic - 7.0f), kRintMagic + 7.0f);
+        ci[j] = (__float_as_uint(t0) & 0xFu) | ((__float_as_uint(t1) & 0xFu) << 4);
     }
-    return __fmul_rn(s2, __fadd_rn(ae, ao));
-#else
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const u64 r = e2m1x2_residual2(mul2(xp[j], inv2));
-        acc = WEIGHTED ? fma2(mul2(wp[j], r), r, acc) : fma2(r, r, acc);
-    }
-    float a, b;
-    upk(acc, a, b);
-    return __fmul_rn(s2, __fadd_rn(a, b));
-#endif
+    return make_uint2(ci[0] | (ci[1] << 8) | (ci[2] << 16) | (ci[3] << 24),
+                      ci[4] | (ci[5] << 8) | (ci[6] << 16) | (ci[7] << 24));
 }
 
-// Error of the zero scale (pattern 0): every code is 0, so the error is the fma sum of x^2
-// (WMSE: RN(w x) x) in the same (even, odd) order, unscaled.
-template <bool WEIGHTED>
-__device__ __forceinline__ float zero_scale_error(const u64 (&xp)[8], const u64 (&wp)[8]) {
-    u64 acc = pk(0.0f, 0.0f);
+// WMSE error of one candidate, binary32 with one accumulator in element order:
+// xhat = RN(q sv), d = RN(|x| - xhat), acc = fma(RN(w d), d, acc) (on magnitudes: RN is odd, so
+// d, RN(w d) d and the sum equal those of the signed values).
+__device__ __forceinline__ float wmse_error(const u64 (&ap)[8], const u64 (&wp)[8], float inv, float sv) {
+    const u64 inv2 = pk(inv, inv);
+    float acc = 0.0f;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc = WEIGHTED ? fma2(mul2(wp[j], xp[j]), xp[j], acc) : fma2(xp[j], xp[j], acc);
-    float a, b;
-    upk(acc, a, b);
-    return __fadd_rn(a, b);
+    for (int j = 0; j < 8; ++j) {
+        float a0, a1, w0, w1, q0, q1;
+        upk(ap[j], a0, a1);
+        upk(wp[j], w0, w1);
+        e2m1x2_decode(e2m1x2(mul2(ap[j], inv2)), q0, q1);
+        const float d0 = __fsub_rn(a0, __fmul_rn(q0, sv));
+        acc = __fmaf_rn(__fmul_rn(w0, d0), d0, acc);
+        const float d1 = __fsub_rn(a1, __fmul_rn(q1, sv));
+        acc = __fmaf_rn(__fmul_rn(w1, d1), d1, acc);
+    }
+    return acc;
 }
 
 // ------------------------------------------------------------------------------------------
 // NVFP4: AbsMax / 4-over-6 / ScaleSweep MSE [-3,+7] / ScaleSweep WMSE [-8,+7] of one block.
-// The block stays in registers for the whole candidate search.  The zero scale, which only
-// enters the window of tiny blocks, is scored before the candidate loop so the loop is
-// branch-free.  ScaleSweep (gist.science/ko/paper/2606.07618), Methodology; 4/6: Adaptive
-// Block-Scaled Data Types (gist.science/ko/paper/2603.28765), Problem.
+// The block stays in registers for the whole candidate search.  ScaleSweep
+// (gist.science/ko/paper/2606.07618), Methodology; 4/6: Adaptive Block-Scaled Data Types
+// (gist.science/ko/paper/2603.28765), Problem.
 // ------------------------------------------------------------------------------------------
-template <int OBJ, bool HAD>
-__device__ __forceinline__ void nvfp4_block(u64 (&xp)[8], const float* __restrict__ imp, int64_t colblk, float S,
-                                            float d6, float d4, const float2* tab, uint2* cdst, uint8_t* sdst) {
-    constexpr bool SWEEP = OBJ == FP4Q_SWEEP_MSE || OBJ == FP4Q_SWEEP_WMSE;
-    constexpr bool WEIGHTED = OBJ == FP4Q_SWEEP_WMSE;
-    constexpr int LO = WEIGHTED ? -8 : -3, HI = 7;
-    u64 wp[8];
-    if (HAD) fwht16(xp);
-    if (WEIGHTED) {
-        const float4* w4 = reinterpret_cast<const float4*>(imp + colblk * 16);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float4 v = __ldg(w4 + j);
-            wp[2 * j] = pk(v.x, v.y);
-            wp[2 * j + 1] = pk(v.z, v.w);
-        }
-    }
+template <int OBJ, bool B16>
+__device__ __forceinline__ void nvfp4_block(const u64 (&xp)[8], const float* __restrict__ imp, int64_t colblk,
+                                            float S, float d6, float d4, const float2* tab, uint2* cdst,
+                                            uint8_t* sdst) {
     int bp = 0;
     if (S > 0.0f) {
         const float ab = block_absmax(xp);
@@ -487,26 +713,56 @@ __device__ __forceinline__ void nvfp4_block(u64 (&xp)[8], const float* __restric
         bp = p0;
         if (OBJ == FP4Q_FOUR_OVER_SIX) {
             const int p4 = e4m3_rne(__fdiv_rn(ab, d4));   // p4 >= p0
-            if (p4 != p0) {
-                const float e0 = p0 == 0 ? zero_scale_error<false>(xp, wp) : sweep_error<false>(xp, wp, tab[p0].x, tab[p0].y);
-                const float e4 = sweep_error<false>(xp, wp, tab[p4].x, tab[p4].y);
-                if (e4 < e0) bp = p4;
+            if (p4 != p0) {   // the two scales compared exactly; a tie keeps max -> 6
+                BlockCtx<B16> c;
+                block_ctx<B16>(xp, ab, S, c);
+                ExactG g[2];
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const float2 e = tab[i ? p4 : p0];
+                    uint32_t q = B16 ? kMagicInt : 0u, x[B16 ? 1 : 4];
+#pragma unroll
+                    for (int b = 0; b < (B16 ? 1 : 4); ++b) x[b] = B16 ? kMagicInt : 0u;
+                    cand_sums<B16, false>(c.ap, c.A, e.x, 0.0f, q, x);
+                    g[i] = exact_G<B16>(__fmul_rn(e.y, c.T), q, x);
+                }
+                if (exact_less(g[1], g[0])) bp = p4;
             }
-        } else if (SWEEP) {
-            // Candidates p0 + k, k = LO .. HI, in increasing offset with strict improvement
-            // (ties keep the lowest offset).  Patterns outside 1 .. 126 score NaN and are never
-            // taken; the zero scale (pattern 0), when it is in the window, is scored first as
-            // the lowest offset.  If every error is +inf the first candidate is kept.
+        } else if (OBJ == FP4Q_SWEEP_MSE) {
+            // below 2^-11 S no element reaches a nonzero code at any candidate: every candidate
+            // ties with the zero scale (p0 is 0 there), the lowest offset
+            if (__fmul_rn(ab, 0x1p11f) >= S) {
+                BlockCtx<B16> c;
+                block_ctx<B16>(xp, ab, S, c);
+                bp = p0 - 3 + window_search<B16, false, 11>(c, tab + p0 - 3, 0.0f, 0.0f);
+            }
+        } else if (OBJ == FP4Q_SWEEP_WMSE) {
+            // candidates p0 - 8 .. p0 + 7 in increasing offset with strict improvement (ties keep
+            // the lowest offset); patterns outside 0..126 score NaN and are never taken; if every
+            // error is +inf the first candidate is kept
+            u64 wp[8], ap[8];
+            const float4* w4 = reinterpret_cast<const float4*>(imp + colblk * 16);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float4 v = __ldg(w4 + j);
+                wp[2 * j] = pk(v.x, v.y);
+                wp[2 * j + 1] = pk(v.z, v.w);
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                float a, b;
+                upk(xp[j], a, b);
+                ap[j] = pk(fabsf(a), fabsf(b));
+            }
             float best = INFINITY;
-            int kb = max(LO, -p0);
-            if (p0 + LO <= 0) best = zero_scale_error<WEIGHTED>(xp, wp);
+            int kb = max(-8, -p0);
             const float2* t = tab + p0;
-#pragma unroll(WEIGHTED ? kWmseUnroll : kMseUnroll)
-            for (int k = LO; k <= HI; ++k) {
-                const float2 c = t[k];
-                const float e = sweep_error<WEIGHTED>(xp, wp, c.x, c.y);
-                if (e < best) {
-                    best = e;
+#pragma unroll
+            for (int k = -8; k <= 7; ++k) {
+                const float2 e = t[k];
+                const float err = wmse_error(ap, wp, e.x, __fmul_rn(e.y, S));
+                if (err < best) {
+                    best = err;
                     kb = k;
                 }
             }
@@ -518,127 +774,50 @@ __device__ __forceinline__ void nvfp4_block(u64 (&xp)[8], const float* __restric
 }
 
 // ------------------------------------------------------------------------------------------
-// IF4 of one block: FP4 (E2M1) vs scaled INT4 at the shared AbsMax scale, lower error kept,
-// indicator in bit 7 of the scale byte.  Adaptive Block-Scaled Data Types
-// (gist.science/ko/paper/2603.28765), Methodology, IF4 structure and the 6/7 method.
-// Both errors are in units of the shared scale: FP4 r = RN(q - y); INT4 z = RN(y RN(7/6)),
-// n = clamp(rint(z), -7, 7), r = RN(RN(n RN(6/7)) - y).
+// IF4 of one block: FP4 (E2M1) vs scaled INT4 at the shared AbsMax scale, the lower exact block
+// error kept (a tie keeps FP4), indicator in bit 7 of the scale byte.  Adaptive Block-Scaled Data
+// Types (gist.science/ko/paper/2603.28765), Methodology, IF4 structure and the 6/7 method.
+// SWEEP: IF4 x ScaleSweep, every candidate scale of the MSE window p0 - 3 .. p0 + 7 under both
+// element types, the lowest (error, offset, FP4 before INT4) -- the IF4 page's type choice
+// searched jointly with ScaleSweep (gist.science/ko/paper/2606.07618), Methodology (MSE window).
 // ------------------------------------------------------------------------------------------
-template <bool HAD>
-__device__ __forceinline__ void if4_block(u64 (&xp)[8], float S, float d6, float K76, float K67, const float2* tab,
-                                          uint2* cdst, uint8_t* sdst) {
-    if (HAD) fwht16(xp);
-    const int p0 = S > 0.0f ? e4m3_rne(__fdiv_rn(block_absmax(xp), d6)) : 0;
-    const float inv = tab[p0].x;
-    const u64 inv2 = pk(inv, inv);
-    u64 accf = pk(0.0f, 0.0f), acci = pk(0.0f, 0.0f);
-    uint32_t cf[8], ci[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const u64 y = mul2(xp[j], inv2);
-        const u64 rf = e2m1x2_code_residual2(y, cf[j]);
-        accf = fma2(rf, rf, accf);
-        // INT4 path on scalar .rn intrinsics (no contraction): z = RN(y RN(7/6)); adding
-        // M = 1.5 * 2^23 rounds z to the nearest integer, ties to even (the sum's ulp is 1), so
-        // t = M + rint(z) exactly; clamping t to [M-7, M+7] clamps n; n = t - M is exact and the
-        // low four bits of t's encoding are n's two's-complement nibble.
-        float y0, y1;
-        upk(y, y0, y1);
-        const float t0 = fminf(fmaxf(__fadd_rn(__fmul_rn(y0, K76), kRintMagic), kRintMagic - 7.0f), kRintMagic + 7.0f);
-        const float t1 = fminf(fmaxf(__fadd_rn(__fmul_rn(y1, K76), kRintMagic), kRintMagic - 7.0f), kRintMagic + 7.0f);
-        const float n0 = __fsub_rn(t0, kRintMagic), n1 = __fsub_rn(t1, kRintMagic);
-        const u64 ri = pk(__fsub_rn(__fmul_rn(n0, K67), y0), __fsub_rn(__fmul_rn(n1, K67), y1));
-        acci = fma2(ri, ri, acci);
-        ci[j] = (__float_as_uint(t0) & 0xFu) | ((__float_as_uint(t1) & 0xFu) << 4);
-    }
-    float a, c;
-    upk(accf, a, c);
-    const float ef = __fadd_rn(a, c);
-    upk(acci, a, c);
-    const float ei = __fadd_rn(a, c);
-    const bool use_int = ei < ef;
-    const uint32_t* cc = use_int ? ci : cf;
-    *cdst = make_uint2(cc[0] | (cc[1] << 8) | (cc[2] << 16) | (cc[3] << 24),
-                       cc[4] | (cc[5] << 8) | (cc[6] << 16) | (cc[7] << 24));
-    *sdst = (uint8_t)(p0 | (use_int ? 0x80 : 0));
-}
-
-// ------------------------------------------------------------------------------------------
-// IF4 x ScaleSweep of one block: every candidate scale of the MSE window p0 - 3 .. p0 + 7 is
-// scored under both element types, error = RN(RN(sv^2) E) (E the residual sum of that type in
-// units of the scale, as above); the zero scale (when in the window) scores the fma sum of x^2
-// for both types.  Candidates in increasing offset, FP4 before INT4, strict improvement: the
-// lowest offset and then FP4 win ties.  Adaptive Block-Scaled Data Types
-// (gist.science/ko/paper/2603.28765), Methodology (IF4 per-block type choice) searched jointly
-// with ScaleSweep (gist.science/ko/paper/2606.07618), Methodology (MSE window).
-// ------------------------------------------------------------------------------------------
-// Residual sums of one block at reciprocal scale inv: FP4 into accf, scaled INT4 into acci
-// (z = RN(y RN(7/6)), n = clamp(rint(z), -7, 7), r = RN(RN(n RN(6/7)) - y)); the INT4 products
-// feeding a subtraction use the scalar .rn intrinsics, which are never contracted.
-__device__ __forceinline__ void if4_sums(const u64 (&xp)[8], float inv, float K76, float K67, float& ef, float& ei) {
-    const u64 inv2 = pk(inv, inv), k76 = pk(K76, K76);
-    u64 accf = pk(0.0f, 0.0f), acci = pk(0.0f, 0.0f);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const u64 y = mul2(xp[j], inv2);
-        const u64 rf = e2m1x2_residual2(y);
-        accf = fma2(rf, rf, accf);
-        float y0, y1, z0, z1;
-        upk(y, y0, y1);
-        upk(mul2(y, k76), z0, z1);   // feeds only the rounding, never an addition
-        const float n0 = fminf(fmaxf(rintf(z0), -7.0f), 7.0f), n1 = fminf(fmaxf(rintf(z1), -7.0f), 7.0f);
-        const u64 ri = pk(__fsub_rn(__fmul_rn(n0, K67), y0), __fsub_rn(__fmul_rn(n1, K67), y1));
-        acci = fma2(ri, ri, acci);
-    }
-    float a, b;
-    upk(accf, a, b);
-    ef = __fadd_rn(a, b);
-    upk(acci, a, b);
-    ei = __fadd_rn(a, b);
-}
-
-template <bool HAD>
-__device__ __forceinline__ void if4_sweep_block(u64 (&xp)[8], float S, float d6, float K76, float K67,
-                                                const float2* tab, uint2* cdst, uint8_t* sdst) {
-    if (HAD) fwht16(xp);
+template <bool SWEEP, bool B16>
+__device__ __forceinline__ void if4_block(const u64 (&xp)[8], float S, float d6, float K76, float K67,
+                                          const float2* tab, uint2* cdst, uint8_t* sdst) {
     int bp = 0;
     bool use_int = false;
     if (S > 0.0f) {
-        const int p0 = e4m3_rne(__fdiv_rn(block_absmax(xp), d6));
-        float best = INFINITY;
-        int kb = max(-3, -p0);   // the first candidate (FP4) if every error is +inf
-        bool ib = false;
-        if (p0 - 3 <= 0) best = zero_scale_error<false>(xp, xp);   // pattern 0: both types alike, FP4 first
-        const float2* t = tab + p0;
+        const float ab = block_absmax(xp);
+        const int p0 = e4m3_rne(__fdiv_rn(ab, d6));
+        bp = p0;
+        if (__fmul_rn(ab, 0x1p11f) >= S) {   // otherwise every candidate ties: FP4 at the lowest offset
+            BlockCtx<B16> c;
+            block_ctx<B16>(xp, ab, S, c);
+            if (SWEEP) {
+                const int i = window_search<B16, true, 11>(c, tab + p0 - 3, K76, K67);
+                bp = p0 - 3 + (i >> 1);
+                use_int = (i & 1) != 0;
+            } else {
+                const float2 e = tab[p0];
+                const float s4 = __fmul_rn(e.y, c.T);
+                uint32_t q = B16 ? kMagicInt : 0u, x[B16 ? 1 : 4];
 #pragma unroll
-        for (int k = -3; k <= 7; ++k) {
-            const float2 c = t[k];
-            float ef, ei;
-            if4_sums(xp, c.x, K76, K67, ef, ei);
-            ef = __fmul_rn(c.y, ef);   // RN(sv^2) E; NaN for the non-candidate patterns
-            ei = __fmul_rn(c.y, ei);
-            if (ef < best) { best = ef; kb = k; ib = false; }
-            if (ei < best) { best = ei; kb = k; ib = true; }
+                for (int b = 0; b < (B16 ? 1 : 4); ++b) x[b] = B16 ? kMagicInt : 0u;
+                cand_sums<B16, false>(c.ap, c.A, e.x, K76, q, x);
+                const ExactG gf = exact_G<B16>(s4, q, x);
+                q = B16 ? kMagicInt : 0u;
+#pragma unroll
+                for (int b = 0; b < (B16 ? 1 : 4); ++b) x[b] = B16 ? kMagicInt : 0u;
+                cand_sums<B16, true>(c.ap, c.A, e.x, K76, q, x);
+                const ExactG gi = exact_G<B16>(__fmul_rn(K67, s4), q, x);
+                use_int = exact_less(gi, gf);
+            }
+        } else if (SWEEP) {
+            bp = max(p0 - 3, 0);
         }
-        bp = p0 + kb;
-        use_int = ib;
     }
     const float inv = tab[bp].x;
-    if (!use_int) {
-        *cdst = block_codes(xp, inv);
-    } else {
-        uint32_t ci[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            float y0, y1;
-            upk(mul2(xp[j], pk(inv, inv)), y0, y1);
-            const int n0 = (int)fminf(fmaxf(rintf(__fmul_rn(y0, K76)), -7.0f), 7.0f);
-            const int n1 = (int)fminf(fmaxf(rintf(__fmul_rn(y1, K76)), -7.0f), 7.0f);
-            ci[j] = ((uint32_t)n0 & 0xFu) | (((uint32_t)n1 & 0xFu) << 4);
-        }
-        *cdst = make_uint2(ci[0] | (ci[1] << 8) | (ci[2] << 16) | (ci[3] << 24),
-                           ci[4] | (ci[5] << 8) | (ci[6] << 16) | (ci[7] << 24));
-    }
+    *cdst = use_int ? block_codes_int4(xp, inv, K76) : block_codes(xp, inv);
     *sdst = (uint8_t)(bp | (use_int ? 0x80 : 0));
 }
 
@@ -655,12 +834,11 @@ enum : int { KIND_IF4 = 4, KIND_IF4_SWEEP = 5 };   // kinds 0..3 are the NVFP4 o
 
 template <int KIND>
 __host__ __device__ constexpr bool q16_persistent() {
-    return KIND == KIND_IF4 || KIND == FP4Q_ABSMAX || KIND == FP4Q_FOUR_OVER_SIX ||
-           ((KIND == FP4Q_SWEEP_MSE || KIND == KIND_IF4_SWEEP) && FP4Q_SWEEP_PERSISTENT);
+    return KIND != FP4Q_SWEEP_WMSE;
 }
 template <int KIND>
 __host__ __device__ constexpr int q16_min_ctas() {   // register cap: CTAs per SM the kernel is compiled for
-    return KIND == FP4Q_SWEEP_WMSE ? 4 : (q16_persistent<KIND>() ? FP4Q_PERSIST_MIN_CTAS : FP4Q_SWEEP_MIN_CTAS);
+    return KIND == FP4Q_SWEEP_MSE || KIND == KIND_IF4_SWEEP ? 3 : (KIND == FP4Q_ABSMAX ? 5 : 4);
 }
 
 template <int IN, int KIND, bool HAD, typename IDX>
@@ -698,9 +876,11 @@ __global__ void __launch_bounds__(kThreads, q16_min_ctas<KIND>())
         unpack16<IN>(rb, xp);
         if (q16_persistent<KIND>() && IN == FP4Q_IN_BF16 && b + G < total)   // next block's loads in flight
             load_raw16<IN>(xv, block_at<IDX, false>(b + G, cols, ld, nb).xoff, rb);
-        if (KIND == KIND_IF4) if4_block<HAD>(xp, S, d6, K76, K67, tab, cdst, sdst);
-        else if (KIND == KIND_IF4_SWEEP) if4_sweep_block<HAD>(xp, S, d6, K76, K67, tab, cdst, sdst);
-        else nvfp4_block<KIND, HAD>(xp, imp, at.b, S, d6, d4, tab, cdst, sdst);
+        if (HAD) fwht16(xp);
+        constexpr bool B16 = IN == FP4Q_IN_BF16 && !HAD;   // bf16 values: 15-bit fixed point
+        if (KIND == KIND_IF4) if4_block<false, B16>(xp, S, d6, K76, K67, tab, cdst, sdst);
+        else if (KIND == KIND_IF4_SWEEP) if4_block<true, B16>(xp, S, d6, K76, K67, tab, cdst, sdst);
+        else nvfp4_block<KIND, B16>(xp, imp, at.b, S, d6, d4, tab, cdst, sdst);
     };
     if (q16_persistent<KIND>()) {
         for (; blk < total; blk += G) one_block(blk);
@@ -755,34 +935,43 @@ __device__ __forceinline__ int mx_exponent(float a, bool ocp) {
     return min(max(e, -127), 127);
 }
 
-// MX scale sweep of one 32-element block (pairs vp): the exponent among e_c - 2 .. e_c with
-// the lowest block error, e_c the ceil rule.  Error at e in units of 4^e: r = RN(q - y) with
-// y = RN(x 2^-e), q = E2M1(y), E = RN(acc_even + acc_odd) of fma(r, r, acc); candidates are
-// compared on RN(E 4^(e - e_c)) (an exact power-of-two factor) in increasing e, strict
-// improvement, so the lowest exponent wins a tie.  Exponents below -127 are not candidates.
-// Bridging the Gap ... Microscaling FP4 (gist.science/ko/paper/2509.23202), Methodology:
-// MXFP4 "Scale Fitting" of the power-of-two scale grid to the data.
-__device__ __forceinline__ int mx_sweep_exponent(const u64 (&vp)[16], int ec) {
-    int be = max(ec - 2, -127);
-    float best = INFINITY;
+// MX scale sweep of one 32-element block (pairs vp, maximum magnitude ab): the exponent among
+// e_c - 2 .. e_c (e_c the ceil rule, none below -127) with the lowest exact block error; the
+// lowest exponent wins a tie.  In the fixed point of the NVFP4 searches, sigma4 = 2^(e + k - 2) is
+// a power of two at least 2^9, so u = sigma4 Q4 - Xi is an integer below 2^41 and
+// G = sigma4 u is exact in binary64.  Bridging the Gap ... Microscaling FP4
+// (gist.science/ko/paper/2509.23202), Methodology: MXFP4 "Scale Fitting" of the power-of-two scale
+// grid to the data.
+template <bool B16>
+__device__ __forceinline__ int mx_sweep_exponent(const u64 (&vp)[16], float ab, int ec) {
+    if (ab == 0.0f) return ec;   // a zero block: every exponent ties, ec = -127 is the only one
+    u64 ap[16];
 #pragma unroll
-    for (int k = -2; k <= 0; ++k) {
-        const int e = ec + k;
-        if (e < -127) continue;
-        const float m = pow2i(-e);
-        const u64 m2 = pk(m, m);
-        u64 acc = pk(0.0f, 0.0f);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const u64 r = e2m1x2_residual2(mul2(vp[j], m2));
-            acc = fma2(r, r, acc);
-        }
+    for (int j = 0; j < 16; ++j) {
         float a, b;
-        upk(acc, a, b);
-        const float err = __fmul_rn(__fadd_rn(a, b), k == -2 ? 0.0625f : (k == -1 ? 0.25f : 1.0f));
-        if (err < best) {
-            best = err;
+        upk(vp[j], a, b);
+        ap[j] = pk(fabsf(a), fabsf(b));
+    }
+    const int k = (B16 ? 14 : 30) - ilog2f(ab);
+    Fixed16<B16, 16> A;
+    fixed_point<B16, 16>(ap, k, A);
+    int be = max(ec - 2, -127);
+    double best = 0.0;
+    bool first = true;
+#pragma unroll
+    for (int d = -2; d <= 0; ++d) {
+        const int e = ec + d;
+        if (e < -127) continue;
+        uint32_t q = 0u, x[B16 ? 1 : 4] = {};
+        cand_sums<B16, false, 16>(ap, A, pow2i(-e), 0.0f, q, x);
+        const double xi = B16 ? (double)x[0]
+                              : (double)x[3] * 16777216.0 + (double)x[2] * 65536.0 + (double)x[1] * 256.0 + (double)x[0];
+        const double s4 = __longlong_as_double((long long)(1023 + e + k - 2) << 52);
+        const double g = __dmul_rn(s4, __fma_rn(s4, (double)q, -xi));
+        if (first || g < best) {
+            best = g;
             be = e;
+            first = false;
         }
     }
     return be;
@@ -848,7 +1037,8 @@ __global__ void __launch_bounds__(kThreads) mxfp4_kernel(const void* __restrict_
         u64 vp[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) vp[j] = pk(v[2 * j], v[2 * j + 1]);
-        const int e = SWEEP ? mx_sweep_exponent(vp, mx_exponent(ab, false)) : mx_exponent(ab, ocp != 0);
+        const int e = SWEEP ? mx_sweep_exponent<IN == FP4Q_IN_BF16 && !HAD>(vp, ab, mx_exponent(ab, false))
+                            : mx_exponent(ab, ocp != 0);
         const float m = pow2i(-e);
         const u64 m2 = pk(m, m);
         uint32_t c[16];
@@ -906,6 +1096,7 @@ __global__ void __launch_bounds__(kThreads) dequant16_kernel(const uint8_t* __re
         const uint32_t sb = __ldg(scales + (tiled ? tiled_scale_offset<int64_t>(r, b, nb) : blk));
         const int p = sb & 0x7F;
         const float sv = p == 0 ? 0.0f : (p == 127 ? __uint_as_float(0x7FC00000u) : __fmul_rn(e4m3_value(p), S));
+        const float gi = __fmul_rn(K67, sv);   // the INT4 block scale RN(RN(6/7) sv)
         float v[16];
         const uint32_t cw[2] = {c.x, c.y};
         if (IF4 && (sb & 0x80)) {
@@ -913,7 +1104,7 @@ __global__ void __launch_bounds__(kThreads) dequant16_kernel(const uint8_t* __re
             for (int i = 0; i < 16; ++i) {
                 const int nib = (cw[i >> 3] >> ((i & 7) * 4)) & 0xF;
                 const int n = nib >= 8 ? nib - 16 : nib;
-                v[i] = __fmul_rn(__fmul_rn((float)n, K67), sv);
+                v[i] = __fmul_rn((float)n, gi);
             }
         } else {
 #pragma unroll
@@ -1151,12 +1342,23 @@ constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_addr[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device (set up on first use).
+// Device address of the scratch array on the current device.  The first call on a device looks
+// it up; later calls check that the cached address still belongs to device memory of this
+// device (a cudaDeviceReset ends the context it lived in, and the next context maps the array
+// afresh), and look it up again if not.
 int noalloc_scratch(void** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return FP4Q_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return FP4Q_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_addr[dev]) {
+        cudaPointerAttributes a;
+        if (cudaPointerGetAttributes(&a, g_noalloc_addr[dev]) != cudaSuccess || a.type != cudaMemoryTypeDevice ||
+            a.device != dev) {
+            (void)cudaGetLastError();   // the failed query leaves no error behind
+            g_noalloc_addr[dev] = nullptr;
+        }
+    }
     if (!g_noalloc_addr[dev]) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return FP4Q_ERR_CUDA;
@@ -1321,13 +1523,19 @@ int fp4q_quantize_noalloc(const void* x, int dtype, int64_t rows, int64_t cols, 
     const int B = fmt == FP4Q_MXFP4 ? 32 : 16;
     const void* aligned_stand_in = reinterpret_cast<const void*>(static_cast<uintptr_t>(256));
     int rc0 = check_common(x, dtype, rows, cols, ld, B, codes, scales, aligned_stand_in);
-    if (rc0 != FP4Q_OK || rows == 0 || cols == 0) return rc0;
+    if (rc0 != FP4Q_OK) return rc0;
+    if (device_status && (reinterpret_cast<uintptr_t>(device_status) & 3u)) return FP4Q_ERR_ALIGNMENT;
+    if (rows == 0 || cols == 0) {   // nothing to quantize: the status word still reports this call
+        if (device_status &&
+            cudaMemsetAsync(device_status, 0, sizeof(uint32_t), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+            return FP4Q_ERR_CUDA;
+        return FP4Q_OK;
+    }
     if (fmt != FP4Q_MXFP4 && !global_scale) return FP4Q_ERR_INVALID_ARG;
     if (fmt == FP4Q_NVFP4 && objective == FP4Q_SWEEP_WMSE) {
         if (!importance) return FP4Q_ERR_INVALID_ARG;
         if (!aligned16(importance)) return FP4Q_ERR_ALIGNMENT;
     }
-    if (device_status && (reinterpret_cast<uintptr_t>(device_status) & 3u)) return FP4Q_ERR_ALIGNMENT;
     void* scratch = nullptr;
     int rc = noalloc_scratch(&scratch);
     if (rc != FP4Q_OK) return rc;

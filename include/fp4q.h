@@ -235,7 +235,9 @@ int fp4q_quantize_host_async(const void* x_host, int dtype, int64_t rows, int64_
 /*
  * Dequantize codes + scales (+ S for NVFP4/IF4) into out [rows][cols], fp32 or (flag
  * FP4Q_F_OUT_BF16) bf16.  NVFP4: RN(q * RN(e(p) S)); IF4 blocks with bit 7 set:
- * RN(RN(n RN(6/7)) * RN(e(p) S)); MXFP4: RN(q * 2^(byte-127)) (byte 0xFF gives NaN).
+ * RN(n * RN(RN(6/7) * RN(e(p) S))) (the INT4 block scale with the 6/7 dequantization folded
+ * in); MXFP4: RN(q * 2^(byte-127)) (byte 0xFF gives NaN).  Each value is the binary32 rounding
+ * of the reconstruction the quantizer's objective measures.
  * inverse_hadamard: apply the normalized transform of the format's block size (32-point for
  * MXFP4, 16-point H_16 / 4 for NVFP4/IF4) to each dequantized block, as butterflies then
  * one multiplication per value (it is its own inverse up to rounding).  global_scale is a device
@@ -257,11 +259,14 @@ int fp4q_dequantize(const uint8_t* codes, const uint8_t* scales, const float* gl
  * It calls no cudaMalloc, cudaFree or other allocating routine.
  *   Arguments and results are those of fp4q_quantize, minus `workspace`.  device_status is
  *   an optional device uint32 (4-byte aligned, may be NULL); it receives the call's
- *   FP4Q_DEVSTAT_* word, copied asynchronously on `stream`.
+ *   FP4Q_DEVSTAT_* word, copied asynchronously on `stream` (FP4Q_DEVSTAT_OK for an empty
+ *   tensor, written by a 4-byte memset on `stream`).
  *   The scratch need does not grow with the tensor, so every shape fp4q_quantize accepts
  *   fits; larger tensors (2^40 elements and up) are rejected with FP4Q_ERR_SHAPE as there.
  *   The first call on a device looks up the array's address (cudaGetSymbolAddress) with
- *   that device current.  Make that first call before any stream capture.
+ *   that device current.  Make that first call before any stream capture.  Later calls check
+ *   the remembered address (cudaPointerGetAttributes) and look it up again after a
+ *   cudaDeviceReset of that device, whose new context maps the array afresh.
  *   Every call clears the scratch on `stream` before using it, and all calls on a device
  *   share it: calls that may run at the same time on the GPU (different streams, different
  *   host threads) race and must be serialized by the caller.
