@@ -71,6 +71,16 @@ def lib():
         L.fp4q_o_if4_quantize.argtypes = [P, i64, i64, i64, C.c_int, C.c_int, P, P, P, P, P, P, P]
         L.fp4q_o_mxfp4_quantize.restype = C.c_int
         L.fp4q_o_mxfp4_quantize.argtypes = [P, i64, i64, i64, C.c_int, C.c_int, C.c_int, P, P, P, P]
+        L.fp4q_o_e2m3_value.restype = C.c_double
+        L.fp4q_o_e2m3_value.argtypes = [C.c_int]
+        L.fp4q_o_e2m3_encode.restype = C.c_int
+        L.fp4q_o_e2m3_encode.argtypes = [C.c_float]
+        L.fp4q_o_global_scale_if6.restype = C.c_float
+        L.fp4q_o_global_scale_if6.argtypes = [C.c_float]
+        L.fp4q_o_if6_quantize.restype = C.c_int
+        L.fp4q_o_if6_quantize.argtypes = [P, i64, i64, i64, C.c_int, P, P, P, P, P, P, P]
+        L.fp4q_o_if6_dequantize.restype = C.c_int
+        L.fp4q_o_if6_dequantize.argtypes = [P, P, C.c_float, i64, i64, P, C.c_int]
         L.fp4q_o_f32_to_bf16.restype = None
         L.fp4q_o_f32_to_bf16.argtypes = [P, i64, P]
         L.fp4q_o_undecided.restype = C.c_long
@@ -255,6 +265,47 @@ def mx_block_errors(x, scales, hadamard=False):
     if lib().fp4q_o_mx_block_errors(_p(x), rows, cols, cols, int(hadamard), _p(scales), _p(err)) < 0:
         raise ValueError("oracle: bad shape")
     return err
+
+
+def e2m3_value(code: int) -> float:
+    return lib().fp4q_o_e2m3_value(int(code))
+
+
+def e2m3_encode(y: float) -> int:
+    return lib().fp4q_o_e2m3_encode(float(y))
+
+
+def if6_quantize(x, S=None):
+    """IF6 (FP6 E2M3 or scaled INT6 per 16-element block, indicator in bit 7 of the E4M3 scale
+    byte): packed 6-bit codes [rows, cols * 3/4], scale bytes [rows, cols/16], S = RN(amax / 1920)
+    and diagnostics (both types' exact errors, runner-up gap and exact-tie flag)."""
+    x = _f32(x)
+    rows, cols = x.shape
+    nb = cols // 16
+    codes = np.zeros((rows, cols * 3 // 4), np.uint8)
+    scales = np.zeros((rows, nb), np.uint8)
+    Sarr = np.array([0.0 if S is None else S], np.float32)
+    ef = np.zeros((rows, nb), np.float64)
+    ei = np.zeros((rows, nb), np.float64)
+    bg = np.zeros((rows, nb), np.float64)
+    bt = np.zeros((rows, nb), np.int32)
+    st = lib().fp4q_o_if6_quantize(_p(x), rows, cols, cols, int(S is not None), _p(Sarr), _p(codes), _p(scales),
+                                   _p(ef), _p(ei), _p(bg), _p(bt))
+    if st < 0:
+        raise ValueError("oracle: bad shape")
+    _decided()
+    return {"codes": codes, "scales": scales, "S": float(Sarr[0]), "status": st, "err_fp": ef, "err_int": ei,
+            "gap": bg, "tie": bt.astype(bool)}
+
+
+def if6_dequantize(codes, scales, S, out_bf16=False):
+    codes = np.ascontiguousarray(codes, np.uint8)
+    scales = np.ascontiguousarray(scales, np.uint8)
+    rows, cols = codes.shape[0], codes.shape[1] * 4 // 3
+    out = np.zeros((rows, cols), np.uint16 if out_bf16 else np.float32)
+    if lib().fp4q_o_if6_dequantize(_p(codes), _p(scales), float(S), rows, cols, _p(out), int(out_bf16)) < 0:
+        raise ValueError("oracle: bad shape")
+    return out
 
 
 def near_ties(r, threshold=1e-6):

@@ -715,6 +715,127 @@ int fp4q_o_mx_block_errors(const float* x, int64_t rows, int64_t cols, int64_t l
 }
 
 /* ------------------------------------------------------------------------------------
+ * IF6  [IF4] "Methodology", extensibility: the same per-block type choice for 6-bit elements
+ * ---------------------------------------------------------------------------------- */
+
+/* FP6 E2M3 magnitude of a 6-bit code (bit 5 = sign, ignored here): 2 exponent bits (bias 1),
+ * 3 mantissa bits; exponent 0 holds the subnormals k/8, k = 0..7; the largest value is 7.5. */
+double fp4q_o_e2m3_value(int code)
+{
+    const int e = (code >> 3) & 3, f = code & 7;
+    return e == 0 ? f / 8.0 : (1.0 + f / 8.0) * ldexp(1.0, e - 1);
+}
+
+/* Round y to the nearest E2M3 value with ties to the even code, saturating at 7.5, sign kept in
+ * bit 5: a scan over the 32 magnitudes. */
+int fp4q_o_e2m3_encode(float y)
+{
+    const int s = signbit(y) ? 0x20 : 0;
+    const double a = fabs((double)y);
+    int best = 0;
+    double bestd = a;
+    for (int c = 1; c < 32; ++c) {
+        const double d = fabs(a - fp4q_o_e2m3_value(c));
+        if (d < bestd || (d == bestd && (c & 1) == 0 && (best & 1) == 1)) { best = c; bestd = d; }
+    }
+    return s | best;
+}
+
+/* The scaled-INT6 code of x at reciprocal scale inv: n = clamp(rint(RN(RN(x*inv) * RN(62/15))), -31, 31). */
+static int int6_code(float x, float inv)
+{
+    const float K = 62.0f / 15.0f;   /* RN(31 / 7.5): the INT6 maximum 31 onto the FP6 maximum 7.5 */
+    const float y = x * inv;
+    float n = rint_even(y * K);
+    if (n > 31.0f) n = 31.0f;
+    if (n < -31.0f) n = -31.0f;
+    return (int)n;
+}
+
+/* Pack the 6-bit fields of one 16-element block into 12 bytes: element i in bits 6i .. 6i+5 of
+ * the block's little-endian 96-bit field. */
+static void pack6(const int* f, uint8_t* dst)
+{
+    memset(dst, 0, 12);
+    for (int i = 0; i < 16; ++i)
+        for (int b = 0; b < 6; ++b)
+            if ((f[i] >> b) & 1) dst[(6 * i + b) >> 3] |= (uint8_t)(1u << ((6 * i + b) & 7));
+}
+
+static int unpack6(const uint8_t* src, int i)
+{
+    int v = 0;
+    for (int b = 0; b < 6; ++b) v |= ((src[(6 * i + b) >> 3] >> ((6 * i + b) & 7)) & 1) << b;
+    return v;
+}
+
+/* S of an IF6 tensor: RN(amax / (256 * 7.5)), the FP6 maximum in place of FP4's 6. */
+float fp4q_o_global_scale_if6(float amax) { return amax / 1920.0f; }
+
+/* IF6 quantization: per 16-element block one E4M3 scale p0 = E4M3(RN(a_b / RN(7.5 S))) shared by
+ * both element types; FP6 codes E2M3(RN(x * inv)) with reconstruction q * sv, INT6 codes n with
+ * reconstruction n * RN(RN(15/62) * sv); INT6 (indicator 0x80 in the scale byte) iff its exact
+ * block error is lower.  codes: [rows][cols * 3 / 4] bytes (12 per block, pack6); FP6 fields are
+ * the E2M3 bits (sign in bit 5), INT6 fields 6-bit two's complement.  err_fp / err_int: both exact
+ * errors (double); gap / tie: the runner-up's relative gap and exact-tie flag. */
+int fp4q_o_if6_quantize(const float* x, int64_t rows, int64_t cols, int64_t ld, int scale_given, float* S_io,
+                        uint8_t* codes, uint8_t* scales, double* blk_err_fp, double* blk_err_int,
+                        double* blk_gap, int* blk_tie)
+{
+    const int B = 16;
+    if (cols % B) return -1;
+    int status = ST_OK;
+    float S;
+    if (scale_given) {
+        S = *S_io;
+        if (!isfinite(S)) status = ST_NONFINITE;
+    } else {
+        float amax;
+        status = tensor_amax(x, rows, cols, ld, &amax);
+        S = status == ST_OK ? fp4q_o_global_scale_if6(amax) : NAN;
+        *S_io = S;
+    }
+    if (status == ST_OK && !scale_range_ok(S)) status = ST_RANGE;
+    const int64_t nb = cols / B;
+    if (status != ST_OK) {
+        memset(codes, 0, (size_t)(rows * cols * 3 / 4));
+        memset(scales, 0, (size_t)(rows * nb));
+        return status;
+    }
+    const float d75 = 7.5f * S, K = 15.0f / 62.0f;   /* RN(7.5 S), RN(15/62) */
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t b = 0; b < nb; ++b) {
+            const float* xb = x + r * ld + b * B;
+            float ab = 0.0f;
+            for (int i = 0; i < B; ++i) ab = fmaxf(ab, fabsf(xb[i]));
+            const int p0 = S > 0.0f ? fp4q_o_e4m3_encode(ab / d75) : 0;
+            float sv, inv;
+            scale_pair(p0, S, &sv, &inv);
+            float mf[16], mi[16];
+            int cf[16], ci[16];
+            for (int i = 0; i < B; ++i) {
+                cf[i] = fp4q_o_e2m3_encode(xb[i] * inv);
+                mf[i] = (float)fp4q_o_e2m3_value(cf[i]);
+                const int n = int6_code(xb[i], inv);
+                mi[i] = (float)abs(n);
+                ci[i] = n & 0x3F;
+            }
+            const long double gf = (long double)sv, gi = (long double)(K * sv);
+            const exact_F ff = block_F(xb, B, mf, gf), fi = block_F(xb, B, mi, gi);
+            const int use_int = F_less(fi, ff);
+            const double ef = block_E(xb, B, mf, gf), ei = block_E(xb, B, mi, gi);
+            pack6(use_int ? ci : cf, codes + r * (cols * 3 / 4) + b * 12);
+            scales[r * nb + b] = (uint8_t)(p0 | (use_int ? 0x80 : 0));
+            if (blk_err_fp) blk_err_fp[r * nb + b] = ef;
+            if (blk_err_int) blk_err_int[r * nb + b] = ei;
+            if (blk_gap) blk_gap[r * nb + b] = rel_gap(use_int ? ei : ef, use_int ? F_diff(fi, ff) : F_diff(ff, fi));
+            if (blk_tie) blk_tie[r * nb + b] = F_equal(ff, fi);
+        }
+    }
+    return ST_OK;
+}
+
+/* ------------------------------------------------------------------------------------
  * Dequantize
  * ---------------------------------------------------------------------------------- */
 
@@ -726,6 +847,36 @@ static uint16_t f32_to_bf16(float f)
     if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x7FFFFFu)) return (uint16_t)((u >> 16) | 0x40);
     u += 0x7FFFu + ((u >> 16) & 1u);
     return (uint16_t)(u >> 16);
+}
+
+int fp4q_o_if6_dequantize(const uint8_t* codes, const uint8_t* scales, float S, int64_t rows, int64_t cols,
+                          void* out, int out_bf16)
+{
+    if (cols % 16) return -1;
+    const int64_t nb = cols / 16;
+    const float K = 15.0f / 62.0f;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t b = 0; b < nb; ++b) {
+            const uint8_t sb = scales[r * nb + b];
+            float sv, inv;
+            scale_pair(sb & 0x7F, S, &sv, &inv);
+            const uint8_t* src = codes + r * (cols * 3 / 4) + b * 12;
+            for (int i = 0; i < 16; ++i) {
+                const int f = unpack6(src, i);
+                float v;
+                if (sb & 0x80) {
+                    const int n = f >= 32 ? f - 64 : f;
+                    v = (float)n * (K * sv);
+                } else {
+                    const float m = (float)fp4q_o_e2m3_value(f);
+                    v = ((f & 0x20) ? -m : m) * sv;
+                }
+                const int64_t idx = r * cols + b * 16 + i;
+                if (out_bf16) ((uint16_t*)out)[idx] = f32_to_bf16(v);
+                else ((float*)out)[idx] = v;
+            }
+        }
+    return ST_OK;
 }
 
 /* Batch form of the bf16 rounding (for its pin). */

@@ -750,6 +750,15 @@ def test_hand_worked(row):
         assert np.array_equal(xh[0], expect)
         return
     expect_exact = _golden_value(expect_tok)
+    if method == "if6":
+        r = O.if6_quantize(_tensor_with(xb, amax=1920.0))
+        assert r["S"] == float(S)
+        assert r["scales"][0, 0] == scale
+        err = r["err_int"][0, 0] if scale & 0x80 else r["err_fp"][0, 0]
+        assert err == float(expect_exact)
+        # both IF6 rows dequantize to themselves (hw16's 31 K = 7.5 - 15 * 2^-26 rounds to 7.5)
+        assert np.array_equal(O.if6_dequantize(r["codes"], r["scales"], r["S"])[0, :16], xb)
+        return
     x = _tensor_with(xb)
     if method.startswith("if4"):
         r = O.if4_quantize(x, sweep="sweep" if method.endswith("sweep") else "absmax")
@@ -853,3 +862,91 @@ def test_if4_sweep_is_the_exact_argmin():
         e, p, t = min(keys)
         assert int(r["scales"][row, j]) == (p | (0x80 if t else 0))
         assert (r["err_int"] if t else r["err_fp"])[row, j] == float(e)
+
+
+# ---------------------------------------------------------------------------------
+# IF6: FP6 E2M3 vs scaled INT6 (Adaptive Block-Scaled Data Types, Methodology, extensibility)
+# ---------------------------------------------------------------------------------
+def e2m3_values_from_format():
+    """FP6 E2M3 magnitudes from the bit layout: 2 exponent bits (bias 1), 3 mantissa bits,
+    exponent 0 subnormal (k/8)."""
+    return [Fr(c & 7, 8) if (c >> 3) == 0 else (1 + Fr(c & 7, 8)) * Fr(2) ** ((c >> 3) - 1) for c in range(32)]
+
+
+E2M3 = e2m3_values_from_format()
+
+
+def nearest_e2m3(y: Fr) -> int:
+    a = abs(y)
+    c = min(range(32), key=lambda c: (abs(a - E2M3[c]), c & 1))
+    return c | (0x20 if y < 0 else 0)
+
+
+def test_e2m3_value_set_and_rounding():
+    assert [Fr(O.e2m3_value(c)) for c in range(32)] == E2M3
+    assert max(E2M3) == Fr(15, 2) and len(set(E2M3)) == 32
+    rng = np.random.default_rng(23)
+    ys = np.concatenate([rng.uniform(-9, 9, 3000), [float(m) for m in E2M3],
+                         [float((E2M3[c] + E2M3[c + 1]) / 2) for c in range(31)]]).astype(np.float32)
+    for y in ys:
+        assert O.e2m3_encode(float(y)) == nearest_e2m3(Fr(float(y))), float(y)
+    assert O.e2m3_encode(100.0) == 31 and O.e2m3_encode(-0.0) == 0x20
+
+
+def _exact_if6(xb, p, S):
+    s = sv_of(p, S)
+    inv = f32(1.0) / f32(s)
+    fp = [E2M3[nearest_e2m3(Fr(float(f32(v) * inv))) & 31] for v in xb]
+    K62 = f32(62.0) / f32(15.0)
+    n = [min(abs(round(Fr(float(f32(f32(v) * inv) * K62)))), 31) for v in xb]
+    g = Fr(float(f32(f32(15.0) / f32(62.0)) * f32(s)))
+    return exact_error(xb, [m * Fr(s) for m in fp]), exact_error(xb, [k * g for k in n])
+
+
+def test_if6_errors_and_choice_are_exact():
+    w = synth.make("cfg4", rows=2, cols=1024)
+    x = synth.as_f32(w)
+    O.inexact_count()
+    r = O.if6_quantize(x)
+    assert O.inexact_count() == 0
+    S = r["S"]
+    assert S == float(f32(np.abs(x).max()) / f32(1920.0))
+    rng = np.random.default_rng(29)
+    ints = 0
+    for row, j in zip(rng.integers(0, 2, 20), rng.integers(0, 64, 20)):
+        xb = x[row, j * 16:(j + 1) * 16]
+        p0 = O.e4m3_encode(float(f32(np.abs(xb).max()) / (f32(7.5) * f32(S))))
+        assert int(r["scales"][row, j]) & 0x7F == p0
+        ef, ei = _exact_if6(xb, p0, S)
+        assert r["err_fp"][row, j] == float(ef) and r["err_int"][row, j] == float(ei)
+        assert bool(r["scales"][row, j] >> 7) == (ei < ef)
+        ints += ei < ef
+    assert 0 < ints < 20
+
+
+def test_if6_packing_and_round_trip():
+    # 6-bit fields, element i at bits 6i..6i+5 of the block's 12 bytes: the dequantized values are
+    # each field decoded (FP6: the E2M3 value, sign bit 5; INT6: two's complement times the INT6
+    # scale) times the block scale, checked field by field against an independent bit reader
+    w = synth.make("cfg3", rows=4, cols=256)
+    x = synth.as_f32(w)
+    r = O.if6_quantize(x)
+    xh = O.if6_dequantize(r["codes"], r["scales"], r["S"])
+    bits = np.unpackbits(r["codes"].reshape(4, -1, 12), axis=2, bitorder="little").reshape(4, -1, 16, 6)
+    fields = (bits * (1 << np.arange(6))).sum(axis=3)
+    for row in range(4):
+        for j in range(16):
+            sb = int(r["scales"][row, j])
+            s = f32(f32(O.e4m3_value(sb & 0x7F)) * f32(r["S"]))
+            for i in range(16):
+                f = int(fields[row, j, i])
+                if sb & 0x80:
+                    n = f - 64 if f >= 32 else f
+                    want = f32(f32(n) * f32(f32(f32(15.0) / f32(62.0)) * s))
+                else:
+                    want = f32(f32(O.e2m3_value(f) * (-1 if f & 0x20 else 1)) * s)
+                assert xh[row, 16 * j + i] == want
+    # a block on the FP6 grid comes back exactly
+    xb = np.array([7.5, 0.125, 3.75, -1.875, 0.5, 6, 0.625, -0.375] + [0] * 8, np.float32)
+    r = O.if6_quantize(_tensor_with(xb, amax=1920.0))
+    assert np.array_equal(O.if6_dequantize(r["codes"], r["scales"], r["S"])[0, :16], xb)
