@@ -47,7 +47,19 @@ WORKLOADS = {
               "NVFP4 ScaleSweep-MSE on 16x16 block-Hadamard-rotated blocks, bf16 activations 8192x4096, "
               "dynamic S of the rotated tensor"),
     "cfg4h": ("cfg4", "if4_had", None, "IF4 on 16x16 block-Hadamard-rotated blocks, bf16 weight 4096x14336"),
+    # the NVFP4 operator ScaleSweep measures its overhead against: AbsMax on the same tensor
+    "cfg3_absmax": ("cfg3", "nvfp4", "absmax",
+                    "NVFP4 AbsMax (one scale per block, no search) dynamic activation quantization, bf16 8192x4096, "
+                    "the same tensor as the ScaleSweep-MSE line"),
 }
+# Dequantization (codes + scales + S -> fp32), on the quantizer's own output of the same tensors
+DEQUANT_WORKLOADS = {
+    "dq_nvfp4": ("cfg3", "nvfp4", "sweep_mse", "NVFP4 dequantize to fp32 of the 8192x4096 activation tensor's "
+                                               "ScaleSweep-MSE codes and scales"),
+    "dq_mxfp4": ("cfg5", "mxfp4", None, "MXFP4 dequantize to fp32 of the 16384x8192 activation tensor's codes and "
+                                        "E8M0 scales"),
+}
+DEQUANT_METRIC = "dequantize GB/s (fp32 out) and % of B200 HBM peak, 1 GPU"
 METRIC = "quantize GB/s (input bf16) and % of B200 HBM peak, 1 GPU, vs CPU oracle"
 # The consumer of the quantized operands (--workload gemm): the block-scaled NVFP4 GEMM on the
 # tcgen05 tensor cores, activations [M][K] (the 8192x4096 activation workload) times a weight
@@ -57,12 +69,13 @@ GEMM_MX_METRIC = "MXFP4 block-scaled GEMM TFLOP/s (tcgen05), 1 GPU"
 GEMM_WORKLOADS = ("gemm", "gemm_mx")
 GEMM_SHAPE = (8192, 14336, 4096)
 # Arithmetic the method itself needs per element for the ALU-bound searches: per candidate
-# scale one multiply (x/s), one E2M1 rounding, one subtraction (residual) and one fused
-# multiply-add (square-accumulate) -- plus, for WMSE, the weight multiply -- over 11 (MSE) or
-# 16 (WMSE) candidates, plus the block maximum and the final multiply + rounding.
+# scale one multiply (x/s), one E2M1 rounding, and the two accumulations of the exact block
+# error (sum q^2 and sum |x| q) -- for WMSE the binary32 residual, weight multiply and fused
+# square-accumulate instead -- over 11 (MSE) or 16 (WMSE) candidates, plus the block maximum and
+# the final multiply + rounding.
 ALU_OPS_PER_ELEMENT = {"sweep_mse": 11 * 4 + 3, "sweep_wmse": 16 * 5 + 3,
                        # IF4 x ScaleSweep: per candidate the FP4 four plus the INT4 pre-scale,
-                       # rounding, clamp, de-scale, residual and square-accumulate
+                       # rounding, clamp, the two accumulations and the code lookup
                        "if4_sweep": 11 * (4 + 6) + 3}
 # the 16-point rotation adds four butterfly additions and one multiplication per element
 ROTATION_OPS_PER_ELEMENT = 4 + 1
@@ -234,9 +247,12 @@ def cpu_baseline_all_cores(w, fmt, obj, budget_s=6.0, cpu_budget_s=30.0):
                       f"shards (S over each shard's rows) on {n} processes, {dt:.1f} s"}
 
 
-def cpu_baseline(w, fmt, obj, budget_s=12.0):
+def cpu_baseline(w, fmt, obj, budget_s=12.0, S=None, gpu=None):
     """The oracle as it stands, single-threaded, on whole rows of the same tensor until about
-    budget_s of CPU time has been spent; returns its throughput in the same unit."""
+    budget_s of CPU time has been spent; returns its throughput in the same unit.  With S (the
+    whole tensor's scale) and gpu = (codes, scales) of the CUDA path for the whole tensor, the
+    same oracle run also checks those rows: mismatching blocks, the near-tie statistic and the
+    reconstruction MSE of both sides (dequantized with the oracle's own decoder)."""
     import oracle as O
     x = O.widen_bf16(w["x"]) if w["dtype"] == "bf16" else w["x"]
     rows, cols = x.shape
@@ -244,26 +260,53 @@ def cpu_baseline(w, fmt, obj, budget_s=12.0):
     done, t0 = 0, time.perf_counter()
     imp = w.get("importance")
     base, had16 = split_fmt(fmt)
+    results = []
     while done < rows and time.perf_counter() - t0 < budget_s:
         xs = x[done:done + chunk]
         if base == "nvfp4":
-            O.nvfp4_quantize(xs, obj, importance=imp, hadamard16=had16)
+            r = O.nvfp4_quantize(xs, obj, importance=imp, hadamard16=had16, S=S)
         elif base == "if4":
-            O.if4_quantize(xs, hadamard16=had16, sweep="sweep" if obj == "if4_sweep" else "absmax")
+            r = O.if4_quantize(xs, hadamard16=had16, sweep="sweep" if obj == "if4_sweep" else "absmax", S=S)
         else:
-            O.mxfp4_quantize(xs, hadamard=fmt.endswith("had"), sweep="sweep" if obj == "mx_sweep" else "rule")
+            r = O.mxfp4_quantize(xs, hadamard=fmt.endswith("had"), sweep="sweep" if obj == "mx_sweep" else "rule")
+        results.append(r)
         done += xs.shape[0]
     dt = time.perf_counter() - t0
     nbytes = algorithmic_bytes(done, cols, fmt, wmse=(obj == "sweep_wmse"))
-    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{done} of {rows} rows of the {rows}x{cols} tensor ({done * cols} elements), "
-                      f"S over the sampled rows, {dt:.1f} s single-threaded"}
+    out = {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+           "sample": f"{done} of {rows} rows of the {rows}x{cols} tensor ({done * cols} elements), "
+                     f"S {'of the whole tensor' if S is not None else 'over the sampled rows'}, {dt:.1f} s single-threaded"}
+    if gpu is not None:
+        oc = np.concatenate([r["codes"] for r in results])
+        osc = np.concatenate([r["scales"] for r in results])
+        gc, gsc = gpu[0][:done], gpu[1][:done]
+        B = 32 if fmt.startswith("mxfp4") else 16
+        bad = (gsc != osc) | (gc.reshape(done, -1, B // 2) != oc.reshape(done, -1, B // 2)).any(axis=2)
+        near = O.near_ties({k: np.concatenate([r[k] for r in results]) for k in ("gap", "tie")})
+        dfmt = "mxfp4" if fmt.startswith("mxfp4") else base
+        xr = O.rotate16(x[:done]) if had16 else x[:done]
+        if fmt.startswith("mxfp4") and fmt.endswith("had"):
+            xr = np.stack([O.hadamard32(v) for v in x[:done].reshape(-1, 32)]).reshape(done, cols)
+        Sd = 0.0 if S is None else S
+        mse_o = float(np.mean((xr.astype(np.float64) - O.dequantize(oc, osc, Sd, dfmt).astype(np.float64)) ** 2))
+        mse_g = float(np.mean((xr.astype(np.float64) - O.dequantize(gc, gsc, Sd, dfmt).astype(np.float64)) ** 2))
+        out["parity"] = {"rows_checked": done, "blocks_checked": int(bad.size), "mismatching_blocks": int(bad.sum()),
+                         "bit_exact": bool(not bad.any()),
+                         "near_tie_frac": round(near["near_frac"], 6), "near_tie_blocks": near["near"],
+                         "exact_tie_blocks": near["exact"],
+                         "recon_mse": mse_g, "recon_mse_oracle": mse_o,
+                         "recon_mse_rel_diff": (abs(mse_g - mse_o) / mse_o) if mse_o > 0 else 0.0,
+                         "how": "the CUDA path's codes and scales of the sampled rows against the oracle's at the "
+                                "whole tensor's S; near ties: runner-up within 1e-6 relative of the best block error"}
+    return out
 
 
 def run_reference(args, rank, world):
     """The oracle on the host cores as the reference arm: K steps, each a bounded row sample."""
     if args.workload in GEMM_WORKLOADS:
         return run_reference_gemm(args, rank, world)
+    if args.workload in DEQUANT_WORKLOADS:
+        return run_reference_dequant(args, rank, world)
     cfg, fmt, obj, desc = WORKLOADS[args.workload]
     from fp4_block_scaled_nvfp4_b200 import synth
     import oracle as O
@@ -301,6 +344,43 @@ def run_reference(args, rank, world):
                        "step_sample_rows": sample_rows},
             "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
                              "sample": f"{sample_rows} rows per step of the {rows}x{cols} tensor"},
+            "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_reference_dequant(args, rank, world):
+    """The oracle's decoder on the host as the reference arm: each step 64 rows."""
+    cfg, fmt, obj, desc = DEQUANT_WORKLOADS[args.workload]
+    from fp4_block_scaled_nvfp4_b200 import synth
+    import oracle as O
+    if rank != 0:
+        return
+    w = synth.make(cfg)
+    rows, cols = w["rows"], w["cols"]
+    sample = 64
+    x = O.widen_bf16(w["x"][:sample * 4])
+    r = O.mxfp4_quantize(x) if fmt == "mxfp4" else O.nvfp4_quantize(x, obj)
+    S = r.get("S", 0.0)
+    B = 32 if fmt == "mxfp4" else 16
+
+    def step(i):
+        a = (i % 4) * sample
+        O.dequantize(r["codes"][a:a + sample], r["scales"][a:a + sample], S, fmt)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    dt = time.perf_counter() - t0
+    per_row = cols // 2 + cols // B + cols * 4
+    val = sample * per_row * args.steps / dt / 1e9
+    line = {"impl": "reference", "metric": DEQUANT_METRIC, "value": round(val, 4), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": desc, "rows": rows, "cols": cols, "step_sample_rows": sample},
+            "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{sample} rows per step of the {rows}x{cols} tensor"},
             "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -522,10 +602,143 @@ def run_ours(args, rank, world):
                        "overlaps the previous step's kernels and D2H (compute stream)"},
     }
     if args.cpu_baseline and world == 1:
-        # the oracle on every host core (reported), and single-threaded (nested)
-        single = cpu_baseline(w, fmt, obj, budget_s=args.cpu_seconds)
+        # the oracle on every host core (reported), and single-threaded (nested); the
+        # single-threaded run works at the whole tensor's S and checks the CUDA path's output
+        # for the rows it covers (the line's correctness fields)
+        c0, s0, g0 = outs[0]
+        S_gpu = None if fmt.startswith("mxfp4") else float(g0.cpu().numpy()[0])
+        single = cpu_baseline(w, fmt, obj, budget_s=args.cpu_seconds, S=S_gpu,
+                              gpu=(c0.cpu().numpy(), s0.cpu().numpy()))
+        line["parity"] = single.pop("parity")
+        if S_gpu is not None:
+            import oracle as O
+            xo = O.widen_bf16(w["x"]) if w["dtype"] == "bf16" else w["x"]
+            S_o = O.tensor_scale(O.rotate16(xo) if had16 else xo)[0]
+            line["parity"]["S_bit_exact"] = bool(np.float32(S_o).view(np.uint32) == np.float32(S_gpu).view(np.uint32))
         line["cpu_baseline"] = cpu_baseline_all_cores(w, fmt, obj, budget_s=args.cpu_seconds / 2)
         line["cpu_baseline"]["single_core"] = single
+    print(json.dumps(line), flush=True)
+
+
+def run_dequant(args, rank, world):
+    """Dequantization throughput: codes + scales (+ S) -> fp32, one kernel per step, on the
+    quantizer's own output for the workload's tensor, over rotating buffer sets."""
+    import torch
+    import torch.distributed as dist
+    import fp4_block_scaled_nvfp4_b200 as fq
+    from fp4_block_scaled_nvfp4_b200 import synth
+    cfg, fmt, obj, desc = DEQUANT_WORKLOADS[args.workload]
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    fq.lib()
+    w = synth.make(cfg)
+    rows, cols = w["rows"], w["cols"]
+    x = device_tensor_from_bits(w["x"], torch).to(dev)
+    codes, scales, gs = fq.quantize(x, fmt, obj or "absmax")
+    B = fq.BLOCK[fmt]
+    in_b = rows * cols // 2 + rows * cols // B + (4 if fmt != "mxfp4" else 0)
+    out_b = rows * cols * 4
+    alg = in_b + out_b
+    nsets = max(2, int(np.ceil(3.0 * L2_BYTES / alg)))
+    sets = [(codes.clone(), scales.clone(), None if gs is None else gs.clone(),
+             torch.empty((rows, cols), dtype=torch.float32, device=dev)) for _ in range(nsets)]
+    del x
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(i):
+        c, sc, g, o = sets[i % nsets]
+        fq.dequantize(c, sc, g, fmt, out=o)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(nsets):
+            step(i)
+    with torch.cuda.stream(stream):
+        graph.replay()
+    torch.cuda.synchronize()
+    cycles = max(1, args.steps // nsets)
+    steps = cycles * nsets
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            start.record()
+            for _ in range(cycles):
+                graph.replay()
+            end.record()
+        end.synchronize()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = start.elapsed_time(end) / steps
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    # end to end through the public API: codes, scales (and S) from pinned host memory, the
+    # dequantize call, the fp32 values back to pinned host memory, every step
+    hosts = [t.cpu().pin_memory() for t in (codes, scales) + ((gs,) if gs is not None else ())]
+    devs = [torch.empty_like(t, device=dev) for t in hosts]
+    out_host = torch.empty((rows, cols), dtype=torch.float32, pin_memory=True)
+    out_dev = torch.empty((rows, cols), dtype=torch.float32, device=dev)
+    e_steps = max(1, min(args.steps, 10))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record()
+        for _ in range(e_steps):
+            for h, d in zip(hosts, devs):
+                d.copy_(h, non_blocking=True)
+            fq.dequantize(devs[0], devs[1], devs[2] if gs is not None else None, fmt, out=out_dev)
+            out_host.copy_(out_dev, non_blocking=True)
+        e1.record()
+    e1.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e_steps
+    if rank != 0:
+        return
+    peak, peak_src = load_peaks()
+    achieved = alg / (ms * 1e-3) / 1e9
+    line = {"metric": DEQUANT_METRIC, "value": round(achieved * world, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": desc, "rows": rows, "cols": cols, "format": fmt, "out_dtype": "fp32",
+                       "parallelism": f"replicas{world}" if world > 1 else "single",
+                       "l2": f"{nsets} rotating buffer sets, {nsets * alg / 2**20:.0f} MB total (> 3x the 126 MB L2)",
+                       "timing": "CUDA graph over the buffer sets, replayed on one stream; CUDA events on that stream"},
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": profiled_traffic(f"{args.workload}:dequant"),
+                         "kernel": "dequant_mx_kernel" if fmt == "mxfp4" else "dequant16_kernel",
+                         "peak_source": f"{peak_src} hbm_gbs (copy, burst) from MEASURED_PEAKS.json"},
+            "kernels_ms": {"dequantize": round(ms, 5)},
+            "gpu_launches": steps, "clocks": clk.summary(),
+            "e2e": {"value": round(alg / (e2e_ms * 1e-3) / 1e9 * world, 3), "unit": "GB/s",
+                    "h2d_bytes_per_step": int(sum(h.numel() * h.element_size() for h in hosts)),
+                    "d2h_bytes_per_step": out_b, "ms_per_step": round(e2e_ms, 4), "steps": e_steps,
+                    "api": "codes, scales and S from pinned host memory, fp4q_dequantize, fp32 values back"}}
+    if args.cpu_baseline and world == 1:
+        import oracle as O
+        hc, hs = hosts[0].numpy(), hosts[1].numpy()
+        S = float(hosts[2].numpy()[0]) if gs is not None else 0.0
+        got = sets[0][3].cpu().numpy()
+        done, t0 = 0, time.perf_counter()
+        chunk = 256
+        same = True
+        while done < rows and time.perf_counter() - t0 < args.cpu_seconds:
+            ref = O.dequantize(hc[done:done + chunk], hs[done:done + chunk], S, fmt)
+            same &= bool(np.array_equal(ref.view(np.uint32), got[done:done + chunk].view(np.uint32)))
+            done += ref.shape[0]
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": round(done * cols * (alg / (rows * cols)) / dt / 1e9, 4), "unit": "GB/s",
+                                "cores": 1, "kind": "oracle",
+                                "sample": f"{done} of {rows} rows dequantized single-threaded, {dt:.1f} s"}
+        line["parity"] = {"rows_checked": done, "bit_exact": same,
+                          "how": "the CUDA path's fp32 values of the sampled rows against the oracle's decoder"}
     print(json.dumps(line), flush=True)
 
 
@@ -713,7 +926,8 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + list(GEMM_WORKLOADS), default="cfg3")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + list(GEMM_WORKLOADS) + sorted(DEQUANT_WORKLOADS),
+                    default="cfg3")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()
@@ -730,6 +944,8 @@ def main():
             run_reference(args, rank, world)
         elif args.workload in GEMM_WORKLOADS:
             run_gemm(args, rank, world)
+        elif args.workload in DEQUANT_WORKLOADS:
+            run_dequant(args, rank, world)
         else:
             run_ours(args, rank, world)
     finally:

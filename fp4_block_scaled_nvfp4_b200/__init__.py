@@ -19,16 +19,21 @@ LIB_PATH = os.path.join(_HERE, "libfp4q.so")
 OK, ERR_INVALID_ARG, ERR_SHAPE, ERR_ALIGNMENT, ERR_UNSUPPORTED, ERR_CUDA = range(6)
 DEVSTAT_OK, DEVSTAT_NONFINITE, DEVSTAT_RANGE, DEVSTAT_TIMEOUT = 0, 1, 2, 4
 IN_F32, IN_BF16 = 0, 1
-FORMATS = {"nvfp4": 0, "if4": 1, "mxfp4": 2}
+FORMATS = {"nvfp4": 0, "if4": 1, "mxfp4": 2, "if6": 3}
 OBJECTIVES = {"absmax": 0, "four_over_six": 1, "sweep_mse": 2, "sweep_wmse": 3}
 F_GLOBAL_SCALE_GIVEN, F_MX_OCP_FLOOR, F_OUT_BF16, F_HADAMARD16, F_HADAMARD32, F_MX_SWEEP, F_IF4_SWEEP = (
     0x1, 0x2, 0x4, 0x8, 0x10, 0x20, 0x40)
 F_SCALE_TILED = 0x80
-BLOCK = {"nvfp4": 16, "if4": 16, "mxfp4": 32}
+BLOCK = {"nvfp4": 16, "if4": 16, "mxfp4": 32, "if6": 16}
+
+
+def code_bytes_per_row(cols: int, fmt: str) -> int:
+    """Bytes of packed codes per row: 4-bit codes (NVFP4, IF4, MXFP4) or 6-bit fields (IF6)."""
+    return cols * 3 // 4 if fmt == "if6" else cols // 2
 
 # Names of every function include/fp4q.h declares (checked against the header by the tests).
-EXPORTS = ("fp4q_workspace_bytes", "fp4q_scale_bytes", "fp4q_nvfp4_gemm", "fp4q_mxfp4_gemm", "fp4q_encode", "fp4q_global_scale", "fp4q_hadamard_global_scale", "fp4q_quantize",
-           "fp4q_hadamard_quantize", "fp4q_dequantize", "fp4q_quantize_noalloc", "fp4q_quantize_host_async", "fp4q_read_device_status", "fp4q_last_launch_count", "fp4q_status_string")
+EXPORTS = ("fp4q_workspace_bytes", "fp4q_scale_bytes", "fp4q_nvfp4_gemm", "fp4q_mxfp4_gemm", "fp4q_gemm", "fp4q_encode", "fp4q_global_scale", "fp4q_hadamard_global_scale", "fp4q_quantize",
+           "fp4q_hadamard_quantize", "fp4q_dequantize", "fp4q_quantize_noalloc", "fp4q_quantize_host_async", "fp4q_read_device_status", "fp4q_last_launch_count", "fp4q_last_cuda_error", "fp4q_status_string")
 
 _lib = None
 
@@ -52,6 +57,8 @@ def lib():
         L.fp4q_nvfp4_gemm.restype = i32
         L.fp4q_nvfp4_gemm.argtypes = [P, P, P, P, P, P, i64, i64, i64, P, i64, P, P]
         L.fp4q_mxfp4_gemm.restype = i32
+        L.fp4q_gemm.restype = i32
+        L.fp4q_gemm.argtypes = [i32, P, P, P, P, P, P, i64, i64, i64, P, i64, u32, P, P]
         L.fp4q_encode.restype = i32
         L.fp4q_encode.argtypes = [P, i64, i32, P, P]
         L.fp4q_mxfp4_gemm.argtypes = [P, P, P, P, i64, i64, i64, P, i64, P, P]
@@ -73,6 +80,8 @@ def lib():
         L.fp4q_read_device_status.argtypes = [P, C.POINTER(C.c_uint32), P]
         L.fp4q_last_launch_count.restype = i32
         L.fp4q_last_launch_count.argtypes = []
+        L.fp4q_last_cuda_error.restype = i32
+        L.fp4q_last_cuda_error.argtypes = []
         L.fp4q_status_string.restype = C.c_char_p
         L.fp4q_status_string.argtypes = [i32]
         _lib = L
@@ -85,7 +94,8 @@ def status_string(rc: int) -> str:
 
 def _check(rc: int, what: str):
     if rc != OK:
-        raise Fp4qError(f"{what}: {status_string(rc)} ({rc})")
+        extra = f", CUDA error {lib().fp4q_last_cuda_error()}" if rc == ERR_CUDA else ""
+        raise Fp4qError(f"{what}: {status_string(rc)} ({rc}{extra})")
 
 
 def _torch():
@@ -127,7 +137,7 @@ def alloc_outputs(rows: int, cols: int, fmt: str, device="cuda", tiled: bool = F
     """(codes, scales, S) device buffers; tiled: a zero-filled 1-D scales buffer in the tiled
     layout of block-scaled GEMMs (scale_bytes(..., tiled=True) bytes)."""
     torch = _torch()
-    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=device)
+    codes = torch.empty((rows, code_bytes_per_row(cols, fmt)), dtype=torch.uint8, device=device)
     if tiled:
         scales = torch.zeros((scale_bytes(rows, cols, fmt, True),), dtype=torch.uint8, device=device)
     else:
@@ -178,7 +188,7 @@ def _check_quantize(x, fmt, objective, importance, codes, scales, gs, tiled, wor
     _dtype_code(x)
     rows, cols = x.shape
     dev = x.device
-    _need(codes, "codes", dev, (torch.uint8,), numel=rows * (cols // 2))
+    _need(codes, "codes", dev, (torch.uint8,), numel=rows * code_bytes_per_row(cols, fmt))
     _need(scales, "scales", dev, (torch.uint8,), numel=scale_bytes(rows, cols, fmt, tiled))
     if fmt != "mxfp4":
         _need(gs, "global scale", dev, (torch.float32,), min_numel=1)
@@ -220,7 +230,8 @@ def quantize(x, fmt: str = "nvfp4", objective: str = "sweep_mse", importance=Non
     if4_sweep: IF4 x ScaleSweep (scale and element type chosen together over the MSE window).
     tiled_scales: NVFP4/MXFP4 scales in the 128x4-tiled layout of block-scaled GEMMs (1-D buffer).
     """
-    fcode, ocode = _format(fmt), _objective(objective)
+    fcode = _format(fmt)
+    ocode = _objective(objective) if fmt == "nvfp4" else 0   # only NVFP4 has objectives
     if x is None or not x.is_cuda or x.dim() != 2 or x.stride(1) != 1:
         raise Fp4qError("x must be a 2-D CUDA tensor with unit column stride")
     rows, cols = x.shape
@@ -287,12 +298,13 @@ def dequantize(codes, scales, global_scale, fmt: str = "nvfp4", inverse_hadamard
     fcode = _format(fmt)
     out_dtype = out_dtype or torch.float32
     if codes is None or not codes.is_cuda or codes.dim() != 2:
-        raise Fp4qError("codes must be a 2-D CUDA tensor [rows, cols/2]")
-    rows, cols = codes.shape[0], codes.shape[1] * 2
+        raise Fp4qError("codes must be a 2-D CUDA tensor [rows, code bytes per row]")
+    rows = codes.shape[0]
+    cols = codes.shape[1] * 4 // 3 if fmt == "if6" else codes.shape[1] * 2
     dev = codes.device
-    if cols % BLOCK[fmt]:
+    if cols % BLOCK[fmt] or code_bytes_per_row(cols, fmt) != codes.shape[1]:
         raise Fp4qError(f"cols must be a multiple of {BLOCK[fmt]}")
-    _need(codes, "codes", dev, (torch.uint8,), numel=rows * (cols // 2))
+    _need(codes, "codes", dev, (torch.uint8,), numel=rows * code_bytes_per_row(cols, fmt))
     _need(scales, "scales", dev, (torch.uint8,), numel=scale_bytes(rows, cols, fmt, tiled_scales))
     if fmt != "mxfp4":
         _need(global_scale, "global_scale", dev, (torch.float32,), min_numel=1)
@@ -314,7 +326,8 @@ def quantize_noalloc(x, fmt: str = "nvfp4", objective: str = "sweep_mse", import
     """quantize() for callers that cannot allocate device memory: the library's own
     per-GPU scratch replaces the workspace (see fp4q_quantize_noalloc in include/fp4q.h).
     Outputs must be passed in `out`; device_status is an optional [1] int32 CUDA tensor."""
-    fcode, ocode = _format(fmt), _objective(objective)
+    fcode = _format(fmt)
+    ocode = _objective(objective) if fmt == "nvfp4" else 0   # only NVFP4 has objectives
     if x is None or not x.is_cuda or x.dim() != 2 or x.stride(1) != 1:
         raise Fp4qError("x must be a 2-D CUDA tensor with unit column stride")
     if out is None:
@@ -354,45 +367,48 @@ def _check_gemm_out(d, M, N, ws):
     torch = _torch()
     if not d.is_cuda or d.dim() != 2 or d.shape[0] != M or d.shape[1] != N or d.stride(1) != 1:
         raise Fp4qError(f"out must be a CUDA [{M}, {N}] tensor with unit column stride")
-    if d.dtype != torch.float32:
-        raise Fp4qError("out must be float32")
+    if d.dtype not in (torch.float32, torch.bfloat16):
+        raise Fp4qError("out must be float32 or bfloat16")
     _need(ws, "workspace", d.device, (torch.uint8,), min_numel=workspace_bytes())
 
 
-def nvfp4_gemm(a, b, out=None, workspace=None, stream=None):
+def nvfp4_gemm(a, b, out=None, workspace=None, stream=None, out_dtype=None):
     """Block-scaled NVFP4 GEMM on the tensor cores: a = (codes [M, K/2], tiled scales, S) and
     b = (codes [N, K/2], tiled scales, S) as returned by quantize(..., tiled_scales=True);
-    returns fp32 [M, N] = S_a S_b A B^T.  M, N multiples of 128, K a multiple of 256."""
+    returns [M, N] = S_a S_b A B^T in fp32, or bf16 (out_dtype=torch.bfloat16, or a bf16 out).
+    M, N multiples of 128, K a multiple of 256."""
     torch = _torch()
     ac, asc, ag = a
     bc, bsc, bg = b
     M, K, N = _check_gemm_operands(ac, asc, bc, bsc, "nvfp4")
-    d = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=ac.device)
+    d = out if out is not None else torch.empty((M, N), dtype=out_dtype or torch.float32, device=ac.device)
     ws = workspace if workspace is not None else new_workspace(ac.device)
     _need(ag, "a's S", ac.device, (torch.float32,), min_numel=1)
     _need(bg, "b's S", ac.device, (torch.float32,), min_numel=1)
     _check_gemm_out(d, M, N, ws)
-    rc = lib().fp4q_nvfp4_gemm(_ptr(ac), _ptr(asc), _ptr(ag), _ptr(bc), _ptr(bsc), _ptr(bg), M, N, K, _ptr(d),
-                               d.stride(0), _ptr(ws), _stream_ptr(stream))
-    _check(rc, "fp4q_nvfp4_gemm")
+    rc = lib().fp4q_gemm(FORMATS["nvfp4"], _ptr(ac), _ptr(asc), _ptr(ag), _ptr(bc), _ptr(bsc), _ptr(bg), M, N, K,
+                         _ptr(d), d.stride(0), F_OUT_BF16 if d.dtype == torch.bfloat16 else 0, _ptr(ws),
+                         _stream_ptr(stream))
+    _check(rc, "fp4q_gemm")
     return d
 
 
-def mxfp4_gemm(a, b, out=None, workspace=None, stream=None):
+def mxfp4_gemm(a, b, out=None, workspace=None, stream=None, out_dtype=None):
     """Block-scaled MXFP4 GEMM on the tensor cores: a = (codes [M, K/2], tiled E8M0 scales) and
     b = (codes [N, K/2], tiled E8M0 scales) as returned by quantize / hadamard_quantize(...,
     "mxfp4", tiled_scales=True) (a third element, the absent tensor scale, is ignored);
-    returns fp32 [M, N] = A B^T.  M, N multiples of 128, K a multiple of 256."""
+    returns [M, N] = A B^T in fp32, or bf16 (out_dtype=torch.bfloat16, or a bf16 out).  M, N
+    multiples of 128, K a multiple of 256."""
     torch = _torch()
     ac, asc = a[0], a[1]
     bc, bsc = b[0], b[1]
     M, K, N = _check_gemm_operands(ac, asc, bc, bsc, "mxfp4")
-    d = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=ac.device)
+    d = out if out is not None else torch.empty((M, N), dtype=out_dtype or torch.float32, device=ac.device)
     ws = workspace if workspace is not None else new_workspace(ac.device)
     _check_gemm_out(d, M, N, ws)
-    rc = lib().fp4q_mxfp4_gemm(_ptr(ac), _ptr(asc), _ptr(bc), _ptr(bsc), M, N, K, _ptr(d), d.stride(0), _ptr(ws),
-                               _stream_ptr(stream))
-    _check(rc, "fp4q_mxfp4_gemm")
+    rc = lib().fp4q_gemm(FORMATS["mxfp4"], _ptr(ac), _ptr(asc), None, _ptr(bc), _ptr(bsc), None, M, N, K, _ptr(d),
+                         d.stride(0), F_OUT_BF16 if d.dtype == torch.bfloat16 else 0, _ptr(ws), _stream_ptr(stream))
+    _check(rc, "fp4q_gemm")
     return d
 
 
@@ -433,7 +449,7 @@ def alloc_host_outputs(rows: int, cols: int, fmt: str):
     """Pinned host buffers for (codes, scales, S)."""
     torch = _torch()
     base, _ = split_fmt(fmt)
-    return (torch.empty((rows, cols // 2), dtype=torch.uint8, pin_memory=True),
+    return (torch.empty((rows, code_bytes_per_row(cols, base)), dtype=torch.uint8, pin_memory=True),
             torch.empty((rows, cols // BLOCK[base]), dtype=torch.uint8, pin_memory=True),
             torch.empty((1,), dtype=torch.float32, pin_memory=True))
 
@@ -481,7 +497,7 @@ class HostQuantizer:
         hc, hs, hg = host_out if host_out is not None else alloc_host_outputs(self.rows, self.cols, self.fmt)
         rc = lib().fp4q_quantize_host_async(
             _ptr(x_host), _dtype_code(x_host), self.rows, self.cols, FORMATS[self.base],
-            _objective(self.objective), _ptr(self.importance), _ptr(hc), _ptr(hs),
+            _objective(self.objective) if self.base == "nvfp4" else 0, _ptr(self.importance), _ptr(hc), _ptr(hs),
             _ptr(hg) if self.base != "mxfp4" else None, _ptr(st["x"]), _ptr(st["codes"]), _ptr(st["scales"]),
             _ptr(st["S"]) if self.base != "mxfp4" else None, _ptr(st["ws"]), self.flags,
             C.c_void_p(self.copy_stream.cuda_stream), C.c_void_p(self.compute_stream.cuda_stream),

@@ -95,9 +95,11 @@ __device__ __forceinline__ int64_t scale_offset(IDX blk, IDX jblocks, bool tiled
 // amax
 // ------------------------------------------------------------------------------------------
 // Combine the per-thread maxima m (magnitude bit patterns) of the CTA, fold them into the
-// workspace word, and let the last CTA write S = RN(RN(amax * post) / 1536) (NaN when any
-// element was NaN or infinite) and, when publish is set, the status word.
-__device__ __forceinline__ void amax_finish(uint32_t m, float post, uint32_t* ws, float* gscale, int publish) {
+// workspace word, and let the last CTA write S = RN(RN(amax * post) / div) (NaN when any
+// element was NaN or infinite) and, when publish is set, the status word.  div = 256 times the
+// element format's largest magnitude: 1536 for FP4 (NVFP4, IF4), 1920 for FP6 (IF6).
+__device__ __forceinline__ void amax_finish(uint32_t m, float post, uint32_t* ws, float* gscale, int publish,
+                                            float div = 1536.0f) {
     m = __reduce_max_sync(0xFFFFFFFFu, m);
     __shared__ uint32_t red[kThreads / 32];
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
@@ -112,7 +114,7 @@ __device__ __forceinline__ void amax_finish(uint32_t m, float post, uint32_t* ws
             const uint32_t bits = atomicExch(&ws[WS_AMAX], 0u);
             atomicExch(&ws[WS_CNT_AMAX], 0u);
             const float S = bits >= 0x7F800000u ? __uint_as_float(0x7FC00000u)
-                                                : __fdiv_rn(__fmul_rn(__uint_as_float(bits), post), 1536.0f);
+                                                : __fdiv_rn(__fmul_rn(__uint_as_float(bits), post), div);
             *gscale = S;
             if (publish) atomicExch(&ws[WS_STATUS], scale_flags(S));
         }
@@ -176,10 +178,10 @@ __device__ __forceinline__ uint32_t amax_partial(const void* __restrict__ xv, in
 template <int IN>
 __global__ void __launch_bounds__(kThreads, 4) amax_kernel(const void* __restrict__ xv, int64_t rows, int64_t cols,
                                                         int64_t ld, uint32_t* __restrict__ ws,
-                                                        float* __restrict__ gscale, int publish) {
+                                                        float* __restrict__ gscale, int publish, float div) {
     const uint32_t m = amax_partial<IN, 8>(xv, rows, cols, ld, (int64_t)blockIdx.x * blockDim.x + threadIdx.x,
                                            (int64_t)gridDim.x * blockDim.x);
-    amax_finish(m, 1.0f, ws, gscale, publish);
+    amax_finish(m, 1.0f, ws, gscale, publish, div);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -423,19 +425,19 @@ struct Fixed16 {
     uint32_t w[B16 ? NP : 2 * NP];
 };
 
-// ap: the block's magnitudes (pairs), k: the shift, from a block maximum a with a 2^k in
-// [2^14, 2^15) (B16) or [2^30, 2^31).
+// xp: the block's values (pairs; their magnitudes are used), k: the shift, from a block maximum a
+// with a 2^k in [2^14, 2^15) (B16) or [2^30, 2^31).
 template <bool B16, int NP = 8>
-__device__ __forceinline__ void fixed_point(const u64 (&ap)[NP], int k, Fixed16<B16, NP>& A) {
+__device__ __forceinline__ void fixed_point(const u64 (&xp)[NP], int k, Fixed16<B16, NP>& A) {
     float fa, fb;
     pow2_split(k, fa, fb);
-    const u64 fa2 = pk(fa, fa);
     if (B16) {
-        const u64 fb2 = pk(fb, fb), mg = pk(kTwo23, kTwo23);
 #pragma unroll
         for (int j = 0; j < NP; ++j) {   // RN(|x| 2^k + 2^23): the integer sits in the low mantissa bits
-            float v0, v1;
-            upk(fma2(mul2(ap[j], fa2), fb2, mg), v0, v1);
+            float x0, x1;
+            upk(xp[j], x0, x1);
+            const float v0 = __fmaf_rn(__fmul_rn(fabsf(x0), fa), fb, kTwo23);
+            const float v1 = __fmaf_rn(__fmul_rn(fabsf(x1), fa), fb, kTwo23);
             A.w[j] = __byte_perm(__float_as_uint(v0), __float_as_uint(v1), 0x5410);
         }
     } else {
@@ -445,9 +447,9 @@ __device__ __forceinline__ void fixed_point(const u64 (&ap)[NP], int k, Fixed16<
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 float v0, v1;
-                upk(mul2(ap[2 * g + h], fa2), v0, v1);
-                a[2 * h] = __float2uint_rz(__fmul_rn(v0, fb));       // exact integers below 2^31
-                a[2 * h + 1] = __float2uint_rz(__fmul_rn(v1, fb));
+                upk(xp[2 * g + h], v0, v1);
+                a[2 * h] = __float2uint_rz(__fmul_rn(__fmul_rn(fabsf(v0), fa), fb));   // exact integers below 2^31
+                a[2 * h + 1] = __float2uint_rz(__fmul_rn(__fmul_rn(fabsf(v1), fa), fb));
             }
             const uint32_t t01 = __byte_perm(a[0], a[1], 0x5140), t23 = __byte_perm(a[2], a[3], 0x5140);
             const uint32_t u01 = __byte_perm(a[0], a[1], 0x7362), u23 = __byte_perm(a[2], a[3], 0x7362);
@@ -460,23 +462,37 @@ __device__ __forceinline__ void fixed_point(const u64 (&ap)[NP], int k, Fixed16<
 }
 
 // 2m of the E2M1 codes of four quotients (bytes in element order): two conversions to E2M1 (round
-// to nearest even, saturating; the quotients are >= 0) and one byte-permute lookup.
+// to nearest even, saturating, sign in bit 3 of each code) and one byte-permute lookup of the
+// magnitude index.  ABS: the quotients are magnitudes, so the sign bits are already clear;
+// otherwise they are masked off first.
+template <bool ABS>
 __device__ __forceinline__ uint32_t mags4_fp4(u64 y01, u64 y23) {
     float y0, y1, y2, y3;
     upk(y01, y0, y1);
     upk(y23, y2, y3);
     uint32_t m;
-    asm("{ .reg .b8 c0, c1; .reg .b16 h; .reg .b32 s;\n"
-        "  cvt.rn.satfinite.e2m1x2.f32 c0, %2, %1;\n"
-        "  cvt.rn.satfinite.e2m1x2.f32 c1, %4, %3;\n"
-        "  mov.b16 h, {c0, c1};\n"
-        "  cvt.u32.u16 s, h;\n"
-        "  prmt.b32 %0, %5, %6, s; }"
-        : "=r"(m) : "f"(y0), "f"(y1), "f"(y2), "f"(y3), "r"(kLutE2M1Lo), "r"(kLutE2M1Hi));
+    if (ABS) {
+        asm("{ .reg .b8 c0, c1; .reg .b16 h; .reg .b32 s;\n"
+            "  cvt.rn.satfinite.e2m1x2.f32 c0, %2, %1;\n"
+            "  cvt.rn.satfinite.e2m1x2.f32 c1, %4, %3;\n"
+            "  mov.b16 h, {c0, c1};\n"
+            "  cvt.u32.u16 s, h;\n"
+            "  prmt.b32 %0, %5, %6, s; }"
+            : "=r"(m) : "f"(y0), "f"(y1), "f"(y2), "f"(y3), "r"(kLutE2M1Lo), "r"(kLutE2M1Hi));
+    } else {
+        asm("{ .reg .b8 c0, c1; .reg .b16 h; .reg .b32 s;\n"
+            "  cvt.rn.satfinite.e2m1x2.f32 c0, %2, %1;\n"
+            "  cvt.rn.satfinite.e2m1x2.f32 c1, %4, %3;\n"
+            "  mov.b16 h, {c0, c1};\n"
+            "  cvt.u32.u16 s, h;\n"
+            "  and.b32 s, s, 0x7777;\n"
+            "  prmt.b32 %0, %5, %6, s; }"
+            : "=r"(m) : "f"(y0), "f"(y1), "f"(y2), "f"(y3), "r"(kLutE2M1Lo), "r"(kLutE2M1Hi));
+    }
     return m;
 }
 
-// 2|n| of the INT4 codes of four quotients y >= 0: n = min(rint(RN(y RN(7/6))), 7), each step a
+// 2|n| of the INT4 codes of four quotients y: |n| = min(rint(RN(|y| RN(7/6))), 7), each step a
 // separate binary32 rounding (scalar intrinsics are never contracted); adding 1.5 2^23 rounds to
 // an integer (ties to even) that sits in the low mantissa bits.
 __device__ __forceinline__ uint32_t mags4_int4(u64 y01, u64 y23, float K76) {
@@ -486,21 +502,22 @@ __device__ __forceinline__ uint32_t mags4_int4(u64 y01, u64 y23, float K76) {
     uint32_t t[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-        t[i] = __float_as_uint(fminf(__fadd_rn(__fmul_rn(y[i], K76), kRintMagic), kRintMagic + 7.0f));
+        t[i] = __float_as_uint(fminf(__fadd_rn(__fmul_rn(fabsf(y[i]), K76), kRintMagic), kRintMagic + 7.0f));
     const uint32_t n = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
     return (n & 0x07070707u) << 1;
 }
 
 // Exact integer sums of one candidate: Q4 = sum M^2 and the X partials (B16: one sum; binary32
 // values: one per byte plane).  q and x start at the caller's value (kMagicInt for B16).
-template <bool B16, bool INT4, int NP = 8>
-__device__ __forceinline__ void cand_sums(const u64 (&ap)[NP], const Fixed16<B16, NP>& A, float inv, float K76, uint32_t& q,
+// ABS: xp holds magnitudes.
+template <bool B16, bool INT4, int NP = 8, bool ABS = false>
+__device__ __forceinline__ void cand_sums(const u64 (&xp)[NP], const Fixed16<B16, NP>& A, float inv, float K76, uint32_t& q,
                                           uint32_t (&x)[B16 ? 1 : 4]) {
     const u64 inv2 = pk(inv, inv);
 #pragma unroll
     for (int g = 0; g < NP / 2; ++g) {
-        const u64 y01 = mul2(ap[2 * g], inv2), y23 = mul2(ap[2 * g + 1], inv2);
-        const uint32_t m4 = INT4 ? mags4_int4(y01, y23, K76) : mags4_fp4(y01, y23);
+        const u64 y01 = mul2(xp[2 * g], inv2), y23 = mul2(xp[2 * g + 1], inv2);
+        const uint32_t m4 = INT4 ? mags4_int4(y01, y23, K76) : mags4_fp4<ABS>(y01, y23);
         q = __dp4a(m4, m4, q);
         if (B16) {
             x[0] = __dp2a_lo(A.w[2 * g], m4, x[0]);
@@ -550,7 +567,28 @@ __device__ __forceinline__ bool exact_less(const ExactG& a, const ExactG& b) {
 }
 
 // Candidates within 2^-20 of the smallest fast score (NaN scores, which mark patterns outside
-// 0..126, are never inside): bit c of the result.
+// 0..126, are never inside): the index of the smallest when it is the only one, else -1.  The
+// count runs on the FMA pipe: d = RN(thr - g) is >= 0 exactly when g <= thr, and
+// sat(d 2^126 + 1) is then 1; it is 0 for d <= -2^-126 and for NaN, and in between only for
+// candidates that are (barely) outside, which can only raise the count -- a count of exactly 1
+// therefore means the smallest is alone inside the margin, and the weighted sum is its index.
+template <int N>
+__device__ __forceinline__ int near_min_unique(const float (&g)[N]) {
+    float m = g[0];
+#pragma unroll
+    for (int c = 1; c < N; ++c) m = fminf(m, g[c]);
+    const float thr = __fmaf_rn(fabsf(m), 0x1p-20f, m);
+    float cnt = 0.0f, idx = 0.0f;
+#pragma unroll
+    for (int c = 0; c < N; ++c) {
+        const float st = __saturatef(__fmaf_rn(__fsub_rn(thr, g[c]), 0x1p126f, 1.0f));
+        cnt = __fadd_rn(cnt, st);
+        idx = __fmaf_rn(st, (float)c, idx);
+    }
+    return cnt == 1.0f ? (int)idx : -1;
+}
+
+// The same candidates as a bit mask (the exact decision's input).
 template <int N>
 __device__ __forceinline__ uint32_t near_min_mask(const float (&g)[N]) {
     float m = g[0];
@@ -568,7 +606,7 @@ __device__ __forceinline__ uint32_t near_min_mask(const float (&g)[N]) {
 // 1..126 hold inv = 0 and e = NaN (pattern 0, the zero scale, holds e = 0).
 template <bool B16>
 struct BlockCtx {
-    u64 ap[8];          // |x| pairs
+    u64 xp[8];          // the block's values (pairs); the searches use their magnitudes
     Fixed16<B16> A;
     float T;            // S 2^(k-2): sigma4 of pattern p is RN(e(p) T) = sv(p) 2^(k-2)
 };
@@ -576,24 +614,20 @@ struct BlockCtx {
 template <bool B16>
 __device__ __forceinline__ void block_ctx(const u64 (&xp)[8], float ab, float S, BlockCtx<B16>& c) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        float a, b;
-        upk(xp[j], a, b);
-        c.ap[j] = pk(fabsf(a), fabsf(b));
-    }
+    for (int j = 0; j < 8; ++j) c.xp[j] = xp[j];
     // an element reaches a nonzero code only from |x| >= sv/4 >= 2^-11 S, so a maximum below that
     // is raised to it (all codes are zero then, and the integers need not be exact)
     const float aeff = fmaxf(ab, __fmul_rn(S, 0x1p-11f));
     const int k = (B16 ? 14 : 30) - ilog2f(aeff);
-    fixed_point<B16>(c.ap, k, c.A);
+    fixed_point<B16>(c.xp, k, c.A);
     float fa, fb;
     pow2_split(k - 2, fa, fb);
     c.T = __fmul_rn(__fmul_rn(S, fa), fb);
 }
 
 // Exact comparison of the candidates in `mask` (bit c = window offset c, INT4 at odd bits when
-// TWO_TYPES); the lowest index wins a tie.
-template <bool B16, bool TWO_TYPES>
+// TWO_TYPES), their sums recomputed; the lowest index wins a tie.  ABS: c.xp holds magnitudes.
+template <bool B16, bool TWO_TYPES, bool ABS>
 __device__ __noinline__ int exact_pick(const BlockCtx<B16>& c, const float2* t, uint32_t mask, float K76, float K67) {
     int best = -1;
     ExactG bg = {0.0, 0.0};
@@ -607,10 +641,10 @@ __device__ __noinline__ int exact_pick(const BlockCtx<B16>& c, const float2* t, 
         for (int b = 0; b < (B16 ? 1 : 4); ++b) x[b] = B16 ? kMagicInt : 0u;
         float s4 = __fmul_rn(e.y, c.T);
         if (int4) {
-            cand_sums<B16, true>(c.ap, c.A, e.x, K76, q, x);
+            cand_sums<B16, true, 8, ABS>(c.xp, c.A, e.x, K76, q, x);
             s4 = __fmul_rn(K67, s4);
         } else {
-            cand_sums<B16, false>(c.ap, c.A, e.x, K76, q, x);
+            cand_sums<B16, false, 8, ABS>(c.xp, c.A, e.x, K76, q, x);
         }
         const ExactG g = exact_G<B16>(s4, q, x);
         if (best < 0 || exact_less(g, bg)) {
@@ -621,10 +655,15 @@ __device__ __noinline__ int exact_pick(const BlockCtx<B16>& c, const float2* t, 
     return best;
 }
 
-// The window search of the NVFP4 MSE sweep (offsets LO..HI around p0, table t = base + p0) or of
-// the IF4 sweep (TWO_TYPES: FP4 and INT4 at each offset, FP4 first); returns the winning index.
-template <bool B16, bool TWO_TYPES, int NOFF>
-__device__ __forceinline__ int window_search(const BlockCtx<B16>& c, const float2* t, float K76, float K67) {
+// The window search of the NVFP4 MSE sweep (offsets 0..NOFF-1 from table entry t = base + p0 - 3)
+// or of the IF4 sweep (TWO_TYPES: FP4 and INT4 at each offset, FP4 first); returns the winning
+// index.  SLOTS (B16 single-type only): per-thread shared memory `slot` keeps each candidate's
+// exact sums, slot[i * kThreads], which the exact decision then reads instead of recomputing.
+// ABS: c.xp holds magnitudes.
+template <bool B16, bool TWO_TYPES, int NOFF, bool SLOTS = false, bool ABS = false>
+__device__ __forceinline__ int window_search(const BlockCtx<B16>& c, const float2* t, float K76, float K67,
+                                             uint2* slot = nullptr) {
+    static_assert(!SLOTS || (B16 && !TWO_TYPES), "slots hold one 32-bit X per candidate");
     constexpr int N = TWO_TYPES ? 2 * NOFF : NOFF;
     float g[N];
 #pragma unroll
@@ -634,20 +673,38 @@ __device__ __forceinline__ int window_search(const BlockCtx<B16>& c, const float
         uint32_t q = B16 ? kMagicInt : 0u, x[B16 ? 1 : 4];
 #pragma unroll
         for (int b = 0; b < (B16 ? 1 : 4); ++b) x[b] = B16 ? kMagicInt : 0u;
-        cand_sums<B16, false>(c.ap, c.A, e.x, K76, q, x);
+        cand_sums<B16, false, 8, ABS>(c.xp, c.A, e.x, K76, q, x);
         g[TWO_TYPES ? 2 * o : o] = fast_G<B16>(s4, q, x);
+        if constexpr (SLOTS) slot[o * kThreads] = make_uint2(q, x[0]);
         if (TWO_TYPES) {
             const float s4i = __fmul_rn(K67, s4);
             q = B16 ? kMagicInt : 0u;
 #pragma unroll
             for (int b = 0; b < (B16 ? 1 : 4); ++b) x[b] = B16 ? kMagicInt : 0u;
-            cand_sums<B16, true>(c.ap, c.A, e.x, K76, q, x);
+            cand_sums<B16, true, 8, ABS>(c.xp, c.A, e.x, K76, q, x);
             g[2 * o + 1] = fast_G<B16>(s4i, q, x);
         }
     }
-    const uint32_t mask = near_min_mask<N>(g);
-    if ((mask & (mask - 1)) == 0) return __ffs(mask) - 1;
-    return exact_pick<B16, TWO_TYPES>(c, t, mask, K76, K67);
+    const int unique = near_min_unique<N>(g);
+    if (unique >= 0) return unique;
+    uint32_t mask = near_min_mask<N>(g);
+    if constexpr (SLOTS) {
+        int best = -1;
+        ExactG bg = {0.0, 0.0};
+        for (; mask; mask &= mask - 1) {
+            const int i = __ffs(mask) - 1;
+            const uint2 qx = slot[i * kThreads];
+            const uint32_t x1[1] = {qx.y};
+            const ExactG eg = exact_G<true>(__fmul_rn(t[i].y, c.T), qx.x, x1);
+            if (best < 0 || exact_less(eg, bg)) {
+                bg = eg;
+                best = i;
+            }
+        }
+        return best;
+    } else {
+        return exact_pick<B16, TWO_TYPES, ABS>(c, t, mask, K76, K67);
+    }
 }
 
 // Packed codes of a block (signed values xp) at reciprocal scale inv: 8 bytes, elements 0..15.
@@ -702,10 +759,13 @@ __device__ __forceinline__ float wmse_error(const u64 (&ap)[8], const u64 (&wp)[
 // (gist.science/ko/paper/2606.07618), Methodology; 4/6: Adaptive Block-Scaled Data Types
 // (gist.science/ko/paper/2603.28765), Problem.
 // ------------------------------------------------------------------------------------------
-template <int OBJ, bool B16>
-__device__ __forceinline__ void nvfp4_block(const u64 (&xp)[8], const float* __restrict__ imp, int64_t colblk,
-                                            float S, float d6, float d4, const float2* tab, uint2* cdst,
-                                            uint8_t* sdst) {
+// SLOTS: `slot` points at this thread's shared-memory slots for the sweep's exact sums.
+// ABS: xp holds the magnitudes and sgn the sign bits at their code positions (bit 4 i + 3).
+template <int OBJ, bool B16, bool SLOTS, bool ABS>
+__device__ __forceinline__ void nvfp4_block(const u64 (&xp)[8], uint2 sgn, const float* __restrict__ imp,
+                                            int64_t colblk, float S, float d6, float d4, const float2* tab,
+                                            uint2* cdst, uint8_t* sdst, uint2* slot) {
+    static_assert(!ABS || OBJ == FP4Q_SWEEP_MSE, "magnitude inputs serve the MSE sweep");
     int bp = 0;
     if (S > 0.0f) {
         const float ab = block_absmax(xp);
@@ -723,7 +783,7 @@ __device__ __forceinline__ void nvfp4_block(const u64 (&xp)[8], const float* __r
                     uint32_t q = B16 ? kMagicInt : 0u, x[B16 ? 1 : 4];
 #pragma unroll
                     for (int b = 0; b < (B16 ? 1 : 4); ++b) x[b] = B16 ? kMagicInt : 0u;
-                    cand_sums<B16, false>(c.ap, c.A, e.x, 0.0f, q, x);
+                    cand_sums<B16, false>(c.xp, c.A, e.x, 0.0f, q, x);
                     g[i] = exact_G<B16>(__fmul_rn(e.y, c.T), q, x);
                 }
                 if (exact_less(g[1], g[0])) bp = p4;
@@ -734,7 +794,7 @@ __device__ __forceinline__ void nvfp4_block(const u64 (&xp)[8], const float* __r
             if (__fmul_rn(ab, 0x1p11f) >= S) {
                 BlockCtx<B16> c;
                 block_ctx<B16>(xp, ab, S, c);
-                bp = p0 - 3 + window_search<B16, false, 11>(c, tab + p0 - 3, 0.0f, 0.0f);
+                bp = p0 - 3 + window_search<B16, false, 11, SLOTS && B16, ABS>(c, tab + p0 - 3, 0.0f, 0.0f, slot);
             }
         } else if (OBJ == FP4Q_SWEEP_WMSE) {
             // candidates p0 - 8 .. p0 + 7 in increasing offset with strict improvement (ties keep
@@ -769,7 +829,9 @@ __device__ __forceinline__ void nvfp4_block(const u64 (&xp)[8], const float* __r
             bp = p0 + kb;
         }
     }
-    *cdst = block_codes(xp, tab[bp].x);
+    uint2 cw = block_codes(xp, tab[bp].x);
+    if (ABS) cw = make_uint2(cw.x | sgn.x, cw.y | sgn.y);
+    *cdst = cw;
     *sdst = (uint8_t)bp;
 }
 
@@ -803,12 +865,12 @@ __device__ __forceinline__ void if4_block(const u64 (&xp)[8], float S, float d6,
                 uint32_t q = B16 ? kMagicInt : 0u, x[B16 ? 1 : 4];
 #pragma unroll
                 for (int b = 0; b < (B16 ? 1 : 4); ++b) x[b] = B16 ? kMagicInt : 0u;
-                cand_sums<B16, false>(c.ap, c.A, e.x, K76, q, x);
+                cand_sums<B16, false>(c.xp, c.A, e.x, K76, q, x);
                 const ExactG gf = exact_G<B16>(s4, q, x);
                 q = B16 ? kMagicInt : 0u;
 #pragma unroll
                 for (int b = 0; b < (B16 ? 1 : 4); ++b) x[b] = B16 ? kMagicInt : 0u;
-                cand_sums<B16, true>(c.ap, c.A, e.x, K76, q, x);
+                cand_sums<B16, true>(c.xp, c.A, e.x, K76, q, x);
                 const ExactG gi = exact_G<B16>(__fmul_rn(K67, s4), q, x);
                 use_int = exact_less(gi, gf);
             }
@@ -847,6 +909,9 @@ __global__ void __launch_bounds__(kThreads, q16_min_ctas<KIND>())
                uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, const float* __restrict__ gscale,
                uint32_t* __restrict__ ws, int tiled) {
     __shared__ float2 s_tab[kTabLen];
+    // exact sums of each thread's 11 sweep candidates (bf16 MSE sweep only), for the rare exact decision
+    constexpr bool kSlots = KIND == FP4Q_SWEEP_MSE && IN == FP4Q_IN_BF16 && !HAD;
+    __shared__ uint2 s_slot[kSlots ? 11 * kThreads : 1];
     const IDX nb = cols / 16;
     const IDX total = rows * nb;
     const IDX G = (IDX)gridDim.x * blockDim.x;
@@ -880,12 +945,170 @@ __global__ void __launch_bounds__(kThreads, q16_min_ctas<KIND>())
         constexpr bool B16 = IN == FP4Q_IN_BF16 && !HAD;   // bf16 values: 15-bit fixed point
         if (KIND == KIND_IF4) if4_block<false, B16>(xp, S, d6, K76, K67, tab, cdst, sdst);
         else if (KIND == KIND_IF4_SWEEP) if4_block<true, B16>(xp, S, d6, K76, K67, tab, cdst, sdst);
-        else nvfp4_block<KIND, B16>(xp, imp, at.b, S, d6, d4, tab, cdst, sdst);
+        else nvfp4_block<KIND, B16, kSlots, false>(xp, make_uint2(0u, 0u), imp, at.b, S, d6, d4, tab, cdst, sdst, s_slot + threadIdx.x);
     };
     if (q16_persistent<KIND>()) {
         for (; blk < total; blk += G) one_block(blk);
     } else if (blk < total) {
         one_block(blk);
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// IF6: FP6 E2M3 vs scaled INT6 per 16-element block, the IF4 idea at 6 bits.  Adaptive
+// Block-Scaled Data Types (gist.science/ko/paper/2603.28765), Methodology ("extensibility" to
+// 6-bit formats): one E4M3 scale per block, p0 = E4M3(RN(a_b / RN(7.5 S))), S = RN(amax / 1920);
+// FP6 codes E2M3(RN(x inv)) reconstructed as q sv; INT6 codes n = clamp(rint(RN(RN(x inv) RN(62/15))),
+// -31, 31) reconstructed as n RN(RN(15/62) sv); INT6 (bit 7 of the scale byte) when its exact block
+// error is lower.  Codes: 6-bit fields, element i at bits 6i..6i+5 of the block's 12 bytes.
+// The exact comparison is the NVFP4 one with M = 8m (FP6, multiples of 1/8 up to 7.5) and
+// M = |n| (INT6): for M = c m the common multiple of E - sum x^2 is a (a Q - X), a = g 2^k / (2c).
+// ------------------------------------------------------------------------------------------
+// 8m of four FP6 codes (bytes, sign bit 5 ignored): e = bits 3..4, f = bits 0..2;
+// 8m = f for e = 0, (8 + f) 2^(e-1) otherwise.
+__device__ __forceinline__ uint32_t e2m3_m8(uint32_t c) {
+    const uint32_t e = (c >> 3) & 3u, f = c & 7u;
+    return e == 0 ? f : (8u + f) << (e - 1);
+}
+
+template <bool B16>
+__device__ __forceinline__ void if6_block(const u64 (&xp)[8], float S, float d75, float K62, float K15,
+                                          const float2* tab, uint8_t* cdst, uint8_t* sdst) {
+    int p0 = 0;
+    bool use_int = false;
+    const float ab = block_absmax(xp);
+    if (S > 0.0f) p0 = e4m3_rne(__fdiv_rn(ab, d75));
+    const float2 te = tab[p0];
+    const float inv = te.x;
+    // below S/(16 * 512) every code of both types is zero: the tie keeps FP6
+    if (S > 0.0f && __fmul_rn(ab, 0x1p13f) >= S) {
+        u64 ap[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            float a, b;
+            upk(xp[j], a, b);
+            ap[j] = pk(fabsf(a), fabsf(b));
+        }
+        // A = |x| 2^k with ab 2^k in [2^15, 2^16) (bf16) or [2^31, 2^32): every element with a
+        // nonzero code of either type (|x| >= sv/16, ab <= 12 sv) is an exact integer
+        const int k = (B16 ? 15 : 31) - ilog2f(ab);
+        Fixed16<B16> A;
+        fixed_point<B16>(ap, k, A);
+        const u64 inv2 = pk(inv, inv);
+        uint32_t qf = 0, qi = 0, xf[B16 ? 1 : 4] = {}, xi[B16 ? 1 : 4] = {};
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            float y[4];
+            upk(mul2(ap[2 * g], inv2), y[0], y[1]);
+            upk(mul2(ap[2 * g + 1], inv2), y[2], y[3]);
+            uint16_t c01, c23;
+            asm("cvt.rn.satfinite.e2m3x2.f32 %0, %1, %2;" : "=h"(c01) : "f"(y[1]), "f"(y[0]));
+            asm("cvt.rn.satfinite.e2m3x2.f32 %0, %1, %2;" : "=h"(c23) : "f"(y[3]), "f"(y[2]));
+            const uint32_t mf = e2m3_m8(c01 & 0xFFu) | (e2m3_m8(c01 >> 8) << 8) | (e2m3_m8(c23 & 0xFFu) << 16) |
+                                (e2m3_m8(c23 >> 8) << 24);
+            uint32_t t[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                t[i] = __float_as_uint(fminf(__fadd_rn(__fmul_rn(y[i], K62), kRintMagic), kRintMagic + 31.0f));
+            const uint32_t mi = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410) &
+                                0x1F1F1F1Fu;
+            qf = __dp4a(mf, mf, qf);
+            qi = __dp4a(mi, mi, qi);
+            if (B16) {
+                xf[0] = __dp2a_lo(A.w[2 * g], mf, xf[0]);
+                xf[0] = __dp2a_hi(A.w[2 * g + 1], mf, xf[0]);
+                xi[0] = __dp2a_lo(A.w[2 * g], mi, xi[0]);
+                xi[0] = __dp2a_hi(A.w[2 * g + 1], mi, xi[0]);
+            } else {
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    xf[b] = __dp4a(A.w[4 * g + b], mf, xf[b]);
+                    xi[b] = __dp4a(A.w[4 * g + b], mi, xi[b]);
+                }
+            }
+        }
+        auto xsum = [](const uint32_t (&x)[B16 ? 1 : 4]) {
+            return B16 ? (double)x[0]
+                       : (double)x[3] * 16777216.0 + (double)x[2] * 65536.0 + (double)x[1] * 256.0 + (double)x[0];
+        };
+        const float sv = __fmul_rn(te.y, S), gi = __fmul_rn(K15, sv);
+        float fa, fb;
+        pow2_split(k - 4, fa, fb);   // FP6: a = sv 2^k / 16
+        const double af = (double)__fmul_rn(__fmul_rn(sv, fa), fb);
+        pow2_split(k - 1, fa, fb);   // INT6: a = RN(RN(15/62) sv) 2^k / 2
+        const double ai = (double)__fmul_rn(__fmul_rn(gi, fa), fb);
+        ExactG g6, gn;
+        const double uf = __fma_rn(af, (double)qf, -xsum(xf)), ui = __fma_rn(ai, (double)qi, -xsum(xi));
+        g6.hi = __dmul_rn(af, uf);
+        g6.lo = __fma_rn(af, uf, -g6.hi);
+        gn.hi = __dmul_rn(ai, ui);
+        gn.lo = __fma_rn(ai, ui, -gn.hi);
+        use_int = exact_less(gn, g6);
+    }
+    // codes of the chosen type from the signed values, packed 6 bits each
+    const u64 inv2 = pk(inv, inv);
+    uint32_t fld[16];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        float y0, y1;
+        upk(mul2(xp[j], inv2), y0, y1);
+        if (use_int) {
+            const float t0 = fminf(fmaxf(__fadd_rn(__fmul_rn(y0, K62), kRintMagic), kRintMagic - 31.0f), kRintMagic + 31.0f);
+            const float t1 = fminf(fmaxf(__fadd_rn(__fmul_rn(y1, K62), kRintMagic), kRintMagic - 31.0f), kRintMagic + 31.0f);
+            fld[2 * j] = __float_as_uint(t0) & 0x3Fu;
+            fld[2 * j + 1] = __float_as_uint(t1) & 0x3Fu;
+        } else {
+            uint16_t c;
+            asm("cvt.rn.satfinite.e2m3x2.f32 %0, %1, %2;" : "=h"(c) : "f"(y1), "f"(y0));
+            fld[2 * j] = c & 0x3Fu;
+            fld[2 * j + 1] = (c >> 8) & 0x3Fu;
+        }
+    }
+    uint32_t w[3] = {0u, 0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int bit = 6 * i;
+        w[bit >> 5] |= fld[i] << (bit & 31);
+        if ((bit & 31) > 26) w[(bit >> 5) + 1] |= fld[i] >> (32 - (bit & 31));
+    }
+    uint32_t* d32 = reinterpret_cast<uint32_t*>(cdst);
+    d32[0] = w[0];
+    d32[1] = w[1];
+    d32[2] = w[2];
+    *sdst = (uint8_t)(p0 | (use_int ? 0x80 : 0));
+}
+
+template <int IN>
+__global__ void __launch_bounds__(kThreads, 4)
+    if6_kernel(const void* __restrict__ xv, int64_t rows, int64_t cols, int64_t ld, uint8_t* __restrict__ codes,
+               uint8_t* __restrict__ scales, const float* __restrict__ gscale, uint32_t* __restrict__ ws) {
+    __shared__ float2 s_tab[kTabLen];
+    const int64_t nb = cols / 16;
+    const int64_t total = rows * nb;
+    const float S = *gscale;
+    const uint32_t flags = scale_flags(S);
+    if (blockIdx.x == 0 && threadIdx.x == 0) ws[WS_STATUS] = flags;
+    build_scale_table(S, s_tab);
+    const float2* tab = s_tab + kTabPad;
+    const float d75 = __fmul_rn(7.5f, S);
+    const float K62 = __fdiv_rn(62.0f, 15.0f), K15 = __fdiv_rn(15.0f, 62.0f);
+    for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < total;
+         blk += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = blk / nb, b = blk - r * nb;
+        uint8_t* cdst = codes + r * (cols * 3 / 4) + b * 12;
+        uint8_t* sdst = scales + blk;
+        if (flags) {   // data out of contract: zero-filled outputs
+            reinterpret_cast<uint32_t*>(cdst)[0] = 0u;
+            reinterpret_cast<uint32_t*>(cdst)[1] = 0u;
+            reinterpret_cast<uint32_t*>(cdst)[2] = 0u;
+            *sdst = 0;
+            continue;
+        }
+        RawBlock16<IN> rb;
+        load_raw16<IN>(xv, r * ld + b * 16, rb);
+        u64 xp[8];
+        unpack16<IN>(rb, xp);
+        if6_block<IN == FP4Q_IN_BF16>(xp, S, d75, K62, K15, tab, cdst, sdst);
     }
 }
 
@@ -963,7 +1186,7 @@ __device__ __forceinline__ int mx_sweep_exponent(const u64 (&vp)[16], float ab, 
         const int e = ec + d;
         if (e < -127) continue;
         uint32_t q = 0u, x[B16 ? 1 : 4] = {};
-        cand_sums<B16, false, 16>(ap, A, pow2i(-e), 0.0f, q, x);
+        cand_sums<B16, false, 16, true>(ap, A, pow2i(-e), 0.0f, q, x);
         const double xi = B16 ? (double)x[0]
                               : (double)x[3] * 16777216.0 + (double)x[2] * 65536.0 + (double)x[1] * 256.0 + (double)x[0];
         const double s4 = __longlong_as_double((long long)(1023 + e + k - 2) << 52);
@@ -1064,7 +1287,10 @@ __device__ __forceinline__ uint32_t bf16_bits(float f) {
 
 template <bool OUT_BF16, int N>
 __device__ __forceinline__ void store_values(void* out, int64_t off, const float (&v)[N]) {
-    if (OUT_BF16) {
+    if (OUT_BF16 && N == 4) {
+        *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(out) + off) =
+            make_uint2(bf16_bits(v[0]) | (bf16_bits(v[1]) << 16), bf16_bits(v[2 % N]) | (bf16_bits(v[3 % N]) << 16));
+    } else if (OUT_BF16) {
         uint4* p = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(out) + off);
 #pragma unroll
         for (int q = 0; q < N / 8; ++q) {
@@ -1077,6 +1303,58 @@ __device__ __forceinline__ void store_values(void* out, int64_t off, const float
         float4* p = reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + off);
 #pragma unroll
         for (int q = 0; q < N / 4; ++q) p[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    }
+}
+
+// Unrotated dequantization with one thread per 4 consecutive elements of a row: each thread reads
+// the 2 bytes of its codes and its block's scale byte and writes one 16-byte (fp32) or 8-byte
+// (bf16) store, so a warp's loads and stores each cover one contiguous stretch of memory.
+// FMT: FP4Q_NVFP4, FP4Q_IF4 (INT4 blocks: RN(n RN(RN(6/7) sv))) or FP4Q_MXFP4 (RN(q 2^e)).
+template <bool OUT_BF16, int FMT>
+__global__ void __launch_bounds__(kThreads) dequant_lin_kernel(const uint8_t* __restrict__ codes,
+                                                               const uint8_t* __restrict__ scales,
+                                                               const float* __restrict__ gscale, int64_t rows,
+                                                               int64_t cols, void* __restrict__ out, int tiled) {
+    constexpr int B = FMT == FP4Q_MXFP4 ? 32 : 16;
+    const float S = FMT == FP4Q_MXFP4 ? 0.0f : *gscale;
+    const float K67 = __fdiv_rn(6.0f, 7.0f);
+    const int64_t q4 = cols / 4, nb = cols / B;
+    const int64_t total = rows * q4;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / q4, c = (i - r * q4) * 4, b = c / B;
+        const uint32_t cw = __ldg(reinterpret_cast<const uint16_t*>(codes + r * (cols / 2) + c / 2));
+        const uint32_t sb = __ldg(scales + (tiled ? tiled_scale_offset<int64_t>(r, b, nb) : r * nb + b));
+        float v[4];
+        if (FMT == FP4Q_MXFP4) {
+            const float m = sb == 0xFFu ? __uint_as_float(0x7FC00000u) : pow2i((int)sb - 127);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float g0, g1;
+                e2m1x2_decode((cw >> (8 * h)) & 0xFFu, g0, g1);
+                v[2 * h] = __fmul_rn(g0, m);
+                v[2 * h + 1] = __fmul_rn(g1, m);
+            }
+        } else {
+            const int p = sb & 0x7F;
+            const float sv = p == 0 ? 0.0f : (p == 127 ? __uint_as_float(0x7FC00000u) : __fmul_rn(e4m3_value(p), S));
+            if (FMT == FP4Q_IF4 && (sb & 0x80)) {
+                const float gi = __fmul_rn(K67, sv);   // the INT4 block scale RN(RN(6/7) sv)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int nib = (cw >> (4 * e)) & 0xF;
+                    v[e] = __fmul_rn((float)(nib >= 8 ? nib - 16 : nib), gi);
+                }
+            } else {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    float g0, g1;
+                    e2m1x2_decode((cw >> (8 * h)) & 0xFFu, g0, g1);
+                    v[2 * h] = __fmul_rn(g0, sv);
+                    v[2 * h + 1] = __fmul_rn(g1, sv);
+                }
+            }
+        }
+        store_values<OUT_BF16>(out, r * cols + c, v);
     }
 }
 
@@ -1153,6 +1431,43 @@ __global__ void __launch_bounds__(kThreads) dequant_mx_kernel(const uint8_t* __r
     }
 }
 
+template <bool OUT_BF16>
+__global__ void __launch_bounds__(kThreads) dequant_if6_kernel(const uint8_t* __restrict__ codes,
+                                                               const uint8_t* __restrict__ scales,
+                                                               const float* __restrict__ gscale, int64_t rows,
+                                                               int64_t cols, void* __restrict__ out) {
+    const float S = *gscale;
+    const float K15 = __fdiv_rn(15.0f, 62.0f);
+    const int64_t nb = cols / 16;
+    const int64_t total = rows * nb;
+    for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < total;
+         blk += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = blk / nb, b = blk - r * nb;
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(codes + r * (cols * 3 / 4) + b * 12);
+        const uint64_t lo = (uint64_t)__ldg(src) | ((uint64_t)__ldg(src + 1) << 32);
+        const uint32_t hi = __ldg(src + 2);
+        const uint32_t sb = __ldg(scales + blk);
+        const int p = sb & 0x7F;
+        const float sv = p == 0 ? 0.0f : (p == 127 ? __uint_as_float(0x7FC00000u) : __fmul_rn(e4m3_value(p), S));
+        const float gi = __fmul_rn(K15, sv);
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int bit = 6 * i;
+            const uint32_t f = bit < 64 ? (uint32_t)((bit <= 58 ? lo >> bit : (lo >> bit) | ((uint64_t)hi << (64 - bit))) & 0x3Fu)
+                                        : (hi >> (bit - 64)) & 0x3Fu;
+            if (sb & 0x80) {
+                const int n = f >= 32 ? (int)f - 64 : (int)f;
+                v[i] = __fmul_rn((float)n, gi);
+            } else {
+                const float m = __fmul_rn((float)e2m3_m8(f), 0.125f);   // exact
+                v[i] = __fmul_rn((f & 0x20u) ? -m : m, sv);
+            }
+        }
+        store_values<OUT_BF16>(out, r * cols + b * 16, v);
+    }
+}
+
 // ------------------------------------------------------------------------------------------
 // Element codec: the hardware conversions every quantize path uses, applied element by element
 // (KIND 0: E2M1 round to nearest even, saturating, the 4-bit code with the sign in bit 3;
@@ -1225,9 +1540,13 @@ int grid_for(K kernel, int64_t work_items, int ctas_per_sm) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+thread_local int g_cuda_error = 0;
+
 int launched(int n) {
     g_launches = n;
-    return cudaGetLastError() == cudaSuccess ? FP4Q_OK : FP4Q_ERR_CUDA;
+    const cudaError_t e = cudaGetLastError();
+    g_cuda_error = (int)e;
+    return e == cudaSuccess ? FP4Q_OK : FP4Q_ERR_CUDA;
 }
 
 int check_common(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld, int B, const uint8_t* codes,
@@ -1266,13 +1585,14 @@ void launch_q16(const void* x, int64_t rows, int64_t cols, int64_t ld, const flo
 // Tensor scale pass: plain amax, or the amax of the 16-point rotated blocks.
 template <int IN>
 void launch_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, uint32_t* ws, float* gs, int publish,
-                 bool had16, cudaStream_t st) {
+                 bool had16, cudaStream_t st, float div = 1536.0f) {
     if (had16) {
         amax_had16_kernel<IN><<<grid_for(amax_had16_kernel<IN>, rows * (cols / 16), 4), kThreads, 0, st>>>(
             x, rows, cols, ld, ws, gs, publish);
     } else {
         const int64_t vecs = rows * cols * (IN == FP4Q_IN_BF16 ? 2 : 4) / 16;
-        amax_kernel<IN><<<grid_for(amax_kernel<IN>, vecs, 4), kThreads, 0, st>>>(x, rows, cols, ld, ws, gs, publish);
+        amax_kernel<IN><<<grid_for(amax_kernel<IN>, vecs, 4), kThreads, 0, st>>>(x, rows, cols, ld, ws, gs, publish,
+                                                                                  div);
     }
 }
 
@@ -1318,6 +1638,16 @@ int launch_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, int f
             mxfp4_kernel<IN, false, false><<<grid_for(mxfp4_kernel<IN, false, false>, nblk, 8), kThreads, 0, st>>>(
                 x, rows, cols, ld, codes, scales, ws, ocp, tiled);
         return launched(1);
+    }
+    if (fmt == FP4Q_IF6) {
+        int n = 0;
+        if (!(flags & FP4Q_F_GLOBAL_SCALE_GIVEN)) {
+            launch_amax<IN>(x, rows, cols, ld, ws, gs, 0, false, st, 1920.0f);
+            ++n;
+        }
+        if6_kernel<IN><<<grid_for(if6_kernel<IN>, rows * (cols / 16), 4), kThreads, 0, st>>>(x, rows, cols, ld, codes,
+                                                                                         scales, gs, ws);
+        return launched(n + 1);
     }
     const bool had16 = (flags & FP4Q_F_HADAMARD16) != 0;
     int n = 0;
@@ -1368,18 +1698,47 @@ int noalloc_scratch(void** out) {
     return FP4Q_OK;
 }
 
+template <bool OUT_BF16, bool IF4, bool HAD>
+void launch_dequant16_as(const uint8_t* codes, const uint8_t* scales, const float* gs, int64_t rows, int64_t cols,
+                         void* out, int tiled, cudaStream_t st) {
+    auto k = dequant16_kernel<OUT_BF16, IF4, HAD>;
+    k<<<grid_for(k, rows * (cols / 16), 8), kThreads, 0, st>>>(codes, scales, gs, rows, cols, out, tiled);
+}
+
+template <bool OUT_BF16, int FMT>
+void launch_dequant_lin(const uint8_t* codes, const uint8_t* scales, const float* gs, int64_t rows, int64_t cols,
+                        void* out, int tiled, cudaStream_t st) {
+    auto k = dequant_lin_kernel<OUT_BF16, FMT>;
+    k<<<grid_for(k, rows * (cols / 4), 8), kThreads, 0, st>>>(codes, scales, gs, rows, cols, out, tiled);
+}
+
 template <bool HAD>
 void launch_dequant16(const uint8_t* codes, const uint8_t* scales, const float* gs, int64_t rows, int64_t cols,
-                      bool if4, bool bf, void* out, int g, int tiled, cudaStream_t st) {
-    if (if4 && bf) dequant16_kernel<true, true, HAD><<<g, kThreads, 0, st>>>(codes, scales, gs, rows, cols, out, tiled);
-    else if (if4) dequant16_kernel<false, true, HAD><<<g, kThreads, 0, st>>>(codes, scales, gs, rows, cols, out, tiled);
-    else if (bf) dequant16_kernel<true, false, HAD><<<g, kThreads, 0, st>>>(codes, scales, gs, rows, cols, out, tiled);
-    else dequant16_kernel<false, false, HAD><<<g, kThreads, 0, st>>>(codes, scales, gs, rows, cols, out, tiled);
+                      bool if4, bool bf, void* out, int tiled, cudaStream_t st) {
+    if (!HAD) {
+        if (if4 && bf) launch_dequant_lin<true, FP4Q_IF4>(codes, scales, gs, rows, cols, out, tiled, st);
+        else if (if4) launch_dequant_lin<false, FP4Q_IF4>(codes, scales, gs, rows, cols, out, tiled, st);
+        else if (bf) launch_dequant_lin<true, FP4Q_NVFP4>(codes, scales, gs, rows, cols, out, tiled, st);
+        else launch_dequant_lin<false, FP4Q_NVFP4>(codes, scales, gs, rows, cols, out, tiled, st);
+        return;
+    }
+    if (if4 && bf) launch_dequant16_as<true, true, HAD>(codes, scales, gs, rows, cols, out, tiled, st);
+    else if (if4) launch_dequant16_as<false, true, HAD>(codes, scales, gs, rows, cols, out, tiled, st);
+    else if (bf) launch_dequant16_as<true, false, HAD>(codes, scales, gs, rows, cols, out, tiled, st);
+    else launch_dequant16_as<false, false, HAD>(codes, scales, gs, rows, cols, out, tiled, st);
+}
+
+template <bool OUT_BF16, bool HAD>
+void launch_dequant_mx(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols, void* out, int tiled,
+                       cudaStream_t st) {
+    auto k = dequant_mx_kernel<OUT_BF16, HAD>;
+    k<<<grid_for(k, rows * (cols / 32), 8), kThreads, 0, st>>>(codes, scales, rows, cols, out, tiled);
 }
 
 // Format, objective and flag checks shared by fp4q_quantize and fp4q_quantize_noalloc.
 int check_quantize_args(int fmt, int objective, uint32_t flags) {
-    if (fmt != FP4Q_NVFP4 && fmt != FP4Q_IF4 && fmt != FP4Q_MXFP4) return FP4Q_ERR_INVALID_ARG;
+    if (fmt != FP4Q_NVFP4 && fmt != FP4Q_IF4 && fmt != FP4Q_MXFP4 && fmt != FP4Q_IF6) return FP4Q_ERR_INVALID_ARG;
+    if (fmt == FP4Q_IF6 && (flags & ~(uint32_t)FP4Q_F_GLOBAL_SCALE_GIVEN)) return FP4Q_ERR_UNSUPPORTED;
     if (flags & ~(FP4Q_F_GLOBAL_SCALE_GIVEN | FP4Q_F_MX_OCP_FLOOR | FP4Q_F_HADAMARD16 | FP4Q_F_HADAMARD32 |
                   FP4Q_F_MX_SWEEP | FP4Q_F_IF4_SWEEP | FP4Q_F_SCALE_TILED))
         return FP4Q_ERR_INVALID_ARG;
@@ -1406,7 +1765,8 @@ extern "C" {
 size_t fp4q_workspace_bytes(void) { return kWorkspaceBytes; }
 
 int64_t fp4q_scale_bytes(int64_t rows, int64_t cols, int fmt, uint32_t flags) {
-    if (fmt != FP4Q_NVFP4 && fmt != FP4Q_IF4 && fmt != FP4Q_MXFP4) return -1;
+    if (fmt != FP4Q_NVFP4 && fmt != FP4Q_IF4 && fmt != FP4Q_MXFP4 && fmt != FP4Q_IF6) return -1;
+    if (fmt == FP4Q_IF6 && (flags & FP4Q_F_SCALE_TILED)) return -1;
     const int64_t B = fmt == FP4Q_MXFP4 ? 32 : 16;
     if (rows < 0 || cols < 0 || cols % B) return -1;
     if (rows > 0 && cols > 0 && rows > ((int64_t)1 << 40) / cols) return -1;
@@ -1487,7 +1847,8 @@ int fp4q_hadamard_quantize(const void* x, int dtype, int64_t rows, int64_t cols,
 int fp4q_dequantize(const uint8_t* codes, const uint8_t* scales, const float* global_scale, int64_t rows,
                     int64_t cols, int fmt, int inverse_hadamard, void* out, uint32_t flags, void* stream) {
     g_launches = 0;
-    if (fmt != FP4Q_NVFP4 && fmt != FP4Q_IF4 && fmt != FP4Q_MXFP4) return FP4Q_ERR_INVALID_ARG;
+    if (fmt != FP4Q_NVFP4 && fmt != FP4Q_IF4 && fmt != FP4Q_MXFP4 && fmt != FP4Q_IF6) return FP4Q_ERR_INVALID_ARG;
+    if (fmt == FP4Q_IF6 && (inverse_hadamard || (flags & FP4Q_F_SCALE_TILED))) return FP4Q_ERR_UNSUPPORTED;
     if (flags & ~(FP4Q_F_OUT_BF16 | FP4Q_F_SCALE_TILED)) return FP4Q_ERR_INVALID_ARG;
     if ((flags & FP4Q_F_SCALE_TILED) && fmt == FP4Q_IF4) return FP4Q_ERR_UNSUPPORTED;
     const int tiled = (flags & FP4Q_F_SCALE_TILED) ? 1 : 0;
@@ -1499,16 +1860,25 @@ int fp4q_dequantize(const uint8_t* codes, const uint8_t* scales, const float* gl
     if (!aligned16(codes) || !aligned16(out)) return FP4Q_ERR_ALIGNMENT;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const bool bf = (flags & FP4Q_F_OUT_BF16) != 0;
-    const int g = grid_for(dequant_mx_kernel<false, true>, rows * (cols / B), 8);
+    if (fmt == FP4Q_IF6) {
+        if (reinterpret_cast<uintptr_t>(codes) & 3u) return FP4Q_ERR_ALIGNMENT;
+        if (bf)
+            dequant_if6_kernel<true><<<grid_for(dequant_if6_kernel<true>, rows * (cols / 16), 8), kThreads, 0, st>>>(
+                codes, scales, global_scale, rows, cols, out);
+        else
+            dequant_if6_kernel<false><<<grid_for(dequant_if6_kernel<false>, rows * (cols / 16), 8), kThreads, 0, st>>>(
+                codes, scales, global_scale, rows, cols, out);
+        return launched(1);
+    }
     if (fmt == FP4Q_MXFP4) {
-        if (bf && inverse_hadamard) dequant_mx_kernel<true, true><<<g, kThreads, 0, st>>>(codes, scales, rows, cols, out, tiled);
-        else if (bf) dequant_mx_kernel<true, false><<<g, kThreads, 0, st>>>(codes, scales, rows, cols, out, tiled);
-        else if (inverse_hadamard) dequant_mx_kernel<false, true><<<g, kThreads, 0, st>>>(codes, scales, rows, cols, out, tiled);
-        else dequant_mx_kernel<false, false><<<g, kThreads, 0, st>>>(codes, scales, rows, cols, out, tiled);
+        if (bf && inverse_hadamard) launch_dequant_mx<true, true>(codes, scales, rows, cols, out, tiled, st);
+        else if (bf) launch_dequant_lin<true, FP4Q_MXFP4>(codes, scales, nullptr, rows, cols, out, tiled, st);
+        else if (inverse_hadamard) launch_dequant_mx<false, true>(codes, scales, rows, cols, out, tiled, st);
+        else launch_dequant_lin<false, FP4Q_MXFP4>(codes, scales, nullptr, rows, cols, out, tiled, st);
     } else if (inverse_hadamard) {
-        launch_dequant16<true>(codes, scales, global_scale, rows, cols, fmt == FP4Q_IF4, bf, out, g, tiled, st);
+        launch_dequant16<true>(codes, scales, global_scale, rows, cols, fmt == FP4Q_IF4, bf, out, tiled, st);
     } else {
-        launch_dequant16<false>(codes, scales, global_scale, rows, cols, fmt == FP4Q_IF4, bf, out, g, tiled, st);
+        launch_dequant16<false>(codes, scales, global_scale, rows, cols, fmt == FP4Q_IF4, bf, out, tiled, st);
     }
     return launched(1);
 }
@@ -1582,7 +1952,8 @@ int fp4q_quantize_host_async(const void* x_host, int dtype, int64_t rows, int64_
     if (rc != FP4Q_OK) return rc;
     const int n = g_launches;
     if (cudaEventRecord(freed, ks) != cudaSuccess) return FP4Q_ERR_CUDA;
-    if (cudaMemcpyAsync(codes_host, codes_dev, (size_t)rows * (size_t)(cols / 2), cudaMemcpyDeviceToHost, ks) !=
+    const size_t code_bytes = (size_t)rows * (size_t)(fmt == FP4Q_IF6 ? cols * 3 / 4 : cols / 2);
+    if (cudaMemcpyAsync(codes_host, codes_dev, code_bytes, cudaMemcpyDeviceToHost, ks) !=
             cudaSuccess ||
         cudaMemcpyAsync(scales_host, scales_dev, (size_t)rows * (size_t)(cols / B), cudaMemcpyDeviceToHost, ks) !=
             cudaSuccess)
@@ -1619,6 +1990,8 @@ int fp4q_read_device_status(const void* workspace, uint32_t* status, void* strea
 }
 
 int fp4q_last_launch_count(void) { return g_launches; }
+
+int fp4q_last_cuda_error(void) { return g_cuda_error; }
 
 const char* fp4q_status_string(int s) {
     switch (s) {

@@ -139,6 +139,32 @@ __device__ __forceinline__ float e4m3_value(int p) {
 __device__ __forceinline__ u64 bf16x2_to_pair(uint32_t w) {
     return pk(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
+// The magnitudes of the pair (sign bits cleared).
+__device__ __forceinline__ u64 bf16x2_to_abs_pair(uint32_t w) {
+    return pk(__uint_as_float((w & 0x7FFFu) << 16), __uint_as_float(w & 0x7FFF0000u));
+}
+// The sign bits of 8 bf16 values (value 2j in the low half of word wj, 2j + 1 in the high half)
+// where E2M1 codes keep them: value i at bit 4 i + 3.  The high bytes of the eight values are
+// gathered, split into even and odd values, and their bit 7 moved to bit 3 (even values).
+__device__ __forceinline__ uint32_t bf16_sign_nibbles8(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
+    const uint32_t t = __byte_perm(w0, w1, 0x7531), u = __byte_perm(w2, w3, 0x7531);
+    const uint32_t ev = __byte_perm(t, u, 0x6420), od = __byte_perm(t, u, 0x7531);
+    return ((ev >> 4) & 0x08080808u) | (od & 0x80808080u);
+}
+// The same from 4 pairs of binary32 values (sign bit 31 of each).
+__device__ __forceinline__ uint32_t f32_sign_nibbles8(u64 p0, u64 p1, u64 p2, u64 p3) {
+    float a[8];
+    upk(p0, a[0], a[1]);
+    upk(p1, a[2], a[3]);
+    upk(p2, a[4], a[5]);
+    upk(p3, a[6], a[7]);
+    uint32_t u[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) u[i] = __float_as_uint(a[i]);
+    const uint32_t ev = __byte_perm(__byte_perm(u[0], u[2], 0x0073), __byte_perm(u[4], u[6], 0x0073), 0x5410);
+    const uint32_t od = __byte_perm(__byte_perm(u[1], u[3], 0x0073), __byte_perm(u[5], u[7], 0x0073), 0x5410);
+    return ((ev >> 4) & 0x08080808u) | (od & 0x80808080u);
+}
 
 // 2^k as a float for k in [-127, 127] (2^-127 is subnormal).
 __device__ __forceinline__ float pow2i(int k) {

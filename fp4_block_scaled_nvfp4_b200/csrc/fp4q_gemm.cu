@@ -12,42 +12,38 @@
 // (tcgen05.mma kind::mxf4nvf4, 16-element E4M3 or 32-element E8M0 scale blocks) accumulating
 // fp32 in tensor memory; the epilogue reads the accumulator back with tcgen05.ld (each warp
 // its lane quarter), multiplies by RN(S_a S_b) (NVFP4) and stores D.
-//   fp4_gemm_kernel<MX> (the one launched; MX selects MXFP4 operands): one CTA per SM over
-//     128 x 256 output tiles, a four-stage ring filled by tensor copies, producer / MMA /
-//     epilogue warps, two overlapping accumulators so the epilogue of a tile overlaps the next
-//     tile's MMAs.
-//   nvfp4_gemm_kernel (build flag FP4Q_GEMM_SIMPLE): 128 x 128 tiles, the same arithmetic in
-//     one stage with plain loads, kept as the reference form of the sequence.
-// Every wait is bounded; one that runs out sets FP4Q_DEVSTAT_TIMEOUT in the status word, stops
-// the CTA's loops, and the CTA still frees its tensor memory.
+//   fp4_gemm_kernel<MX, OUT_BF16>: one CTA per SM over 128 x 256 output tiles, a four-stage
+//     ring filled by tensor copies, producer / MMA / epilogue warps, two overlapping
+//     accumulators so the epilogue of a tile overlaps the next tile's MMAs; D in fp32 or bf16.
+// Every wait is bounded; one that runs out sets FP4Q_DEVSTAT_TIMEOUT in the status word and
+// stops the CTA's loops.  Before the CTA frees its tensor memory and leaves, the MMA thread waits
+// (bounded) for its tensor-core operations to finish and the producer for the copies it armed.
 #include <atomic>
 #include <cstdint>
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "fp4q.h"
 
-#ifndef FP4Q_GEMM_SIMPLE
-#define FP4Q_GEMM_SIMPLE 0   // 1: the single-stage kernel with plain loads instead of the pipelined one
+// Failure-path test build only (compiled into a separate library by the test suite's build):
+// the MMA thread treats its first wait as timed out, before any copy has landed or any MMA has
+// been issued, so that the bounded exit path runs; never set in the product library.
+#ifndef FP4Q_GEMM_FAIL_FIRST_WAIT
+#define FP4Q_GEMM_FAIL_FIRST_WAIT 0
 #endif
 
 namespace fp4q {
 
 extern thread_local int g_launches;
+extern thread_local int g_cuda_error;
 
 namespace gemm {
 
-constexpr int kTM = 128, kTN = 128, kTK = 256;     // CTA tile and K per stage
-constexpr int kThreads = 128;
-constexpr uint32_t kTmemCols = 256;                // accumulator 128 + scale factors 16 + 16
-constexpr uint32_t kColSFA = 128, kColSFB = 144;
-constexpr int kTileBytes = kTM * kTK / 2;          // 16 KB of codes per operand and stage
+constexpr int kTM = 128, kTN = 128, kTK = 256;     // M tile, narrow N tile, K per stage
+constexpr int kTileBytes = kTM * kTK / 2;          // 16 KB of A codes per stage
 constexpr int kSfBytes = 4 * 512;                  // four 128x4 scale atoms per operand and stage
-constexpr int kSmemBytes = 2 * kTileBytes + 2 * kSfBytes + 64;
-// The request is padded so that at most two CTAs share an SM: two allocations of 256 tensor
-// memory columns fill the 512 an SM has, so no allocation ever waits for another CTA.
-[[maybe_unused]] constexpr int kSmemAlloc = (kSmemBytes + 1024) > 100 * 1024 ? (kSmemBytes + 1024) : 100 * 1024;
 constexpr uint32_t kWaitPolls = 1u << 22;          // bounded mbarrier wait
 
 // Shared-memory matrix descriptor (sm_100 tensor-core operand): start address, leading and
@@ -78,131 +74,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
         if (done) return true;
     }
     return false;
-}
-
-__global__ void __launch_bounds__(kThreads, 1)
-    nvfp4_gemm_kernel(const uint8_t* __restrict__ a, const uint8_t* __restrict__ sfa, const float* __restrict__ sa,
-                      const uint8_t* __restrict__ b, const uint8_t* __restrict__ sfb, const float* __restrict__ sb,
-                      int K, float* __restrict__ d, int64_t ldd, uint32_t* __restrict__ status) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    uint8_t* sA = smem;
-    uint8_t* sB = smem + kTileBytes;
-    uint8_t* sSFA = smem + 2 * kTileBytes;
-    uint8_t* sSFB = sSFA + kSfBytes;
-    uint64_t* mbar = reinterpret_cast<uint64_t*>(sSFB + kSfBytes);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mbar + 1);
-    __shared__ int s_fail;
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t m0 = (int64_t)blockIdx.y * kTM, n0 = (int64_t)blockIdx.x * kTN;
-    const int64_t rowbytes = K / 2;
-    const int64_t jt = K / 64;                        // scale atoms per 128-row tile along K
-
-    if (warp == 0) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                     :: "r"(smem_u32(tmem_slot)), "r"(kTmemCols) : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-    }
-    if (tid == 0) {
-        s_fail = 0;
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" :: "r"(smem_u32(mbar)) : "memory");
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-    __syncthreads();
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    const uint32_t tmem = *tmem_slot;
-
-    const int KT = K / kTK;
-    uint32_t parity = 0;
-    for (int kt = 0; kt < KT; ++kt) {
-        // operand tiles: 16-byte chunk c of row r goes to chunk c ^ (r % 8) of that row
-        const uint8_t* ga = a + m0 * rowbytes + (int64_t)kt * (kTK / 2);
-        const uint8_t* gb = b + n0 * rowbytes + (int64_t)kt * (kTK / 2);
-        for (int i = tid; i < kTM * 8; i += kThreads) {
-            const int r = i >> 3, c = i & 7;
-            const uint4 va = __ldg(reinterpret_cast<const uint4*>(ga + r * rowbytes + c * 16));
-            const uint4 vb = __ldg(reinterpret_cast<const uint4*>(gb + r * rowbytes + c * 16));
-            *reinterpret_cast<uint4*>(sA + r * 128 + ((c ^ (r & 7)) << 4)) = va;
-            *reinterpret_cast<uint4*>(sB + r * 128 + ((c ^ (r & 7)) << 4)) = vb;
-        }
-        // scale atoms of this stage: atoms 4 kt .. 4 kt + 3 of the row tile, contiguous
-        {
-            const uint4* gsa = reinterpret_cast<const uint4*>(sfa + ((int64_t)blockIdx.y * jt + 4 * kt) * 512);
-            const uint4* gsb = reinterpret_cast<const uint4*>(sfb + ((int64_t)blockIdx.x * jt + 4 * kt) * 512);
-            reinterpret_cast<uint4*>(sSFA)[tid] = __ldg(gsa + tid);
-            reinterpret_cast<uint4*>(sSFB)[tid] = __ldg(gsb + tid);
-        }
-        // the tensor core reads shared memory through the async proxy
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncthreads();
-        if (tid == 0) {
-            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t da = smem_desc(smem_u32(sSFA + kk * 512), 16, 128, 0);
-                const uint64_t db = smem_desc(smem_u32(sSFB + kk * 512), 16, 128, 0);
-                asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" :: "r"(tmem + kColSFA + 4 * kk), "l"(da)
-                             : "memory");
-                asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" :: "r"(tmem + kColSFB + 4 * kk), "l"(db)
-                             : "memory");
-            }
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t adesc = smem_desc(smem_u32(sA + kk * 32), 16, 1024, 2);
-                const uint64_t bdesc = smem_desc(smem_u32(sB + kk * 32), 16, 1024, 2);
-                const uint32_t accumulate = (kt > 0 || kk > 0) ? 1u : 0u;
-                asm volatile(
-                    "{ .reg .pred p;\n"
-                    "  setp.ne.b32 p, %4, 0;\n"
-                    "  tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p; }"
-                    :: "r"(tmem), "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate),
-                       "r"(tmem + kColSFA + 4 * kk), "r"(tmem + kColSFB + 4 * kk)
-                    : "memory");
-            }
-            asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-                         :: "r"(smem_u32(mbar)) : "memory");
-        }
-        // the MMAs have read the shared tiles before anyone refills them
-        if (!mbar_wait(smem_u32(mbar), parity)) s_fail = 1;
-        parity ^= 1u;
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        __syncthreads();
-        if (s_fail) break;
-    }
-
-    if (!s_fail) {
-        const float scale = __fmul_rn(*sa, *sb);
-        float* drow = d + (m0 + warp * 32 + lane) * ldd + n0;
-#pragma unroll 1
-        for (int c0 = 0; c0 < kTN; c0 += 32) {
-            uint32_t v[32];
-            asm volatile(
-                "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-                "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-                "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-                : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-                  "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
-                  "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
-                  "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
-                  "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-                : "r"(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0)
-                : "memory");
-            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-            for (int j = 0; j < 32; j += 4)
-                *reinterpret_cast<float4*>(drow + c0 + j) =
-                    make_float4(__fmul_rn(__uint_as_float(v[j]), scale), __fmul_rn(__uint_as_float(v[j + 1]), scale),
-                                __fmul_rn(__uint_as_float(v[j + 2]), scale), __fmul_rn(__uint_as_float(v[j + 3]), scale));
-        }
-    } else if (tid == 0) {
-        atomicOr(status, (uint32_t)FP4Q_DEVSTAT_TIMEOUT);
-    }
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-    __syncthreads();
-    if (warp == 0)
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(kTmemCols) : "memory");
 }
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -254,7 +125,7 @@ constexpr int kPThreads = 192;
 constexpr uint32_t kPTmemCols = 512;
 constexpr uint32_t kAcc1 = 192;                            // first column of the odd tiles' accumulator
 constexpr uint32_t kPColSFA = 448, kPColSFB = 464;
-constexpr int kPersistSmem = kPStages * kPStageBytes + 1024 + 256;
+constexpr int kPersistSmem = kPStages * kPStageBytes + 1024 + 256;   // ring, alignment, barriers
 constexpr uint32_t kIdescN256 = (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(kTM >> 4) << 24);
 
 // MX = false: NVFP4 operands (E4M3 factor per 16 elements, tensor scales S_a, S_b); MX = true:
@@ -263,12 +134,12 @@ constexpr uint32_t kIdescN256 = (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) <
 // four, and each K = 64 MMA reads two of a 32-bit column's four factor bytes: the byte offset
 // (0 or 2) goes into the tensor-memory address's top bits and the instruction descriptor's
 // factor-id fields.
-template <bool MX>
+template <bool MX, bool OUT_BF16>
 __global__ void __launch_bounds__(kPThreads, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                                  const uint8_t* __restrict__ sfa, const float* __restrict__ sa,
                                  const uint8_t* __restrict__ sfb, const float* __restrict__ sb, int K, int m_tiles,
-                                 int n_tiles, int n_last_wide, float* __restrict__ d, int64_t ldd,
+                                 int n_tiles, int n_last_wide, void* __restrict__ dv, int64_t ldd,
                                  uint32_t* __restrict__ status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -276,7 +147,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
     uint64_t* empty = full + kPStages;
     uint64_t* acc_full = empty + kPStages;
     uint64_t* acc_free = acc_full + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_free + 1);
+    uint64_t* drained = acc_free + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 1);
     __shared__ volatile int s_fail;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -301,6 +173,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
         }
         mbar_init(smem_u32(acc_full), 1);
         mbar_init(smem_u32(acc_free), 4);   // one arrival per epilogue warp
+        mbar_init(smem_u32(drained), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(&tma_a)) : "memory");
         asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(&tma_b)) : "memory");
@@ -362,7 +235,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
             const uint32_t tacc = tmem + ((j & 1) ? kAcc1 : 0u);
             for (int kt = 0; kt < KT; ++kt, ++g) {
                 const uint32_t s = g % kPStages, round = g / kPStages;
-                if (!mbar_wait(smem_u32(full + s), round & 1u)) { s_fail = 1; break; }
+                if ((FP4Q_GEMM_FAIL_FIRST_WAIT && g == 0) || !mbar_wait(smem_u32(full + s), round & 1u)) {
+                    s_fail = 1;
+                    break;
+                }
                 asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
                 uint8_t* st = smem + s * kPStageBytes;
                 uint8_t* ssf = st + kTileBytes + kBTileBytes;
@@ -436,7 +312,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
             const int first = (!odd && nchunks == 8) ? 6 : 0;
             const int shared_chunks = odd ? 2 : (nchunks == 8 ? 2 : 0);
             const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (odd ? kAcc1 : 0u);
-            float* drow = d + ((int64_t)mt * kTM + q * 32 + lane) * ldd + (int64_t)nt * kBN;
+            const int64_t drow = ((int64_t)mt * kTM + q * 32 + lane) * ldd + (int64_t)nt * kBN;
             for (int i = 0; i <= nchunks; ++i) {
                 if (i == shared_chunks) {
                     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -447,25 +323,55 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 const int c = (first + i) % nchunks;
                 uint32_t v[32];
                 tmem_ld32(tbase + (uint32_t)(c * 32), v);
+                if constexpr (OUT_BF16) {   // RN(RN(acc * scale)) to bf16, nearest even
+                    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(dv) + drow + c * 32);
 #pragma unroll
-                for (int e = 0; e < 32; e += 4)
-                    *reinterpret_cast<float4*>(drow + c * 32 + e) = make_float4(
-                        __fmul_rn(__uint_as_float(v[e]), scale), __fmul_rn(__uint_as_float(v[e + 1]), scale),
-                        __fmul_rn(__uint_as_float(v[e + 2]), scale), __fmul_rn(__uint_as_float(v[e + 3]), scale));
+                    for (int e = 0; e < 32; e += 8) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int h = 0; h < 4; ++h) {
+                            const __nv_bfloat162 p = __floats2bfloat162_rn(
+                                __fmul_rn(__uint_as_float(v[e + 2 * h]), scale),
+                                __fmul_rn(__uint_as_float(v[e + 2 * h + 1]), scale));
+                            w[h] = *reinterpret_cast<const uint32_t*>(&p);
+                        }
+                        dst[e / 8] = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                } else {
+                    float* drp = reinterpret_cast<float*>(dv) + drow + c * 32;
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4)
+                        *reinterpret_cast<float4*>(drp + e) = make_float4(
+                            __fmul_rn(__uint_as_float(v[e]), scale), __fmul_rn(__uint_as_float(v[e + 1]), scale),
+                            __fmul_rn(__uint_as_float(v[e + 2]), scale), __fmul_rn(__uint_as_float(v[e + 3]), scale));
+                }
             }
         }
     }
     __syncwarp();
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
-    if (s_fail && tid == 0) {
-        atomicOr(status, (uint32_t)FP4Q_DEVSTAT_TIMEOUT);
-        // a wait gave up: before the CTA leaves, let the copies it armed land in its shared
-        // memory (the last stage armed in each ring slot; each wait is again bounded)
-        for (uint32_t i = 0; i < (uint32_t)kPStages && i < issued; ++i) {
-            const uint32_t gi = issued - 1 - i;
-            mbar_wait(smem_u32(full + gi % kPStages), (gi / kPStages) & 1u);
+    if (s_fail) {
+        if (tid == 32) {
+            // a wait gave up: the MMA thread's tensor-core operations (MMAs and scale copies into
+            // tensor memory) finish before the memory they use is freed; the commit arrives once
+            // all of them have (the wait is again bounded)
+            asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                         :: "r"(smem_u32(drained)) : "memory");
+            mbar_wait(smem_u32(drained), 0u);
         }
+        if (tid == 0) {
+            atomicOr(status, (uint32_t)FP4Q_DEVSTAT_TIMEOUT);
+            // the copies the producer armed land in this CTA's shared memory before it leaves (the
+            // last stage armed in each ring slot; each wait is again bounded)
+            for (uint32_t i = 0; i < (uint32_t)kPStages && i < issued; ++i) {
+                const uint32_t gi = issued - 1 - i;
+                mbar_wait(smem_u32(full + gi % kPStages), (gi / kPStages) & 1u);
+            }
+        }
+        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+        __syncthreads();
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     }
     __syncwarp();
     if (warp == 0)
@@ -493,11 +399,17 @@ bool smem_attribute_set(int bytes) {
 }
 
 // Shared host path of the two entry points: argument checks, tensor maps, launch.
-template <bool MX>
+template <bool MX, bool OUT_BF16>
 int launch(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global_scale, const uint8_t* b_codes,
-           const uint8_t* b_scales, const float* b_global_scale, int64_t M, int64_t N, int64_t K, float* d, int64_t ldd,
+           const uint8_t* b_scales, const float* b_global_scale, int64_t M, int64_t N, int64_t K, void* d, int64_t ldd,
            void* workspace, void* stream) {
     g_launches = 0;
+    g_cuda_error = 0;
+    // a CUDA call that fails leaves its code for fp4q_last_cuda_error
+    auto cuda_failed = [](cudaError_t e) {
+        g_cuda_error = (int)e;
+        return e != cudaSuccess;
+    };
     if (M < 0 || N < 0 || K < 0 || M % kTM || N % kTN || K % kTK || ldd < N) return FP4Q_ERR_SHAPE;
     if (M / kTM > 65535 || K > (1 << 30)) return FP4Q_ERR_SHAPE;
     if (M == 0 || N == 0 || K == 0) return FP4Q_OK;
@@ -505,30 +417,26 @@ int launch(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_globa
     if (!MX && (!a_global_scale || !b_global_scale)) return FP4Q_ERR_INVALID_ARG;
     auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
     if (!al16(a_codes) || !al16(a_scales) || !al16(b_codes) || !al16(b_scales) || !al16(d) || !al16(workspace) ||
-        ldd % 4)
+        ldd % (OUT_BF16 ? 8 : 4))
         return FP4Q_ERR_ALIGNMENT;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     uint32_t* status = reinterpret_cast<uint32_t*>(workspace);
-    if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return FP4Q_ERR_CUDA;
-#if FP4Q_GEMM_SIMPLE
-    if (MX) return FP4Q_ERR_UNSUPPORTED;
-    if (!smem_attribute_set<nvfp4_gemm_kernel>(kSmemAlloc)) return FP4Q_ERR_CUDA;
-    const dim3 grid((unsigned)(N / kTN), (unsigned)(M / kTM));
-    nvfp4_gemm_kernel<<<grid, kThreads, kSmemAlloc, st>>>(a_codes, a_scales, a_global_scale, b_codes, b_scales,
-                                                          b_global_scale, (int)K, d, ldd, status);
-#else
+    if (cuda_failed(cudaMemsetAsync(status, 0, sizeof(uint32_t), st))) return FP4Q_ERR_CUDA;
     // the tensor-copy descriptors of A and B: [rows][K/2] bytes, 128-byte-wide boxes of 128 (A) or
     // 256 (B) rows, 128-byte swizzle
     static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
     if (!encode) {
         void* fn = nullptr;
         cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        if (cuda_failed(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q)) ||
             q != cudaDriverEntryPointSuccess || !fn)
             return FP4Q_ERR_CUDA;
         encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
-    if (!smem_attribute_set<fp4_gemm_kernel<MX>>(kPersistSmem)) return FP4Q_ERR_CUDA;
+    if (!smem_attribute_set<fp4_gemm_kernel<MX, OUT_BF16>>(kPersistSmem)) {
+        g_cuda_error = (int)cudaGetLastError();
+        return FP4Q_ERR_CUDA;
+    }
     CUtensorMap ta, tb;
     auto make = [&](CUtensorMap* m, const uint8_t* base, int64_t rows, int box_rows) {
         const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
@@ -539,7 +447,10 @@ int launch(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_globa
                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
     };
-    if (!make(&ta, a_codes, M, kTM) || !make(&tb, b_codes, N, kBN)) return FP4Q_ERR_CUDA;
+    if (!make(&ta, a_codes, M, kTM) || !make(&tb, b_codes, N, kBN)) {
+        g_cuda_error = -1;   // the tensor-map encoder refused the operands
+        return FP4Q_ERR_CUDA;
+    }
     static int sms = 0;
     if (!sms) {
         int dev = 0;
@@ -549,11 +460,10 @@ int launch(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_globa
     }
     const int m_tiles = (int)(M / kTM), n_tiles = (int)((N + kBN - 1) / kBN);
     const int tiles = m_tiles * n_tiles;
-    fp4_gemm_kernel<MX><<<tiles < sms ? tiles : sms, kPThreads, kPersistSmem, st>>>(
+    fp4_gemm_kernel<MX, OUT_BF16><<<tiles < sms ? tiles : sms, kPThreads, kPersistSmem, st>>>(
         ta, tb, a_scales, a_global_scale, b_scales, b_global_scale, (int)K, m_tiles, n_tiles, (int)(N % kBN == 0), d,
         ldd, status);
-#endif
-    if (cudaGetLastError() != cudaSuccess) return FP4Q_ERR_CUDA;
+    if (cuda_failed(cudaGetLastError())) return FP4Q_ERR_CUDA;
     g_launches = 1;
     return FP4Q_OK;
 }
@@ -561,17 +471,36 @@ int launch(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_globa
 }  // namespace gemm
 }  // namespace fp4q
 
+extern "C" int fp4q_gemm(int fmt, const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global_scale,
+                         const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global_scale, int64_t M,
+                         int64_t N, int64_t K, void* d, int64_t ldd, uint32_t flags, void* workspace, void* stream) {
+    fp4q::g_launches = 0;
+    if (flags & ~(uint32_t)FP4Q_F_OUT_BF16) return FP4Q_ERR_INVALID_ARG;
+    const bool bf = (flags & FP4Q_F_OUT_BF16) != 0;
+    if (fmt == FP4Q_NVFP4)
+        return bf ? fp4q::gemm::launch<false, true>(a_codes, a_scales, a_global_scale, b_codes, b_scales, b_global_scale,
+                                                    M, N, K, d, ldd, workspace, stream)
+                  : fp4q::gemm::launch<false, false>(a_codes, a_scales, a_global_scale, b_codes, b_scales,
+                                                     b_global_scale, M, N, K, d, ldd, workspace, stream);
+    if (fmt == FP4Q_MXFP4)
+        return bf ? fp4q::gemm::launch<true, true>(a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, M, N, K, d,
+                                                   ldd, workspace, stream)
+                  : fp4q::gemm::launch<true, false>(a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, M, N, K, d,
+                                                    ldd, workspace, stream);
+    return fmt == FP4Q_IF4 ? FP4Q_ERR_UNSUPPORTED : FP4Q_ERR_INVALID_ARG;
+}
+
 extern "C" int fp4q_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global_scale,
                                const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global_scale,
                                int64_t M, int64_t N, int64_t K, float* d, int64_t ldd, void* workspace,
                                void* stream) {
-    return fp4q::gemm::launch<false>(a_codes, a_scales, a_global_scale, b_codes, b_scales, b_global_scale, M, N, K, d,
-                                     ldd, workspace, stream);
+    return fp4q_gemm(FP4Q_NVFP4, a_codes, a_scales, a_global_scale, b_codes, b_scales, b_global_scale, M, N, K, d, ldd,
+                     0, workspace, stream);
 }
 
 extern "C" int fp4q_mxfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* b_codes,
                                const uint8_t* b_scales, int64_t M, int64_t N, int64_t K, float* d, int64_t ldd,
                                void* workspace, void* stream) {
-    return fp4q::gemm::launch<true>(a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, M, N, K, d, ldd, workspace,
-                                    stream);
+    return fp4q_gemm(FP4Q_MXFP4, a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, M, N, K, d, ldd, 0, workspace,
+                     stream);
 }

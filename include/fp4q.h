@@ -71,6 +71,14 @@
 #include <stddef.h>
 #include <stdint.h>
 
+/* Exported entry points (the library is built with hidden visibility: nothing else is exported,
+ * so two builds of it loaded into one process keep their internal state apart). */
+#if defined(__GNUC__)
+#define FP4Q_API __attribute__((visibility("default")))
+#else
+#define FP4Q_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -88,7 +96,7 @@ typedef enum {
  * its tensor-core work (its output is then incomplete). */
 enum { FP4Q_DEVSTAT_OK = 0, FP4Q_DEVSTAT_NONFINITE = 1, FP4Q_DEVSTAT_RANGE = 2, FP4Q_DEVSTAT_TIMEOUT = 4 };
 enum { FP4Q_IN_F32 = 0, FP4Q_IN_BF16 = 1 };
-enum { FP4Q_NVFP4 = 0, FP4Q_IF4 = 1, FP4Q_MXFP4 = 2 };
+enum { FP4Q_NVFP4 = 0, FP4Q_IF4 = 1, FP4Q_MXFP4 = 2, FP4Q_IF6 = 3 };
 enum { FP4Q_ABSMAX = 0, FP4Q_FOUR_OVER_SIX = 1, FP4Q_SWEEP_MSE = 2, FP4Q_SWEEP_WMSE = 3 };
 
 #define FP4Q_F_GLOBAL_SCALE_GIVEN 0x1u  /* quantize: read S from *global_scale (no amax pass) */
@@ -110,7 +118,7 @@ enum { FP4Q_ABSMAX = 0, FP4Q_FOUR_OVER_SIX = 1, FP4Q_SWEEP_MSE = 2, FP4Q_SWEEP_W
                                            window p0-3 .. p0+7 (see the arithmetic above)      */
 
 /* Size in bytes of the workspace every quantize call needs (a small constant). */
-size_t fp4q_workspace_bytes(void);
+FP4Q_API size_t fp4q_workspace_bytes(void);
 
 /*
  * Size in bytes of the scales buffer of a rows x cols tensor in format fmt: rows * cols/B
@@ -125,7 +133,7 @@ size_t fp4q_workspace_bytes(void);
  * scales as written (fp4q_nvfp4_gemm and fp4q_mxfp4_gemm do).  IF4 has no tiled form (its indicator bit is not a consumer format).
  * Returns -1 for an unknown format or a bad shape.
  */
-int64_t fp4q_scale_bytes(int64_t rows, int64_t cols, int fmt, uint32_t flags);
+FP4Q_API int64_t fp4q_scale_bytes(int64_t rows, int64_t cols, int fmt, uint32_t flags);
 
 /*
  * Quantize x into codes + scales (+ S).
@@ -156,7 +164,7 @@ int64_t fp4q_scale_bytes(int64_t rows, int64_t cols, int fmt, uint32_t flags);
  * Launches: NVFP4/IF4 without a given S: an amax kernel then the quantize kernel;
  * otherwise one kernel.  Empty tensors launch nothing.
  */
-int fp4q_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+FP4Q_API int fp4q_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld,
                   int fmt, int objective, const float* importance,
                   uint8_t* codes, uint8_t* scales, float* global_scale,
                   void* workspace, uint32_t flags, void* stream);
@@ -169,7 +177,7 @@ int fp4q_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int64_t 
  * Passing the result to fp4q_quantize with FP4Q_F_GLOBAL_SCALE_GIVEN performs exactly the
  * work of a call without the flag.  cols * element size must be a multiple of 16 bytes.
  */
-int fp4q_global_scale(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+FP4Q_API int fp4q_global_scale(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld,
                       float* global_scale, void* workspace, void* stream);
 
 /*
@@ -181,7 +189,7 @@ int fp4q_global_scale(const void* x, int dtype, int64_t rows, int64_t cols, int6
  * overflows, gives S = NaN.  Status, workspace and errors as fp4q_global_scale.  Use: a
  * row-sharded tensor reduces the per-shard S values by maximum.
  */
-int fp4q_hadamard_global_scale(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+FP4Q_API int fp4q_hadamard_global_scale(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld,
                                int had_size, float* global_scale, void* workspace, void* stream);
 
 /*
@@ -194,7 +202,7 @@ int fp4q_hadamard_global_scale(const void* x, int dtype, int64_t rows, int64_t c
  * fmt = FP4Q_MXFP4.  Dequantized values are in the rotated domain.  flags: 0,
  * FP4Q_F_MX_OCP_FLOOR or FP4Q_F_MX_SWEEP (the MX scale sweep on the rotated blocks).
  */
-int fp4q_hadamard_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+FP4Q_API int fp4q_hadamard_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld,
                            int had_size, uint8_t* codes, uint8_t* scales,
                            void* workspace, uint32_t flags, void* stream);
 
@@ -225,7 +233,7 @@ int fp4q_hadamard_quantize(const void* x, int dtype, int64_t rows, int64_t cols,
  * event after it).  Errors as fp4q_quantize; the device status lands in the set's
  * workspace.  Launch count as fp4q_quantize (copies are not counted).
  */
-int fp4q_quantize_host_async(const void* x_host, int dtype, int64_t rows, int64_t cols,
+FP4Q_API int fp4q_quantize_host_async(const void* x_host, int dtype, int64_t rows, int64_t cols,
                              int fmt, int objective, const float* importance,
                              uint8_t* codes_host, uint8_t* scales_host, float* S_host,
                              void* x_dev, uint8_t* codes_dev, uint8_t* scales_dev, float* S_dev,
@@ -244,7 +252,7 @@ int fp4q_quantize_host_async(const void* x_host, int dtype, int64_t rows, int64_
  * pointer (ignored for MXFP4).  out must be 16-byte aligned.  flags: FP4Q_F_OUT_BF16 and
  * FP4Q_F_SCALE_TILED (scales in the tiled layout of fp4q_scale_bytes; NVFP4 and MXFP4).
  */
-int fp4q_dequantize(const uint8_t* codes, const uint8_t* scales, const float* global_scale,
+FP4Q_API int fp4q_dequantize(const uint8_t* codes, const uint8_t* scales, const float* global_scale,
                     int64_t rows, int64_t cols, int fmt, int inverse_hadamard,
                     void* out, uint32_t flags, void* stream);
 
@@ -271,7 +279,7 @@ int fp4q_dequantize(const uint8_t* codes, const uint8_t* scales, const float* gl
  *   share it: calls that may run at the same time on the GPU (different streams, different
  *   host threads) race and must be serialized by the caller.
  */
-int fp4q_quantize_noalloc(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+FP4Q_API int fp4q_quantize_noalloc(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld,
                           int fmt, int objective, const float* importance,
                           uint8_t* codes, uint8_t* scales, float* global_scale,
                           uint32_t* device_status, uint32_t flags, void* stream);
@@ -289,16 +297,20 @@ int fp4q_quantize_noalloc(const void* x, int dtype, int64_t rows, int64_t cols, 
  * FP4Q_ERR_ALIGNMENT.  NaN inputs give whatever the hardware conversion gives.
  */
 enum { FP4Q_CODEC_E2M1 = 0, FP4Q_CODEC_E4M3 = 1 };
-int fp4q_encode(const float* x, int64_t n, int kind, uint8_t* out, void* stream);
+FP4Q_API int fp4q_encode(const float* x, int64_t n, int kind, uint8_t* out, void* stream);
 
 /* Copy the device status word of `workspace` to *status (blocks until `stream` is done). */
-int fp4q_read_device_status(const void* workspace, uint32_t* status, void* stream);
+FP4Q_API int fp4q_read_device_status(const void* workspace, uint32_t* status, void* stream);
 
 /* Number of kernel launches the most recent successful call on this thread issued. */
-int fp4q_last_launch_count(void);
+FP4Q_API int fp4q_last_launch_count(void);
+
+/* The cudaError_t value behind the most recent FP4Q_ERR_CUDA on this thread from a launching call
+ * (0 after a successful launch; -1 when the GEMM's tensor-map encoder refused its operands). */
+FP4Q_API int fp4q_last_cuda_error(void);
 
 /* Static description of a status code. */
-const char* fp4q_status_string(int status);
+FP4Q_API const char* fp4q_status_string(int status);
 
 /*
  * Block-scaled NVFP4 GEMM on the B200 tensor cores (tcgen05), the consumer of two quantized
@@ -314,9 +326,11 @@ const char* fp4q_status_string(int status);
  * d: fp32 [M][ldd], ldd >= N, ldd a multiple of 4; all pointers device memory, 16-byte
  * aligned.  M and N multiples of 128, K a multiple of 256 (FP4Q_ERR_SHAPE otherwise).
  * workspace: fp4q_workspace_bytes() bytes; its word 0 receives the device status
- * (FP4Q_DEVSTAT_TIMEOUT if a bounded wait for the tensor cores ran out).  One launch.
+ * (FP4Q_DEVSTAT_TIMEOUT if a bounded wait for the tensor cores ran out; the kernel then lets its
+ * tensor-core operations and armed copies finish, each again with a bounded wait, frees its
+ * tensor memory and returns, so the context stays usable).  One launch.
  */
-int fp4q_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global_scale,
+FP4Q_API int fp4q_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global_scale,
                     const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global_scale,
                     int64_t M, int64_t N, int64_t K, float* d, int64_t ldd, void* workspace,
                     void* stream);
@@ -331,9 +345,24 @@ int fp4q_nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float
  * the Gap ... Microscaling FP4, "Methodology": rotations folded into the adjacent weights).
  * Shapes, alignment, layout of d, workspace and errors as for fp4q_nvfp4_gemm.
  */
-int fp4q_mxfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* b_codes,
+FP4Q_API int fp4q_mxfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* b_codes,
                     const uint8_t* b_scales, int64_t M, int64_t N, int64_t K, float* d, int64_t ldd,
                     void* workspace, void* stream);
+
+/*
+ * Either GEMM with a choice of output type: fmt FP4Q_NVFP4 (arguments as fp4q_nvfp4_gemm) or
+ * FP4Q_MXFP4 (as fp4q_mxfp4_gemm; the global-scale pointers are ignored).  d is fp32 [M][ldd]
+ * (ldd a multiple of 4) or, with flags = FP4Q_F_OUT_BF16, bf16 [M][ldd] (ldd a multiple of 8):
+ * the fp32 value RN(acc * RN(S_a S_b)) rounded to the nearest bf16, ties to even.  The pages
+ * leave the consumer's output type open; bf16 is the usual activation type of the layer after
+ * the GEMM and halves the bytes D takes.  Errors: FP4Q_ERR_INVALID_ARG (unknown format or flag),
+ * FP4Q_ERR_UNSUPPORTED (FP4Q_IF4: its indicator bit is not a tensor-core operand format), and
+ * those of fp4q_nvfp4_gemm.
+ */
+FP4Q_API int fp4q_gemm(int fmt, const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global_scale,
+              const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global_scale,
+              int64_t M, int64_t N, int64_t K, void* d, int64_t ldd, uint32_t flags,
+              void* workspace, void* stream);
 
 #ifdef __cplusplus
 }

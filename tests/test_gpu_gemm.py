@@ -156,3 +156,28 @@ def test_full_size_gemm_sampled(mx):
     got = d[torch.from_numpy(rows).cuda()][:, torch.from_numpy(cols).cuda()].cpu().numpy().astype(np.float64)
     mag = np.abs(da) @ np.abs(db).T
     assert np.all(np.abs(got - ref) <= 2e-5 * mag + 1e-30), float(np.max(np.abs(got - ref) / (mag + 1e-30)))
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 384, 1024), (128, 256, 512)])
+def test_gemm_bf16_output(M, N, K):
+    # bf16 D: each value is the fp32 result RN(acc * RN(S_a S_b)) rounded to bf16 (nearest even),
+    # checked against the fp32 launch of the same operands rounded by the oracle's bf16 rounding
+    (qa, ra), (qb, rb) = _operand("cfg3", M, K, "sweep_mse"), _operand("cfg2", N, K, "sweep_mse")
+    ws = fq.new_workspace()
+    d32 = fq.nvfp4_gemm(qa, qb, workspace=ws)
+    d16 = fq.nvfp4_gemm(qa, qb, workspace=ws, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert fq.read_device_status(ws) == fq.DEVSTAT_OK
+    want = O.f32_to_bf16(d32.cpu().numpy())
+    got = d16.view(torch.int16).cpu().numpy().view(np.uint16).ravel()
+    assert np.array_equal(got, want)
+    # the MXFP4 GEMM with rotated operands rounds its fp32 result the same way
+    xa = torch.from_numpy(synth.make("cfg3", rows=M, cols=K)["x"].view(np.int16)).view(torch.bfloat16).cuda()
+    xb = torch.from_numpy(synth.make("cfg2", rows=N, cols=K)["x"].view(np.int16)).view(torch.bfloat16).cuda()
+    a = fq.hadamard_quantize(xa, tiled_scales=True)
+    b = fq.hadamard_quantize(xb, tiled_scales=True)
+    m32 = fq.mxfp4_gemm(a, b, workspace=ws)
+    m16 = fq.mxfp4_gemm(a, b, workspace=ws, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert np.array_equal(m16.view(torch.int16).cpu().numpy().view(np.uint16).ravel(),
+                          O.f32_to_bf16(m32.cpu().numpy()))
