@@ -66,7 +66,12 @@ METRIC = "quantize GB/s (input bf16) and % of B200 HBM peak, 1 GPU, vs CPU oracl
 # [N][K] (Llama-3-8B-shaped MLP up-projection, 14336x4096, Student-t weights), K contiguous.
 GEMM_METRIC = "NVFP4 block-scaled GEMM TFLOP/s (tcgen05), 1 GPU"
 GEMM_MX_METRIC = "MXFP4 block-scaled GEMM TFLOP/s (tcgen05), 1 GPU"
-GEMM_WORKLOADS = ("gemm", "gemm_mx")
+GEMM_DYN_METRIC = ("NVFP4 dynamic-activation GEMM TFLOP/s (amax + ScaleSweep quantize of the activation, then the "
+                   "tcgen05 GEMM), 1 GPU")
+# gemm / gemm_mx: the GEMM alone on pre-quantized operands (fp32 D); gemm_bf16: the same with bf16 D;
+# gemm_dyn: each step quantizes the bf16 activation (amax + ScaleSweep-MSE, tiled scales) and runs the
+# NVFP4 GEMM against the pre-quantized weight with bf16 D
+GEMM_WORKLOADS = ("gemm", "gemm_mx", "gemm_bf16", "gemm_dyn")
 GEMM_SHAPE = (8192, 14336, 4096)
 # Arithmetic the method itself needs per element for the ALU-bound searches: per candidate
 # scale one multiply (x/s), one E2M1 rounding, and the two accumulations of the exact block
@@ -404,28 +409,28 @@ def run_ours(args, rank, world):
     in_bytes = x_host.numel() * 2
     alg = algorithmic_bytes(rows, cols, fmt, wmse=(obj == "sweep_wmse"))
     out_bytes = rows * cols // 2 + rows * cols // (32 if fmt.startswith("mxfp4") else 16)
-    nsets = max(2, int(np.ceil(2.5 * L2_BYTES / (in_bytes + out_bytes))))
+    nsets = max(2, int(np.ceil(3.0 * L2_BYTES / (in_bytes + out_bytes))))
     xs = [x_host.to(dev) for _ in range(nsets)]
     base, had16 = split_fmt(fmt)
     outs = [fq.alloc_outputs(rows, cols, "mxfp4" if fmt.startswith("mxfp4") else base, dev) for _ in range(nsets)]
     imp = torch.from_numpy(w["importance"]).to(dev) if obj == "sweep_wmse" else None
-    ws = fq.new_workspace(dev)
+    wss = [fq.new_workspace(dev) for _ in range(nsets)]   # one per buffer set: steps may overlap
     launches_per_step = 0
 
     def amax(s):
-        fq.global_scale(xs[s], out=outs[s][2], workspace=ws, hadamard16=had16)
+        fq.global_scale(xs[s], out=outs[s][2], workspace=wss[s], hadamard16=had16)
         return 1
 
     def quant(s):
         c, sc, g = outs[s]
         if fmt.startswith("mxfp4"):   # one kernel, no tensor scale
             if fmt.endswith("had"):
-                fq.hadamard_quantize(xs[s], out=(c, sc, None), workspace=ws, mx_sweep=(obj == "mx_sweep"))
+                fq.hadamard_quantize(xs[s], out=(c, sc, None), workspace=wss[s], mx_sweep=(obj == "mx_sweep"))
             else:
-                fq.quantize(xs[s], "mxfp4", out=(c, sc, None), workspace=ws, mx_sweep=(obj == "mx_sweep"))
+                fq.quantize(xs[s], "mxfp4", out=(c, sc, None), workspace=wss[s], mx_sweep=(obj == "mx_sweep"))
         else:
-            fq.quantize(xs[s], base, obj or "absmax", importance=imp, global_scale=g, out=(c, sc, g), workspace=ws,
-                        hadamard16=had16, if4_sweep=(obj == "if4_sweep"))
+            fq.quantize(xs[s], base, obj or "absmax", importance=imp, global_scale=g, out=(c, sc, g),
+                        workspace=wss[s], hadamard16=had16, if4_sweep=(obj == "if4_sweep"))
         return 1
 
     def step(s):
@@ -448,11 +453,41 @@ def run_ours(args, rank, world):
     # costs several microseconds): one per buffer set, for a remainder of steps, and one that
     # runs every set once in turn
     graphs = [capture(lambda s=s: step(s)) for s in range(nsets)]
-    cycle = capture(lambda: [step(s) for s in range(nsets)])
+    two_pass = not fmt.startswith("mxfp4")
+    side = torch.cuda.Stream(device=dev)
+
+    def pipelined_cycle():
+        # every set's amax + quantize in turn, with the next set's amax pass (HBM-bound) on a
+        # second stream under this set's quantize (compute-bound); each quantize waits for its
+        # own set's amax, and each amax for the quantize two sets back (at most one of each runs)
+        done_amax, done_quant = [], []
+        fork = torch.cuda.Event()
+        fork.record(stream)
+        side.wait_event(fork)
+        for s in range(nsets):
+            with torch.cuda.stream(side):
+                if s >= 2:
+                    side.wait_event(done_quant[s - 2])
+                amax(s)
+                e = torch.cuda.Event()
+                e.record(side)
+                done_amax.append(e)
+            stream.wait_event(done_amax[s])
+            quant(s)
+            e = torch.cuda.Event()
+            e.record(stream)
+            done_quant.append(e)
+        join = torch.cuda.Event()
+        join.record(side)
+        stream.wait_event(join)
+
+    cycle = capture(pipelined_cycle if two_pass else (lambda: [step(s) for s in range(nsets)]))
+    serial_cycle = capture(lambda: [step(s) for s in range(nsets)]) if two_pass else cycle
     with torch.cuda.stream(stream):
         for s in range(nsets):
             graphs[s].replay()
         cycle.replay()
+        serial_cycle.replay()
     torch.cuda.synchronize()
     full_cycles, rest = divmod(args.steps, nsets)
 
@@ -477,6 +512,23 @@ def run_ours(args, rank, world):
         t = torch.tensor([ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
+
+    # the same steps with no overlap between them (one stream, amax then quantize per step)
+    serial_ms = ms
+    if two_pass:
+        with torch.cuda.stream(stream):
+            start.record()
+            for _ in range(full_cycles):
+                serial_cycle.replay()
+            for i in range(rest):
+                graphs[i].replay()
+            end.record()
+        end.synchronize()
+        serial_ms = start.elapsed_time(end)
+        if world > 1:
+            t = torch.tensor([serial_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            serial_ms = float(t.item())
 
     # per-kernel launch durations for the roofline: the same launches, one kernel kind at a
     # time (every buffer set in turn, so reads still come from HBM), timed with CUDA events on
@@ -515,8 +567,8 @@ def run_ours(args, rank, world):
     step_dist = {"p10": pick(0.1), "p50": pick(0.5), "p90": pick(0.9), "steps": n_dist,
                  "how": "each step between its own CUDA events on the launching stream"}
 
-    # status of the last step must be clean
-    st = fq.read_device_status(ws)
+    # every buffer set's status word must be clean
+    st = next((v for v in (fq.read_device_status(w_) for w_ in wss) if v), 0)
 
     # end to end through the public API with host buffers: every step copies its input in
     # from pinned memory, quantizes, and copies codes, scales and S out; two staging sets let
@@ -583,14 +635,20 @@ def run_ours(args, rank, world):
                    "method": obj or fmt, "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": f"{nsets} rotating input/output buffer sets, {nsets * (in_bytes + out_bytes) / 2**20:.0f} MB "
                          f"total (> 2x the 126 MB L2)",
-                   "timing": "CUDA graph of one step per buffer set (no timing nodes inside), replayed in turn on one "
-                             "stream; CUDA events on that stream"},
+                   "timing": ("CUDA graph over the buffer sets (no timing nodes inside); each step's amax pass runs on "
+                              "a second stream under the previous step's quantize kernel, each quantize after its own "
+                              "amax; CUDA events on the launching stream" if two_pass else
+                              "CUDA graph over the buffer sets (no timing nodes inside), replayed on one stream; CUDA "
+                              "events on that stream")},
         "hbm_frac": round(value / world / peak, 4),
         "input_gbps": round(in_bytes * args.steps * world / (ms * 1e-3) / 1e9, 2),
         "elements_per_s": round(rows * cols * args.steps * world / (ms * 1e-3), 1),
         "kernels_ms": {"amax": (None if t_amax is None else round(t_amax, 5)), "quantize": round(tq, 5),
                        "how": f"each kernel alone, {kernel_reps} launches over the rotating buffer sets, CUDA events"},
         "step_ms": step_dist,
+        "serial": {"value": round(alg * args.steps * world / (serial_ms * 1e-3) / 1e9, 2),
+                   "ms_per_step": round(serial_ms / args.steps, 5),
+                   "how": "the same steps with no overlap: amax then quantize per step on one stream"},
         "roofline": roofline,
         "device_status": st,
         "gpu_launches": launches_per_step * args.steps,
@@ -776,6 +834,10 @@ def run_reference_gemm(args, rank, world):
         return
     M, N, K = GEMM_SHAPE
     mx = args.workload == "gemm_mx"
+    if args.workload == "gemm_dyn":
+        print(json.dumps({"impl": "reference", "unavailable": "the dynamic GEMM line has no CPU arm; the oracle's "
+                          "quantize and GEMM are timed by the quantize and gemm workloads"}), flush=True)
+        return
     wa = synth.make("cfg3", rows=16 * max(1, args.steps + args.warmup), cols=K)
     wb = synth.make("cfg2", rows=1024, cols=K)
     if mx:
@@ -819,14 +881,28 @@ def run_gemm(args, rank, world):
     dev = torch.device("cuda", local)
     fq.lib()
     mx = args.workload == "gemm_mx"
+    dyn = args.workload == "gemm_dyn"
+    out_bf16 = args.workload in ("gemm_bf16", "gemm_dyn")
     gemm = fq.mxfp4_gemm if mx else fq.nvfp4_gemm
     (M, N, K), qa, qb, wa, wb = gemm_operands(torch, fq, synth, dev, mx=mx)
-    d = torch.empty((M, N), dtype=torch.float32, device=dev)
+    d = torch.empty((M, N), dtype=torch.bfloat16 if out_bf16 else torch.float32, device=dev)
     ws = fq.new_workspace(dev)
     stream = torch.cuda.Stream(device=dev)
+    if dyn:
+        # the activation in bf16, quantized every step into qa's buffers (S, codes, tiled scales)
+        xa = device_tensor_from_bits(wa["x"], torch).to(dev)
+        ws_q = fq.new_workspace(dev)
+
+        def one_step():
+            fq.global_scale(xa, out=qa[2], workspace=ws_q)
+            fq.quantize(xa, "nvfp4", "sweep_mse", global_scale=qa[2], out=qa, workspace=ws_q, tiled_scales=True)
+            gemm(qa, qb, out=d, workspace=ws)
+    else:
+        def one_step():
+            gemm(qa, qb, out=d, workspace=ws)
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
-            gemm(qa, qb, out=d, workspace=ws)
+            one_step()
     torch.cuda.synchronize()
     flops = 2.0 * M * N * K
     steps = args.steps
@@ -839,7 +915,7 @@ def run_gemm(args, rank, world):
         with torch.cuda.stream(stream):
             start.record()
             for _ in range(steps):
-                gemm(qa, qb, out=d, workspace=ws)
+                one_step()
             end.record()
         end.synchronize()
     torch.cuda.synchronize()
@@ -851,10 +927,20 @@ def run_gemm(args, rank, world):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
     st = fq.read_device_status(ws)
+    gemm_only_ms = ms
+    if dyn:   # the GEMM alone on the same operands, for the split of the step
+        st = st or fq.read_device_status(ws_q)
+        with torch.cuda.stream(stream):
+            start.record()
+            for _ in range(steps):
+                gemm(qa, qb, out=d, workspace=ws)
+            end.record()
+        end.synchronize()
+        gemm_only_ms = start.elapsed_time(end) / steps
     # end to end through the public API: operands (codes, tiled scales, S) copied in from pinned
     # host memory, the GEMM, and the fp32 product copied back, every step
     hosts = [t.cpu().pin_memory() for t in (*qa, *qb)]
-    d_host = torch.empty((M, N), dtype=torch.float32, pin_memory=True)
+    d_host = torch.empty((M, N), dtype=d.dtype, pin_memory=True)
     devs = [torch.empty_like(t, device=dev) for t in hosts]
     e_steps = max(1, min(steps, 5))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -877,15 +963,19 @@ def run_gemm(args, rank, world):
         return
     peak, peak_src = fp4_peak_tflops()
     tf = flops / (ms * 1e-3) / 1e12
-    line = {"metric": GEMM_MX_METRIC if mx else GEMM_METRIC, "value": round(tf * world, 1), "unit": "TFLOP/s",
-            "n_gpus": world, "steps": steps,
+    out_desc = "bf16 out" if out_bf16 else "fp32 out"
+    workload = ("MXFP4 GEMM, activations 8192x4096 (activation workload) times weight 14336x4096 (Student-t), both "
+                "rotated by the 32-point block Hadamard, K contiguous, tiled E8M0 scales, fp32 out") if mx else (
+               "NVFP4 GEMM, activations 8192x4096 (activation workload, sweep-MSE) times weight 14336x4096 "
+               f"(Student-t, sweep-MSE), K contiguous, tiled scales, {out_desc}")
+    if dyn:
+        workload = ("per step: amax + ScaleSweep-MSE quantization of the bf16 activation 8192x4096 (tiled scales), "
+                    "then the NVFP4 GEMM against the pre-quantized 14336x4096 weight, bf16 out")
+    line = {"metric": GEMM_DYN_METRIC if dyn else (GEMM_MX_METRIC if mx else GEMM_METRIC), "value": round(tf * world, 1),
+            "unit": "TFLOP/s", "n_gpus": world, "steps": steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "e2m1xe2m1->f32", "data": "synthetic",
-            "config": {"workload": ("MXFP4 GEMM, activations 8192x4096 (activation workload) times weight 14336x4096 "
-                                    "(Student-t), both rotated by the 32-point block Hadamard, K contiguous, tiled "
-                                    "E8M0 scales, fp32 out") if mx else
-                                   ("NVFP4 GEMM, activations 8192x4096 (activation workload, sweep-MSE) times weight "
-                                    "14336x4096 (Student-t, sweep-MSE), K contiguous, tiled scales, fp32 out"),
+            "vs_baseline": None, "dtype": "e2m1xe2m1->" + ("bf16" if out_bf16 else "f32"), "data": "synthetic",
+            "config": {"workload": workload,
                        "M": M, "N": N, "K": K, "parallelism": f"replicas{world}" if world > 1 else "single",
                        "l2": "operands 46 MB stay L2-resident across steps (a GEMM reuses them by design)",
                        "timing": "CUDA events around back-to-back launches on one stream"},
@@ -893,7 +983,7 @@ def run_gemm(args, rank, world):
                          "frac": round(tf / peak, 4), "traffic": profiled_traffic(f"{args.workload}:gemm", GEMM_SOURCES),
                          "kernel": f"fp4_gemm_kernel<{'true' if mx else 'false'}>",
                          "peak_source": peak_src},
-            "device_status": st, "gpu_launches": steps, "clocks": clk.summary(),
+            "device_status": st, "gpu_launches": steps * (3 if dyn else 1), "clocks": clk.summary(),
             "e2e": {"value": round(flops / (e2e_ms * 1e-3) / 1e12 * world, 3), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": int(sum(h.numel() * h.element_size() for h in hosts)),
                     "d2h_bytes_per_step": M * N * 4, "ms_per_step": round(e2e_ms, 3), "steps": e_steps,

@@ -462,9 +462,9 @@ __device__ __forceinline__ void fixed_point(const u64 (&xp)[NP], int k, Fixed16<
 }
 
 // 2m of the E2M1 codes of four quotients (bytes in element order): two conversions to E2M1 (round
-// to nearest even, saturating, sign in bit 3 of each code) and one byte-permute lookup of the
-// magnitude index.  ABS: the quotients are magnitudes, so the sign bits are already clear;
-// otherwise they are masked off first.
+// to nearest even, saturating, sign in bit 3 of each code), the two code bytes joined over a zero
+// high half into the selector, and one byte-permute lookup of the magnitude index.  ABS: the
+// quotients are magnitudes, so the sign bits are clear; otherwise they are masked off first.
 template <bool ABS>
 __device__ __forceinline__ uint32_t mags4_fp4(u64 y01, u64 y23) {
     float y0, y1, y2, y3;
@@ -472,19 +472,21 @@ __device__ __forceinline__ uint32_t mags4_fp4(u64 y01, u64 y23) {
     upk(y23, y2, y3);
     uint32_t m;
     if (ABS) {
-        asm("{ .reg .b8 c0, c1; .reg .b16 h; .reg .b32 s;\n"
+        asm("{ .reg .b8 c0, c1; .reg .b16 h0, h1; .reg .b32 s;\n"
             "  cvt.rn.satfinite.e2m1x2.f32 c0, %2, %1;\n"
             "  cvt.rn.satfinite.e2m1x2.f32 c1, %4, %3;\n"
-            "  mov.b16 h, {c0, c1};\n"
-            "  cvt.u32.u16 s, h;\n"
+            "  mov.b16 h0, {c0, c1};\n"
+            "  mov.b16 h1, 0;\n"
+            "  mov.b32 s, {h0, h1};\n"
             "  prmt.b32 %0, %5, %6, s; }"
             : "=r"(m) : "f"(y0), "f"(y1), "f"(y2), "f"(y3), "r"(kLutE2M1Lo), "r"(kLutE2M1Hi));
     } else {
-        asm("{ .reg .b8 c0, c1; .reg .b16 h; .reg .b32 s;\n"
+        asm("{ .reg .b8 c0, c1; .reg .b16 h0, h1; .reg .b32 s;\n"
             "  cvt.rn.satfinite.e2m1x2.f32 c0, %2, %1;\n"
             "  cvt.rn.satfinite.e2m1x2.f32 c1, %4, %3;\n"
-            "  mov.b16 h, {c0, c1};\n"
-            "  cvt.u32.u16 s, h;\n"
+            "  mov.b16 h0, {c0, c1};\n"
+            "  mov.b16 h1, 0;\n"
+            "  mov.b32 s, {h0, h1};\n"
             "  and.b32 s, s, 0x7777;\n"
             "  prmt.b32 %0, %5, %6, s; }"
             : "=r"(m) : "f"(y0), "f"(y1), "f"(y2), "f"(y3), "r"(kLutE2M1Lo), "r"(kLutE2M1Hi));
@@ -626,9 +628,10 @@ __device__ __forceinline__ void block_ctx(const u64 (&xp)[8], float ab, float S,
 }
 
 // Exact comparison of the candidates in `mask` (bit c = window offset c, INT4 at odd bits when
-// TWO_TYPES), their sums recomputed; the lowest index wins a tie.  ABS: c.xp holds magnitudes.
+// TWO_TYPES), their sums recomputed; the lowest index wins a tie.  The branch that reaches it is
+// rare; inlined, it needs no call frame and no spills around a call.  ABS: c.xp holds magnitudes.
 template <bool B16, bool TWO_TYPES, bool ABS>
-__device__ __noinline__ int exact_pick(const BlockCtx<B16>& c, const float2* t, uint32_t mask, float K76, float K67) {
+__device__ __forceinline__ int exact_pick(const BlockCtx<B16>& c, const float2* t, uint32_t mask, float K76, float K67) {
     int best = -1;
     ExactG bg = {0.0, 0.0};
     for (; mask; mask &= mask - 1) {
@@ -657,13 +660,11 @@ __device__ __noinline__ int exact_pick(const BlockCtx<B16>& c, const float2* t, 
 
 // The window search of the NVFP4 MSE sweep (offsets 0..NOFF-1 from table entry t = base + p0 - 3)
 // or of the IF4 sweep (TWO_TYPES: FP4 and INT4 at each offset, FP4 first); returns the winning
-// index.  SLOTS (B16 single-type only): per-thread shared memory `slot` keeps each candidate's
-// exact sums, slot[i * kThreads], which the exact decision then reads instead of recomputing.
-// ABS: c.xp holds magnitudes.
-template <bool B16, bool TWO_TYPES, int NOFF, bool SLOTS = false, bool ABS = false>
-__device__ __forceinline__ int window_search(const BlockCtx<B16>& c, const float2* t, float K76, float K67,
-                                             uint2* slot = nullptr) {
-    static_assert(!SLOTS || (B16 && !TWO_TYPES), "slots hold one 32-bit X per candidate");
+// index.  Each candidate's fast score is kept; only when another candidate lies within the
+// margin of the smallest are the close ones' sums recomputed and compared exactly.  ABS: c.xp
+// holds magnitudes.
+template <bool B16, bool TWO_TYPES, int NOFF, bool ABS = false>
+__device__ __forceinline__ int window_search(const BlockCtx<B16>& c, const float2* t, float K76, float K67) {
     constexpr int N = TWO_TYPES ? 2 * NOFF : NOFF;
     float g[N];
 #pragma unroll
@@ -675,7 +676,6 @@ __device__ __forceinline__ int window_search(const BlockCtx<B16>& c, const float
         for (int b = 0; b < (B16 ? 1 : 4); ++b) x[b] = B16 ? kMagicInt : 0u;
         cand_sums<B16, false, 8, ABS>(c.xp, c.A, e.x, K76, q, x);
         g[TWO_TYPES ? 2 * o : o] = fast_G<B16>(s4, q, x);
-        if constexpr (SLOTS) slot[o * kThreads] = make_uint2(q, x[0]);
         if (TWO_TYPES) {
             const float s4i = __fmul_rn(K67, s4);
             q = B16 ? kMagicInt : 0u;
@@ -687,24 +687,7 @@ __device__ __forceinline__ int window_search(const BlockCtx<B16>& c, const float
     }
     const int unique = near_min_unique<N>(g);
     if (unique >= 0) return unique;
-    uint32_t mask = near_min_mask<N>(g);
-    if constexpr (SLOTS) {
-        int best = -1;
-        ExactG bg = {0.0, 0.0};
-        for (; mask; mask &= mask - 1) {
-            const int i = __ffs(mask) - 1;
-            const uint2 qx = slot[i * kThreads];
-            const uint32_t x1[1] = {qx.y};
-            const ExactG eg = exact_G<true>(__fmul_rn(t[i].y, c.T), qx.x, x1);
-            if (best < 0 || exact_less(eg, bg)) {
-                bg = eg;
-                best = i;
-            }
-        }
-        return best;
-    } else {
-        return exact_pick<B16, TWO_TYPES, ABS>(c, t, mask, K76, K67);
-    }
+    return exact_pick<B16, TWO_TYPES, ABS>(c, t, near_min_mask<N>(g), K76, K67);
 }
 
 // Packed codes of a block (signed values xp) at reciprocal scale inv: 8 bytes, elements 0..15.
@@ -759,12 +742,12 @@ __device__ __forceinline__ float wmse_error(const u64 (&ap)[8], const u64 (&wp)[
 // (gist.science/ko/paper/2606.07618), Methodology; 4/6: Adaptive Block-Scaled Data Types
 // (gist.science/ko/paper/2603.28765), Problem.
 // ------------------------------------------------------------------------------------------
-// SLOTS: `slot` points at this thread's shared-memory slots for the sweep's exact sums.
-// ABS: xp holds the magnitudes and sgn the sign bits at their code positions (bit 4 i + 3).
-template <int OBJ, bool B16, bool SLOTS, bool ABS>
+// ABS (the MSE sweep): xp holds the magnitudes and sgn the sign bits at their code positions
+// (bit 4 i + 3), put back into the codes at the end.
+template <int OBJ, bool B16, bool ABS>
 __device__ __forceinline__ void nvfp4_block(const u64 (&xp)[8], uint2 sgn, const float* __restrict__ imp,
                                             int64_t colblk, float S, float d6, float d4, const float2* tab,
-                                            uint2* cdst, uint8_t* sdst, uint2* slot) {
+                                            uint2* cdst, uint8_t* sdst) {
     static_assert(!ABS || OBJ == FP4Q_SWEEP_MSE, "magnitude inputs serve the MSE sweep");
     int bp = 0;
     if (S > 0.0f) {
@@ -794,7 +777,7 @@ __device__ __forceinline__ void nvfp4_block(const u64 (&xp)[8], uint2 sgn, const
             if (__fmul_rn(ab, 0x1p11f) >= S) {
                 BlockCtx<B16> c;
                 block_ctx<B16>(xp, ab, S, c);
-                bp = p0 - 3 + window_search<B16, false, 11, SLOTS && B16, ABS>(c, tab + p0 - 3, 0.0f, 0.0f, slot);
+                bp = p0 - 3 + window_search<B16, false, 11, ABS>(c, tab + p0 - 3, 0.0f, 0.0f);
             }
         } else if (OBJ == FP4Q_SWEEP_WMSE) {
             // candidates p0 - 8 .. p0 + 7 in increasing offset with strict improvement (ties keep
@@ -887,10 +870,10 @@ __device__ __forceinline__ void if4_block(const u64 (&xp)[8], float S, float d6,
 // The NVFP4 / IF4 quantize kernel (KIND = the NVFP4 objective, or KIND_IF4).  Each thread
 // walks the blocks tid, tid + G, ... (G threads in the grid) with the next block's loads in
 // flight while the current one is searched; the CTA builds its scale table once.  The host
-// picks the grid per kind: one block per thread (G >= blocks: the loop runs once) for the
-// ScaleSweep searches, one persistent wave for the light IF4 / AbsMax / 4-6 kinds, whose
-// per-CTA start-up (S, table, first loads) would otherwise not be amortized.  The status
-// word depends only on S, so CTA 0 writes it.
+// picks the grid per kind: one block per thread (G >= blocks: the loop runs once) for the WMSE
+// search, one persistent wave (the CTAs that fit on the SMs) for the other kinds, whose per-CTA
+// start-up (S, table, first loads) would otherwise not be amortized.  The status word depends
+// only on S, so CTA 0 writes it.
 // ------------------------------------------------------------------------------------------
 enum : int { KIND_IF4 = 4, KIND_IF4_SWEEP = 5 };   // kinds 0..3 are the NVFP4 objectives
 
@@ -909,9 +892,6 @@ __global__ void __launch_bounds__(kThreads, q16_min_ctas<KIND>())
                uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, const float* __restrict__ gscale,
                uint32_t* __restrict__ ws, int tiled) {
     __shared__ float2 s_tab[kTabLen];
-    // exact sums of each thread's 11 sweep candidates (bf16 MSE sweep only), for the rare exact decision
-    constexpr bool kSlots = KIND == FP4Q_SWEEP_MSE && IN == FP4Q_IN_BF16 && !HAD;
-    __shared__ uint2 s_slot[kSlots ? 11 * kThreads : 1];
     const IDX nb = cols / 16;
     const IDX total = rows * nb;
     const IDX G = (IDX)gridDim.x * blockDim.x;
@@ -937,15 +917,40 @@ __global__ void __launch_bounds__(kThreads, q16_min_ctas<KIND>())
             return;
         }
         if (IN != FP4Q_IN_BF16) load_raw16<IN>(xv, at.xoff, rb);
+        // the MSE sweep searches on magnitudes and puts the signs back into the codes at the end
+        constexpr bool kAbs = KIND == FP4Q_SWEEP_MSE;
+        constexpr bool kRawSigns = kAbs && IN == FP4Q_IN_BF16 && !HAD;
         u64 xp[8];
-        unpack16<IN>(rb, xp);
+        uint2 sgn = make_uint2(0u, 0u);
+        if constexpr (kRawSigns) {
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const uint4 v = rb.v[q];
+                (q ? sgn.y : sgn.x) = bf16_sign_nibbles8(v.x, v.y, v.z, v.w);
+                xp[4 * q] = bf16x2_to_abs_pair(v.x);
+                xp[4 * q + 1] = bf16x2_to_abs_pair(v.y);
+                xp[4 * q + 2] = bf16x2_to_abs_pair(v.z);
+                xp[4 * q + 3] = bf16x2_to_abs_pair(v.w);
+            }
+        } else {
+            unpack16<IN>(rb, xp);
+        }
         if (q16_persistent<KIND>() && IN == FP4Q_IN_BF16 && b + G < total)   // next block's loads in flight
             load_raw16<IN>(xv, block_at<IDX, false>(b + G, cols, ld, nb).xoff, rb);
         if (HAD) fwht16(xp);
+        if constexpr (kAbs && !kRawSigns) {
+            sgn = make_uint2(f32_sign_nibbles8(xp[0], xp[1], xp[2], xp[3]), f32_sign_nibbles8(xp[4], xp[5], xp[6], xp[7]));
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                float a0, a1;
+                upk(xp[j], a0, a1);
+                xp[j] = pk(fabsf(a0), fabsf(a1));
+            }
+        }
         constexpr bool B16 = IN == FP4Q_IN_BF16 && !HAD;   // bf16 values: 15-bit fixed point
         if (KIND == KIND_IF4) if4_block<false, B16>(xp, S, d6, K76, K67, tab, cdst, sdst);
         else if (KIND == KIND_IF4_SWEEP) if4_block<true, B16>(xp, S, d6, K76, K67, tab, cdst, sdst);
-        else nvfp4_block<KIND, B16, kSlots, false>(xp, make_uint2(0u, 0u), imp, at.b, S, d6, d4, tab, cdst, sdst, s_slot + threadIdx.x);
+        else nvfp4_block<KIND, B16, kAbs>(xp, sgn, imp, at.b, S, d6, d4, tab, cdst, sdst);
     };
     if (q16_persistent<KIND>()) {
         for (; blk < total; blk += G) one_block(blk);

@@ -165,7 +165,6 @@ __device__ __forceinline__ uint32_t f32_sign_nibbles8(u64 p0, u64 p1, u64 p2, u6
     const uint32_t od = __byte_perm(__byte_perm(u[1], u[3], 0x0073), __byte_perm(u[5], u[7], 0x0073), 0x5410);
     return ((ev >> 4) & 0x08080808u) | (od & 0x80808080u);
 }
-
 // 2^k as a float for k in [-127, 127] (2^-127 is subnormal).
 __device__ __forceinline__ float pow2i(int k) {
     return k >= -126 ? __int_as_float((k + 127) << 23) : __int_as_float(0x00400000);
