@@ -25,4 +25,4 @@ def test_algorithmic_bytes_match_the_contract(rows, cols, fmt, in_bytes, wmse, w
 def test_every_bench_workload_has_a_shape_and_method():
     for name, (cfg, fmt, obj, desc) in bench.WORKLOADS.items():
         assert cfg.startswith("cfg") and fmt and desc
-    assert "cfg3" in bench.WORKLOADS and set(bench.GEMM_WORKLOADS) == {"gemm", "gemm_mx"}
+    assert "cfg3" in bench.WORKLOADS and set(bench.GEMM_WORKLOADS) == {"gemm", "gemm_mx", "gemm_bf16", "gemm_dyn"}
