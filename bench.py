@@ -47,6 +47,9 @@ WORKLOADS = {
               "NVFP4 ScaleSweep-MSE on 16x16 block-Hadamard-rotated blocks, bf16 activations 8192x4096, "
               "dynamic S of the rotated tensor"),
     "cfg4h": ("cfg4", "if4_had", None, "IF4 on 16x16 block-Hadamard-rotated blocks, bf16 weight 4096x14336"),
+    "cfg4i6": ("cfg4", "if6", None,
+               "IF6 per-block FP6 (E2M3) / scaled INT6 selection, 6-bit codes, S = amax/1920, bf16 weight "
+               "4096x14336, 0.02*t4"),
     # the NVFP4 operator ScaleSweep measures its overhead against: AbsMax on the same tensor
     "cfg3_absmax": ("cfg3", "nvfp4", "absmax",
                     "NVFP4 AbsMax (one scale per block, no search) dynamic activation quantization, bf16 8192x4096, "
@@ -94,10 +97,15 @@ def split_fmt(fmt):
 L2_BYTES = 126 * 2 ** 20
 
 
+def code_bytes(n, fmt):
+    """Bytes of packed element codes for n elements: 4 bits (FP4 formats) or 6 bits (IF6)."""
+    return n * 3 // 4 if fmt == "if6" else n // 2
+
+
 def algorithmic_bytes(rows, cols, fmt, in_bytes=2, wmse=False):
     B = 32 if fmt.startswith("mxfp4") else 16
     n = rows * cols
-    b = n * in_bytes + n // 2 + n // B
+    b = n * in_bytes + code_bytes(n, fmt) + n // B
     if not fmt.startswith("mxfp4"):
         b += 4
     if wmse:
@@ -217,6 +225,8 @@ def _oracle_rows(args):
         O.nvfp4_quantize(xs, obj, importance=imp, hadamard16=had16)
     elif base == "if4":
         O.if4_quantize(xs, hadamard16=had16, sweep="sweep" if obj == "if4_sweep" else "absmax")
+    elif base == "if6":
+        O.if6_quantize(xs)
     else:
         O.mxfp4_quantize(xs, hadamard=fmt.endswith("had"), sweep="sweep" if obj == "mx_sweep" else "rule")
     return xs.shape[0]
@@ -272,6 +282,8 @@ def cpu_baseline(w, fmt, obj, budget_s=12.0, S=None, gpu=None):
             r = O.nvfp4_quantize(xs, obj, importance=imp, hadamard16=had16, S=S)
         elif base == "if4":
             r = O.if4_quantize(xs, hadamard16=had16, sweep="sweep" if obj == "if4_sweep" else "absmax", S=S)
+        elif base == "if6":
+            r = O.if6_quantize(xs, S=S)
         else:
             r = O.mxfp4_quantize(xs, hadamard=fmt.endswith("had"), sweep="sweep" if obj == "mx_sweep" else "rule")
         results.append(r)
@@ -286,15 +298,17 @@ def cpu_baseline(w, fmt, obj, budget_s=12.0, S=None, gpu=None):
         osc = np.concatenate([r["scales"] for r in results])
         gc, gsc = gpu[0][:done], gpu[1][:done]
         B = 32 if fmt.startswith("mxfp4") else 16
-        bad = (gsc != osc) | (gc.reshape(done, -1, B // 2) != oc.reshape(done, -1, B // 2)).any(axis=2)
+        cb = code_bytes(B, base)   # code bytes per block
+        bad = (gsc != osc) | (gc.reshape(done, -1, cb) != oc.reshape(done, -1, cb)).any(axis=2)
         near = O.near_ties({k: np.concatenate([r[k] for r in results]) for k in ("gap", "tie")})
         dfmt = "mxfp4" if fmt.startswith("mxfp4") else base
         xr = O.rotate16(x[:done]) if had16 else x[:done]
         if fmt.startswith("mxfp4") and fmt.endswith("had"):
             xr = np.stack([O.hadamard32(v) for v in x[:done].reshape(-1, 32)]).reshape(done, cols)
         Sd = 0.0 if S is None else S
-        mse_o = float(np.mean((xr.astype(np.float64) - O.dequantize(oc, osc, Sd, dfmt).astype(np.float64)) ** 2))
-        mse_g = float(np.mean((xr.astype(np.float64) - O.dequantize(gc, gsc, Sd, dfmt).astype(np.float64)) ** 2))
+        deq = (lambda c, sc: O.if6_dequantize(c, sc, Sd)) if base == "if6" else (lambda c, sc: O.dequantize(c, sc, Sd, dfmt))
+        mse_o = float(np.mean((xr.astype(np.float64) - deq(oc, osc).astype(np.float64)) ** 2))
+        mse_g = float(np.mean((xr.astype(np.float64) - deq(gc, gsc).astype(np.float64)) ** 2))
         out["parity"] = {"rows_checked": done, "blocks_checked": int(bad.size), "mismatching_blocks": int(bad.sum()),
                          "bit_exact": bool(not bad.any()),
                          "near_tie_frac": round(near["near_frac"], 6), "near_tie_blocks": near["near"],
@@ -331,6 +345,8 @@ def run_reference(args, rank, world):
             O.nvfp4_quantize(xs, obj, importance=imp, hadamard16=had16)
         elif base == "if4":
             O.if4_quantize(xs, hadamard16=had16, sweep="sweep" if obj == "if4_sweep" else "absmax")
+        elif base == "if6":
+            O.if6_quantize(xs)
         else:
             O.mxfp4_quantize(xs, hadamard=fmt.endswith("had"), sweep="sweep" if obj == "mx_sweep" else "rule")
 
@@ -408,7 +424,7 @@ def run_ours(args, rank, world):
     x_host = device_tensor_from_bits(w["x"], torch)
     in_bytes = x_host.numel() * 2
     alg = algorithmic_bytes(rows, cols, fmt, wmse=(obj == "sweep_wmse"))
-    out_bytes = rows * cols // 2 + rows * cols // (32 if fmt.startswith("mxfp4") else 16)
+    out_bytes = code_bytes(rows * cols, fmt) + rows * cols // (32 if fmt.startswith("mxfp4") else 16)
     nsets = max(2, int(np.ceil(3.0 * L2_BYTES / (in_bytes + out_bytes))))
     xs = [x_host.to(dev) for _ in range(nsets)]
     base, had16 = split_fmt(fmt)
@@ -433,8 +449,14 @@ def run_ours(args, rank, world):
                         workspace=wss[s], hadamard16=had16, if4_sweep=(obj == "if4_sweep"))
         return 1
 
+    if fmt == "if6":   # its own tensor scale (amax / 1920): one public call runs the amax pass and the quantizer
+        def quant(s):
+            c, sc, g = outs[s]
+            fq.quantize(xs[s], "if6", out=(c, sc, g), workspace=wss[s])
+            return 2
+
     def step(s):
-        return (0 if fmt.startswith("mxfp4") else amax(s)) + quant(s)
+        return (0 if fmt.startswith("mxfp4") or fmt == "if6" else amax(s)) + quant(s)
 
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
@@ -453,7 +475,7 @@ def run_ours(args, rank, world):
     # costs several microseconds): one per buffer set, for a remainder of steps, and one that
     # runs every set once in turn
     graphs = [capture(lambda s=s: step(s)) for s in range(nsets)]
-    two_pass = not fmt.startswith("mxfp4")
+    two_pass = not (fmt.startswith("mxfp4") or fmt == "if6")
     side = torch.cuda.Stream(device=dev)
 
     def pipelined_cycle():
@@ -550,7 +572,7 @@ def run_ours(args, rank, world):
         return a.elapsed_time(b) / kernel_reps
 
     t_q = time_kernel(quant)
-    t_amax = None if fmt.startswith("mxfp4") else time_kernel(amax)
+    t_amax = None if not two_pass else time_kernel(amax)
 
     # per-step distribution: up to 200 steps, each between its own pair of CUDA events on the
     # stream (the buffer sets in turn)
@@ -671,7 +693,7 @@ def run_ours(args, rank, world):
         if S_gpu is not None:
             import oracle as O
             xo = O.widen_bf16(w["x"]) if w["dtype"] == "bf16" else w["x"]
-            S_o = O.tensor_scale(O.rotate16(xo) if had16 else xo)[0]
+            S_o = O.if6_tensor_scale(xo) if base == "if6" else O.tensor_scale(O.rotate16(xo) if had16 else xo)[0]
             line["parity"]["S_bit_exact"] = bool(np.float32(S_o).view(np.uint32) == np.float32(S_gpu).view(np.uint32))
         line["cpu_baseline"] = cpu_baseline_all_cores(w, fmt, obj, budget_s=args.cpu_seconds / 2)
         line["cpu_baseline"]["single_core"] = single

@@ -531,6 +531,70 @@ __device__ __forceinline__ void cand_sums(const u64 (&xp)[NP], const Fixed16<B16
     }
 }
 
+// IF4 at one scale, bf16 values.  The FP4 sums of cand_sums, and the block's signed E2M1 code word
+// (the conversions the sums already made, before their sign bits are masked off).
+__device__ __forceinline__ uint2 fp4_sums_codes(const u64 (&xp)[8], const Fixed16<true>& A, float inv, uint32_t& q,
+                                                uint32_t& x) {
+    const u64 inv2 = pk(inv, inv);
+    uint32_t h[4];
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+        float y0, y1, y2, y3;
+        upk(mul2(xp[2 * g], inv2), y0, y1);
+        upk(mul2(xp[2 * g + 1], inv2), y2, y3);
+        uint32_t m4;
+        asm("{ .reg .b8 c0, c1; .reg .b16 h0, h1; .reg .b32 t;\n"
+            "  cvt.rn.satfinite.e2m1x2.f32 c0, %3, %2;\n"
+            "  cvt.rn.satfinite.e2m1x2.f32 c1, %5, %4;\n"
+            "  mov.b16 h0, {c0, c1};\n"
+            "  mov.b16 h1, 0;\n"
+            "  mov.b32 %1, {h0, h1};\n"
+            "  and.b32 t, %1, 0x7777;\n"
+            "  prmt.b32 %0, %6, %7, t; }"
+            : "=r"(m4), "=r"(h[g]) : "f"(y0), "f"(y1), "f"(y2), "f"(y3), "r"(kLutE2M1Lo), "r"(kLutE2M1Hi));
+        q = __dp4a(m4, m4, q);
+        x = __dp2a_lo(A.w[2 * g], m4, x);
+        x = __dp2a_hi(A.w[2 * g + 1], m4, x);
+    }
+    return make_uint2(__byte_perm(h[0], h[1], 0x5410), __byte_perm(h[2], h[3], 0x5410));
+}
+
+// IF4 at one scale, bf16 values: the INT4 sums in binary32 and the block's INT4 code word.
+// n = rint(RN(RN(x inv) RN(7/6))) rides in the low mantissa bits of v = RN(z + 1.5 2^23), clamped
+// to [-7, 7] when CLAMP (at a normal, unsaturated base pattern |y| <= 6.4 (1 + 2^-21): the E4M3
+// rounding of a_b / RN(6 S) is within 1/16, so |z| stays below 7.5 and it needs none); the low
+// nibble of v's bits is n's two's complement code.  xs = sum x n and qs = sum n^2 are exact in
+// binary32: every product x n with n != 0 is a multiple of ulp(a_b) 2^-4 (|x| >= a_b / 15 there,
+// and x has 8 significant bits) and the sum stays below 2^19 such units.  In the fixed point of
+// the FP4 sums (A = |x| 2^k, M = 2|n|): X = 2^(k+1) xs and Q4 = 4 qs.
+template <bool CLAMP>
+__device__ __forceinline__ uint2 int4_sums_f(const u64 (&xp)[8], float inv, float K76, float& qs, float& xs) {
+    const u64 inv2 = pk(inv, inv), mag2 = pk(kRintMagic, kRintMagic);
+    u64 xa = 0ull, qa = 0ull;   // +0.0f pairs
+    uint32_t cw[2] = {0u, 0u};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        float y0, y1;
+        upk(mul2(xp[j], inv2), y0, y1);
+        float v0 = __fadd_rn(__fmul_rn(y0, K76), kRintMagic), v1 = __fadd_rn(__fmul_rn(y1, K76), kRintMagic);
+        if (CLAMP) {
+            v0 = fminf(fmaxf(v0, kRintMagic - 7.0f), kRintMagic + 7.0f);
+            v1 = fminf(fmaxf(v1, kRintMagic - 7.0f), kRintMagic + 7.0f);
+        }
+        const u64 n2 = sub2(pk(v0, v1), mag2);   // exact
+        xa = fma2(xp[j], n2, xa);
+        qa = fma2(n2, n2, qa);
+        const uint32_t byte = (__float_as_uint(v0) & 0xFu) | ((__float_as_uint(v1) & 0xFu) << 4);
+        cw[j >> 2] |= byte << (8 * (j & 3));
+    }
+    float a, b;
+    upk(xa, a, b);
+    xs = __fadd_rn(a, b);
+    upk(qa, a, b);
+    qs = __fadd_rn(a, b);
+    return make_uint2(cw[0], cw[1]);
+}
+
 // The fast score G~ of a candidate from its sums, and its exact value in binary64.
 template <bool B16>
 __device__ __forceinline__ float fast_G(float s4, uint32_t q, const uint32_t (&x)[B16 ? 1 : 4]) {
@@ -559,6 +623,15 @@ __device__ __forceinline__ ExactG exact_G(float s4, uint32_t q, const uint32_t (
     }
     const double s = (double)s4;
     const double u = __fma_rn(s, q4, -xi);   // exact: fewer than 45 significant bits
+    ExactG g;
+    g.hi = __dmul_rn(s, u);
+    g.lo = __fma_rn(s, u, -g.hi);
+    return g;
+}
+// The same from the binary32 INT4 sums of int4_sums_f (Q4 = 4 qs, X = 2^(k+1) xs, both exact).
+__device__ __forceinline__ ExactG exact_G_int4f(float s4, float qs, float xs, int k) {
+    const double s = (double)s4;
+    const double u = __fma_rn(s, 4.0 * (double)qs, -ldexp((double)xs, k + 1));   // exact, as in exact_G
     ExactG g;
     g.hi = __dmul_rn(s, u);
     g.lo = __fma_rn(s, u, -g.hi);
@@ -611,6 +684,7 @@ struct BlockCtx {
     u64 xp[8];          // the block's values (pairs); the searches use their magnitudes
     Fixed16<B16> A;
     float T;            // S 2^(k-2): sigma4 of pattern p is RN(e(p) T) = sv(p) 2^(k-2)
+    int k;              // the fixed-point shift: A = |x| 2^k
 };
 
 template <bool B16>
@@ -625,6 +699,7 @@ __device__ __forceinline__ void block_ctx(const u64 (&xp)[8], float ab, float S,
     float fa, fb;
     pow2_split(k - 2, fa, fb);
     c.T = __fmul_rn(__fmul_rn(S, fa), fb);
+    c.k = k;
 }
 
 // Exact comparison of the candidates in `mask` (bit c = window offset c, INT4 at odd bits when
@@ -690,14 +765,27 @@ __device__ __forceinline__ int window_search(const BlockCtx<B16>& c, const float
     return exact_pick<B16, TWO_TYPES, ABS>(c, t, near_min_mask<N>(g), K76, K67);
 }
 
-// Packed codes of a block (signed values xp) at reciprocal scale inv: 8 bytes, elements 0..15.
+// Packed codes of a block (signed values xp) at reciprocal scale inv: 8 bytes, elements 0..15; the
+// code bytes of each 8 elements are joined with two half-word packs.
 __device__ __forceinline__ uint2 block_codes(const u64 (&xp)[8], float inv) {
     const u64 inv2 = pk(inv, inv);
-    uint32_t c[8];
+    uint32_t w[2];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) c[j] = e2m1x2(mul2(xp[j], inv2));
-    return make_uint2(c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24),
-                      c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24));
+    for (int h = 0; h < 2; ++h) {
+        float y[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) upk(mul2(xp[4 * h + j], inv2), y[2 * j], y[2 * j + 1]);
+        asm("{ .reg .b8 c0, c1, c2, c3; .reg .b16 h0, h1;\n"
+            "  cvt.rn.satfinite.e2m1x2.f32 c0, %2, %1;\n"
+            "  cvt.rn.satfinite.e2m1x2.f32 c1, %4, %3;\n"
+            "  cvt.rn.satfinite.e2m1x2.f32 c2, %6, %5;\n"
+            "  cvt.rn.satfinite.e2m1x2.f32 c3, %8, %7;\n"
+            "  mov.b16 h0, {c0, c1};\n"
+            "  mov.b16 h1, {c2, c3};\n"
+            "  mov.b32 %0, {h0, h1}; }"
+            : "=r"(w[h]) : "f"(y[0]), "f"(y[1]), "f"(y[2]), "f"(y[3]), "f"(y[4]), "f"(y[5]), "f"(y[6]), "f"(y[7]));
+    }
+    return make_uint2(w[0], w[1]);
 }
 // INT4 codes of a block at reciprocal scale inv: n = clamp(rint(RN(RN(x inv) RN(7/6))), -7, 7) as
 // 4-bit two's complement nibbles (the low bits of 1.5 2^23 + n).
@@ -842,17 +930,32 @@ __device__ __forceinline__ void if4_block(const u64 (&xp)[8], float S, float d6,
                 const int i = window_search<B16, true, 11>(c, tab + p0 - 3, K76, K67);
                 bp = p0 - 3 + (i >> 1);
                 use_int = (i & 1) != 0;
+            } else if constexpr (B16) {
+                // both element types at p0, each type's codes taken from its own evaluation
+                const float2 e = tab[p0];
+                const float s4 = __fmul_rn(e.y, c.T);
+                uint32_t q = kMagicInt, x[1] = {kMagicInt};
+                const uint2 cw_fp = fp4_sums_codes(c.xp, c.A, e.x, q, x[0]);
+                const ExactG gf = exact_G<true>(s4, q, x);
+                float qs, xs;
+                // below pattern 8 (subnormal) and at 126 (where a_b / RN(6 S) may exceed the largest
+                // E4M3 value when S is given) |y| can pass 6.4, so the INT4 codes are clamped there
+                const uint2 cw_int = p0 >= 8 && p0 < 126 ? int4_sums_f<false>(c.xp, e.x, K76, qs, xs)
+                                                         : int4_sums_f<true>(c.xp, e.x, K76, qs, xs);
+                const ExactG gi = exact_G_int4f(__fmul_rn(K67, s4), qs, xs, c.k);
+                use_int = exact_less(gi, gf);
+                *cdst = use_int ? cw_int : cw_fp;
+                *sdst = (uint8_t)(bp | (use_int ? 0x80 : 0));
+                return;
             } else {
                 const float2 e = tab[p0];
                 const float s4 = __fmul_rn(e.y, c.T);
-                uint32_t q = B16 ? kMagicInt : 0u, x[B16 ? 1 : 4];
-#pragma unroll
-                for (int b = 0; b < (B16 ? 1 : 4); ++b) x[b] = B16 ? kMagicInt : 0u;
+                uint32_t q = 0u, x[4] = {0u, 0u, 0u, 0u};
                 cand_sums<B16, false>(c.xp, c.A, e.x, K76, q, x);
                 const ExactG gf = exact_G<B16>(s4, q, x);
-                q = B16 ? kMagicInt : 0u;
+                q = 0u;
 #pragma unroll
-                for (int b = 0; b < (B16 ? 1 : 4); ++b) x[b] = B16 ? kMagicInt : 0u;
+                for (int b = 0; b < 4; ++b) x[b] = 0u;
                 cand_sums<B16, true>(c.xp, c.A, e.x, K76, q, x);
                 const ExactG gi = exact_G<B16>(__fmul_rn(K67, s4), q, x);
                 use_int = exact_less(gi, gf);

@@ -275,6 +275,12 @@ def e2m3_encode(y: float) -> int:
     return lib().fp4q_o_e2m3_encode(float(y))
 
 
+def if6_tensor_scale(x) -> float:
+    """IF6's tensor scale of a whole float32 tensor: S = RN(max|x| / 1920) (finite tensors)."""
+    x = _f32(x)
+    return float(lib().fp4q_o_global_scale_if6(float(np.max(np.abs(x))) if x.size else 0.0))
+
+
 def if6_quantize(x, S=None):
     """IF6 (FP6 E2M3 or scaled INT6 per 16-element block, indicator in bit 7 of the E4M3 scale
     byte): packed 6-bit codes [rows, cols * 3/4], scale bytes [rows, cols/16], S = RN(amax / 1920)
