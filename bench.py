@@ -656,7 +656,7 @@ def run_ours(args, rank, world):
         "config": {"workload": desc, "rows": rows, "cols": cols, "input_dtype": w["dtype"],
                    "method": obj or fmt, "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": f"{nsets} rotating input/output buffer sets, {nsets * (in_bytes + out_bytes) / 2**20:.0f} MB "
-                         f"total (> 2x the 126 MB L2)",
+                         f"total (at least 3x the 126 MB L2)",
                    "timing": ("CUDA graph over the buffer sets (no timing nodes inside); each step's amax pass runs on "
                               "a second stream under the previous step's quantize kernel, each quantize after its own "
                               "amax; CUDA events on the launching stream" if two_pass else

@@ -1079,6 +1079,26 @@ __device__ __forceinline__ uint32_t e2m3_m8(uint32_t c) {
     return e == 0 ? f : (8u + f) << (e - 1);
 }
 
+// 8m of the FP6 codes of four non-negative quotients (bytes in element order): two conversions to
+// E2M3, their decode to f16 pairs, RN(8 m + 1024) in f16 (exact: 8m is an integer below 64, so
+// the sum sits in [1024, 2048) where the f16 step is 1) leaves 8m in the low byte of each half,
+// and one byte permute gathers the four bytes.
+__device__ __forceinline__ uint32_t m8x4_fp6(float y0, float y1, float y2, float y3) {
+    uint32_t m;
+    asm("{ .reg .b16 c01, c23; .reg .b32 h01, h23, e8, k;\n"
+        "  cvt.rn.satfinite.e2m3x2.f32 c01, %2, %1;\n"
+        "  cvt.rn.satfinite.e2m3x2.f32 c23, %4, %3;\n"
+        "  cvt.rn.f16x2.e2m3x2 h01, c01;\n"
+        "  cvt.rn.f16x2.e2m3x2 h23, c23;\n"
+        "  mov.b32 e8, 0x48004800;\n"
+        "  mov.b32 k, 0x64006400;\n"
+        "  fma.rn.f16x2 h01, h01, e8, k;\n"
+        "  fma.rn.f16x2 h23, h23, e8, k;\n"
+        "  prmt.b32 %0, h01, h23, 0x6420; }"
+        : "=r"(m) : "f"(y0), "f"(y1), "f"(y2), "f"(y3));
+    return m;
+}
+
 template <bool B16>
 __device__ __forceinline__ void if6_block(const u64 (&xp)[8], float S, float d75, float K62, float K15,
                                           const float2* tab, uint8_t* cdst, uint8_t* sdst) {
@@ -1109,11 +1129,7 @@ __device__ __forceinline__ void if6_block(const u64 (&xp)[8], float S, float d75
             float y[4];
             upk(mul2(ap[2 * g], inv2), y[0], y[1]);
             upk(mul2(ap[2 * g + 1], inv2), y[2], y[3]);
-            uint16_t c01, c23;
-            asm("cvt.rn.satfinite.e2m3x2.f32 %0, %1, %2;" : "=h"(c01) : "f"(y[1]), "f"(y[0]));
-            asm("cvt.rn.satfinite.e2m3x2.f32 %0, %1, %2;" : "=h"(c23) : "f"(y[3]), "f"(y[2]));
-            const uint32_t mf = e2m3_m8(c01 & 0xFFu) | (e2m3_m8(c01 >> 8) << 8) | (e2m3_m8(c23 & 0xFFu) << 16) |
-                                (e2m3_m8(c23 >> 8) << 24);
+            const uint32_t mf = m8x4_fp6(y[0], y[1], y[2], y[3]);
             uint32_t t[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i)
@@ -1202,8 +1218,14 @@ __global__ void __launch_bounds__(kThreads, 4)
     const float K62 = __fdiv_rn(62.0f, 15.0f), K15 = __fdiv_rn(15.0f, 62.0f);
     for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < total;
          blk += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = blk / nb, b = blk - r * nb;
-        uint8_t* cdst = codes + r * (cols * 3 / 4) + b * 12;
+        // codes and scales are dense (12 bytes and 1 byte per block); the input row pitch needs
+        // the row index only when rows are padded
+        int64_t xoff = blk * 16;
+        if (ld != cols) {
+            const int64_t r = blk / nb;
+            xoff = r * ld + (blk - r * nb) * 16;
+        }
+        uint8_t* cdst = codes + blk * 12;
         uint8_t* sdst = scales + blk;
         if (flags) {   // data out of contract: zero-filled outputs
             reinterpret_cast<uint32_t*>(cdst)[0] = 0u;
@@ -1213,7 +1235,7 @@ __global__ void __launch_bounds__(kThreads, 4)
             continue;
         }
         RawBlock16<IN> rb;
-        load_raw16<IN>(xv, r * ld + b * 16, rb);
+        load_raw16<IN>(xv, xoff, rb);
         u64 xp[8];
         unpack16<IN>(rb, xp);
         if6_block<IN == FP4Q_IN_BF16>(xp, S, d75, K62, K15, tab, cdst, sdst);
