@@ -17,28 +17,39 @@
  *          Microscaling FP4 (gist.science/ko/paper/2509.23202), "Methodology"; scale rule
  *          "block maximum onto the largest codeword": TORQ (gist.science/ko/paper/
  *          2605.19561), "Method", S-step.
+ *   IF6    16-element blocks of 6-bit codes, per block the lower-MSE of FP6 (E2M3, largest
+ *          value 7.5) and scaled INT6 ([-31, 31], x 62/15 before rounding, x 15/62 on
+ *          dequantization), indicator in the scale byte's sign bit (1 = INT6): the IF4
+ *          construction at 6 bits, Adaptive Block-Scaled Data Types, "Methodology"
+ *          (extensibility to 6-bit types).
  *
- * Arithmetic (identical on every path; every step one binary32 operation rounded to
- * nearest even, no contraction, no flush-to-zero):
- *   S = RN(amax/1536); p0 = E4M3_RNE(RN(a_b / RN(6 S))); p4 = E4M3_RNE(RN(a_b / RN(4 S)));
- *   candidate p: sv = RN(e(p) S), inv = RN(1/sv) (sv = inv = 0 for p = 0);
- *   y = RN(x inv); q = E2M1_RNE_satfinite(y); r = RN(q - y) (the quantizer's rounding error
- *   in units of the scale); E = RN(acc_even + acc_odd), acc_par = fma(r, r, acc_par) over the
- *   block's even / odd positions in order (WMSE: fma(RN(w r), r, acc)); error = RN(RN(sv^2) E),
- *   i.e. the block MSE sum (x - q s)^2 = s^2 sum (x/s - q)^2 evaluated on the binary32
- *   quotient y; for p = 0 the error is the same fma sum over x itself.  The lowest offset
- *   wins a tie of the computed errors.
- *   IF4 INT4: z = RN(y RN(7/6)), n = clamp(rint(z), -7, 7), v = RN(n RN(6/7)),
- *   r = RN(v - y); both paths share s, so INT4 iff E_int < E_fp.
+ * Arithmetic (identical on every path).  RN is one binary32 operation rounded to nearest even,
+ * with no contraction and no flush-to-zero:
+ *   S = RN(amax/1536) (IF6: RN(amax/1920)); p0 = E4M3_RNE(RN(a_b / RN(6 S))) (IF6: RN(7.5 S));
+ *   p4 = E4M3_RNE(RN(a_b / RN(4 S))) (4/6 only).
+ *   candidate pattern p: sv = RN(e(p) S), inv = RN(1/sv) (sv = inv = 0 for p = 0);
+ *   codes: y = RN(x inv), q = E2M1_RNE_satfinite(y); the reconstruction is q sv (exact).
+ *   MSE objectives (4/6, the sweep, IF4, IF6, the IF4 sweep, the MX sweep): the block error
+ *   E = sum_i (x_i - xhat_i)^2 of the exact reconstructions, compared EXACTLY (the library
+ *   decides it in integer and binary64 arithmetic with no rounding in the comparison); the
+ *   lowest offset wins a tie (4/6: the max->6 scale; IF4, IF6: FP first; the IF4 sweep: lowest
+ *   offset, then FP4; the MX sweep: the lowest exponent).  ScaleSweep, "Methodology": the
+ *   objective is the block's reconstruction error.
+ *   WMSE (importance-weighted): binary32, one accumulator per candidate in element order:
+ *   xhat = RN(q sv), d = RN(x - xhat), acc = fma(RN(w d), d, acc); the lowest (acc, offset)
+ *   wins; NaN never wins; if every acc is +inf the first candidate is kept.
+ *   IF4 INT4: n = clamp(rint(RN(y RN(7/6))), -7, 7), reconstruction n g with g = RN(RN(6/7) sv)
+ *   (the INT4 block's own binary32 scale); INT4 iff its exact error is lower.
  *   IF4 x ScaleSweep (flag FP4Q_F_IF4_SWEEP): every MSE-window candidate p0-3 .. p0+7 under both
- *   types, error RN(RN(sv^2) E_type) (the zero scale: the fma sum of x^2 for both); the
- *   lowest (error, offset, type) wins with FP4 before INT4.  Adaptive Block-Scaled Data Types,
- *   "Methodology" (IF4 type choice) searched jointly with ScaleSweep, "Methodology".
+ *   types, exact errors; the lowest (error, offset, type) wins with FP4 before INT4.  Adaptive
+ *   Block-Scaled Data Types, "Methodology" (IF4 type choice) searched jointly with ScaleSweep,
+ *   "Methodology".
+ *   IF6: FP6 codes E2M3_RNE_satfinite(y), reconstruction q sv; INT6 codes
+ *   n = clamp(rint(RN(y RN(62/15))), -31, 31), reconstruction n RN(RN(15/62) sv).
  *   MXFP4: e = smallest integer with a_b <= 6 * 2^e (flag FP4Q_F_MX_OCP_FLOOR: floor(log2
- *   a_b) - 2), clamped to [-127,127]; y = RN(x 2^-e).
+ *   a_b) - 2), clamped to [-127,127]; y = RN(x 2^-e), reconstruction q 2^e.
  *   MX scale sweep (flag FP4Q_F_MX_SWEEP): e among e_c - 2 .. e_c (e_c the ceil rule, none
- *   below -127) minimizing RN(E 4^(e - e_c)), E = RN(acc_even + acc_odd) of fma(r, r, acc),
- *   r = RN(q - y) at that e; the lowest e wins a tie.  Bridging the Gap ... Microscaling FP4,
+ *   below -127) with the lowest exact block error.  Bridging the Gap ... Microscaling FP4,
  *   "Methodology": MXFP4 "Scale Fitting" of the power-of-two grid to the data, read as
  *   ScaleSweep's block-MSE search over E8M0 neighbours; exponents above e_c can only tie (the
  *   grid at 2^(e_c+1) below 6*2^e_c is a subset of the grid at 2^e_c).
@@ -49,9 +60,12 @@
  *   codes    [rows][cols/2] bytes; element 2k in the low nibble of byte k, 2k+1 in the high
  *            nibble; nibble = sign << 3 | E2M1 magnitude index (IF4 INT4 blocks: 4-bit two's
  *            complement of n).  16-byte aligned; cols/2 bytes per row, no padding.
- *   scales   [rows][cols/B] bytes, B = 16 (NVFP4/IF4: E4M3 pattern, IF4 indicator in bit 7)
- *            or 32 (MXFP4: E8M0 byte e+127, 0xFF marks a block with a non-finite input).
- *   global_scale  one float (NVFP4/IF4): written with S, or read when
+ *            IF6: [rows][cols*3/4] bytes, 12 per block, element i of a block in bits
+ *            6i .. 6i+5 of the block's little-endian 96-bit field (FP6: sign << 5 | E2M3
+ *            magnitude bits; INT6: 6-bit two's complement of n).
+ *   scales   [rows][cols/B] bytes, B = 16 (NVFP4/IF4/IF6: E4M3 pattern, IF4/IF6 indicator in
+ *            bit 7) or 32 (MXFP4: E8M0 byte e+127, 0xFF marks a block with a non-finite input).
+ *   global_scale  one float (NVFP4/IF4/IF6): written with S, or read when
  *            FP4Q_F_GLOBAL_SCALE_GIVEN is set.
  *   workspace fp4q_workspace_bytes() bytes, 16-byte aligned, ZERO-FILLED ONCE by the caller
  *            before its first use; every call leaves it zeroed again except word 0.  Word 0
@@ -150,7 +164,8 @@ FP4Q_API int64_t fp4q_scale_bytes(int64_t rows, int64_t cols, int fmt, uint32_t 
  *   with FP4Q_F_MX_OCP_FLOOR: FP4Q_ERR_INVALID_ARG), FP4Q_F_IF4_SWEEP (IF4 only, else
  *   FP4Q_ERR_UNSUPPORTED; combines with FP4Q_F_HADAMARD16 and FP4Q_F_GLOBAL_SCALE_GIVEN),
  *   FP4Q_F_SCALE_TILED (NVFP4 and MXFP4: scales in the tiled layout of fp4q_scale_bytes; IF4:
- *   FP4Q_ERR_UNSUPPORTED).
+ *   FP4Q_ERR_UNSUPPORTED).  fmt FP4Q_IF6 (objective ignored) takes FP4Q_F_GLOBAL_SCALE_GIVEN
+ *   only (S = RN(amax/1920) otherwise); every other flag returns FP4Q_ERR_UNSUPPORTED.
  * FP4Q_F_HADAMARD16: every 16-element block is first rotated by the normalized Sylvester
  *   Hadamard matrix H_16 / 4 (butterflies h = 1, 2, 4, 8 in binary32, then one exact
  *   multiplication by 1/4 per value), and the whole method -- S, the block scales, the
@@ -244,8 +259,10 @@ FP4Q_API int fp4q_quantize_host_async(const void* x_host, int dtype, int64_t row
  * Dequantize codes + scales (+ S for NVFP4/IF4) into out [rows][cols], fp32 or (flag
  * FP4Q_F_OUT_BF16) bf16.  NVFP4: RN(q * RN(e(p) S)); IF4 blocks with bit 7 set:
  * RN(n * RN(RN(6/7) * RN(e(p) S))) (the INT4 block scale with the 6/7 dequantization folded
- * in); MXFP4: RN(q * 2^(byte-127)) (byte 0xFF gives NaN).  Each value is the binary32 rounding
- * of the reconstruction the quantizer's objective measures.
+ * in); MXFP4: RN(q * 2^(byte-127)) (byte 0xFF gives NaN); IF6 (codes as fp4q_quantize writes
+ * them): RN(q * RN(e(p) S)) for FP6 blocks, RN(n * RN(RN(15/62) * RN(e(p) S))) for INT6 blocks
+ * (no inverse_hadamard, no tiled scales).  Each value is the binary32 rounding of the
+ * reconstruction the quantizer's objective measures.
  * inverse_hadamard: apply the normalized transform of the format's block size (32-point for
  * MXFP4, 16-point H_16 / 4 for NVFP4/IF4) to each dequantized block, as butterflies then
  * one multiplication per value (it is its own inverse up to rounding).  global_scale is a device

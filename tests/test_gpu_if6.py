@@ -83,3 +83,29 @@ def test_if6_full_size_sampled():
     r = O.if6_quantize(x[rows], S=S6)
     assert np.array_equal(scales.cpu().numpy()[rows], r["scales"])
     assert np.array_equal(codes.cpu().numpy()[rows], r["codes"])
+
+
+def test_if6_padded_rows_and_nonfinite():
+    # a row pitch larger than the width (the kernel's padded-row addressing), bit-exact against
+    # the oracle on the unpadded values; then a NaN: status NONFINITE and zero-filled outputs
+    w = synth.make("cfg4", rows=10, cols=1024)
+    x = O.widen_bf16(w["x"])
+    full = _dev(w)
+    padded = torch.zeros((10, 1024 + 48), dtype=torch.bfloat16, device="cuda")
+    padded[:, :1024] = full
+    view = padded[:, :1024]
+    assert view.stride(0) == 1024 + 48
+    ws = fq.new_workspace()
+    codes, scales, g = fq.quantize(view, "if6", workspace=ws)
+    torch.cuda.synchronize()
+    r = O.if6_quantize(x)
+    assert fq.read_device_status(ws) == r["status"] == 0
+    assert np.float32(g.cpu().numpy()[0]).view(np.uint32) == np.float32(r["S"]).view(np.uint32)
+    assert np.array_equal(scales.cpu().numpy(), r["scales"])
+    assert np.array_equal(codes.cpu().numpy(), r["codes"])
+    bad = full.clone()
+    bad[3, 100] = float("nan")
+    codes, scales, g = fq.quantize(bad, "if6", workspace=ws)
+    torch.cuda.synchronize()
+    assert fq.read_device_status(ws) == fq.DEVSTAT_NONFINITE
+    assert not codes.any() and not scales.any()

@@ -191,6 +191,19 @@ def test_padded_rows_and_given_scale():
     gc, gsc, _, st, _ = run_gpu(full, "if4", S=S)
     r = O.if4_quantize(oracle_x(w), S=S)
     assert_same_codes(gc, gsc, r["codes"], r["scales"])
+    # IF4 and its sweep on the padded view, at the tensor's own S
+    for sweep in (False, True):
+        gc, gsc, gS, st, _ = run_gpu(view, "if4", if4_sweep=sweep)
+        r = O.if4_quantize(oracle_x(w), sweep="sweep" if sweep else "absmax")
+        assert st == r["status"] == 0 and f32_bits(gS) == f32_bits(r["S"])
+        assert_same_codes(gc, gsc, r["codes"], r["scales"])
+    # a given S far below the tensor's: base patterns saturate at 126, where the INT4 codes clamp
+    S = float(np.float32(r["S"]) / np.float32(64))
+    gc, gsc, _, st, _ = run_gpu(full, "if4", S=S)
+    r = O.if4_quantize(oracle_x(w), S=S)
+    assert st == r["status"]
+    assert np.any((r["scales"] & 0x7F) == 0x7E)
+    assert_same_codes(gc, gsc, r["codes"], r["scales"])
 
 
 # ------------------------------------------------------------------------------------------
