@@ -72,54 +72,6 @@ __device__ __forceinline__ u64 e2m1x2_decode(uint32_t c) {
     return pk(a, b);
 }
 
-// Quantizer residuals of a pair in units of the scale: with y = (y0, y1), codes
-// q = E2M1(y) and r = RN(q - y) per lane (q is exact in f16, the subtraction is one binary32
-// rounding).  Encode, decode and subtract in one block so no value leaves its register.
-__device__ __forceinline__ void e2m1x2_residual(u64 y, float& r0, float& r1) {
-    float a, b;
-    upk(y, a, b);
-    asm("{ .reg .b8 t; .reg .b32 h; .reg .f16 p, q;\n"
-        "  cvt.rn.satfinite.e2m1x2.f32 t, %3, %2;\n"
-        "  cvt.rn.f16x2.e2m1x2 h, t;\n"
-        "  mov.b32 {p, q}, h;\n"
-        "  sub.rn.f32.f16 %0, p, %2;\n"
-        "  sub.rn.f32.f16 %1, q, %3; }"
-        : "=f"(r0), "=f"(r1) : "f"(a), "f"(b));
-}
-
-// The same residual pair returned as one packed register pair (for f32x2 accumulation).
-__device__ __forceinline__ u64 e2m1x2_residual2(u64 y) {
-    u64 r;
-    asm("{ .reg .b8 t; .reg .b32 h; .reg .f16 p, q; .reg .f32 a, b, r0, r1;\n"
-        "  mov.b64 {a, b}, %1;\n"
-        "  cvt.rn.satfinite.e2m1x2.f32 t, b, a;\n"
-        "  cvt.rn.f16x2.e2m1x2 h, t;\n"
-        "  mov.b32 {p, q}, h;\n"
-        "  sub.rn.f32.f16 r0, p, a;\n"
-        "  sub.rn.f32.f16 r1, q, b;\n"
-        "  mov.b64 %0, {r0, r1}; }"
-        : "=l"(r) : "l"(y));
-    return r;
-}
-
-// Codes and residuals of a pair from one conversion: `code` receives the packed E2M1 byte
-// (low nibble = y0), the return value the pair r = RN(q - y).
-__device__ __forceinline__ u64 e2m1x2_code_residual2(u64 y, uint32_t& code) {
-    u64 r;
-    asm("{ .reg .b8 t; .reg .b16 c16; .reg .b32 h; .reg .f16 p, q; .reg .f32 a, b, r0, r1;\n"
-        "  mov.b64 {a, b}, %2;\n"
-        "  cvt.rn.satfinite.e2m1x2.f32 t, b, a;\n"
-        "  mov.b16 c16, {t, 0};\n"
-        "  cvt.u32.u16 %1, c16;\n"
-        "  cvt.rn.f16x2.e2m1x2 h, t;\n"
-        "  mov.b32 {p, q}, h;\n"
-        "  sub.rn.f32.f16 r0, p, a;\n"
-        "  sub.rn.f32.f16 r1, q, b;\n"
-        "  mov.b64 %0, {r0, r1}; }"
-        : "=l"(r), "=r"(code) : "l"(y));
-    return r;
-}
-
 // ---- E4M3 (FN) ----------------------------------------------------------------------------
 // Bit pattern of the nearest E4M3 value (ties to even, saturating at 448) of a finite v >= 0.
 __device__ __forceinline__ int e4m3_rne(float v) {
