@@ -427,11 +427,20 @@ struct Fixed16 {
 
 // xp: the block's values (pairs; their magnitudes are used), k: the shift, from a block maximum a
 // with a 2^k in [2^14, 2^15) (B16) or [2^30, 2^31).
-template <bool B16, int NP = 8>
+// ABS: xp holds magnitudes (bf16 values: packed multiplies, exact as the scalar ones).
+template <bool B16, int NP = 8, bool ABS = false>
 __device__ __forceinline__ void fixed_point(const u64 (&xp)[NP], int k, Fixed16<B16, NP>& A) {
     float fa, fb;
     pow2_split(k, fa, fb);
-    if (B16) {
+    if (B16 && ABS) {
+        const u64 fa2 = pk(fa, fa), fb2 = pk(fb, fb), m2 = pk(kTwo23, kTwo23);
+#pragma unroll
+        for (int j = 0; j < NP; ++j) {   // |x| 2^k + 2^23 (every step exact for the elements that count)
+            float v0, v1;
+            upk(fma2(mul2(xp[j], fa2), fb2, m2), v0, v1);
+            A.w[j] = __byte_perm(__float_as_uint(v0), __float_as_uint(v1), 0x5410);
+        }
+    } else if (B16) {
 #pragma unroll
         for (int j = 0; j < NP; ++j) {   // RN(|x| 2^k + 2^23): the integer sits in the low mantissa bits
             float x0, x1;
@@ -687,7 +696,7 @@ struct BlockCtx {
     int k;              // the fixed-point shift: A = |x| 2^k
 };
 
-template <bool B16>
+template <bool B16, bool ABS = false>
 __device__ __forceinline__ void block_ctx(const u64 (&xp)[8], float ab, float S, BlockCtx<B16>& c) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) c.xp[j] = xp[j];
@@ -695,7 +704,7 @@ __device__ __forceinline__ void block_ctx(const u64 (&xp)[8], float ab, float S,
     // is raised to it (all codes are zero then, and the integers need not be exact)
     const float aeff = fmaxf(ab, __fmul_rn(S, 0x1p-11f));
     const int k = (B16 ? 14 : 30) - ilog2f(aeff);
-    fixed_point<B16>(c.xp, k, c.A);
+    fixed_point<B16, 8, ABS>(c.xp, k, c.A);
     float fa, fb;
     pow2_split(k - 2, fa, fb);
     c.T = __fmul_rn(__fmul_rn(S, fa), fb);
@@ -864,7 +873,7 @@ __device__ __forceinline__ void nvfp4_block(const u64 (&xp)[8], uint2 sgn, const
             // ties with the zero scale (p0 is 0 there), the lowest offset
             if (__fmul_rn(ab, 0x1p11f) >= S) {
                 BlockCtx<B16> c;
-                block_ctx<B16>(xp, ab, S, c);
+                block_ctx<B16, ABS>(xp, ab, S, c);
                 bp = p0 - 3 + window_search<B16, false, 11, ABS>(c, tab + p0 - 3, 0.0f, 0.0f);
             }
         } else if (OBJ == FP4Q_SWEEP_WMSE) {
@@ -1307,7 +1316,7 @@ __device__ __forceinline__ int mx_sweep_exponent(const u64 (&vp)[16], float ab, 
     }
     const int k = (B16 ? 14 : 30) - ilog2f(ab);
     Fixed16<B16, 16> A;
-    fixed_point<B16, 16>(ap, k, A);
+    fixed_point<B16, 16, true>(ap, k, A);
     int be = max(ec - 2, -127);
     double best = 0.0;
     bool first = true;
