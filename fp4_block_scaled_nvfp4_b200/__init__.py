@@ -32,7 +32,7 @@ def code_bytes_per_row(cols: int, fmt: str) -> int:
     return cols * 3 // 4 if fmt == "if6" else cols // 2
 
 # Names of every function include/fp4q.h declares (checked against the header by the tests).
-EXPORTS = ("fp4q_workspace_bytes", "fp4q_scale_bytes", "fp4q_nvfp4_gemm", "fp4q_mxfp4_gemm", "fp4q_gemm", "fp4q_encode", "fp4q_global_scale", "fp4q_hadamard_global_scale", "fp4q_quantize",
+EXPORTS = ("fp4q_workspace_bytes", "fp4q_scale_bytes", "fp4q_nvfp4_gemm", "fp4q_mxfp4_gemm", "fp4q_gemm", "fp4q_encode", "fp4q_global_scale", "fp4q_if6_global_scale", "fp4q_hadamard_global_scale", "fp4q_quantize",
            "fp4q_hadamard_quantize", "fp4q_dequantize", "fp4q_quantize_noalloc", "fp4q_quantize_host_async", "fp4q_read_device_status", "fp4q_last_launch_count", "fp4q_last_cuda_error", "fp4q_status_string")
 
 _lib = None
@@ -66,6 +66,8 @@ def lib():
         L.fp4q_quantize.argtypes = [P, i32, i64, i64, i64, i32, i32, P, P, P, P, P, u32, P]
         L.fp4q_global_scale.restype = i32
         L.fp4q_global_scale.argtypes = [P, i32, i64, i64, i64, P, P, P]
+        L.fp4q_if6_global_scale.restype = i32
+        L.fp4q_if6_global_scale.argtypes = [P, i32, i64, i64, i64, P, P, P]
         L.fp4q_hadamard_global_scale.restype = i32
         L.fp4q_hadamard_global_scale.argtypes = [P, i32, i64, i64, i64, i32, P, P, P]
         L.fp4q_hadamard_quantize.restype = i32
@@ -250,9 +252,9 @@ def quantize(x, fmt: str = "nvfp4", objective: str = "sweep_mse", importance=Non
     return codes, scales, (gs if fmt != "mxfp4" else None)
 
 
-def global_scale(x, out=None, workspace=None, stream=None, hadamard16: bool = False):
+def global_scale(x, out=None, workspace=None, stream=None, hadamard16: bool = False, fmt: str = "nvfp4"):
     """Tensor scale S = RN(max|x| / 1536) as a [1] float32 CUDA tensor (amax pass only);
-    hadamard16: of the 16-point block-rotated tensor."""
+    hadamard16: of the 16-point block-rotated tensor; fmt "if6": IF6's S = RN(max|x| / 1920)."""
     torch = _torch()
     if x is None or not x.is_cuda or x.dim() != 2 or x.stride(1) != 1:
         raise Fp4qError("x must be a 2-D CUDA tensor with unit column stride")
@@ -262,7 +264,14 @@ def global_scale(x, out=None, workspace=None, stream=None, hadamard16: bool = Fa
     ws = workspace if workspace is not None else new_workspace(x.device)
     _need(gs, "out", x.device, (torch.float32,), min_numel=1)
     _need(ws, "workspace", x.device, (torch.uint8,), min_numel=workspace_bytes())
-    if hadamard16:
+    if fmt not in ("nvfp4", "if4", "if6"):
+        raise Fp4qError(f"no tensor scale for format {fmt!r}")
+    if fmt == "if6":
+        if hadamard16:
+            raise Fp4qError("IF6 has no rotated form")
+        rc = lib().fp4q_if6_global_scale(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), _ptr(gs), _ptr(ws),
+                                         _stream_ptr(stream))
+    elif hadamard16:
         rc = lib().fp4q_hadamard_global_scale(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), 16, _ptr(gs),
                                               _ptr(ws), _stream_ptr(stream))
     else:

@@ -1943,7 +1943,7 @@ namespace fp4q {
 // fp4q_global_scale (plain, granule = 16 bytes of a row) and fp4q_hadamard_global_scale
 // (rotated blocks, granule = 16 elements).
 int global_scale_impl(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld, bool had16,
-                      float* global_scale, void* workspace, void* stream) {
+                      float* global_scale, void* workspace, void* stream, float div = 1536.0f) {
     g_launches = 0;
     if (dtype != FP4Q_IN_F32 && dtype != FP4Q_IN_BF16) return FP4Q_ERR_INVALID_ARG;
     const int es = dtype == FP4Q_IN_BF16 ? 2 : 4;
@@ -1954,8 +1954,8 @@ int global_scale_impl(const void* x, int dtype, int64_t rows, int64_t cols, int6
     if (!aligned16(x) || !aligned16(workspace) || (ld * es) % 16) return FP4Q_ERR_ALIGNMENT;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     uint32_t* ws = reinterpret_cast<uint32_t*>(workspace);
-    if (dtype == FP4Q_IN_BF16) launch_amax<FP4Q_IN_BF16>(x, rows, cols, ld, ws, global_scale, 1, had16, st);
-    else launch_amax<FP4Q_IN_F32>(x, rows, cols, ld, ws, global_scale, 1, had16, st);
+    if (dtype == FP4Q_IN_BF16) launch_amax<FP4Q_IN_BF16>(x, rows, cols, ld, ws, global_scale, 1, had16, st, div);
+    else launch_amax<FP4Q_IN_F32>(x, rows, cols, ld, ws, global_scale, 1, had16, st, div);
     return launched(1);
 }
 }  // namespace fp4q
@@ -1965,6 +1965,11 @@ extern "C" {
 int fp4q_global_scale(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld, float* global_scale,
                       void* workspace, void* stream) {
     return global_scale_impl(x, dtype, rows, cols, ld, false, global_scale, workspace, stream);
+}
+
+int fp4q_if6_global_scale(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld, float* global_scale,
+                          void* workspace, void* stream) {
+    return global_scale_impl(x, dtype, rows, cols, ld, false, global_scale, workspace, stream, 1920.0f);
 }
 
 int fp4q_hadamard_global_scale(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld, int had_size,

@@ -196,6 +196,16 @@ FP4Q_API int fp4q_global_scale(const void* x, int dtype, int64_t rows, int64_t c
                       float* global_scale, void* workspace, void* stream);
 
 /*
+ * IF6's tensor scale: S = RN(max|x| / 1920) (7.5, the FP6 maximum, in place of FP4's 6; Adaptive
+ * Block-Scaled Data Types, "Methodology", the IF4 construction at 6 bits).  Status, workspace,
+ * shapes and errors as fp4q_global_scale; passing the result to fp4q_quantize(FP4Q_IF6) with
+ * FP4Q_F_GLOBAL_SCALE_GIVEN performs exactly the work of a call without the flag.  Use: a
+ * row-sharded tensor reduces the per-shard S values by maximum.
+ */
+FP4Q_API int fp4q_if6_global_scale(const void* x, int dtype, int64_t rows, int64_t cols, int64_t ld,
+                          float* global_scale, void* workspace, void* stream);
+
+/*
  * Tensor scale of the block-rotated tensor: S = RN(max|H x| / 1536), H x being every
  * 16-element block of every row rotated by H_16 / 4 exactly as fp4q_quantize does under
  * FP4Q_F_HADAMARD16 (so this S with FP4Q_F_GLOBAL_SCALE_GIVEN | FP4Q_F_HADAMARD16

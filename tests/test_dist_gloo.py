@@ -50,9 +50,12 @@ def _worker(rank, world, port, results):
         s_rot_loc, _ = O.tensor_scale(O.rotate16(shard))
         s_rot = reduce_global_scale(torch.tensor([s_rot_loc], dtype=torch.float32))
         rot = O.nvfp4_quantize(shard, "sweep_mse", S=float(s_rot.item()), hadamard16=True)
+        # IF6: its own tensor scale RN(amax / 1920), reduced the same way
+        s6 = reduce_global_scale(torch.tensor([O.if6_tensor_scale(shard)], dtype=torch.float32))
+        q6 = O.if6_quantize(shard, S=float(s6.item()))
         results[rank] = (float(s_all.item()), codes["codes"].tobytes(), codes["scales"].tobytes(),
                          float(s_bad.item()), slowest, float(s_rot.item()), rot["codes"].tobytes(),
-                         rot["scales"].tobytes())
+                         rot["scales"].tobytes(), float(s6.item()), q6["codes"].tobytes(), q6["scales"].tobytes())
     finally:
         dist.destroy_process_group()
 
@@ -69,9 +72,13 @@ def test_sharded_scale_matches_whole_tensor():
     x = O.widen_bf16(w["x"])
     whole = O.nvfp4_quantize(x, "sweep_mse")
     whole_rot = O.nvfp4_quantize(x, "sweep_mse", hadamard16=True)
+    whole6 = O.if6_quantize(x)
     assert whole_rot["S"] != whole["S"]
     for rank in range(world):
-        s_all, c, sc, s_bad, slowest, s_rot, c_rot, sc_rot = results[rank]
+        s_all, c, sc, s_bad, slowest, s_rot, c_rot, sc_rot, s6, c6, sc6 = results[rank]
+        assert np.float32(s6).view(np.uint32) == np.float32(whole6["S"]).view(np.uint32)
+        assert c6 == whole6["codes"][rank * 16:(rank + 1) * 16].tobytes()
+        assert sc6 == whole6["scales"][rank * 16:(rank + 1) * 16].tobytes()
         assert np.float32(s_rot).view(np.uint32) == np.float32(whole_rot["S"]).view(np.uint32)
         assert c_rot == whole_rot["codes"][rank * 16:(rank + 1) * 16].tobytes()
         assert sc_rot == whole_rot["scales"][rank * 16:(rank + 1) * 16].tobytes()

@@ -35,7 +35,8 @@ def nccl_group():
 
 
 @pytest.mark.parametrize("fmt,obj,had16", [("nvfp4", "sweep_mse", False), ("nvfp4", "sweep_mse", True),
-                                           ("if4", "absmax", False), ("mxfp4", "absmax", False)])
+                                           ("if4", "absmax", False), ("if6", "absmax", False),
+                                           ("mxfp4", "absmax", False)])
 def test_sharded_quantize_over_nccl_matches_the_single_call(nccl_group, fmt, obj, had16):
     w = synth.make("cfg3", rows=256, cols=4096)
     x = torch.from_numpy(w["x"].view(np.int16)).view(torch.bfloat16).cuda()

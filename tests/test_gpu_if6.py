@@ -109,3 +109,33 @@ def test_if6_padded_rows_and_nonfinite():
     torch.cuda.synchronize()
     assert fq.read_device_status(ws) == fq.DEVSTAT_NONFINITE
     assert not codes.any() and not scales.any()
+
+
+@pytest.mark.parametrize("cfg,rows,cols", [("cfg4", 40, 14336), ("cfg1", None, None)])
+def test_if6_global_scale_entry_point(cfg, rows, cols):
+    # fp4q_if6_global_scale alone gives the S that an IF6 quantize computes, and passing it back
+    # reproduces that call's codes and scales
+    w = synth.make(cfg, rows=rows, cols=cols)
+    x = O.widen_bf16(w["x"]) if w["dtype"] == "bf16" else np.asarray(w["x"], np.float32)
+    xd = _dev(w)
+    ws = fq.new_workspace()
+    g = fq.global_scale(xd, workspace=ws, fmt="if6")
+    torch.cuda.synchronize()
+    assert np.float32(g.cpu().numpy()[0]).view(np.uint32) == np.float32(O.if6_tensor_scale(x)).view(np.uint32)
+    c0, s0, g0 = fq.quantize(xd, "if6", workspace=ws)
+    c1, s1, _ = fq.quantize(xd, "if6", global_scale=g, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(g.view(torch.int32), g0.view(torch.int32))
+    assert torch.equal(c0, c1) and torch.equal(s0, s1)
+    # a non-finite element gives S = NaN and the NONFINITE status; the next call (a zero tensor)
+    # overwrites the status word with its own
+    z = torch.zeros(4, 64, dtype=torch.bfloat16, device="cuda")
+    z[2, 9] = float("nan")
+    gn = fq.global_scale(z, workspace=ws, fmt="if6")
+    torch.cuda.synchronize()
+    assert torch.isnan(gn).all() and fq.read_device_status(ws) & fq.DEVSTAT_NONFINITE
+    z[2, 9] = 0
+    gz = fq.global_scale(z, workspace=ws, fmt="if6")
+    torch.cuda.synchronize()
+    assert float(gz.item()) == 0.0
+    assert fq.read_device_status(ws) == O.if6_quantize(np.zeros((4, 64), np.float32))["status"]
