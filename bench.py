@@ -513,44 +513,62 @@ def run_ours(args, rank, world):
     torch.cuda.synchronize()
     full_cycles, rest = divmod(args.steps, nsets)
 
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    # the batched form (NVFP4 / IF4 without rotation or WMSE): the K steps' tensors, the buffer
+    # sets in turn, in one fp4q_quantize_batch call -- one amax kernel, then K quantize kernels,
+    # each also taking the next tensor's amax
+    fused = two_pass and not had16 and obj != "sweep_wmse"
+    if fused:
+        def plan_over(k):
+            return fq.BatchPlan([xs[i % nsets] for i in range(k)], base, obj or "absmax",
+                                outs=[outs[i % nsets] for i in range(k)], workspace=wss[0],
+                                if4_sweep=(obj == "if4_sweep"))
+        plan = plan_over(args.steps)
+        with torch.cuda.stream(stream):
+            plan_over(max(args.warmup, nsets + 1))(stream)
+        torch.cuda.synchronize()
+        batch_graph = capture(lambda: plan(stream))   # the K + 1 launches as one CUDA graph
+        with torch.cuda.stream(stream):
+            batch_graph.replay()
+        torch.cuda.synchronize()
+
+    def timed(run):
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
         with torch.cuda.stream(stream):
             start.record()
-            for _ in range(full_cycles):
-                cycle.replay()
-            for i in range(rest):
-                graphs[i].replay()
+            run()
             end.record()
         end.synchronize()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    ms = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        t_ms = start.elapsed_time(end)
+        if world > 1:
+            t = torch.tensor([t_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            t_ms = float(t.item())
+        return t_ms
+
+    def run_cycles():
+        for _ in range(full_cycles):
+            cycle.replay()
+        for i in range(rest):
+            graphs[i].replay()
+
+    with ClockSampler(local) as clk:
+        ms = timed(batch_graph.replay if fused else run_cycles)
+    two_stream_ms = timed(run_cycles) if fused else None
 
     # the same steps with no overlap between them (one stream, amax then quantize per step)
-    serial_ms = ms
-    if two_pass:
-        with torch.cuda.stream(stream):
-            start.record()
-            for _ in range(full_cycles):
-                serial_cycle.replay()
-            for i in range(rest):
-                graphs[i].replay()
-            end.record()
-        end.synchronize()
-        serial_ms = start.elapsed_time(end)
-        if world > 1:
-            t = torch.tensor([serial_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            serial_ms = float(t.item())
+    def run_serial():
+        for _ in range(full_cycles):
+            serial_cycle.replay()
+        for i in range(rest):
+            graphs[i].replay()
+
+    serial_ms = timed(run_serial) if two_pass else ms
 
     # per-kernel launch durations for the roofline: the same launches, one kernel kind at a
     # time (every buffer set in turn, so reads still come from HBM), timed with CUDA events on
@@ -626,15 +644,26 @@ def run_ours(args, rank, world):
     value = alg * args.steps * world / (ms * 1e-3) / 1e9
     tq = t_q
     kernel_key = f"{args.workload}:quantize"
+    kernel_name = "quantize (" + (obj or fmt) + ")"
+    t_fused = None
+    if fused:
+        # the dominant kernel of the timed region: K quantize kernels that also take the next
+        # tensor's amax, and one amax kernel (timed alone above) for the first tensor
+        t_fused = (ms - t_amax) / args.steps
+        tq = t_fused
+        kernel_key = f"{args.workload}:quantize_next"
+        kernel_name += " + the next tensor's amax"
     achieved = alg / (tq * 1e-3) / 1e9
     clocks = clk.summary()
     traffic = profiled_traffic(kernel_key)
     hbm_roof = {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": "quantize (" + (obj or fmt) + ")",
+                "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": kernel_name,
                 "peak_source": f"{peak_src} hbm_gbs (copy, burst) from MEASURED_PEAKS.json"}
     ops = ALU_OPS_PER_ELEMENT.get(obj or fmt)
     if ops is not None and had16:
         ops += ROTATION_OPS_PER_ELEMENT
+    if ops is not None and fused:
+        ops += 1   # the tensor maximum
     if ops is not None:
         # the candidate search is bound by plain FP32/convert arithmetic, not by HBM: the peak is
         # 148 SMs x 128 FP32 lanes x the SM clock sampled during the timed region
@@ -643,7 +672,7 @@ def run_ours(args, rank, world):
         alu_peak = sms * 128 * mhz * 1e6 / 1e9
         alu_ach = ops * rows * cols / (tq * 1e-3) / 1e9
         roofline = {"bound": "alu", "achieved": round(alu_ach, 1), "peak": round(alu_peak, 1), "unit": "Gop/s",
-                    "frac": round(alu_ach / alu_peak, 4), "traffic": traffic, "kernel": "quantize (" + obj + ")",
+                    "frac": round(alu_ach / alu_peak, 4), "traffic": traffic, "kernel": kernel_name,
                     "ops_per_element": ops,
                     "peak_source": f"{sms} SMs x 128 FP32 lanes x {mhz:.0f} MHz (median SM clock in the timed region)",
                     "hbm": {k: hbm_roof[k] for k in ("achieved", "peak", "unit", "frac")}}
@@ -657,7 +686,11 @@ def run_ours(args, rank, world):
                    "method": obj or fmt, "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": f"{nsets} rotating input/output buffer sets, {nsets * (in_bytes + out_bytes) / 2**20:.0f} MB "
                          f"total (at least 3x the 126 MB L2)",
-                   "timing": ("CUDA graph over the buffer sets (no timing nodes inside); each step's amax pass runs on "
+                   "timing": ("one fp4q_quantize_batch call over the K steps' tensors (the buffer sets in turn), "
+                              "captured as a CUDA graph: an amax kernel for the first tensor, then K quantize "
+                              "kernels, each also taking the next tensor's amax; CUDA events on the launching "
+                              "stream" if fused else
+                              "CUDA graph over the buffer sets (no timing nodes inside); each step's amax pass runs on "
                               "a second stream under the previous step's quantize kernel, each quantize after its own "
                               "amax; CUDA events on the launching stream" if two_pass else
                               "CUDA graph over the buffer sets (no timing nodes inside), replayed on one stream; CUDA "
@@ -665,15 +698,22 @@ def run_ours(args, rank, world):
         "hbm_frac": round(value / world / peak, 4),
         "input_gbps": round(in_bytes * args.steps * world / (ms * 1e-3) / 1e9, 2),
         "elements_per_s": round(rows * cols * args.steps * world / (ms * 1e-3), 1),
-        "kernels_ms": {"amax": (None if t_amax is None else round(t_amax, 5)), "quantize": round(tq, 5),
-                       "how": f"each kernel alone, {kernel_reps} launches over the rotating buffer sets, CUDA events"},
+        "kernels_ms": {"amax": (None if t_amax is None else round(t_amax, 5)), "quantize": round(t_q, 5),
+                       "how": f"each kernel alone, {kernel_reps} launches over the rotating buffer sets, CUDA events",
+                       **({"quantize_next_amax": round(t_fused, 5),
+                           "how_next": "the timed region's K batched quantize kernels: (region - one amax) / K"}
+                          if fused else {})},
         "step_ms": step_dist,
         "serial": {"value": round(alg * args.steps * world / (serial_ms * 1e-3) / 1e9, 2),
                    "ms_per_step": round(serial_ms / args.steps, 5),
                    "how": "the same steps with no overlap: amax then quantize per step on one stream"},
+        **({"two_stream": {"value": round(alg * args.steps * world / (two_stream_ms * 1e-3) / 1e9, 2),
+                           "ms_per_step": round(two_stream_ms / args.steps, 5),
+                           "how": "the same steps as separate amax and quantize kernels, each amax on a second "
+                                  "stream under the previous step's quantize"}} if fused else {}),
         "roofline": roofline,
         "device_status": st,
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": args.steps + 1 if fused else launches_per_step * args.steps,
         "clocks": clocks,
         "e2e": {"value": round(alg / (e2e_ms * 1e-3) / 1e9 * world, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4), "steps": e2e_steps,

@@ -32,7 +32,7 @@ def code_bytes_per_row(cols: int, fmt: str) -> int:
     return cols * 3 // 4 if fmt == "if6" else cols // 2
 
 # Names of every function include/fp4q.h declares (checked against the header by the tests).
-EXPORTS = ("fp4q_workspace_bytes", "fp4q_scale_bytes", "fp4q_nvfp4_gemm", "fp4q_mxfp4_gemm", "fp4q_gemm", "fp4q_encode", "fp4q_global_scale", "fp4q_if6_global_scale", "fp4q_hadamard_global_scale", "fp4q_quantize",
+EXPORTS = ("fp4q_workspace_bytes", "fp4q_scale_bytes", "fp4q_nvfp4_gemm", "fp4q_mxfp4_gemm", "fp4q_gemm", "fp4q_encode", "fp4q_global_scale", "fp4q_if6_global_scale", "fp4q_quantize_batch", "fp4q_hadamard_global_scale", "fp4q_quantize",
            "fp4q_hadamard_quantize", "fp4q_dequantize", "fp4q_quantize_noalloc", "fp4q_quantize_host_async", "fp4q_read_device_status", "fp4q_last_launch_count", "fp4q_last_cuda_error", "fp4q_status_string")
 
 _lib = None
@@ -64,6 +64,8 @@ def lib():
         L.fp4q_mxfp4_gemm.argtypes = [P, P, P, P, i64, i64, i64, P, i64, P, P]
         L.fp4q_quantize.restype = i32
         L.fp4q_quantize.argtypes = [P, i32, i64, i64, i64, i32, i32, P, P, P, P, P, u32, P]
+        L.fp4q_quantize_batch.restype = i32
+        L.fp4q_quantize_batch.argtypes = [i32, P, i32, i32, i32, P, u32, P]
         L.fp4q_global_scale.restype = i32
         L.fp4q_global_scale.argtypes = [P, i32, i64, i64, i64, P, P, P]
         L.fp4q_if6_global_scale.restype = i32
@@ -250,6 +252,98 @@ def quantize(x, fmt: str = "nvfp4", objective: str = "sweep_mse", importance=Non
                              _ptr(gs) if fmt != "mxfp4" else None, _ptr(ws), flags, _stream_ptr(stream))
     _check(rc, "fp4q_quantize")
     return codes, scales, (gs if fmt != "mxfp4" else None)
+
+
+class _Tensor(C.Structure):
+    """fp4q_tensor of include/fp4q.h."""
+    _fields_ = [("x", C.c_void_p), ("rows", C.c_int64), ("cols", C.c_int64), ("ld", C.c_int64),
+                ("importance", C.c_void_p), ("codes", C.c_void_p), ("scales", C.c_void_p),
+                ("global_scale", C.c_void_p)]
+
+
+class BatchPlan:
+    """A checked, marshalled fp4q_quantize_batch call over fixed buffers, for callers that run
+    the same batch repeatedly (the descriptors are built once; each call is the C call only).
+
+    xs: 2-D CUDA tensors of one dtype on one device; fmt "nvfp4" or "if4".
+    importance: one float32 [cols] tensor per input (SWEEP_WMSE), or None.
+    global_scales: one [1] float32 tensor per input to use as S (no amax passes), or None.
+    outs: optional list of preallocated (codes, scales, S) tuples (entries may repeat: later
+    tensors overwrite earlier results, as separate calls would).
+    """
+
+    def __init__(self, xs, fmt: str = "nvfp4", objective: str = "sweep_mse", importance=None, global_scales=None,
+                 outs=None, workspace=None, hadamard16: bool = False, if4_sweep: bool = False,
+                 tiled_scales: bool = False):
+        if fmt not in ("nvfp4", "if4"):
+            raise Fp4qError(f"a batch holds nvfp4 or if4 tensors, not {fmt!r}")
+        self.fcode = _format(fmt)
+        self.ocode = _objective(objective) if fmt == "nvfp4" else 0
+        xs = list(xs)
+        n = len(xs)
+        for name, seq in (("importance", importance), ("global_scales", global_scales), ("outs", outs)):
+            if seq is not None and len(seq) != n:
+                raise Fp4qError(f"{name} must have one entry per tensor")
+        self.n, self.results, self.dcode, self.ws = n, [], IN_BF16, None
+        self.arr = (_Tensor * max(n, 1))()
+        self.flags = _flags(global_scales, False, hadamard16, False, if4_sweep, tiled_scales)
+        self._keep = (xs, importance, global_scales)
+        if n == 0:
+            return
+        dev = xs[0].device if xs[0] is not None else None
+        dcode = None
+        for i, x in enumerate(xs):
+            if x is None or not x.is_cuda or x.dim() != 2 or (x.numel() and x.stride(1) != 1):
+                raise Fp4qError("every input must be a 2-D CUDA tensor with unit column stride")
+            if x.device != dev:
+                raise Fp4qError("every input must be on the same device")
+            code = _dtype_code(x)
+            if dcode is not None and code != dcode:
+                raise Fp4qError("every input must have the same dtype")
+            dcode = code
+            rows, cols = x.shape
+            if cols % 16:
+                raise Fp4qError("cols must be a multiple of 16")
+            codes, scales, gs = outs[i] if outs is not None else alloc_outputs(rows, cols, fmt, dev,
+                                                                               tiled=tiled_scales)
+            if global_scales is not None:
+                gs = global_scales[i]
+            if x.numel() == 0:   # skipped by the library; nothing is read or written
+                self.arr[i] = _Tensor(None, rows, cols, cols, None, None, None, None)
+                self.results.append((codes, scales, gs))
+                continue
+            imp = importance[i] if importance is not None else None
+            _check_quantize(x, fmt, objective, imp, codes, scales, gs, tiled_scales)
+            ld = x.stride(0) if rows > 1 else cols   # the row pitch of a tensor with one row or none is unused
+            self.arr[i] = _Tensor(x.data_ptr(), rows, cols, ld, None if imp is None else imp.data_ptr(),
+                                  codes.data_ptr(), scales.data_ptr(), gs.data_ptr())
+            self.results.append((codes, scales, gs))
+        torch = _torch()
+        ws = workspace if workspace is not None else new_workspace(dev)
+        _need(ws, "workspace", dev, (torch.uint8, torch.int32, torch.int64, torch.float32))
+        if ws.numel() * ws.element_size() < workspace_bytes():
+            raise Fp4qError(f"workspace must hold at least {workspace_bytes()} bytes")
+        self.dcode, self.ws = dcode, ws
+
+    def __call__(self, stream=None):
+        """Run the batch on `stream` (default: the current stream); returns [(codes, scales, S)]."""
+        if self.n:
+            rc = lib().fp4q_quantize_batch(self.n, C.cast(self.arr, C.c_void_p), self.dcode, self.fcode, self.ocode,
+                                           _ptr(self.ws), self.flags, _stream_ptr(stream))
+            _check(rc, "fp4q_quantize_batch")
+        return self.results
+
+
+def quantize_batch(xs, fmt: str = "nvfp4", objective: str = "sweep_mse", importance=None, global_scales=None,
+                   outs=None, workspace=None, stream=None, hadamard16: bool = False, if4_sweep: bool = False,
+                   tiled_scales: bool = False):
+    """NVFP4 / IF4 quantization of a sequence of 2-D CUDA tensors of one dtype in one call
+    (fp4q_quantize_batch): the results of quantize() on each, with each tensor's amax pass folded
+    into the previous tensor's quantize kernel.  Arguments as BatchPlan; returns the list of
+    (codes, scales, S)."""
+    return BatchPlan(xs, fmt, objective, importance=importance, global_scales=global_scales, outs=outs,
+                     workspace=workspace, hadamard16=hadamard16, if4_sweep=if4_sweep,
+                     tiled_scales=tiled_scales)(stream)
 
 
 def global_scale(x, out=None, workspace=None, stream=None, hadamard16: bool = False, fmt: str = "nvfp4"):

@@ -9,9 +9,9 @@ ROOT = os.path.dirname(PKG)
 SRCS = [os.path.join(HERE, "fp4q.cu"), os.path.join(HERE, "fp4q_gemm.cu")]
 DEPS = SRCS + [os.path.join(HERE, "fp4q_device.cuh"), os.path.join(ROOT, "include", "fp4q.h")]
 LIB = os.path.join(PKG, "libfp4q.so")
-# The GEMM failure-path test library: the product sources built with the MMA thread's first
-# wait treated as timed out (FP4Q_GEMM_FAIL_FIRST_WAIT); loaded only by tests/test_gpu_gemm_failure.py.
-TEST_LIB = os.path.join(PKG, "libfp4q_gemm_failtest.so")
+# The failure-path test library: the product sources built with the GEMM MMA thread's first wait
+# treated as timed out (FP4Q_GEMM_FAIL_FIRST_WAIT); loaded only by tests/test_gpu_gemm_failure.py.
+TEST_LIB = os.path.join(PKG, "libfp4q_failtest.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
          "--fmad=false", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "-shared", "-Xptxas", "-v",

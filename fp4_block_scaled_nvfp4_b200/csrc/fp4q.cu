@@ -29,6 +29,7 @@
 #include <cmath>
 #include <cstdint>
 #include <mutex>
+#include <vector>
 #include <cuda_runtime.h>
 
 #include "fp4q.h"
@@ -121,6 +122,27 @@ __device__ __forceinline__ void amax_finish(uint32_t m, float post, uint32_t* ws
     }
 }
 
+// Fold one 16-byte vector into a running maximum of magnitude bit patterns: per 16-bit half for
+// bf16 (amax_bits turns the pair into float bits), per word for fp32.
+template <int IN>
+__device__ __forceinline__ void amax_fold(uint32_t& m, const uint4 v) {
+    if (IN == FP4Q_IN_BF16) {
+        uint32_t t;
+        const uint32_t mk = 0x7FFF7FFFu;
+        asm("max.u16x2 %0, %1, %2;" : "=r"(t) : "r"(v.x & mk), "r"(v.y & mk));
+        asm("max.u16x2 %0, %0, %1;" : "+r"(t) : "r"(v.z & mk));
+        asm("max.u16x2 %0, %0, %1;" : "+r"(t) : "r"(v.w & mk));
+        asm("max.u16x2 %0, %0, %1;" : "+r"(m) : "r"(t));
+    } else {
+        const uint32_t mk = 0x7FFFFFFFu;
+        m = max(m, max(max(v.x & mk, v.y & mk), max(v.z & mk, v.w & mk)));
+    }
+}
+template <int IN>
+__device__ __forceinline__ uint32_t amax_bits(uint32_t m) {
+    return IN == FP4Q_IN_BF16 ? max(m & 0xFFFFu, m >> 16) << 16 : m;   // bf16 bits -> f32 bits
+}
+
 // Largest magnitude of the elements in the 16-byte vectors first, first + step, ... of a
 // rows x cols tensor with row pitch ld, as float bits (NaN and Inf order above every finite
 // value as integers).  U loads are kept in flight per thread on contiguous tensors.
@@ -132,19 +154,7 @@ __device__ __forceinline__ uint32_t amax_partial(const void* __restrict__ xv, in
     uint32_t m = 0;
     const uint4* base = reinterpret_cast<const uint4*>(xv);
     const int64_t ldv = ld * (IN == FP4Q_IN_BF16 ? 2 : 4) / 16;
-    auto fold = [&](const uint4 v) {
-        if (IN == FP4Q_IN_BF16) {
-            uint32_t t;
-            const uint32_t mk = 0x7FFF7FFFu;
-            asm("max.u16x2 %0, %1, %2;" : "=r"(t) : "r"(v.x & mk), "r"(v.y & mk));
-            asm("max.u16x2 %0, %0, %1;" : "+r"(t) : "r"(v.z & mk));
-            asm("max.u16x2 %0, %0, %1;" : "+r"(t) : "r"(v.w & mk));
-            asm("max.u16x2 %0, %0, %1;" : "+r"(m) : "r"(t));
-        } else {
-            const uint32_t mk = 0x7FFFFFFFu;
-            m = max(m, max(max(v.x & mk, v.y & mk), max(v.z & mk, v.w & mk)));
-        }
-    };
+    auto fold = [&](const uint4 v) { amax_fold<IN>(m, v); };
     auto at = [&](int64_t i) -> const uint4* {
         if (ldv == vpr) return base + i;
         const int64_t r = i / vpr;
@@ -171,8 +181,7 @@ __device__ __forceinline__ uint32_t amax_partial(const void* __restrict__ xv, in
         }
     }
     for (; i < total; i += step) fold(__ldg(at(i)));
-    if (IN == FP4Q_IN_BF16) m = max(m & 0xFFFFu, m >> 16) << 16;   // bf16 bits -> f32 bits
-    return m;
+    return amax_bits<IN>(m);
 }
 
 template <int IN>
@@ -998,12 +1007,58 @@ __host__ __device__ constexpr int q16_min_ctas() {   // register cap: CTAs per S
     return KIND == FP4Q_SWEEP_MSE || KIND == KIND_IF4_SWEEP ? 3 : (KIND == FP4Q_ABSMAX ? 5 : 4);
 }
 
-template <int IN, int KIND, bool HAD, typename IDX>
+// The next tensor of a batch (fp4q_quantize_batch): same element type; its S is written to gs.
+template <typename IDX>
+struct NextTensor {
+    const void* x;
+    IDX rows, cols, ld;
+    float* gs;
+};
+
+// 16-byte vector i of a tensor, counted row by row.
+template <int IN, typename IDX>
+__device__ __forceinline__ const uint4* vec_at(const NextTensor<IDX>& t, IDX i) {
+    constexpr int es = IN == FP4Q_IN_BF16 ? 2 : 4;
+    const IDX vpr = t.cols * es / 16, ldv = t.ld * es / 16;
+    const uint4* base = reinterpret_cast<const uint4*>(t.x);
+    if (ldv == vpr) return base + i;
+    const IDX r = i / vpr;
+    return base + r * ldv + (i - r * vpr);
+}
+
+// The next tensor's amax, folded while this tensor is quantized.  Thread t owns the vectors
+// t, t + G, t + 2G, ... of the next tensor and takes two of them per block it quantizes: the
+// pair is copied into the thread's own shared-memory slots by cp.async one block ahead and
+// folded after the following block, so its HBM reads overlap the candidate search and hold
+// no registers meanwhile.  Only the issuing thread reads a slot, so the group wait orders it.
+template <int IN, typename IDX>
+__device__ __forceinline__ void next_stage(const NextTensor<IDX>& t, IDX ntot, IDX v, IDX G, uint4* s) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const IDX i = v + (IDX)u * G;
+        if (i < ntot) {
+            const uint32_t dst = (uint32_t)__cvta_generic_to_shared(s + u * kThreads + threadIdx.x);
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(vec_at<IN>(t, i)) : "memory");
+        }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int IN, typename IDX>
+__device__ __forceinline__ void next_fold(IDX ntot, IDX v, IDX G, const uint4* s, uint32_t& m) {
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+        if (v + (IDX)u * G < ntot) amax_fold<IN>(m, s[u * kThreads + threadIdx.x]);
+}
+
+template <int IN, int KIND, bool HAD, typename IDX, bool NEXT>
 __global__ void __launch_bounds__(kThreads, q16_min_ctas<KIND>())
     q16_kernel(const void* __restrict__ xv, IDX rows, IDX cols, IDX ld, const float* __restrict__ imp,
                uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, const float* __restrict__ gscale,
-               uint32_t* __restrict__ ws, int tiled) {
+               uint32_t* __restrict__ ws, int tiled, NextTensor<IDX> nx, int status_or) {
+    static_assert(!NEXT || (q16_persistent<KIND>() && !HAD), "the next tensor's amax rides on the persistent loop");
     __shared__ float2 s_tab[kTabLen];
+    __shared__ uint4 s_nx[NEXT ? 2 * kThreads : 1];
     const IDX nb = cols / 16;
     const IDX total = rows * nb;
     const IDX G = (IDX)gridDim.x * blockDim.x;
@@ -1014,7 +1069,10 @@ __global__ void __launch_bounds__(kThreads, q16_min_ctas<KIND>())
     if (IN == FP4Q_IN_BF16 && blk < total) load_raw16<IN>(xv, block_at<IDX, false>(blk, cols, ld, nb).xoff, rb);
     const float S = *gscale;
     const uint32_t flags = scale_flags(S);
-    if (blockIdx.x == 0 && threadIdx.x == 0) ws[WS_STATUS] = flags;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        if (status_or) atomicOr(&ws[WS_STATUS], flags);
+        else ws[WS_STATUS] = flags;
+    }
     build_scale_table(S, s_tab);
     const float2* tab = s_tab + kTabPad;
     const float d6 = __fmul_rn(6.0f, S), d4 = __fmul_rn(4.0f, S);
@@ -1064,7 +1122,21 @@ __global__ void __launch_bounds__(kThreads, q16_min_ctas<KIND>())
         else if (KIND == KIND_IF4_SWEEP) if4_block<true, B16>(xp, S, d6, K76, K67, tab, cdst, sdst);
         else nvfp4_block<KIND, B16, kAbs>(xp, sgn, imp, at.b, S, d6, d4, tab, cdst, sdst);
     };
-    if (q16_persistent<KIND>()) {
+    if constexpr (NEXT) {
+        const IDX ntot = nx.rows * (nx.cols * (IN == FP4Q_IN_BF16 ? 2 : 4) / 16);
+        IDX nv = blk;
+        uint32_t nm = 0;
+        next_stage<IN>(nx, ntot, nv, G, s_nx);
+        for (; blk < total; blk += G) {
+            one_block(blk);
+            next_fold<IN>(ntot, nv, G, s_nx, nm);
+            nv += 2 * G;
+            next_stage<IN>(nx, ntot, nv, G, s_nx);
+        }
+        next_fold<IN>(ntot, nv, G, s_nx, nm);
+        for (nv += 2 * G; nv < ntot; nv += G) amax_fold<IN>(nm, __ldg(vec_at<IN>(nx, nv)));
+        amax_finish(amax_bits<IN>(nm), 1.0f, ws, nx.gs, 0);
+    } else if (q16_persistent<KIND>()) {
         for (; blk < total; blk += G) one_block(blk);
     } else if (blk < total) {
         one_block(blk);
@@ -1700,25 +1772,48 @@ int check_common(const void* x, int dtype, int64_t rows, int64_t cols, int64_t l
     return FP4Q_OK;
 }
 
-// The NVFP4 / IF4 kernel; 32-bit index arithmetic when the tensor allows it.
+// Batch context of a q16 launch: the next tensor whose amax the launch folds (null: none) and
+// whether the status word is ORed (later tensors of a batch) rather than written.
+struct BatchLink {
+    const NextTensor<int64_t>* next = nullptr;
+    int status_or = 0;
+};
+
+// The NVFP4 / IF4 kernel; 32-bit index arithmetic when the tensors allow it.
 template <int IN, int KIND, bool HAD, typename IDX>
 void launch_q16_as(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* imp, uint8_t* codes,
-                   uint8_t* scales, float* gs, uint32_t* ws, int tiled, cudaStream_t st) {
-    auto kernel = q16_kernel<IN, KIND, HAD, IDX>;
+                   uint8_t* scales, float* gs, uint32_t* ws, int tiled, cudaStream_t st, BatchLink bl) {
     const int64_t total = rows * (cols / 16);
+    if constexpr (q16_persistent<KIND>() && !HAD) {
+        if (bl.next) {
+            const NextTensor<int64_t>& n = *bl.next;
+            const NextTensor<IDX> nx = {n.x, (IDX)n.rows, (IDX)n.cols, (IDX)n.ld, n.gs};
+            const int64_t nvec = n.rows * (n.cols * (IN == FP4Q_IN_BF16 ? 2 : 4) / 16);
+            auto kernel = q16_kernel<IN, KIND, HAD, IDX, true>;
+            // two of the next tensor's vectors ride on each block: size the wave for the larger need
+            const int grid = grid_for(kernel, total > nvec / 2 ? total : nvec / 2, q16_min_ctas<KIND>());
+            kernel<<<grid, kThreads, 0, st>>>(x, (IDX)rows, (IDX)cols, (IDX)ld, imp, codes, scales, gs, ws, tiled, nx,
+                                              bl.status_or);
+            return;
+        }
+    }
+    auto kernel = q16_kernel<IN, KIND, HAD, IDX, false>;
     const int grid = q16_persistent<KIND>() ? grid_for(kernel, total, q16_min_ctas<KIND>())
                                             : (int)((total + kThreads - 1) / kThreads);
-    kernel<<<grid, kThreads, 0, st>>>(x, (IDX)rows, (IDX)cols, (IDX)ld, imp, codes, scales, gs, ws, tiled);
+    const NextTensor<IDX> none = {nullptr, 0, 0, 0, nullptr};
+    kernel<<<grid, kThreads, 0, st>>>(x, (IDX)rows, (IDX)cols, (IDX)ld, imp, codes, scales, gs, ws, tiled, none,
+                                      bl.status_or);
 }
 
 template <int IN, int KIND, bool HAD>
 void launch_q16(const void* x, int64_t rows, int64_t cols, int64_t ld, const float* imp, uint8_t* codes,
-                uint8_t* scales, float* gs, uint32_t* ws, int tiled, cudaStream_t st) {
+                uint8_t* scales, float* gs, uint32_t* ws, int tiled, cudaStream_t st, BatchLink bl) {
     const int64_t total = rows * (cols / 16);
-    if (total < ((int64_t)1 << 31) && rows * ld < ((int64_t)1 << 31))
-        launch_q16_as<IN, KIND, HAD, uint32_t>(x, rows, cols, ld, imp, codes, scales, gs, ws, tiled, st);
+    const bool small_next = !bl.next || bl.next->rows * bl.next->ld < ((int64_t)1 << 31);
+    if (total < ((int64_t)1 << 31) && rows * ld < ((int64_t)1 << 31) && small_next)
+        launch_q16_as<IN, KIND, HAD, uint32_t>(x, rows, cols, ld, imp, codes, scales, gs, ws, tiled, st, bl);
     else
-        launch_q16_as<IN, KIND, HAD, int64_t>(x, rows, cols, ld, imp, codes, scales, gs, ws, tiled, st);
+        launch_q16_as<IN, KIND, HAD, int64_t>(x, rows, cols, ld, imp, codes, scales, gs, ws, tiled, st, bl);
 }
 
 // Tensor scale pass: plain amax, or the amax of the 16-point rotated blocks.
@@ -1737,21 +1832,28 @@ void launch_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, uint32_t
 
 template <int IN, bool HAD>
 void launch_nvfp4_if4(const void* x, int64_t rows, int64_t cols, int64_t ld, int fmt, int obj, const float* imp,
-                      uint8_t* codes, uint8_t* scales, float* gs, uint32_t* ws, uint32_t flags, cudaStream_t st) {
+                      uint8_t* codes, uint8_t* scales, float* gs, uint32_t* ws, uint32_t flags, cudaStream_t st,
+                      BatchLink bl = BatchLink()) {
     const int tiled = (flags & FP4Q_F_SCALE_TILED) ? 1 : 0;
     if (fmt == FP4Q_IF4) {
-        if (flags & FP4Q_F_IF4_SWEEP) launch_q16<IN, KIND_IF4_SWEEP, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, tiled, st);
-        else launch_q16<IN, KIND_IF4, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, tiled, st);
+        if (flags & FP4Q_F_IF4_SWEEP)
+            launch_q16<IN, KIND_IF4_SWEEP, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, tiled, st, bl);
+        else
+            launch_q16<IN, KIND_IF4, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, tiled, st, bl);
         return;
     }
     switch (obj) {
-        case FP4Q_ABSMAX: launch_q16<IN, FP4Q_ABSMAX, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, tiled, st); break;
-        case FP4Q_FOUR_OVER_SIX:
-            launch_q16<IN, FP4Q_FOUR_OVER_SIX, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, tiled, st);
+        case FP4Q_ABSMAX:
+            launch_q16<IN, FP4Q_ABSMAX, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, tiled, st, bl);
             break;
-        case FP4Q_SWEEP_MSE: launch_q16<IN, FP4Q_SWEEP_MSE, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, tiled, st); break;
+        case FP4Q_FOUR_OVER_SIX:
+            launch_q16<IN, FP4Q_FOUR_OVER_SIX, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, tiled, st, bl);
+            break;
+        case FP4Q_SWEEP_MSE:
+            launch_q16<IN, FP4Q_SWEEP_MSE, HAD>(x, rows, cols, ld, imp, codes, scales, gs, ws, tiled, st, bl);
+            break;
         default:   // WMSE is rejected with the rotation before any launch
-            if (!HAD) launch_q16<IN, FP4Q_SWEEP_WMSE, false>(x, rows, cols, ld, imp, codes, scales, gs, ws, tiled, st);
+            if (!HAD) launch_q16<IN, FP4Q_SWEEP_WMSE, false>(x, rows, cols, ld, imp, codes, scales, gs, ws, tiled, st, bl);
             break;
     }
 }
@@ -1935,6 +2037,77 @@ int fp4q_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int64_t 
                                              ws, flags, st);
     return launch_quantize<FP4Q_IN_F32>(x, rows, cols, ld, fmt, objective, importance, codes, scales, global_scale, ws,
                                         flags, st);
+}
+
+}  // extern "C"
+
+namespace fp4q {
+// fp4q_quantize_batch: the non-empty tensors in order.  Without a given S, the first one's amax
+// pass is its own kernel and every quantize kernel also folds the following tensor's amax
+// (persistent kinds, no rotation); WMSE and the rotated forms run each tensor's amax pass as its
+// own kernel.  The status word is cleared first and every quantize kernel ORs its flags into it.
+template <int IN>
+int batch_impl(const fp4q_tensor* t, const int* live, int m, int fmt, int obj, uint32_t* ws, uint32_t flags,
+               cudaStream_t st) {
+    if (cudaMemsetAsync(ws + WS_STATUS, 0, sizeof(uint32_t), st) != cudaSuccess) return launched(0);
+    const bool given = (flags & FP4Q_F_GLOBAL_SCALE_GIVEN) != 0, had16 = (flags & FP4Q_F_HADAMARD16) != 0;
+    const bool fused = !given && !had16 && !(fmt == FP4Q_NVFP4 && obj == FP4Q_SWEEP_WMSE);
+    auto rides = [&](int k) { return fused && k > 0; };   // a tensor's amax rides on the previous kernel
+    int n = 0;
+    for (int k = 0; k < m; ++k) {
+        const fp4q_tensor& a = t[live[k]];
+        if (!given && !rides(k)) {
+            launch_amax<IN>(a.x, a.rows, a.cols, a.ld, ws, a.global_scale, 0, had16, st);
+            ++n;
+        }
+        NextTensor<int64_t> nx = {nullptr, 0, 0, 0, nullptr};
+        BatchLink bl;
+        bl.status_or = 1;
+        if (k + 1 < m && rides(k + 1)) {
+            const fp4q_tensor& b = t[live[k + 1]];
+            nx = {b.x, b.rows, b.cols, b.ld, b.global_scale};
+            bl.next = &nx;
+        }
+        if (had16)
+            launch_nvfp4_if4<IN, true>(a.x, a.rows, a.cols, a.ld, fmt, obj, a.importance, a.codes, a.scales,
+                                       a.global_scale, ws, flags, st, bl);
+        else
+            launch_nvfp4_if4<IN, false>(a.x, a.rows, a.cols, a.ld, fmt, obj, a.importance, a.codes, a.scales,
+                                        a.global_scale, ws, flags, st, bl);
+        ++n;
+    }
+    return launched(n);
+}
+}  // namespace fp4q
+
+extern "C" {
+
+int fp4q_quantize_batch(int n, const fp4q_tensor* tensors, int dtype, int fmt, int objective, void* workspace,
+                        uint32_t flags, void* stream) {
+    g_launches = 0;
+    if (n < 0 || (n > 0 && !tensors)) return FP4Q_ERR_INVALID_ARG;
+    int rc = check_quantize_args(fmt, objective, flags);
+    if (rc != FP4Q_OK) return rc;
+    if (fmt != FP4Q_NVFP4 && fmt != FP4Q_IF4) return FP4Q_ERR_UNSUPPORTED;
+    std::vector<int> live;
+    for (int i = 0; i < n; ++i) {
+        const fp4q_tensor& a = tensors[i];
+        rc = check_common(a.x, dtype, a.rows, a.cols, a.ld, 16, a.codes, a.scales, workspace);
+        if (rc != FP4Q_OK) return rc;
+        if (a.rows == 0 || a.cols == 0) continue;
+        if (!a.global_scale) return FP4Q_ERR_INVALID_ARG;
+        if (fmt == FP4Q_NVFP4 && objective == FP4Q_SWEEP_WMSE) {
+            if (!a.importance) return FP4Q_ERR_INVALID_ARG;
+            if (!aligned16(a.importance)) return FP4Q_ERR_ALIGNMENT;
+        }
+        live.push_back(i);
+    }
+    if (live.empty()) return FP4Q_OK;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t* ws = reinterpret_cast<uint32_t*>(workspace);
+    if (dtype == FP4Q_IN_BF16)
+        return batch_impl<FP4Q_IN_BF16>(tensors, live.data(), (int)live.size(), fmt, objective, ws, flags, st);
+    return batch_impl<FP4Q_IN_F32>(tensors, live.data(), (int)live.size(), fmt, objective, ws, flags, st);
 }
 
 }  // extern "C"

@@ -196,6 +196,43 @@ FP4Q_API int fp4q_global_scale(const void* x, int dtype, int64_t rows, int64_t c
                       float* global_scale, void* workspace, void* stream);
 
 /*
+ * One tensor of a batch (fp4q_quantize_batch).  Members as the fp4q_quantize arguments of the
+ * same names: x [rows][ld] (device, bf16 or fp32 as the batch's dtype), codes, scales,
+ * global_scale (device; written with S, or read under FP4Q_F_GLOBAL_SCALE_GIVEN) and, for
+ * SWEEP_WMSE only, importance (device float[cols], else NULL).  Caller-owned.
+ */
+typedef struct fp4q_tensor {
+    const void* x;
+    int64_t rows, cols, ld;
+    const float* importance;
+    uint8_t* codes;
+    uint8_t* scales;
+    float* global_scale;
+} fp4q_tensor;
+
+/*
+ * NVFP4 or IF4 quantization of n tensors in order, with the results of n fp4q_quantize calls
+ * (same dtype, fmt, objective and flags; every tensor gets its own S = RN(amax/1536) from its
+ * own elements, ScaleSweep, "Methodology"): codes, scale bytes and S bit for bit identical.
+ * A sequence of tensors (the layers of a model, a stream of activations) leaves the HBM-bound
+ * amax pass and the arithmetic-bound search of each tensor side by side: here the quantize
+ * kernel of tensor i also reads tensor i+1 and writes its S, so that read overlaps the search
+ * instead of running as a pass of its own.
+ *   tensors    host array of n descriptors (read during the call only); empty tensors are
+ *              skipped.  The inputs must not overlap any output of the batch.
+ *   workspace  as fp4q_quantize; word 0 receives the OR of the tensors' device statuses (a
+ *              batch of only empty tensors leaves it unchanged).
+ *   flags      as fp4q_quantize.
+ * Launches (NVFP4 AbsMax, 4/6 and sweep-MSE, IF4 and the IF4 sweep, no rotation, S not given):
+ * one amax kernel for the first non-empty tensor, then one quantize kernel per tensor, m + 1
+ * for m non-empty tensors.  With FP4Q_F_GLOBAL_SCALE_GIVEN: m quantize kernels.  SWEEP_WMSE and
+ * FP4Q_F_HADAMARD16 keep the amax pass as its own kernel per tensor (2m).  MXFP4 and IF6:
+ * FP4Q_ERR_UNSUPPORTED.  Errors: as fp4q_quantize, for every tensor, before anything runs.
+ */
+FP4Q_API int fp4q_quantize_batch(int n, const fp4q_tensor* tensors, int dtype, int fmt, int objective,
+                        void* workspace, uint32_t flags, void* stream);
+
+/*
  * IF6's tensor scale: S = RN(max|x| / 1920) (7.5, the FP6 maximum, in place of FP4's 6; Adaptive
  * Block-Scaled Data Types, "Methodology", the IF4 construction at 6 bits).  Status, workspace,
  * shapes and errors as fp4q_global_scale; passing the result to fp4q_quantize(FP4Q_IF6) with

@@ -186,3 +186,34 @@ def test_host_async_validation():
     assert call(flags=0x40) == fq.ERR_UNSUPPORTED                 # IF4 sweep on NVFP4
     assert call(flags=0x20) == fq.ERR_UNSUPPORTED                 # MX sweep on NVFP4
     assert call(rows=0, x_host=None, x_dev=None) == fq.OK and L.fp4q_last_launch_count() == 0
+
+
+def test_quantize_batch_rejects_before_launch():
+    L = fq.lib()
+    F = FAKE
+    T = fq._Tensor
+
+    def call(ts, fmt=0, obj=2, flags=0, dtype=1, ws=F, n=None):
+        arr = (T * max(1, len(ts)))(*ts)
+        return L.fp4q_quantize_batch(len(ts) if n is None else n, C.cast(arr, C.c_void_p), dtype, fmt, obj, ws,
+                                     flags, None)
+
+    good = lambda **kw: T(kw.get("x", F), kw.get("rows", 4), kw.get("cols", 64), kw.get("ld", 64),
+                          kw.get("imp", None), kw.get("codes", F), kw.get("scales", F), kw.get("gs", F))
+    assert call([good()], n=-1) == fq.ERR_INVALID_ARG
+    assert L.fp4q_quantize_batch(2, None, 1, 0, 2, F, 0, None) == fq.ERR_INVALID_ARG
+    assert call([good()], fmt=2) == fq.ERR_UNSUPPORTED                  # MXFP4: no tensor scale to batch
+    assert call([good()], fmt=3) == fq.ERR_UNSUPPORTED                  # IF6
+    assert call([good()], fmt=9) == fq.ERR_INVALID_ARG
+    assert call([good(), good(cols=24)]) == fq.ERR_SHAPE                # checked for every tensor
+    assert call([good(), good(ld=32)]) == fq.ERR_SHAPE
+    assert call([good(), good(x=F + 8)]) == fq.ERR_ALIGNMENT
+    assert call([good(), good(gs=None)]) == fq.ERR_INVALID_ARG
+    assert call([good(imp=F), good(imp=None)], obj=3) == fq.ERR_INVALID_ARG  # WMSE needs each importance
+    assert call([good(imp=F), good(imp=F + 4)], obj=3) == fq.ERR_ALIGNMENT
+    assert call([good()], dtype=5) == fq.ERR_INVALID_ARG
+    assert call([good()], ws=None) == fq.ERR_INVALID_ARG
+    # empty tensors are skipped: a batch of only empty tensors launches nothing
+    assert call([good(rows=0, x=None, codes=None, scales=None, gs=None), good(cols=0)]) == fq.OK
+    assert L.fp4q_last_launch_count() == 0
+    assert call([]) == fq.OK and L.fp4q_last_launch_count() == 0

@@ -1,5 +1,5 @@
 """The GEMM's bounded-wait failure path, exercised without a fault: a test build of the library
-(libfp4q_gemm_failtest.so, the same sources with FP4Q_GEMM_FAIL_FIRST_WAIT) makes the MMA thread
+(libfp4q_failtest.so, the same sources with FP4Q_GEMM_FAIL_FIRST_WAIT) makes the MMA thread
 treat its first wait as timed out.  The call must return, report FP4Q_DEVSTAT_TIMEOUT in the
 status word once the stream is done (the producer's own wait for a free ring slot then runs out
 as well, after its bounded polls), and leave the context usable: the product library's next GEMM
@@ -17,7 +17,7 @@ import oracle as O
 import fp4_block_scaled_nvfp4_b200 as fq
 from fp4_block_scaled_nvfp4_b200 import synth
 
-TEST_LIB = os.path.join(os.path.dirname(fq.__file__), "libfp4q_gemm_failtest.so")
+TEST_LIB = os.path.join(os.path.dirname(fq.__file__), "libfp4q_failtest.so")
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -25,7 +25,7 @@ def _need_cuda():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     if not os.path.exists(TEST_LIB):
-        pytest.fail("libfp4q_gemm_failtest.so is not built (__graft_entry__.build() builds it)")
+        pytest.fail("libfp4q_failtest.so is not built (__graft_entry__.build() builds it)")
     fq.lib()
 
 
