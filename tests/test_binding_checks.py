@@ -40,3 +40,18 @@ def test_noalloc_needs_outputs():
     x = torch.zeros(4, 32)
     with pytest.raises(fq.Fp4qError):
         fq.quantize_noalloc(x, "nvfp4", "absmax", out=None)
+
+
+def test_batch_rejects_before_the_library():
+    x = torch.zeros(4, 32)
+    with pytest.raises(fq.Fp4qError, match="nvfp4 or if4"):
+        fq.quantize_batch([x], "mxfp4")
+    with pytest.raises(fq.Fp4qError, match="nvfp4 or if4"):
+        fq.quantize_batch([x], "if6")
+    with pytest.raises(fq.Fp4qError, match="objective"):
+        fq.quantize_batch([x], "nvfp4", "sweep-mse")
+    with pytest.raises(fq.Fp4qError, match="one entry per tensor"):
+        fq.quantize_batch([x, x], "nvfp4", global_scales=[torch.ones(1)])
+    with pytest.raises(fq.Fp4qError, match="CUDA"):
+        fq.quantize_batch([x], "nvfp4", "absmax")
+    assert fq.quantize_batch([], "nvfp4") == []
