@@ -688,8 +688,10 @@ def run_ours(args, rank, world):
                          f"total (at least 3x the 126 MB L2)",
                    "timing": ("one fp4q_quantize_batch call over the K steps' tensors (the buffer sets in turn), "
                               "captured as a CUDA graph: an amax kernel for the first tensor, then K quantize "
-                              "kernels, each also taking the next tensor's amax; CUDA events on the launching "
-                              "stream" if fused else
+                              "kernels, each also taking the next tensor's amax" +
+                              ("; the AbsMax kernel marks that read evict-last in L2, so the tensor's second read "
+                               "(its quantization, one kernel later) comes mostly from L2" if obj == "absmax" else "") +
+                              "; CUDA events on the launching stream" if fused else
                               "CUDA graph over the buffer sets (no timing nodes inside); each step's amax pass runs on "
                               "a second stream under the previous step's quantize kernel, each quantize after its own "
                               "amax; CUDA events on the launching stream" if two_pass else
