@@ -55,3 +55,48 @@ def test_header_compiles_as_c_and_the_abi_links(tmp_path):
     assert out.returncode == 0, out.stderr
     run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert run.returncode == 0 and run.stdout.strip() == "ok", (run.returncode, run.stdout, run.stderr)
+
+
+LAYOUT = r"""
+#include <stddef.h>
+#include <stdio.h>
+#include "fp4q.h"
+
+int main(void) {
+    fp4q_tensor t[2];
+    memset(t, 0, sizeof t);
+    printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(fp4q_tensor), offsetof(fp4q_tensor, x),
+           offsetof(fp4q_tensor, rows), offsetof(fp4q_tensor, cols), offsetof(fp4q_tensor, ld),
+           offsetof(fp4q_tensor, importance), offsetof(fp4q_tensor, codes), offsetof(fp4q_tensor, scales),
+           offsetof(fp4q_tensor, global_scale));
+    /* a batch of empty tensors returns before anything runs */
+    t[0].cols = 64; t[0].ld = 64; t[1].rows = 3;
+    return fp4q_quantize_batch(2, t, FP4Q_IN_BF16, FP4Q_NVFP4, FP4Q_SWEEP_MSE, (void*)0x10000, 0u, NULL) == FP4Q_OK &&
+           fp4q_last_launch_count() == 0 ? 0 : 1;
+}
+"""
+
+
+def test_batch_descriptor_layout_matches_the_binding(tmp_path):
+    # the binding's ctypes fp4q_tensor must have the header struct's size and field offsets
+    import ctypes as C
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    lib = fq.LIB_PATH
+    if not os.path.exists(lib):
+        pytest.skip("library not built")
+    src = tmp_path / "layout.c"
+    src.write_text("#include <string.h>\n" + LAYOUT)
+    exe = tmp_path / "layout"
+    cmd = [gcc, "-std=c11", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"), str(src),
+           lib, "-Wl,-rpath," + os.path.dirname(lib), "-o", str(exe)]
+    out = subprocess.run(cmd, capture_output=True, text=True)
+    assert out.returncode == 0, out.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0, (run.stdout, run.stderr)
+    got = [int(v) for v in run.stdout.split()]
+    T = fq._Tensor
+    want = [C.sizeof(T)] + [getattr(T, f).offset for f in
+                            ("x", "rows", "cols", "ld", "importance", "codes", "scales", "global_scale")]
+    assert got == want
